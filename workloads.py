@@ -1,0 +1,151 @@
+"""Seeded synthetic inputs for the QJL key-compression workloads.
+
+This module is shared by the tests, the smoke check and the bench, and is the
+only thing the CUDA path and the CPU oracle have in common.  It holds no step
+of the method: it only draws keys, values and queries with the shapes and
+distributions of the five workloads below and records how it drew them.
+
+Workloads (keys/values/queries are synthetic; there are no model weights):
+  single   1 head, d=128, m=256, 1024 fp32 keys and 1 fp32 query N(0,1);
+           values N(0,1) stored as bf16; quantize + one decode step.
+  gqa      GQA decode: batch 8, 32 query heads / 8 KV heads, d=128, m=256,
+           context 32768; bf16 keys N(0,1) with 4 outlier channels x10;
+           bf16 values N(0,1); one query token per sequence.
+  long     MHA decode: batch 1, 32 heads, d=128, m=256, context 131072; bf16
+           keys k_t = r_t g_t with g_t ~ N(0, I) and r_t ~ lognormal(0, 0.5);
+           bf16 values N(0,1).
+  prefill  quantization of 65536 tokens x 32 layers x 8 KV heads, d=128,
+           m=256; bf16 keys N(0,1) with 4 outlier channels x10.
+  sweep    m in {64,128,256,512} x d in {64,128}; batch 16, 32 heads MHA,
+           context 16384; bf16 keys and values N(0,1).
+
+Recipe details that the workload descriptions leave open:
+  * the sketch seed is 0 for every workload;
+  * data seeds: workload index i (1..5) gives torch generator seeds
+    1000*i + {0: keys, 1: values, 2: queries, 3: outlier channels,
+    4: per-token norms};
+  * outlier channels: the first 4 entries of a seeded permutation of range(d);
+  * queries are N(0,1) in the key dtype, scaled by ``q_scale`` (default 1);
+  * softmax scale 1/sqrt(d).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int              # 1..5, selects the data seeds
+    B: int                  # batch
+    Hq: int                 # query heads
+    Hkv: int                # KV heads
+    T: int                  # context length (keys per (b, kv-head))
+    d: int                  # head dimension
+    m: int                  # sketch rows
+    key_dtype: torch.dtype  # dtype keys and queries are stored in
+    outliers: int = 0       # number of outlier channels scaled by 10
+    lognormal_sigma: float = 0.0  # per-token norm spread (0 = none)
+    sketch_seed: int = 0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def n_keys(self) -> int:
+        return self.B * self.Hkv * self.T
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+SINGLE = Workload("single", 1, 1, 1, 1, 1024, 128, 256, torch.float32)
+GQA = Workload("gqa", 2, 8, 32, 8, 32768, 128, 256, torch.bfloat16, outliers=4)
+LONG = Workload("long", 3, 1, 32, 32, 131072, 128, 256, torch.bfloat16,
+                lognormal_sigma=0.5)
+# prefill: 65536 tokens x 32 layers x 8 KV heads, laid out as B=32 layers,
+# Hkv=8 heads, T=65536 tokens (no queries; quantization only)
+PREFILL = Workload("prefill", 4, 32, 8, 8, 65536, 128, 256, torch.bfloat16,
+                   outliers=4)
+SWEEP_BASE = Workload("sweep", 5, 16, 32, 32, 16384, 128, 256, torch.bfloat16)
+SWEEP_M = (64, 128, 256, 512)
+SWEEP_D = (64, 128)
+
+ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE)}
+
+
+def sweep_points():
+    return [SWEEP_BASE.with_(m=m, d=d) for d in SWEEP_D for m in SWEEP_M]
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def outlier_channels(w: Workload) -> torch.Tensor:
+    if w.outliers == 0:
+        return torch.empty(0, dtype=torch.long)
+    perm = torch.randperm(w.d, generator=_gen("cpu", 1000 * w.index + 3))
+    return perm[: w.outliers].sort().values
+
+
+def _fill_normal(out: torch.Tensor, gen: torch.Generator, rows_per_chunk: int,
+                 scale_cols: torch.Tensor | None, row_scale=None):
+    """Fill a [rows, d] view with N(0,1) draws chunk by chunk (bounded temp)."""
+    rows, d = out.shape
+    for r0 in range(0, rows, rows_per_chunk):
+        r1 = min(rows, r0 + rows_per_chunk)
+        x = torch.randn((r1 - r0, d), generator=gen, device=out.device,
+                        dtype=torch.float32)
+        if scale_cols is not None and scale_cols.numel():
+            x[:, scale_cols.to(out.device)] *= 10.0
+        if row_scale is not None:
+            x *= row_scale[r0:r1, None].to(out.device)
+        out[r0:r1].copy_(x)
+
+
+def keys(w: Workload, device="cpu", rows_per_chunk: int = 1 << 20):
+    """Keys [B, Hkv, T, d] in w.key_dtype."""
+    K = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=w.key_dtype, device=device)
+    flat = K.view(-1, w.d)
+    row_scale = None
+    if w.lognormal_sigma > 0:
+        z = torch.randn(flat.shape[0], generator=_gen(device, 1000 * w.index + 4),
+                        device=device, dtype=torch.float32)
+        row_scale = torch.exp(w.lognormal_sigma * z)
+    _fill_normal(flat, _gen(device, 1000 * w.index + 0), rows_per_chunk,
+                 outlier_channels(w), row_scale)
+    return K
+
+
+def values(w: Workload, device="cpu", rows_per_chunk: int = 1 << 20):
+    """Values [B, Hkv, T, d] in bf16 (fp32 draws rounded to bf16)."""
+    V = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.bfloat16, device=device)
+    _fill_normal(V.view(-1, w.d), _gen(device, 1000 * w.index + 1),
+                 rows_per_chunk, None)
+    return V
+
+
+def queries(w: Workload, device="cpu", q_scale: float = 1.0):
+    """One query token per (b, query head): [B, Hq, d] in w.key_dtype."""
+    Q = torch.randn((w.B, w.Hq, w.d), generator=_gen(device, 1000 * w.index + 2),
+                    device=device, dtype=torch.float32) * q_scale
+    return Q.to(w.key_dtype)
+
+
+def random_keys(n: int, d: int, seed: int, dtype=torch.bfloat16, device="cpu",
+                scale: float = 1.0):
+    """Plain N(0, scale^2) keys [n, d] for edge-case tests."""
+    x = torch.randn((n, d), generator=_gen(device, seed), device=device,
+                    dtype=torch.float32) * scale
+    return x.to(dtype)
