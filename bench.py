@@ -1,0 +1,459 @@
+"""Benchmark: QJL key quantization + compressed-key decode attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>]
+
+A step is one pass of the whole hot path over one batch of the workload:
+quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
+run one decode step of attention over the compressed cache
+(jl_decode_attention: query projection, scorer, combine).  The default
+workload is GQA decode: batch 8, 32 query / 8 KV heads, d=128, m=256, context
+32768.  Inputs are seeded synthetic tensors (workloads.py) already resident
+in HBM; they exceed L2 (126 MB), so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own batch of the same workload
+(independent sequences, no data-path collective), timing is the max over ranks
+and ``value`` counts the keys of all ranks ("scaling": "weak").
+
+The JSON line also carries: per-phase CUDA-event timings, the roofline of the
+dominant kernel (algorithmic bytes / measured duration against the measured
+HBM copy bandwidth), the end-to-end number through the Python binding with
+pinned host buffers (H2D copies of the step's inputs and D2H of its output
+inside the timed region), SM clocks sampled during the timed region, and the
+float64 oracle timed on a bounded sample on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------
+# helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def pick_workload(name: str) -> workloads.Workload:
+    if name.startswith("sweep"):
+        # sweep-m<M>-d<D>
+        m = int(name.split("-m")[1].split("-")[0])
+        d = int(name.split("-d")[1])
+        return workloads.SWEEP_BASE.with_(m=m, d=d)
+    return workloads.ALL[name]
+
+
+def kernel_source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "bit_jl_key_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e:
+        return None
+    if e.get("source_hash") != kernel_source_hash(e["sources"]):
+        return None
+    return e
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sms, maxs, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 9:
+                continue
+            try:
+                sms.append(float(c[1]))
+                maxs.append(float(c[2]))
+                power.append(float(c[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, c[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes
+
+def quantize_bytes(w, n_keys):
+    """Read the keys, write codes + fp16 norms (the sketch is 64 KB, L2)."""
+    kb = 2 if w.key_dtype == torch.bfloat16 else 4
+    return n_keys * (w.d * kb + w.m // 8 + 2)
+
+
+def decode_bytes(w):
+    """Per KV key: code (m/8 B) + fp16 norm (2 B) + bf16 value row (2d B)."""
+    return w.B * w.Hkv * w.T * (w.m // 8 + 2 + 2 * w.d)
+
+
+# --------------------------------------------------------------------------
+# our arm
+
+def run_ours(args, rank, world, local_rank):
+    import bit_jl_key_b200 as jl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload)
+    decode = w.name != "prefill"
+    peak, peak_kind = load_peaks()
+
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)
+    Kf = K.view(-1, w.d)
+    n_keys = Kf.shape[0]
+    W = w.m // 32
+    signs = torch.empty((n_keys, W), dtype=torch.int32, device=dev)
+    norms = torch.empty((n_keys,), dtype=torch.float16, device=dev)
+    if decode:
+        V = workloads.values(w, dev)
+        Q = workloads.queries(w, dev)
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        ws_bytes = jl.jl_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d)
+        ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+        sg4 = signs.view(w.B, w.Hkv, w.T, W)
+        nr3 = norms.view(w.B, w.Hkv, w.T)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + (3 if decode else 0)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        jl.jl_quantize_keys(Kf, S, signs, norms)
+        if ev is not None:
+            ev[1].record(stream)
+        if decode:
+            jl.jl_decode_attention(Q, S, sg4, nr3, V, softmax_scale=w.softmax_scale,
+                                   out=out, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+
+    # timed region: whole steps, plus per-phase events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    d_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if decode else 0.0
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step = float(t.item())
+    keys_all = n_keys * world
+    value = keys_all / (ms_step * 1e-3)
+
+    # ---- end to end through the binding with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hK = K.cpu().pin_memory()
+        del K
+        torch.cuda.empty_cache()
+        Kd = torch.empty(hK.shape, dtype=hK.dtype, device=dev)
+        h2d = hK.numel() * hK.element_size()
+        if decode:
+            hV = V.cpu().pin_memory()
+            hQ = Q.cpu().pin_memory()
+            hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+            Vd, Qd = V, Q
+            h2d += hV.numel() * hV.element_size() + hQ.numel() * hQ.element_size()
+            d2h = hOut.numel() * hOut.element_size()
+        else:
+            hSig = torch.empty(signs.shape, dtype=signs.dtype).pin_memory()
+            hNrm = torch.empty(norms.shape, dtype=norms.dtype).pin_memory()
+            d2h = hSig.numel() * 4 + hNrm.numel() * 2
+
+        def e2e_step():
+            Kd.copy_(hK, non_blocking=True)
+            if decode:
+                Vd.copy_(hV, non_blocking=True)
+                Qd.copy_(hQ, non_blocking=True)
+            jl.jl_quantize_keys(Kd.view(-1, w.d), S, signs, norms)
+            if decode:
+                jl.jl_decode_attention(Qd, S, sg4, nr3, Vd,
+                                       softmax_scale=w.softmax_scale, out=out,
+                                       workspace=ws)
+                hOut.copy_(out, non_blocking=True)
+            else:
+                hSig.copy_(signs, non_blocking=True)
+                hNrm.copy_(norms, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e_steps = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": keys_all / (e_ms * 1e-3), "unit": "keys/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    # ---- roofline of the dominant kernel
+    qb = quantize_bytes(w, n_keys)
+    phases = {"quantize": {"ms": q_ms, "keys_per_s": n_keys / (q_ms * 1e-3),
+                           "tokens_per_s": w.B * w.T / (q_ms * 1e-3),
+                           "algorithmic_bytes": qb,
+                           "GB_per_s": qb / (q_ms * 1e-3) / 1e9}}
+    phases["quantize"]["frac_of_hbm_peak"] = phases["quantize"]["GB_per_s"] / peak
+    if decode:
+        db = decode_bytes(w)
+        phases["decode"] = {"ms": d_ms, "keys_scored_per_s": n_keys / (d_ms * 1e-3),
+                            "head_key_pairs_per_s": w.B * w.Hq * w.T / (d_ms * 1e-3),
+                            "algorithmic_bytes": db,
+                            "GB_per_s": db / (d_ms * 1e-3) / 1e9}
+        phases["decode"]["frac_of_hbm_peak"] = phases["decode"]["GB_per_s"] / peak
+    dom = max(phases, key=lambda k: phases[k]["ms"])
+    traffic = ncu_traffic({"quantize": "quantize", "decode": "decode"}[dom] + ":" + w.name)
+    roof = {"kernel": {"quantize": "jl_quantize_keys", "decode": "jl_decode_attention"}[dom],
+            "bound": "hbm", "achieved": phases[dom]["GB_per_s"], "peak": peak,
+            "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+            "frac": phases[dom]["GB_per_s"] / peak,
+            "algorithmic_bytes_per_launch": phases[dom]["algorithmic_bytes"],
+            "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
+
+    clocks = clk.summary()
+    line = {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": value, "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} "
+                               f"d={w.d} m={w.m}",
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"dp{world}",
+                   "l2": "inputs exceed L2 (126 MB); no flush"},
+        "phases": phases,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+
+def oracle_sample(w: workloads.Workload):
+    """A bounded sample of the workload for the float64 oracle: the first
+    (b, kv-head) unit of keys/values and its G query heads (prefill: the first
+    16384 keys).  Returns (callable running one oracle step, keys per step,
+    description)."""
+    import numpy as np
+    import oracle
+
+    S64 = oracle.sketch(w.m, w.d, w.sketch_seed)
+    if w.name == "prefill":
+        n = 16384
+        Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()
+
+        def run():
+            oracle.quantize(Kf, S64)
+        return run, n, f"first {n} keys of the workload's recipe (quantize only)"
+    T = w.T if w.name != "long" else 32768
+    sub = w.with_(B=1, Hkv=1, Hq=w.G, T=T)
+    K = workloads.keys(sub).double().numpy()
+    V = workloads.values(sub).double().numpy()
+    Q = workloads.queries(sub).double().numpy()
+
+    def run():
+        sig, nrm, n16, _ = oracle.quantize(K.reshape(-1, w.d), S64)
+        oracle.decode(Q, S64, sig.reshape(1, 1, T, w.m // 32),
+                      oracle.fp16_bits_to_f64(n16).reshape(1, 1, T), V,
+                      w.softmax_scale)
+    return run, T, (f"one (b, kv-head) unit: {T} keys, {w.G} query heads, "
+                    f"quantize + decode in float64")
+
+
+def time_oracle(w, steps=1, warmup=0):
+    import oracle
+    run, keys, desc = oracle_sample(w)
+    for _ in range(warmup):
+        run()
+    t = time.perf_counter()
+    for _ in range(steps):
+        run()
+    dt = (time.perf_counter() - t) / steps
+    return {"value": keys / dt, "unit": "keys/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "sample": desc, "s_per_step": dt}
+
+
+def run_reference(args, rank, world):
+    w = pick_workload(args.workload)
+    if rank != 0:
+        return None
+    cb = time_oracle(w, steps=args.steps, warmup=args.warmup)
+    return {
+        "impl": "reference",
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": cb["value"], "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": cb["s_per_step"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} "
+                               f"d={w.d} m={w.m}",
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"dp{world}"},
+        "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": cb["value"], "unit": "keys/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local_rank))
+    try:
+        # the oracle runs before any GPU work on rank 0 (bounded sample)
+        cb = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cb = time_oracle(pick_workload(args.workload), steps=1)
+        line = run_ours(args, rank, world, local_rank)
+        if cb is not None:
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+"""bit_jl_key_b200 -- QJL sign-bit key compression and compressed-key decode
+attention on NVIDIA B200 (sm_100a).
+
+This module is a thin ctypes binding over ``libjlkey.so`` (C ABI in
+``include/jlkey.h``).  It only marshals torch tensors into pointers, sizes and
+the current CUDA stream; every step of the computation runs in the library's
+CUDA kernels.  There is no CPU fallback: if the library is missing or a call
+fails, an exception is raised.
+
+Functions (same names as the C entry points):
+  jl_sketch_init(m, d, seed)            -> S  (bf16 [m, d])
+  jl_quantize_keys(K, S)                -> (signs int32 [n, m/32], norms fp16 [n])
+  jl_quantize_keys_simt(K, S)           -> same, SIMT-core kernel
+  jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int
+  jl_decode_attention(Q, S, signs, norms, V, ...) -> out bf16 [B, Hq, d]
+  jl_device_error()                     -> int (0 = no device fault reported)
+
+Sign codes are returned as torch.int32 tensors holding the uint32 words bit
+for bit (torch has no general uint32 arithmetic); word w of a key holds sketch
+rows 32w..32w+31, LSB first, bit = 1 iff (S k)_i >= 0.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjlkey.so")
+
+JL_BF16 = 0
+JL_F32 = 1
+JL_OK = 0
+JL_ERR_INVALID_ARG = -1
+JL_ERR_UNSUPPORTED = -2
+JL_ERR_WORKSPACE = -3
+JL_ERR_CUDA = -4
+JL_ERR_DEVICE = -5
+
+EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
+            "jl_quantize_keys_simt", "jl_decode_workspace_bytes",
+            "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64")
+
+_lib = None
+
+
+class JLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+def load():
+    """Load libjlkey.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m bit_jl_key_b200.build` "
+            "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.jl_status_string.restype = ctypes.c_char_p
+    L.jl_status_string.argtypes = [i32]
+    L.jl_sketch_init.restype = i32
+    L.jl_sketch_init.argtypes = [vp, i32, i32, ctypes.c_uint64, vp]
+    for name in ("jl_quantize_keys", "jl_quantize_keys_simt"):
+        f = getattr(L, name)
+        f.restype = i32
+        f.argtypes = [vp, i32, i64, i64, vp, i32, i32, vp, vp, vp]
+    L.jl_decode_workspace_bytes.restype = sz
+    L.jl_decode_workspace_bytes.argtypes = [i32, i32, i32, i64, i32, i32]
+    L.jl_decode_attention.restype = i32
+    L.jl_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32,
+                                      i64, i32, i32, ctypes.c_float, vp, vp,
+                                      vp, sz, vp]
+    L.jl_device_error.restype = i32
+    L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
+    L.jl_bf16_from_f64.restype = ctypes.c_uint16
+    L.jl_bf16_from_f64.argtypes = [ctypes.c_double]
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().jl_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != JL_OK:
+        raise JLError(status, where)
+
+
+def _stream(t: torch.Tensor | None = None, stream=None):
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libjlkey works on CUDA tensors only (no CPU fallback)")
+
+
+# --------------------------------------------------------------------------
+
+def jl_sketch_init(m: int, d: int, seed: int = 0, device=None, out=None,
+                   stream=None) -> torch.Tensor:
+    """The m x d bf16 Gaussian sketch regenerated from ``seed``."""
+    if out is None:
+        out = torch.empty((m, d), dtype=torch.bfloat16,
+                          device=device if device is not None else "cuda")
+    _need_cuda(out)
+    assert out.dtype == torch.bfloat16 and out.is_contiguous() and out.shape == (m, d)
+    _check(load().jl_sketch_init(_ptr(out), m, d, ctypes.c_uint64(seed),
+                                 _stream(out, stream)), "jl_sketch_init")
+    return out
+
+
+def _quantize(name, K, S, signs, norms, stream):
+    L = load()
+    if K.dim() != 2:
+        K = K.reshape(-1, K.shape[-1])
+    n, d = K.shape
+    m = S.shape[0]
+    _need_cuda(K, S)
+    if K.stride(1) != 1:
+        raise ValueError("keys must have unit stride along d")
+    if K.dtype == torch.bfloat16:
+        kt = JL_BF16
+    elif K.dtype == torch.float32:
+        kt = JL_F32
+    else:
+        raise TypeError(f"unsupported key dtype {K.dtype}")
+    assert S.dtype == torch.bfloat16 and S.is_contiguous() and S.shape[1] == d
+    if signs is None:
+        signs = torch.empty((n, m // 32), dtype=torch.int32, device=K.device)
+    if norms is None:
+        norms = torch.empty((n,), dtype=torch.float16, device=K.device)
+    assert signs.dtype == torch.int32 and signs.is_contiguous() and signs.numel() == n * (m // 32)
+    assert norms.dtype == torch.float16 and norms.is_contiguous() and norms.numel() == n
+    _check(getattr(L, name)(_ptr(K), kt, n, K.stride(0) if n > 0 else d, _ptr(S),
+                            m, d, _ptr(signs), _ptr(norms), _stream(K, stream)),
+           name)
+    return signs, norms
+
+
+def jl_quantize_keys(K, S, signs=None, norms=None, stream=None):
+    """Sign codes and fp16 norms of the rows of K ([..., d], bf16 or fp32)."""
+    return _quantize("jl_quantize_keys", K, S, signs, norms, stream)
+
+
+def jl_quantize_keys_simt(K, S, signs=None, norms=None, stream=None):
+    """Same as jl_quantize_keys, computed on the SIMT cores."""
+    return _quantize("jl_quantize_keys_simt", K, S, signs, norms, stream)
+
+
+def jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int:
+    return int(load().jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d))
+
+
+def jl_decode_attention(Q, S, signs, norms, V, softmax_scale=None, out=None,
+                        scores=None, want_scores=False, workspace=None,
+                        stream=None):
+    """One decode step over compressed keys.
+
+    Q [B, Hq, d] (bf16/fp32); signs [B, Hkv, T, m/32] int32; norms [B, Hkv, T]
+    fp16; V [B, Hkv, T, d] bf16.  Returns out [B, Hq, d] bf16, or
+    (out, scores [B, Hq, T] fp32) when ``want_scores`` (or ``scores`` given).
+    """
+    L = load()
+    B, Hq, d = Q.shape
+    Bv, Hkv, T, dv = V.shape
+    m = S.shape[0]
+    _need_cuda(Q, S, signs, norms, V)
+    assert Bv == B and dv == d
+    assert signs.shape == (B, Hkv, T, m // 32) and signs.dtype == torch.int32
+    assert norms.shape == (B, Hkv, T) and norms.dtype == torch.float16
+    assert V.dtype == torch.bfloat16
+    for t in (Q, S, signs, norms, V):
+        if not t.is_contiguous():
+            raise ValueError("decode inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    if Q.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"unsupported query dtype {Q.dtype}")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=Q.device)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
+    need = jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_decode_attention(_ptr(Q), qt, _ptr(S), _ptr(signs), _ptr(norms),
+                                 _ptr(V), B, Hq, Hkv, T, m, d,
+                                 ctypes.c_float(softmax_scale), _ptr(out),
+                                 _ptr(scores), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream(Q, stream)),
+           "jl_decode_attention")
+    if scores is not None:
+        return out, scores
+    return out
+
+
+def jl_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    code = ctypes.c_int(0)
+    st = load().jl_device_error(ctypes.byref(code), _stream(None, stream))
+    if st not in (JL_OK, JL_ERR_DEVICE):
+        raise JLError(st, "jl_device_error")
+    return int(code.value)
+
+
+def jl_bf16_from_f64(x: float) -> int:
+    return int(load().jl_bf16_from_f64(float(x)))

@@ -1,0 +1,201 @@
+// api.cu -- the extern "C" entry points of libjlkey (include/jlkey.h).
+//
+// Every entry point validates its arguments on the host before launching
+// anything and returns a status code; no exception crosses the boundary.
+#include "jl_common.cuh"
+#include "jl_internal.h"
+
+#include <mutex>
+
+namespace jlk {
+
+__device__ int g_device_error = 0;
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_attr_mu;
+int g_sm_count[kMaxDevices];
+int g_smem_optin[kMaxDevices];
+int *g_err_ptr[kMaxDevices];
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return dev;
+}
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_sm_count[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess || v <= 0)
+      v = 148;
+    g_sm_count[dev] = v;
+  }
+  return g_sm_count[dev];
+}
+
+int *device_error_ptr() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+int device_max_smem_optin() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 227 * 1024;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_smem_optin[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                               dev) != cudaSuccess || v <= 0)
+      v = 227 * 1024;
+    g_smem_optin[dev] = v;
+  }
+  return g_smem_optin[dev];
+}
+
+}  // namespace jlk
+
+namespace {
+
+bool aligned(const void *p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+bool supported_md(int m, int d) {
+  return (d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512);
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? JL_OK : JL_ERR_CUDA; }
+
+int validate_quantize(const void *K, jl_dtype kt, int64_t n, int64_t ldk,
+                      const uint16_t *S, int m, int d, const uint32_t *signs,
+                      const uint16_t *norms) {
+  if (kt != JL_BF16 && kt != JL_F32) return JL_ERR_INVALID_ARG;
+  if (n < 0) return JL_ERR_INVALID_ARG;
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (n == 0) return JL_OK;
+  if (!K || !S || !signs || !norms) return JL_ERR_INVALID_ARG;
+  if (ldk < d) return JL_ERR_INVALID_ARG;
+  const size_t esz = (kt == JL_F32) ? 4 : 2;
+  if (!aligned(K, 16) || ((size_t)ldk * esz) % 16 != 0) return JL_ERR_INVALID_ARG;
+  if (!aligned(S, 16) || !aligned(signs, 16) || !aligned(norms, 2))
+    return JL_ERR_INVALID_ARG;
+  return JL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *jl_status_string(int status) {
+  switch (status) {
+    case JL_OK: return "ok";
+    case JL_ERR_INVALID_ARG: return "invalid argument (null pointer, bad size or misaligned buffer)";
+    case JL_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128, m one of 64/128/256/512)";
+    case JL_ERR_WORKSPACE: return "workspace missing or smaller than jl_decode_workspace_bytes()";
+    case JL_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case JL_ERR_DEVICE: return "a kernel reported a device-side fault";
+    default: return "unknown status";
+  }
+}
+
+int jl_sketch_init(uint16_t *S, int m, int d, uint64_t seed,
+                   jl_stream_t stream) {
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (!S || !aligned(S, 16)) return JL_ERR_INVALID_ARG;
+  return from_cuda(jlk::launch_sketch(S, m, d, seed, (cudaStream_t)stream));
+}
+
+int jl_quantize_keys_simt(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                          int64_t key_stride, const uint16_t *S, int m, int d,
+                          uint32_t *signs, uint16_t *norms,
+                          jl_stream_t stream) {
+  int st = validate_quantize(K, key_dtype, n_keys, key_stride, S, m, d, signs,
+                             norms);
+  if (st != JL_OK || n_keys == 0) return st;
+  return from_cuda(jlk::launch_quantize_simt(K, key_dtype == JL_F32, n_keys,
+                                             key_stride, S, m, d, signs, norms,
+                                             (cudaStream_t)stream));
+}
+
+int jl_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                     int64_t key_stride, const uint16_t *S, int m, int d,
+                     uint32_t *signs, uint16_t *norms, jl_stream_t stream) {
+  int st = validate_quantize(K, key_dtype, n_keys, key_stride, S, m, d, signs,
+                             norms);
+  if (st != JL_OK || n_keys == 0) return st;
+  if (key_dtype == JL_BF16 && jlk::quantize_tc_supported(m, d, key_stride, K)) {
+    return from_cuda(jlk::launch_quantize_tc(
+        reinterpret_cast<const uint16_t *>(K), n_keys, key_stride, S, m, d,
+        signs, norms, (cudaStream_t)stream));
+  }
+  return from_cuda(jlk::launch_quantize_simt(K, key_dtype == JL_F32, n_keys,
+                                             key_stride, S, m, d, signs, norms,
+                                             (cudaStream_t)stream));
+}
+
+size_t jl_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m,
+                                 int d) {
+  jlk::DecodePlan p;
+  if (B == 0) return 0;
+  if (!jlk::make_decode_plan(B, Hq, Hkv, T, m, d, &p)) return 0;
+  return p.total_bytes;
+}
+
+int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                        const uint32_t *signs, const uint16_t *norms,
+                        const uint16_t *V, int B, int Hq, int Hkv, int64_t T,
+                        int m, int d, float softmax_scale, uint16_t *out,
+                        float *scores, void *workspace, size_t workspace_bytes,
+                        jl_stream_t stream) {
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0)
+    return JL_ERR_INVALID_ARG;
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;  // NaN
+  if (B == 0) return JL_OK;
+  if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(S, 16) || !aligned(signs, 16) ||
+      !aligned(norms, 2) || !aligned(V, 16) || !aligned(out, 4) ||
+      (scores && !aligned(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  jlk::DecodePlan p;
+  if (!jlk::make_decode_plan(B, Hq, Hkv, T, m, d, &p)) return JL_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
+    return JL_ERR_WORKSPACE;
+  return from_cuda(jlk::launch_decode(p, Q, q_dtype == JL_F32, S, signs, norms,
+                                      V, softmax_scale, out, scores, workspace,
+                                      (cudaStream_t)stream));
+}
+
+int jl_device_error(int *code, jl_stream_t stream) {
+  if (!code) return JL_ERR_INVALID_ARG;
+  *code = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    return JL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, jlk::g_device_error, sizeof(int)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(jlk::g_device_error, &zero, sizeof(int)) !=
+        cudaSuccess)
+      return JL_ERR_CUDA;
+  }
+  *code = v;
+  return v ? JL_ERR_DEVICE : JL_OK;
+}
+
+}  // extern "C"

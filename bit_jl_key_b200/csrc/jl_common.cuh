@@ -1,0 +1,106 @@
+// jl_common.cuh -- internal helpers shared by the libjlkey kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/jlkey.h"
+
+namespace jlk {
+
+// Device error word (one per device, defined in api.cu).  Kernels never trap:
+// a kernel that detects a fault (a bounded wait that ran out, an impossible
+// index) records a code through the pointer it was given (first fault wins)
+// and returns early.  device_error_ptr() is the word's device address for the
+// current device.
+int *device_error_ptr();
+
+enum DeviceErr : int {
+  DERR_NONE = 0,
+  DERR_TC_WAIT_TIMEOUT = 1,    // tensor-core quantizer: a pipeline wait ran out
+  DERR_TC_TMEM_ALLOC = 2,      // tensor-core quantizer: TMEM allocation failed
+  DERR_DECODE_PLAN = 3,        // decode: inconsistent work split
+};
+
+__device__ __forceinline__ void record_device_error(int *err, int code) {
+  atomicCAS(err, 0, code);
+}
+
+// Number of SMs of the current device (cached per device, thread-safe).
+int device_sm_count();
+// Max dynamic shared memory per block (opt-in) of the current device.
+int device_max_smem_optin();
+
+// ---------------------------------------------------------------------------
+// bf16 helpers on raw bit patterns.
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+// Pack two floats into a bf16x2 register (lo -> bits 0..15), round to nearest.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float bf16_round_f32(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_80+ instructions that sm_100a keeps).
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte async copy global -> shared, L2 only; src_bytes < 16 zero-fills.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src,
+                                            int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// 8-byte async copy global -> shared; src_bytes < 8 zero-fills.
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void *src,
+                                           int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// D[16x8] += A[16x16] * B[16x8], bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0,
+                                               uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four transposed 8x8 b16 matrices from shared memory.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t &r0,
+                                                  uint32_t &r1, uint32_t &r2,
+                                                  uint32_t &r3) {
+  asm volatile(
+      "ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+}  // namespace jlk

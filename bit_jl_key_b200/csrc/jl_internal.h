@@ -1,0 +1,54 @@
+// jl_internal.h -- launchers behind the C ABI (host side, internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/jlkey.h"
+
+namespace jlk {
+
+cudaError_t launch_sketch(uint16_t *S, int m, int d, uint64_t seed,
+                          cudaStream_t stream);
+
+// SIMT quantizer: any supported (m, d), bf16 or fp32 keys.
+cudaError_t launch_quantize_simt(const void *K, bool keys_f32, int64_t n,
+                                 int64_t ldk, const uint16_t *S, int m, int d,
+                                 uint32_t *signs, uint16_t *norms,
+                                 cudaStream_t stream);
+
+// Tensor-core (tcgen05 + TMA) quantizer for bf16 keys.  Returns
+// cudaErrorNotSupported when the shape is outside its envelope, in which case
+// the caller falls back to the SIMT path.
+cudaError_t launch_quantize_tc(const uint16_t *K, int64_t n, int64_t ldk,
+                               const uint16_t *S, int m, int d,
+                               uint32_t *signs, uint16_t *norms,
+                               cudaStream_t stream);
+bool quantize_tc_supported(int m, int d, int64_t ldk, const void *K);
+
+// Decode: work split shared by the workspace query and the launch.
+struct DecodePlan {
+  int B, Hq, Hkv, m, d;
+  int64_t T;
+  int G;         // query heads per KV head
+  int HG;        // head groups per KV head (groups of at most 8 heads)
+  int units;     // B * Hkv * HG
+  int64_t nb_u;  // 32-key blocks per unit
+  int64_t NB;    // units * nb_u
+  int W;         // warps launched (each takes a contiguous run of blocks)
+  int slots;     // partial-state slots per unit
+  size_t u_bytes;        // fp32 query projections [B][Hq][m]
+  size_t partial_bytes;  // fp32 [units][slots][8][d + 2]
+  size_t total_bytes;
+};
+bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
+                      DecodePlan *plan);
+
+cudaError_t launch_decode(const DecodePlan &p, const void *Q, bool q_f32,
+                          const uint16_t *S, const uint32_t *signs,
+                          const uint16_t *norms, const uint16_t *V,
+                          float softmax_scale, uint16_t *out, float *scores,
+                          void *workspace, cudaStream_t stream);
+
+}  // namespace jlk

@@ -1,0 +1,185 @@
+/*
+ * jlkey.h -- C ABI of libjlkey: QJL sign-bit compression of attention keys
+ * and decode attention that reads only the compressed keys, on NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *  - "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+ *    Quantization", section "QJL: one bit, zero parameters, unbiased inner
+ *    products": a Gaussian sketch S with i.i.d. N(0,1) entries, regenerated
+ *    from a seed; the quantizer Q(x) = sign(S x); the dequantizer
+ *    Q^-1(z) = sqrt(pi/2)/d * S^T z; the estimator is unbiased (property 1)
+ *    with variance shrinking with the number of sketch rows (property 2).
+ *  - "QJL: 1-Bit Quantized JL Transform for KV Cache Quantization with Zero
+ *    Overhead", Abstract: quantize one vector (the key) with QJL and apply
+ *    the plain JL transform to the other (the query): the asymmetric
+ *    estimator.  No per-block zero point or scale is stored.
+ *  - same blog page, section "PolarQuant": the radius (norm) that a
+ *    direction code drops is stored once per vector in floating point.
+ *
+ * With m sketch rows (S is m x d) the library computes, per key k:
+ *     code(k) = sign(S k)       (m bits, 1 = non-negative)
+ *     norm(k) = ||k||_2         (IEEE binary16)
+ * and, per query q and key k, the score
+ *     s(q,k) = sqrt(pi/2)/m * norm(k) * sum_i (S q)_i * sign(S k)_i
+ * which estimates <q,k> (with m = d this is <q, Q^-1(Q(k))> * ||k||).  Decode
+ * attention returns  out = sum_t softmax_t(softmax_scale * s(q,k_t)) * v_t.
+ *
+ * Conventions for every entry point:
+ *  - Memory: every buffer is allocated and owned by the caller (device memory
+ *    unless stated).  The library allocates nothing, frees nothing and keeps
+ *    no pointer after it returns.
+ *  - Execution: work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and the call returns without synchronising,
+ *    except jl_device_error, which synchronises `stream`.
+ *  - Errors: a negative status is returned.  Argument errors are detected
+ *    before anything is launched.  JL_ERR_CUDA reports a failed launch.
+ *    Kernels never trap; a kernel that detects a fault sets a device error
+ *    word that jl_device_error reads and clears.
+ *  - Layouts: row-major, innermost index last.  bf16 values are passed as
+ *    uint16_t bit patterns, binary16 norms likewise.
+ *  - Supported shapes: d in {64, 128}; m in {64, 128, 256, 512}.
+ *  - Thread safety: entry points may be called concurrently from several host
+ *    threads; the only process-wide state is a per-device cache of device
+ *    attributes.
+ */
+#ifndef JLKEY_H
+#define JLKEY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JL_API __attribute__((visibility("default")))
+#else
+#define JL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream). */
+typedef struct CUstream_st *jl_stream_t;
+
+/* Element type of keys and queries. */
+typedef enum { JL_BF16 = 0, JL_F32 = 1 } jl_dtype;
+
+enum {
+    JL_OK = 0,
+    JL_ERR_INVALID_ARG = -1, /* null pointer, negative size, misalignment   */
+    JL_ERR_UNSUPPORTED = -2, /* a shape outside the supported set           */
+    JL_ERR_WORKSPACE = -3,   /* workspace pointer null or smaller than asked */
+    JL_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    JL_ERR_DEVICE = -5       /* a kernel reported a fault (jl_device_error) */
+};
+
+/* Human-readable text of a status code (static storage). */
+JL_API const char *jl_status_string(int status);
+
+/*
+ * jl_sketch_init -- the Gaussian sketch S, regenerated from `seed`.
+ * Defines: "The Geometry of Forgetting ...", section "QJL: one bit, zero
+ * parameters, unbiased inner products" (S with i.i.d. N(0,1) entries, shared
+ * by every vector and rebuilt from a seed).
+ *   S    : out, device, m x d bf16, row-major, 16-byte aligned.
+ *   Element e = i*d + j is the Box-Muller normal (cosine branch) of the
+ *   SplitMix64 outputs 2e and 2e+1 of `seed` (outputs taken from the
+ *   generator's counter form: output n = mix(seed + (n+1) * 0x9E3779B97F4A7C15)),
+ *   each mapped to the uniform ((x >> 12) + 1/2) * 2^-52, then rounded to
+ *   bf16 (nearest, ties to even).
+ * Errors: JL_ERR_INVALID_ARG (S null/misaligned), JL_ERR_UNSUPPORTED (m, d).
+ */
+JL_API int jl_sketch_init(uint16_t *S, int m, int d, uint64_t seed,
+                   jl_stream_t stream);
+
+/*
+ * jl_quantize_keys -- code(k) and norm(k) for n_keys keys.
+ * Defines: same section, quantizer equation Q(x) = sign(S x), plus the norm
+ * kept beside the code ("PolarQuant" section: one radius per vector).
+ *   K          : in, device, n_keys rows of d elements of `key_dtype`, row r
+ *                starting at element r * key_stride; 16-byte aligned base,
+ *                key_stride * sizeof(element) a multiple of 16 bytes.
+ *   key_dtype  : JL_BF16 (tensor-core path) or JL_F32.
+ *   S          : in, device, m x d bf16 from jl_sketch_init (16-byte aligned).
+ *   signs      : out, device, n_keys x (m/32) uint32, 16-byte aligned.  Bit i
+ *                of the code is bit (i % 32) of word i / 32 (LSB first) and
+ *                is 1 iff (S k)_i >= 0.
+ *   norms      : out, device, n_keys binary16 (||k||_2 rounded to nearest),
+ *                2-byte aligned.
+ * n_keys == 0 is a no-op.  Projections are accumulated in fp32 from exact
+ * bf16 x bf16 products; a coordinate with |(S k)_i| within the fp32
+ * accumulation error of 0 may take either sign.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_CUDA.
+ */
+JL_API int jl_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                     int64_t key_stride, const uint16_t *S, int m, int d,
+                     uint32_t *signs, uint16_t *norms, jl_stream_t stream);
+
+/*
+ * jl_quantize_keys_simt -- the same result as jl_quantize_keys computed with
+ * plain fp32 FMA on the SIMT cores (no tensor cores).  Serves fp32 keys and
+ * cross-checks the tensor-core path.  Same arguments and errors.
+ */
+JL_API int jl_quantize_keys_simt(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                          int64_t key_stride, const uint16_t *S, int m, int d,
+                          uint32_t *signs, uint16_t *norms,
+                          jl_stream_t stream);
+
+/*
+ * jl_decode_workspace_bytes -- device scratch that jl_decode_attention needs
+ * for these shapes (query projections and split-context partial softmax
+ * states).  Depends on the shapes only.  Returns 0 for unsupported shapes.
+ */
+JL_API size_t jl_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m,
+                                 int d);
+
+/*
+ * jl_decode_attention -- one decode step of attention over compressed keys.
+ * Defines: the asymmetric estimator ("QJL ..." Abstract; "The Geometry of
+ * Forgetting ...", QJL section, dequantizer equation with m rows, scaled by
+ * the stored norm) used as the attention logit, then softmax and the value
+ * sum.  Query head h reads KV head h / (Hq / Hkv).
+ *   Q        : in, device, B x Hq x d of `q_dtype` (one token per sequence),
+ *              16-byte aligned.
+ *   S        : in, device, m x d bf16 (the sketch the keys were coded with).
+ *   signs    : in, device, B x Hkv x T x (m/32) uint32 codes, 16-byte aligned.
+ *   norms    : in, device, B x Hkv x T binary16 key norms, 2-byte aligned.
+ *   V        : in, device, B x Hkv x T x d bf16 values, 16-byte aligned.
+ *   softmax_scale : logit = softmax_scale * s(q, k_t) (typically 1/sqrt(d)).
+ *   out      : out, device, B x Hq x d bf16, 4-byte aligned.
+ *   scores   : optional out (NULL to skip), device, B x Hq x T fp32: the
+ *              estimator s(q, k_t) before softmax_scale, 4-byte aligned.
+ *   workspace: device scratch of at least jl_decode_workspace_bytes(...),
+ *              256-byte aligned; contents on entry are ignored.
+ * B == 0 is a no-op.  T must be >= 1 (softmax over an empty context is
+ * undefined).  Hq must be a multiple of Hkv.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
+ * JL_ERR_CUDA.
+ */
+JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                        const uint32_t *signs, const uint16_t *norms,
+                        const uint16_t *V, int B, int Hq, int Hkv, int64_t T,
+                        int m, int d, float softmax_scale, uint16_t *out,
+                        float *scores, void *workspace, size_t workspace_bytes,
+                        jl_stream_t stream);
+
+/*
+ * jl_device_error -- synchronise `stream`, then read and clear the device
+ * error word of the current device (0 = no fault reported).  *code receives
+ * the word.  Returns JL_OK, JL_ERR_DEVICE when the word was non-zero, or
+ * JL_ERR_CUDA.
+ */
+JL_API int jl_device_error(int *code, jl_stream_t stream);
+
+/*
+ * jl_bf16_from_f64 -- host helper: the bf16 code (round to nearest, ties to
+ * even, directly from float64) that jl_sketch_init applies to each normal.
+ */
+JL_API uint16_t jl_bf16_from_f64(double x);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JLKEY_H */

@@ -1,0 +1,146 @@
+"""Host-side checks of libjlkey that need no GPU.
+
+The library must load, export every entry point include/jlkey.h declares, and
+reject bad arguments before launching anything.  The host copy of the
+sketch's bf16 rounding is compared with the oracle's rounding.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_jl_key_b200 as jl
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"JL_API\s+[\w\s\*]*?\b(jl_\w+)\s*\(", src)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_jl_key_b200 import build
+    build.build()
+    return jl.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(jl.EXPORTED)
+
+
+def test_status_strings(lib):
+    for st in (jl.JL_OK, jl.JL_ERR_INVALID_ARG, jl.JL_ERR_UNSUPPORTED,
+               jl.JL_ERR_WORKSPACE, jl.JL_ERR_CUDA, jl.JL_ERR_DEVICE):
+        s = jl.status_string(st)
+        assert s and s != "unknown status"
+    assert jl.status_string(12345) == "unknown status"
+
+
+def test_host_bf16_rounding_matches_oracle(lib):
+    rng = np.random.default_rng(0)
+    vals = list(rng.normal(size=2000)) + list(rng.normal(size=200) * 1e-38)
+    vals += [1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -40, -(1 + 2 ** -8),
+             0.0, -0.0, 3e38, -3.5e38, 2 ** -133, 2 ** -134, 3 * 2 ** -134, 1e-300]
+    for x in vals:
+        assert jl.jl_bf16_from_f64(float(x)) == oracle.f64_to_bf16_bits(float(x)), x
+
+
+def test_workspace_query(lib):
+    f = jl.jl_decode_workspace_bytes
+    assert f(8, 32, 8, 32768, 256, 128) > 8 * 32 * 256 * 4
+    assert f(1, 1, 1, 1024, 256, 128) > 0
+    assert f(0, 32, 8, 1024, 256, 128) == 0        # nothing to do
+    assert f(1, 6, 4, 1024, 256, 128) == 0         # Hq not a multiple of Hkv
+    assert f(1, 1, 1, 1024, 96, 128) == 0          # unsupported m
+    assert f(1, 1, 1, 1024, 256, 96) == 0          # unsupported d
+    assert f(1, 1, 1, 0, 256, 128) == 0            # empty context
+    # depends on shapes only
+    assert f(2, 16, 4, 777, 128, 64) == f(2, 16, 4, 777, 128, 64)
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p((1 << 20) + 2)
+
+
+def test_sketch_argument_errors(lib):
+    assert lib.jl_sketch_init(NULL, 256, 128, 0, NULL) == jl.JL_ERR_INVALID_ARG
+    assert lib.jl_sketch_init(MISALIGNED, 256, 128, 0, NULL) == jl.JL_ERR_INVALID_ARG
+    assert lib.jl_sketch_init(FAKE, 100, 128, 0, NULL) == jl.JL_ERR_UNSUPPORTED
+    assert lib.jl_sketch_init(FAKE, 256, 32, 0, NULL) == jl.JL_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["jl_quantize_keys", "jl_quantize_keys_simt"])
+def test_quantize_argument_errors(lib, name):
+    f = getattr(lib, name)
+    ok = dict(K=FAKE, kt=jl.JL_BF16, n=10, ldk=128, S=FAKE, m=256, d=128,
+              signs=FAKE, norms=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["K"], a["kt"], a["n"], a["ldk"], a["S"], a["m"], a["d"],
+                 a["signs"], a["norms"], NULL)
+
+    assert call(n=0) == jl.JL_OK                     # empty: no-op
+    assert call(n=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(K=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(S=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(signs=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(norms=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(K=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(ldk=100) == jl.JL_ERR_INVALID_ARG     # < d
+    assert call(ldk=130) == jl.JL_ERR_INVALID_ARG     # 260 B not a 16 B multiple
+    assert call(kt=7) == jl.JL_ERR_INVALID_ARG
+    assert call(m=96) == jl.JL_ERR_UNSUPPORTED
+    assert call(d=80, ldk=80) == jl.JL_ERR_UNSUPPORTED
+
+
+def test_decode_argument_errors(lib):
+    f = lib.jl_decode_attention
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, S=FAKE, signs=FAKE, norms=FAKE, V=FAKE,
+              B=2, Hq=8, Hkv=2, T=100, m=256, d=128, scale=0.1, out=FAKE,
+              scores=NULL, ws=FAKE, wsb=1 << 40)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["Q"], a["qt"], a["S"], a["signs"], a["norms"], a["V"],
+                 a["B"], a["Hq"], a["Hkv"], a["T"], a["m"], a["d"],
+                 ctypes.c_float(a["scale"]), a["out"], a["scores"], a["ws"],
+                 a["wsb"], NULL)
+
+    assert call(B=0) == jl.JL_OK                     # empty batch: no-op
+    assert call(T=0) == jl.JL_ERR_INVALID_ARG        # empty context
+    assert call(Hq=6, Hkv=4) == jl.JL_ERR_INVALID_ARG
+    assert call(Hkv=0) == jl.JL_ERR_INVALID_ARG
+    assert call(qt=5) == jl.JL_ERR_INVALID_ARG
+    assert call(m=48) == jl.JL_ERR_UNSUPPORTED
+    assert call(d=256) == jl.JL_ERR_UNSUPPORTED
+    for k in ("Q", "S", "signs", "norms", "V", "out"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(V=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(signs=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == jl.JL_ERR_INVALID_ARG
+    assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
+    need = jl.jl_decode_workspace_bytes(2, 8, 2, 100, 256, 128)
+    assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == jl.JL_ERR_WORKSPACE
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        jl.jl_quantize_keys(torch.zeros(4, 128, dtype=torch.bfloat16),
+                            torch.zeros(256, 128, dtype=torch.bfloat16))
