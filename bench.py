@@ -56,7 +56,12 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def pick_workload(name: str) -> workloads.Workload:
+def pick_workload(name: str, batch: int = 0) -> workloads.Workload:
+    w = _pick(name)
+    return w.with_(B=batch) if batch else w
+
+
+def _pick(name: str) -> workloads.Workload:
     if name.startswith("sweep"):
         # sweep-m<M>-d<D>
         m = int(name.split("-m")[1].split("-")[0])
@@ -168,7 +173,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload)
+    w = pick_workload(args.workload, args.batch)
     decode = w.name != "prefill"
     peak, peak_kind = load_peaks()
 
@@ -386,7 +391,7 @@ def time_oracle(w, steps=1, warmup=0):
 
 
 def run_reference(args, rank, world):
-    w = pick_workload(args.workload)
+    w = pick_workload(args.workload, args.batch)
     if rank != 0:
         return None
     cb = time_oracle(w, steps=args.steps, warmup=args.warmup)
@@ -416,6 +421,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -444,7 +451,7 @@ def main():
         # the oracle runs before any GPU work on rank 0 (bounded sample)
         cb = None
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cb = time_oracle(pick_workload(args.workload), steps=1)
+            cb = time_oracle(pick_workload(args.workload, args.batch), steps=1)
         line = run_ours(args, rank, world, local_rank)
         if cb is not None:
             line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
