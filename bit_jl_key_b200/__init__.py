@@ -38,10 +38,13 @@ JL_ERR_UNSUPPORTED = -2
 JL_ERR_WORKSPACE = -3
 JL_ERR_CUDA = -4
 JL_ERR_DEVICE = -5
+JL_ERR_SCRATCH_LIMIT = -6
+DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_quantize_keys_simt", "jl_decode_workspace_bytes",
-            "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64")
+            "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64",
+            "jl_decode_attention_noalloc")
 
 _lib = None
 
@@ -77,6 +80,10 @@ def load():
     L.jl_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32,
                                       i64, i32, i32, ctypes.c_float, vp, vp,
                                       vp, sz, vp]
+    L.jl_decode_attention_noalloc.restype = i32
+    L.jl_decode_attention_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32,
+                                              i32, i64, i32, i32, ctypes.c_float,
+                                              vp, vp, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.jl_bf16_from_f64.restype = ctypes.c_uint16
@@ -208,6 +215,43 @@ def jl_decode_attention(Q, S, signs, norms, V, softmax_scale=None, out=None,
                                  workspace.numel() * workspace.element_size(),
                                  _stream(Q, stream)),
            "jl_decode_attention")
+    if scores is not None:
+        return out, scores
+    return out
+
+
+def jl_decode_attention_noalloc(Q, S, signs, norms, V, softmax_scale=None,
+                                out=None, scores=None, want_scores=False,
+                                stream=None):
+    """jl_decode_attention without a workspace, for callers that cannot
+    allocate device memory where they call it (plugins inside an engine that
+    owns all device memory, latency-critical paths).  The library's static
+    device scratch (DECODE_STATIC_SCRATCH_BYTES, held by every GPU that loads
+    the library) replaces the workspace; calls must not overlap on a GPU, and
+    shapes needing more scratch raise JLError(JL_ERR_SCRATCH_LIMIT).  Output
+    tensors passed in are used as given; when ``out``/``scores`` are None this
+    wrapper creates them with torch, as it would for any caller."""
+    L = load()
+    B, Hq, d = Q.shape
+    _, Hkv, T, _ = V.shape
+    m = S.shape[0]
+    _need_cuda(Q, S, signs, norms, V)
+    for t in (Q, S, signs, norms, V):
+        if not t.is_contiguous():
+            raise ValueError("decode inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=Q.device)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
+    _check(L.jl_decode_attention_noalloc(_ptr(Q), qt, _ptr(S), _ptr(signs),
+                                         _ptr(norms), _ptr(V), B, Hq, Hkv, T,
+                                         m, d, ctypes.c_float(softmax_scale),
+                                         _ptr(out), _ptr(scores),
+                                         _stream(Q, stream)),
+           "jl_decode_attention_noalloc")
     if scores is not None:
         return out, scores
     return out

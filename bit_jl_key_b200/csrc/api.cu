@@ -107,6 +107,7 @@ const char *jl_status_string(int status) {
     case JL_ERR_WORKSPACE: return "workspace missing or smaller than jl_decode_workspace_bytes()";
     case JL_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case JL_ERR_DEVICE: return "a kernel reported a device-side fault";
+    case JL_ERR_SCRATCH_LIMIT: return "shapes need more scratch than the static decode scratch (JL_DECODE_STATIC_SCRATCH_BYTES); use jl_decode_attention with a workspace";
     default: return "unknown status";
   }
 }

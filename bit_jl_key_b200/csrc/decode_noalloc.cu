@@ -1,0 +1,90 @@
+// decode_noalloc.cu -- decode attention for callers that cannot allocate.
+//
+// jl_decode_attention needs device scratch (the query projections and the
+// per-split softmax states) that its caller allocates.  Some callers cannot
+// allocate device memory where they call us: a plugin running inside an
+// engine that owns all device memory through its own pool and hands the
+// plugin no allocator, or code on a latency-critical path where cudaMalloc
+// and cudaFree would stall the device.  jl_decode_attention_noalloc serves
+// them: it runs the same kernels with a scratch buffer that lives in this
+// file as a statically sized __device__ array, so the call allocates nothing.
+//
+// Costs and rules of that design:
+//  - every GPU that loads the library holds JL_DECODE_STATIC_SCRATCH_BYTES
+//    of device memory for the array until the process exits;
+//  - all calls share the one array, so two calls whose kernels overlap on a
+//    GPU (for example on two streams) race and corrupt each other's result;
+//  - shapes whose scratch would exceed the array are rejected before any
+//    launch;
+//  - the array's device address is looked up once per device, on the first
+//    call made with that device current.
+#include "jl_common.cuh"
+#include "jl_internal.h"
+
+#include <mutex>
+
+namespace {
+
+static __device__ __align__(256) unsigned char
+    g_decode_scratch[JL_DECODE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxDevices];
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// array's name stands for a host-side shadow, not device memory, so kernels
+// must be given the address the runtime reports for the current device.
+cudaError_t scratch_address(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int jl_decode_attention_noalloc(
+    const void *Q, jl_dtype q_dtype, const uint16_t *S, const uint32_t *signs,
+    const uint16_t *norms, const uint16_t *V, int B, int Hq, int Hkv,
+    int64_t T, int m, int d, float softmax_scale, uint16_t *out,
+    float *scores, jl_stream_t stream) {
+  // same argument checks as jl_decode_attention, minus the workspace
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0)
+    return JL_ERR_INVALID_ARG;
+  if (!((d == 64 || d == 128) &&
+        (m == 64 || m == 128 || m == 256 || m == 512)))
+    return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
+  if (B == 0) return JL_OK;
+  if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
+  auto misaligned = [](const void *p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) != 0;
+  };
+  if (misaligned(Q, 16) || misaligned(S, 16) || misaligned(signs, 16) ||
+      misaligned(norms, 2) || misaligned(V, 16) || misaligned(out, 4) ||
+      (scores && misaligned(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  jlk::DecodePlan p;
+  if (!jlk::make_decode_plan(B, Hq, Hkv, T, m, d, &p)) return JL_ERR_UNSUPPORTED;
+  if (p.total_bytes > (size_t)JL_DECODE_STATIC_SCRATCH_BYTES)
+    return JL_ERR_SCRATCH_LIMIT;
+  void *scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return JL_ERR_CUDA;
+  // Nothing in the scratch has to start at zero: the kernels read only
+  // elements written earlier in the same call.
+  const cudaError_t e = jlk::launch_decode(p, Q, q_dtype == JL_F32, S, signs,
+                                           norms, V, softmax_scale, out, scores,
+                                           scratch, (cudaStream_t)stream);
+  return e == cudaSuccess ? JL_OK : JL_ERR_CUDA;
+}

@@ -71,7 +71,8 @@ enum {
     JL_ERR_UNSUPPORTED = -2, /* a shape outside the supported set           */
     JL_ERR_WORKSPACE = -3,   /* workspace pointer null or smaller than asked */
     JL_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
-    JL_ERR_DEVICE = -5       /* a kernel reported a fault (jl_device_error) */
+    JL_ERR_DEVICE = -5,      /* a kernel reported a fault (jl_device_error) */
+    JL_ERR_SCRATCH_LIMIT = -6 /* shapes need more than the static scratch    */
 };
 
 /* Human-readable text of a status code (static storage). */
@@ -163,6 +164,38 @@ JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *
                         int m, int d, float softmax_scale, uint16_t *out,
                         float *scores, void *workspace, size_t workspace_bytes,
                         jl_stream_t stream);
+
+/*
+ * jl_decode_attention_noalloc -- jl_decode_attention for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this entry point
+ * exists for deployment, not for the method.
+ * Some callers cannot call cudaMalloc where they call this library: plugins
+ * hosted by an engine that owns all device memory through its own pool and
+ * gives them no allocator, and code on latency-critical paths where
+ * allocating or freeing would stall the device.  This variant takes the same
+ * inputs and outputs as jl_decode_attention (same meaning, layout, alignment
+ * and errors) but no workspace: its scratch is a statically sized device
+ * array inside the library, JL_DECODE_STATIC_SCRATCH_BYTES long, which every
+ * GPU that loads the library holds until the process exits.  It allocates
+ * and frees nothing.
+ *  - Limit: shapes for which jl_decode_workspace_bytes(...) exceeds
+ *    JL_DECODE_STATIC_SCRATCH_BYTES are rejected with JL_ERR_SCRATCH_LIMIT
+ *    before anything is launched (use jl_decode_attention with a workspace).
+ *  - Sharing: every call uses the same array, which keeps the previous call's
+ *    contents (no part of it needs to start at zero).  Calls whose kernels
+ *    overlap on a GPU, e.g. on two streams, race on it and give wrong
+ *    results: serialise them.
+ *  - Set-up: the first call made with a given device current looks up the
+ *    array's device address on that device; make that first call before any
+ *    stream capture.
+ */
+#define JL_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,
+                                       const uint16_t *S, const uint32_t *signs,
+                                       const uint16_t *norms, const uint16_t *V,
+                                       int B, int Hq, int Hkv, int64_t T, int m,
+                                       int d, float softmax_scale, uint16_t *out,
+                                       float *scores, jl_stream_t stream);
 
 /*
  * jl_device_error -- synchronise `stream`, then read and clear the device
