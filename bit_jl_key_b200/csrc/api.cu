@@ -137,7 +137,7 @@ int jl_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
   int st = validate_quantize(K, key_dtype, n_keys, key_stride, S, m, d, signs,
                              norms);
   if (st != JL_OK || n_keys == 0) return st;
-  if (key_dtype == JL_BF16 && jlk::quantize_tc_supported(m, d, key_stride, K)) {
+  if (key_dtype == JL_BF16 && jlk::quantize_tc_supported(m, d, n_keys, key_stride, K)) {
     return from_cuda(jlk::launch_quantize_tc(
         reinterpret_cast<const uint16_t *>(K), n_keys, key_stride, S, m, d,
         signs, norms, (cudaStream_t)stream));

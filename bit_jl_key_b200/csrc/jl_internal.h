@@ -25,7 +25,7 @@ cudaError_t launch_quantize_tc(const uint16_t *K, int64_t n, int64_t ldk,
                                const uint16_t *S, int m, int d,
                                uint32_t *signs, uint16_t *norms,
                                cudaStream_t stream);
-bool quantize_tc_supported(int m, int d, int64_t ldk, const void *K);
+bool quantize_tc_supported(int m, int d, int64_t n, int64_t ldk, const void *K);
 
 // Decode: work split shared by the workspace query and the launch.
 struct DecodePlan {

@@ -1,20 +1,472 @@
-// quantize_tc.cu -- tensor-core (tcgen05 + TMA) QJL quantizer for bf16 keys.
+// quantize_tc.cu -- QJL key codes on the 5th-generation tensor cores.
+//
+// Quantizer Q(k) = sign(S k) of "The Geometry of Forgetting: How Three Papers
+// Cracked KV Cache Quantization", section "QJL: one bit, zero parameters,
+// unbiased inner products", for a tile of 128 keys at a time, plus the key
+// norm kept beside the code (same page, "PolarQuant" section).
+//
+// The projection P = K S^T (M = 128 keys, N = m sketch rows, K = d) is a
+// dense bf16 contraction: tcgen05.mma with both operands in shared memory
+// (TMA-loaded, 128-byte swizzle, K-major) and the fp32 accumulator in tensor
+// memory.  Only the sign of each accumulator element survives, so P never
+// leaves the SM.
+//
+// One persistent CTA per SM, 10 warps with fixed roles:
+//   warp 0     TMA producer: S once, then one 128 x d key tile per stage of
+//              a STAGES-deep shared-memory ring.
+//   warp 1     owns the TMEM allocation; lane 0 issues the MMAs of a tile
+//              into one of two TMEM accumulators (one for m = 512) and
+//              commits them to the barriers that free the key stage and
+//              publish the accumulator.
+//   warps 2-5  sign epilogue: warp w reads TMEM lanes 32*(w%4).. (its lane
+//              quadrant), 32 columns per tcgen05.ld, and packs the 32 sign
+//              bits of a word with one funnel shift per value; then releases
+//              the accumulator and stores the code row.
+//   warps 6-9  norm epilogue: each thread sums the squares of one key row
+//              straight from the swizzled stage in shared memory, then frees
+//              the stage (together with the MMA commit).
+// Every mbarrier wait is bounded (about 2 s of GPU time); a wait that runs
+// out records DERR_TC_WAIT_TIMEOUT in the device error word, tells the other
+// roles to stop, and the CTA still drains its copies and frees its TMEM.
 #include "jl_common.cuh"
 #include "jl_internal.h"
 
-namespace jlk {
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
-bool quantize_tc_supported(int m, int d, int64_t ldk, const void *K) {
-  (void)m; (void)d; (void)ldk; (void)K;
-  return false;
+#include <mutex>
+
+namespace jlk {
+namespace tc {
+
+constexpr int BM = 128;           // keys per tile (MMA M)
+constexpr int NWARPS = 10;
+constexpr int THREADS = NWARPS * 32;
+constexpr int SMEM_BUDGET = 220 * 1024;
+constexpr unsigned long long WAIT_NS = 2000000000ull;  // bounded waits: 2 s
+
+template <int M, int D>
+struct Cfg {
+  static constexpr int KCH = D / 64;                 // 128-byte swizzle columns
+  static constexpr int A_CHUNK = BM * 128;           // one swizzle column of a tile
+  static constexpr int A_STAGE = BM * D * 2;
+  static constexpr int S_CHUNK = M * 128;
+  static constexpr int S_BYTES = M * D * 2;
+  static constexpr int NH = (M > 256) ? 2 : 1;       // MMAs per K step (N halves)
+  static constexpr int NMMA = M / NH;                // N of one MMA (<= 256)
+  static constexpr int ACC = (M > 256) ? 1 : 2;      // accumulator buffers
+  static constexpr int TMEM_COLS = (ACC * M < 32) ? 32 : ACC * M;
+  static constexpr int STAGES_RAW = (SMEM_BUDGET - S_BYTES) / A_STAGE;
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  static constexpr int WORDS = M / 32;
+  // dynamic smem: [S][A stages][barriers]
+  static constexpr int OFF_A = S_BYTES;
+  static constexpr int OFF_BAR = OFF_A + STAGES * A_STAGE;
+  static constexpr int NBAR = 2 * STAGES + 2 * ACC + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + align slack
+  static_assert(STAGES >= 2, "key ring needs two stages");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "tmem");
+};
+
+struct Params {
+  int64_t n;
+  int64_t num_tiles;
+  uint32_t *signs;
+  uint16_t *norms;
+  int *err;
+};
+
+// --------------------------------------------------------------------------
+// PTX wrappers
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map,
+                                            int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// K-major operand, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);          // start address
+  d |= (uint64_t)1u << 16;                          // leading byte offset (unused)
+  d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset
+  d |= (uint64_t)1u << 46;                          // descriptor version
+  d |= (uint64_t)2u << 61;                          // SWIZZLE_128B
+  return d;
+}
+__device__ __forceinline__ void mma_bf16_ss(uint32_t tmem_d, uint64_t adesc,
+                                            uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+        "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+        "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+// Bounded wait on a barrier phase; false when the wait ran out or another
+// role gave up (then the error word is set and the shared abort flag raised).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
+                                           volatile int *abort_flag, int *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > WAIT_NS) {
+        *abort_flag = 1;
+        record_device_error(err, DERR_TC_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+template <int M, int D>
+__global__ void __launch_bounds__(THREADS, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_s,
+                       const Params p) {
+  using C = Cfg<M, D>;
+  extern __shared__ uint8_t tc_smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  const uint32_t raw = smem_u32(tc_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = tc_smem_raw + (base - raw);
+  const uint32_t sS = base;
+  const uint32_t sA = base + C::OFF_A;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + C::ACC + a); };
+  const uint32_t sfull_bar = bar0 + 8u * (2 * C::STAGES + 2 * C::ACC);
+  uint32_t *tmem_holder =
+      reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+  volatile int *abort_flag =
+      reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1 + 4);   // MMA commit + 4 norm warps
+    }
+    for (int a = 0; a < C::ACC; ++a) {
+      mbar_init(tfull_bar(a), 1);       // MMA commit
+      mbar_init(tempty_bar(a), 4);      // 4 sign warps
+    }
+    mbar_init(sfull_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+        "tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::"r"(
+            smem_u32(tmem_holder)),
+        "n"(C::TMEM_COLS)
+        : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int64_t ntiles = p.num_tiles;
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(sfull_bar, C::S_BYTES);
+      for (int kc = 0; kc < C::KCH; ++kc)
+        for (int h = 0; h < C::NH; ++h)
+          tma_load_2d(sS + kc * C::S_CHUNK + h * C::NMMA * 128, &tmap_s, kc * 64,
+                      h * C::NMMA, sfull_bar);
+      int64_t i = 0;
+      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        const int s = (int)(i % C::STAGES);
+        const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
+        if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.err)) break;
+        mbar_expect_tx(full_bar(s), C::A_STAGE);
+        for (int kc = 0; kc < C::KCH; ++kc)
+          tma_load_2d(sA + s * C::A_STAGE + kc * C::A_CHUNK, &tmap_k, kc * 64,
+                      (int)(tile * BM), full_bar(s));
+      }
+      // drain: the last stages issued must have landed before the CTA exits
+      const int64_t issued = i;
+      for (int64_t j = (issued > C::STAGES ? issued - C::STAGES : 0); j < issued; ++j) {
+        const int s = (int)(j % C::STAGES);
+        const uint32_t ph = (uint32_t)((j / C::STAGES) & 1);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(full_bar(s), ph) && globaltimer() - t0 < WAIT_NS) {
+        }
+      }
+      {
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(sfull_bar, 0) && globaltimer() - t0 < WAIT_NS) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4)                 // D: fp32
+                                 | (1u << 7) | (1u << 10)  // A, B: bf16
+                                 | ((uint32_t)(C::NMMA >> 3) << 17)  // N
+                                 | ((uint32_t)(BM >> 4) << 24);      // M
+      bool ok = wait_phase(sfull_bar, 0, abort_flag, p.err);
+      int64_t i = 0;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
+        const int s = (int)(i % C::STAGES);
+        const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
+        const int a = (int)(i % C::ACC);
+        const uint32_t aph = (uint32_t)((i / C::ACC) & 1);
+        if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err)) break;
+        if (!wait_phase(full_bar(s), ph, abort_flag, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+          const uint64_t adesc =
+              smem_desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
+#pragma unroll
+          for (int h = 0; h < C::NH; ++h) {
+            const uint64_t bdesc = smem_desc_sw128(
+                sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
+            mma_bf16_ss(tmem_base + a * M + h * C::NMMA, adesc, bdesc, idesc,
+                        kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(empty_bar(s));
+        mma_commit(tfull_bar(a));
+      }
+      // drain: the last accumulator's MMAs must be complete before TMEM is freed
+      if (i > 0) {
+        const int64_t j = i - 1;
+        const int a = (int)(j % C::ACC);
+        const uint32_t aph = (uint32_t)((j / C::ACC) & 1);
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(tfull_bar(a), aph) && globaltimer() - t0 < WAIT_NS) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---------------- sign epilogue (TMEM lane quadrant warp % 4)
+    const int q = warp & 3;
+    int64_t i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int a = (int)(i % C::ACC);
+      const uint32_t aph = (uint32_t)((i / C::ACC) & 1);
+      if (!wait_phase(tfull_bar(a), aph, abort_flag, p.err)) break;
+      __syncwarp();
+      tc_fence_after();
+      // 4 code words (128 columns) per step: at most 4 TMEM slices are live,
+      // whatever the number of sketch rows
+      constexpr int GW = C::WORDS < 4 ? C::WORDS : 4;
+      const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * M);
+      const int64_t row = tile * BM + 32 * q + lane;
+      uint32_t *dst = p.signs + row * C::WORDS;
+      const bool live = row < p.n;
+#pragma unroll 1
+      for (int w0 = 0; w0 < C::WORDS; w0 += GW) {
+        uint32_t words[GW];
+#pragma unroll
+        for (int w = 0; w < GW; ++w) {
+          uint32_t v[32];
+          tmem_ld32(trow + 32 * (w0 + w), v);
+          tmem_ld_wait();
+          uint32_t word = 0;
+#pragma unroll
+          for (int j = 31; j >= 0; --j) word = __funnelshift_l(v[j], word, 1);
+          words[w] = ~word;  // bit j = 1 iff column 32(w0+w) + j is >= 0
+        }
+        if (live) {
+          if constexpr (GW == 2)
+            *reinterpret_cast<uint2 *>(dst + w0) = make_uint2(words[0], words[1]);
+          else
+            *reinterpret_cast<uint4 *>(dst + w0) =
+                make_uint4(words[0], words[1], words[2], words[3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(a));
+    }
+  } else {
+    // ---------------- norm epilogue: rows 32*(warp-6) .. +31 of each tile
+    const int r = 32 * (warp - 6) + lane;
+    int64_t i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int s = (int)(i % C::STAGES);
+      const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
+      if (!wait_phase(full_bar(s), ph, abort_flag, p.err)) break;
+      float ss0 = 0.f, ss1 = 0.f;
+      const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + r * 128;
+#pragma unroll
+      for (int kc = 0; kc < C::KCH; ++kc) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(
+              rowp + kc * C::A_CHUNK + ((c ^ (r & 7)) << 4));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(w4[e] << 16);
+            const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+            ss0 = fmaf(lo, lo, ss0);
+            ss1 = fmaf(hi, hi, ss1);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+      const int64_t row = tile * BM + r;
+      if (row < p.n) p.norms[row] = __half_as_ushort(__float2half_rn(sqrtf(ss0 + ss1)));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
+                 "n"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------------------
+// host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] with row pitch `pitch_elems`, boxes of
+// 64 columns (128 B) x box_rows rows, 128-byte swizzle, zero fill out of range.
+bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols,
+              uint64_t pitch_elems, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int M, int D>
+cudaError_t launch_t(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *S,
+                     uint32_t *signs, uint16_t *norms, cudaStream_t stream) {
+  using C = Cfg<M, D>;
+  CUtensorMap mk, ms;
+  if (!make_map(&mk, K, (uint64_t)n, D, (uint64_t)ldk, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&ms, S, M, D, D, (uint32_t)C::NMMA)) return cudaErrorInvalidValue;
+  int *err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  Params p{n, (n + BM - 1) / BM, signs, norms, err};
+  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<M, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
+  quantize_tc_kernel<M, D><<<(int)grid, THREADS, C::SMEM, stream>>>(mk, ms, p);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+bool quantize_tc_supported(int m, int d, int64_t n, int64_t ldk, const void *K) {
+  if (!((d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512)))
+    return false;
+  if (n < 1 || n >= ((int64_t)1 << 31)) return false;  // tensor-map row extent
+  if ((reinterpret_cast<uintptr_t>(K) & 15u) != 0 || ((ldk * 2) & 15) != 0) return false;
+  if (ldk >= ((int64_t)1 << 39)) return false;
+  return tc::encode_fn() != nullptr;
 }
 
 cudaError_t launch_quantize_tc(const uint16_t *K, int64_t n, int64_t ldk,
-                               const uint16_t *S, int m, int d,
-                               uint32_t *signs, uint16_t *norms,
-                               cudaStream_t stream) {
-  (void)K; (void)n; (void)ldk; (void)S; (void)m; (void)d; (void)signs;
-  (void)norms; (void)stream;
+                               const uint16_t *S, int m, int d, uint32_t *signs,
+                               uint16_t *norms, cudaStream_t stream) {
+#define JL_CASE(MM, DD) \
+  if (m == MM && d == DD) return tc::launch_t<MM, DD>(K, n, ldk, S, signs, norms, stream);
+  JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
+  JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
+#undef JL_CASE
   return cudaErrorNotSupported;
 }
 
