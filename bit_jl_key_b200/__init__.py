@@ -28,7 +28,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libjlkey.so")
+# JLKEY_LIBRARY may name another build of the same library (e.g. to compare
+# two builds of a kernel); by default the in-tree build is loaded.
+LIB_PATH = os.environ.get("JLKEY_LIBRARY") or os.path.join(_HERE, "libjlkey.so")
 
 JL_BF16 = 0
 JL_F32 = 1

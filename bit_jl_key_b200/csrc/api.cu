@@ -51,6 +51,20 @@ int *device_error_ptr() {
   return g_err_ptr[dev];
 }
 
+void *tensor_map_encoder() {
+  static std::once_flag once;
+  static void *fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = p;
+  });
+  return fn;
+}
+
 int device_max_smem_optin() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 227 * 1024;
@@ -169,7 +183,7 @@ int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
   if (B == 0) return JL_OK;
   if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
   if (!aligned(Q, 16) || !aligned(S, 16) || !aligned(signs, 16) ||
-      !aligned(norms, 2) || !aligned(V, 16) || !aligned(out, 4) ||
+      !aligned(norms, 16) || !aligned(V, 16) || !aligned(out, 4) ||
       (scores && !aligned(scores, 4)))
     return JL_ERR_INVALID_ARG;
   jlk::DecodePlan p;

@@ -15,10 +15,14 @@
 //   2. scorer   a fixed grid of warps; the (unit, 32-key block) space is cut
 //               into equal contiguous runs, one per warp.  A unit is one
 //               (b, kv head, group of <= 8 query heads).  Each warp streams
-//               its blocks through a 3-stage cp.async ring (codes + values),
-//               scores them on tensor cores, keeps an online softmax and a
-//               P.V accumulator per head, and writes one partial state per
-//               unit it touched.
+//               its blocks through its own ring of shared-memory stages: one
+//               lane loads the block's values with a 3-D bulk-tensor copy
+//               (TMA, 128-byte swizzle, rows past the context zero-filled),
+//               every lane copies a slice of the sign codes with cp.async,
+//               and both complete on the stage's mbarrier.  The warp scores
+//               the block on tensor cores, keeps an online softmax and a P.V
+//               accumulator per head, and writes one partial state per unit
+//               it touched.
 //   3. combine  log-sum-exp merge of the partial states -> bf16 output.
 //
 // Scoring on tensor cores.  For 8 keys and one 16-wide slice of the sketch
@@ -32,48 +36,61 @@
 //   ((w << (15 - p)) & 0x80008000) ^ 0xBF80BF80.
 // The score accumulator layout equals the B-operand layout of the P.V product
 // D[16 dims x 8 heads] += V^T[16 dims x 16 keys] * P[16 keys x 8 heads], so P
-// goes from registers straight into the second MMA; V^T comes from shared
-// memory through ldmatrix.trans on an XOR-swizzled tile.
+// goes from registers straight into the second MMA; V^T comes from the
+// swizzled stage through ldmatrix.trans, conflict-free.
 #include "jl_common.cuh"
 #include "jl_internal.h"
 
+#include <cudaTypedefs.h>
 #include <math.h>
 
 namespace jlk {
 
-constexpr int DEC_KB = 32;      // keys per block
-constexpr int DEC_WARPS = 4;    // warps per CTA (independent pipelines)
-constexpr int DEC_STAGES = 3;   // blocks in the per-warp ring
-constexpr int DEC_HPAD = 8;     // head slots per unit
-constexpr int DEC_SM_COUNT = 148;  // B200; fixes the work split per shape
+constexpr int DEC_KB = 32;         // keys per block
+constexpr int DEC_WARPS = 4;       // warps per CTA (independent pipelines)
+constexpr int DEC_HPAD = 8;        // head slots per unit
+constexpr int DEC_SM_COUNT = 148;  // B200 SMs: bounds the workspace per shape
+constexpr int DEC_MAX_CTAS_SM = 4;
+constexpr int DEC_NORM_AREA = 96;  // per stage: 40 fp16 norms (aligned superset)
+#ifndef JL_DECODE_S8
+#define JL_DECODE_S8 0
+#endif
+constexpr bool DEC_S8 = JL_DECODE_S8 != 0;  // int8 scoring MMA (else bf16)
 
 template <int M, int D>
 struct DecCfg {
-  static constexpr int WORDS = M / 32;                 // code words per key
+  static constexpr int STAGES = 2;                     // blocks in the ring
   static constexpr int KEY_SIGN_BYTES = M / 8;
   static constexpr int SIGN_BYTES = DEC_KB * KEY_SIGN_BYTES;
-  static constexpr int V_BYTES = DEC_KB * D * 2;
-  static constexpr int STAGE_BYTES = SIGN_BYTES + V_BYTES;
-  static constexpr int NC = M / 16;                    // 16-wide k slices
-  static constexpr bool A_SMEM = (M > 256);            // A fragments in smem
+  static constexpr int V_BYTES = DEC_KB * D * 2;       // 4 or 8 KB
+  static constexpr int V_BOX = DEC_KB * 128;           // one 64-column box
+  static constexpr int STAGE_BYTES = (V_BYTES + SIGN_BYTES + 1023) / 1024 * 1024;
+  // scoring MMA: bf16 m16n8k16 (16 coordinates per slice) or s8 m16n8k32 (32)
+  static constexpr int KS = DEC_S8 ? 32 : 16;
+  static constexpr int NC = M / KS;                    // k slices
+  static constexpr int A_REGS = 4 * NC;
+  static constexpr bool A_SMEM = A_REGS > 64;          // A fragments in smem
   static constexpr int A_SMEM_BYTES = A_SMEM ? NC * 32 * 16 : 0;
-  static constexpr int WARP_BYTES = DEC_STAGES * STAGE_BYTES + A_SMEM_BYTES;
-  static constexpr int CTA_BYTES = DEC_WARPS * WARP_BYTES;
+  static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + A_SMEM_BYTES;
+  static constexpr int OFF_NORM = DEC_WARPS * WARP_BYTES;
+  static constexpr int OFF_BAR = OFF_NORM + DEC_WARPS * STAGES * DEC_NORM_AREA;
+  static constexpr int CTA_BYTES = OFF_BAR + DEC_WARPS * STAGES * 8 + 1024;  // + align
   static constexpr int LW = (M >= 128) ? M / 128 : 1;  // code words a lane reads
   static constexpr int SIGN_CHUNK = (M >= 128) ? 16 : 8;
+  static constexpr int SIGN_CHUNKS = SIGN_BYTES / SIGN_CHUNK;  // multiple of 32
   static constexpr int DT = D / 16;                    // 16-dim output tiles
-  static constexpr int VCH = D / 8;                    // 16-byte chunks per row
+  static_assert(SIGN_CHUNKS % 32 == 0, "sign chunks per lane");
+  static_assert(STAGE_BYTES % 1024 == 0 && WARP_BYTES % 1024 == 0, "swizzle atoms");
 };
 
 struct DecParams {
   const float *U;           // [B][Hq][M]
   const uint32_t *signs;    // [B][Hkv][T][M/32]
   const uint16_t *norms;    // [B][Hkv][T]
-  const uint16_t *V;        // [B][Hkv][T][D]
   float *partials;          // [units][slots][8][D + 2]
   float *scores;            // nullable [B][Hq][T]
   int *err;                 // device error word
-  int64_t T, nb_u, NB;
+  int64_t T, nb_u, NB, n_keys;
   int Hq, Hkv, G, HG, W, slots;
   float coef;               // sqrt(pi/2) / m
   float scale_log2;         // softmax_scale * log2(e)
@@ -119,107 +136,134 @@ __global__ void __launch_bounds__(128) qproj_kernel(const void *__restrict__ Q,
 
 // ---------------------------------------------------------------------------
 // 2. scorer
-template <int M, int D>
-struct WarpRing {
-  using C = DecCfg<M, D>;
-  uint8_t *base;  // this warp's smem
-  __device__ __forceinline__ uint8_t *sign(int s) const {
-    return base + s * C::STAGE_BYTES;
-  }
-  __device__ __forceinline__ uint8_t *val(int s) const {
-    return base + s * C::STAGE_BYTES + C::SIGN_BYTES;
-  }
-  __device__ __forceinline__ uint8_t *afrag() const {
-    return base + DEC_STAGES * C::STAGE_BYTES;
+
+// Position of a block in the (unit, block) space, advanced without division.
+struct BlockPos {
+  int64_t u;    // unit
+  int64_t blk;  // block within the unit
+  __device__ __forceinline__ void next(int64_t nb_u) {
+    if (++blk == nb_u) {
+      blk = 0;
+      ++u;
+    }
   }
 };
 
-// Issue the async copies of block b into stage s; returns this lane's key norm
-// (lane l holds key l of the block, 0 beyond the context).
 template <int M, int D>
-__device__ __forceinline__ float issue_block(const DecParams &p,
-                                             const WarpRing<M, D> &ring,
-                                             int64_t b, int64_t bend, int s,
-                                             int lane) {
+struct Ring {
   using C = DecCfg<M, D>;
-  float nrm = 0.f;
-  if (b < bend) {
-    const int64_t u = b / p.nb_u;
-    const int64_t blk = b - u * p.nb_u;
-    const int64_t kvi = u / p.HG;
-    const int64_t key0 = blk * DEC_KB;
-    const int nval = (int)((p.T - key0) < DEC_KB ? (p.T - key0) : DEC_KB);
-    const int64_t gkey = kvi * p.T + key0;
-    // codes: contiguous SIGN_BYTES for the block
-    const uint8_t *sg = reinterpret_cast<const uint8_t *>(p.signs) +
-                        gkey * C::KEY_SIGN_BYTES;
-    const uint32_t sdst = smem_u32(ring.sign(s));
-#pragma unroll
-    for (int e = lane; e < C::SIGN_BYTES / C::SIGN_CHUNK; e += 32) {
-      const int key = e * C::SIGN_CHUNK / C::KEY_SIGN_BYTES;
-      const bool ok = key < nval;
-      const void *src = ok ? (const void *)(sg + e * C::SIGN_CHUNK)
-                           : (const void *)p.signs;
-      if (C::SIGN_CHUNK == 16)
-        cp_async_16(sdst + e * 16, src, ok ? 16 : 0);
-      else
-        cp_async_8(sdst + e * 8, src, ok ? 8 : 0);
-    }
-    // values: 32 rows of D bf16, 16-byte chunk c of row r stored at chunk
-    // c ^ (r & 7) so that ldmatrix.trans reads are conflict-free
-    const uint16_t *vg = p.V + gkey * D;
-    const uint32_t vdst = smem_u32(ring.val(s));
-#pragma unroll
-    for (int e = lane; e < DEC_KB * C::VCH; e += 32) {
-      const int key = e / C::VCH;
-      const int c = e - key * C::VCH;
-      const bool ok = key < nval;
-      const void *src = ok ? (const void *)(vg + (int64_t)key * D + c * 8)
-                           : (const void *)p.V;
-      cp_async_16(vdst + key * (2 * D) + ((c ^ (key & 7)) << 4), src,
-                  ok ? 16 : 0);
-    }
-    if (lane < nval) nrm = __half2float(__ushort_as_half(__ldg(p.norms + gkey + lane)));
+  uint32_t base;   // this warp's stages (1024-aligned)
+  uint32_t nbase;  // this warp's norm areas
+  uint32_t bbase;  // this warp's barriers
+  __device__ __forceinline__ uint32_t val(int s) const { return base + s * C::STAGE_BYTES; }
+  __device__ __forceinline__ uint32_t sign(int s) const {
+    return base + s * C::STAGE_BYTES + C::V_BYTES;
   }
-  cp_async_commit();
-  return nrm;
+  __device__ __forceinline__ uint32_t afrag() const { return base + C::STAGES * C::STAGE_BYTES; }
+  __device__ __forceinline__ uint32_t norm(int s) const { return nbase + s * DEC_NORM_AREA; }
+  __device__ __forceinline__ uint32_t bar(int s) const { return bbase + 8 * s; }
+};
+
+// Start the copies of block `pos` into stage s: values by one 3-D bulk-tensor
+// copy per 64 columns (lane 0), codes and norms by cp.async (all lanes).
+template <int M, int D>
+__device__ __forceinline__ void issue_block(const DecParams &p, const CUtensorMap *vmap,
+                                            const Ring<M, D> &ring, const BlockPos &pos,
+                                            int s, int lane) {
+  using C = DecCfg<M, D>;
+  const int64_t kvi = p.HG == 1 ? pos.u : pos.u / p.HG;
+  const int64_t key0 = pos.blk * DEC_KB;
+  const int64_t left = p.T - key0;
+  const int nval = left < DEC_KB ? (int)left : DEC_KB;
+  const int64_t gkey = kvi * p.T + key0;
+  // codes: SIGN_BYTES contiguous bytes, a slice per lane, zero past the context
+  const uint8_t *sg = reinterpret_cast<const uint8_t *>(p.signs) + gkey * C::KEY_SIGN_BYTES;
+  const uint32_t sdst = ring.sign(s);
+#pragma unroll
+  for (int e = lane; e < C::SIGN_CHUNKS; e += 32) {
+    const bool ok = e * C::SIGN_CHUNK < nval * C::KEY_SIGN_BYTES;
+    const void *src = ok ? (const void *)(sg + e * C::SIGN_CHUNK) : (const void *)p.signs;
+    if constexpr (C::SIGN_CHUNK == 16)
+      cp_async_16(sdst + e * 16, src, ok ? 16 : 0);
+    else
+      cp_async_8(sdst + e * 8, src, ok ? 8 : 0);
+  }
+  // norms: the 16-byte-aligned run of 8-norm groups covering the block
+  // (at most 5 groups); key k of the block lands at element (gkey & 7) + k
+  if (lane < 5) {
+    const int64_t first = (gkey & ~(int64_t)7) + 8 * lane;
+    const int64_t avail = p.n_keys - first;
+    const bool ok = first < gkey + nval && avail > 0;
+    const int nbytes = ok ? (avail >= 8 ? 16 : (int)avail * 2) : 0;
+    cp_async_16(ring.norm(s) + 16 * lane, ok ? (const void *)(p.norms + first)
+                                             : (const void *)p.norms, nbytes);
+  }
+  cp_async_mbar_arrive(ring.bar(s));
+  __syncwarp();
+  if (lane == 0) {
+    mbar_expect_tx(ring.bar(s), C::V_BYTES);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h)
+      tma_load_3d(ring.val(s) + h * C::V_BOX, vmap, h * 64, (int)key0, (int)kvi, ring.bar(s));
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
+         ((uint32_t)(d & 0xFF) << 24);
 }
 
 template <int M, int D>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
-    decode_scorer_kernel(const DecParams p) {
+    decode_scorer_kernel(const __grid_constant__ CUtensorMap vmap, const DecParams p) {
   using C = DecCfg<M, D>;
-  extern __shared__ __align__(128) uint8_t dsmem[];
+  extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int w = blockIdx.x * DEC_WARPS + wid;
   if (w >= p.W) return;
   const int g = lane >> 2;  // group id: head row / key column / dim row
   const int t = lane & 3;   // thread in group
-  WarpRing<M, D> ring{dsmem + wid * C::WARP_BYTES};
+  const uint32_t cta = (smem_u32(dsmem_raw) + 1023u) & ~1023u;
+  const Ring<M, D> ring{cta + wid * C::WARP_BYTES,
+                        cta + C::OFF_NORM + wid * C::STAGES * DEC_NORM_AREA,
+                        cta + C::OFF_BAR + wid * C::STAGES * 8};
 
   const int64_t bbeg = (int64_t)w * p.NB / p.W;
   const int64_t bend = (int64_t)(w + 1) * p.NB / p.W;
+  const int64_t nblk = bend - bbeg;
+
+  if (lane == 0)
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(ring.bar(s), 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  __syncwarp();
 
   // prologue: fill the ring
-  float nrm[DEC_STAGES];
+  BlockPos ipos{bbeg / p.nb_u, bbeg - (bbeg / p.nb_u) * p.nb_u};
+  const BlockPos pos0 = ipos;
 #pragma unroll
-  for (int s = 0; s < DEC_STAGES; ++s)
-    nrm[s] = issue_block<M, D>(p, ring, bbeg + s, bend, s, lane);
+  for (int s = 0; s < C::STAGES; ++s) {
+    if (s < nblk) {
+      issue_block<M, D>(p, &vmap, ring, ipos, s, lane);
+      ipos.next(p.nb_u);
+    }
+  }
 
   // per-unit state
-  int64_t cur_u = -1;
+  int64_t cur_u = -1, kv_base = 0;
   int Gg = 0, b_idx = 0, hq0 = 0;
   float mx = -INFINITY, lsum = 0.f;
+  float hscale = 0.f;   // int8 scoring: value of one unit of S q for head g
+  int usum = 0;         // int8 scoring: sum of the quantized S q of head g
   float acc[C::DT][4];
   uint32_t afr[C::A_SMEM ? 1 : C::NC][4];
+  bool failed = false;
 
   auto flush = [&](int64_t u) {
     float l = lsum;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int f = warp_of_block(u * p.nb_u, p.NB, p.W);
-    const int slot = w - f;
+    const int slot = w - warp_of_block(u * p.nb_u, p.NB, p.W);
     if (slot < 0 || slot >= p.slots) {
       record_device_error(p.err, DERR_DECODE_PLAN);
       return;
@@ -244,11 +288,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     }
   };
 
-  for (int64_t b = bbeg; b < bend; ++b) {
-    const int s = (int)((b - bbeg) % DEC_STAGES);
-    const int64_t u = b / p.nb_u;
-    const int64_t key0 = (b - u * p.nb_u) * DEC_KB;
-    const int nval = (int)((p.T - key0) < DEC_KB ? (p.T - key0) : DEC_KB);
+  BlockPos pos = pos0;
+  for (int64_t i = 0; i < nblk; ++i) {
+    const int s = (int)(i % C::STAGES);
+    const int64_t u = pos.u;
+    const int64_t key0 = pos.blk * DEC_KB;
+    const int64_t left = p.T - key0;
+    const int nval = left < DEC_KB ? (int)left : DEC_KB;
 
     if (u != cur_u) {
       if (cur_u >= 0) flush(cur_u);
@@ -256,6 +302,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       const int64_t kvi = u / p.HG;
       const int hg = (int)(u - kvi * p.HG);
       const int hkv = (int)(kvi % p.Hkv);
+      kv_base = kvi * p.T;
       b_idx = (int)(kvi / p.Hkv);
       hq0 = hkv * p.G + hg * DEC_HPAD;
       Gg = min(DEC_HPAD, p.G - hg * DEC_HPAD);
@@ -264,98 +311,214 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
       for (int dt = 0; dt < C::DT; ++dt)
         acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
-      // A fragments: rows 0..7 bf16(u), rows 8..15 bf16(u - bf16(u))
       const float *urow = p.U + ((int64_t)b_idx * p.Hq + hq0 + g) * M;
       const bool live = g < Gg;
+      if constexpr (DEC_S8) {
+        // S q of head g as integers: u ~= hscale * (256 hi + lo), |256 hi + lo|
+        // <= 32000, hi and lo int8 (rows g and g + 8 of the A operand)
+        float amax = 0.f;
+        for (int q = 0; q < M / 16; ++q) {
+          const int Qr = t * (M / 16) + q;
+          const int ib = 32 * (Qr >> 3) + (Qr & 7);
 #pragma unroll
-      for (int c = 0; c < C::NC; ++c) {
-        uint32_t a4[4];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int Qp = t * (M / 8) + 2 * c + r;  // pair index in the key code
-          const int ilo = 32 * (Qp >> 4) + (Qp & 15);
-          const float x0 = live ? urow[ilo] : 0.f;
-          const float x1 = live ? urow[ilo + 16] : 0.f;
-          const float h0 = bf16_round_f32(x0), h1 = bf16_round_f32(x1);
-          a4[2 * r] = pack_bf16x2(h0, h1);
-          a4[2 * r + 1] = pack_bf16x2(x0 - h0, x1 - h1);
+          for (int j = 0; j < 4; ++j) amax = fmaxf(amax, live ? fabsf(urow[ib + 8 * j]) : 0.f);
         }
-        if constexpr (C::A_SMEM) {
-          reinterpret_cast<uint4 *>(ring.afrag())[c * 32 + lane] =
-              make_uint4(a4[0], a4[1], a4[2], a4[3]);
-        } else {
-          afr[c][0] = a4[0]; afr[c][1] = a4[1];
-          afr[c][2] = a4[2]; afr[c][3] = a4[3];
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        hscale = amax > 0.f ? amax / 32000.f : 0.f;
+        const float inv = amax > 0.f ? 32000.f / amax : 0.f;
+        int lsum_i = 0;
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          uint32_t a4[4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int Qr = t * (M / 16) + 2 * c + r;  // byte-register index in the code
+            const int ib = 32 * (Qr >> 3) + (Qr & 7);
+            int hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int ui = live ? __float2int_rn(urow[ib + 8 * j] * inv) : 0;
+              lsum_i += ui;
+              hi[j] = (ui + 128) >> 8;
+              lo[j] = ui - (hi[j] << 8);
+            }
+            a4[r == 0 ? 0 : 2] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
+            a4[r == 0 ? 1 : 3] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
+          }
+          if constexpr (C::A_SMEM) {
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                             ring.afrag() + (c * 32 + lane) * 16),
+                         "r"(a4[0]), "r"(a4[1]), "r"(a4[2]), "r"(a4[3])
+                         : "memory");
+          } else {
+            afr[c][0] = a4[0]; afr[c][1] = a4[1];
+            afr[c][2] = a4[2]; afr[c][3] = a4[3];
+          }
+        }
+        lsum_i += __shfl_xor_sync(0xffffffffu, lsum_i, 1);
+        lsum_i += __shfl_xor_sync(0xffffffffu, lsum_i, 2);
+        usum = lsum_i;
+      } else {
+        // A fragments: rows 0..7 bf16(u), rows 8..15 bf16(u - bf16(u))
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c) {
+          uint32_t a4[4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int Qp = t * (M / 8) + 2 * c + r;  // pair index in the key code
+            const int ilo = 32 * (Qp >> 4) + (Qp & 15);
+            const float x0 = live ? urow[ilo] : 0.f;
+            const float x1 = live ? urow[ilo + 16] : 0.f;
+            const float h0 = bf16_round_f32(x0), h1 = bf16_round_f32(x1);
+            a4[2 * r] = pack_bf16x2(h0, h1);
+            a4[2 * r + 1] = pack_bf16x2(x0 - h0, x1 - h1);
+          }
+          if constexpr (C::A_SMEM) {
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                             ring.afrag() + (c * 32 + lane) * 16),
+                         "r"(a4[0]), "r"(a4[1]), "r"(a4[2]), "r"(a4[3])
+                         : "memory");
+          } else {
+            afr[c][0] = a4[0]; afr[c][1] = a4[1];
+            afr[c][2] = a4[2]; afr[c][3] = a4[3];
+          }
         }
       }
       if constexpr (C::A_SMEM) __syncwarp();
     }
 
-    cp_async_wait<DEC_STAGES - 1>();
-    __syncwarp();
+    if (!mbar_wait_bounded(ring.bar(s), (uint32_t)((i / C::STAGES) & 1))) {
+      record_device_error(p.err, DERR_DECODE_WAIT_TIMEOUT);
+      failed = true;
+      break;
+    }
 
-    // ---- scores for the 4 groups of 8 keys
-    const uint8_t *sg = ring.sign(s);
+    // ---- code words of the 4 groups of 8 keys (lane: key kg*8 + g)
+    const uint32_t sg = ring.sign(s);
     uint32_t wd[4][C::LW];
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
-      const uint8_t *kp = sg + (kg * 8 + g) * C::KEY_SIGN_BYTES;
-      if constexpr (M >= 128) {
-#pragma unroll
-        for (int i = 0; i < C::LW; ++i)
-          wd[kg][i] = reinterpret_cast<const uint32_t *>(kp)[t * C::LW + i];
+      const uint32_t kp = sg + (kg * 8 + g) * C::KEY_SIGN_BYTES;
+      if constexpr (C::LW == 4) {
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                     : "=r"(wd[kg][0]), "=r"(wd[kg][1]), "=r"(wd[kg][2]), "=r"(wd[kg][3])
+                     : "r"(kp + t * 16));
+      } else if constexpr (C::LW == 2) {
+        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];\n"
+                     : "=r"(wd[kg][0]), "=r"(wd[kg][1])
+                     : "r"(kp + t * 8));
+      } else if constexpr (M == 128) {
+        asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][0]) : "r"(kp + t * 4));
       } else {
-        wd[kg][0] = reinterpret_cast<const uint32_t *>(kp)[t >> 1];
+        asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][0]) : "r"(kp + (t >> 1) * 4));
       }
     }
-    float sc[4][4];
+
+    // ---- raw estimator sum_i u_i sign_i for head g, keys kg*8 + 2t + j
+    float raw[4][2];
+    if constexpr (DEC_S8) {
+      int sc[4][4];
 #pragma unroll
-    for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0.f;
-    const int pbase = (M >= 128) ? 0 : 8 * (t & 1);
+      for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0;
+      const int pbase = (M >= 128) ? 0 : 4 * (t & 1);
 #pragma unroll
-    for (int c = 0; c < C::NC; ++c) {
-      uint32_t a0, a1, a2, a3;
-      if constexpr (C::A_SMEM) {
-        const uint4 v = reinterpret_cast<const uint4 *>(ring.afrag())[c * 32 + lane];
-        a0 = v.x; a1 = v.y; a2 = v.z; a3 = v.w;
-      } else {
-        a0 = afr[c][0]; a1 = afr[c][1]; a2 = afr[c][2]; a3 = afr[c][3];
-      }
-      const int q0 = 2 * c, q1 = 2 * c + 1;
-#pragma unroll
-      for (int kg = 0; kg < 4; ++kg) {
-        uint32_t w0, w1;
-        int p0, p1;
-        if constexpr (M >= 128) {
-          w0 = wd[kg][q0 >> 4]; p0 = q0 & 15;
-          w1 = wd[kg][q1 >> 4]; p1 = q1 & 15;
+      for (int c = 0; c < C::NC; ++c) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (C::A_SMEM) {
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                       : "r"(ring.afrag() + (c * 32 + lane) * 16));
         } else {
-          w0 = w1 = wd[kg][0]; p0 = pbase + q0; p1 = pbase + q1;
+          a0 = afr[c][0]; a1 = afr[c][1]; a2 = afr[c][2]; a3 = afr[c][3];
         }
-        const uint32_t b0 = ((w0 << (15 - p0)) & 0x80008000u) ^ 0xBF80BF80u;
-        const uint32_t b1 = ((w1 << (15 - p1)) & 0x80008000u) ^ 0xBF80BF80u;
-        mma_bf16_16816(sc[kg], a0, a1, a2, a3, b0, b1);
+        const int q0 = 2 * c, q1 = 2 * c + 1;
+#pragma unroll
+        for (int kg = 0; kg < 4; ++kg) {
+          uint32_t w0, w1;
+          int p0, p1;
+          if constexpr (M >= 128) {
+            w0 = wd[kg][q0 >> 3]; p0 = q0 & 7;
+            w1 = wd[kg][q1 >> 3]; p1 = q1 & 7;
+          } else {
+            w0 = w1 = wd[kg][0]; p0 = pbase + q0; p1 = pbase + q1;
+          }
+          // bytes j = bits p + 8j: {0, 1} per coordinate
+          const uint32_t b0 = (w0 >> p0) & 0x01010101u;
+          const uint32_t b1 = (w1 >> p1) & 0x01010101u;
+          mma_s8_16832(sc[kg], a0, a1, a2, a3, b0, b1);
+        }
       }
+      // sum_i u_i sign_i = hscale * (2 * sum_{bit=1} u_int - sum u_int)
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          raw[kg][j] = hscale * (float)(2 * (sc[kg][j] * 256 + sc[kg][j + 2]) - usum);
+    } else {
+      float sc[4][4];
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0.f;
+      const int pbase = (M >= 128) ? 0 : 8 * (t & 1);
+#pragma unroll
+      for (int c = 0; c < C::NC; ++c) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (C::A_SMEM) {
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                       : "r"(ring.afrag() + (c * 32 + lane) * 16));
+        } else {
+          a0 = afr[c][0]; a1 = afr[c][1]; a2 = afr[c][2]; a3 = afr[c][3];
+        }
+        const int q0 = 2 * c, q1 = 2 * c + 1;
+#pragma unroll
+        for (int kg = 0; kg < 4; ++kg) {
+          uint32_t w0, w1;
+          int p0, p1;
+          if constexpr (M >= 128) {
+            w0 = wd[kg][q0 >> 4]; p0 = q0 & 15;
+            w1 = wd[kg][q1 >> 4]; p1 = q1 & 15;
+          } else {
+            w0 = w1 = wd[kg][0]; p0 = pbase + q0; p1 = pbase + q1;
+          }
+          const uint32_t b0 = ((w0 << (15 - p0)) & 0x80008000u) ^ 0xBF80BF80u;
+          const uint32_t b1 = ((w1 << (15 - p1)) & 0x80008000u) ^ 0xBF80BF80u;
+          mma_bf16_16816(sc[kg], a0, a1, a2, a3, b0, b1);
+        }
+      }
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) raw[kg][j] = sc[kg][j] + sc[kg][j + 2];
     }
 
     // ---- estimator, masking, online softmax (head g, keys kg*8 + 2t + j)
     float l2[4][2];
     float bmax = -INFINITY;
+    const uint32_t nrow = ring.norm(s) + (uint32_t)((kv_base + key0) & 7) * 2;
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int key = kg * 8 + 2 * t + j;
-        const float raw = sc[kg][j] + sc[kg][j + 2];
-        const float nk = __shfl_sync(0xffffffffu, nrm[0], key);
-        const float sval = p.coef * nk * raw;
-        const bool ok = key < nval;
-        if (p.scores != nullptr && ok && g < Gg)
+        unsigned short hb;
+        asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(hb) : "r"(nrow + key * 2));
+        const float nk = __half2float(__ushort_as_half(hb));
+        const float sval = (p.coef * nk) * raw[kg][j];
+        l2[kg][j] = sval * p.scale_log2;
+        if (p.scores != nullptr && key < nval && g < Gg)
           p.scores[((int64_t)b_idx * p.Hq + hq0 + g) * p.T + key0 + key] = sval;
-        l2[kg][j] = ok ? sval * p.scale_log2 : -INFINITY;
-        bmax = fmaxf(bmax, l2[kg][j]);
       }
     }
+    if (nval < DEC_KB) {
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          if (kg * 8 + 2 * t + j >= nval) l2[kg][j] = -INFINITY;
+    }
+#pragma unroll
+    for (int kg = 0; kg < 4; ++kg) bmax = fmaxf(bmax, fmaxf(l2[kg][0], l2[kg][1]));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
     bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));
     const float mnew = fmaxf(mx, bmax);
@@ -380,33 +543,43 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       acc[dt][2] *= al0; acc[dt][3] *= al1;
     }
 
-    // ---- P.V: two k-steps of 16 keys
-    const uint32_t vbase = smem_u32(ring.val(s));
+    // ---- P.V: two k-steps of 16 keys over the swizzled value tile
+    const uint32_t vbase = ring.val(s);
     const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
       const uint32_t pb0 = pack_bf16x2(pr[2 * jj][0], pr[2 * jj][1]);
       const uint32_t pb1 = pack_bf16x2(pr[2 * jj + 1][0], pr[2 * jj + 1][1]);
-      const int key = 16 * jj + rr + 8 * (mi >> 1);
+      const uint32_t krow = vbase + (16 * jj + rr + 8 * (mi >> 1)) * 128;
 #pragma unroll
       for (int dt = 0; dt < C::DT; ++dt) {
-        const int ch = 2 * dt + (mi & 1);
-        const uint32_t addr = vbase + key * (2 * D) + ((ch ^ rr) << 4);
+        const int ch = 2 * dt + (mi & 1);  // 16-byte chunk along d
+        const uint32_t addr = krow + (ch >> 3) * C::V_BOX + (((ch & 7) ^ rr) << 4);
         uint32_t v0, v1, v2, v3;
         ldmatrix_x4_trans(addr, v0, v1, v2, v3);
         mma_bf16_16816(acc[dt], v0, v1, v2, v3, pb0, pb1);
       }
     }
 
-    // ---- refill this stage with block b + STAGES
+    // ---- refill this stage with the block STAGES ahead
     __syncwarp();
-#pragma unroll
-    for (int i = 0; i < DEC_STAGES - 1; ++i) nrm[i] = nrm[i + 1];
-    nrm[DEC_STAGES - 1] =
-        issue_block<M, D>(p, ring, b + DEC_STAGES, bend, s, lane);
+    if (i + C::STAGES < nblk) {
+      issue_block<M, D>(p, &vmap, ring, ipos, s, lane);
+      ipos.next(p.nb_u);
+    }
+    pos.next(p.nb_u);
+  }
+  if (failed) {
+    // let the copies already started land before the warp's smem goes away
+    for (int k = 0; k < C::STAGES; ++k) {
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(ring.bar(k), 0) && !mbar_try_wait(ring.bar(k), 1) &&
+             globaltimer() - t0 < WAIT_LIMIT_NS) {
+      }
+    }
+    return;
   }
   if (cur_u >= 0) flush(cur_u);
-  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -441,22 +614,8 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
 
 // ---------------------------------------------------------------------------
 // planning and launch
-template <int M, int D>
-static int ctas_per_sm() {
-  const int smem_sm = 228 * 1024;
-  int k = smem_sm / (DecCfg<M, D>::CTA_BYTES + 1024);
-  if (k > 3) k = 3;
-  if (k < 1) k = 1;
-  return k;
-}
-
-static int dispatch_ctas_per_sm(int m, int d) {
-#define JL_CASE(MM, DD) \
-  if (m == MM && d == DD) return ctas_per_sm<MM, DD>();
-  JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
-  JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
-#undef JL_CASE
-  return 0;
+static bool supported(int m, int d) {
+  return (d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512);
 }
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -464,8 +623,8 @@ static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
                       DecodePlan *pl) {
   if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv) return false;
-  const int k = dispatch_ctas_per_sm(m, d);
-  if (k == 0) return false;
+  if ((int64_t)B * Hkv >= ((int64_t)1 << 31) || T >= ((int64_t)1 << 31)) return false;
+  if (!supported(m, d)) return false;
   DecodePlan p{};
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.m = m; p.d = d;
   p.G = Hq / Hkv;
@@ -473,8 +632,11 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
   p.units = B * Hkv * p.HG;
   p.nb_u = (T + DEC_KB - 1) / DEC_KB;
   p.NB = (int64_t)p.units * p.nb_u;
-  const int64_t wt = (int64_t)DEC_SM_COUNT * k * DEC_WARPS;
-  p.W = (int)(p.NB < wt ? p.NB : wt);
+  // the launch uses at most W_bound warps (B200 SMs x max CTAs per SM); the
+  // partial-state layout is sized for that bound so that it depends on the
+  // shapes only
+  const int64_t wb = (int64_t)DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS;
+  p.W = (int)(p.NB < wb ? p.NB : wb);
   p.slots = (int)((p.W + p.units - 1) / p.units) + 1;
   p.u_bytes = round_up((size_t)B * Hq * m * sizeof(float), 256);
   p.partial_bytes = round_up(
@@ -482,6 +644,22 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
   p.total_bytes = p.u_bytes + p.partial_bytes;
   *pl = p;
   return true;
+}
+
+// V viewed as [B*Hkv][T][d] bf16; boxes of 64 columns x 32 rows x 1 unit with
+// the 128-byte swizzle; rows past T are zero-filled.
+static bool make_value_map(CUtensorMap *map, const uint16_t *V, int64_t units_kv,
+                           int64_t T, int d) {
+  auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)units_kv};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)T * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)DEC_KB, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(V), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int M, int D>
@@ -495,6 +673,11 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   float *U = reinterpret_cast<float *>(workspace);
   float *partials =
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
+  CUtensorMap vmap;
+  if (!make_value_map(&vmap, V, (int64_t)pl.B * pl.Hkv, pl.T, D))
+    return cudaErrorInvalidValue;
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
   const int bh = pl.B * pl.Hq;
   if (q_f32)
     qproj_kernel<M, D, true><<<bh, 128, 0, stream>>>(Q, S, U);
@@ -502,12 +685,12 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
     qproj_kernel<M, D, false><<<bh, 128, 0, stream>>>(Q, S, U);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (device_error_ptr() == nullptr) return cudaErrorInvalidSymbol;
 
   DecParams p;
-  p.U = U; p.signs = signs; p.norms = norms; p.V = V; p.partials = partials;
-  p.scores = scores; p.err = device_error_ptr(); p.T = pl.T; p.nb_u = pl.nb_u; p.NB = pl.NB;
-  p.Hq = pl.Hq; p.Hkv = pl.Hkv; p.G = pl.G; p.HG = pl.HG; p.W = pl.W;
+  p.U = U; p.signs = signs; p.norms = norms; p.partials = partials;
+  p.scores = scores; p.err = err; p.T = pl.T; p.nb_u = pl.nb_u; p.NB = pl.NB;
+  p.n_keys = (int64_t)pl.B * pl.Hkv * pl.T;
+  p.Hq = pl.Hq; p.Hkv = pl.Hkv; p.G = pl.G; p.HG = pl.HG;
   p.slots = pl.slots;
   p.coef = (float)(sqrt(M_PI / 2.0) / (double)M);
   p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
@@ -515,13 +698,22 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::CTA_BYTES);
   if (e != cudaSuccess) return e;
-  const int ctas = (pl.W + DEC_WARPS - 1) / DEC_WARPS;
-  decode_scorer_kernel<M, D><<<ctas, DEC_WARPS * 32, C::CTA_BYTES, stream>>>(p);
+  // one wave of resident CTAs, never more warps than the plan's bound
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_scorer_kernel<M, D>,
+                                                    DEC_WARPS * 32, C::CTA_BYTES);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > DEC_MAX_CTAS_SM) per_sm = DEC_MAX_CTAS_SM;
+  const int64_t wave = (int64_t)device_sm_count() * per_sm * DEC_WARPS;
+  p.W = (int)(wave < pl.W ? wave : pl.W);
+  const int ctas = (p.W + DEC_WARPS - 1) / DEC_WARPS;
+  decode_scorer_kernel<M, D><<<ctas, DEC_WARPS * 32, C::CTA_BYTES, stream>>>(vmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<D><<<bh, D, 0, stream>>>(partials, out, pl.Hq, pl.Hkv,
                                                  pl.G, pl.HG, pl.nb_u, pl.NB,
-                                                 pl.W, pl.slots);
+                                                 p.W, pl.slots);
   return cudaGetLastError();
 }
 

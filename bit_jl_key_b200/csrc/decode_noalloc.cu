@@ -72,7 +72,7 @@ extern "C" int jl_decode_attention_noalloc(
     return (reinterpret_cast<uintptr_t>(p) % a) != 0;
   };
   if (misaligned(Q, 16) || misaligned(S, 16) || misaligned(signs, 16) ||
-      misaligned(norms, 2) || misaligned(V, 16) || misaligned(out, 4) ||
+      misaligned(norms, 16) || misaligned(V, 16) || misaligned(out, 4) ||
       (scores && misaligned(scores, 4)))
     return JL_ERR_INVALID_ARG;
   jlk::DecodePlan p;

@@ -145,7 +145,7 @@ JL_API size_t jl_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m
  *              16-byte aligned.
  *   S        : in, device, m x d bf16 (the sketch the keys were coded with).
  *   signs    : in, device, B x Hkv x T x (m/32) uint32 codes, 16-byte aligned.
- *   norms    : in, device, B x Hkv x T binary16 key norms, 2-byte aligned.
+ *   norms    : in, device, B x Hkv x T binary16 key norms, 16-byte aligned.
  *   V        : in, device, B x Hkv x T x d bf16 values, 16-byte aligned.
  *   softmax_scale : logit = softmax_scale * s(q, k_t) (typically 1/sqrt(d)).
  *   out      : out, device, B x Hq x d bf16, 4-byte aligned.

@@ -132,6 +132,7 @@ def test_decode_argument_errors(lib):
         assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
     assert call(V=MISALIGNED) == jl.JL_ERR_INVALID_ARG
     assert call(signs=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(norms=ctypes.c_void_p((1 << 20) + 8)) == jl.JL_ERR_INVALID_ARG
     assert call(scale=float("nan")) == jl.JL_ERR_INVALID_ARG
     assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
     need = jl.jl_decode_workspace_bytes(2, 8, 2, 100, 256, 128)
