@@ -151,6 +151,21 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def reduce_max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (the only collective the bench
+    uses; the data path has none)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Units of all ranks over the slowest rank's time (weak scaling)."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 # --------------------------------------------------------------------------
 # algorithmic bytes
 
@@ -236,13 +251,9 @@ def run_ours(args, rank, world, local_rank):
     if jl.jl_device_error() != 0:
         raise RuntimeError("device error in the timed region")
 
-    ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = reduce_max_over_ranks(ms_total / args.steps, world, dev)
     keys_all = n_keys * world
-    value = keys_all / (ms_step * 1e-3)
+    value = whole_job_rate(n_keys, world, ms_step)
 
     # ---- end to end through the binding with pinned host buffers
     e2e = None
@@ -290,12 +301,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         barrier()
-        e_ms = e0.elapsed_time(e1) / e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": keys_all / (e_ms * 1e-3), "unit": "keys/s",
+        e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+        e2e = {"value": whole_job_rate(n_keys, world, e_ms), "unit": "keys/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 

@@ -44,6 +44,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <utility>
+
 namespace jlk {
 
 constexpr int DEC_KB = 32;         // keys per block
@@ -51,13 +53,14 @@ constexpr int DEC_WARPS = 4;       // warps per CTA (independent pipelines)
 constexpr int DEC_HPAD = 8;        // head slots per unit
 constexpr int DEC_SM_COUNT = 148;  // B200 SMs: bounds the workspace per shape
 constexpr int DEC_MAX_CTAS_SM = 4;
-constexpr int DEC_NORM_AREA = 96;  // per stage: 40 fp16 norms (aligned superset)
-#ifndef JL_DECODE_S8
-#define JL_DECODE_S8 0
+constexpr int DEC_NORM_AREA = 128; // per stage: 40 fp16 norms; bulk-tensor copies need
+                                   // a 128-byte-aligned destination
+// Scoring MMA per shape: 0 = chosen by decode_use_s8(), 1 = bf16, 2 = int8.
+#ifndef JL_DECODE_SCORE
+#define JL_DECODE_SCORE 0
 #endif
-constexpr bool DEC_S8 = JL_DECODE_S8 != 0;  // int8 scoring MMA (else bf16)
 
-template <int M, int D>
+template <int M, int D, bool S8>
 struct DecCfg {
   static constexpr int STAGES = 2;                     // blocks in the ring
   static constexpr int KEY_SIGN_BYTES = M / 8;
@@ -66,7 +69,7 @@ struct DecCfg {
   static constexpr int V_BOX = DEC_KB * 128;           // one 64-column box
   static constexpr int STAGE_BYTES = (V_BYTES + SIGN_BYTES + 1023) / 1024 * 1024;
   // scoring MMA: bf16 m16n8k16 (16 coordinates per slice) or s8 m16n8k32 (32)
-  static constexpr int KS = DEC_S8 ? 32 : 16;
+  static constexpr int KS = S8 ? 32 : 16;
   static constexpr int NC = M / KS;                    // k slices
   static constexpr int A_REGS = 4 * NC;
   static constexpr bool A_SMEM = A_REGS > 64;          // A fragments in smem
@@ -96,6 +99,19 @@ struct DecParams {
   float scale_log2;         // softmax_scale * log2(e)
 };
 
+// Bulk-tensor maps of one decode call.  Values always go through `value`
+// (3-D, [B*Hkv][T][d], 128-byte swizzle).  When the context length keeps
+// every unit's codes and norms 16-byte aligned (T % 8 == 0), `sign` and
+// `norm` map them as [B*Hkv][T*words] and [B*Hkv][T] and one lane fetches a
+// whole block; otherwise every lane copies a slice with cp.async.
+struct DecMaps {
+  CUtensorMap value;
+  CUtensorMap sign;
+  CUtensorMap norm;
+  int tma_codes;  // 1: codes and norms by bulk-tensor copy
+  int sign_elem;  // bytes per element of the sign map (4 or 8)
+};
+
 // warp that owns block b when NB blocks are cut into W contiguous runs
 // starting at floor(w * NB / W)
 __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
@@ -104,34 +120,53 @@ __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
 }
 
 // ---------------------------------------------------------------------------
-// 1. query projection u = S q (fp32 accumulate)
+// 1. query projection u = S q (fp32 accumulate).  A CTA projects QPB queries;
+// thread i owns sketch row i, reads it once (16-byte loads, L2-resident) and
+// applies it to all QPB queries held in shared memory.
+constexpr int QPB = 8;
+
 template <int M, int D, bool QF32>
-__global__ void __launch_bounds__(128) qproj_kernel(const void *__restrict__ Q,
-                                                    const uint16_t *__restrict__ S,
-                                                    float *__restrict__ U) {
-  __shared__ float qs[D];
-  const int bh = blockIdx.x;
-  for (int j = threadIdx.x; j < D; j += blockDim.x) {
-    qs[j] = QF32 ? reinterpret_cast<const float *>(Q)[(int64_t)bh * D + j]
-                 : bf16_bits_to_f32(
-                       reinterpret_cast<const uint16_t *>(Q)[(int64_t)bh * D + j]);
+__global__ void __launch_bounds__(M) qproj_kernel(const void *__restrict__ Q,
+                                                  const uint16_t *__restrict__ S,
+                                                  float *__restrict__ U, int nq) {
+  __shared__ float qs[QPB][D];
+  griddep_launch_dependents();  // let the scorer start its copies now
+  const int q0 = blockIdx.x * QPB;
+  const int nloc = min(QPB, nq - q0);
+  for (int e = threadIdx.x; e < QPB * D; e += M) {
+    const int j = e / D, c = e - j * D;
+    float v = 0.f;
+    if (j < nloc) {
+      const int64_t idx = (int64_t)(q0 + j) * D + c;
+      v = QF32 ? reinterpret_cast<const float *>(Q)[idx]
+               : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[idx]);
+    }
+    qs[j][c] = v;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < M; i += blockDim.x) {
-    const uint4 *row = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
-    float acc = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = __ldg(row + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const int i = threadIdx.x;
+  const uint4 *row = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
+  float acc[QPB];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc = fmaf(__uint_as_float(w[e] << 16), qs[c * 8 + 2 * e], acc);
-        acc = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), qs[c * 8 + 2 * e + 1], acc);
+  for (int j = 0; j < QPB; ++j) acc[j] = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 v = __ldg(row + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float s0 = __uint_as_float(w[e] << 16);
+      const float s1 = __uint_as_float(w[e] & 0xFFFF0000u);
+#pragma unroll
+      for (int j = 0; j < QPB; ++j) {
+        acc[j] = fmaf(s0, qs[j][c * 8 + 2 * e], acc[j]);
+        acc[j] = fmaf(s1, qs[j][c * 8 + 2 * e + 1], acc[j]);
       }
     }
-    U[(int64_t)bh * M + i] = acc;
   }
+#pragma unroll
+  for (int j = 0; j < QPB; ++j)
+    if (j < nloc) U[(int64_t)(q0 + j) * M + i] = acc[j];
 }
 
 // ---------------------------------------------------------------------------
@@ -149,9 +184,9 @@ struct BlockPos {
   }
 };
 
-template <int M, int D>
+template <int M, int D, bool S8>
 struct Ring {
-  using C = DecCfg<M, D>;
+  using C = DecCfg<M, D, S8>;
   uint32_t base;   // this warp's stages (1024-aligned)
   uint32_t nbase;  // this warp's norm areas
   uint32_t bbase;  // this warp's barriers
@@ -166,13 +201,26 @@ struct Ring {
 
 // Start the copies of block `pos` into stage s: values by one 3-D bulk-tensor
 // copy per 64 columns (lane 0), codes and norms by cp.async (all lanes).
-template <int M, int D>
-__device__ __forceinline__ void issue_block(const DecParams &p, const CUtensorMap *vmap,
-                                            const Ring<M, D> &ring, const BlockPos &pos,
+template <int M, int D, bool S8>
+__device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &maps,
+                                            const Ring<M, D, S8> &ring, const BlockPos &pos,
                                             int s, int lane) {
-  using C = DecCfg<M, D>;
+  using C = DecCfg<M, D, S8>;
   const int64_t kvi = p.HG == 1 ? pos.u : pos.u / p.HG;
   const int64_t key0 = pos.blk * DEC_KB;
+  if (maps.tma_codes) {
+    if (lane == 0) {
+      mbar_expect_tx(ring.bar(s), C::V_BYTES + C::SIGN_BYTES + 2 * DEC_KB);
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_load_3d(ring.val(s) + h * C::V_BOX, &maps.value, h * 64, (int)key0, (int)kvi,
+                    ring.bar(s));
+      tma_load_2d(ring.sign(s), &maps.sign,
+                  (int)(key0 * C::KEY_SIGN_BYTES / maps.sign_elem), (int)kvi, ring.bar(s));
+      tma_load_2d(ring.norm(s), &maps.norm, (int)key0, (int)kvi, ring.bar(s));
+    }
+    return;
+  }
   const int64_t left = p.T - key0;
   const int nval = left < DEC_KB ? (int)left : DEC_KB;
   const int64_t gkey = kvi * p.T + key0;
@@ -204,19 +252,190 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const CUtensorMa
     mbar_expect_tx(ring.bar(s), C::V_BYTES);
 #pragma unroll
     for (int h = 0; h < D / 64; ++h)
-      tma_load_3d(ring.val(s) + h * C::V_BOX, vmap, h * 64, (int)key0, (int)kvi, ring.bar(s));
+      tma_load_3d(ring.val(s) + h * C::V_BOX, &maps.value, h * 64, (int)key0, (int)kvi,
+                  ring.bar(s));
   }
 }
+
 
 __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
          ((uint32_t)(d & 0xFF) << 24);
 }
 
-template <int M, int D>
+// The lane's 32-coordinate runs of u: lane t of a quad owns code words
+// t*M/128 .. (M >= 128), or half of word t/2 (M = 64).  run(k) gives the
+// start of the k-th run of `len` consecutive coordinates.
+template <int M>
+struct LaneRuns {
+  static constexpr int WORDS = (M >= 128) ? M / 128 : 1;
+};
+
+__device__ __forceinline__ float4 ldg4(const float *p) {
+  return __ldg(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ float f4c(const float4 &v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// A fragments of one unit for the lane (g, t): rows 0..7 of the scoring MMA
+// hold the high part of S q of the <= 8 heads, rows 8..15 the low part.
+//   bf16: hi = bf16(u), lo = bf16(u - hi)
+//   int8: u ~= hscale * (256 hi + lo), |256 hi + lo| <= 32000, usum = sum of
+//         256 hi + lo over the head's coordinates.
+// u is read as whole 16-byte vectors of the lane's own coordinate runs.
+template <int M, int D, bool S8>
+__device__ __forceinline__ void build_afrags(const float *urow, bool live, int t,
+                                             const Ring<M, D, S8> &ring,
+                                             uint32_t (&afr)[DecCfg<M, D, S8>::A_SMEM ? 1 : DecCfg<M, D, S8>::NC][4],
+                                             float &hscale, int &usum) {
+  using C = DecCfg<M, D, S8>;
+  auto put = [&](int c, const uint32_t (&a4)[4]) {
+    if constexpr (C::A_SMEM) {
+      const int lane = (threadIdx.x & 31);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                       ring.afrag() + (c * 32 + lane) * 16),
+                   "r"(a4[0]), "r"(a4[1]), "r"(a4[2]), "r"(a4[3])
+                   : "memory");
+    } else {
+      afr[c][0] = a4[0]; afr[c][1] = a4[1]; afr[c][2] = a4[2]; afr[c][3] = a4[3];
+    }
+  };
+  if constexpr (!S8) {
+    if constexpr (M >= 128) {
+#pragma unroll
+      for (int lw = 0; lw < LaneRuns<M>::WORDS; ++lw) {
+        const float *src = urow + 32 * (t * LaneRuns<M>::WORDS + lw);
+        float4 x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
+        // pair p of the word: coordinates p and p + 16 -> chunk 8 lw + p/2, slot p&1
+#pragma unroll
+        for (int c2 = 0; c2 < 8; ++c2) {
+          uint32_t a4[4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int pp = 2 * c2 + r;
+            const float x0 = f4c(x[pp >> 2], pp & 3), x1 = f4c(x[(pp + 16) >> 2], pp & 3);
+            const float h0 = bf16_round_f32(x0), h1 = bf16_round_f32(x1);
+            a4[2 * r] = pack_bf16x2(h0, h1);
+            a4[2 * r + 1] = pack_bf16x2(x0 - h0, x1 - h1);
+          }
+          put(8 * lw + c2, a4);
+        }
+      }
+    } else {
+      // M = 64: pairs 8(t&1) .. +7 of word t/2
+      const float *src = urow + 32 * (t >> 1) + 8 * (t & 1);
+      float4 x[4];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
+        x[2 + k] = live ? ldg4(src + 16 + 4 * k) : make_float4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a4[4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int q = 2 * c + r;
+          const float x0 = f4c(x[q >> 2], q & 3), x1 = f4c(x[2 + (q >> 2)], q & 3);
+          const float h0 = bf16_round_f32(x0), h1 = bf16_round_f32(x1);
+          a4[2 * r] = pack_bf16x2(h0, h1);
+          a4[2 * r + 1] = pack_bf16x2(x0 - h0, x1 - h1);
+        }
+        put(c, a4);
+      }
+    }
+    (void)hscale; (void)usum;
+  } else {
+    // pass 1: the head's largest |u| (4 lanes of the quad together)
+    float amax = 0.f;
+    if (live) {
+      if constexpr (M >= 128) {
+#pragma unroll
+        for (int lw = 0; lw < LaneRuns<M>::WORDS; ++lw) {
+          const float *src = urow + 32 * (t * LaneRuns<M>::WORDS + lw);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 v = ldg4(src + 4 * k);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+          }
+        }
+      } else {
+        const float *src = urow + 32 * (t >> 1) + 4 * (t & 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 v = ldg4(src + 8 * j);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+      }
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    hscale = amax > 0.f ? amax / 32000.f : 0.f;
+    const float inv = amax > 0.f ? 32000.f / amax : 0.f;
+    int isum = 0;
+    auto quant = [&](float x, int &hi, int &lo) {
+      const int ui = __float2int_rn(x * inv);
+      isum += ui;
+      hi = (ui + 128) >> 8;
+      lo = ui - (hi << 8);
+    };
+    // pass 2: byte register p of a word holds coordinates p + 8j, j = 0..3
+    if constexpr (M >= 128) {
+#pragma unroll
+      for (int lw = 0; lw < LaneRuns<M>::WORDS; ++lw) {
+        const float *src = urow + 32 * (t * LaneRuns<M>::WORDS + lw);
+        float4 x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          uint32_t a4[4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int pp = 2 * c2 + r;
+            int hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) quant(f4c(x[(pp + 8 * j) >> 2], pp & 3), hi[j], lo[j]);
+            a4[2 * r] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
+            a4[2 * r + 1] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
+          }
+          put(4 * lw + c2, a4);
+        }
+      }
+    } else {
+      const float *src = urow + 32 * (t >> 1) + 4 * (t & 1);
+      float4 x[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] = live ? ldg4(src + 8 * j) : make_float4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t a4[4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int q = 2 * c + r;
+          int hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) quant(f4c(x[j], q), hi[j], lo[j]);
+          a4[2 * r] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
+          a4[2 * r + 1] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        put(c, a4);
+      }
+    }
+    isum += __shfl_xor_sync(0xffffffffu, isum, 1);
+    isum += __shfl_xor_sync(0xffffffffu, isum, 2);
+    usum = isum;
+  }
+  if constexpr (C::A_SMEM) __syncwarp();
+}
+
+template <int M, int D, bool S8>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
-    decode_scorer_kernel(const __grid_constant__ CUtensorMap vmap, const DecParams p) {
-  using C = DecCfg<M, D>;
+    decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
+  using C = DecCfg<M, D, S8>;
   extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -225,7 +444,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   const int g = lane >> 2;  // group id: head row / key column / dim row
   const int t = lane & 3;   // thread in group
   const uint32_t cta = (smem_u32(dsmem_raw) + 1023u) & ~1023u;
-  const Ring<M, D> ring{cta + wid * C::WARP_BYTES,
+  const Ring<M, D, S8> ring{cta + wid * C::WARP_BYTES,
                         cta + C::OFF_NORM + wid * C::STAGES * DEC_NORM_AREA,
                         cta + C::OFF_BAR + wid * C::STAGES * 8};
 
@@ -244,10 +463,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
   for (int s = 0; s < C::STAGES; ++s) {
     if (s < nblk) {
-      issue_block<M, D>(p, &vmap, ring, ipos, s, lane);
+      issue_block<M, D, S8>(p, maps, ring, ipos, s, lane);
       ipos.next(p.nb_u);
     }
   }
+
+  // the query projections come from the previous kernel on the stream, which
+  // may still be running (programmatic dependent launch): wait for it only
+  // now, after the first copies are on their way
+  griddep_wait();
 
   // per-unit state
   int64_t cur_u = -1, kv_base = 0;
@@ -312,79 +536,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       for (int dt = 0; dt < C::DT; ++dt)
         acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
       const float *urow = p.U + ((int64_t)b_idx * p.Hq + hq0 + g) * M;
-      const bool live = g < Gg;
-      if constexpr (DEC_S8) {
-        // S q of head g as integers: u ~= hscale * (256 hi + lo), |256 hi + lo|
-        // <= 32000, hi and lo int8 (rows g and g + 8 of the A operand)
-        float amax = 0.f;
-        for (int q = 0; q < M / 16; ++q) {
-          const int Qr = t * (M / 16) + q;
-          const int ib = 32 * (Qr >> 3) + (Qr & 7);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) amax = fmaxf(amax, live ? fabsf(urow[ib + 8 * j]) : 0.f);
-        }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        hscale = amax > 0.f ? amax / 32000.f : 0.f;
-        const float inv = amax > 0.f ? 32000.f / amax : 0.f;
-        int lsum_i = 0;
-#pragma unroll
-        for (int c = 0; c < C::NC; ++c) {
-          uint32_t a4[4];
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int Qr = t * (M / 16) + 2 * c + r;  // byte-register index in the code
-            const int ib = 32 * (Qr >> 3) + (Qr & 7);
-            int hi[4], lo[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int ui = live ? __float2int_rn(urow[ib + 8 * j] * inv) : 0;
-              lsum_i += ui;
-              hi[j] = (ui + 128) >> 8;
-              lo[j] = ui - (hi[j] << 8);
-            }
-            a4[r == 0 ? 0 : 2] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
-            a4[r == 0 ? 1 : 3] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
-          }
-          if constexpr (C::A_SMEM) {
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
-                             ring.afrag() + (c * 32 + lane) * 16),
-                         "r"(a4[0]), "r"(a4[1]), "r"(a4[2]), "r"(a4[3])
-                         : "memory");
-          } else {
-            afr[c][0] = a4[0]; afr[c][1] = a4[1];
-            afr[c][2] = a4[2]; afr[c][3] = a4[3];
-          }
-        }
-        lsum_i += __shfl_xor_sync(0xffffffffu, lsum_i, 1);
-        lsum_i += __shfl_xor_sync(0xffffffffu, lsum_i, 2);
-        usum = lsum_i;
-      } else {
-        // A fragments: rows 0..7 bf16(u), rows 8..15 bf16(u - bf16(u))
-#pragma unroll
-        for (int c = 0; c < C::NC; ++c) {
-          uint32_t a4[4];
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int Qp = t * (M / 8) + 2 * c + r;  // pair index in the key code
-            const int ilo = 32 * (Qp >> 4) + (Qp & 15);
-            const float x0 = live ? urow[ilo] : 0.f;
-            const float x1 = live ? urow[ilo + 16] : 0.f;
-            const float h0 = bf16_round_f32(x0), h1 = bf16_round_f32(x1);
-            a4[2 * r] = pack_bf16x2(h0, h1);
-            a4[2 * r + 1] = pack_bf16x2(x0 - h0, x1 - h1);
-          }
-          if constexpr (C::A_SMEM) {
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
-                             ring.afrag() + (c * 32 + lane) * 16),
-                         "r"(a4[0]), "r"(a4[1]), "r"(a4[2]), "r"(a4[3])
-                         : "memory");
-          } else {
-            afr[c][0] = a4[0]; afr[c][1] = a4[1];
-            afr[c][2] = a4[2]; afr[c][3] = a4[3];
-          }
-        }
-      }
+      build_afrags<M, D, S8>(urow, g < Gg, t, ring, afr, hscale, usum);
       if constexpr (C::A_SMEM) __syncwarp();
     }
 
@@ -417,7 +569,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 
     // ---- raw estimator sum_i u_i sign_i for head g, keys kg*8 + 2t + j
     float raw[4][2];
-    if constexpr (DEC_S8) {
+    if constexpr (S8) {
       int sc[4][4];
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0;
@@ -495,7 +647,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // ---- estimator, masking, online softmax (head g, keys kg*8 + 2t + j)
     float l2[4][2];
     float bmax = -INFINITY;
-    const uint32_t nrow = ring.norm(s) + (uint32_t)((kv_base + key0) & 7) * 2;
+    const uint32_t nrow =
+        ring.norm(s) + (maps.tma_codes ? 0u : (uint32_t)((kv_base + key0) & 7) * 2);
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
 #pragma unroll
@@ -537,10 +690,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // rescale the accumulator: lane holds heads 2t and 2t+1
     const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
     const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
+    if (__any_sync(0xffffffffu, (al0 != 1.f) || (al1 != 1.f))) {
 #pragma unroll
-    for (int dt = 0; dt < C::DT; ++dt) {
-      acc[dt][0] *= al0; acc[dt][1] *= al1;
-      acc[dt][2] *= al0; acc[dt][3] *= al1;
+      for (int dt = 0; dt < C::DT; ++dt) {
+        acc[dt][0] *= al0; acc[dt][1] *= al1;
+        acc[dt][2] *= al0; acc[dt][3] *= al1;
+      }
     }
 
     // ---- P.V: two k-steps of 16 keys over the swizzled value tile
@@ -564,11 +719,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // ---- refill this stage with the block STAGES ahead
     __syncwarp();
     if (i + C::STAGES < nblk) {
-      issue_block<M, D>(p, &vmap, ring, ipos, s, lane);
+      issue_block<M, D, S8>(p, maps, ring, ipos, s, lane);
       ipos.next(p.nb_u);
     }
     pos.next(p.nb_u);
   }
+  griddep_launch_dependents();
   if (failed) {
     // let the copies already started land before the warp's smem goes away
     for (int k = 0; k < C::STAGES; ++k) {
@@ -583,11 +739,20 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 }
 
 // ---------------------------------------------------------------------------
-// 3. combine the partial states of each (b, query head)
+// 3. combine the partial states of each (b, query head).  Warp 0 reads every
+// slot's (max, sum) at once and leaves the slot weights in shared memory; then
+// each thread (one output dimension) sums its weighted column with several
+// loads in flight.
+// one unit can be split over every warp of the launch: at most W_bound + 1
+constexpr int COMB_MAX_SLOTS = DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS + 1;
+
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(
     const float *__restrict__ partials, uint16_t *__restrict__ out, int Hq,
     int Hkv, int G, int HG, int64_t nb_u, int64_t NB, int W, int slots) {
+  __shared__ float wts[COMB_MAX_SLOTS];
+  __shared__ float inv_l;
+  griddep_wait();  // every partial state of the scorer is needed
   const int bh = blockIdx.x;
   const int b = bh / Hq, hq = bh - b * Hq;
   const int hkv = hq / G, hl = hq - hkv * G;
@@ -595,21 +760,32 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
   const int64_t u = ((int64_t)b * Hkv + hkv) * HG + hg;
   const int f = warp_of_block(u * nb_u, NB, W);
   const int l = warp_of_block((u + 1) * nb_u - 1, NB, W);
-  const int n = min(l - f + 1, slots);
+  const int n = min(min(l - f + 1, slots), COMB_MAX_SLOTS);
   const float *rec0 = partials + (size_t)u * slots * DEC_HPAD * (D + 2) +
                       (size_t)hh * (D + 2);
   const size_t sstride = (size_t)DEC_HPAD * (D + 2);
-  float Mx = -INFINITY;
-  for (int s = 0; s < n; ++s) Mx = fmaxf(Mx, rec0[s * sstride + D]);
-  float L = 0.f, o = 0.f;
-  const int dim = threadIdx.x;
-  for (int s = 0; s < n; ++s) {
-    const float *rec = rec0 + s * sstride;
-    const float wgt = fast_exp2(rec[D] - Mx);
-    L = fmaf(wgt, rec[D + 1], L);
-    o = fmaf(wgt, rec[dim], o);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float mx = -INFINITY;
+    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, rec0[s * sstride + D]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float L = 0.f;
+    for (int s = lane; s < n; s += 32) {
+      const float wgt = fast_exp2(rec0[s * sstride + D] - mx);
+      wts[s] = wgt;
+      L = fmaf(wgt, rec0[s * sstride + D + 1], L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) inv_l = 1.f / L;
   }
-  out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o / L));
+  __syncthreads();
+  const int dim = threadIdx.x;
+  float o = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < n; ++s) o = fmaf(wts[s], rec0[s * sstride + dim], o);
+  out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o * inv_l));
 }
 
 // ---------------------------------------------------------------------------
@@ -637,7 +813,7 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
   // shapes only
   const int64_t wb = (int64_t)DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS;
   p.W = (int)(p.NB < wb ? p.NB : wb);
-  p.slots = (int)((p.W + p.units - 1) / p.units) + 1;
+  p.slots = (int)((p.W + p.units - 1) / p.units) + 1;  // <= W_bound + 1 <= 2369
   p.u_bytes = round_up((size_t)B * Hq * m * sizeof(float), 256);
   p.partial_bytes = round_up(
       (size_t)p.units * p.slots * DEC_HPAD * (d + 2) * sizeof(float), 256);
@@ -646,43 +822,96 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
   return true;
 }
 
-// V viewed as [B*Hkv][T][d] bf16; boxes of 64 columns x 32 rows x 1 unit with
-// the 128-byte swizzle; rows past T are zero-filled.
-static bool make_value_map(CUtensorMap *map, const uint16_t *V, int64_t units_kv,
-                           int64_t T, int d) {
+// Tensor maps of one call (see DecMaps).
+static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
+                      const uint16_t *norms, int64_t units_kv, int64_t T, int m, int d) {
   auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)units_kv};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)T * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)DEC_KB, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(V), dims,
-            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  {  // values [B*Hkv][T][d]: 64 columns x 32 rows x 1 unit, 128-byte swizzle
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)units_kv};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)T * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)DEC_KB, 1};
+    if (fn(&mp->value, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(V),
+           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  mp->tma_codes = 0;
+  mp->sign_elem = (m > 256) ? 8 : 4;
+  if (T % 8 != 0) return true;  // per-unit rows not 16-byte aligned: cp.async path
+  {  // codes [B*Hkv][T * m/8 bytes] as 4- or 8-byte elements, one block per box
+    const int es = mp->sign_elem;
+    cuuint64_t dims[2] = {(cuuint64_t)(T * (m / 8) / es), (cuuint64_t)units_kv};
+    cuuint64_t strides[1] = {(cuuint64_t)T * (m / 8)};
+    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * (m / 8) / es), 1};
+    if (fn(&mp->sign, es == 8 ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
+           2, const_cast<uint32_t *>(signs), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return true;
+  }
+  {  // norms [B*Hkv][T] binary16, 32 per box
+    cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)units_kv};
+    cuuint64_t strides[1] = {(cuuint64_t)T * 2};
+    cuuint32_t box[2] = {(cuuint32_t)DEC_KB, 1};
+    if (fn(&mp->norm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(norms), dims,
+           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return true;
+  }
+  mp->tma_codes = 1;
+  return true;
 }
 
-template <int M, int D>
+// Scoring MMA for a shape: int8 (half the sign-expansion work and MMAs per
+// key) unless a bf16 build is forced; see the measurements in the design
+// notes for the per-shape choice.
+static bool decode_use_s8(int G, int m) {
+  if (JL_DECODE_SCORE == 1) return false;
+  if (JL_DECODE_SCORE == 2) return true;
+  return G == 1 || m > 256;
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <int M, int D, bool S8>
 static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
                                    bool q_f32, const uint16_t *S,
                                    const uint32_t *signs, const uint16_t *norms,
                                    const uint16_t *V, float softmax_scale,
                                    uint16_t *out, float *scores,
                                    void *workspace, cudaStream_t stream) {
-  using C = DecCfg<M, D>;
+  using C = DecCfg<M, D, S8>;
   float *U = reinterpret_cast<float *>(workspace);
   float *partials =
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
-  CUtensorMap vmap;
-  if (!make_value_map(&vmap, V, (int64_t)pl.B * pl.Hkv, pl.T, D))
+  DecMaps maps;
+  if (!make_maps(&maps, V, signs, norms, (int64_t)pl.B * pl.Hkv, pl.T, M, D))
     return cudaErrorInvalidValue;
   int *err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidSymbol;
   const int bh = pl.B * pl.Hq;
+  const int qblocks = (bh + QPB - 1) / QPB;
   if (q_f32)
-    qproj_kernel<M, D, true><<<bh, 128, 0, stream>>>(Q, S, U);
+    qproj_kernel<M, D, true><<<qblocks, M, 0, stream>>>(Q, S, U, bh);
   else
-    qproj_kernel<M, D, false><<<bh, 128, 0, stream>>>(Q, S, U);
+    qproj_kernel<M, D, false><<<qblocks, M, 0, stream>>>(Q, S, U, bh);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -694,27 +923,24 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   p.slots = pl.slots;
   p.coef = (float)(sqrt(M_PI / 2.0) / (double)M);
   p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
-  e = cudaFuncSetAttribute(decode_scorer_kernel<M, D>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::CTA_BYTES);
+  auto kern = decode_scorer_kernel<M, D, S8>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::CTA_BYTES);
   if (e != cudaSuccess) return e;
   // one wave of resident CTAs, never more warps than the plan's bound
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_scorer_kernel<M, D>,
-                                                    DEC_WARPS * 32, C::CTA_BYTES);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DEC_WARPS * 32,
+                                                    C::CTA_BYTES);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   if (per_sm > DEC_MAX_CTAS_SM) per_sm = DEC_MAX_CTAS_SM;
   const int64_t wave = (int64_t)device_sm_count() * per_sm * DEC_WARPS;
   p.W = (int)(wave < pl.W ? wave : pl.W);
   const int ctas = (p.W + DEC_WARPS - 1) / DEC_WARPS;
-  decode_scorer_kernel<M, D><<<ctas, DEC_WARPS * 32, C::CTA_BYTES, stream>>>(vmap, p);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(ctas), dim3(DEC_WARPS * 32), C::CTA_BYTES, stream, maps, p);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<D><<<bh, D, 0, stream>>>(partials, out, pl.Hq, pl.Hkv,
-                                                 pl.G, pl.HG, pl.nb_u, pl.NB,
-                                                 p.W, pl.slots);
-  return cudaGetLastError();
+  return launch_pdl(decode_combine_kernel<D>, dim3(bh), dim3(D), 0, stream,
+                    (const float *)partials, out, pl.Hq, pl.Hkv, pl.G, pl.HG, pl.nb_u,
+                    pl.NB, p.W, pl.slots);
 }
 
 cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
@@ -722,11 +948,15 @@ cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
                           const uint16_t *norms, const uint16_t *V,
                           float softmax_scale, uint16_t *out, float *scores,
                           void *workspace, cudaStream_t stream) {
-#define JL_CASE(MM, DD)                                                       \
-  if (pl.m == MM && pl.d == DD)                                               \
-    return launch_decode_t<MM, DD>(pl, Q, q_f32, S, signs, norms, V,          \
-                                   softmax_scale, out, scores, workspace,     \
-                                   stream);
+  const bool s8 = decode_use_s8(pl.G, pl.m);
+#define JL_CASE(MM, DD)                                                         \
+  if (pl.m == MM && pl.d == DD)                                                 \
+    return s8 ? launch_decode_t<MM, DD, true>(pl, Q, q_f32, S, signs, norms, V, \
+                                              softmax_scale, out, scores,       \
+                                              workspace, stream)                \
+              : launch_decode_t<MM, DD, false>(pl, Q, q_f32, S, signs, norms, V, \
+                                               softmax_scale, out, scores,      \
+                                               workspace, stream);
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
 #undef JL_CASE

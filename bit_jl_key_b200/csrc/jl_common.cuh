@@ -175,6 +175,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; griddep_wait() blocks
+// until the predecessor has completed and its writes are visible, and
+// griddep_launch_dependents() lets the next kernel start early.  Both are
+// no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // Host: the driver's cuTensorMapEncodeTiled (through the runtime's entry
 // point query, so the library does not link libcuda); null if unavailable.
 void *tensor_map_encoder();

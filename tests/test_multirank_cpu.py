@@ -1,0 +1,72 @@
+"""Multi-rank host logic of the bench on CPU (gloo, world size 2).
+
+The decode and quantize path shards by independent (batch, kv-head) units, so
+ranks run independent batches and the only collective is the max over ranks
+of the step time.  This checks that reduction and the whole-job rate, and
+that the reference arm prints on rank 0 only.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, times, out_q):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = bench.reduce_max_over_ranks(times[rank], world, torch.device("cpu"))
+        rate = bench.whole_job_rate(1000, world, ms)
+        out_q.put((rank, ms, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_rate():
+    world = 2
+    times = [3.0, 5.0]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, times, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, rate in res:
+        assert ms == 5.0
+        assert rate == pytest.approx(2 * 1000 / 5e-3)
+
+
+def test_single_rank_rate_is_plain():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max_over_ranks(2.5, 1, torch.device("cpu")) == 2.5
+    assert bench.whole_job_rate(500, 1, 2.0) == pytest.approx(250000.0)
+
+
+def test_reference_arm_prints_on_rank_zero_only():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0", "--workload", "single"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
