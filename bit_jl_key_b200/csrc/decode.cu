@@ -120,53 +120,36 @@ __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
 }
 
 // ---------------------------------------------------------------------------
-// 1. query projection u = S q (fp32 accumulate).  A CTA projects QPB queries;
-// thread i owns sketch row i, reads it once (16-byte loads, L2-resident) and
-// applies it to all QPB queries held in shared memory.
-constexpr int QPB = 8;
-
+// 1. query projection u = S q (fp32 accumulate).  One CTA per query, thread i
+// owns sketch row i and issues all of its 16-byte loads before the first
+// multiply (one memory round trip; S is L2-resident after the first call).
 template <int M, int D, bool QF32>
 __global__ void __launch_bounds__(M) qproj_kernel(const void *__restrict__ Q,
                                                   const uint16_t *__restrict__ S,
-                                                  float *__restrict__ U, int nq) {
-  __shared__ float qs[QPB][D];
+                                                  float *__restrict__ U) {
+  __shared__ float qs[D];
   griddep_launch_dependents();  // let the scorer start its copies now
-  const int q0 = blockIdx.x * QPB;
-  const int nloc = min(QPB, nq - q0);
-  for (int e = threadIdx.x; e < QPB * D; e += M) {
-    const int j = e / D, c = e - j * D;
-    float v = 0.f;
-    if (j < nloc) {
-      const int64_t idx = (int64_t)(q0 + j) * D + c;
-      v = QF32 ? reinterpret_cast<const float *>(Q)[idx]
-               : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[idx]);
-    }
-    qs[j][c] = v;
-  }
-  __syncthreads();
+  const int bh = blockIdx.x;
   const int i = threadIdx.x;
-  const uint4 *row = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
-  float acc[QPB];
+  uint4 row[D / 8];
+  const uint4 *src = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
 #pragma unroll
-  for (int j = 0; j < QPB; ++j) acc[j] = 0.f;
-#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) row[c] = __ldg(src + c);
+  for (int j = i; j < D; j += M)
+    qs[j] = QF32 ? reinterpret_cast<const float *>(Q)[(int64_t)bh * D + j]
+                 : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[(int64_t)bh * D + j]);
+  __syncthreads();
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
   for (int c = 0; c < D / 8; ++c) {
-    const uint4 v = __ldg(row + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t w[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float s0 = __uint_as_float(w[e] << 16);
-      const float s1 = __uint_as_float(w[e] & 0xFFFF0000u);
-#pragma unroll
-      for (int j = 0; j < QPB; ++j) {
-        acc[j] = fmaf(s0, qs[j][c * 8 + 2 * e], acc[j]);
-        acc[j] = fmaf(s1, qs[j][c * 8 + 2 * e + 1], acc[j]);
-      }
+      acc0 = fmaf(__uint_as_float(w[e] << 16), qs[c * 8 + 2 * e], acc0);
+      acc1 = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), qs[c * 8 + 2 * e + 1], acc1);
     }
   }
-#pragma unroll
-  for (int j = 0; j < QPB; ++j)
-    if (j < nloc) U[(int64_t)(q0 + j) * M + i] = acc[j];
+  U[(int64_t)bh * M + i] = acc0 + acc1;
 }
 
 // ---------------------------------------------------------------------------
@@ -765,16 +748,23 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
                       (size_t)hh * (D + 2);
   const size_t sstride = (size_t)DEC_HPAD * (D + 2);
   if (threadIdx.x < 32) {
+    // (max, sum) of every slot in one round of loads; slots past 32 per lane
+    // are rare (one unit spread over more than 32 warps)
     const int lane = threadIdx.x;
     float mx = -INFINITY;
-    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, rec0[s * sstride + D]);
+    for (int s = lane; s < n; s += 32) {
+      const float ms = rec0[s * sstride + D];
+      wts[s] = ms;
+      mx = fmaxf(mx, ms);
+    }
+    const float lsl = lane < n ? rec0[lane * sstride + D + 1] : 0.f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float L = 0.f;
     for (int s = lane; s < n; s += 32) {
-      const float wgt = fast_exp2(rec0[s * sstride + D] - mx);
+      const float wgt = fast_exp2(wts[s] - mx);
       wts[s] = wgt;
-      L = fmaf(wgt, rec0[s * sstride + D + 1], L);
+      L = fmaf(wgt, s == lane ? lsl : rec0[s * sstride + D + 1], L);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -782,9 +772,14 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
   }
   __syncthreads();
   const int dim = threadIdx.x;
+  // the first 32 slots: every load issued before the first multiply
+  float v[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) v[s] = s < n ? rec0[s * sstride + dim] : 0.f;
   float o = 0.f;
-#pragma unroll 8
-  for (int s = 0; s < n; ++s) o = fmaf(wts[s], rec0[s * sstride + dim], o);
+#pragma unroll
+  for (int s = 0; s < 32; ++s) o = s < n ? fmaf(wts[s], v[s], o) : o;
+  for (int s = 32; s < n; ++s) o = fmaf(wts[s], rec0[s * sstride + dim], o);
   out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o * inv_l));
 }
 
@@ -907,11 +902,10 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   int *err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidSymbol;
   const int bh = pl.B * pl.Hq;
-  const int qblocks = (bh + QPB - 1) / QPB;
   if (q_f32)
-    qproj_kernel<M, D, true><<<qblocks, M, 0, stream>>>(Q, S, U, bh);
+    qproj_kernel<M, D, true><<<bh, M, 0, stream>>>(Q, S, U);
   else
-    qproj_kernel<M, D, false><<<qblocks, M, 0, stream>>>(Q, S, U, bh);
+    qproj_kernel<M, D, false><<<bh, M, 0, stream>>>(Q, S, U);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 

@@ -8,7 +8,7 @@
 
 #include <cuda.h>
 
-#include "../../include/jlkey.h"
+#include "jlkey.h"
 
 namespace jlk {
 

@@ -5,7 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/jlkey.h"
+#include "jlkey.h"
 
 namespace jlk {
 

@@ -40,22 +40,32 @@ namespace jlk {
 namespace tc {
 
 constexpr int BM = 128;           // keys per tile (MMA M)
-constexpr int NWARPS = 10;
-constexpr int THREADS = NWARPS * 32;
+// Sign-epilogue warps per TMEM lane quadrant: 0 = chosen per shape.
+#ifndef JL_QTC_SIGN_WARPS
+#define JL_QTC_SIGN_WARPS 0
+#endif
 constexpr int SMEM_BUDGET = 220 * 1024;
 constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
 
 template <int M, int D>
 struct Cfg {
+  // two sign warps per quadrant when the epilogue has many columns per byte
+  // of key read (m >= 4 d) or a single accumulator (m = 512)
+  static constexpr int SQ = JL_QTC_SIGN_WARPS ? JL_QTC_SIGN_WARPS
+                                              : ((M >= 4 * D || M > 256) ? 2 : 1);
+  static constexpr int NWARPS = 2 + 4 * SQ + 4;
+  static constexpr int THREADS = NWARPS * 32;
+  static constexpr int FIRST_NORM_WARP = 2 + 4 * SQ;
   static constexpr int KCH = D / 64;                 // 128-byte swizzle columns
   static constexpr int A_CHUNK = BM * 128;           // one swizzle column of a tile
   static constexpr int A_STAGE = BM * D * 2;
   static constexpr int S_CHUNK = M * 128;
   static constexpr int S_BYTES = M * D * 2;
-  static constexpr int NH = (M > 256) ? 2 : 1;       // MMAs per K step (N halves)
+  static constexpr int NH = (M > 256) ? 2 : 1;       // N halves (work items) per tile
   static constexpr int NMMA = M / NH;                // N of one MMA (<= 256)
-  static constexpr int ACC = (M > 256) ? 1 : 2;      // accumulator buffers
-  static constexpr int TMEM_COLS = (ACC * M < 32) ? 32 : ACC * M;
+  static constexpr int ACC = 2;                      // accumulator buffers (items)
+  static constexpr int TMEM_COLS = ACC * NMMA;
+  static constexpr int WORDS_ITEM = NMMA / 32;       // code words per item
   static constexpr int STAGES_RAW = (SMEM_BUDGET - S_BYTES) / A_STAGE;
   static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
   static constexpr int WORDS = M / 32;
@@ -148,7 +158,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
 
 // --------------------------------------------------------------------------
 template <int M, int D>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_s,
                        const Params p) {
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < C::ACC; ++a) {
       mbar_init(tfull_bar(a), 1);       // MMA commit
-      mbar_init(tempty_bar(a), 4);      // 4 sign warps
+      mbar_init(tempty_bar(a), 4 * C::SQ);  // the sign warps
     }
     mbar_init(sfull_bar, 1);
     *abort_flag = 0;
@@ -242,87 +252,98 @@ __global__ void __launch_bounds__(THREADS, 1)
                                  | ((uint32_t)(C::NMMA >> 3) << 17)  // N
                                  | ((uint32_t)(BM >> 4) << 24);      // M
       bool ok = wait_phase(sfull_bar, 0, abort_flag, p.err);
-      int64_t i = 0;
+      int64_t i = 0, j = 0;  // tiles and items (tile x N-half) issued
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
         const int s = (int)(i % C::STAGES);
         const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
-        const int a = (int)(i % C::ACC);
-        const uint32_t aph = (uint32_t)((i / C::ACC) & 1);
-        if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err)) break;
         if (!wait_phase(full_bar(s), ph, abort_flag, p.err)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-          const uint64_t adesc =
-              smem_desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
-#pragma unroll
-          for (int h = 0; h < C::NH; ++h) {
-            const uint64_t bdesc = smem_desc_sw128(
-                sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
-            mma_bf16_ss(tmem_base + a * M + h * C::NMMA, adesc, bdesc, idesc,
-                        kk > 0 ? 1u : 0u);
+        for (int h = 0; h < C::NH; ++h, ++j) {
+          const int a = (int)(j & 1);
+          const uint32_t aph = (uint32_t)((j >> 1) & 1);
+          if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+            const uint64_t adesc =
+                smem_desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
+            const uint64_t bdesc =
+                smem_desc_sw128(sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
+            mma_bf16_ss(tmem_base + a * C::NMMA, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(tfull_bar(a));
         }
+        if (!ok) break;
         mma_commit(empty_bar(s));
-        mma_commit(tfull_bar(a));
       }
       // drain: the last accumulator's MMAs must be complete before TMEM is freed
-      if (i > 0) {
-        const int64_t j = i - 1;
-        const int a = (int)(j % C::ACC);
-        const uint32_t aph = (uint32_t)((j / C::ACC) & 1);
+      if (j > 0) {
+        const int64_t jl = j - 1;
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(tfull_bar(a), aph) && globaltimer() - t0 < WAIT_NS) {
+        while (!mbar_try_wait(tfull_bar((int)(jl & 1)), (uint32_t)((jl >> 1) & 1)) &&
+               globaltimer() - t0 < WAIT_NS) {
         }
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ---------------- sign epilogue (TMEM lane quadrant warp % 4)
+  } else if (warp < C::FIRST_NORM_WARP) {
+    // ---------------- sign epilogue: TMEM lane quadrant warp % 4, and the
+    // k-th of the quadrant's SQ shares of each item's code words
     const int q = warp & 3;
-    int64_t i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-      const int a = (int)(i % C::ACC);
-      const uint32_t aph = (uint32_t)((i / C::ACC) & 1);
-      if (!wait_phase(tfull_bar(a), aph, abort_flag, p.err)) break;
-      __syncwarp();
-      tc_fence_after();
-      // 4 code words (128 columns) per step: at most 4 TMEM slices are live,
-      // whatever the number of sketch rows
-      constexpr int GW = C::WORDS < 4 ? C::WORDS : 4;
-      const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * M);
+    const int k = (warp - 2) >> 2;
+    constexpr int WPW = C::WORDS_ITEM / C::SQ;  // code words per sign warp and item
+    constexpr int GW = WPW < 4 ? WPW : 4;       // words per 16/8/4-byte store
+    int64_t j = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
       const int64_t row = tile * BM + 32 * q + lane;
-      uint32_t *dst = p.signs + row * C::WORDS;
       const bool live = row < p.n;
+      for (int h = 0; h < C::NH; ++h, ++j) {
+        const int a = (int)(j & 1);
+        const uint32_t aph = (uint32_t)((j >> 1) & 1);
+        if (!wait_phase(tfull_bar(a), aph, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * C::NMMA);
+        uint32_t *dst = p.signs + row * C::WORDS + h * C::WORDS_ITEM;
+        // GW words (32 columns each) per step bound the live TMEM slices
 #pragma unroll 1
-      for (int w0 = 0; w0 < C::WORDS; w0 += GW) {
-        uint32_t words[GW];
+        for (int w0 = k * WPW; w0 < (k + 1) * WPW; w0 += GW) {
+          uint32_t words[GW];
 #pragma unroll
-        for (int w = 0; w < GW; ++w) {
-          uint32_t v[32];
-          tmem_ld32(trow + 32 * (w0 + w), v);
-          tmem_ld_wait();
-          uint32_t word = 0;
+          for (int w = 0; w < GW; ++w) {
+            uint32_t v[32];
+            tmem_ld32(trow + 32 * (w0 + w), v);
+            tmem_ld_wait();
+            uint32_t word = 0;
 #pragma unroll
-          for (int j = 31; j >= 0; --j) word = __funnelshift_l(v[j], word, 1);
-          words[w] = ~word;  // bit j = 1 iff column 32(w0+w) + j is >= 0
+            for (int jj = 31; jj >= 0; --jj) word = __funnelshift_l(v[jj], word, 1);
+            words[w] = ~word;  // bit jj = 1 iff that column is >= 0
+          }
+          if (live) {
+            if constexpr (GW == 1)
+              dst[w0] = words[0];
+            else if constexpr (GW == 2)
+              *reinterpret_cast<uint2 *>(dst + w0) = make_uint2(words[0], words[1]);
+            else
+              *reinterpret_cast<uint4 *>(dst + w0) =
+                  make_uint4(words[0], words[1], words[2], words[3]);
+          }
         }
-        if (live) {
-          if constexpr (GW == 2)
-            *reinterpret_cast<uint2 *>(dst + w0) = make_uint2(words[0], words[1]);
-          else
-            *reinterpret_cast<uint4 *>(dst + w0) =
-                make_uint4(words[0], words[1], words[2], words[3]);
-        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(a));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(a));
     }
   } else {
     // ---------------- norm epilogue: rows 32*(warp-6) .. +31 of each tile
-    const int r = 32 * (warp - 6) + lane;
+    const int r = 32 * (warp - C::FIRST_NORM_WARP) + lane;
     int64_t i = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = (int)(i % C::STAGES);
@@ -399,7 +420,7 @@ cudaError_t launch_t(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  quantize_tc_kernel<M, D><<<(int)grid, THREADS, C::SMEM, stream>>>(mk, ms, p);
+  quantize_tc_kernel<M, D><<<(int)grid, C::THREADS, C::SMEM, stream>>>(mk, ms, p);
   return cudaGetLastError();
 }
 

@@ -136,6 +136,14 @@ DECODE_CASES = [
     (1, 3, 3, 4096, 512, 64, torch.bfloat16, 4.0),   # peaked softmax
     (3, 6, 2, 2049, 128, 128, torch.float32, 1.0),
     (1, 8, 8, 8192, 64, 128, torch.bfloat16, 1.0),
+    # head groups of 8 on the bulk-tensor copy path (T % 8 == 0)
+    (1, 16, 1, 1024, 256, 128, torch.bfloat16, 2.0),
+    (2, 12, 1, 512, 128, 64, torch.bfloat16, 1.0),
+    # int8 scoring (one head per KV head, or m = 512) on both copy paths
+    (1, 4, 4, 2048, 256, 128, torch.bfloat16, 3.0),
+    (1, 4, 4, 1001, 128, 64, torch.bfloat16, 1.0),
+    (1, 2, 2, 512, 512, 128, torch.bfloat16, 2.0),
+    (2, 4, 1, 777, 512, 64, torch.bfloat16, 1.0),
 ]
 
 
