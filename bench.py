@@ -180,6 +180,30 @@ def decode_bytes(w):
     return w.B * w.Hkv * w.T * (w.m // 8 + 2 + 2 * w.d)
 
 
+def score_error(jl, w, Q, S, signs, norms, V, K, max_rows=16):
+    """Normalised error of the GPU estimator against the exact inner product
+    on sampled (b, query head) rows: rms over keys of (s - <q,k>) / (|q||k|),
+    next to the closed form sqrt((pi/2 - 1/d) / m) of the estimator's variance
+    for independent Gaussian q, k.  Measurement only (exact products by a
+    plain fp32 matmul of the stored bf16 values)."""
+    out, sc = jl.jl_decode_attention(Q, S, signs, norms, V,
+                                     softmax_scale=w.softmax_scale, want_scores=True)
+    rows = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    step = max(1, len(rows) // max_rows)
+    errs = []
+    for (b, h) in rows[::step][:max_rows]:
+        q = Q[b, h].float()
+        k = K[b, h // w.G].float()
+        exact = k @ q
+        denom = k.norm(dim=1) * q.norm()
+        errs.append(((sc[b, h] - exact) / denom).double())
+    e = torch.cat(errs)
+    return {"rms_normalised": float(torch.sqrt(torch.mean(e * e))),
+            "predicted": math.sqrt((math.pi / 2 - 1.0 / w.d) / w.m),
+            "bits_per_key": w.m + 16, "bits_per_coordinate": (w.m + 16) / w.d,
+            "samples": int(e.numel())}
+
+
 # --------------------------------------------------------------------------
 # our arm
 
@@ -254,6 +278,11 @@ def run_ours(args, rank, world, local_rank):
     ms_step = reduce_max_over_ranks(ms_total / args.steps, world, dev)
     keys_all = n_keys * world
     value = whole_job_rate(n_keys, world, ms_step)
+
+    # ---- estimator quality on sampled heads (untimed)
+    score_err = None
+    if decode and not args.no_score_error:
+        score_err = score_error(jl, w, Q, S, sg4, nr3, V, K)
 
     # ---- end to end through the binding with pinned host buffers
     e2e = None
@@ -343,6 +372,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs exceed L2 (126 MB); no flush"},
         "phases": phases,
         "roofline": roof,
+        "score_error": score_err,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -432,6 +462,7 @@ def main():
                     help="override the workload's batch (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-score-error", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
