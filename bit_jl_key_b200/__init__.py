@@ -46,7 +46,8 @@ DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_quantize_keys_simt", "jl_decode_workspace_bytes",
             "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64",
-            "jl_decode_attention_noalloc")
+            "jl_decode_attention_noalloc", "jl_decode_paged_workspace_bytes",
+            "jl_decode_attention_paged")
 
 _lib = None
 
@@ -86,6 +87,12 @@ def load():
     L.jl_decode_attention_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32,
                                               i32, i64, i32, i32, ctypes.c_float,
                                               vp, vp, vp]
+    L.jl_decode_paged_workspace_bytes.restype = sz
+    L.jl_decode_paged_workspace_bytes.argtypes = [i32, i32, i32, i64, i32, i32]
+    L.jl_decode_attention_paged.restype = i32
+    L.jl_decode_attention_paged.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
+                                            vp, i32, vp, i32, i32, i32, i64, i32, i32,
+                                            ctypes.c_float, vp, vp, vp, sz, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.jl_bf16_from_f64.restype = ctypes.c_uint16
@@ -254,6 +261,62 @@ def jl_decode_attention_noalloc(Q, S, signs, norms, V, softmax_scale=None,
                                          _ptr(out), _ptr(scores),
                                          _stream(Q, stream)),
            "jl_decode_attention_noalloc")
+    if scores is not None:
+        return out, scores
+    return out
+
+
+def jl_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d) -> int:
+    return int(load().jl_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d))
+
+
+def jl_decode_attention_paged(Q, S, sign_pages, norm_pages, value_pages, block_table,
+                              seq_lens, max_len, K_new=None, V_new=None,
+                              softmax_scale=None, out=None, scores=None,
+                              want_scores=False, workspace=None, stream=None):
+    """One decode step over a paged compressed cache of ragged sequences.
+
+    Q [B, Hq, d]; pools sign_pages int32 [P_n, Hkv, P, m/32], norm_pages fp16
+    [P_n, Hkv, P], value_pages bf16 [P_n, Hkv, P, d]; block_table int32
+    [B, max_pages]; seq_lens int32 [B] (device, not modified).  With K_new
+    [B, Hkv, d] and V_new [B, Hkv, d] the new key of every sequence is
+    quantized and stored at position seq_lens[b] first, and attention covers
+    seq_lens[b] + 1 keys.  Returns out [B, Hq, d] (and scores [B, Hq, max_len]).
+    """
+    L = load()
+    B, Hq, d = Q.shape
+    num_pages, Hkv, P, W = sign_pages.shape
+    m = W * 32
+    _need_cuda(Q, S, sign_pages, norm_pages, value_pages, block_table, seq_lens, K_new, V_new)
+    assert S.shape == (m, d) and S.dtype == torch.bfloat16
+    assert norm_pages.shape == (num_pages, Hkv, P) and norm_pages.dtype == torch.float16
+    assert value_pages.shape == (num_pages, Hkv, P, d) and value_pages.dtype == torch.bfloat16
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == B
+    assert seq_lens.dtype == torch.int32 and seq_lens.shape == (B,)
+    for t in (Q, S, sign_pages, norm_pages, value_pages, block_table, seq_lens, K_new, V_new):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("paged decode inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    kt = JL_BF16
+    if K_new is not None:
+        assert K_new.shape == (B, Hkv, d) and V_new is not None and V_new.shape == (B, Hkv, d)
+        kt = JL_F32 if K_new.dtype == torch.float32 else JL_BF16
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=Q.device)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, max_len), dtype=torch.float32, device=Q.device)
+    need = jl_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_decode_attention_paged(
+        _ptr(Q), qt, _ptr(K_new), kt, _ptr(V_new), _ptr(S), _ptr(sign_pages),
+        _ptr(norm_pages), _ptr(value_pages), num_pages, P, _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, max_len, m, d,
+        ctypes.c_float(softmax_scale), _ptr(out), _ptr(scores), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(Q, stream)),
+        "jl_decode_attention_paged")
     if scores is not None:
         return out, scores
     return out

@@ -195,6 +195,53 @@ int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
                                       (cudaStream_t)stream));
 }
 
+size_t jl_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len, int m,
+                                       int d) {
+  jlk::DecodePlan p;
+  if (B == 0) return 0;
+  if (!jlk::make_paged_plan(B, Hq, Hkv, max_len, m, d, &p)) return 0;
+  return p.total_bytes;
+}
+
+int jl_decode_attention_paged(
+    const void *Q, jl_dtype q_dtype, const void *K_new, jl_dtype k_dtype,
+    const uint16_t *V_new, const uint16_t *S, uint32_t *sign_pages,
+    uint16_t *norm_pages, uint16_t *value_pages, int num_pages, int page_tokens,
+    const int32_t *block_table, int max_pages, const int32_t *seq_lens, int B, int Hq,
+    int Hkv, int64_t max_len, int m, int d, float softmax_scale, uint16_t *out,
+    float *scores, void *workspace, size_t workspace_bytes, jl_stream_t stream) {
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (K_new && k_dtype != JL_BF16 && k_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || max_len < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
+  if (num_pages < 1 || max_pages < 1 || page_tokens < 32 || page_tokens % 32 != 0)
+    return JL_ERR_INVALID_ARG;
+  if ((int64_t)max_pages * page_tokens < max_len) return JL_ERR_INVALID_ARG;
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
+  if (B == 0) return JL_OK;
+  if (!Q || !S || !sign_pages || !norm_pages || !value_pages || !block_table || !seq_lens ||
+      !out)
+    return JL_ERR_INVALID_ARG;
+  if (K_new && !V_new) return JL_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(S, 16) || !aligned(sign_pages, 16) ||
+      !aligned(norm_pages, 16) || !aligned(value_pages, 16) || !aligned(out, 4) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || (K_new && !aligned(K_new, 16)) ||
+      (V_new && !aligned(V_new, 16)) || (scores && !aligned(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  jlk::DecodePlan p;
+  if (!jlk::make_paged_plan(B, Hq, Hkv, max_len, m, d, &p)) return JL_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
+    return JL_ERR_WORKSPACE;
+  jlk::PagedArgs a;
+  a.Q = Q; a.q_f32 = q_dtype == JL_F32;
+  a.K_new = K_new; a.k_f32 = k_dtype == JL_F32; a.V_new = V_new; a.S = S;
+  a.sign_pages = sign_pages; a.norm_pages = norm_pages; a.value_pages = value_pages;
+  a.num_pages = num_pages; a.page_tokens = page_tokens;
+  a.block_table = block_table; a.max_pages = max_pages; a.seq_lens = seq_lens;
+  a.softmax_scale = softmax_scale; a.out = out; a.scores = scores; a.workspace = workspace;
+  return from_cuda(jlk::launch_decode_paged(p, a, (cudaStream_t)stream));
+}
+
 int jl_device_error(int *code, jl_stream_t stream) {
   if (!code) return JL_ERR_INVALID_ARG;
   *code = 0;

@@ -90,13 +90,21 @@ struct DecParams {
   const float *U;           // [B][Hq][M]
   const uint32_t *signs;    // [B][Hkv][T][M/32]
   const uint16_t *norms;    // [B][Hkv][T]
-  float *partials;          // [units][slots][8][D + 2]
+  float *partials;          // [W + units records][8][D + 2]
   float *scores;            // nullable [B][Hq][T]
   int *err;                 // device error word
   int64_t T, nb_u, NB, n_keys;
-  int Hq, Hkv, G, HG, W, slots;
+  int Hq, Hkv, G, HG, W, slots;  // slots: partial records (W bound + units)
   float coef;               // sqrt(pi/2) / m
   float scale_log2;         // softmax_scale * log2(e)
+  int64_t score_stride;     // row stride of `scores` (T, or max_len when paged)
+  // paged cache (PAGED kernels): unit u = (b, kv head, head group) owns blocks
+  // unit_off[u] .. unit_off[u+1] of the flat block space, written by the prep
+  // kernel from seq_lens; its keys live in pages block_table[b][*]
+  const int64_t *unit_off;  // [units + 1]
+  const int32_t *seq_lens;  // [B]
+  const int32_t *block_table;  // [B][max_pages]
+  int max_pages, page_tokens, append, units;
 };
 
 // Bulk-tensor maps of one decode call.  Values always go through `value`
@@ -155,17 +163,75 @@ __global__ void __launch_bounds__(M) qproj_kernel(const void *__restrict__ Q,
 // ---------------------------------------------------------------------------
 // 2. scorer
 
-// Position of a block in the (unit, block) space, advanced without division.
+// Position of a block in the (unit, block) space, advanced without division,
+// with the geometry of its unit: blocks nb, keys len, kv row kvi = b*Hkv + hkv.
 struct BlockPos {
   int64_t u;    // unit
   int64_t blk;  // block within the unit
-  __device__ __forceinline__ void next(int64_t nb_u) {
-    if (++blk == nb_u) {
-      blk = 0;
-      ++u;
-    }
-  }
+  int64_t nb;   // blocks of unit u
+  int64_t len;  // keys of unit u
+  int64_t kvi;  // b * Hkv + kv head of unit u
 };
+
+template <bool PAGED>
+__device__ __forceinline__ void pos_load_unit(const DecParams &p, BlockPos &pos) {
+  pos.kvi = p.HG == 1 ? pos.u : pos.u / p.HG;
+  if constexpr (PAGED) {
+    pos.nb = p.unit_off[pos.u + 1] - p.unit_off[pos.u];
+    // an invalid length (past the bound) was reported by the prep kernel,
+    // which also capped the unit's blocks; keep every access inside the bound
+    const int64_t len = (int64_t)p.seq_lens[pos.kvi / p.Hkv] + p.append;
+    pos.len = len < p.T ? len : p.T;
+  } else {
+    pos.nb = p.nb_u;
+    pos.len = p.T;
+  }
+}
+
+// Position of flat block b (which must exist).
+template <bool PAGED>
+__device__ __forceinline__ BlockPos pos_of_block(const DecParams &p, int64_t b) {
+  BlockPos pos;
+  if constexpr (PAGED) {
+    // last unit whose first block is <= b (empty units share their offset)
+    int64_t lo = 0, hi = p.units - 1;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (p.unit_off[mid] <= b) lo = mid; else hi = mid - 1;
+    }
+    pos.u = lo;
+    pos.blk = b - p.unit_off[lo];
+  } else {
+    pos.u = b / p.nb_u;
+    pos.blk = b - pos.u * p.nb_u;
+  }
+  pos_load_unit<PAGED>(p, pos);
+  return pos;
+}
+
+template <bool PAGED>
+__device__ __forceinline__ void pos_next(const DecParams &p, BlockPos &pos) {
+  if (++pos.blk < pos.nb) return;
+  pos.blk = 0;
+  if constexpr (PAGED) {
+    // skip units without blocks; never step past the last unit
+    do {
+      if (pos.u + 1 >= p.units) return;
+      ++pos.u;
+      pos_load_unit<PAGED>(p, pos);
+    } while (pos.nb == 0);
+  } else {
+    ++pos.u;
+    pos_load_unit<PAGED>(p, pos);
+  }
+}
+
+// First flat block of unit u.
+template <bool PAGED>
+__device__ __forceinline__ int64_t unit_first_block(const DecParams &p, int64_t u) {
+  if constexpr (PAGED) return p.unit_off[u];
+  else return u * p.nb_u;
+}
 
 template <int M, int D, bool S8>
 struct Ring {
@@ -184,23 +250,31 @@ struct Ring {
 
 // Start the copies of block `pos` into stage s: values by one 3-D bulk-tensor
 // copy per 64 columns (lane 0), codes and norms by cp.async (all lanes).
-template <int M, int D, bool S8>
+template <int M, int D, bool S8, bool PAGED>
 __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &maps,
                                             const Ring<M, D, S8> &ring, const BlockPos &pos,
                                             int s, int lane) {
   using C = DecCfg<M, D, S8>;
-  const int64_t kvi = p.HG == 1 ? pos.u : pos.u / p.HG;
+  const int64_t kvi = pos.kvi;
   const int64_t key0 = pos.blk * DEC_KB;
-  if (maps.tma_codes) {
+  if (PAGED || maps.tma_codes) {
     if (lane == 0) {
+      // row (y) within the tensor's unit (z): the sequence itself, or the page
+      // holding this block (row within the page) for a paged cache
+      int y = (int)key0, z = (int)kvi;
+      if constexpr (PAGED) {
+        const int64_t b = kvi / p.Hkv;
+        const int page = p.block_table[b * p.max_pages + (int)(key0 / p.page_tokens)];
+        y = (int)(key0 % p.page_tokens);
+        z = page * p.Hkv + (int)(kvi - b * p.Hkv);
+      }
       mbar_expect_tx(ring.bar(s), C::V_BYTES + C::SIGN_BYTES + 2 * DEC_KB);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h)
-        tma_load_3d(ring.val(s) + h * C::V_BOX, &maps.value, h * 64, (int)key0, (int)kvi,
-                    ring.bar(s));
-      tma_load_2d(ring.sign(s), &maps.sign,
-                  (int)(key0 * C::KEY_SIGN_BYTES / maps.sign_elem), (int)kvi, ring.bar(s));
-      tma_load_2d(ring.norm(s), &maps.norm, (int)key0, (int)kvi, ring.bar(s));
+        tma_load_3d(ring.val(s) + h * C::V_BOX, &maps.value, h * 64, y, z, ring.bar(s));
+      tma_load_2d(ring.sign(s), &maps.sign, (int)((int64_t)y * C::KEY_SIGN_BYTES / maps.sign_elem),
+                  z, ring.bar(s));
+      tma_load_2d(ring.norm(s), &maps.norm, y, z, ring.bar(s));
     }
     return;
   }
@@ -415,7 +489,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
   if constexpr (C::A_SMEM) __syncwarp();
 }
 
-template <int M, int D, bool S8>
+template <int M, int D, bool S8, bool PAGED>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
     decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
   using C = DecCfg<M, D, S8>;
@@ -424,6 +498,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   const int wid = threadIdx.x >> 5;
   const int w = blockIdx.x * DEC_WARPS + wid;
   if (w >= p.W) return;
+  // a paged call's work plan (and its appended keys) come from the prep kernel
+  if constexpr (PAGED) griddep_wait();
+  const int64_t NB = PAGED ? p.unit_off[p.units] : p.NB;
+  // a paged call is launched for the bound; with fewer blocks than warps the
+  // first NB warps take one block each and the rest have nothing to do (no
+  // warp may own an empty run: the combine reads a record from every warp
+  // between a unit's first and last)
+  const int Wn = PAGED ? (int)(NB < p.W ? NB : p.W) : p.W;
+  if (w >= Wn) return;
   const int g = lane >> 2;  // group id: head row / key column / dim row
   const int t = lane & 3;   // thread in group
   const uint32_t cta = (smem_u32(dsmem_raw) + 1023u) & ~1023u;
@@ -431,9 +514,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
                         cta + C::OFF_NORM + wid * C::STAGES * DEC_NORM_AREA,
                         cta + C::OFF_BAR + wid * C::STAGES * 8};
 
-  const int64_t bbeg = (int64_t)w * p.NB / p.W;
-  const int64_t bend = (int64_t)(w + 1) * p.NB / p.W;
+  const int64_t bbeg = (int64_t)w * NB / Wn;
+  const int64_t bend = (int64_t)(w + 1) * NB / Wn;
   const int64_t nblk = bend - bbeg;
+  if (nblk <= 0) return;
 
   if (lane == 0)
     for (int s = 0; s < C::STAGES; ++s) mbar_init(ring.bar(s), 1);
@@ -441,20 +525,20 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   __syncwarp();
 
   // prologue: fill the ring
-  BlockPos ipos{bbeg / p.nb_u, bbeg - (bbeg / p.nb_u) * p.nb_u};
+  BlockPos ipos = pos_of_block<PAGED>(p, bbeg);
   const BlockPos pos0 = ipos;
 #pragma unroll
   for (int s = 0; s < C::STAGES; ++s) {
     if (s < nblk) {
-      issue_block<M, D, S8>(p, maps, ring, ipos, s, lane);
-      ipos.next(p.nb_u);
+      issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+      pos_next<PAGED>(p, ipos);
     }
   }
 
   // the query projections come from the previous kernel on the stream, which
   // may still be running (programmatic dependent launch): wait for it only
   // now, after the first copies are on their way
-  griddep_wait();
+  if constexpr (!PAGED) griddep_wait();
 
   // per-unit state
   int64_t cur_u = -1, kv_base = 0;
@@ -470,12 +554,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     float l = lsum;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int slot = w - warp_of_block(u * p.nb_u, p.NB, p.W);
-    if (slot < 0 || slot >= p.slots) {
+    // the warps of unit u are warp_of_block(first block of u) .. ; warp w's
+    // record for unit u is w + u: a warp's records are consecutive, and the
+    // next warp's first record comes after its last
+    const int64_t rec_idx = (int64_t)w + u;
+    if (rec_idx >= p.slots) {
       record_device_error(p.err, DERR_DECODE_PLAN);
       return;
     }
-    float *rec = p.partials + ((size_t)u * p.slots + slot) * DEC_HPAD * (D + 2);
+    float *rec = p.partials + (size_t)rec_idx * DEC_HPAD * (D + 2);
     if (t == 0 && g < Gg) {
       rec[g * (D + 2) + D] = mx;
       rec[g * (D + 2) + D + 1] = l;
@@ -500,13 +587,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     const int s = (int)(i % C::STAGES);
     const int64_t u = pos.u;
     const int64_t key0 = pos.blk * DEC_KB;
-    const int64_t left = p.T - key0;
+    const int64_t left = pos.len - key0;
     const int nval = left < DEC_KB ? (int)left : DEC_KB;
 
     if (u != cur_u) {
       if (cur_u >= 0) flush(cur_u);
       cur_u = u;
-      const int64_t kvi = u / p.HG;
+      const int64_t kvi = pos.kvi;
       const int hg = (int)(u - kvi * p.HG);
       const int hkv = (int)(kvi % p.Hkv);
       kv_base = kvi * p.T;
@@ -527,6 +614,24 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       record_device_error(p.err, DERR_DECODE_WAIT_TIMEOUT);
       failed = true;
       break;
+    }
+    if constexpr (PAGED) {
+      // a page's slots past the sequence's last key hold whatever was there:
+      // zero those value rows so that p = 0 cannot meet a NaN
+      if (nval < DEC_KB) {
+        const uint32_t vb = ring.val(s);
+        for (int e = lane; e < (DEC_KB - nval) * (D / 64) * 8; e += 32) {
+          const int row = nval + e / ((D / 64) * 8);
+          const int rest = e - (row - nval) * ((D / 64) * 8);
+          const uint32_t addr = vb + (rest >> 3) * C::V_BOX + row * 128 + (rest & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};\n" ::"r"(addr), "r"(0)
+                       : "memory");
+        }
+        // the stage is refilled by bulk-tensor copies later: order these
+        // generic-proxy writes before them
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncwarp();
+      }
     }
 
     // ---- code words of the 4 groups of 8 keys (lane: key kg*8 + g)
@@ -643,7 +748,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
         const float sval = (p.coef * nk) * raw[kg][j];
         l2[kg][j] = sval * p.scale_log2;
         if (p.scores != nullptr && key < nval && g < Gg)
-          p.scores[((int64_t)b_idx * p.Hq + hq0 + g) * p.T + key0 + key] = sval;
+          p.scores[((int64_t)b_idx * p.Hq + hq0 + g) * p.score_stride + key0 + key] = sval;
       }
     }
     if (nval < DEC_KB) {
@@ -702,10 +807,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // ---- refill this stage with the block STAGES ahead
     __syncwarp();
     if (i + C::STAGES < nblk) {
-      issue_block<M, D, S8>(p, maps, ring, ipos, s, lane);
-      ipos.next(p.nb_u);
+      issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+      pos_next<PAGED>(p, ipos);
     }
-    pos.next(p.nb_u);
+    pos_next<PAGED>(p, pos);
   }
   griddep_launch_dependents();
   if (failed) {
@@ -729,10 +834,11 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 // one unit can be split over every warp of the launch: at most W_bound + 1
 constexpr int COMB_MAX_SLOTS = DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS + 1;
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(D) decode_combine_kernel(
     const float *__restrict__ partials, uint16_t *__restrict__ out, int Hq,
-    int Hkv, int G, int HG, int64_t nb_u, int64_t NB, int W, int slots) {
+    int Hkv, int G, int HG, int64_t nb_u, int64_t NB_fixed, int W, int slots,
+    const int64_t *__restrict__ unit_off, int units) {
   __shared__ float wts[COMB_MAX_SLOTS];
   __shared__ float inv_l;
   griddep_wait();  // every partial state of the scorer is needed
@@ -741,10 +847,26 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
   const int hkv = hq / G, hl = hq - hkv * G;
   const int hg = hl / DEC_HPAD, hh = hl - hg * DEC_HPAD;
   const int64_t u = ((int64_t)b * Hkv + hkv) * HG + hg;
-  const int f = warp_of_block(u * nb_u, NB, W);
-  const int l = warp_of_block((u + 1) * nb_u - 1, NB, W);
-  const int n = min(min(l - f + 1, slots), COMB_MAX_SLOTS);
-  const float *rec0 = partials + (size_t)u * slots * DEC_HPAD * (D + 2) +
+  int64_t first, last, NB;
+  if constexpr (PAGED) {
+    NB = unit_off[units];
+    first = unit_off[u];
+    last = unit_off[u + 1] - 1;
+    if (last < first) {  // nothing to attend over: zeros
+      out[(int64_t)bh * D + threadIdx.x] = 0;
+      return;
+    }
+  } else {
+    NB = NB_fixed;
+    first = u * nb_u;
+    last = (u + 1) * nb_u - 1;
+  }
+  if constexpr (PAGED) W = (int)(NB < W ? NB : W);  // as the scorer
+  const int f = warp_of_block(first, NB, W);
+  const int l = warp_of_block(last, NB, W);
+  const int n = min(l - f + 1, COMB_MAX_SLOTS);
+  // records of unit u: warp w wrote record w + u (see the scorer's flush)
+  const float *rec0 = partials + (size_t)((int64_t)f + u) * DEC_HPAD * (D + 2) +
                       (size_t)hh * (D + 2);
   const size_t sstride = (size_t)DEC_HPAD * (D + 2);
   if (threadIdx.x < 32) {
@@ -784,6 +906,124 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// 4. paged calls: one prep launch does the query projections (CTAs
+// [0, B*Hq)), appends each sequence's new key (CTAs [B*Hq, B*Hq + B*Hkv) when
+// keys are given) and writes the work plan (last CTA).
+struct PrepParams {
+  const void *Q;
+  const uint16_t *S;
+  float *U;
+  int nq;                       // B * Hq
+  const void *K_new;            // B x Hkv x d, nullable
+  const uint16_t *V_new;        // B x Hkv x d
+  uint32_t *sign_pages;
+  uint16_t *norm_pages;
+  uint16_t *value_pages;
+  int num_pages, page_tokens, max_pages;
+  const int32_t *block_table;
+  const int32_t *seq_lens;
+  int B, Hkv, HG, units, append;
+  int64_t max_len;
+  int64_t *unit_off;            // [units + 1]
+  int *err;
+};
+
+template <int M, int D, bool QF32, bool KF32>
+__global__ void __launch_bounds__(M) paged_prep_kernel(const PrepParams pp) {
+  __shared__ float sh[D];
+  __shared__ int64_t scan[M];
+  const int bid = blockIdx.x;
+  const int i = threadIdx.x;
+  if (bid < pp.nq) {
+    // ---- query projection u = S q (as qproj_kernel)
+    uint4 row[D / 8];
+    const uint4 *src = reinterpret_cast<const uint4 *>(pp.S + (int64_t)i * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) row[c] = __ldg(src + c);
+    for (int j = i; j < D; j += M)
+      sh[j] = QF32 ? reinterpret_cast<const float *>(pp.Q)[(int64_t)bid * D + j]
+                   : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(pp.Q)[(int64_t)bid * D + j]);
+    __syncthreads();
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint32_t w[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc0 = fmaf(__uint_as_float(w[e] << 16), sh[c * 8 + 2 * e], acc0);
+        acc1 = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), sh[c * 8 + 2 * e + 1], acc1);
+      }
+    }
+    pp.U[(int64_t)bid * M + i] = acc0 + acc1;
+    return;
+  }
+  const int nappend = pp.append ? pp.B * pp.Hkv : 0;
+  if (bid < pp.nq + nappend) {
+    // ---- append: quantize key kvi = b*Hkv + hkv and store it at position
+    // seq_lens[b] of its sequence (thread i: sketch row i; a ballot per warp
+    // packs 32 code bits)
+    const int kvi = bid - pp.nq;
+    const int b = kvi / pp.Hkv, hkv = kvi - b * pp.Hkv;
+    for (int j = i; j < D; j += M)
+      sh[j] = KF32 ? reinterpret_cast<const float *>(pp.K_new)[(int64_t)kvi * D + j]
+                   : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(pp.K_new)[(int64_t)kvi * D + j]);
+    __syncthreads();
+    const int64_t pos = pp.seq_lens[b];
+    const int64_t pidx = pos / pp.page_tokens;
+    const int page = (pos >= 0 && pidx < pp.max_pages)
+                         ? pp.block_table[(int64_t)b * pp.max_pages + pidx] : -1;
+    if (page < 0 || page >= pp.num_pages || pos + 1 > pp.max_len) {
+      if (i == 0) record_device_error(pp.err, DERR_DECODE_PLAN);
+      return;
+    }
+    const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
+    const uint16_t *srow = pp.S + (int64_t)i * D;
+    float y = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) y = fmaf(bf16_bits_to_f32(srow[j]), sh[j], y);
+    const uint32_t word = __ballot_sync(0xffffffffu, y >= 0.f);
+    if ((i & 31) == 0) pp.sign_pages[slot * (M / 32) + (i >> 5)] = word;
+    if (i < 32) {
+      float ss = 0.f;
+      for (int j = i; j < D; j += 32) ss = fmaf(sh[j], sh[j], ss);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (i == 0) pp.norm_pages[slot] = __half_as_ushort(__float2half_rn(sqrtf(ss)));
+    }
+    for (int j = i; j < D; j += M) pp.value_pages[slot * D + j] = pp.V_new[(int64_t)kvi * D + j];
+    return;
+  }
+  // ---- work plan: unit u owns ceil(len/32) blocks, len = seq_lens[b] (+1)
+  int64_t carry = 0;
+  for (int base = 0; base < pp.units; base += M) {
+    const int u = base + i;
+    int64_t nb = 0;
+    if (u < pp.units) {
+      const int b = (u / pp.HG) / pp.Hkv;
+      int64_t len = (int64_t)pp.seq_lens[b] + pp.append;
+      if (len < 0) len = 0;
+      if (len > pp.max_len) {
+        record_device_error(pp.err, DERR_DECODE_PLAN);
+        len = pp.max_len;
+      }
+      nb = (len + DEC_KB - 1) / DEC_KB;
+    }
+    scan[i] = nb;
+    __syncthreads();
+    for (int o = 1; o < M; o <<= 1) {  // inclusive scan (Hillis-Steele)
+      const int64_t v = i >= o ? scan[i - o] : 0;
+      __syncthreads();
+      scan[i] += v;
+      __syncthreads();
+    }
+    if (u < pp.units) pp.unit_off[u] = carry + scan[i] - nb;
+    carry += scan[M - 1];
+    __syncthreads();
+  }
+  if (i == 0) pp.unit_off[pp.units] = carry;
+}
+
+// ---------------------------------------------------------------------------
 // planning and launch
 static bool supported(int m, int d) {
   return (d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512);
@@ -791,10 +1031,13 @@ static bool supported(int m, int d) {
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
-                      DecodePlan *pl) {
+// Warps are launched one wave at a time (SMs x resident CTAs x 4), never more
+// than this bound, which sizes the partial records: W_bound + units of them.
+constexpr int64_t DEC_W_BOUND = (int64_t)DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS;
+
+static bool plan_common(int B, int Hq, int Hkv, int64_t T, int m, int d, DecodePlan *pl) {
   if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv) return false;
-  if ((int64_t)B * Hkv >= ((int64_t)1 << 31) || T >= ((int64_t)1 << 31)) return false;
+  if ((int64_t)B * Hkv >= ((int64_t)1 << 24) || T >= ((int64_t)1 << 31)) return false;
   if (!supported(m, d)) return false;
   DecodePlan p{};
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.T = T; p.m = m; p.d = d;
@@ -803,17 +1046,25 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
   p.units = B * Hkv * p.HG;
   p.nb_u = (T + DEC_KB - 1) / DEC_KB;
   p.NB = (int64_t)p.units * p.nb_u;
-  // the launch uses at most W_bound warps (B200 SMs x max CTAs per SM); the
-  // partial-state layout is sized for that bound so that it depends on the
-  // shapes only
-  const int64_t wb = (int64_t)DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS;
-  p.W = (int)(p.NB < wb ? p.NB : wb);
-  p.slots = (int)((p.W + p.units - 1) / p.units) + 1;  // <= W_bound + 1 <= 2369
+  p.W = (int)(p.NB < DEC_W_BOUND ? p.NB : DEC_W_BOUND);
+  p.records = p.W + p.units;
   p.u_bytes = round_up((size_t)B * Hq * m * sizeof(float), 256);
-  p.partial_bytes = round_up(
-      (size_t)p.units * p.slots * DEC_HPAD * (d + 2) * sizeof(float), 256);
-  p.total_bytes = p.u_bytes + p.partial_bytes;
+  p.partial_bytes = round_up((size_t)p.records * DEC_HPAD * (d + 2) * sizeof(float), 256);
   *pl = p;
+  return true;
+}
+
+bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, DecodePlan *pl) {
+  if (!plan_common(B, Hq, Hkv, T, m, d, pl)) return false;
+  pl->off_bytes = 0;
+  pl->total_bytes = pl->u_bytes + pl->partial_bytes;
+  return true;
+}
+
+bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d, DecodePlan *pl) {
+  if (!plan_common(B, Hq, Hkv, max_len, m, d, pl)) return false;
+  pl->off_bytes = round_up((size_t)(pl->units + 1) * sizeof(int64_t), 256);
+  pl->total_bytes = pl->u_bytes + pl->off_bytes + pl->partial_bytes;
   return true;
 }
 
@@ -823,7 +1074,7 @@ static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
   auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!fn) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
-  {  // values [B*Hkv][T][d]: 64 columns x 32 rows x 1 unit, 128-byte swizzle
+  {  // values [units][T][d]: 64 columns x 32 rows x 1 unit, 128-byte swizzle
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)units_kv};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)T * d * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)DEC_KB, 1};
@@ -836,7 +1087,7 @@ static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
   mp->tma_codes = 0;
   mp->sign_elem = (m > 256) ? 8 : 4;
   if (T % 8 != 0) return true;  // per-unit rows not 16-byte aligned: cp.async path
-  {  // codes [B*Hkv][T * m/8 bytes] as 4- or 8-byte elements, one block per box
+  {  // codes [units][T * m/8 bytes] as 4- or 8-byte elements, one block per box
     const int es = mp->sign_elem;
     cuuint64_t dims[2] = {(cuuint64_t)(T * (m / 8) / es), (cuuint64_t)units_kv};
     cuuint64_t strides[1] = {(cuuint64_t)T * (m / 8)};
@@ -847,7 +1098,7 @@ static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return true;
   }
-  {  // norms [B*Hkv][T] binary16, 32 per box
+  {  // norms [units][T] binary16, 32 per box
     cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)units_kv};
     cuuint64_t strides[1] = {(cuuint64_t)T * 2};
     cuuint32_t box[2] = {(cuuint32_t)DEC_KB, 1};
@@ -885,6 +1136,46 @@ static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *partials,
+                        const uint32_t *signs, const uint16_t *norms, float *scores,
+                        float softmax_scale, int m, int *err) {
+  p = DecParams{};
+  p.U = U; p.signs = signs; p.norms = norms; p.partials = partials;
+  p.scores = scores; p.err = err; p.T = pl.T; p.nb_u = pl.nb_u; p.NB = pl.NB;
+  p.n_keys = (int64_t)pl.B * pl.Hkv * pl.T;
+  p.Hq = pl.Hq; p.Hkv = pl.Hkv; p.G = pl.G; p.HG = pl.HG;
+  p.slots = pl.records;
+  p.coef = (float)(sqrt(M_PI / 2.0) / (double)m);
+  p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
+  p.score_stride = pl.T;
+  p.units = pl.units;
+}
+
+// Launch the scorer (one wave, <= the plan's warp bound) and the combine.
+template <int M, int D, bool S8, bool PAGED>
+static cudaError_t launch_scorer_combine(const DecodePlan &pl, DecParams &p, const DecMaps &maps,
+                                         uint16_t *out, cudaStream_t stream) {
+  using C = DecCfg<M, D, S8>;
+  auto kern = decode_scorer_kernel<M, D, S8, PAGED>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::CTA_BYTES);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DEC_WARPS * 32,
+                                                    C::CTA_BYTES);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > DEC_MAX_CTAS_SM) per_sm = DEC_MAX_CTAS_SM;
+  const int64_t wave = (int64_t)device_sm_count() * per_sm * DEC_WARPS;
+  p.W = (int)(wave < pl.W ? wave : pl.W);
+  const int ctas = (p.W + DEC_WARPS - 1) / DEC_WARPS;
+  e = launch_pdl(kern, dim3(ctas), dim3(DEC_WARPS * 32), C::CTA_BYTES, stream, maps, p);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_combine_kernel<D, PAGED>, dim3(pl.B * pl.Hq), dim3(D), 0, stream,
+                    (const float *)p.partials, out, pl.Hq, pl.Hkv, pl.G, pl.HG, pl.nb_u,
+                    pl.NB, p.W, pl.records, p.unit_off, pl.units);
+}
+
 template <int M, int D, bool S8>
 static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
                                    bool q_f32, const uint16_t *S,
@@ -892,7 +1183,6 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
                                    const uint16_t *V, float softmax_scale,
                                    uint16_t *out, float *scores,
                                    void *workspace, cudaStream_t stream) {
-  using C = DecCfg<M, D, S8>;
   float *U = reinterpret_cast<float *>(workspace);
   float *partials =
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
@@ -908,33 +1198,9 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
     qproj_kernel<M, D, false><<<bh, M, 0, stream>>>(Q, S, U);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-
   DecParams p;
-  p.U = U; p.signs = signs; p.norms = norms; p.partials = partials;
-  p.scores = scores; p.err = err; p.T = pl.T; p.nb_u = pl.nb_u; p.NB = pl.NB;
-  p.n_keys = (int64_t)pl.B * pl.Hkv * pl.T;
-  p.Hq = pl.Hq; p.Hkv = pl.Hkv; p.G = pl.G; p.HG = pl.HG;
-  p.slots = pl.slots;
-  p.coef = (float)(sqrt(M_PI / 2.0) / (double)M);
-  p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
-  auto kern = decode_scorer_kernel<M, D, S8>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::CTA_BYTES);
-  if (e != cudaSuccess) return e;
-  // one wave of resident CTAs, never more warps than the plan's bound
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DEC_WARPS * 32,
-                                                    C::CTA_BYTES);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm > DEC_MAX_CTAS_SM) per_sm = DEC_MAX_CTAS_SM;
-  const int64_t wave = (int64_t)device_sm_count() * per_sm * DEC_WARPS;
-  p.W = (int)(wave < pl.W ? wave : pl.W);
-  const int ctas = (p.W + DEC_WARPS - 1) / DEC_WARPS;
-  e = launch_pdl(kern, dim3(ctas), dim3(DEC_WARPS * 32), C::CTA_BYTES, stream, maps, p);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(decode_combine_kernel<D>, dim3(bh), dim3(D), 0, stream,
-                    (const float *)partials, out, pl.Hq, pl.Hkv, pl.G, pl.HG, pl.nb_u,
-                    pl.NB, p.W, pl.slots);
+  fill_params(p, pl, U, partials, signs, norms, scores, softmax_scale, M, err);
+  return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
 }
 
 cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
@@ -951,6 +1217,100 @@ cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
               : launch_decode_t<MM, DD, false>(pl, Q, q_f32, S, signs, norms, V, \
                                                softmax_scale, out, scores,      \
                                                workspace, stream);
+  JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
+  JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
+#undef JL_CASE
+  return cudaErrorNotSupported;
+}
+
+// Paged pools: values [num_pages*Hkv][P][d], codes [num_pages*Hkv][P*m/8 bytes],
+// norms [num_pages*Hkv][P]; every block is one box inside one page.
+static bool make_paged_maps(DecMaps *mp, const PagedArgs &a, int Hkv, int m, int d) {
+  auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!fn) return false;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const uint64_t rows = (uint64_t)a.num_pages * Hkv, P = (uint64_t)a.page_tokens;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)d, P, rows};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, P * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)DEC_KB, 1};
+    if (fn(&mp->value, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.value_pages, dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  mp->sign_elem = (m > 256) ? 8 : 4;
+  {
+    const int es = mp->sign_elem;
+    cuuint64_t dims[2] = {(cuuint64_t)(P * (m / 8) / es), rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(P * (m / 8))};
+    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * (m / 8) / es), 1};
+    if (fn(&mp->sign, es == 8 ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
+           2, a.sign_pages, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    cuuint64_t dims[2] = {P, rows};
+    cuuint64_t strides[1] = {P * 2};
+    cuuint32_t box[2] = {(cuuint32_t)DEC_KB, 1};
+    if (fn(&mp->norm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.norm_pages, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  mp->tma_codes = 1;
+  return true;
+}
+
+template <int M, int D, bool S8>
+static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
+                                  cudaStream_t stream) {
+  uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
+  float *U = reinterpret_cast<float *>(ws);
+  int64_t *unit_off = reinterpret_cast<int64_t *>(ws + pl.u_bytes);
+  float *partials = reinterpret_cast<float *>(ws + pl.u_bytes + pl.off_bytes);
+  DecMaps maps;
+  if (!make_paged_maps(&maps, a, pl.Hkv, M, D)) return cudaErrorInvalidValue;
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
+  PrepParams pp;
+  pp.Q = a.Q; pp.S = a.S; pp.U = U; pp.nq = pl.B * pl.Hq;
+  pp.K_new = a.K_new; pp.V_new = a.V_new;
+  pp.sign_pages = a.sign_pages; pp.norm_pages = a.norm_pages; pp.value_pages = a.value_pages;
+  pp.num_pages = a.num_pages; pp.page_tokens = a.page_tokens; pp.max_pages = a.max_pages;
+  pp.block_table = a.block_table; pp.seq_lens = a.seq_lens;
+  pp.B = pl.B; pp.Hkv = pl.Hkv; pp.HG = pl.HG; pp.units = pl.units;
+  pp.append = a.K_new != nullptr;
+  pp.max_len = pl.T;
+  pp.unit_off = unit_off;
+  pp.err = err;
+  const int prep_ctas = pp.nq + (pp.append ? pl.B * pl.Hkv : 0) + 1;
+  if (a.q_f32) {
+    if (a.k_f32) paged_prep_kernel<M, D, true, true><<<prep_ctas, M, 0, stream>>>(pp);
+    else paged_prep_kernel<M, D, true, false><<<prep_ctas, M, 0, stream>>>(pp);
+  } else {
+    if (a.k_f32) paged_prep_kernel<M, D, false, true><<<prep_ctas, M, 0, stream>>>(pp);
+    else paged_prep_kernel<M, D, false, false><<<prep_ctas, M, 0, stream>>>(pp);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  DecParams p;
+  fill_params(p, pl, U, partials, nullptr, nullptr, a.scores, a.softmax_scale, M, err);
+  p.unit_off = unit_off; p.seq_lens = a.seq_lens; p.block_table = a.block_table;
+  p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
+  p.score_stride = pl.T;
+  return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);
+}
+
+cudaError_t launch_decode_paged(const DecodePlan &pl, const PagedArgs &a,
+                                cudaStream_t stream) {
+  const bool s8 = decode_use_s8(pl.G, pl.m);
+#define JL_CASE(MM, DD)                                            \
+  if (pl.m == MM && pl.d == DD)                                    \
+    return s8 ? launch_paged_t<MM, DD, true>(pl, a, stream)        \
+              : launch_paged_t<MM, DD, false>(pl, a, stream);
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
 #undef JL_CASE

@@ -30,25 +30,50 @@ bool quantize_tc_supported(int m, int d, int64_t n, int64_t ldk, const void *K);
 // Decode: work split shared by the workspace query and the launch.
 struct DecodePlan {
   int B, Hq, Hkv, m, d;
-  int64_t T;
+  int64_t T;     // keys per unit (contiguous cache) or the bound max_len (paged)
   int G;         // query heads per KV head
   int HG;        // head groups per KV head (groups of at most 8 heads)
   int units;     // B * Hkv * HG
-  int64_t nb_u;  // 32-key blocks per unit
-  int64_t NB;    // units * nb_u
-  int W;         // warps launched (each takes a contiguous run of blocks)
-  int slots;     // partial-state slots per unit
+  int64_t nb_u;  // 32-key blocks per unit (paged: the bound)
+  int64_t NB;    // units * nb_u (paged: the bound)
+  int W;         // bound on the warps launched
+  int records;   // partial-state records: W + units
   size_t u_bytes;        // fp32 query projections [B][Hq][m]
-  size_t partial_bytes;  // fp32 [units][slots][8][d + 2]
+  size_t off_bytes;      // paged: int64 block offsets [units + 1]
+  size_t partial_bytes;  // fp32 [records][8][d + 2]
   size_t total_bytes;
 };
 bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
                       DecodePlan *plan);
+bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d,
+                     DecodePlan *plan);
 
 cudaError_t launch_decode(const DecodePlan &p, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,
                           const uint16_t *norms, const uint16_t *V,
                           float softmax_scale, uint16_t *out, float *scores,
                           void *workspace, cudaStream_t stream);
+
+struct PagedArgs {
+  const void *Q;
+  bool q_f32;
+  const void *K_new;  // nullable: no append
+  bool k_f32;
+  const uint16_t *V_new;
+  const uint16_t *S;
+  uint32_t *sign_pages;
+  uint16_t *norm_pages;
+  uint16_t *value_pages;
+  int num_pages, page_tokens;
+  const int32_t *block_table;
+  int max_pages;
+  const int32_t *seq_lens;
+  float softmax_scale;
+  uint16_t *out;
+  float *scores;
+  void *workspace;
+};
+cudaError_t launch_decode_paged(const DecodePlan &p, const PagedArgs &a,
+                                cudaStream_t stream);
 
 }  // namespace jlk

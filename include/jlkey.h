@@ -166,6 +166,61 @@ JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *
                         jl_stream_t stream);
 
 /*
+ * jl_decode_paged_workspace_bytes -- device scratch jl_decode_attention_paged
+ * needs (query projections, the per-call work plan and split partial
+ * states) for B sequences of at most max_len keys each (counting the key a
+ * call appends).  Depends on the shapes only; 0 for unsupported shapes.
+ */
+JL_API size_t jl_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len,
+                                              int m, int d);
+
+/*
+ * jl_decode_attention_paged -- one decode step of a batch of sequences of
+ * different lengths whose compressed cache lives in a pool of fixed-size
+ * pages, optionally appending each sequence's new key first.
+ * Defines: the quantizer Q(k) = sign(S k) with the stored norm ("The Geometry
+ * of Forgetting ...", QJL and PolarQuant sections) applied to the new key, and
+ * the asymmetric estimator of jl_decode_attention used as the attention logit
+ * over each sequence's keys.
+ *   Q           : in, B x Hq x d of q_dtype (16-byte aligned): the new token's
+ *                 queries.
+ *   K_new       : in or NULL, B x Hkv x d of k_dtype (16-byte aligned): the new
+ *                 token's keys.  When given, key t = seq_lens[b] of sequence b
+ *                 is written first: its code and binary16 norm (the
+ *                 quantizer of jl_quantize_keys) and its value V_new[b][h]
+ *                 go to page block_table[b][t / page_tokens], slot
+ *                 t % page_tokens, and the step attends over seq_lens[b] + 1
+ *                 keys.  Without K_new it attends over seq_lens[b] keys.
+ *   V_new       : in, B x Hkv x d bf16 (required with K_new).
+ *   S           : in, m x d bf16 sketch.
+ *   sign_pages  : in/out, num_pages x Hkv x page_tokens x (m/32) uint32.
+ *   norm_pages  : in/out, num_pages x Hkv x page_tokens binary16.
+ *   value_pages : in/out, num_pages x Hkv x page_tokens x d bf16.
+ *                 The three pools are 16-byte aligned.
+ *   page_tokens : keys per page, a multiple of 32.
+ *   block_table : in, B x max_pages int32 page ids (device); entries past a
+ *                 sequence's last page are not read.
+ *   seq_lens    : in, B int32 (device): keys already cached per sequence.
+ *                 Not modified (the caller advances it after an append).
+ *   max_len     : bound on seq_lens[b] (+1 with K_new), used to size the
+ *                 work split and the workspace.
+ *   scores      : optional out, B x Hq x max_len fp32 (row stride max_len).
+ *   workspace   : >= jl_decode_paged_workspace_bytes(...), 256-byte aligned.
+ * A sequence with no key to attend over (seq_lens[b] == 0, no K_new) gets an
+ * output of zeros.  Values past a sequence's last key inside its last page
+ * are never read into the result, whatever they hold.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
+ * JL_ERR_CUDA.
+ */
+JL_API int jl_decode_attention_paged(
+    const void *Q, jl_dtype q_dtype, const void *K_new, jl_dtype k_dtype,
+    const uint16_t *V_new, const uint16_t *S, uint32_t *sign_pages,
+    uint16_t *norm_pages, uint16_t *value_pages, int num_pages, int page_tokens,
+    const int32_t *block_table, int max_pages, const int32_t *seq_lens, int B, int Hq,
+    int Hkv, int64_t max_len, int m, int d, float softmax_scale, uint16_t *out,
+    float *scores, void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
+/*
  * jl_decode_attention_noalloc -- jl_decode_attention for callers that cannot
  * allocate device memory.  The paper has no counterpart: this entry point
  * exists for deployment, not for the method.

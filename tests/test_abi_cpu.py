@@ -145,3 +145,49 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         jl.jl_quantize_keys(torch.zeros(4, 128, dtype=torch.bfloat16),
                             torch.zeros(256, 128, dtype=torch.bfloat16))
+
+
+def test_paged_workspace_query(lib):
+    f = jl.jl_decode_paged_workspace_bytes
+    assert f(4, 32, 8, 4096, 256, 128) > 4 * 32 * 256 * 4
+    assert f(0, 32, 8, 4096, 256, 128) == 0
+    assert f(1, 6, 4, 4096, 256, 128) == 0
+    assert f(1, 1, 1, 0, 256, 128) == 0
+    # sized by the bound, so never below the contiguous plan at that length
+    assert f(4, 32, 8, 4096, 256, 128) >= jl.jl_decode_workspace_bytes(4, 32, 8, 4096, 256, 128)
+
+
+def test_paged_decode_argument_errors(lib):
+    f = lib.jl_decode_attention_paged
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, Kn=FAKE, kt=jl.JL_BF16, Vn=FAKE, S=FAKE,
+              sp=FAKE, np_=FAKE, vp=FAKE, npages=16, P=64, table=FAKE, maxp=4,
+              lens=FAKE, B=2, Hq=8, Hkv=2, max_len=256, m=256, d=128, scale=0.1,
+              out=FAKE, scores=NULL, ws=FAKE, wsb=1 << 40)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["Q"], a["qt"], a["Kn"], a["kt"], a["Vn"], a["S"], a["sp"], a["np_"],
+                 a["vp"], a["npages"], a["P"], a["table"], a["maxp"], a["lens"], a["B"],
+                 a["Hq"], a["Hkv"], a["max_len"], a["m"], a["d"],
+                 ctypes.c_float(a["scale"]), a["out"], a["scores"], a["ws"], a["wsb"], NULL)
+
+    assert call(B=0) == jl.JL_OK
+    assert call(P=48) == jl.JL_ERR_INVALID_ARG          # page not a whole number of 32-key blocks
+    assert call(P=0) == jl.JL_ERR_INVALID_ARG
+    assert call(maxp=3) == jl.JL_ERR_INVALID_ARG        # 3 * 64 < max_len
+    assert call(npages=0) == jl.JL_ERR_INVALID_ARG
+    assert call(max_len=0) == jl.JL_ERR_INVALID_ARG
+    assert call(Hq=6, Hkv=4) == jl.JL_ERR_INVALID_ARG
+    assert call(kt=9) == jl.JL_ERR_INVALID_ARG
+    assert call(Vn=NULL) == jl.JL_ERR_INVALID_ARG        # key without its value
+    assert call(m=96) == jl.JL_ERR_UNSUPPORTED
+    for k in ("Q", "S", "sp", "np_", "vp", "table", "lens", "out"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(vp=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(Kn=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(lens=ctypes.c_void_p((1 << 20) + 2)) == jl.JL_ERR_INVALID_ARG
+    assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
+    need = jl.jl_decode_paged_workspace_bytes(2, 8, 2, 256, 256, 128)
+    assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
+    # without a new key, the key dtype is not looked at
+    assert call(Kn=NULL, Vn=NULL, kt=9, ws=NULL) == jl.JL_ERR_WORKSPACE
