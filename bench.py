@@ -1,7 +1,7 @@
 """Benchmark: QJL key quantization + compressed-key decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -10,6 +10,12 @@ run one decode step of attention over the compressed cache
 workload is GQA decode: batch 8, 32 query / 8 KV heads, d=128, m=256, context
 32768.  Inputs are seeded synthetic tensors (workloads.py) already resident
 in HBM; they exceed L2 (126 MB), so no flush is needed between steps.
+
+The paged-gqa workload times a serving step instead: one
+jl_decode_attention_paged call that appends every sequence's new key and
+value to a shuffled page pool and attends over its ragged context (the cache
+is filled once, untimed; the lengths stay fixed from step to step, so every
+step rewrites the same slots).
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload
 (independent sequences, no data-path collective), timing is the max over ranks
@@ -207,9 +213,138 @@ def score_error(jl, w, Q, S, signs, norms, V, K, max_rows=16):
 # --------------------------------------------------------------------------
 # our arm
 
+def _barrier(world, dev):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
+
+def run_paged(args, rank, world, local_rank):
+    """Serving step over a paged cache: append + decode in one call."""
+    import bit_jl_key_b200 as jl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload, args.batch)
+    peak, peak_kind = load_peaks()
+    P = workloads.PAGE_TOKENS
+    lens, table, num_pages = workloads.paged_layout(w, P)
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    # fill the pool (untimed): keys and values of every slot, quantized in place
+    pool = w.with_(B=num_pages, T=P)
+    Kp = workloads.keys(pool, dev)
+    sign_pages = torch.empty((num_pages, w.Hkv, P, w.m // 32), dtype=torch.int32, device=dev)
+    norm_pages = torch.empty((num_pages, w.Hkv, P), dtype=torch.float16, device=dev)
+    jl.jl_quantize_keys(Kp.view(-1, w.d), S, sign_pages.view(-1, w.m // 32), norm_pages.view(-1))
+    del Kp
+    value_pages = workloads.values(pool, dev)
+    Q = workloads.queries(w, dev)
+    Kn, Vn = workloads.new_tokens(w, dev)
+    seq = lens.to(dev)
+    tab = table.to(dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((jl.jl_decode_paged_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d),),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    attended = int((lens.long() + 1).sum()) * w.Hkv     # KV keys scored per step
+
+    def step():
+        jl.jl_decode_attention_paged(Q, S, sign_pages, norm_pages, value_pages, tab, seq,
+                                     w.T, K_new=Kn, V_new=Vn, softmax_scale=w.softmax_scale,
+                                     out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        _barrier(world, dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        _barrier(world, dev)
+    ms_step = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    d_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    # end to end: the step's new query, key and value (and the lengths) from
+    # pinned host memory, the output back to it; the cache stays resident
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, Kn, Vn))
+        hL = lens.clone().pin_memory()
+        hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hL))
+        d2h = hOut.numel() * hOut.element_size()
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            Kn.copy_(hK, non_blocking=True)
+            Vn.copy_(hV, non_blocking=True)
+            seq.copy_(hL, non_blocking=True)
+            step()
+            hOut.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        _barrier(world, dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        _barrier(world, dev)
+        e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        e2e = {"value": whole_job_rate(attended, world, e_ms), "unit": "keys/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    per_key = w.m // 8 + 2 + 2 * w.d
+    db = attended * per_key
+    gbs = db / (d_ms * 1e-3) / 1e9
+    traffic = ncu_traffic("decode:" + w.name)
+    phases = {"decode": {"ms": d_ms, "keys_scored_per_s": attended / (d_ms * 1e-3),
+                         "head_key_pairs_per_s": attended * w.G / (d_ms * 1e-3),
+                         "algorithmic_bytes": db, "GB_per_s": gbs,
+                         "frac_of_hbm_peak": gbs / peak,
+                         "appended_keys": w.B * w.Hkv}}
+    roof = {"kernel": "jl_decode_attention_paged", "bound": "hbm", "achieved": gbs,
+            "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+            "frac": gbs / peak, "algorithmic_bytes_per_launch": db,
+            "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
+    return {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": whole_job_rate(attended, world, ms_step), "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} max_len={w.T} "
+                               f"d={w.d} m={w.m} page={P} lens={lens.tolist()} + 1 appended",
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"dp{world}",
+                   "l2": "cache exceeds L2 (126 MB); no flush"},
+        "phases": phases,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
+    if args.workload == "paged-gqa":
+        return run_paged(args, rank, world, local_rank)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = pick_workload(args.workload, args.batch)

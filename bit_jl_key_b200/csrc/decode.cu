@@ -98,13 +98,12 @@ struct DecParams {
   float coef;               // sqrt(pi/2) / m
   float scale_log2;         // softmax_scale * log2(e)
   int64_t score_stride;     // row stride of `scores` (T, or max_len when paged)
-  // paged cache (PAGED kernels): unit u = (b, kv head, head group) owns blocks
-  // unit_off[u] .. unit_off[u+1] of the flat block space, written by the prep
-  // kernel from seq_lens; its keys live in pages block_table[b][*]
-  const int64_t *unit_off;  // [units + 1]
+  // paged cache (PAGED kernels): sequence b holds UH = Hkv * HG consecutive
+  // units, each of paged_blocks(b) blocks, so the flat block space follows
+  // from seq_lens alone; the keys live in pages block_table[b][*]
   const int32_t *seq_lens;  // [B]
   const int32_t *block_table;  // [B][max_pages]
-  int max_pages, page_tokens, append, units;
+  int max_pages, page_tokens, append, units, B, UH;
 };
 
 // Bulk-tensor maps of one decode call.  Values always go through `value`
@@ -120,6 +119,16 @@ struct DecMaps {
   int sign_elem;  // bytes per element of the sign map (4 or 8)
 };
 
+// Paged cache: blocks of every unit of sequence b, ceil(len / 32) with
+// len = seq_lens[b] (+1 when the call appends a key) kept inside [0, max_len];
+// a length past the bound is reported by the combine.
+__device__ __forceinline__ int64_t paged_blocks(const int32_t *seq_lens, int b, int append,
+                                                int64_t max_len) {
+  int64_t len = (int64_t)__ldg(seq_lens + b) + append;
+  len = len < 0 ? 0 : (len > max_len ? max_len : len);
+  return (len + DEC_KB - 1) / DEC_KB;
+}
+
 // warp that owns block b when NB blocks are cut into W contiguous runs
 // starting at floor(w * NB / W)
 __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
@@ -128,36 +137,86 @@ __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
 }
 
 // ---------------------------------------------------------------------------
-// 1. query projection u = S q (fp32 accumulate).  One CTA per query, thread i
-// owns sketch row i and issues all of its 16-byte loads before the first
-// multiply (one memory round trip; S is L2-resident after the first call).
-template <int M, int D, bool QF32>
-__global__ void __launch_bounds__(M) qproj_kernel(const void *__restrict__ Q,
-                                                  const uint16_t *__restrict__ S,
-                                                  float *__restrict__ U) {
-  __shared__ float qs[D];
-  griddep_launch_dependents();  // let the scorer start its copies now
-  const int bh = blockIdx.x;
-  const int i = threadIdx.x;
-  uint4 row[D / 8];
-  const uint4 *src = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
+// 1. query projection u = S q (fp32 accumulate), four vectors per CTA.
+//
+// y[j][i] = sum_c S[i][c] x_j[c] for x_j = X[x0 + j], j < nx <= 4, written to
+// dst[j * M + i].  256 threads: warp w takes sketch rows w, w + 8, ... in
+// chunks of 8 rows; lane l holds columns [l*CPL, (l+1)*CPL) of a row, so every
+// load of a row is one coalesced 128- or 256-byte line.  The 32 partial sums a
+// lane has for a chunk (8 rows x 4 vectors) are combined by a butterfly
+// reduce-scatter: 31 shuffles leave lane l with the complete sum of entry l.
+constexpr int PROJ_THREADS = 256;
+constexpr int PROJ_VECS = 4;
+
+template <int M, int D, bool XF32>
+__device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
+                                         const void *__restrict__ X, int64_t x0,
+                                         int nx, float *dst) {
+  constexpr int CPL = D / 32;   // columns per lane
+  constexpr int CH = 8;         // rows per chunk
+  constexpr int RPW = M / 8;    // rows per warp
+  static_assert(CH * PROJ_VECS == 32 && RPW % CH == 0, "projection tiling");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float x[PROJ_VECS][CPL];
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) row[c] = __ldg(src + c);
-  for (int j = i; j < D; j += M)
-    qs[j] = QF32 ? reinterpret_cast<const float *>(Q)[(int64_t)bh * D + j]
-                 : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[(int64_t)bh * D + j]);
-  __syncthreads();
-  float acc0 = 0.f, acc1 = 0.f;
+  for (int j = 0; j < PROJ_VECS; ++j)
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint32_t w[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      acc0 = fmaf(__uint_as_float(w[e] << 16), qs[c * 8 + 2 * e], acc0);
-      acc1 = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), qs[c * 8 + 2 * e + 1], acc1);
+    for (int c = 0; c < CPL; ++c) {
+      const int64_t e = (x0 + j) * D + lane * CPL + c;
+      x[j][c] = j >= nx ? 0.f
+                : XF32  ? reinterpret_cast<const float *>(X)[e]
+                        : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(X)[e]);
     }
+#pragma unroll
+  for (int r0 = 0; r0 < RPW; r0 += CH) {
+    uint32_t sw[CH][CPL / 2];
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const uint16_t *row = S + (int64_t)(warp + 8 * (r0 + k)) * D + lane * CPL;
+      if constexpr (CPL == 4) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2 *>(row));
+        sw[k][0] = t.x;
+        sw[k][1] = t.y;
+      } else {
+        sw[k][0] = __ldg(reinterpret_cast<const uint32_t *>(row));
+      }
+    }
+    float v[32];
+#pragma unroll
+    for (int k = 0; k < CH; ++k)
+#pragma unroll
+      for (int j = 0; j < PROJ_VECS; ++j) {
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL / 2; ++c) {
+          a = fmaf(__uint_as_float(sw[k][c] << 16), x[j][2 * c], a);
+          a = fmaf(__uint_as_float(sw[k][c] & 0xFFFF0000u), x[j][2 * c + 1], a);
+        }
+        v[k * PROJ_VECS + j] = a;
+      }
+#pragma unroll
+    for (int st = 16; st >= 1; st >>= 1) {
+      const bool upper = (lane & st) != 0;
+#pragma unroll
+      for (int k = 0; k < st; ++k) {
+        const float send = upper ? v[k] : v[k + st];
+        const float keep = upper ? v[k + st] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+      }
+    }
+    const int k = lane / PROJ_VECS, j = lane % PROJ_VECS;
+    if (j < nx) dst[(int64_t)j * M + warp + 8 * (r0 + k)] = v[0];
   }
-  U[(int64_t)bh * M + i] = acc0 + acc1;
+}
+
+template <int M, int D, bool QF32>
+__global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restrict__ Q,
+                                                             const uint16_t *__restrict__ S,
+                                                             float *__restrict__ U, int nq) {
+  griddep_launch_dependents();  // let the scorer start its copies now
+  const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
+  const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
+  project4<M, D, QF32>(S, Q, x0, nx, U + x0 * M);
 }
 
 // ---------------------------------------------------------------------------
@@ -171,49 +230,108 @@ struct BlockPos {
   int64_t nb;   // blocks of unit u
   int64_t len;  // keys of unit u
   int64_t kvi;  // b * Hkv + kv head of unit u
+  // paged cache only: the block's page within its sequence (pidx), its first
+  // row in that page (y), the sequence's block-table row, the kv head, and
+  // the pool page itself once looked up (load_page); kept up to date without
+  // divisions as the position advances
+  int pidx, y, hkv, page;
+  const int32_t *trow;
 };
 
 template <bool PAGED>
 __device__ __forceinline__ void pos_load_unit(const DecParams &p, BlockPos &pos) {
   pos.kvi = p.HG == 1 ? pos.u : pos.u / p.HG;
   if constexpr (PAGED) {
-    pos.nb = p.unit_off[pos.u + 1] - p.unit_off[pos.u];
-    // an invalid length (past the bound) was reported by the prep kernel,
-    // which also capped the unit's blocks; keep every access inside the bound
-    const int64_t len = (int64_t)p.seq_lens[pos.kvi / p.Hkv] + p.append;
-    pos.len = len < p.T ? len : p.T;
+    const int b = (int)pos.kvi / p.Hkv;  // kv rows < 2^24 (checked by the plan)
+    pos.hkv = (int)pos.kvi - b * p.Hkv;
+    pos.trow = p.block_table + (int64_t)b * p.max_pages;
+    pos.nb = paged_blocks(p.seq_lens, b, p.append, p.T);
+    // keep every access inside the bound, whatever the length says
+    const int64_t len = (int64_t)__ldg(p.seq_lens + b) + p.append;
+    pos.len = len < 0 ? 0 : (len < p.T ? len : p.T);
   } else {
     pos.nb = p.nb_u;
     pos.len = p.T;
   }
 }
 
-// Position of flat block b (which must exist).
-template <bool PAGED>
+// Position of flat block b (which must exist), contiguous cache.
 __device__ __forceinline__ BlockPos pos_of_block(const DecParams &p, int64_t b) {
   BlockPos pos;
-  if constexpr (PAGED) {
-    // last unit whose first block is <= b (empty units share their offset)
-    int64_t lo = 0, hi = p.units - 1;
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (p.unit_off[mid] <= b) lo = mid; else hi = mid - 1;
-    }
-    pos.u = lo;
-    pos.blk = b - p.unit_off[lo];
-  } else {
-    pos.u = b / p.nb_u;
-    pos.blk = b - pos.u * p.nb_u;
-  }
-  pos_load_unit<PAGED>(p, pos);
+  pos.u = b / p.nb_u;
+  pos.blk = b - pos.u * p.nb_u;
+  pos_load_unit<false>(p, pos);
   return pos;
 }
 
-template <bool PAGED>
+// Paged cache, whole warp: total blocks NB of the flat space (sum over the
+// sequences of UH * paged_blocks), the same in every lane.  Not inlined: it
+// runs once per warp and keeps its registers out of the streaming loop.
+__device__ __noinline__ int64_t paged_total(const int32_t *seq_lens, int B, int append,
+                                            int64_t max_len, int UH, int lane) {
+  int64_t tot = 0;
+  for (int b = lane; b < B; b += 32) tot += paged_blocks(seq_lens, b, append, max_len);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  return tot * UH;
+}
+
+// Paged cache, whole warp: the sequence whose range of the flat block space
+// holds block bb (b = -1 if none does), with the range's first block and the
+// blocks of each of its units.  A scan over the sequences, 32 at a time.
+struct SeqHit {
+  int64_t start, nbs;
+  int b;
+};
+__device__ __noinline__ SeqHit paged_find(const int32_t *seq_lens, int B, int append,
+                                          int64_t max_len, int UH, int64_t bb, int lane) {
+  int64_t carry = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int64_t n = b < B ? paged_blocks(seq_lens, b, append, max_len) * UH : 0;
+    int64_t incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int64_t excl = carry + incl - n;
+    const uint32_t hit = __ballot_sync(0xffffffffu, n > 0 && excl <= bb && bb < excl + n);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      SeqHit h;
+      h.start = __shfl_sync(0xffffffffu, excl, src);
+      h.nbs = __shfl_sync(0xffffffffu, n, src) / UH;
+      h.b = b0 + src;
+      return h;
+    }
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  SeqHit none;
+  none.start = none.nbs = 0;
+  none.b = -1;
+  return none;
+}
+
+// TRACK: keep the page fields up to date (positions that issue copies).
+template <bool PAGED, bool TRACK = true>
 __device__ __forceinline__ void pos_next(const DecParams &p, BlockPos &pos) {
-  if (++pos.blk < pos.nb) return;
+  if (++pos.blk < pos.nb) {
+    if constexpr (PAGED && TRACK) {
+      pos.y += DEC_KB;  // pages hold a whole number of blocks
+      if (pos.y == p.page_tokens) {
+        pos.y = 0;
+        ++pos.pidx;
+      }
+    }
+    return;
+  }
   pos.blk = 0;
   if constexpr (PAGED) {
+    if constexpr (TRACK) {
+      pos.y = 0;
+      pos.pidx = 0;
+    }
     // skip units without blocks; never step past the last unit
     do {
       if (pos.u + 1 >= p.units) return;
@@ -226,11 +344,12 @@ __device__ __forceinline__ void pos_next(const DecParams &p, BlockPos &pos) {
   }
 }
 
-// First flat block of unit u.
-template <bool PAGED>
-__device__ __forceinline__ int64_t unit_first_block(const DecParams &p, int64_t u) {
-  if constexpr (PAGED) return p.unit_off[u];
-  else return u * p.nb_u;
+// Paged cache: look up the pool page of the block at `pos` ahead of the copy
+// that needs it, so that the table read is not on the issue path.  `pos` is
+// always a block of its unit or block 0 of a unit, so the entry read lies
+// inside the sequence's row of the table.
+__device__ __forceinline__ void load_page(BlockPos &pos) {
+  pos.page = __ldg(pos.trow + pos.pidx);
 }
 
 template <int M, int D, bool S8>
@@ -263,10 +382,8 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
       // holding this block (row within the page) for a paged cache
       int y = (int)key0, z = (int)kvi;
       if constexpr (PAGED) {
-        const int64_t b = kvi / p.Hkv;
-        const int page = p.block_table[b * p.max_pages + (int)(key0 / p.page_tokens)];
-        y = (int)(key0 % p.page_tokens);
-        z = page * p.Hkv + (int)(kvi - b * p.Hkv);
+        y = pos.y;
+        z = pos.page * p.Hkv + pos.hkv;
       }
       mbar_expect_tx(ring.bar(s), C::V_BYTES + C::SIGN_BYTES + 2 * DEC_KB);
 #pragma unroll
@@ -498,13 +615,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   const int wid = threadIdx.x >> 5;
   const int w = blockIdx.x * DEC_WARPS + wid;
   if (w >= p.W) return;
-  // a paged call's work plan (and its appended keys) come from the prep kernel
-  if constexpr (PAGED) griddep_wait();
-  const int64_t NB = PAGED ? p.unit_off[p.units] : p.NB;
-  // a paged call is launched for the bound; with fewer blocks than warps the
-  // first NB warps take one block each and the rest have nothing to do (no
-  // warp may own an empty run: the combine reads a record from every warp
-  // between a unit's first and last)
+  // a paged call plans its split from seq_lens (an input, not written by the
+  // prep kernel that runs before this one); it is launched for the bound, so
+  // with fewer blocks than warps the first NB warps take one block each and
+  // the rest have nothing to do (no warp may own an empty run: the combine
+  // reads a record from every warp between a unit's first and last)
+  const int64_t NB =
+      PAGED ? paged_total(p.seq_lens, p.B, p.append, p.T, p.UH, lane) : p.NB;
   const int Wn = PAGED ? (int)(NB < p.W ? NB : p.W) : p.W;
   if (w >= Wn) return;
   const int g = lane >> 2;  // group id: head row / key column / dim row
@@ -525,20 +642,50 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   __syncwarp();
 
   // prologue: fill the ring
-  BlockPos ipos = pos_of_block<PAGED>(p, bbeg);
+  BlockPos ipos;
+  if constexpr (PAGED) {
+    const SeqHit h = paged_find(p.seq_lens, p.B, p.append, p.T, p.UH, bbeg, lane);
+    if (h.b < 0) {
+      if (lane == 0) record_device_error(p.err, DERR_DECODE_PLAN);
+      return;
+    }
+    const int64_t r = bbeg - h.start;
+    const int64_t uin = r / h.nbs;
+    ipos.u = (int64_t)h.b * p.UH + uin;
+    ipos.blk = r - uin * h.nbs;
+    pos_load_unit<true>(p, ipos);
+    const int key0 = (int)ipos.blk * DEC_KB;  // < max_len < 2^31
+    ipos.pidx = key0 / p.page_tokens;
+    ipos.y = key0 - ipos.pidx * p.page_tokens;
+    load_page(ipos);
+  } else {
+    ipos = pos_of_block(p, bbeg);
+  }
   const BlockPos pos0 = ipos;
+  int issued = 0;
 #pragma unroll
   for (int s = 0; s < C::STAGES; ++s) {
     if (s < nblk) {
+      // the block holding the key this call appends is written by the prep
+      // kernel: copy it only after the wait below
+      if (PAGED && p.append && ipos.blk == ipos.nb - 1) break;
       issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
       pos_next<PAGED>(p, ipos);
+      if constexpr (PAGED) load_page(ipos);
+      ++issued;
     }
   }
 
-  // the query projections come from the previous kernel on the stream, which
-  // may still be running (programmatic dependent launch): wait for it only
-  // now, after the first copies are on their way
-  if constexpr (!PAGED) griddep_wait();
+  // the query projections (and a paged call's appended keys) come from the
+  // previous kernel on the stream, which may still be running (programmatic
+  // dependent launch): wait for it only now, after the first copies are on
+  // their way
+  griddep_wait();
+  for (int s = issued; s < C::STAGES && s < nblk; ++s) {
+    issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+    pos_next<PAGED>(p, ipos);
+    if constexpr (PAGED) load_page(ipos);
+  }
 
   // per-unit state
   int64_t cur_u = -1, kv_base = 0;
@@ -593,11 +740,11 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     if (u != cur_u) {
       if (cur_u >= 0) flush(cur_u);
       cur_u = u;
-      const int64_t kvi = pos.kvi;
-      const int hg = (int)(u - kvi * p.HG);
-      const int hkv = (int)(kvi % p.Hkv);
-      kv_base = kvi * p.T;
-      b_idx = (int)(kvi / p.Hkv);
+      const int kvi = (int)pos.kvi;  // < 2^24 (checked by the plan)
+      const int hg = (int)u - kvi * p.HG;
+      b_idx = kvi / p.Hkv;
+      const int hkv = kvi - b_idx * p.Hkv;
+      kv_base = (int64_t)kvi * p.T;
       hq0 = hkv * p.G + hg * DEC_HPAD;
       Gg = min(DEC_HPAD, p.G - hg * DEC_HPAD);
       mx = -INFINITY;
@@ -809,8 +956,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     if (i + C::STAGES < nblk) {
       issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
       pos_next<PAGED>(p, ipos);
+      if constexpr (PAGED) load_page(ipos);
     }
-    pos_next<PAGED>(p, pos);
+    pos_next<PAGED, false>(p, pos);
   }
   griddep_launch_dependents();
   if (failed) {
@@ -835,33 +983,63 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 constexpr int COMB_MAX_SLOTS = DEC_SM_COUNT * DEC_MAX_CTAS_SM * DEC_WARPS + 1;
 
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(D) decode_combine_kernel(
-    const float *__restrict__ partials, uint16_t *__restrict__ out, int Hq,
-    int Hkv, int G, int HG, int64_t nb_u, int64_t NB_fixed, int W, int slots,
-    const int64_t *__restrict__ unit_off, int units) {
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
+                                                           uint16_t *__restrict__ out) {
   __shared__ float wts[COMB_MAX_SLOTS];
   __shared__ float inv_l;
-  griddep_wait();  // every partial state of the scorer is needed
+  __shared__ int64_t red[2][D / 32];
+  const float *__restrict__ partials = p.partials;
+  const int Hq = p.Hq, G = p.G;
+  int W = p.W;
   const int bh = blockIdx.x;
   const int b = bh / Hq, hq = bh - b * Hq;
   const int hkv = hq / G, hl = hq - hkv * G;
   const int hg = hl / DEC_HPAD, hh = hl - hg * DEC_HPAD;
-  const int64_t u = ((int64_t)b * Hkv + hkv) * HG + hg;
+  const int64_t u = ((int64_t)b * p.Hkv + hkv) * p.HG + hg;
   int64_t first, last, NB;
   if constexpr (PAGED) {
-    NB = unit_off[units];
-    first = unit_off[u];
-    last = unit_off[u + 1] - 1;
-    if (last < first) {  // nothing to attend over: zeros
+    // the unit's blocks in the flat space: those of the sequences before b,
+    // then this sequence's units in order (as the scorer's plan)
+    int64_t pre = 0, tot = 0;
+    for (int bb = threadIdx.x; bb < p.B; bb += D) {
+      const int64_t n = paged_blocks(p.seq_lens, bb, p.append, p.T);
+      tot += n;
+      pre += bb < b ? n : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+      red[0][threadIdx.x >> 5] = tot;
+      red[1][threadIdx.x >> 5] = pre;
+    }
+    __syncthreads();
+    tot = pre = 0;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      tot += red[0][k];
+      pre += red[1][k];
+    }
+    const int64_t nbs = paged_blocks(p.seq_lens, b, p.append, p.T);
+    if (threadIdx.x == 0 && hq == 0 &&
+        (int64_t)__ldg(p.seq_lens + b) + p.append > p.T)
+      record_device_error(p.err, DERR_DECODE_PLAN);  // length past the bound
+    if (nbs == 0) {  // nothing to attend over: zeros
       out[(int64_t)bh * D + threadIdx.x] = 0;
       return;
     }
+    NB = tot * p.UH;
+    first = pre * p.UH + (u - (int64_t)b * p.UH) * nbs;
+    last = first + nbs - 1;
+    W = (int)(NB < W ? NB : W);  // as the scorer
   } else {
-    NB = NB_fixed;
-    first = u * nb_u;
-    last = (u + 1) * nb_u - 1;
+    NB = p.NB;
+    first = u * p.nb_u;
+    last = (u + 1) * p.nb_u - 1;
   }
-  if constexpr (PAGED) W = (int)(NB < W ? NB : W);  // as the scorer
+  griddep_wait();  // every partial state of the scorer is needed
   const int f = warp_of_block(first, NB, W);
   const int l = warp_of_block(last, NB, W);
   const int n = min(l - f + 1, COMB_MAX_SLOTS);
@@ -906,9 +1084,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// 4. paged calls: one prep launch does the query projections (CTAs
-// [0, B*Hq)), appends each sequence's new key (CTAs [B*Hq, B*Hq + B*Hkv) when
-// keys are given) and writes the work plan (last CTA).
+// 4. paged calls: one prep launch of 256-thread CTAs does the query
+// projections (four queries per CTA) and, when keys are given, appends each
+// sequence's new key (four keys per CTA).  The scorer and the combine derive
+// the work split from seq_lens themselves.
 struct PrepParams {
   const void *Q;
   const uint16_t *S;
@@ -922,105 +1101,71 @@ struct PrepParams {
   int num_pages, page_tokens, max_pages;
   const int32_t *block_table;
   const int32_t *seq_lens;
-  int B, Hkv, HG, units, append;
+  int B, Hkv, append;
   int64_t max_len;
-  int64_t *unit_off;            // [units + 1]
   int *err;
 };
 
 template <int M, int D, bool QF32, bool KF32>
-__global__ void __launch_bounds__(M) paged_prep_kernel(const PrepParams pp) {
-  __shared__ float sh[D];
-  __shared__ int64_t scan[M];
+__global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepParams pp) {
+  __shared__ float ys[PROJ_VECS][M];
+  // launched early behind the previous kernel on the stream (programmatic
+  // dependent launch): wait for it before reading anything, then let the
+  // scorer be scheduled; it waits for this grid's results where it needs them
+  griddep_wait();
+  griddep_launch_dependents();
   const int bid = blockIdx.x;
   const int i = threadIdx.x;
-  if (bid < pp.nq) {
-    // ---- query projection u = S q (as qproj_kernel)
-    uint4 row[D / 8];
-    const uint4 *src = reinterpret_cast<const uint4 *>(pp.S + (int64_t)i * D);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) row[c] = __ldg(src + c);
-    for (int j = i; j < D; j += M)
-      sh[j] = QF32 ? reinterpret_cast<const float *>(pp.Q)[(int64_t)bid * D + j]
-                   : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(pp.Q)[(int64_t)bid * D + j]);
-    __syncthreads();
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint32_t w[4] = {row[c].x, row[c].y, row[c].z, row[c].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc0 = fmaf(__uint_as_float(w[e] << 16), sh[c * 8 + 2 * e], acc0);
-        acc1 = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), sh[c * 8 + 2 * e + 1], acc1);
-      }
-    }
-    pp.U[(int64_t)bid * M + i] = acc0 + acc1;
+  const int qctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS;
+  if (bid < qctas) {
+    // ---- query projections u = S q, four queries per CTA
+    const int64_t x0 = (int64_t)bid * PROJ_VECS;
+    const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)pp.nq - x0);
+    project4<M, D, QF32>(pp.S, pp.Q, x0, nx, pp.U + x0 * M);
     return;
   }
-  const int nappend = pp.append ? pp.B * pp.Hkv : 0;
-  if (bid < pp.nq + nappend) {
-    // ---- append: quantize key kvi = b*Hkv + hkv and store it at position
-    // seq_lens[b] of its sequence (thread i: sketch row i; a ballot per warp
-    // packs 32 code bits)
-    const int kvi = bid - pp.nq;
-    const int b = kvi / pp.Hkv, hkv = kvi - b * pp.Hkv;
-    for (int j = i; j < D; j += M)
-      sh[j] = KF32 ? reinterpret_cast<const float *>(pp.K_new)[(int64_t)kvi * D + j]
-                   : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(pp.K_new)[(int64_t)kvi * D + j]);
+  const int nkv = pp.B * pp.Hkv;
+  const int actas = pp.append ? (nkv + PROJ_VECS - 1) / PROJ_VECS : 0;
+  if (bid < qctas + actas) {
+    // ---- append: quantize keys kvi = b*Hkv + hkv (four per CTA) and store
+    // each at position seq_lens[b] of its sequence
+    const int x0 = (bid - qctas) * PROJ_VECS;
+    const int nx = min(PROJ_VECS, nkv - x0);
+    project4<M, D, KF32>(pp.S, pp.K_new, x0, nx, &ys[0][0]);
     __syncthreads();
+    const int lane = i & 31, j = i >> 5;  // warp j stores key x0 + j
+    if (j >= nx) return;
+    const int kvi = x0 + j;
+    const int b = kvi / pp.Hkv, hkv = kvi - b * pp.Hkv;
     const int64_t pos = pp.seq_lens[b];
     const int64_t pidx = pos / pp.page_tokens;
     const int page = (pos >= 0 && pidx < pp.max_pages)
                          ? pp.block_table[(int64_t)b * pp.max_pages + pidx] : -1;
     if (page < 0 || page >= pp.num_pages || pos + 1 > pp.max_len) {
-      if (i == 0) record_device_error(pp.err, DERR_DECODE_PLAN);
+      if (lane == 0) record_device_error(pp.err, DERR_DECODE_PLAN);
       return;
     }
     const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
-    const uint16_t *srow = pp.S + (int64_t)i * D;
-    float y = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < D; ++j) y = fmaf(bf16_bits_to_f32(srow[j]), sh[j], y);
-    const uint32_t word = __ballot_sync(0xffffffffu, y >= 0.f);
-    if ((i & 31) == 0) pp.sign_pages[slot * (M / 32) + (i >> 5)] = word;
-    if (i < 32) {
-      float ss = 0.f;
-      for (int j = i; j < D; j += 32) ss = fmaf(sh[j], sh[j], ss);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (i == 0) pp.norm_pages[slot] = __half_as_ushort(__float2half_rn(sqrtf(ss)));
+    for (int w = 0; w < M / 32; ++w) {  // bit l of word w: coordinate 32w + l >= 0
+      const uint32_t word = __ballot_sync(0xffffffffu, ys[j][w * 32 + lane] >= 0.f);
+      if (lane == 0) pp.sign_pages[slot * (M / 32) + w] = word;
     }
-    for (int j = i; j < D; j += M) pp.value_pages[slot * D + j] = pp.V_new[(int64_t)kvi * D + j];
+    float ss = 0.f;
+    for (int c = lane; c < D; c += 32) {
+      const float x = KF32 ? reinterpret_cast<const float *>(pp.K_new)[(int64_t)kvi * D + c]
+                           : bf16_bits_to_f32(
+                                 reinterpret_cast<const uint16_t *>(pp.K_new)[(int64_t)kvi * D + c]);
+      ss = fmaf(x, x, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) pp.norm_pages[slot] = __half_as_ushort(__float2half_rn(sqrtf(ss)));
+    const uint32_t *vsrc = reinterpret_cast<const uint32_t *>(pp.V_new + (int64_t)kvi * D);
+    uint32_t *vdst = reinterpret_cast<uint32_t *>(pp.value_pages + slot * D);
+    for (int c = lane; c < D / 2; c += 32) vdst[c] = vsrc[c];
     return;
   }
-  // ---- work plan: unit u owns ceil(len/32) blocks, len = seq_lens[b] (+1)
-  int64_t carry = 0;
-  for (int base = 0; base < pp.units; base += M) {
-    const int u = base + i;
-    int64_t nb = 0;
-    if (u < pp.units) {
-      const int b = (u / pp.HG) / pp.Hkv;
-      int64_t len = (int64_t)pp.seq_lens[b] + pp.append;
-      if (len < 0) len = 0;
-      if (len > pp.max_len) {
-        record_device_error(pp.err, DERR_DECODE_PLAN);
-        len = pp.max_len;
-      }
-      nb = (len + DEC_KB - 1) / DEC_KB;
-    }
-    scan[i] = nb;
-    __syncthreads();
-    for (int o = 1; o < M; o <<= 1) {  // inclusive scan (Hillis-Steele)
-      const int64_t v = i >= o ? scan[i - o] : 0;
-      __syncthreads();
-      scan[i] += v;
-      __syncthreads();
-    }
-    if (u < pp.units) pp.unit_off[u] = carry + scan[i] - nb;
-    carry += scan[M - 1];
-    __syncthreads();
-  }
-  if (i == 0) pp.unit_off[pp.units] = carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -1056,16 +1201,14 @@ static bool plan_common(int B, int Hq, int Hkv, int64_t T, int m, int d, DecodeP
 
 bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, DecodePlan *pl) {
   if (!plan_common(B, Hq, Hkv, T, m, d, pl)) return false;
-  pl->off_bytes = 0;
   pl->total_bytes = pl->u_bytes + pl->partial_bytes;
   return true;
 }
 
 bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d, DecodePlan *pl) {
-  if (!plan_common(B, Hq, Hkv, max_len, m, d, pl)) return false;
-  pl->off_bytes = round_up((size_t)(pl->units + 1) * sizeof(int64_t), 256);
-  pl->total_bytes = pl->u_bytes + pl->off_bytes + pl->partial_bytes;
-  return true;
+  // the same scratch as a contiguous call at the bound: the split itself is
+  // derived on the device from the lengths and needs no storage
+  return make_decode_plan(B, Hq, Hkv, max_len, m, d, pl);
 }
 
 // Tensor maps of one call (see DecMaps).
@@ -1149,6 +1292,8 @@ static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *par
   p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634074);
   p.score_stride = pl.T;
   p.units = pl.units;
+  p.B = pl.B;
+  p.UH = pl.Hkv * pl.HG;
 }
 
 // Launch the scorer (one wave, <= the plan's warp bound) and the combine.
@@ -1172,8 +1317,7 @@ static cudaError_t launch_scorer_combine(const DecodePlan &pl, DecParams &p, con
   e = launch_pdl(kern, dim3(ctas), dim3(DEC_WARPS * 32), C::CTA_BYTES, stream, maps, p);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_combine_kernel<D, PAGED>, dim3(pl.B * pl.Hq), dim3(D), 0, stream,
-                    (const float *)p.partials, out, pl.Hq, pl.Hkv, pl.G, pl.HG, pl.nb_u,
-                    pl.NB, p.W, pl.records, p.unit_off, pl.units);
+                    (const DecParams)p, out);
 }
 
 template <int M, int D, bool S8>
@@ -1192,10 +1336,11 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   int *err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidSymbol;
   const int bh = pl.B * pl.Hq;
+  const int qctas = (bh + PROJ_VECS - 1) / PROJ_VECS;
   if (q_f32)
-    qproj_kernel<M, D, true><<<bh, M, 0, stream>>>(Q, S, U);
+    qproj_kernel<M, D, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh);
   else
-    qproj_kernel<M, D, false><<<bh, M, 0, stream>>>(Q, S, U);
+    qproj_kernel<M, D, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecParams p;
@@ -1269,8 +1414,7 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
                                   cudaStream_t stream) {
   uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
   float *U = reinterpret_cast<float *>(ws);
-  int64_t *unit_off = reinterpret_cast<int64_t *>(ws + pl.u_bytes);
-  float *partials = reinterpret_cast<float *>(ws + pl.u_bytes + pl.off_bytes);
+  float *partials = reinterpret_cast<float *>(ws + pl.u_bytes);
   DecMaps maps;
   if (!make_paged_maps(&maps, a, pl.Hkv, M, D)) return cudaErrorInvalidValue;
   int *err = device_error_ptr();
@@ -1281,24 +1425,25 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   pp.sign_pages = a.sign_pages; pp.norm_pages = a.norm_pages; pp.value_pages = a.value_pages;
   pp.num_pages = a.num_pages; pp.page_tokens = a.page_tokens; pp.max_pages = a.max_pages;
   pp.block_table = a.block_table; pp.seq_lens = a.seq_lens;
-  pp.B = pl.B; pp.Hkv = pl.Hkv; pp.HG = pl.HG; pp.units = pl.units;
+  pp.B = pl.B; pp.Hkv = pl.Hkv;
   pp.append = a.K_new != nullptr;
   pp.max_len = pl.T;
-  pp.unit_off = unit_off;
   pp.err = err;
-  const int prep_ctas = pp.nq + (pp.append ? pl.B * pl.Hkv : 0) + 1;
-  if (a.q_f32) {
-    if (a.k_f32) paged_prep_kernel<M, D, true, true><<<prep_ctas, M, 0, stream>>>(pp);
-    else paged_prep_kernel<M, D, true, false><<<prep_ctas, M, 0, stream>>>(pp);
-  } else {
-    if (a.k_f32) paged_prep_kernel<M, D, false, true><<<prep_ctas, M, 0, stream>>>(pp);
-    else paged_prep_kernel<M, D, false, false><<<prep_ctas, M, 0, stream>>>(pp);
-  }
-  cudaError_t e = cudaGetLastError();
+  const int nkv = pl.B * pl.Hkv;
+  const int prep_ctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS +
+                        (pp.append ? (nkv + PROJ_VECS - 1) / PROJ_VECS : 0);
+  const dim3 pg(prep_ctas), pb(PROJ_THREADS);
+  cudaError_t e;
+  if (a.q_f32)
+    e = a.k_f32 ? launch_pdl(paged_prep_kernel<M, D, true, true>, pg, pb, 0, stream, pp)
+                : launch_pdl(paged_prep_kernel<M, D, true, false>, pg, pb, 0, stream, pp);
+  else
+    e = a.k_f32 ? launch_pdl(paged_prep_kernel<M, D, false, true>, pg, pb, 0, stream, pp)
+                : launch_pdl(paged_prep_kernel<M, D, false, false>, pg, pb, 0, stream, pp);
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, nullptr, nullptr, a.scores, a.softmax_scale, M, err);
-  p.unit_off = unit_off; p.seq_lens = a.seq_lens; p.block_table = a.block_table;
+  p.seq_lens = a.seq_lens; p.block_table = a.block_table;
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
   return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);

@@ -39,7 +39,6 @@ struct DecodePlan {
   int W;         // bound on the warps launched
   int records;   // partial-state records: W + units
   size_t u_bytes;        // fp32 query projections [B][Hq][m]
-  size_t off_bytes;      // paged: int64 block offsets [units + 1]
   size_t partial_bytes;  // fp32 [records][8][d + 2]
   size_t total_bytes;
 };

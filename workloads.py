@@ -18,12 +18,18 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
            m=256; bf16 keys N(0,1) with 4 outlier channels x10.
   sweep    m in {64,128,256,512} x d in {64,128}; batch 16, 32 heads MHA,
            context 16384; bf16 keys and values N(0,1).
+  paged-gqa  serving step of the gqa shapes over a paged cache: batch 8,
+           32 / 8 heads, d=128, m=256; sequence lengths uniform in
+           [16384, 32767) plus the appended key (bound 32768); pages of 64
+           tokens assigned in a shuffled order; cache contents drawn as for
+           gqa.
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
   * data seeds: workload index i (1..5) gives torch generator seeds
     1000*i + {0: keys, 1: values, 2: queries, 3: outlier channels,
-    4: per-token norms};
+    4: per-token norms, 5: sequence lengths, 6: page order, 7: appended
+    keys, 8: appended values};
   * outlier channels: the first 4 entries of a seeded permutation of range(d);
   * queries are N(0,1) in the key dtype, scaled by ``q_scale`` (default 1);
   * softmax scale 1/sqrt(d).
@@ -79,7 +85,12 @@ SWEEP_BASE = Workload("sweep", 5, 16, 32, 32, 16384, 128, 256, torch.bfloat16)
 SWEEP_M = (64, 128, 256, 512)
 SWEEP_D = (64, 128)
 
-ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE)}
+# paged-gqa: T is the length bound (max_len) of the paged cache
+PAGED_GQA = Workload("paged-gqa", 6, 8, 32, 8, 32768, 128, 256, torch.bfloat16,
+                     outliers=4)
+PAGE_TOKENS = 64
+
+ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA)}
 
 
 def sweep_points():
@@ -149,3 +160,35 @@ def random_keys(n: int, d: int, seed: int, dtype=torch.bfloat16, device="cpu",
     x = torch.randn((n, d), generator=_gen(device, seed), device=device,
                     dtype=torch.float32) * scale
     return x.to(dtype)
+
+
+def paged_layout(w: Workload, page_tokens: int = PAGE_TOKENS, spare_pages: int = 16):
+    """Sequence lengths and a shuffled block table for a paged cache.
+
+    Lengths are uniform in [T/2, T-1) so that the appended key still fits the
+    bound T; sequence b owns ceil((len_b + 1) / page_tokens) pages, taken from
+    a seeded permutation of the pool.  Returns (lens int32 [B], block_table
+    int32 [B, max_pages] with -1 in unused entries, num_pages).
+    """
+    g = _gen("cpu", 1000 * w.index + 5)
+    lens = torch.randint(w.T // 2, w.T - 1, (w.B,), generator=g, dtype=torch.int64)
+    per_seq = [-(-(int(L) + 1) // page_tokens) for L in lens]
+    max_pages = -(-w.T // page_tokens)
+    num_pages = sum(per_seq) + spare_pages
+    perm = torch.randperm(num_pages, generator=_gen("cpu", 1000 * w.index + 6))
+    table = torch.full((w.B, max_pages), -1, dtype=torch.int32)
+    k = 0
+    for b, n in enumerate(per_seq):
+        table[b, :n] = perm[k:k + n].to(torch.int32)
+        k += n
+    return lens.to(torch.int32), table, num_pages
+
+
+def new_tokens(w: Workload, device="cpu"):
+    """The key and value each sequence appends in a decode step: [B, Hkv, d]
+    each, drawn like the cache's keys (outlier channels included) and values."""
+    K = torch.empty((w.B * w.Hkv, w.d), dtype=w.key_dtype, device=device)
+    _fill_normal(K, _gen(device, 1000 * w.index + 7), 1 << 20, outlier_channels(w))
+    V = torch.empty((w.B * w.Hkv, w.d), dtype=torch.bfloat16, device=device)
+    _fill_normal(V, _gen(device, 1000 * w.index + 8), 1 << 20, None)
+    return K.view(w.B, w.Hkv, w.d), V.view(w.B, w.Hkv, w.d)
