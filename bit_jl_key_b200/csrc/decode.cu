@@ -121,7 +121,7 @@ struct DecMaps {
 
 // Paged cache: blocks of every unit of sequence b, ceil(len / 32) with
 // len = seq_lens[b] (+1 when the call appends a key) kept inside [0, max_len];
-// a length past the bound is reported by the combine.
+// a length outside the bound is reported by the combine.
 __device__ __forceinline__ int64_t paged_blocks(const int32_t *seq_lens, int b, int append,
                                                 int64_t max_len) {
   int64_t len = (int64_t)__ldg(seq_lens + b) + append;
@@ -1023,9 +1023,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
       pre += red[1][k];
     }
     const int64_t nbs = paged_blocks(p.seq_lens, b, p.append, p.T);
-    if (threadIdx.x == 0 && hq == 0 &&
-        (int64_t)__ldg(p.seq_lens + b) + p.append > p.T)
-      record_device_error(p.err, DERR_DECODE_PLAN);  // length past the bound
+    if (threadIdx.x == 0 && hq == 0) {  // a length outside [0, bound]
+      const int64_t len = __ldg(p.seq_lens + b);
+      if (len < 0 || len + p.append > p.T) record_device_error(p.err, DERR_DECODE_PLAN);
+    }
     if (nbs == 0) {  // nothing to attend over: zeros
       out[(int64_t)bh * D + threadIdx.x] = 0;
       return;

@@ -167,9 +167,10 @@ JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *
 
 /*
  * jl_decode_paged_workspace_bytes -- device scratch jl_decode_attention_paged
- * needs (query projections, the per-call work plan and split partial
- * states) for B sequences of at most max_len keys each (counting the key a
- * call appends).  Depends on the shapes only; 0 for unsupported shapes.
+ * needs (query projections and split partial states) for B sequences of at
+ * most max_len keys each (counting the key a call appends).  Depends on the
+ * shapes only (the device-side lengths never change it); 0 for unsupported
+ * shapes.
  */
 JL_API size_t jl_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len,
                                               int m, int d);
@@ -202,13 +203,18 @@ JL_API size_t jl_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t ma
  *                 sequence's last page are not read.
  *   seq_lens    : in, B int32 (device): keys already cached per sequence.
  *                 Not modified (the caller advances it after an append).
+ *                 A length outside [0, max_len] (max_len - 1 with K_new)
+ *                 records a device error (jl_device_error) and the
+ *                 sequence is clipped to the bound.
  *   max_len     : bound on seq_lens[b] (+1 with K_new), used to size the
  *                 work split and the workspace.
  *   scores      : optional out, B x Hq x max_len fp32 (row stride max_len).
  *   workspace   : >= jl_decode_paged_workspace_bytes(...), 256-byte aligned.
  * A sequence with no key to attend over (seq_lens[b] == 0, no K_new) gets an
  * output of zeros.  Values past a sequence's last key inside its last page
- * are never read into the result, whatever they hold.
+ * are never read into the result, whatever they hold.  The page that
+ * receives an appended key must belong to that sequence alone: the other
+ * sequences' keys are read while the new keys are being written.
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
  * JL_ERR_CUDA.
  */

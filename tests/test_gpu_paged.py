@@ -139,3 +139,36 @@ def test_paged_equals_contiguous_decode():
                                        V.contiguous(), table, seq, T)
     mabs, rel = H.output_errors(H.f64(out), H.f64(ref))
     assert mabs <= 1e-2 and rel <= 1e-2
+
+
+def test_paged_length_past_bound_reports_error_and_recovers():
+    # a length at the bound with a key to append cannot fit: the kernels clip
+    # the sequence, skip the write and record an error; the next valid call
+    # is unaffected
+    torch.cuda.set_device(0)
+    B, Hq, Hkv, d, m, P = 2, 4, 2, 128, 256, 32
+    lens = [64, 10]
+    max_len = 65
+    S, S64, table, (sp, npg, vp), keys, vals = _setup(B, Hq, Hkv, d, m, P, lens, max_len, 11,
+                                                      garbage=False)
+    Q = workloads.random_keys(B * Hq, d, 60).reshape(B, Hq, d).cuda()
+    Kn = workloads.random_keys(B * Hkv, d, 61).reshape(B, Hkv, d).cuda()
+    Vn = workloads.random_keys(B * Hkv, d, 62).reshape(B, Hkv, d).cuda()
+    tab = torch.from_numpy(table).cuda()
+    assert jl.jl_device_error() == 0
+    bad = torch.tensor([65, 10], dtype=torch.int32, device="cuda")
+    jl.jl_decode_attention_paged(Q, S, sp, npg, vp, tab, bad, max_len, K_new=Kn, V_new=Vn)
+    assert jl.jl_device_error() == 3          # inconsistent work split / bound
+    assert jl.jl_device_error() == 0          # reading clears it
+    good = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    out = jl.jl_decode_attention_paged(Q, S, sp, npg, vp, tab, good, max_len)
+    torch.cuda.synchronize()
+    assert jl.jl_device_error() == 0
+    scale = 1.0 / math.sqrt(d)
+    for b in range(B):
+        sig = np.stack([oracle.quantize(H.f64(keys[b][h]), S64)[0] for h in range(Hkv)])
+        n16 = np.stack([oracle.quantize(H.f64(keys[b][h]), S64)[2] for h in range(Hkv)])
+        ref_out, _ = oracle.decode(H.f64(Q[b].cpu())[None], S64, sig[None],
+                                   oracle.fp16_bits_to_f64(n16)[None], H.f64(vals[b])[None], scale)
+        mabs, rel = H.output_errors(H.f64(out[b])[None], ref_out)
+        assert mabs <= H.OUT_ABS and rel <= 1e-2, (b, mabs, rel)
