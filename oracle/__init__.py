@@ -69,6 +69,9 @@ def lib():
         L.jlo_scores.restype = None
         L.jlo_scores.argtypes = [ctypes.c_long, ctypes.c_int, _f64p, _u32p,
                                  _f64p, _f64p]
+        L.jlo_dequantize.restype = None
+        L.jlo_dequantize.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                     _u32p, _f64p, _f64p, _f64p]
         L.jlo_decode.restype = None
         L.jlo_decode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_long, ctypes.c_int, ctypes.c_int,
@@ -193,6 +196,24 @@ def estimate(q, k, S) -> float:
     signs, norms, _, _ = quantize(np.asarray(k, np.float64)[None, :], S)
     u = project(np.asarray(q, np.float64)[None, :], S)[0]
     return float(scores(u, signs, norms)[0])
+
+
+def dequantize(signs, norms, S) -> np.ndarray:
+    """Q^-1: khat = sqrt(pi/2)/m * ||k|| * S^T z for each code.
+
+    signs uint32 [n, m/32]; norms [n] (float64 values of the stored norms);
+    S [m, d].  Returns float64 [n, d].
+    """
+    signs = _c(signs, np.uint32)
+    norms = _c(norms, np.float64).reshape(-1)
+    S = _c(S, np.float64)
+    m, d = S.shape
+    n = signs.shape[0]
+    assert signs.shape == (n, m // 32) and norms.shape == (n,)
+    out = np.empty((n, d), dtype=np.float64)
+    lib().jlo_dequantize(n, d, m, _ptr(signs, _u32p), _ptr(norms, _f64p),
+                         _ptr(S, _f64p), _ptr(out, _f64p))
+    return out
 
 
 def decode(Q, S, signs, norms, V, softmax_scale: float, want_scores=False):

@@ -202,6 +202,31 @@ void jlo_scores(long T, int m, const double *u, const uint32_t *signs,
         out[t] = jlo_estimate_one(m, u, signs + t * words, norms[t]);
 }
 
+/* Dequantizer [GEO-QJL] Q^-1(z) = sqrt(pi/2)/d * S^T z, taken with m sketch
+ * rows and with the stored norm restoring the magnitude [GEO-POLAR]:
+ *   khat = sqrt(pi/2)/m * ||k|| * S^T z,   z_i = +1 if bit i is set, else -1
+ *   signs : n x (m/32) words, LSB-first
+ *   norms : n norms (float64 values of the stored norms)
+ *   S     : m x d (float64), row-major
+ *   out   : n x d reconstructions */
+void jlo_dequantize(long n, int d, int m, const uint32_t *signs,
+                    const double *norms, const double *S, double *out)
+{
+    int words = m / 32;
+    #pragma omp parallel for schedule(static)
+    for (long t = 0; t < n; ++t) {
+        const uint32_t *code = signs + t * words;
+        for (int j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < m; ++i) {
+                double z = ((code[i / 32] >> (i % 32)) & 1u) ? 1.0 : -1.0;
+                acc += S[(long)i * d + j] * z;
+            }
+            out[t * d + j] = sqrt(JLO_PI / 2.0) / (double)m * norms[t] * acc;
+        }
+    }
+}
+
 /* ---------------------------------------------------------------------- */
 /* Decode attention over compressed keys: the attention logits are the inner
  * products that the estimator of [GEO-QJL] approximates.  One query token per

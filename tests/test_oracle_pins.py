@@ -356,3 +356,76 @@ def test_qjl_code_has_no_block_constants():
     # 1 + 16/128 bits per coordinate, independent of any block size
     assert oracle.qjl_bits_per_coordinate(128, 128, 16) == 1.125
     assert oracle.qjl_bits_per_coordinate(256, 128, 16) == 2.125
+
+
+# --------------------------------------------------------------------------
+# dequantizer Q^-1 ("The Geometry of Forgetting ...", QJL section), with m
+# rows and the stored norm: khat = sqrt(pi/2)/m * ||k|| * S^T sign(S k)
+
+def test_dequantizer_hand_fixture():
+    fx = _golden("qjl_dequant_fixture.json")
+    d, m = fx["d"], fx["m"]
+    S = np.zeros((m, d))
+    S[:2] = np.array(fx["S_rows_0_1"], dtype=np.float64)
+    for key in fx["keys"]:
+        k = np.array(key["k"], dtype=np.float64)
+        signs, norms, _, _ = oracle.quantize(k[None], S)
+        assert int(signs[0, 0]) == key["code"]
+        assert norms[0] ** 2 == pytest.approx(key["norm_sq"], rel=1e-15)
+        khat = oracle.dequantize(signs, norms, S)[0]
+        want = math.sqrt(math.pi / 2) / m * math.sqrt(key["norm_sq"]) * np.array(key["StZ"])
+        assert np.allclose(khat, want, rtol=1e-14, atol=1e-15)
+
+
+def test_dequantizer_inner_product_equals_estimator():
+    # <y, Q^-1(Q(k))> is the asymmetric estimator, whatever y is: this ties
+    # the dequantizer's orientation (S^T z, not S z) and constant to the
+    # estimator, which is pinned on its own above
+    rng = np.random.default_rng(31)
+    d, m, n = 24, 96, 40
+    S = rng.standard_normal((m, d))
+    K = rng.standard_normal((n, d))
+    Y = rng.standard_normal((n, d)) * 3
+    signs, norms, _, _ = oracle.quantize(K, S)
+    khat = oracle.dequantize(signs, norms, S)
+    U = oracle.project(Y, S)
+    for i in range(n):
+        est = oracle.scores(U[i], signs[i:i + 1], norms[i:i + 1])[0]
+        assert Y[i] @ khat[i] == pytest.approx(est, rel=1e-12, abs=1e-12)
+
+
+def _reconstructions(k, m, R, seed):
+    rng = np.random.default_rng(seed)
+    d = k.shape[0]
+    out = np.empty((R, d))
+    for r in range(R):
+        S = rng.standard_normal((m, d))
+        signs, norms, _, _ = oracle.quantize(k[None], S)
+        out[r] = oracle.dequantize(signs, norms, S)[0]
+    return out
+
+
+def test_dequantizer_unbiased():
+    # E_S[khat] = sqrt(pi/2)/m ||k|| * m * E[s sign(s.k)] = k
+    rng = np.random.default_rng(40)
+    d, m, R = 10, 64, 4000
+    k = rng.standard_normal(d) * 2
+    rec = _reconstructions(k, m, R, 41)
+    sem = rec.std(axis=0, ddof=1) / math.sqrt(R)
+    assert np.all(np.abs(rec.mean(axis=0) - k) < 5 * sem)
+
+
+@pytest.mark.parametrize("m", [32, 128, 512])
+def test_reconstruction_mse_closed_form(m):
+    # D_mse of the page, for this quantizer: E||k - khat||^2 =
+    # ||k||^2 ((pi/2) d - 1) / m  (E||khat||^2 = ||k||^2 ((pi/2) d/m + (m-1)/m)
+    # for i.i.d. N(0,1) rows, minus ||k||^2 since khat is unbiased)
+    rng = np.random.default_rng(50 + m)
+    d, R = 16, 1500
+    k = rng.standard_normal(d)
+    rec = _reconstructions(k, m, R, 60 + m)
+    err = np.sum((rec - k) ** 2, axis=1) / (k @ k)
+    pred = (math.pi / 2 * d - 1) / m
+    sem = err.std(ddof=1) / math.sqrt(R)
+    assert abs(err.mean() - pred) < 5 * sem
+    assert err.mean() == pytest.approx(pred, rel=0.08)
