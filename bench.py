@@ -1,7 +1,7 @@
 """Benchmark: QJL key quantization + compressed-key decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -16,6 +16,10 @@ jl_decode_attention_paged call that appends every sequence's new key and
 value to a shuffled page pool and attends over its ragged context (the cache
 is filled once, untimed; the lengths stay fixed from step to step, so every
 step rewrites the same slots).
+
+The dequant-gqa workload times the explicit dequantizer: one
+jl_dequantize_keys call turning the gqa cache's codes and norms back into
+bf16 keys.
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload
 (independent sequences, no data-path collective), timing is the max over ranks
@@ -192,6 +196,18 @@ def decode_bytes(w):
     return w.B * w.Hkv * w.T * (w.m // 8 + 2 + 2 * w.d)
 
 
+def reconstruction_error(jl, w, S, signs, norms, K, rows=65536):
+    """Measured D_mse of the dequantizer on the first rows of the cache:
+    mean over keys of ||k - khat||^2 / ||k||^2, beside the closed form
+    ((pi/2) d - 1) / m for a Gaussian sketch.  Measurement only."""
+    n = min(rows, signs.shape[0])
+    khat = jl.jl_dequantize_keys(signs[:n], norms[:n], S).float()
+    k = K.reshape(-1, w.d)[:n].float()
+    rel = ((khat - k) ** 2).sum(1) / (k * k).sum(1)
+    return {"mean_rel_sq_error": float(rel.mean()),
+            "predicted": (math.pi / 2 * w.d - 1) / w.m, "samples": n}
+
+
 def score_error(jl, w, Q, S, signs, norms, V, K, max_rows=16):
     """Normalised error of the GPU estimator against the exact inner product
     on sampled (b, query head) rows: rms over keys of (s - <q,k>) / (|q||k|),
@@ -345,11 +361,107 @@ def run_paged(args, rank, world, local_rank):
     }
 
 
+def run_dequant(args, rank, world, local_rank):
+    """Explicit dequantizer over the gqa cache's codes: khat in bf16."""
+    import bit_jl_key_b200 as jl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload, args.batch)
+    peak, peak_kind = load_peaks()
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)
+    signs, norms = jl.jl_quantize_keys(K.view(-1, w.d), S)      # untimed set-up
+    recon = None if args.no_score_error else reconstruction_error(jl, w, S, signs, norms, K)
+    del K
+    torch.cuda.empty_cache()
+    n = signs.shape[0]
+    out = torch.empty((n, w.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        jl.jl_dequantize_keys(signs, norms, S, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        _barrier(world, dev)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        _barrier(world, dev)
+    ms = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    e2e = None
+    if not args.no_e2e:
+        hS = signs.cpu().pin_memory()
+        hN = norms.cpu().pin_memory()
+        hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            signs.copy_(hS, non_blocking=True)
+            norms.copy_(hN, non_blocking=True)
+            step()
+            hOut.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        _barrier(world, dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e_steps = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        _barrier(world, dev)
+        e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+        e2e = {"value": whole_job_rate(n, world, e_ms), "unit": "keys/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": hS.numel() * 4 + hN.numel() * 2,
+               "d2h_bytes_per_step": hOut.numel() * 2}
+
+    nbytes = n * (w.m // 8 + 2 + 2 * w.d)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    traffic = ncu_traffic("dequant:" + w.name)
+    return {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": whole_job_rate(n, world, ms), "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: {n} codes, m={w.m}, d={w.d} -> bf16 keys",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                   "l2": "inputs and outputs exceed L2 (126 MB); no flush"},
+        "phases": {"dequantize": {"ms": ms, "keys_per_s": n / (ms * 1e-3),
+                                  "algorithmic_bytes": nbytes, "GB_per_s": gbs,
+                                  "frac_of_hbm_peak": gbs / peak,
+                                  "tflops": n * 2 * w.m * w.d / (ms * 1e-3) / 1e12}},
+        "roofline": {"kernel": "jl_dequantize_keys", "bound": "hbm", "achieved": gbs,
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": gbs / peak, "algorithmic_bytes_per_launch": nbytes,
+                     "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
+        "reconstruction_error": recon,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
     if args.workload == "paged-gqa":
         return run_paged(args, rank, world, local_rank)
+    if args.workload == "dequant-gqa":
+        return run_dequant(args, rank, world, local_rank)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = pick_workload(args.workload, args.batch)
@@ -432,9 +544,10 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_rate(n_keys, world, ms_step)
 
     # ---- estimator quality on sampled heads (untimed)
-    score_err = None
+    score_err = recon_err = None
     if decode and not args.no_score_error:
         score_err = score_error(jl, w, Q, S, sg4, nr3, V, K)
+        recon_err = reconstruction_error(jl, w, S, signs, norms, K)
 
     # ---- end to end through the binding with pinned host buffers
     e2e = None
@@ -526,6 +639,7 @@ def run_ours(args, rank, world, local_rank):
         "phase_timing": "each phase alone: K back-to-back calls, CUDA events at the ends",
         "roofline": roof,
         "score_error": score_err,
+        "reconstruction_error": recon_err,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -545,6 +659,15 @@ def oracle_sample(w: workloads.Workload):
     import oracle
 
     S64 = oracle.sketch(w.m, w.d, w.sketch_seed)
+    if w.name == "dequant-gqa":
+        n = 16384
+        Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()
+        sig, _, n16, _ = oracle.quantize(Kf, S64)          # set-up, untimed
+        n64 = oracle.fp16_bits_to_f64(n16)
+
+        def run():
+            oracle.dequantize(sig, n64, S64)
+        return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
     if w.name == "prefill":
         n = 16384
         Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()

@@ -47,7 +47,7 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_quantize_keys_simt", "jl_decode_workspace_bytes",
             "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64",
             "jl_decode_attention_noalloc", "jl_decode_paged_workspace_bytes",
-            "jl_decode_attention_paged")
+            "jl_decode_attention_paged", "jl_dequantize_keys")
 
 _lib = None
 
@@ -87,6 +87,8 @@ def load():
     L.jl_decode_attention_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32,
                                               i32, i64, i32, i32, ctypes.c_float,
                                               vp, vp, vp]
+    L.jl_dequantize_keys.restype = i32
+    L.jl_dequantize_keys.argtypes = [vp, vp, i64, vp, i32, i32, vp, vp]
     L.jl_decode_paged_workspace_bytes.restype = sz
     L.jl_decode_paged_workspace_bytes.argtypes = [i32, i32, i32, i64, i32, i32]
     L.jl_decode_attention_paged.restype = i32
@@ -178,6 +180,27 @@ def jl_quantize_keys(K, S, signs=None, norms=None, stream=None):
 def jl_quantize_keys_simt(K, S, signs=None, norms=None, stream=None):
     """Same as jl_quantize_keys, computed on the SIMT cores."""
     return _quantize("jl_quantize_keys_simt", K, S, signs, norms, stream)
+
+
+def jl_dequantize_keys(signs, norms, S, out=None, stream=None):
+    """khat = sqrt(pi/2)/m * ||k|| * S^T z for each code: [n, d] bf16."""
+    L = load()
+    m, d = S.shape
+    _need_cuda(signs, norms, S, out)
+    assert signs.dtype == torch.int32 and signs.shape[-1] == m // 32
+    assert norms.dtype == torch.float16 and S.dtype == torch.bfloat16
+    signs2 = signs.reshape(-1, m // 32)
+    n = signs2.shape[0]
+    assert norms.numel() == n
+    for t in (signs2, norms, S):
+        if not t.is_contiguous():
+            raise ValueError("dequantize inputs must be contiguous")
+    if out is None:
+        out = torch.empty((n, d), dtype=torch.bfloat16, device=signs.device)
+    assert out.dtype == torch.bfloat16 and out.numel() == n * d and out.is_contiguous()
+    _check(L.jl_dequantize_keys(_ptr(signs2), _ptr(norms), n, _ptr(S), m, d, _ptr(out),
+                                _stream(signs, stream)), "jl_dequantize_keys")
+    return out
 
 
 def jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int:

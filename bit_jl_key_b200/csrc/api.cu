@@ -161,6 +161,19 @@ int jl_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
                                              (cudaStream_t)stream));
 }
 
+int jl_dequantize_keys(const uint32_t *signs, const uint16_t *norms, int64_t n_keys,
+                       const uint16_t *S, int m, int d, uint16_t *out, jl_stream_t stream) {
+  if (n_keys < 0) return JL_ERR_INVALID_ARG;
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (n_keys == 0) return JL_OK;
+  if (!signs || !norms || !S || !out) return JL_ERR_INVALID_ARG;
+  if (!aligned(signs, 16) || !aligned(norms, 2) || !aligned(S, 16) || !aligned(out, 16))
+    return JL_ERR_INVALID_ARG;
+  if (n_keys >= ((int64_t)1 << 40)) return JL_ERR_UNSUPPORTED;
+  return from_cuda(jlk::launch_dequantize_tc(signs, norms, n_keys, S, m, d, out,
+                                             (cudaStream_t)stream));
+}
+
 size_t jl_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m,
                                  int d) {
   jlk::DecodePlan p;

@@ -27,6 +27,11 @@ cudaError_t launch_quantize_tc(const uint16_t *K, int64_t n, int64_t ldk,
                                cudaStream_t stream);
 bool quantize_tc_supported(int m, int d, int64_t n, int64_t ldk, const void *K);
 
+// Tensor-core dequantizer khat = sqrt(pi/2)/m * ||k|| * S^T z (bf16 out).
+cudaError_t launch_dequantize_tc(const uint32_t *signs, const uint16_t *norms, int64_t n,
+                                 const uint16_t *S, int m, int d, uint16_t *out,
+                                 cudaStream_t stream);
+
 // Decode: work split shared by the workspace query and the launch.
 struct DecodePlan {
   int B, Hq, Hkv, m, d;

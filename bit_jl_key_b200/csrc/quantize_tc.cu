@@ -136,6 +136,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
+// The same wait, tied to the registers of one load: code that reads v after
+// it cannot be moved above it.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
+                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
+                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+// Code word of 32 accumulator columns: bit j = 1 iff column j is >= 0
+// (sign bit clear).  One funnel shift per column moves its sign bit in; four
+// independent chains of 8 (one per byte) keep the dependency chain short.
+__device__ __forceinline__ uint32_t pack_signs(const uint32_t (&v)[32]) {
+  uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+  for (int jj = 7; jj >= 0; --jj) {
+    c0 = __funnelshift_l(v[jj], c0, 1);
+    c1 = __funnelshift_l(v[8 + jj], c1, 1);
+    c2 = __funnelshift_l(v[16 + jj], c2, 1);
+    c3 = __funnelshift_l(v[24 + jj], c3, 1);
+  }
+  return ~(c0 | (c1 << 8) | (c2 << 16) | (c3 << 24));
+}
 
 // Bounded wait on a barrier phase; false when the wait ran out or another
 // role gave up (then the error word is set and the shared abort flag raised).
@@ -311,29 +338,34 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
         __syncwarp();
         tc_fence_after();
         const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * C::NMMA);
-        uint32_t *dst = p.signs + row * C::WORDS + h * C::WORDS_ITEM;
-        // GW words (32 columns each) per step bound the live TMEM slices
-#pragma unroll 1
-        for (int w0 = k * WPW; w0 < (k + 1) * WPW; w0 += GW) {
-          uint32_t words[GW];
+        uint32_t *dst = p.signs + row * C::WORDS + h * C::WORDS_ITEM + k * WPW;
+        // this warp's WPW code words; the TMEM loads are double-buffered so
+        // that the load of word w + 1 is in flight while word w is packed
+        uint32_t words[WPW];
+        uint32_t va[32], vb[32];
+        const uint32_t tcol = trow + 32 * (k * WPW);
+        tmem_ld32(tcol, va);
 #pragma unroll
-          for (int w = 0; w < GW; ++w) {
-            uint32_t v[32];
-            tmem_ld32(trow + 32 * (w0 + w), v);
-            tmem_ld_wait();
-            uint32_t word = 0;
-#pragma unroll
-            for (int jj = 31; jj >= 0; --jj) word = __funnelshift_l(v[jj], word, 1);
-            words[w] = ~word;  // bit jj = 1 iff that column is >= 0
+        for (int w = 0; w < WPW; w += 2) {
+          tmem_ld_wait(va);
+          if (w + 1 < WPW) tmem_ld32(tcol + 32 * (w + 1), vb);
+          words[w] = pack_signs(va);
+          if (w + 1 < WPW) {
+            tmem_ld_wait(vb);
+            if (w + 2 < WPW) tmem_ld32(tcol + 32 * (w + 2), va);
+            words[w + 1] = pack_signs(vb);
           }
-          if (live) {
+        }
+        if (live) {
+#pragma unroll
+          for (int w = 0; w < WPW; w += GW) {
             if constexpr (GW == 1)
-              dst[w0] = words[0];
+              dst[w] = words[w];
             else if constexpr (GW == 2)
-              *reinterpret_cast<uint2 *>(dst + w0) = make_uint2(words[0], words[1]);
+              *reinterpret_cast<uint2 *>(dst + w) = make_uint2(words[w], words[w + 1]);
             else
-              *reinterpret_cast<uint4 *>(dst + w0) =
-                  make_uint4(words[0], words[1], words[2], words[3]);
+              *reinterpret_cast<uint4 *>(dst + w) =
+                  make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
           }
         }
         tc_fence_before();

@@ -166,6 +166,28 @@ JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *
                         jl_stream_t stream);
 
 /*
+ * jl_dequantize_keys -- explicit dequantizer of the codes.
+ * Defines: Q^-1(z) = sqrt(pi/2)/d * S^T z ("The Geometry of Forgetting: How
+ * Three Papers Cracked KV Cache Quantization", section "QJL: one bit, zero
+ * parameters, unbiased inner products"), taken with m sketch rows and with
+ * the stored norm restoring the magnitude ("PolarQuant" section):
+ *     khat_t = sqrt(pi/2)/m * ||k_t|| * S^T z_t,   z_ti = +1 if bit i is set,
+ * so that <q, khat_t> is the asymmetric estimator and E||k - khat||^2 is the
+ * page's D_mse, ||k||^2 ((pi/2) d - 1) / m for a Gaussian S.
+ *   signs  : in, n_keys x (m/32) uint32 codes (jl_quantize_keys layout),
+ *            16-byte aligned.
+ *   norms  : in, n_keys binary16 norms.
+ *   S      : in, m x d bf16 sketch, 16-byte aligned.
+ *   out    : out, n_keys x d bf16 (round to nearest), 16-byte aligned.
+ * Computed on the tensor cores with fp32 accumulation.  n_keys == 0 is a
+ * no-op.  Errors: JL_ERR_INVALID_ARG (null or misaligned pointer, n_keys < 0),
+ * JL_ERR_UNSUPPORTED (m, d), JL_ERR_CUDA.
+ */
+JL_API int jl_dequantize_keys(const uint32_t *signs, const uint16_t *norms, int64_t n_keys,
+                              const uint16_t *S, int m, int d, uint16_t *out,
+                              jl_stream_t stream);
+
+/*
  * jl_decode_paged_workspace_bytes -- device scratch jl_decode_attention_paged
  * needs (query projections and split partial states) for B sequences of at
  * most max_len keys each (counting the key a call appends).  Depends on the

@@ -191,3 +191,22 @@ def test_paged_decode_argument_errors(lib):
     assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
     # without a new key, the key dtype is not looked at
     assert call(Kn=NULL, Vn=NULL, kt=9, ws=NULL) == jl.JL_ERR_WORKSPACE
+
+
+def test_dequantize_argument_errors(lib):
+    f = lib.jl_dequantize_keys
+    ok = dict(signs=FAKE, norms=FAKE, n=10, S=FAKE, m=256, d=128, out=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["signs"], a["norms"], a["n"], a["S"], a["m"], a["d"], a["out"], NULL)
+
+    assert call(n=0) == jl.JL_OK
+    assert call(n=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(m=96) == jl.JL_ERR_UNSUPPORTED
+    assert call(d=32) == jl.JL_ERR_UNSUPPORTED
+    for k in ("signs", "norms", "S", "out"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(signs=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(out=ctypes.c_void_p((1 << 20) + 8)) == jl.JL_ERR_INVALID_ARG
+    assert call(norms=ctypes.c_void_p((1 << 20) + 1)) == jl.JL_ERR_INVALID_ARG

@@ -23,6 +23,8 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
            [16384, 32767) plus the appended key (bound 32768); pages of 64
            tokens assigned in a shuffled order; cache contents drawn as for
            gqa.
+  dequant-gqa  the gqa cache's 2,097,152 codes (m=256) and norms turned back
+           into bf16 keys of d=128 (codes made from gqa's keys).
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -90,7 +92,10 @@ PAGED_GQA = Workload("paged-gqa", 6, 8, 32, 8, 32768, 128, 256, torch.bfloat16,
                      outliers=4)
 PAGE_TOKENS = 64
 
-ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA)}
+# dequant-gqa: the codes of the gqa cache turned back into bf16 keys
+DEQUANT_GQA = GQA.with_(name="dequant-gqa")
+
+ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA)}
 
 
 def sweep_points():
