@@ -216,6 +216,25 @@ def dequantize(signs, norms, S) -> np.ndarray:
     return out
 
 
+def search_topk(Q, S, signs, norms, k: int):
+    """Inner-product search over a QJL-compressed index: for each query q,
+    the k index vectors with the largest estimated <q, x> (the asymmetric
+    estimator, as in decode), best first; ties go to the lower index.
+
+    Q [nq, d]; signs [N, m/32]; norms [N] (float64 values of the stored
+    norms).  Returns (idx int64 [nq, k], scores float64 [nq, k], all scores
+    float64 [nq, N]).  The ordering step is a library sort.
+    """
+    Q = _c(Q, np.float64)
+    U = project(Q, S)
+    N = signs.shape[0]
+    allsc = np.stack([scores(U[i], signs, norms) for i in range(U.shape[0])])
+    # descending by score, ascending by index among equal scores
+    order = np.lexsort((np.broadcast_to(np.arange(N), allsc.shape), -allsc), axis=-1)
+    idx = order[:, :k]
+    return idx, np.take_along_axis(allsc, idx, axis=1), allsc
+
+
 def decode(Q, S, signs, norms, V, softmax_scale: float, want_scores=False):
     """Decode attention over compressed keys.
 

@@ -429,3 +429,38 @@ def test_reconstruction_mse_closed_form(m):
     sem = err.std(ddof=1) / math.sqrt(R)
     assert abs(err.mean() - pred) < 5 * sem
     assert err.mean() == pytest.approx(pred, rel=0.08)
+
+
+# --------------------------------------------------------------------------
+# inner-product search over a compressed index (the final section of "The
+# Geometry of Forgetting ...": the same quantizer for any store of vectors
+# read through inner products)
+
+def test_search_topk_brute_force_tiny():
+    rng = np.random.default_rng(70)
+    d, m, N, nq, k = 8, 32, 40, 5, 6
+    S = rng.standard_normal((m, d))
+    X = rng.standard_normal((N, d))
+    X[7] = X[3]                                   # an exact tie
+    Q = rng.standard_normal((nq, d))
+    signs, norms, _, _ = oracle.quantize(X, S)
+    idx, sc, _ = oracle.search_topk(Q, S, signs, norms, k)
+    for i in range(nq):
+        est = [oracle.estimate(Q[i], X[j], S) for j in range(N)]
+        want = sorted(range(N), key=lambda j: (-est[j], j))[:k]
+        assert list(idx[i]) == want
+        assert np.allclose(sc[i], [est[j] for j in want], rtol=1e-12)
+
+
+def test_search_recovers_exact_top1_with_many_rows():
+    # the estimator concentrates as m grows, so the estimated best match of a
+    # planted near-duplicate is the exact best match
+    rng = np.random.default_rng(71)
+    d, N = 32, 300
+    X = rng.standard_normal((N, d))
+    Q = X[[11, 200, 57]] * 1.0 + 0.05 * rng.standard_normal((3, d))
+    exact = np.argmax(Q @ X.T, axis=1)
+    S = rng.standard_normal((4096, d))
+    signs, norms, _, _ = oracle.quantize(X, S)
+    idx, _, _ = oracle.search_topk(Q, S, signs, norms, 1)
+    assert list(idx[:, 0]) == list(exact)
