@@ -1,7 +1,7 @@
 """Benchmark: QJL key quantization + compressed-key decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -16,6 +16,10 @@ jl_decode_attention_paged call that appends every sequence's new key and
 value to a shuffled page pool and attends over its ragged context (the cache
 is filled once, untimed; the lengths stay fixed from step to step, so every
 step rewrites the same slots).
+
+The search workload times one jl_search_topk call: the top-10 index vectors
+of each of 128 queries over 8,388,608 compressed vectors (scores on the
+tensor cores; the roofline is the tensor peak).
 
 The dequant-gqa workload times the explicit dequantizer: one
 jl_dequantize_keys call turning the gqa cache's codes and norms back into
@@ -63,6 +67,9 @@ FALLBACK_HBM_GBS = 6650.0
 # --------------------------------------------------------------------------
 # helpers
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -70,6 +77,17 @@ def load_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_tensor_peak():
+    """Dense bf16 tensor peak (burst figure: the kernel is timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured bf16_tflops (fp16 runs at the bf16 rate)"
+    return FALLBACK_BF16_TFLOPS, "fallback bf16 TFLOP/s"
 
 
 def pick_workload(name: str, batch: int = 0) -> workloads.Workload:
@@ -455,9 +473,111 @@ def run_dequant(args, rank, world, local_rank):
     }
 
 
+def run_search(args, rank, world, local_rank):
+    """Top-k inner-product search over a compressed index."""
+    import bit_jl_key_b200 as jl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload, args.batch)
+    k = workloads.SEARCH_K
+    hbm_peak, _ = load_peaks()
+    tpeak, tkind = load_tensor_peak()
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)                                    # index vectors, untimed
+    signs, norms = jl.jl_quantize_keys(K.view(-1, w.d), S)
+    del K
+    torch.cuda.empty_cache()
+    Q = workloads.queries(w, dev).view(-1, w.d)
+    N, nq = signs.shape[0], Q.shape[0]
+    ws = torch.empty((jl.jl_search_workspace_bytes(nq, w.m, w.d, k),), dtype=torch.uint8,
+                     device=dev)
+    oi = torch.empty((nq, k), dtype=torch.int32, device=dev)
+    osc = torch.empty((nq, k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        jl.jl_search_topk(Q, S, signs, norms, k, out_index=oi, out_scores=osc, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        _barrier(world, dev)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        _barrier(world, dev)
+    ms = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    e2e = None
+    if not args.no_e2e:
+        # the queries from pinned host memory, the top-k lists back to it
+        hQ = Q.cpu().pin_memory()
+        hI = torch.empty(oi.shape, dtype=oi.dtype).pin_memory()
+        hS = torch.empty(osc.shape, dtype=osc.dtype).pin_memory()
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            step()
+            hI.copy_(oi, non_blocking=True)
+            hS.copy_(osc, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        _barrier(world, dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        _barrier(world, dev)
+        e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        e2e = {"value": whole_job_rate(N * nq, world, e_ms), "unit": "query-vector pairs/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": hQ.numel() * hQ.element_size(),
+               "d2h_bytes_per_step": hI.numel() * 4 + hS.numel() * 4}
+
+    flops = 2.0 * w.m * N * nq                 # the estimator's m multiply-adds per pair
+    tflops = flops / (ms * 1e-3) / 1e12
+    nbytes = N * (w.m // 8 + 2)
+    return {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": whole_job_rate(N * nq, world, ms), "unit": "query-vector pairs/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: {nq} queries x {N} vectors, d={w.d}, m={w.m}, "
+                               f"top-{k}",
+                   "global_batch": nq * world, "seq_len": N, "parallelism": f"dp{world}",
+                   "l2": "index (285 MB of codes and norms) exceeds L2; no flush"},
+        "phases": {"search": {"ms": ms, "pairs_per_s": N * nq / (ms * 1e-3),
+                              "tflops": tflops, "frac_of_tensor_peak": tflops / tpeak,
+                              "index_bytes": nbytes,
+                              "index_GB_per_s": nbytes / (ms * 1e-3) / 1e9,
+                              "frac_of_hbm_peak": nbytes / (ms * 1e-3) / 1e9 / hbm_peak}},
+        "roofline": {"kernel": "jl_search_topk", "bound": "tensor", "achieved": tflops,
+                     "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s",
+                     "frac": tflops / tpeak, "algorithmic_flops_per_launch": flops,
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
+    if args.workload == "search":
+        return run_search(args, rank, world, local_rank)
     if args.workload == "paged-gqa":
         return run_paged(args, rank, world, local_rank)
     if args.workload == "dequant-gqa":
@@ -659,6 +779,17 @@ def oracle_sample(w: workloads.Workload):
     import oracle
 
     S64 = oracle.sketch(w.m, w.d, w.sketch_seed)
+    if w.name == "search":
+        n, nq = 262144, 4
+        X = workloads.keys(w.with_(T=n)).view(-1, w.d).double().numpy()
+        sig, _, n16, _ = oracle.quantize(X, S64)            # set-up, untimed
+        n64 = oracle.fp16_bits_to_f64(n16)
+        Qs = workloads.queries(w).view(-1, w.d)[:nq].double().numpy()
+
+        def run():
+            oracle.search_topk(Qs, S64, sig, n64, workloads.SEARCH_K)
+        return run, n * nq, (f"{nq} queries x the first {n} index vectors of the workload's "
+                             f"recipe (scores + top-{workloads.SEARCH_K})")
     if w.name == "dequant-gqa":
         n = 16384
         Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()
@@ -690,6 +821,10 @@ def oracle_sample(w: workloads.Workload):
                     f"quantize + decode in float64")
 
 
+def unit_of(w) -> str:
+    return "query-vector pairs/s" if w.name == "search" else "keys/s"
+
+
 def time_oracle(w, steps=1, warmup=0):
     import oracle
     run, keys, desc = oracle_sample(w)
@@ -699,7 +834,7 @@ def time_oracle(w, steps=1, warmup=0):
     for _ in range(steps):
         run()
     dt = (time.perf_counter() - t) / steps
-    return {"value": keys / dt, "unit": "keys/s", "cores": oracle.max_threads(),
+    return {"value": keys / dt, "unit": unit_of(w), "cores": oracle.max_threads(),
             "kind": "oracle", "sample": desc, "s_per_step": dt}
 
 
@@ -711,7 +846,7 @@ def run_reference(args, rank, world):
     return {
         "impl": "reference",
         "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
-        "value": cb["value"], "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "value": cb["value"], "unit": unit_of(w), "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": cb["s_per_step"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded, workloads.py)",
@@ -720,7 +855,7 @@ def run_reference(args, rank, world):
                    "global_batch": w.B * world, "seq_len": w.T,
                    "parallelism": f"dp{world}"},
         "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
-        "e2e": {"value": cb["value"], "unit": "keys/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": cb["value"], "unit": unit_of(w), "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 

@@ -47,7 +47,8 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_quantize_keys_simt", "jl_decode_workspace_bytes",
             "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64",
             "jl_decode_attention_noalloc", "jl_decode_paged_workspace_bytes",
-            "jl_decode_attention_paged", "jl_dequantize_keys")
+            "jl_decode_attention_paged", "jl_dequantize_keys", "jl_search_workspace_bytes",
+            "jl_search_topk")
 
 _lib = None
 
@@ -87,6 +88,11 @@ def load():
     L.jl_decode_attention_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32,
                                               i32, i64, i32, i32, ctypes.c_float,
                                               vp, vp, vp]
+    L.jl_search_workspace_bytes.restype = sz
+    L.jl_search_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.jl_search_topk.restype = i32
+    L.jl_search_topk.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp, i64, i32, vp, vp, vp, sz,
+                                 vp]
     L.jl_dequantize_keys.restype = i32
     L.jl_dequantize_keys.argtypes = [vp, vp, i64, vp, i32, i32, vp, vp]
     L.jl_decode_paged_workspace_bytes.restype = sz
@@ -201,6 +207,40 @@ def jl_dequantize_keys(signs, norms, S, out=None, stream=None):
     _check(L.jl_dequantize_keys(_ptr(signs2), _ptr(norms), n, _ptr(S), m, d, _ptr(out),
                                 _stream(signs, stream)), "jl_dequantize_keys")
     return out
+
+
+def jl_search_workspace_bytes(n_queries, m, d, k) -> int:
+    return int(load().jl_search_workspace_bytes(n_queries, m, d, k))
+
+
+def jl_search_topk(Q, S, signs, norms, k, out_index=None, out_scores=None, workspace=None,
+                   stream=None):
+    """Top-k inner-product search of the queries Q [nq, d] over the index
+    (signs [N, m/32] int32, norms [N] fp16).  Returns (index int32 [nq, k],
+    scores fp32 [nq, k]), best first."""
+    L = load()
+    m, d = S.shape
+    nq = Q.shape[0]
+    _need_cuda(Q, S, signs, norms)
+    assert Q.dim() == 2 and Q.shape[1] == d
+    assert signs.dtype == torch.int32 and signs.shape[1] == m // 32
+    assert norms.dtype == torch.float16 and norms.numel() == signs.shape[0]
+    for t in (Q, S, signs, norms):
+        if not t.is_contiguous():
+            raise ValueError("search inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    if out_index is None:
+        out_index = torch.empty((nq, k), dtype=torch.int32, device=Q.device)
+    if out_scores is None:
+        out_scores = torch.empty((nq, k), dtype=torch.float32, device=Q.device)
+    need = jl_search_workspace_bytes(nq, m, d, k)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_search_topk(_ptr(Q), qt, nq, _ptr(S), m, d, _ptr(signs), _ptr(norms),
+                            signs.shape[0], k, _ptr(out_index), _ptr(out_scores),
+                            _ptr(workspace), workspace.numel(), _stream(Q, stream)),
+           "jl_search_topk")
+    return out_index, out_scores
 
 
 def jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int:

@@ -174,6 +174,32 @@ int jl_dequantize_keys(const uint32_t *signs, const uint16_t *norms, int64_t n_k
                                              (cudaStream_t)stream));
 }
 
+size_t jl_search_workspace_bytes(int n_queries, int m, int d, int k) {
+  if (n_queries < 0 || k < 1 || k > JL_SEARCH_MAX_K || !supported_md(m, d)) return 0;
+  return jlk::search_workspace_bytes(n_queries, m, k);
+}
+
+int jl_search_topk(const void *Q, jl_dtype q_dtype, int n_queries, const uint16_t *S, int m,
+                   int d, const uint32_t *signs, const uint16_t *norms, int64_t n_index, int k,
+                   int32_t *out_index, float *out_scores, void *workspace,
+                   size_t workspace_bytes, jl_stream_t stream) {
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (n_queries < 0 || n_index < 1 || k < 1 || k > JL_SEARCH_MAX_K) return JL_ERR_INVALID_ARG;
+  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
+  if (n_index >= ((int64_t)1 << 31)) return JL_ERR_UNSUPPORTED;
+  if (n_queries == 0) return JL_OK;
+  if (!Q || !S || !signs || !norms || !out_index || !out_scores) return JL_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(S, 16) || !aligned(signs, 16) || !aligned(norms, 2) ||
+      !aligned(out_index, 4) || !aligned(out_scores, 4))
+    return JL_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) ||
+      workspace_bytes < jlk::search_workspace_bytes(n_queries, m, k))
+    return JL_ERR_WORKSPACE;
+  return from_cuda(jlk::launch_search(Q, q_dtype == JL_F32, n_queries, S, m, d, signs, norms,
+                                      n_index, k, out_index, out_scores, workspace,
+                                      (cudaStream_t)stream));
+}
+
 size_t jl_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m,
                                  int d) {
   jlk::DecodePlan p;

@@ -1349,6 +1349,24 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
 }
 
+cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S, float *U,
+                                    int nq, int m, int d, cudaStream_t stream) {
+  if (nq <= 0) return cudaSuccess;
+  const int ctas = (nq + PROJ_VECS - 1) / PROJ_VECS;
+#define JL_CASE(MM, DD)                                                              \
+  if (m == MM && d == DD) {                                                          \
+    if (q_f32)                                                                       \
+      qproj_kernel<MM, DD, true><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq);    \
+    else                                                                             \
+      qproj_kernel<MM, DD, false><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq);   \
+    return cudaGetLastError();                                                       \
+  }
+  JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
+  JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
+#undef JL_CASE
+  return cudaErrorNotSupported;
+}
+
 cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,
                           const uint16_t *norms, const uint16_t *V,

@@ -32,6 +32,17 @@ cudaError_t launch_dequantize_tc(const uint32_t *signs, const uint16_t *norms, i
                                  const uint16_t *S, int m, int d, uint16_t *out,
                                  cudaStream_t stream);
 
+// u = S q for nq queries (fp32 [nq][m]).
+cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S, float *U,
+                                    int nq, int m, int d, cudaStream_t stream);
+
+// Inner-product top-k search over a compressed index (search_tc.cu).
+size_t search_workspace_bytes(int nq, int m, int k);
+cudaError_t launch_search(const void *Q, bool q_f32, int nq, const uint16_t *S, int m, int d,
+                          const uint32_t *signs, const uint16_t *norms, int64_t N, int k,
+                          int32_t *out_idx, float *out_scores, void *workspace,
+                          cudaStream_t stream);
+
 // Decode: work split shared by the workspace query and the launch.
 struct DecodePlan {
   int B, Hq, Hkv, m, d;

@@ -1,0 +1,761 @@
+// search_tc.cu -- inner-product top-k search over a QJL-compressed index.
+//
+// "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+// Quantization", final section: the quantizer serves any store of
+// high-dimensional vectors that is read through inner products (vector
+// databases, retrieval, recommendation).  Here each index vector x is kept as
+// its QJL code z = sign(S x) and norm, and a query q is scored against every
+// vector with the asymmetric estimator of the QJL section,
+//     s(q, x) = sqrt(pi/2)/m * ||x|| * <S q, z>,
+// keeping the k best vectors per query.
+//
+// One pass handles up to 128 queries.  For a tile of 256 index vectors the
+// scores form a dense contraction D[128 queries][256 vectors] = U Z^T
+// (M = 128, N = 256, K = m) on the tensor cores:
+//   * U = S q (projected by the query-projection kernel) is rounded to fp16
+//     with a power-of-two scale per query (relative error <= 2^-11 per
+//     coordinate) and written once into tensor memory as the A operand;
+//   * the B operand is Z scaled by each vector's norm, +-||x|| in fp16 (the
+//     norms are stored in binary16, and a product with the fp16 U is exact
+//     in fp32), expanded from the code bits into shared memory one K-chunk of
+//     64 coordinates (32 KB) at a time: an fp16 pair holds coordinates
+//     (p, p + 16) of a code word, ((w << (15 - p)) & 0x80008000) ^
+//     (0x80008000 | ||x|| ||x||), and U's columns use the same order;
+//   * the accumulator (256 fp32 columns) sits in tensor memory beside U.
+// Each epilogue lane owns one query and keeps its best KT scores (before the
+// query's positive output scale) in registers.  Per 32 columns the hot path
+// is the group maximum and one comparison with the list's bound: the larger
+// of the list's own KT-th best and the best KT-th best any list of the query
+// has published so far (a lower bound on the final KT-th best, shared
+// through an atomic maximum in global memory).  Only a lane whose group
+// passes parks its 32 scores in a private row of shared memory and inserts
+// the qualifying ones.  A second kernel merges the lists of each query.
+// Before the full pass, the same kernel scores the queries against a spread
+// sample of the index tiles, and the merge kernel turns each query's 16th
+// best sample score into its starting bound (a valid lower bound on the
+// final 16th best: the sample is part of the index), so that very few scores
+// of the full pass reach the insertion path.
+//
+// One persistent CTA per SM, 9 warps with fixed roles:
+//   warps 0-3  expand: thread t owns rows t and t + 128 of every tile.
+//   warps 4-7  U into tensor memory first, then the epilogue: lane quadrant
+//              warp % 4 = queries 32 (warp % 4) .. + 31, one list per query.
+//   warp 8     owns the TMEM allocation; lane 0 issues the MMAs.
+// Every mbarrier wait is bounded; a wait that runs out records
+// DERR_TC_WAIT_TIMEOUT and the CTA still frees its TMEM.
+#include "jl_common.cuh"
+#include "jl_internal.h"
+
+#include <math.h>
+
+namespace jlk {
+namespace srch {
+
+constexpr int QM = 128;                        // queries per pass (MMA M)
+constexpr int BN = 256;                        // index vectors per tile (MMA N)
+constexpr int CHUNK_K = 64;                    // coordinates per Z chunk
+constexpr int CHUNK_BYTES = BN * CHUNK_K * 2;  // 32 KB
+constexpr int EXP_WARPS = 4, EPI_WARPS = 4;
+constexpr int LISTS = 1;                       // lists per query and CTA
+constexpr int PARK_ROWS = 4;                   // groups a lane can park per tile
+constexpr int MMA_WARP = EXP_WARPS + EPI_WARPS;
+constexpr int THREADS = (MMA_WARP + 1) * 32;
+constexpr int CODE_SLOTS = 3;
+constexpr int TMEM_COLS = 512;
+constexpr int MAX_CTAS = 256;                  // bounds the per-CTA lists
+constexpr int MERGE_THREADS = 256;
+constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
+
+template <int M>
+struct Cfg {
+  static constexpr int KCH = M / CHUNK_K;
+  static constexpr int U_COLS = M / 2;         // fp16 pairs
+  static constexpr int D_COL = U_COLS;         // accumulator columns [D_COL, D_COL + 256)
+  static constexpr int RING = M > 256 ? 3 : 4;
+  static constexpr int CODE_ROW = M / 8;
+  static constexpr int CODE_WORDS = M / 32;
+  static constexpr int OFF_Z = 0;
+  static constexpr int OFF_C = OFF_Z + RING * CHUNK_BYTES;
+  // per epilogue lane: PARK_ROWS rows of 33 floats (parked groups)
+  static constexpr int OFF_P = OFF_C + CODE_SLOTS * BN * CODE_ROW;
+  static constexpr int OFF_BAR = OFF_P + EPI_WARPS * 32 * PARK_ROWS * 33 * 4;
+  static constexpr int NBAR = 2 * RING + 2;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static_assert(D_COL + BN <= TMEM_COLS, "tensor memory columns");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct Params {
+  const uint32_t *signs;   // N x m/32
+  const uint16_t *norms;   // N binary16
+  const float *U;          // QM x m (rows >= nq ignored)
+  float *part_val;         // [MAX_CTAS][LISTS][QM][KT]
+  int32_t *part_idx;
+  unsigned *gbound;        // [QM] order-preserving codes of the shared bounds (0 = none)
+  float *qscale;           // [QM] output scale of each query's scores
+  int64_t N;
+  int64_t num_tiles;       // tiles of this launch: tile0 + j * tile_step, j < num_tiles
+  int64_t tile0, tile_step;
+  int nq;
+  float coef;              // sqrt(pi/2) / m
+  int *err;
+};
+
+// --------------------------------------------------------------------------
+// PTX wrappers
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+// D (tensor memory) += A (tensor memory) * B (shared memory), fp16 inputs
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+        "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+        "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
+                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
+                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+      "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+      "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
+                                           volatile int *abort_flag, int *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > WAIT_NS) {
+        *abort_flag = 1;
+        record_device_error(err, DERR_TC_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Copy code rows `row0` and `row0 + 128` (M/8 bytes each) into shared memory
+// with cp.async, zero fill past the end, as one commit group.
+template <int M>
+__device__ __forceinline__ void copy_code_rows(uint32_t dst0, uint32_t dst1, const uint32_t *signs,
+                                               int64_t row0, int64_t N) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t row = row0 + 128 * h;
+    const bool live = row < N;
+    const uint32_t dst = h ? dst1 : dst0;
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(signs + (live ? row : 0) * (M / 32));
+    if constexpr (M >= 128) {
+#pragma unroll
+      for (int q = 0; q < M / 128; ++q) cp_async_16(dst + 16 * q, src + 16 * q, live ? 16 : 0);
+    } else {
+      cp_async_8(dst, src, live ? 8 : 0);
+    }
+  }
+  cp_async_commit();
+}
+
+// Expand two 32-bit code words into one 128-byte row of a B chunk (fp16
+// +-||x||, pair j of word h at 16-byte unit 4 h + j / 4), swizzled by
+// (row & 7); x = 0x80008000 | the norm's bits in both halves.
+__device__ __forceinline__ void expand_row(uint8_t *chunk, int r, uint32_t w0, uint32_t w1,
+                                           uint32_t x) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t w = half ? w1 : w0;
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4) {
+      uint32_t q[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * u4 + e;
+        q[e] = ((w << (15 - j)) & 0x80008000u) ^ x;
+      }
+      const int unit = 4 * half + u4;
+      *reinterpret_cast<uint4 *>(chunk + r * 128 + ((unit ^ (r & 7)) << 4)) =
+          make_uint4(q[0], q[1], q[2], q[3]);
+    }
+  }
+}
+
+// Order-preserving code of a float (larger float <-> larger code; never 0 for
+// a number), and back.
+__device__ __forceinline__ unsigned ord_code(float f) {
+  const unsigned b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord_float(unsigned c) {
+  if (c == 0u) return -INFINITY;
+  return __uint_as_float((c & 0x80000000u) ? (c & 0x7FFFFFFFu) : ~c);
+}
+
+// A query's list of its KT best (score, index): filled in order, then the
+// minimum is replaced.  All indexing is static so the list stays in registers.
+template <int KT>
+struct TopList {
+  float val[KT];
+  int32_t idx[KT];
+  int cnt;
+  float thr;  // the smallest kept score once the list is full, else -inf
+
+  __device__ __forceinline__ void init() {
+    cnt = 0;
+    thr = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < KT; ++e) {
+      val[e] = -INFINITY;
+      idx[e] = -1;
+    }
+  }
+  __device__ __forceinline__ float min_val() const {
+    float mv = val[0];
+#pragma unroll
+    for (int e = 1; e < KT; ++e) mv = fminf(mv, val[e]);
+    return mv;
+  }
+  __device__ __forceinline__ void insert(float s, int32_t i) {
+    if (cnt < KT) {
+#pragma unroll
+      for (int e = 0; e < KT; ++e)
+        if (e == cnt) {
+          val[e] = s;
+          idx[e] = i;
+        }
+      if (++cnt == KT) thr = min_val();
+    } else {
+      bool done = false;
+#pragma unroll
+      for (int e = 0; e < KT; ++e)
+        if (!done && val[e] == thr) {
+          val[e] = s;
+          idx[e] = i;
+          done = true;
+        }
+      thr = min_val();
+    }
+  }
+};
+
+// --------------------------------------------------------------------------
+template <int M, int KT>
+__global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
+  using C = Cfg<M>;
+  extern __shared__ uint8_t sr_smem_raw[];
+  const uint32_t raw = smem_u32(sr_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = sr_smem_raw + (base - raw);
+  const uint32_t sZ = base + C::OFF_Z;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  auto zfull_bar = [&](int s) { return bar0 + 8u * s; };
+  auto zempty_bar = [&](int s) { return bar0 + 8u * (C::RING + s); };
+  const uint32_t dfull_bar = bar0 + 8u * (2 * C::RING);
+  const uint32_t dempty_bar = bar0 + 8u * (2 * C::RING + 1);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+  volatile int *abort_flag =
+      reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::RING; ++s) {
+      mbar_init(zfull_bar(s), EXP_WARPS);
+      mbar_init(zempty_bar(s), 1);
+    }
+    mbar_init(dfull_bar, 1);
+    mbar_init(dempty_bar, EPI_WARPS);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == MMA_WARP) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+        "tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::"r"(
+            smem_u32(tmem_holder)),
+        "n"(TMEM_COLS)
+        : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // ---- U into tensor memory (warps 4-7, lane quadrant warp % 4): fp16 pairs
+  // (u_{32b+j}, u_{32b+j+16}) at column 16 b + j, scaled by 2^e per query
+  if (warp >= EXP_WARPS && warp < MMA_WARP) {
+    const int q = warp & 3;
+    const int qi = 32 * q + lane;
+    const bool valid = qi < p.nq;
+    const float *urow = p.U + (int64_t)(valid ? qi : 0) * M;
+    float mx = 0.f;
+    if (valid)
+      for (int i = 0; i < M; ++i) mx = fmaxf(mx, fabsf(urow[i]));
+    int ex = 0;
+    if (mx > 0.f) frexpf(mx, &ex);          // mx = f 2^ex, f in [0.5, 1)
+    const float scale = ldexpf(1.f, 15 - ex);  // max |u| scale in [2^14, 2^15)
+    // output scale of the query's scores: sqrt(pi/2)/m * 2^-e
+    if (blockIdx.x == 0) p.qscale[qi] = p.coef * ldexpf(1.f, ex - 15);
+#pragma unroll 1
+    for (int c0 = 0; c0 < C::U_COLS; c0 += 32) {
+      uint32_t v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = c0 + e, b = c >> 4, j = c & 15;
+        const float lo = valid ? urow[32 * b + j] * scale : 0.f;
+        const float hi = valid ? urow[32 * b + j + 16] * scale : 0.f;
+        __half2 h = __floats2half2_rn(lo, hi);
+        v[e] = *reinterpret_cast<uint32_t *>(&h);
+      }
+      tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int64_t ntiles = p.num_tiles;
+  auto tile_at = [&](int64_t j) { return p.tile0 + j * p.tile_step; };  // rows past N: zero codes
+  if (warp < EXP_WARPS) {
+    // ---------------- expand: rows t and t + 128 of every tile
+    const int t = threadIdx.x;
+    const uint32_t crow0 = base + C::OFF_C + t * C::CODE_ROW;
+    auto slot0 = [&](int64_t it) { return crow0 + (uint32_t)((it % CODE_SLOTS) * BN * C::CODE_ROW); };
+    for (int k = 0; k < CODE_SLOTS - 1; ++k) {
+      const int64_t row0 = tile_at((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BN + t;
+      copy_code_rows<M>(slot0(k), slot0(k) + 128 * C::CODE_ROW, p.signs, row0, p.N);
+    }
+    int64_t c = 0, it = 0;
+    bool ok = true;
+    // the two rows' norms (0 past the end), one tile ahead: B holds +-||x||
+    auto norm_of = [&](int64_t row) -> uint32_t {
+      return row < p.N ? (uint32_t)__ldg(p.norms + row) & 0x7FFFu : 0u;
+    };
+    uint32_t n0 = norm_of(tile_at(blockIdx.x) * BN + t), n1 = norm_of(tile_at(blockIdx.x) * BN + t + 128);
+    for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++it) {
+      const int64_t nrow = tile_at(j + gridDim.x) * BN + t;
+      const uint32_t nn0 = norm_of(nrow), nn1 = norm_of(nrow + 128);
+      {
+        const int64_t row0 = tile_at(j + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BN + t;
+        const uint32_t d0 = slot0(it + CODE_SLOTS - 1);
+        copy_code_rows<M>(d0, d0 + 128 * C::CODE_ROW, p.signs, row0, p.N);
+      }
+      const uint32_t x0 = 0x80008000u | (n0 << 16) | n0;
+      const uint32_t x1 = 0x80008000u | (n1 << 16) | n1;
+      cp_async_wait<CODE_SLOTS - 1>();
+      uint32_t c0w[C::CODE_WORDS], c1w[C::CODE_WORDS];
+      {
+        const uint32_t *s0 = reinterpret_cast<const uint32_t *>(gbase + (slot0(it) - base));
+        const uint32_t *s1 = s0 + 128 * (C::CODE_ROW / 4);
+#pragma unroll
+        for (int i = 0; i < C::CODE_WORDS; ++i) {
+          c0w[i] = s0[i];
+          c1w[i] = s1[i];
+        }
+      }
+#pragma unroll
+      for (int kc = 0; kc < C::KCH; ++kc, ++c) {
+        const int s = (int)(c % C::RING);
+        const uint32_t ph = (uint32_t)((c / C::RING) & 1);
+        if (!wait_phase(zempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t *chunk = gbase + C::OFF_Z + s * CHUNK_BYTES;
+        expand_row(chunk, t, c0w[2 * kc], c0w[2 * kc + 1], x0);
+        expand_row(chunk, t + 128, c1w[2 * kc], c1w[2 * kc + 1], x1);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(zfull_bar(s));
+      }
+      n0 = nn0;
+      n1 = nn1;
+    }
+    cp_async_wait<0>();
+  } else if (warp < MMA_WARP) {
+    // ---------------- epilogue: lane = query 32 (warp % 4) + lane; half h
+    // of the warps takes the 32-column groups g = h, h + 2, ...
+    const int q = warp & 3;
+    const int ew = warp - EXP_WARPS;
+    const int h = 0;
+    const int qi = 32 * q + lane;
+    float *park = reinterpret_cast<float *>(gbase + C::OFF_P) + (ew * 32 + lane) * (PARK_ROWS * 33);
+    // the list holds scores before the query's output scale (positive, so
+    // the order is the same)
+    TopList<KT> list;
+    list.init();
+    float published = -INFINITY;
+    // insert the qualifying scores of a group held in row[32] (shared memory)
+    auto insert_row = [&](const float *row, int g, int nvalid, int64_t base_row, float gb) {
+      const float thr = list.thr;
+      uint32_t hits = 0;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float sc = row[e];
+        hits |= (32 * g + e < nvalid && sc > thr && sc >= gb) ? (1u << e) : 0u;
+      }
+#pragma unroll 1
+      while (hits) {
+        const int e = __ffs(hits) - 1;
+        hits &= hits - 1;
+        const float sc = row[e];
+        if (sc > list.thr) list.insert(sc, (int32_t)(base_row + 32 * g + e));
+      }
+    };
+    int64_t tt = 0;
+    for (int64_t j = blockIdx.x; j < ntiles; j += gridDim.x, ++tt) {
+      const int64_t base_row = tile_at(j) * BN;
+      const int nvalid = (int)((p.N - base_row) < BN ? (p.N - base_row) : BN);
+      // the query's shared bound: scores below it cannot make the top KT
+      const float gb = ord_float(*reinterpret_cast<volatile unsigned *>(p.gbound + qi));
+      if (!wait_phase(dfull_bar, (uint32_t)(tt & 1), abort_flag, p.err)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)C::D_COL;
+      // the tile's 8 groups of 32 columns: while the accumulator is held only
+      // the group maxima are taken; groups that may qualify are parked and
+      // inserted once the accumulator is released (or when the rows are full)
+      int np = 0;          // parked groups
+      uint32_t pgs = 0;    // their group numbers, 4 bits each
+      // one group: its maximum (a tree, depth 5), parked if it may qualify
+      auto scan_group = [&](uint32_t (&v)[32], int g) {
+        float m16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m16[e] = fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 16]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) m16[e] = fmaxf(m16[e], m16[e + w]);
+        if (m16[0] > list.thr && m16[0] >= gb) {
+          float *row = park + np * 33;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) row[e] = __uint_as_float(v[e]);
+          pgs |= (uint32_t)g << (4 * np);
+          ++np;
+        }
+      };
+      auto flush = [&]() {
+#pragma unroll 1
+        for (int r = 0; r < np; ++r)
+          insert_row(park + r * 33, (int)((pgs >> (4 * r)) & 15u), nvalid, base_row, gb);
+        np = 0;
+        pgs = 0;
+      };
+      // the tile's 8 groups of 32 columns, two at a time with the next load in
+      // flight: while the accumulator is held only the group maxima are
+      // taken; groups that may qualify are parked and inserted after the
+      // accumulator is released (or when all rows are in use)
+      uint32_t va[32], vb[32];
+      tmem_ld32(trow, va);
+#pragma unroll 1
+      for (int g = 0; g < BN / 32; g += 2) {
+        tmem_ld_wait(va);
+        tmem_ld32(trow + 32 * (g + 1), vb);
+        scan_group(va, g);
+        tmem_ld_wait(vb);
+        if (g + 2 < BN / 32) {
+          tmem_ld32(trow + 32 * (g + 2), va);
+        } else {  // the accumulator is read: free it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dempty_bar);
+        }
+        scan_group(vb, g + 1);
+        // at most two groups park per pair: flush before the rows run out,
+        // and after the last pair (one call site keeps the code small)
+        if (np > PARK_ROWS - 2 || (g + 2 >= BN / 32 && np > 0)) flush();
+      }
+      // publish a better bound once the list is full
+      if (list.cnt == KT && list.thr > published) {
+        published = list.thr;
+        atomicMax(p.gbound + qi, ord_code(published));
+      }
+      __syncwarp();
+    }
+    // this warp's list for the query (unsorted, before the output scale;
+    // empty entries are -inf / -1)
+    const int64_t o = (((int64_t)blockIdx.x * LISTS + h) * QM + qi) * KT;
+#pragma unroll
+    for (int e = 0; e < KT; ++e) {
+      p.part_val[o + e] = list.val[e];
+      p.part_idx[o + e] = list.idx[e];
+    }
+  } else {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4)                        // D: fp32
+                                 | (0u << 7) | (0u << 10)         // A, B: fp16
+                                 | ((uint32_t)(BN >> 3) << 17)    // N
+                                 | ((uint32_t)(QM >> 4) << 24);   // M
+      int64_t c = 0, tt = 0;
+      bool ok = true;
+      for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++tt) {
+        if (!wait_phase(dempty_bar, (uint32_t)((tt & 1) ^ 1), abort_flag, p.err)) break;
+        tc_fence_after();
+        for (int kc = 0; kc < C::KCH; ++kc, ++c) {
+          const int s = (int)(c % C::RING);
+          const uint32_t ph = (uint32_t)((c / C::RING) & 1);
+          if (!wait_phase(zfull_bar(s), ph, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < CHUNK_K / 16; ++kk) {
+            const uint32_t atm = tmem_base + (uint32_t)(kc * 32 + kk * 8);
+            const uint64_t bdesc = smem_desc_sw128(sZ + s * CHUNK_BYTES + kk * 32);
+            mma_f16_ts(tmem_base + C::D_COL, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(zempty_bar(s));
+        }
+        if (!ok) break;
+        mma_commit(dfull_bar);
+      }
+      if (tt > 0 && ok) {  // the last tile's MMAs complete before TMEM is freed
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(dfull_bar, (uint32_t)((tt - 1) & 1)) &&
+               globaltimer() - t0 < WAIT_NS) {
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
+                 "n"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------------------
+// Merge: per query, the k best of all CTAs' lists, best first (ties to the
+// lower index); entries beyond the candidates are (-1, -inf).  Output mode
+// writes them (scores times the query's output scale); bound mode writes the
+// k-th best as the query's shared bound (none if fewer than k candidates).
+__device__ __forceinline__ bool better(float a, int32_t ia, float b, int32_t ib) {
+  return a > b || (a == b && (unsigned)ia < (unsigned)ib);
+}
+
+__global__ void __launch_bounds__(MERGE_THREADS) search_merge_kernel(
+    const float *__restrict__ part_val, const int32_t *__restrict__ part_idx, int ctas, int kt,
+    int k, const float *__restrict__ qscale, int32_t *__restrict__ out_idx,
+    float *__restrict__ out_scores, unsigned *__restrict__ bound_out) {
+  extern __shared__ uint8_t mg_smem[];
+  const int ncand = ctas * LISTS * kt;
+  float *cv = reinterpret_cast<float *>(mg_smem);
+  int32_t *ci = reinterpret_cast<int32_t *>(cv + ncand);
+  __shared__ float wv[MERGE_THREADS / 32];
+  __shared__ int32_t wi[MERGE_THREADS / 32];
+  __shared__ int wpos[MERGE_THREADS / 32];
+  const int qi = blockIdx.x;
+  for (int e = threadIdx.x; e < ncand; e += MERGE_THREADS) {
+    const int list = e / kt, j = e - list * kt;  // list = cta * LISTS + half
+    const int64_t o = ((int64_t)list * QM + qi) * kt + j;
+    cv[e] = part_val[o];
+    ci[e] = part_idx[o];
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int32_t bi = -1;
+    int bp = -1;
+    for (int e = threadIdx.x; e < ncand; e += MERGE_THREADS)
+      if (ci[e] >= 0 && (bp < 0 || better(cv[e], ci[e], bv, bi))) {
+        bv = cv[e];
+        bi = ci[e];
+        bp = e;
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const int op = __shfl_xor_sync(0xffffffffu, bp, o);
+      if (op >= 0 && (bp < 0 || better(ov, oi, bv, bi))) {
+        bv = ov;
+        bi = oi;
+        bp = op;
+      }
+    }
+    if (lane == 0) {
+      wv[w] = bv;
+      wi[w] = bi;
+      wpos[w] = bp;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float fv = -INFINITY;
+      int32_t fi = -1;
+      int fp = -1;
+      for (int x = 0; x < MERGE_THREADS / 32; ++x)
+        if (wpos[x] >= 0 && (fp < 0 || better(wv[x], wi[x], fv, fi))) {
+          fv = wv[x];
+          fi = wi[x];
+          fp = wpos[x];
+        }
+      if (bound_out) {
+        if (r == k - 1) bound_out[qi] = fp >= 0 ? ord_code(fv) : 0u;
+      } else {
+        out_idx[(int64_t)qi * k + r] = fi;
+        out_scores[(int64_t)qi * k + r] = fp >= 0 ? fv * qscale[qi] : -INFINITY;
+      }
+      if (fp >= 0) ci[fp] = -1;  // taken
+    }
+    __syncthreads();
+  }
+}
+
+// list length per query and CTA (k <= JL_SEARCH_MAX_K = 16): a longer list
+// would not fit the epilogue's registers
+static int list_len(int) { return 16; }
+
+template <int M, int KT>
+static cudaError_t launch_pass(const Params &p, int grid, cudaStream_t stream) {
+  using C = Cfg<M>;
+  cudaError_t e = cudaFuncSetAttribute(search_tc_kernel<M, KT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  search_tc_kernel<M, KT><<<grid, THREADS, C::SMEM, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace srch
+
+size_t search_workspace_bytes(int nq, int m, int k) {
+  (void)nq;
+  const size_t u = (size_t)srch::QM * m * sizeof(float);
+  const size_t lists = (size_t)srch::MAX_CTAS * srch::LISTS * srch::QM * srch::list_len(k);
+  return (u + 255) / 256 * 256 + lists * (sizeof(float) + sizeof(int32_t)) +
+         srch::QM * (sizeof(unsigned) + sizeof(float)) + 256;
+}
+
+cudaError_t launch_search(const void *Q, bool q_f32, int nq, const uint16_t *S, int m, int d,
+                          const uint32_t *signs, const uint16_t *norms, int64_t N, int k,
+                          int32_t *out_idx, float *out_scores, void *workspace,
+                          cudaStream_t stream) {
+  using namespace srch;
+  int *err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  const int kt = list_len(k);
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  float *U = reinterpret_cast<float *>(ws);
+  const size_t u_bytes = ((size_t)QM * m * sizeof(float) + 255) / 256 * 256;
+  float *part_val = reinterpret_cast<float *>(ws + u_bytes);
+  int32_t *part_idx = reinterpret_cast<int32_t *>(part_val + (size_t)MAX_CTAS * LISTS * QM * kt);
+  unsigned *gbound = reinterpret_cast<unsigned *>(part_idx + (size_t)MAX_CTAS * LISTS * QM * kt);
+  float *qscale = reinterpret_cast<float *>(gbound + QM);
+  const int64_t num_tiles = (N + BN - 1) / BN;
+  int64_t grid64 = device_sm_count();
+  if (grid64 > MAX_CTAS) grid64 = MAX_CTAS;
+  if (grid64 > num_tiles) grid64 = num_tiles;
+  const int grid = (int)grid64;
+  const size_t qbytes = (size_t)d * (q_f32 ? 4 : 2);
+  const size_t msmem = (size_t)grid * LISTS * kt * (sizeof(float) + sizeof(int32_t));
+  cudaError_t e = cudaFuncSetAttribute(search_merge_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+  if (e != cudaSuccess) return e;
+  for (int q0 = 0; q0 < nq; q0 += QM) {
+    const int nqp = nq - q0 < QM ? nq - q0 : QM;
+    e = launch_query_projection(reinterpret_cast<const uint8_t *>(Q) + (size_t)q0 * qbytes,
+                                q_f32, S, U, nqp, m, d, stream);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(gbound, 0, QM * sizeof(unsigned), stream);  // no bound yet
+    if (e != cudaSuccess) return e;
+    Params p{signs, norms, U, part_val, part_idx, gbound, qscale, N, num_tiles, 0, 1, nqp,
+             (float)(1.2533141373155002512 / (double)m), err};
+    auto run = [&](const Params &pp) -> cudaError_t {
+#define JL_CASE(MM) \
+      if (m == MM) return launch_pass<MM, 16>(pp, grid, stream);
+      JL_CASE(64) JL_CASE(128) JL_CASE(256) JL_CASE(512)
+#undef JL_CASE
+      return cudaErrorNotSupported;
+    };
+    // warm start: about 4 tiles per CTA spread over the index, merged into
+    // each query's starting bound (the 16th best of the sample)
+    const int64_t sample_step = num_tiles / ((int64_t)grid * 4);
+    if (sample_step >= 2) {
+      Params ps = p;
+      ps.tile_step = sample_step;
+      ps.num_tiles = (num_tiles + sample_step - 1) / sample_step;
+      e = run(ps);
+      if (e != cudaSuccess) return e;
+      search_merge_kernel<<<nqp, MERGE_THREADS, msmem, stream>>>(
+          part_val, part_idx, grid, kt, kt, qscale, nullptr, nullptr, gbound);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    e = run(p);
+    if (e != cudaSuccess) return e;
+    search_merge_kernel<<<nqp, MERGE_THREADS, msmem, stream>>>(
+        part_val, part_idx, grid, kt, k, qscale, out_idx + (size_t)q0 * k,
+        out_scores + (size_t)q0 * k, nullptr);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace jlk

@@ -187,6 +187,48 @@ JL_API int jl_dequantize_keys(const uint32_t *signs, const uint16_t *norms, int6
                               const uint16_t *S, int m, int d, uint16_t *out,
                               jl_stream_t stream);
 
+/* Largest k of jl_search_topk. */
+#define JL_SEARCH_MAX_K 16
+
+/*
+ * jl_search_workspace_bytes -- device scratch jl_search_topk needs (query
+ * projections of one pass of 128 queries and the per-CTA candidate lists).
+ * Depends on the shapes only; 0 for unsupported shapes or k outside
+ * [1, JL_SEARCH_MAX_K].
+ */
+JL_API size_t jl_search_workspace_bytes(int n_queries, int m, int d, int k);
+
+/*
+ * jl_search_topk -- inner-product search over a QJL-compressed index.
+ * Defines: "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+ * Quantization", final section (the quantizer serves any store of vectors
+ * read through inner products: vector databases, retrieval), with the
+ * asymmetric estimator of the QJL section as the similarity:
+ *     s(q, x_j) = sqrt(pi/2)/m * ||x_j|| * <S q, sign(S x_j)>.
+ * For every query, the k index vectors with the largest s, best first; equal
+ * scores go to the lower index.
+ *   Q          : in, n_queries x d of q_dtype (16-byte aligned).
+ *   S          : in, m x d bf16 sketch.
+ *   signs      : in, n_index x (m/32) uint32 codes (jl_quantize_keys layout),
+ *                16-byte aligned.
+ *   norms      : in, n_index binary16 norms.
+ *   out_index  : out, n_queries x k int32 (-1 past the last vector when
+ *                k > n_index).
+ *   out_scores : out, n_queries x k fp32 (-inf where out_index is -1).
+ *   workspace  : >= jl_search_workspace_bytes(...), 256-byte aligned.
+ * Queries are handled 128 at a time.  The scores are computed on the tensor
+ * cores with the query projection rounded to fp16 (a power-of-two scale per
+ * query keeps its largest coordinate in [2^14, 2^15)), so they agree with the
+ * float64 estimator to about 3e-4 of the score scale; near-ties may order
+ * differently.  n_queries == 0 is a no-op.  Errors: JL_ERR_INVALID_ARG
+ * (n_index < 1, k outside [1, JL_SEARCH_MAX_K], bad pointer), JL_ERR_UNSUPPORTED,
+ * JL_ERR_WORKSPACE, JL_ERR_CUDA.
+ */
+JL_API int jl_search_topk(const void *Q, jl_dtype q_dtype, int n_queries, const uint16_t *S,
+                          int m, int d, const uint32_t *signs, const uint16_t *norms,
+                          int64_t n_index, int k, int32_t *out_index, float *out_scores,
+                          void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
 /*
  * jl_decode_paged_workspace_bytes -- device scratch jl_decode_attention_paged
  * needs (query projections and split partial states) for B sequences of at

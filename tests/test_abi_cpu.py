@@ -210,3 +210,29 @@ def test_dequantize_argument_errors(lib):
     assert call(signs=MISALIGNED) == jl.JL_ERR_INVALID_ARG
     assert call(out=ctypes.c_void_p((1 << 20) + 8)) == jl.JL_ERR_INVALID_ARG
     assert call(norms=ctypes.c_void_p((1 << 20) + 1)) == jl.JL_ERR_INVALID_ARG
+
+
+def test_search_argument_errors(lib):
+    f = lib.jl_search_topk
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, nq=4, S=FAKE, m=256, d=128, signs=FAKE, norms=FAKE,
+              N=1000, k=10, oi=FAKE, os=FAKE, ws=FAKE, wsb=1 << 40)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["Q"], a["qt"], a["nq"], a["S"], a["m"], a["d"], a["signs"], a["norms"],
+                 a["N"], a["k"], a["oi"], a["os"], a["ws"], a["wsb"], NULL)
+
+    assert call(nq=0) == jl.JL_OK
+    assert call(nq=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(N=0) == jl.JL_ERR_INVALID_ARG
+    assert call(k=0) == jl.JL_ERR_INVALID_ARG
+    assert call(k=17) == jl.JL_ERR_INVALID_ARG
+    assert call(qt=3) == jl.JL_ERR_INVALID_ARG
+    assert call(m=100) == jl.JL_ERR_UNSUPPORTED
+    for key in ("Q", "S", "signs", "norms", "oi", "os"):
+        assert call(**{key: NULL}) == jl.JL_ERR_INVALID_ARG, key
+    assert call(signs=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
+    need = jl.jl_search_workspace_bytes(4, 256, 128, 10)
+    assert need > 0 and call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
+    assert jl.jl_search_workspace_bytes(4, 256, 128, 17) == 0

@@ -25,6 +25,8 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
            gqa.
   dequant-gqa  the gqa cache's 2,097,152 codes (m=256) and norms turned back
            into bf16 keys of d=128 (codes made from gqa's keys).
+  search   top-10 inner-product search of 128 bf16 N(0,1) queries over an index
+           of 8,388,608 N(0,1) vectors (d=128) kept as QJL codes (m=256).
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -95,7 +97,13 @@ PAGE_TOKENS = 64
 # dequant-gqa: the codes of the gqa cache turned back into bf16 keys
 DEQUANT_GQA = GQA.with_(name="dequant-gqa")
 
-ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA)}
+# search: 128 queries against an index of 8,388,608 vectors (as keys of one
+# sequence: B = Hkv = 1, T = index size; Hq = queries)
+SEARCH = Workload("search", 7, 1, 128, 1, 8388608, 128, 256, torch.bfloat16)
+SEARCH_K = 10
+
+ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA,
+                           SEARCH)}
 
 
 def sweep_points():
