@@ -14,6 +14,10 @@ Functions (same names as the C entry points):
   jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int
   jl_decode_attention(Q, S, signs, norms, V, ...) -> out bf16 [B, Hq, d]
   jl_device_error()                     -> int (0 = no device fault reported)
+  jl_turbo_codebook(d, mse_bits)        -> centroids (list of float)
+  jl_turbo_rotation_init(d, seed)       -> (Pi bf16 [d, d], Pinv fp32 [d, d])
+  jl_turbo_quantize_keys(K, Pi, S, mse_bits) -> (codes int32 [n, words], norms fp16 [n, 2])
+  jl_turbo_decode_attention(Q, Pinv, S, codes, norms, V, mse_bits, ...) -> out bf16
 
 Sign codes are returned as torch.int32 tensors holding the uint32 words bit
 for bit (torch has no general uint32 arithmetic); word w of a key holds sketch
@@ -48,7 +52,9 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_decode_attention", "jl_device_error", "jl_bf16_from_f64",
             "jl_decode_attention_noalloc", "jl_decode_paged_workspace_bytes",
             "jl_decode_attention_paged", "jl_dequantize_keys", "jl_search_workspace_bytes",
-            "jl_search_topk")
+            "jl_search_topk", "jl_turbo_codebook", "jl_turbo_rotation_workspace_bytes",
+            "jl_turbo_rotation_init", "jl_turbo_quantize_keys", "jl_turbo_decode_workspace_bytes",
+            "jl_turbo_decode_attention")
 
 _lib = None
 
@@ -101,6 +107,19 @@ def load():
     L.jl_decode_attention_paged.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
                                             vp, i32, vp, i32, i32, i32, i64, i32, i32,
                                             ctypes.c_float, vp, vp, vp, sz, vp]
+    L.jl_turbo_codebook.restype = i32
+    L.jl_turbo_codebook.argtypes = [i32, i32, vp]
+    L.jl_turbo_rotation_workspace_bytes.restype = sz
+    L.jl_turbo_rotation_workspace_bytes.argtypes = [i32]
+    L.jl_turbo_rotation_init.restype = i32
+    L.jl_turbo_rotation_init.argtypes = [vp, vp, i32, ctypes.c_uint64, vp, sz, vp]
+    L.jl_turbo_quantize_keys.restype = i32
+    L.jl_turbo_quantize_keys.argtypes = [vp, i32, i64, i64, vp, vp, i32, i32, i32, vp, vp, vp]
+    L.jl_turbo_decode_workspace_bytes.restype = sz
+    L.jl_turbo_decode_workspace_bytes.argtypes = [i32, i32, i32, i64, i32, i32, i32]
+    L.jl_turbo_decode_attention.restype = i32
+    L.jl_turbo_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i64,
+                                            i32, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.jl_bf16_from_f64.restype = ctypes.c_uint16
@@ -396,3 +415,110 @@ def jl_device_error(stream=None) -> int:
 
 def jl_bf16_from_f64(x: float) -> int:
     return int(load().jl_bf16_from_f64(float(x)))
+
+
+# --------------------------------------------------------------------------
+# TurboQuant-prod keys
+
+def turbo_code_words(mse_bits: int, m: int, d: int) -> int:
+    """uint32 words of one key's code: mse_bits cell planes of d bits, then m
+    residual sign bits."""
+    return (mse_bits * d + m) // 32
+
+
+def jl_turbo_codebook(d: int, mse_bits: int):
+    """The 2^mse_bits Lloyd-Max centroids of the rotated-coordinate density
+    (ascending, as float), computed by the library on the host."""
+    L = load()
+    buf = (ctypes.c_float * (1 << mse_bits))()
+    _check(L.jl_turbo_codebook(d, mse_bits, ctypes.cast(buf, ctypes.c_void_p)),
+           "jl_turbo_codebook")
+    return [float(v) for v in buf]
+
+
+def jl_turbo_rotation_workspace_bytes(d: int) -> int:
+    return int(load().jl_turbo_rotation_workspace_bytes(d))
+
+
+def jl_turbo_rotation_init(d: int, seed: int, device=None, stream=None):
+    """(Pi bf16 [d, d], Pinv fp32 [d, d]) regenerated from ``seed``."""
+    L = load()
+    dev = device if device is not None else "cuda"
+    Pi = torch.empty((d, d), dtype=torch.bfloat16, device=dev)
+    Pinv = torch.empty((d, d), dtype=torch.float32, device=dev)
+    ws = torch.empty((max(jl_turbo_rotation_workspace_bytes(d), 1),), dtype=torch.uint8,
+                     device=dev)
+    _check(L.jl_turbo_rotation_init(_ptr(Pi), _ptr(Pinv), d, ctypes.c_uint64(seed), _ptr(ws),
+                                    ws.numel(), _stream(Pi, stream)), "jl_turbo_rotation_init")
+    return Pi, Pinv
+
+
+def jl_turbo_quantize_keys(K, Pi, S, mse_bits: int, codes=None, norms=None, stream=None):
+    """TurboQuant-prod codes (int32 [n, words]) and norms (fp16 [n, 2]:
+    ||k||, ||rt||) of the rows of K ([..., d] bf16)."""
+    L = load()
+    if K.dim() != 2:
+        K = K.reshape(-1, K.shape[-1])
+    n, d = K.shape
+    m = S.shape[0]
+    _need_cuda(K, Pi, S)
+    if K.stride(1) != 1:
+        raise ValueError("keys must have unit stride along d")
+    if K.dtype != torch.bfloat16:
+        raise TypeError("the TurboQuant quantizer takes bf16 keys")
+    assert Pi.dtype == torch.bfloat16 and Pi.is_contiguous() and Pi.shape == (d, d)
+    assert S.dtype == torch.bfloat16 and S.is_contiguous() and S.shape[1] == d
+    words = turbo_code_words(mse_bits, m, d)
+    if codes is None:
+        codes = torch.empty((n, words), dtype=torch.int32, device=K.device)
+    if norms is None:
+        norms = torch.empty((n, 2), dtype=torch.float16, device=K.device)
+    assert codes.dtype == torch.int32 and codes.is_contiguous() and codes.numel() == n * words
+    assert norms.dtype == torch.float16 and norms.is_contiguous() and norms.numel() == 2 * n
+    _check(L.jl_turbo_quantize_keys(_ptr(K), JL_BF16, n, K.stride(0) if n > 0 else d, _ptr(Pi),
+                                    _ptr(S), m, d, mse_bits, _ptr(codes), _ptr(norms),
+                                    _stream(K, stream)), "jl_turbo_quantize_keys")
+    return codes, norms
+
+
+def jl_turbo_decode_workspace_bytes(B, Hq, Hkv, T, m, d, mse_bits) -> int:
+    return int(load().jl_turbo_decode_workspace_bytes(B, Hq, Hkv, T, m, d, mse_bits))
+
+
+def jl_turbo_decode_attention(Q, Pinv, S, codes, norms, V, mse_bits, softmax_scale=None,
+                              out=None, scores=None, want_scores=False, workspace=None,
+                              stream=None):
+    """One decode step over TurboQuant-prod keys.
+
+    Q [B, Hq, d] (bf16/fp32); codes [B, Hkv, T, words] int32; norms
+    [B, Hkv, T, 2] fp16; V [B, Hkv, T, d] bf16.  Returns out [B, Hq, d] bf16,
+    or (out, scores [B, Hq, T] fp32) when ``want_scores`` (or ``scores``)."""
+    L = load()
+    B, Hq, d = Q.shape
+    m = S.shape[0]
+    Hkv, T = V.shape[1], V.shape[2]
+    words = turbo_code_words(mse_bits, m, d)
+    _need_cuda(Q, Pinv, S, codes, norms, V, out, scores)
+    assert codes.dtype == torch.int32 and codes.shape == (B, Hkv, T, words)
+    assert norms.dtype == torch.float16 and norms.shape == (B, Hkv, T, 2)
+    assert V.dtype == torch.bfloat16 and V.shape == (B, Hkv, T, d)
+    assert Pinv.dtype == torch.float32 and Pinv.shape == (d, d)
+    for t in (Q, Pinv, S, codes, norms, V):
+        if not t.is_contiguous():
+            raise ValueError("decode inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=Q.device)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
+    need = jl_turbo_decode_workspace_bytes(B, Hq, Hkv, T, m, d, mse_bits)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_turbo_decode_attention(_ptr(Q), qt, _ptr(Pinv), _ptr(S), _ptr(codes),
+                                       _ptr(norms), _ptr(V), B, Hq, Hkv, T, m, d, mse_bits,
+                                       ctypes.c_float(softmax_scale), _ptr(out), _ptr(scores),
+                                       _ptr(workspace), workspace.numel(), _stream(Q, stream)),
+           "jl_turbo_decode_attention")
+    return (out, scores) if scores is not None else out

@@ -281,6 +281,81 @@ int jl_decode_attention_paged(
   return from_cuda(jlk::launch_decode_paged(p, a, (cudaStream_t)stream));
 }
 
+int jl_turbo_codebook(int d, int mse_bits, float *centroids) {
+  if (!centroids) return JL_ERR_INVALID_ARG;
+  if (d < 3 || d > 4096 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+    return JL_ERR_UNSUPPORTED;
+  return jlk::turbo_codebook(d, mse_bits, centroids, nullptr) ? JL_OK : JL_ERR_UNSUPPORTED;
+}
+
+size_t jl_turbo_rotation_workspace_bytes(int d) { return jlk::turbo_rotation_workspace_bytes(d); }
+
+int jl_turbo_rotation_init(uint16_t *Pi, float *Pinv, int d, uint64_t seed, void *workspace,
+                           size_t workspace_bytes, jl_stream_t stream) {
+  if (d != 64 && d != 128) return JL_ERR_UNSUPPORTED;
+  if (!Pi || !Pinv || !aligned(Pi, 16) || !aligned(Pinv, 16)) return JL_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) ||
+      workspace_bytes < jlk::turbo_rotation_workspace_bytes(d))
+    return JL_ERR_WORKSPACE;
+  return from_cuda(
+      jlk::launch_turbo_rotation(Pi, Pinv, d, seed, workspace, (cudaStream_t)stream));
+}
+
+int jl_turbo_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                           int64_t key_stride, const uint16_t *Pi, const uint16_t *S, int m,
+                           int d, int mse_bits, uint32_t *codes, uint16_t *norms,
+                           jl_stream_t stream) {
+  if (key_dtype != JL_BF16 && key_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (n_keys < 0) return JL_ERR_INVALID_ARG;
+  if (key_dtype != JL_BF16 || m != 128 || d != 128 || mse_bits < 1 ||
+      mse_bits > JL_TURBO_MAX_MSE_BITS)
+    return JL_ERR_UNSUPPORTED;
+  if (n_keys == 0) return JL_OK;
+  if (!K || !Pi || !S || !codes || !norms || key_stride < d) return JL_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || ((size_t)key_stride * 2) % 16 != 0 || !aligned(Pi, 16) ||
+      !aligned(S, 16) || !aligned(codes, 16) || !aligned(norms, 4))
+    return JL_ERR_INVALID_ARG;
+  if (n_keys >= ((int64_t)1 << 31) || key_stride >= ((int64_t)1 << 39)) return JL_ERR_UNSUPPORTED;
+  return from_cuda(jlk::launch_turbo_quantize(reinterpret_cast<const uint16_t *>(K), n_keys,
+                                              key_stride, Pi, S, m, d, mse_bits, codes, norms,
+                                              (cudaStream_t)stream));
+}
+
+size_t jl_turbo_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m, int d,
+                                       int mse_bits) {
+  jlk::DecodePlan p;
+  if (B == 0) return 0;
+  if (!jlk::make_turbo_decode_plan(B, Hq, Hkv, T, m, d, mse_bits, &p)) return 0;
+  return p.total_bytes;
+}
+
+int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv,
+                              const uint16_t *S, const uint32_t *codes, const uint16_t *norms,
+                              const uint16_t *V, int B, int Hq, int Hkv, int64_t T, int m,
+                              int d, int mse_bits, float softmax_scale, uint16_t *out,
+                              float *scores, void *workspace, size_t workspace_bytes,
+                              jl_stream_t stream) {
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
+  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > 2) return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
+  if (B == 0) return JL_OK;
+  if (!Q || !Pinv || !S || !codes || !norms || !V || !out) return JL_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(Pinv, 16) || !aligned(S, 16) || !aligned(codes, 16) ||
+      !aligned(norms, 16) || !aligned(V, 16) || !aligned(out, 4) ||
+      (scores && !aligned(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  jlk::DecodePlan p;
+  if (!jlk::make_turbo_decode_plan(B, Hq, Hkv, T, m, d, mse_bits, &p)) return JL_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
+    return JL_ERR_WORKSPACE;
+  double walsh[3];
+  if (!jlk::turbo_codebook(d, mse_bits, nullptr, walsh)) return JL_ERR_UNSUPPORTED;
+  return from_cuda(jlk::launch_turbo_decode(p, mse_bits, Q, q_dtype == JL_F32, Pinv, S, codes,
+                                            norms, V, walsh, softmax_scale, out, scores,
+                                            workspace, (cudaStream_t)stream));
+}
+
 int jl_device_error(int *code, jl_stream_t stream) {
   if (!code) return JL_ERR_INVALID_ARG;
   *code = 0;

@@ -60,29 +60,38 @@ constexpr int DEC_NORM_AREA = 128; // per stage: 40 fp16 norms; bulk-tensor copi
 #define JL_DECODE_SCORE 0
 #endif
 
-template <int M, int D, bool S8>
+// TB > 0: TurboQuant-prod codes, TB cell bit planes of D bits ahead of the M
+// residual sign bits, scored as TB + 1 sign contractions (see turbo_scores).
+template <int M, int D, bool S8, int TB = 0>
 struct DecCfg {
   static constexpr int STAGES = 2;                     // blocks in the ring
-  static constexpr int KEY_SIGN_BYTES = M / 8;
+  static constexpr int CODE_BITS = TB * D + M;         // bits per key
+  static constexpr int KEY_SIGN_BYTES = CODE_BITS / 8;
   static constexpr int SIGN_BYTES = DEC_KB * KEY_SIGN_BYTES;
   static constexpr int V_BYTES = DEC_KB * D * 2;       // 4 or 8 KB
   static constexpr int V_BOX = DEC_KB * 128;           // one 64-column box
   static constexpr int STAGE_BYTES = (V_BYTES + SIGN_BYTES + 1023) / 1024 * 1024;
   // scoring MMA: bf16 m16n8k16 (16 coordinates per slice) or s8 m16n8k32 (32)
   static constexpr int KS = S8 ? 32 : 16;
-  static constexpr int NC = M / KS;                    // k slices
+  static constexpr int NC = CODE_BITS / KS;            // k slices
+  static constexpr int NC_MSE = TB * D / KS;           // slices of the cell planes
   static constexpr int A_REGS = 4 * NC;
   static constexpr bool A_SMEM = A_REGS > 64;          // A fragments in smem
   static constexpr int A_SMEM_BYTES = A_SMEM ? NC * 32 * 16 : 0;
   static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + A_SMEM_BYTES;
+  // per stage: the block's norms (TB > 0: two binary16 per key), with room
+  // for the 16-byte-aligned groups of the cp.async path
+  static constexpr int NORM_BYTES = TB ? 4 : 2;
+  static constexpr int NORM_AREA = TB ? 2 * DEC_NORM_AREA : DEC_NORM_AREA;
   static constexpr int OFF_NORM = DEC_WARPS * WARP_BYTES;
-  static constexpr int OFF_BAR = OFF_NORM + DEC_WARPS * STAGES * DEC_NORM_AREA;
+  static constexpr int OFF_BAR = OFF_NORM + DEC_WARPS * STAGES * NORM_AREA;
   static constexpr int CTA_BYTES = OFF_BAR + DEC_WARPS * STAGES * 8 + 1024;  // + align
-  static constexpr int LW = (M >= 128) ? M / 128 : 1;  // code words a lane reads
+  static constexpr int LW = (CODE_BITS >= 128) ? CODE_BITS / 128 : 1;  // code words a lane reads
   static constexpr int SIGN_CHUNK = (M >= 128) ? 16 : 8;
   static constexpr int SIGN_CHUNKS = SIGN_BYTES / SIGN_CHUNK;  // multiple of 32
   static constexpr int DT = D / 16;                    // 16-dim output tiles
   static_assert(SIGN_CHUNKS % 32 == 0, "sign chunks per lane");
+  static_assert(TB == 0 || (!S8 && D == 128 && M % 128 == 0), "cell-plane codes: bf16, d = 128");
   static_assert(STAGE_BYTES % 1024 == 0 && WARP_BYTES % 1024 == 0, "swizzle atoms");
 };
 
@@ -151,7 +160,7 @@ constexpr int PROJ_VECS = 4;
 template <int M, int D, bool XF32>
 __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
                                          const void *__restrict__ X, int64_t x0,
-                                         int nx, float *dst) {
+                                         int nx, float *dst, int dst_stride = M) {
   constexpr int CPL = D / 32;   // columns per lane
   constexpr int CH = 8;         // rows per chunk
   constexpr int RPW = M / 8;    // rows per warp
@@ -205,7 +214,7 @@ __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
       }
     }
     const int k = lane / PROJ_VECS, j = lane % PROJ_VECS;
-    if (j < nx) dst[(int64_t)j * M + warp + 8 * (r0 + k)] = v[0];
+    if (j < nx) dst[(int64_t)j * dst_stride + warp + 8 * (r0 + k)] = v[0];
   }
 }
 
@@ -217,6 +226,48 @@ __global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restr
   const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
   const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
   project4<M, D, QF32>(S, Q, x0, nx, U + x0 * M);
+}
+
+// TurboQuant-prod query rows, four queries per CTA: w = Pinv^T q (so that
+// <w, Pi x> = <q, x> for the stored bf16 Pi), then the row
+//   [wc_0 w, ..., wc_{TB-1} w, S w]
+// whose dot product with the +-1 expansion of a key's code [planes, signs]
+// gives the two raw sums of the score: the cell planes' part is
+// <w, c[cell]> because c_j = sum_p wc_p (2 bit_p(j) - 1) for the symmetric
+// codebook (its single-bit Walsh coefficients; the others vanish for
+// TB <= 2).
+template <int M, int D, int TB, bool QF32>
+__global__ void __launch_bounds__(PROJ_THREADS)
+    turbo_qproj_kernel(const void *__restrict__ Q, const float *__restrict__ Pinv,
+                       const uint16_t *__restrict__ S, float *__restrict__ U, int nq, float wc0,
+                       float wc1) {
+  griddep_launch_dependents();
+  constexpr int MT = TB * D + M;
+  __shared__ float wsm[PROJ_VECS * D];
+  const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
+  const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
+  for (int e = threadIdx.x; e < PROJ_VECS * D; e += PROJ_THREADS) {
+    const int j = e / D, i = e - (e / D) * D;
+    float acc = 0.f;
+    if (j < nx) {
+      const int64_t qb = (x0 + j) * D;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
+        const float qc = QF32 ? reinterpret_cast<const float *>(Q)[qb + c]
+                              : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[qb + c]);
+        acc = fmaf(__ldg(Pinv + c * D + i), qc, acc);
+      }
+    }
+    wsm[e] = acc;
+  }
+  __syncthreads();
+  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TB * D, MT);
+  for (int e = threadIdx.x; e < nx * D; e += PROJ_THREADS) {
+    const int j = e / D, i = e - (e / D) * D;
+    float *row = U + (x0 + j) * MT;
+    row[i] = wc0 * wsm[e];
+    if constexpr (TB > 1) row[D + i] = wc1 * wsm[e];
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -352,9 +403,9 @@ __device__ __forceinline__ void load_page(BlockPos &pos) {
   pos.page = __ldg(pos.trow + pos.pidx);
 }
 
-template <int M, int D, bool S8>
+template <int M, int D, bool S8, int TB = 0>
 struct Ring {
-  using C = DecCfg<M, D, S8>;
+  using C = DecCfg<M, D, S8, TB>;
   uint32_t base;   // this warp's stages (1024-aligned)
   uint32_t nbase;  // this warp's norm areas
   uint32_t bbase;  // this warp's barriers
@@ -363,17 +414,17 @@ struct Ring {
     return base + s * C::STAGE_BYTES + C::V_BYTES;
   }
   __device__ __forceinline__ uint32_t afrag() const { return base + C::STAGES * C::STAGE_BYTES; }
-  __device__ __forceinline__ uint32_t norm(int s) const { return nbase + s * DEC_NORM_AREA; }
+  __device__ __forceinline__ uint32_t norm(int s) const { return nbase + s * C::NORM_AREA; }
   __device__ __forceinline__ uint32_t bar(int s) const { return bbase + 8 * s; }
 };
 
 // Start the copies of block `pos` into stage s: values by one 3-D bulk-tensor
 // copy per 64 columns (lane 0), codes and norms by cp.async (all lanes).
-template <int M, int D, bool S8, bool PAGED>
+template <int M, int D, bool S8, bool PAGED, int TB = 0>
 __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &maps,
-                                            const Ring<M, D, S8> &ring, const BlockPos &pos,
+                                            const Ring<M, D, S8, TB> &ring, const BlockPos &pos,
                                             int s, int lane) {
-  using C = DecCfg<M, D, S8>;
+  using C = DecCfg<M, D, S8, TB>;
   const int64_t kvi = pos.kvi;
   const int64_t key0 = pos.blk * DEC_KB;
   if (PAGED || maps.tma_codes) {
@@ -385,7 +436,7 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
         y = pos.y;
         z = pos.page * p.Hkv + pos.hkv;
       }
-      mbar_expect_tx(ring.bar(s), C::V_BYTES + C::SIGN_BYTES + 2 * DEC_KB);
+      mbar_expect_tx(ring.bar(s), C::V_BYTES + C::SIGN_BYTES + C::NORM_BYTES * DEC_KB);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h)
         tma_load_3d(ring.val(s) + h * C::V_BOX, &maps.value, h * 64, y, z, ring.bar(s));
@@ -410,15 +461,19 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
     else
       cp_async_8(sdst + e * 8, src, ok ? 8 : 0);
   }
-  // norms: the 16-byte-aligned run of 8-norm groups covering the block
-  // (at most 5 groups); key k of the block lands at element (gkey & 7) + k
-  if (lane < 5) {
-    const int64_t first = (gkey & ~(int64_t)7) + 8 * lane;
+  // norms: the 16-byte-aligned run of G-key groups covering the block (G = 8
+  // binary16 norms, or 4 pairs); key k of the block lands at key slot
+  // (gkey % G) + k
+  constexpr int G = 16 / C::NORM_BYTES;
+  constexpr int GROUPS = (DEC_KB + G - 1) / G + 1;
+  if (lane < GROUPS) {
+    const int64_t first = (gkey & ~(int64_t)(G - 1)) + G * lane;
     const int64_t avail = p.n_keys - first;
     const bool ok = first < gkey + nval && avail > 0;
-    const int nbytes = ok ? (avail >= 8 ? 16 : (int)avail * 2) : 0;
-    cp_async_16(ring.norm(s) + 16 * lane, ok ? (const void *)(p.norms + first)
-                                             : (const void *)p.norms, nbytes);
+    const int nbytes = ok ? (avail >= G ? 16 : (int)avail * C::NORM_BYTES) : 0;
+    const uint8_t *nb = reinterpret_cast<const uint8_t *>(p.norms);
+    cp_async_16(ring.norm(s) + 16 * lane,
+                ok ? (const void *)(nb + first * C::NORM_BYTES) : (const void *)nb, nbytes);
   }
   cp_async_mbar_arrive(ring.bar(s));
   __syncwarp();
@@ -458,12 +513,12 @@ __device__ __forceinline__ float f4c(const float4 &v, int i) {
 //   int8: u ~= hscale * (256 hi + lo), |256 hi + lo| <= 32000, usum = sum of
 //         256 hi + lo over the head's coordinates.
 // u is read as whole 16-byte vectors of the lane's own coordinate runs.
-template <int M, int D, bool S8>
+template <int M, int D, bool S8, int TB = 0>
 __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t,
-                                             const Ring<M, D, S8> &ring,
-                                             uint32_t (&afr)[DecCfg<M, D, S8>::A_SMEM ? 1 : DecCfg<M, D, S8>::NC][4],
+                                             const Ring<M, D, S8, TB> &ring,
+                                             uint32_t (&afr)[DecCfg<M, D, S8, TB>::A_SMEM ? 1 : DecCfg<M, D, S8, TB>::NC][4],
                                              float &hscale, int &usum) {
-  using C = DecCfg<M, D, S8>;
+  using C = DecCfg<M, D, S8, TB>;
   auto put = [&](int c, const uint32_t (&a4)[4]) {
     if constexpr (C::A_SMEM) {
       const int lane = (threadIdx.x & 31);
@@ -476,10 +531,13 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
     }
   };
   if constexpr (!S8) {
-    if constexpr (M >= 128) {
+    if constexpr (C::CODE_BITS >= 128) {
 #pragma unroll
-      for (int lw = 0; lw < LaneRuns<M>::WORDS; ++lw) {
-        const float *src = urow + 32 * (t * LaneRuns<M>::WORDS + lw);
+      for (int lw = 0; lw < C::LW; ++lw) {
+        // code word of the lane's run lw: contiguous runs, or (cell planes)
+        // interleaved so that run lw of the four lanes is one plane
+        const int word = TB ? 4 * lw + t : t * C::LW + lw;
+        const float *src = urow + 32 * word;
         float4 x[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
@@ -606,10 +664,10 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
   if constexpr (C::A_SMEM) __syncwarp();
 }
 
-template <int M, int D, bool S8, bool PAGED>
+template <int M, int D, bool S8, bool PAGED, int TB = 0>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
     decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
-  using C = DecCfg<M, D, S8>;
+  using C = DecCfg<M, D, S8, TB>;
   extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -627,8 +685,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   const int g = lane >> 2;  // group id: head row / key column / dim row
   const int t = lane & 3;   // thread in group
   const uint32_t cta = (smem_u32(dsmem_raw) + 1023u) & ~1023u;
-  const Ring<M, D, S8> ring{cta + wid * C::WARP_BYTES,
-                        cta + C::OFF_NORM + wid * C::STAGES * DEC_NORM_AREA,
+  const Ring<M, D, S8, TB> ring{cta + wid * C::WARP_BYTES,
+                        cta + C::OFF_NORM + wid * C::STAGES * C::NORM_AREA,
                         cta + C::OFF_BAR + wid * C::STAGES * 8};
 
   const int64_t bbeg = (int64_t)w * NB / Wn;
@@ -669,7 +727,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       // the block holding the key this call appends is written by the prep
       // kernel: copy it only after the wait below
       if (PAGED && p.append && ipos.blk == ipos.nb - 1) break;
-      issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+      issue_block<M, D, S8, PAGED, TB>(p, maps, ring, ipos, s, lane);
       pos_next<PAGED>(p, ipos);
       if constexpr (PAGED) load_page(ipos);
       ++issued;
@@ -682,7 +740,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   // their way
   griddep_wait();
   for (int s = issued; s < C::STAGES && s < nblk; ++s) {
-    issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+    issue_block<M, D, S8, PAGED, TB>(p, maps, ring, ipos, s, lane);
     pos_next<PAGED>(p, ipos);
     if constexpr (PAGED) load_page(ipos);
   }
@@ -752,8 +810,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
       for (int dt = 0; dt < C::DT; ++dt)
         acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
-      const float *urow = p.U + ((int64_t)b_idx * p.Hq + hq0 + g) * M;
-      build_afrags<M, D, S8>(urow, g < Gg, t, ring, afr, hscale, usum);
+      const float *urow = p.U + ((int64_t)b_idx * p.Hq + hq0 + g) * C::CODE_BITS;
+      build_afrags<M, D, S8, TB>(urow, g < Gg, t, ring, afr, hscale, usum);
       if constexpr (C::A_SMEM) __syncwarp();
     }
 
@@ -787,7 +845,11 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
       const uint32_t kp = sg + (kg * 8 + g) * C::KEY_SIGN_BYTES;
-      if constexpr (C::LW == 4) {
+      if constexpr (TB > 0) {
+#pragma unroll
+        for (int lw = 0; lw < C::LW; ++lw)
+          asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][lw]) : "r"(kp + (4 * lw + t) * 4));
+      } else if constexpr (C::LW == 4) {
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
                      : "=r"(wd[kg][0]), "=r"(wd[kg][1]), "=r"(wd[kg][2]), "=r"(wd[kg][3])
                      : "r"(kp + t * 16));
@@ -803,7 +865,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     }
 
     // ---- raw estimator sum_i u_i sign_i for head g, keys kg*8 + 2t + j
-    float raw[4][2];
+    // (cell-plane codes: raw over the planes, rawq over the residual signs)
+    float raw[4][2], rawq[4][2];
     if constexpr (S8) {
       int sc[4][4];
 #pragma unroll
@@ -843,10 +906,14 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
         for (int j = 0; j < 2; ++j)
           raw[kg][j] = hscale * (float)(2 * (sc[kg][j] * 256 + sc[kg][j + 2]) - usum);
     } else {
-      float sc[4][4];
+      float sc[4][4], sq[4][4];
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0.f;
-      const int pbase = (M >= 128) ? 0 : 8 * (t & 1);
+      if constexpr (TB > 0) {
+#pragma unroll
+        for (int kg = 0; kg < 4; ++kg) sq[kg][0] = sq[kg][1] = sq[kg][2] = sq[kg][3] = 0.f;
+      }
+      const int pbase = (C::CODE_BITS >= 128) ? 0 : 8 * (t & 1);
 #pragma unroll
       for (int c = 0; c < C::NC; ++c) {
         uint32_t a0, a1, a2, a3;
@@ -862,7 +929,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
         for (int kg = 0; kg < 4; ++kg) {
           uint32_t w0, w1;
           int p0, p1;
-          if constexpr (M >= 128) {
+          if constexpr (C::CODE_BITS >= 128) {
             w0 = wd[kg][q0 >> 4]; p0 = q0 & 15;
             w1 = wd[kg][q1 >> 4]; p1 = q1 & 15;
           } else {
@@ -870,29 +937,47 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           }
           const uint32_t b0 = ((w0 << (15 - p0)) & 0x80008000u) ^ 0xBF80BF80u;
           const uint32_t b1 = ((w1 << (15 - p1)) & 0x80008000u) ^ 0xBF80BF80u;
-          mma_bf16_16816(sc[kg], a0, a1, a2, a3, b0, b1);
+          if (TB > 0 && c >= C::NC_MSE)
+            mma_bf16_16816(sq[kg], a0, a1, a2, a3, b0, b1);
+          else
+            mma_bf16_16816(sc[kg], a0, a1, a2, a3, b0, b1);
         }
       }
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) raw[kg][j] = sc[kg][j] + sc[kg][j + 2];
+        for (int j = 0; j < 2; ++j) {
+          raw[kg][j] = sc[kg][j] + sc[kg][j + 2];
+          if constexpr (TB > 0) rawq[kg][j] = sq[kg][j] + sq[kg][j + 2];
+        }
     }
 
     // ---- estimator, masking, online softmax (head g, keys kg*8 + 2t + j)
     float l2[4][2];
     float bmax = -INFINITY;
+    constexpr int NG = 16 / C::NORM_BYTES;  // keys per 16-byte norm group
     const uint32_t nrow =
-        ring.norm(s) + (maps.tma_codes ? 0u : (uint32_t)((kv_base + key0) & 7) * 2);
+        ring.norm(s) +
+        (maps.tma_codes ? 0u : (uint32_t)((kv_base + key0) & (NG - 1)) * C::NORM_BYTES);
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int key = kg * 8 + 2 * t + j;
-        unsigned short hb;
-        asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(hb) : "r"(nrow + key * 2));
-        const float nk = __half2float(__ushort_as_half(hb));
-        const float sval = (p.coef * nk) * raw[kg][j];
+        float sval;
+        if constexpr (TB > 0) {
+          // s = ||k|| (<w, c[cell]> + sqrt(pi/2)/m ||rt|| <S w, sign(S rt)>)
+          uint32_t nb;
+          asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(nb) : "r"(nrow + key * 4));
+          const float nk = __half2float(__ushort_as_half((unsigned short)(nb & 0xFFFFu)));
+          const float nr = __half2float(__ushort_as_half((unsigned short)(nb >> 16)));
+          sval = nk * fmaf(p.coef * nr, rawq[kg][j], raw[kg][j]);
+        } else {
+          unsigned short hb;
+          asm volatile("ld.shared.u16 %0, [%1];\n" : "=h"(hb) : "r"(nrow + key * 2));
+          const float nk = __half2float(__ushort_as_half(hb));
+          sval = (p.coef * nk) * raw[kg][j];
+        }
         l2[kg][j] = sval * p.scale_log2;
         if (p.scores != nullptr && key < nval && g < Gg)
           p.scores[((int64_t)b_idx * p.Hq + hq0 + g) * p.score_stride + key0 + key] = sval;
@@ -954,7 +1039,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // ---- refill this stage with the block STAGES ahead
     __syncwarp();
     if (i + C::STAGES < nblk) {
-      issue_block<M, D, S8, PAGED>(p, maps, ring, ipos, s, lane);
+      issue_block<M, D, S8, PAGED, TB>(p, maps, ring, ipos, s, lane);
       pos_next<PAGED>(p, ipos);
       if constexpr (PAGED) load_page(ipos);
     }
@@ -1214,7 +1299,9 @@ bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d, Deco
 
 // Tensor maps of one call (see DecMaps).
 static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
-                      const uint16_t *norms, int64_t units_kv, int64_t T, int m, int d) {
+                      const uint16_t *norms, int64_t units_kv, int64_t T, int m, int d,
+                      int code_bytes = 0, int norm_bytes = 2) {
+  if (code_bytes == 0) code_bytes = m / 8;
   auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!fn) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
@@ -1229,24 +1316,26 @@ static bool make_maps(DecMaps *mp, const uint16_t *V, const uint32_t *signs,
       return false;
   }
   mp->tma_codes = 0;
-  mp->sign_elem = (m > 256) ? 8 : 4;
+  mp->sign_elem = (DEC_KB * code_bytes / 4 > 256) ? 8 : 4;
   if (T % 8 != 0) return true;  // per-unit rows not 16-byte aligned: cp.async path
-  {  // codes [units][T * m/8 bytes] as 4- or 8-byte elements, one block per box
+  {  // codes [units][T * code_bytes] as 4- or 8-byte elements, one block per box
     const int es = mp->sign_elem;
-    cuuint64_t dims[2] = {(cuuint64_t)(T * (m / 8) / es), (cuuint64_t)units_kv};
-    cuuint64_t strides[1] = {(cuuint64_t)T * (m / 8)};
-    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * (m / 8) / es), 1};
+    cuuint64_t dims[2] = {(cuuint64_t)(T * code_bytes / es), (cuuint64_t)units_kv};
+    cuuint64_t strides[1] = {(cuuint64_t)T * code_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * code_bytes / es), 1};
     if (fn(&mp->sign, es == 8 ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
            2, const_cast<uint32_t *>(signs), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return true;
   }
-  {  // norms [units][T] binary16, 32 per box
+  {  // norms [units][T] binary16 (or binary16 pairs as 4-byte elements), 32 per box
     cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)units_kv};
-    cuuint64_t strides[1] = {(cuuint64_t)T * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)T * norm_bytes};
     cuuint32_t box[2] = {(cuuint32_t)DEC_KB, 1};
-    if (fn(&mp->norm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(norms), dims,
+    if (fn(&mp->norm,
+           norm_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+           const_cast<uint16_t *>(norms), dims,
            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return true;
@@ -1298,11 +1387,11 @@ static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *par
 }
 
 // Launch the scorer (one wave, <= the plan's warp bound) and the combine.
-template <int M, int D, bool S8, bool PAGED>
+template <int M, int D, bool S8, bool PAGED, int TB = 0>
 static cudaError_t launch_scorer_combine(const DecodePlan &pl, DecParams &p, const DecMaps &maps,
                                          uint16_t *out, cudaStream_t stream) {
-  using C = DecCfg<M, D, S8>;
-  auto kern = decode_scorer_kernel<M, D, S8, PAGED>;
+  using C = DecCfg<M, D, S8, TB>;
+  auto kern = decode_scorer_kernel<M, D, S8, PAGED, TB>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::CTA_BYTES);
   if (e != cudaSuccess) return e;
@@ -1347,6 +1436,62 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   DecParams p;
   fill_params(p, pl, U, partials, signs, norms, scores, softmax_scale, M, err);
   return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
+}
+
+bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int bits,
+                            DecodePlan *pl) {
+  if (m != 128 || d != 128 || bits < 1 || bits > 2) return false;
+  if (!plan_common(B, Hq, Hkv, T, m, d, pl)) return false;
+  pl->u_bytes = round_up((size_t)B * Hq * (bits * d + m) * sizeof(float), 256);
+  pl->total_bytes = pl->u_bytes + pl->partial_bytes;
+  return true;
+}
+
+template <int TB>
+static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bool q_f32,
+                                         const float *Pinv, const uint16_t *S,
+                                         const uint32_t *codes, const uint16_t *norms,
+                                         const uint16_t *V, const double *walsh,
+                                         float softmax_scale, uint16_t *out, float *scores,
+                                         void *workspace, cudaStream_t stream) {
+  constexpr int M = 128, D = 128;
+  float *U = reinterpret_cast<float *>(workspace);
+  float *partials =
+      reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
+  DecMaps maps;
+  if (!make_maps(&maps, V, codes, norms, (int64_t)pl.B * pl.Hkv, pl.T, M, D,
+                 DecCfg<M, D, false, TB>::KEY_SIGN_BYTES, 4))
+    return cudaErrorInvalidValue;
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
+  const int bh = pl.B * pl.Hq;
+  const int qctas = (bh + PROJ_VECS - 1) / PROJ_VECS;
+  const float wc0 = (float)walsh[0], wc1 = (float)walsh[1];
+  if (q_f32)
+    turbo_qproj_kernel<M, D, TB, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh,
+                                                                          wc0, wc1);
+  else
+    turbo_qproj_kernel<M, D, TB, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh,
+                                                                           wc0, wc1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  DecParams p;
+  fill_params(p, pl, U, partials, codes, norms, scores, softmax_scale, M, err);
+  return launch_scorer_combine<M, D, false, false, TB>(pl, p, maps, out, stream);
+}
+
+cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, bool q_f32,
+                                const float *Pinv, const uint16_t *S, const uint32_t *codes,
+                                const uint16_t *norms, const uint16_t *V, const double *walsh,
+                                float softmax_scale, uint16_t *out, float *scores,
+                                void *workspace, cudaStream_t stream) {
+  if (bits == 1)
+    return launch_turbo_decode_t<1>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
+                                    softmax_scale, out, scores, workspace, stream);
+  if (bits == 2)
+    return launch_turbo_decode_t<2>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
+                                    softmax_scale, out, scores, workspace, stream);
+  return cudaErrorNotSupported;
 }
 
 cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S, float *U,

@@ -1,6 +1,7 @@
 // jl_internal.h -- launchers behind the C ABI (host side, internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -43,6 +44,24 @@ cudaError_t launch_search(const void *Q, bool q_f32, int nq, const uint16_t *S, 
                           int32_t *out_idx, float *out_scores, void *workspace,
                           cudaStream_t stream);
 
+// 2-D bf16 tensor map [rows][cols] (pitch in elements), boxes of 64 columns x
+// box_rows rows, 128-byte swizzle (quantize_tc.cu).
+namespace tc {
+bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols,
+              uint64_t pitch_elems, uint32_t box_rows);
+}
+
+// TurboQuant-prod (turbo_tc.cu): the stage-one codebook (host, cached; false
+// for unsupported d / bits), its single-bit Walsh coefficients, the rotation
+// and its inverse, and the tensor-core quantizer (d = m = 128, bf16 keys).
+bool turbo_codebook(int d, int bits, float *centroids, double *walsh);
+size_t turbo_rotation_workspace_bytes(int d);
+cudaError_t launch_turbo_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t seed, void *ws,
+                                  cudaStream_t stream);
+cudaError_t launch_turbo_quantize(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *Pi,
+                                  const uint16_t *S, int m, int d, int bits, uint32_t *codes,
+                                  uint16_t *norms, cudaStream_t stream);
+
 // Decode: work split shared by the workspace query and the launch.
 struct DecodePlan {
   int B, Hq, Hkv, m, d;
@@ -62,6 +81,15 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
                       DecodePlan *plan);
 bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d,
                      DecodePlan *plan);
+
+// TurboQuant-prod decode (decode.cu): d = m = 128, bits 1 or 2.
+bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int bits,
+                            DecodePlan *plan);
+cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, bool q_f32,
+                                const float *Pinv, const uint16_t *S, const uint32_t *codes,
+                                const uint16_t *norms, const uint16_t *V, const double *walsh,
+                                float softmax_scale, uint16_t *out, float *scores,
+                                void *workspace, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodePlan &p, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,

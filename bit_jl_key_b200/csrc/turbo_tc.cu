@@ -1,0 +1,712 @@
+// turbo_tc.cu -- TurboQuant-prod keys: codebook, rotation, quantizer.
+//
+// "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+// Quantization":
+//  * section "Random rotation, and what high dimensions do to your
+//    intuitions": Pi from orthogonalising a Gaussian matrix; a coordinate of a
+//    rotated unit vector has the density
+//        f(x) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - x^2)^((d-3)/2);
+//  * section "TurboQuant: bridging MSE and inner product, in two stages": the
+//    Lloyd-Max codebook of f for the first b-1 bits of every rotated
+//    coordinate, then QJL on the residual.
+//
+// Codebook (host, float64, once per (d, bits)): Lloyd's two conditions
+// alternated on the positive half of the even density -- boundaries at the
+// midpoints of neighbouring centroids, each centroid the mean of f over its
+// cell.  Cell masses by composite Gauss-Legendre quadrature of f, first
+// moments from the antiderivative of x (1 - x^2)^((d-3)/2).
+//
+// Rotation (device, float64, init time): G from the sketch generator,
+// Gram-Schmidt column by column with one re-orthogonalisation pass (the
+// positive-diagonal QR factor), rounded to bf16; then the inverse of the bf16
+// matrix by Newton-Schulz iterations X <- X (2I - Pi X) from X = Pi^T.
+//
+// Quantizer (tensor cores), per tile of 128 keys:
+//   MMA 1   D = K Pi^T             (K: TMA-loaded bf16 tile; Pi resident)
+//   epilogue A  (one thread per key): y = D / ||k||; cells by a branch-free
+//           binary search over the boundaries (the cell bits are the code's
+//           planes); rt = bf16(y - c[cell]) written to tensor memory as the
+//           A operand of
+//   MMA 2   D = rt S^T             (S resident; D reuses MMA 1's columns)
+//   epilogue B  sign words of D.
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 epilogue (TMEM lane quadrant
+// warp % 4).  Two accumulators: the epilogue runs A of tile t, then B of tile
+// t - 1, so MMA 2 of one tile overlaps epilogue A of the next.  Every wait is
+// bounded; a wait that runs out records DERR_TC_WAIT_TIMEOUT, tells the other
+// roles to stop, and the CTA drains its copies and frees its tensor memory.
+#include "jl_common.cuh"
+#include "jl_internal.h"
+#include "jl_rng.cuh"
+#include "jl_tc.cuh"
+
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+namespace jlk {
+namespace turbo {
+
+// --------------------------------------------------------------------------
+// codebook (host)
+
+struct GaussLegendre {
+  std::vector<double> x, w;  // nodes and weights on [-1, 1]
+  explicit GaussLegendre(int n) : x(n), w(n) {
+    // Newton's method on the Legendre polynomial P_n from the Chebyshev-like
+    // initial guesses cos(pi (i + 3/4) / (n + 1/2))
+    for (int i = 0; i < (n + 1) / 2; ++i) {
+      double z = cos(M_PI * (i + 0.75) / (n + 0.5)), dp = 0.0;
+      for (int it = 0; it < 100; ++it) {
+        double p0 = 1.0, p1 = z;
+        for (int k = 2; k <= n; ++k) {
+          const double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+          p0 = p1;
+          p1 = p2;
+        }
+        dp = n * (z * p1 - p0) / (z * z - 1.0);
+        const double dz = p1 / dp;
+        z -= dz;
+        if (fabs(dz) < 1e-16) break;
+      }
+      x[i] = -z;
+      x[n - 1 - i] = z;
+      w[i] = w[n - 1 - i] = 2.0 / ((1.0 - z * z) * dp * dp);
+    }
+  }
+};
+
+struct Density {
+  int d;
+  double logc;  // log of Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2))
+  explicit Density(int dd)
+      : d(dd), logc(lgamma(dd / 2.0) - 0.5 * log(M_PI) - lgamma((dd - 1) / 2.0)) {}
+  double f(double x) const {
+    const double s = 1.0 - x * x;
+    if (s <= 0.0) return d == 3 ? exp(logc) : 0.0;
+    return exp(logc + 0.5 * (d - 3) * log(s));
+  }
+  // int_lo^hi x f(x) dx
+  double moment(double lo, double hi) const {
+    auto F = [&](double x) {
+      const double s = 1.0 - x * x;
+      return s <= 0.0 ? 0.0 : -exp(0.5 * (d - 1) * log(s)) / (d - 1);
+    };
+    return exp(logc) * (F(hi) - F(lo));
+  }
+  // int_lo^hi f(x) dx: composite Gauss-Legendre over panels of width <=
+  // 1/(8 sqrt(d)) (a fraction of the density's spread)
+  double mass(double lo, double hi, const GaussLegendre &gl) const {
+    // beyond 15 standard deviations (1/sqrt(d) each) f is below e^-110 of its
+    // peak: leave that tail out of the panels
+    hi = fmin(hi, fmax(0.0, 15.0 / sqrt((double)d)));
+    const double width = hi - lo;
+    if (width <= 0.0) return 0.0;
+    const double pw = 0.125 / sqrt((double)d);
+    const int panels = (int)ceil(width / pw) < 1 ? 1 : (int)ceil(width / pw);
+    const double h = width / panels;
+    double s = 0.0;
+    for (int p = 0; p < panels; ++p) {
+      const double a = lo + p * h, mid = a + 0.5 * h;
+      double ps = 0.0;
+      for (size_t k = 0; k < gl.x.size(); ++k) ps += gl.w[k] * f(mid + 0.5 * h * gl.x[k]);
+      s += 0.5 * h * ps;
+    }
+    return s;
+  }
+};
+
+// Positive half a_0 < ... < a_{H-1} of the symmetric L = 2H-level quantizer.
+static std::vector<double> lloyd_max_half(int d, int bits) {
+  const int H = 1 << (bits - 1);
+  const Density den(d);
+  const GaussLegendre gl(16);
+  std::vector<double> a(H), t(H + 1);
+  const double sd = 1.0 / sqrt((double)d);
+  for (int i = 0; i < H; ++i) a[i] = fmin((i + 0.5) * 2.5 * sd / H, 1.0 - (H - i) * 1e-3);
+  // stop once a sweep moves no centroid by more than 1e-14 of the largest
+  // (far below the float rounding of the result)
+  for (int it = 0; it < 100000; ++it) {
+    t[0] = 0.0;
+    t[H] = 1.0;
+    for (int i = 1; i < H; ++i) t[i] = 0.5 * (a[i - 1] + a[i]);
+    double move = 0.0;
+    for (int i = 0; i < H; ++i) {
+      const double nm = den.moment(t[i], t[i + 1]) / den.mass(t[i], t[i + 1], gl);
+      move = fmax(move, fabs(nm - a[i]));
+      a[i] = nm;
+    }
+    if (move <= 1e-14 * a[H - 1]) break;
+  }
+  return a;
+}
+
+struct Codebook {
+  int L = 0;
+  double c[8];      // centroids, ascending
+  float cf[8];      // as float
+  float thr[7];     // float((c_i + c_{i+1}) / 2)
+  double walsh[3];  // c_j = sum_p walsh[p] * (2 bit_p(j) - 1)  (bits <= 2)
+};
+
+static const Codebook *codebook(int d, int bits) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, Codebook> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(d, bits);
+  auto it = cache.find(key);
+  if (it != cache.end()) return &it->second;
+  const std::vector<double> a = lloyd_max_half(d, bits);
+  Codebook cb;
+  const int H = (int)a.size();
+  cb.L = 2 * H;
+  for (int i = 0; i < H; ++i) {
+    cb.c[H + i] = a[i];
+    cb.c[H - 1 - i] = -a[i];
+  }
+  for (int j = 0; j < cb.L; ++j) cb.cf[j] = (float)cb.c[j];
+  for (int j = 0; j + 1 < cb.L; ++j) cb.thr[j] = (float)(0.5 * (cb.c[j] + cb.c[j + 1]));
+  // Walsh coefficients of the single-bit terms: (1/L) sum_j c_j e_p(j)
+  for (int p = 0; p < 3; ++p) {
+    double s = 0.0;
+    if (p < bits)
+      for (int j = 0; j < cb.L; ++j) s += cb.c[j] * (((j >> p) & 1) ? 1.0 : -1.0);
+    cb.walsh[p] = s / cb.L;
+  }
+  return &cache.emplace(key, cb).first->second;
+}
+
+// --------------------------------------------------------------------------
+// rotation (device, float64)
+
+constexpr int ROT_THREADS = 256;
+
+// One CTA.  Shared memory: Qc (column j of Q contiguous), v, r.
+template <int D>
+__global__ void __launch_bounds__(ROT_THREADS) rot_gram_schmidt_kernel(uint64_t seed,
+                                                                        uint16_t *Pi,
+                                                                        double *Pit64) {
+  extern __shared__ double rot_smem[];
+  double *Qc = rot_smem;        // [D][D]
+  double *v = Qc + D * D;       // [D]
+  double *r = v + D;            // [D]
+  double *red = r + D;          // [ROT_THREADS / 32]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = ROT_THREADS / 32;
+  for (int j = 0; j < D; ++j) {
+    if (tid < D) v[tid] = gauss_at(seed, (uint64_t)tid * D + j);  // G[tid][j]
+    __syncthreads();
+    for (int pass = 0; pass < 2; ++pass) {
+      // r_i = <q_i, v> for i < j
+      for (int i = warp; i < j; i += NW) {
+        double s = 0.0;
+        for (int k = lane; k < D; k += 32) s += Qc[i * D + k] * v[k];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) r[i] = s;
+      }
+      __syncthreads();
+      if (tid < D) {
+        double s = 0.0;
+        for (int i = 0; i < j; ++i) s += Qc[i * D + tid] * r[i];
+        v[tid] -= s;
+      }
+      __syncthreads();
+    }
+    double s = tid < D ? v[tid] * v[tid] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[warp] = s;
+    __syncthreads();
+    double nn = 0.0;
+    for (int w = 0; w < NW; ++w) nn += red[w];
+    const double inv = 1.0 / sqrt(nn);
+    if (tid < D) Qc[j * D + tid] = v[tid] * inv;
+    __syncthreads();
+  }
+  for (int e = tid; e < D * D; e += ROT_THREADS) {
+    const int i = e / D, j = e - i * D;  // Pi[i][j] = Q[i][j] = Qc[j][i]
+    const uint16_t b = bf16_from_f64_bits(Qc[j * D + i]);
+    Pi[e] = b;
+    Pit64[e] = (double)__uint_as_float((uint32_t)b << 16);
+  }
+}
+
+// out = alpha * A B + beta * C  (n x n, row-major float64); 16 x 16 tiles
+__global__ void rot_gemm_kernel(const double *A, const double *B, const double *C,
+                                double alpha, double beta, double *out, int n) {
+  __shared__ double ta[16][17], tb[16][17];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int row = blockIdx.y * 16 + ty, col = blockIdx.x * 16 + tx;
+  double s = 0.0;
+  for (int k0 = 0; k0 < n; k0 += 16) {
+    ta[ty][tx] = A[row * n + k0 + tx];
+    tb[ty][tx] = B[(k0 + ty) * n + col];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) s += ta[ty][k] * tb[k][tx];
+    __syncthreads();
+  }
+  out[row * n + col] = alpha * s + (C ? beta * C[row * n + col] : 0.0);
+}
+
+__global__ void rot_transpose_kernel(const double *A, double *out, int n) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < n * n) {
+    const int i = e / n, j = e - i * n;
+    out[j * n + i] = A[e];
+  }
+}
+
+__global__ void rot_to_f32_kernel(const double *A, float *out, int n) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < n * n) out[e] = (float)A[e];
+}
+
+constexpr int NS_ITERS = 6;
+
+size_t rotation_workspace_bytes(int d) {
+  if (d != 64 && d != 128) return 0;
+  return 4 * (size_t)d * d * sizeof(double);
+}
+
+cudaError_t launch_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t seed, void *ws,
+                            cudaStream_t stream) {
+  double *P64 = reinterpret_cast<double *>(ws);
+  double *X = P64 + (size_t)d * d, *Xn = X + (size_t)d * d, *T = Xn + (size_t)d * d;
+  const size_t smem = ((size_t)d * d + 2 * d + ROT_THREADS / 32) * sizeof(double);
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(rot_gram_schmidt_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rot_gram_schmidt_kernel<128><<<1, ROT_THREADS, smem, stream>>>(seed, Pi, P64);
+  } else {
+    rot_gram_schmidt_kernel<64><<<1, ROT_THREADS, smem, stream>>>(seed, Pi, P64);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nn = d * d;
+  rot_transpose_kernel<<<(nn + 255) / 256, 256, 0, stream>>>(P64, X, d);
+  const dim3 g(d / 16, d / 16), b(16, 16);
+  for (int it = 0; it < NS_ITERS; ++it) {
+    rot_gemm_kernel<<<g, b, 0, stream>>>(P64, X, nullptr, 1.0, 0.0, T, d);  // T = Pi X
+    rot_gemm_kernel<<<g, b, 0, stream>>>(X, T, X, -1.0, 2.0, Xn, d);        // 2X - X T
+    double *tmp = X;
+    X = Xn;
+    Xn = tmp;
+  }
+  rot_to_f32_kernel<<<(nn + 255) / 256, 256, 0, stream>>>(X, Pinv, d);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------------------
+// quantizer (tensor cores), d = m = 128
+
+constexpr int BM = 128;
+constexpr int QD = 128;   // head dim = rotation size
+constexpr int QM = 128;   // residual sketch rows
+
+template <int TB>
+struct QCfg {
+  static constexpr int KCH = QD / 64;
+  static constexpr int A_CHUNK = BM * 128;      // one 64-column swizzle column of a tile
+  static constexpr int A_STAGE = BM * QD * 2;   // 32 KB
+  static constexpr int W_CHUNK = 128 * 128;     // 128 rows x 64 columns of Pi or S
+  static constexpr int W_BYTES = 128 * QD * 2;  // 32 KB
+  static constexpr int STAGES = 4;
+  static constexpr int OFF_PI = 0;
+  static constexpr int OFF_S = W_BYTES;
+  static constexpr int OFF_A = 2 * W_BYTES;
+  static constexpr int OFF_BAR = OFF_A + STAGES * A_STAGE;
+  static constexpr int NBAR = 2 * STAGES + 4 * 2 + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+  static constexpr int THREADS = 6 * 32;
+  static constexpr int WORDS = TB * QD / 32 + QM / 32;
+  static constexpr int PW = QD / 32;            // words per plane
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int A2_COL = 256;            // bf16 residual rows (64 columns each)
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct QParams {
+  int64_t n;
+  int64_t num_tiles;
+  uint32_t *codes;
+  uint32_t *norms;  // (||k|| | ||rt|| << 16) binary16 pairs
+  int *err;
+  float thr[7];
+  float cent[8];
+};
+
+// Cell of y by binary search over the boundaries (ties go to the lower cell);
+// the bits of the cell index go to the plane words at bit e; returns
+// y - c[cell].
+template <int TB>
+__device__ __forceinline__ float cell_residual(float y, const float (&t)[7], const float (&c)[8],
+                                               uint32_t (&pw)[TB], int e) {
+  if constexpr (TB == 1) {
+    const bool b0 = y > t[0];
+    pw[0] |= (uint32_t)b0 << e;
+    return y - (b0 ? c[1] : c[0]);
+  } else if constexpr (TB == 2) {
+    const bool b1 = y > t[1];
+    const bool b0 = y > (b1 ? t[2] : t[0]);
+    pw[1] |= (uint32_t)b1 << e;
+    pw[0] |= (uint32_t)b0 << e;
+    const float hi = b1 ? c[3] : c[1], lo = b1 ? c[2] : c[0];
+    return y - (b0 ? hi : lo);
+  } else {
+    const bool b2 = y > t[3];
+    const bool b1 = y > (b2 ? t[5] : t[1]);
+    const float t0 = b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]);
+    const bool b0 = y > t0;
+    pw[2] |= (uint32_t)b2 << e;
+    pw[1] |= (uint32_t)b1 << e;
+    pw[0] |= (uint32_t)b0 << e;
+    const float c01 = b0 ? c[1] : c[0], c23 = b0 ? c[3] : c[2];
+    const float c45 = b0 ? c[5] : c[4], c67 = b0 ? c[7] : c[6];
+    const float lo = b1 ? c23 : c01, hi = b1 ? c67 : c45;
+    return y - (b2 ? hi : lo);
+  }
+}
+
+template <int TB>
+__global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
+    turbo_quantize_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                          const __grid_constant__ CUtensorMap tmap_pi,
+                          const __grid_constant__ CUtensorMap tmap_s, const QParams p) {
+  using C = QCfg<TB>;
+  extern __shared__ uint8_t tq_smem_raw[];
+  const uint32_t raw = smem_u32(tq_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *gbase = tq_smem_raw + (base - raw);
+  const uint32_t sPi = base + C::OFF_PI, sS = base + C::OFF_S, sA = base + C::OFF_A;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  auto kfull = [&](int s) { return bar0 + 8u * s; };
+  auto kempty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto d1full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+  auto afull = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
+  auto d2full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 4 + a); };
+  auto dempty = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 6 + a); };
+  const uint32_t wfull = bar0 + 8u * (2 * C::STAGES + 8);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
+  volatile int *abort_flag =
+      reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(kfull(s), 1);
+      mbar_init(kempty(s), 1 + 4);  // MMA commit + 4 epilogue warps (norms)
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(d1full(a), 1);
+      mbar_init(afull(a), 4);
+      mbar_init(d2full(a), 1);
+      mbar_init(dempty(a), 4);
+    }
+    mbar_init(wfull, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
+        "tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::"r"(
+            smem_u32(tmem_holder)),
+        "n"(C::TMEM_COLS)
+        : "memory");
+  }
+  tcx::fence_before();
+  __syncthreads();
+  tcx::fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  // tiles of this CTA: blockIdx.x + t * gridDim.x, t < cnt
+  const int64_t cnt =
+      p.num_tiles > blockIdx.x ? (p.num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(wfull, 2 * C::W_BYTES);
+      for (int kc = 0; kc < C::KCH; ++kc) {
+        tma_load_2d(sPi + kc * C::W_CHUNK, &tmap_pi, kc * 64, 0, wfull);
+        tma_load_2d(sS + kc * C::W_CHUNK, &tmap_s, kc * 64, 0, wfull);
+      }
+      int64_t t = 0;
+      for (; t < cnt; ++t) {
+        const int s = (int)(t % C::STAGES);
+        const uint32_t ph = (uint32_t)((t / C::STAGES) & 1);
+        if (!tcx::wait_phase(kempty(s), ph ^ 1u, abort_flag, p.err)) break;
+        const int64_t tile = blockIdx.x + t * gridDim.x;
+        mbar_expect_tx(kfull(s), C::A_STAGE);
+        for (int kc = 0; kc < C::KCH; ++kc)
+          tma_load_2d(sA + s * C::A_STAGE + kc * C::A_CHUNK, &tmap_k, kc * 64,
+                      (int)(tile * BM), kfull(s));
+      }
+      for (int64_t j = (t > C::STAGES ? t - C::STAGES : 0); j < t; ++j)
+        tcx::drain_wait(kfull((int)(j % C::STAGES)), (uint32_t)((j / C::STAGES) & 1));
+      tcx::drain_wait(wfull, 0);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tcx::idesc_f16(BM, 128, 1);
+      bool ok = tcx::wait_phase(wfull, 0, abort_flag, p.err);
+      int64_t issued2 = 0;
+      for (int64_t t = 0; ok && t <= cnt; ++t) {
+        if (t < cnt) {
+          const int s = (int)(t % C::STAGES);
+          const int a = (int)(t & 1);
+          if (!tcx::wait_phase(kfull(s), (uint32_t)((t / C::STAGES) & 1), abort_flag, p.err) ||
+              !tcx::wait_phase(dempty(a), (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tcx::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < QD / 16; ++kk) {
+            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+            const uint64_t ad = tcx::desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
+            const uint64_t bd = tcx::desc_sw128(sPi + (kk >> 2) * C::W_CHUNK + koff);
+            tcx::mma_ss(tmem_base + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          tcx::commit(d1full(a));
+          tcx::commit(kempty(s));
+        }
+        if (t >= 1) {
+          const int64_t u = t - 1;
+          const int a = (int)(u & 1);
+          if (!tcx::wait_phase(afull(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tcx::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < QD / 16; ++kk) {
+            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+            const uint64_t bd = tcx::desc_sw128(sS + (kk >> 2) * C::W_CHUNK + koff);
+            tcx::mma_ts(tmem_base + a * 128, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
+                        kk > 0 ? 1u : 0u);
+          }
+          tcx::commit(d2full(a));
+          ++issued2;
+        }
+      }
+      // the last products must be complete before tensor memory is freed
+      if (issued2 > 0) {
+        const int64_t u = issued2 - 1;
+        tcx::drain_wait(d2full((int)(u & 1)), (uint32_t)((u >> 1) & 1));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: key row 32 * (warp % 4) + lane of each tile
+    const int q = warp & 3;
+    const int r = 32 * q + lane;
+    const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16);
+    float t[7], c[8];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) t[i] = p.thr[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = p.cent[i];
+    bool ok = true;
+    for (int64_t it = 0; ok && it <= cnt; ++it) {
+      if (it < cnt) {
+        // ---- A: norm, cells, residual of tile it
+        const int s = (int)(it % C::STAGES);
+        const int a = (int)(it & 1);
+        const int64_t row = (blockIdx.x + it * gridDim.x) * BM + r;
+        if (!tcx::wait_phase(kfull(s), (uint32_t)((it / C::STAGES) & 1), abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        float ss0 = 0.f, ss1 = 0.f;
+        {
+          const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + r * 128;
+#pragma unroll
+          for (int kc = 0; kc < C::KCH; ++kc)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(rowp + kc * C::A_CHUNK +
+                                                               ((ch ^ (r & 7)) << 4));
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w4[e] << 16);
+                const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+                ss0 = fmaf(lo, lo, ss0);
+                ss1 = fmaf(hi, hi, ss1);
+              }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(kempty(s));
+        const float nk = sqrtf(ss0 + ss1);
+        const float inv = nk > 0.f ? 1.f / nk : 0.f;
+        if (!tcx::wait_phase(d1full(a), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tcx::fence_after();
+        uint32_t planes[TB][C::PW];
+        float rs0 = 0.f, rs1 = 0.f;
+        uint32_t va[32], vb[32];
+        const uint32_t dcol = trow + (uint32_t)(a * 128);
+        const uint32_t acol = trow + (uint32_t)(C::A2_COL + a * 64);
+        auto chunk = [&](const uint32_t (&v)[32], int ch) {
+          uint32_t pw[TB];
+#pragma unroll
+          for (int pp = 0; pp < TB; ++pp) pw[pp] = 0u;
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float r0 = cell_residual<TB>(__uint_as_float(v[e]) * inv, t, c, pw, e);
+            const float r1 = cell_residual<TB>(__uint_as_float(v[e + 1]) * inv, t, c, pw, e + 1);
+            const uint32_t b = pack_bf16x2(r0, r1);
+            pk[e >> 1] = b;
+            const float lo = __uint_as_float(b << 16), hi = __uint_as_float(b & 0xFFFF0000u);
+            rs0 = fmaf(lo, lo, rs0);
+            rs1 = fmaf(hi, hi, rs1);
+          }
+          tcx::st16(acol + 16 * ch, pk);
+#pragma unroll
+          for (int pp = 0; pp < TB; ++pp) planes[pp][ch] = pw[pp];
+        };
+        tcx::ld32(dcol, va);
+        tcx::ld_wait(va);
+        tcx::ld32(dcol + 32, vb);
+        chunk(va, 0);
+        tcx::ld_wait(vb);
+        tcx::ld32(dcol + 64, va);
+        chunk(vb, 1);
+        tcx::ld_wait(va);
+        tcx::ld32(dcol + 96, vb);
+        chunk(va, 2);
+        tcx::ld_wait(vb);
+        chunk(vb, 3);
+        tcx::st_wait();
+        tcx::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull(a));
+        if (row < p.n) {
+          uint32_t *dst = p.codes + row * C::WORDS;
+#pragma unroll
+          for (int pp = 0; pp < TB; ++pp)
+            *reinterpret_cast<uint4 *>(dst + pp * C::PW) =
+                make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
+          const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
+          const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
+          p.norms[row] = n16 | (r16 << 16);
+        }
+      }
+      if (it >= 1) {
+        // ---- B: residual sign words of tile it - 1
+        const int64_t u = it - 1;
+        const int a = (int)(u & 1);
+        const int64_t row = (blockIdx.x + u * gridDim.x) * BM + r;
+        if (!tcx::wait_phase(d2full(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tcx::fence_after();
+        uint32_t w[4];
+        uint32_t va[32], vb[32];
+        const uint32_t dcol = trow + (uint32_t)(a * 128);
+        tcx::ld32(dcol, va);
+        tcx::ld_wait(va);
+        tcx::ld32(dcol + 32, vb);
+        w[0] = tcx::sign_word(va);
+        tcx::ld_wait(vb);
+        tcx::ld32(dcol + 64, va);
+        w[1] = tcx::sign_word(vb);
+        tcx::ld_wait(va);
+        tcx::ld32(dcol + 96, vb);
+        w[2] = tcx::sign_word(va);
+        tcx::ld_wait(vb);
+        w[3] = tcx::sign_word(vb);
+        tcx::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dempty(a));
+        if (row < p.n)
+          *reinterpret_cast<uint4 *>(p.codes + row * C::WORDS + TB * C::PW) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+
+  tcx::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tcx::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
+                 "n"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+template <int TB>
+static cudaError_t launch_quantize_t(const uint16_t *K, int64_t n, int64_t ldk,
+                                     const uint16_t *Pi, const uint16_t *S, const Codebook &cb,
+                                     uint32_t *codes, uint16_t *norms, cudaStream_t stream) {
+  using C = QCfg<TB>;
+  CUtensorMap mk, mpi, ms;
+  if (!tc::make_map(&mk, K, (uint64_t)n, QD, (uint64_t)ldk, BM) ||
+      !tc::make_map(&mpi, Pi, QD, QD, QD, 128) || !tc::make_map(&ms, S, QM, QD, QD, 128))
+    return cudaErrorInvalidValue;
+  QParams p{};
+  p.n = n;
+  p.num_tiles = (n + BM - 1) / BM;
+  p.codes = codes;
+  p.norms = reinterpret_cast<uint32_t *>(norms);
+  p.err = device_error_ptr();
+  if (!p.err) return cudaErrorInvalidSymbol;
+  for (int i = 0; i < 7; ++i) p.thr[i] = i + 1 < cb.L ? cb.thr[i] : 0.f;
+  for (int i = 0; i < 8; ++i) p.cent[i] = i < cb.L ? cb.cf[i] : 0.f;
+  cudaError_t e = cudaFuncSetAttribute(turbo_quantize_kernel<TB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
+  turbo_quantize_kernel<TB><<<(int)grid, C::THREADS, C::SMEM, stream>>>(mk, mpi, ms, p);
+  return cudaGetLastError();
+}
+
+}  // namespace turbo
+
+bool turbo_codebook(int d, int bits, float *centroids, double *walsh) {
+  if (d < 3 || d > 4096 || bits < 1 || bits > 3) return false;
+  const turbo::Codebook *cb = turbo::codebook(d, bits);
+  if (centroids)
+    for (int j = 0; j < cb->L; ++j) centroids[j] = cb->cf[j];
+  if (walsh)
+    for (int p = 0; p < 3; ++p) walsh[p] = cb->walsh[p];
+  return true;
+}
+
+size_t turbo_rotation_workspace_bytes(int d) { return turbo::rotation_workspace_bytes(d); }
+
+cudaError_t launch_turbo_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t seed, void *ws,
+                                  cudaStream_t stream) {
+  return turbo::launch_rotation(Pi, Pinv, d, seed, ws, stream);
+}
+
+cudaError_t launch_turbo_quantize(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *Pi,
+                                  const uint16_t *S, int m, int d, int bits, uint32_t *codes,
+                                  uint16_t *norms, cudaStream_t stream) {
+  if (m != turbo::QM || d != turbo::QD) return cudaErrorNotSupported;
+  const turbo::Codebook *cb = turbo::codebook(d, bits);
+  switch (bits) {
+    case 1: return turbo::launch_quantize_t<1>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
+    case 2: return turbo::launch_quantize_t<2>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
+    case 3: return turbo::launch_quantize_t<3>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace jlk

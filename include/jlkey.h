@@ -322,6 +322,120 @@ JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,
                                        int d, float softmax_scale, uint16_t *out,
                                        float *scores, jl_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * TurboQuant-prod keys.
+ * Defines: "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+ * Quantization", sections "Random rotation, and what high dimensions do to
+ * your intuitions" (a rotation Pi from an orthogonalised Gaussian matrix; the
+ * density f(x) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - x^2)^((d-3)/2)
+ * of each coordinate of a rotated unit vector) and "TurboQuant: bridging MSE
+ * and inner product, in two stages" (b-1 bits per coordinate from the
+ * Lloyd-Max codebook of f, one more bit from QJL on the residual; unbiased).
+ *
+ * Per key k (d = 128; the residual sketch S is m x d with m = 128):
+ *   x = k / ||k||  (0 for k = 0),  y = Pi x  (Pi: the stored bf16 rotation)
+ *   cell_i = number of codebook boundaries strictly below y_i
+ *   rt = bf16(y - c[cell])           (nearest, ties to even)
+ *   code = cell bit planes, then sign(S rt);  norms = (||k||, ||rt||) binary16
+ * and per query q, with w = Pi^{-T} q (Pinv from jl_turbo_rotation_init):
+ *   s(q, k) = ||k|| * ( <w, c[cell]> + sqrt(pi/2)/m * ||rt|| * <S w, sign(S rt)> ).
+ * For an exactly orthogonal Pi the QJL stage in this rotated frame is the
+ * pages' construction in distribution (S Pi^T is again an i.i.d. Gaussian
+ * matrix); mapping the query with the inverse transpose of the stored Pi
+ * keeps <w, y> = <q, x> exact, so s is unbiased up to the bf16 rounding of
+ * the residual and the binary16 norms.
+ *
+ * Code layout, per key: words = mse_bits * d/32 + m/32 uint32; plane p
+ * (p < mse_bits) is words [p*d/32, (p+1)*d/32) and holds bit p of every
+ * coordinate's cell (coordinate i at bit i % 32 of word i / 32 of the
+ * plane); the QJL code follows (jl_quantize_keys layout).  norms: n x 2
+ * binary16, element 0 = ||k||, element 1 = ||rt||.
+ * -------------------------------------------------------------------------*/
+#define JL_TURBO_MAX_MSE_BITS 3
+
+/*
+ * jl_turbo_codebook -- the stage-one codebook: the 2^mse_bits centroids
+ * c_0 < ... < c_{L-1} of the Lloyd-Max quantizer of f (centroid = mean of f
+ * over its cell, cells bounded by the midpoints of neighbouring centroids),
+ * computed in float64 by this library and rounded to float.
+ *   centroids : out, HOST memory, 2^mse_bits floats.
+ * Errors: JL_ERR_INVALID_ARG (null), JL_ERR_UNSUPPORTED (d < 3, d > 4096,
+ * mse_bits outside [1, JL_TURBO_MAX_MSE_BITS]).
+ */
+JL_API int jl_turbo_codebook(int d, int mse_bits, float *centroids);
+
+/* Device scratch of jl_turbo_rotation_init (0 for unsupported d). */
+JL_API size_t jl_turbo_rotation_workspace_bytes(int d);
+
+/*
+ * jl_turbo_rotation_init -- the rotation and its query map from `seed`.
+ *   Pi   : out, device, d x d bf16, row-major, 16-byte aligned: Q of the
+ *          factorisation G = Q R with diag(R) > 0, G[i][j] the normal of
+ *          element i*d + j of the jl_sketch_init generator with this seed,
+ *          rounded to bf16 (nearest, ties to even).  Orthogonalised in
+ *          float64 (Gram-Schmidt with re-orthogonalisation).
+ *   Pinv : out, device, d x d fp32, row-major, 16-byte aligned: the inverse
+ *          of the bf16 Pi (float64 Newton-Schulz iterations, then rounded).
+ *          The decode maps each query as w = Pinv^T q.
+ *   workspace : device scratch of jl_turbo_rotation_workspace_bytes(d).
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED (d not 64 or 128),
+ * JL_ERR_WORKSPACE, JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_rotation_init(uint16_t *Pi, float *Pinv, int d, uint64_t seed,
+                                  void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
+
+/*
+ * jl_turbo_quantize_keys -- TurboQuant-prod codes and norms of n_keys keys.
+ *   K        : in, device, bf16 keys, row r at element r * key_stride
+ *              (16-byte aligned, stride * 2 a multiple of 16 bytes).
+ *   Pi       : in, device, d x d bf16 rotation (jl_turbo_rotation_init).
+ *   S        : in, device, m x d bf16 residual sketch (jl_sketch_init).
+ *   codes    : out, device, n_keys x words uint32 (layout above), 16-byte
+ *              aligned.
+ *   norms    : out, device, n_keys x 2 binary16, 4-byte aligned.
+ * Computed on the tensor cores (both products fp32-accumulated from exact
+ * bf16 operands).  A coordinate within the fp32 error of a boundary may take
+ * either cell; a residual coordinate within that error of a bf16 rounding
+ * midpoint may round either way, and a sign within the resulting error of 0
+ * either sign.  n_keys == 0 is a no-op.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED (d, m not 128; key dtype
+ * not bf16; mse_bits outside [1, JL_TURBO_MAX_MSE_BITS]), JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
+                                  int64_t key_stride, const uint16_t *Pi, const uint16_t *S,
+                                  int m, int d, int mse_bits, uint32_t *codes,
+                                  uint16_t *norms, jl_stream_t stream);
+
+/* Device scratch of jl_turbo_decode_attention (0 for unsupported shapes). */
+JL_API size_t jl_turbo_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int m,
+                                              int d, int mse_bits);
+
+/*
+ * jl_turbo_decode_attention -- one decode step over TurboQuant-prod keys:
+ * logit = softmax_scale * s(q, k_t), softmax over the context, value sum.
+ * Query head h reads KV head h / (Hq / Hkv).
+ *   Q      : in, device, B x Hq x d of `q_dtype`, 16-byte aligned.
+ *   Pinv   : in, device, d x d fp32 (jl_turbo_rotation_init).
+ *   S      : in, device, m x d bf16 residual sketch.
+ *   codes  : in, device, B x Hkv x T x words uint32, 16-byte aligned.
+ *   norms  : in, device, B x Hkv x T x 2 binary16, 16-byte aligned.
+ *   V      : in, device, B x Hkv x T x d bf16, 16-byte aligned.
+ *   out    : out, device, B x Hq x d bf16.
+ *   scores : optional out, B x Hq x T fp32 (s before softmax_scale).
+ *   workspace : device scratch of jl_turbo_decode_workspace_bytes(...).
+ * Supported: d = m = 128, mse_bits 1 or 2.  B == 0 is a no-op; T >= 1.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
+ * JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv,
+                                     const uint16_t *S, const uint32_t *codes,
+                                     const uint16_t *norms, const uint16_t *V, int B, int Hq,
+                                     int Hkv, int64_t T, int m, int d, int mse_bits,
+                                     float softmax_scale, uint16_t *out, float *scores,
+                                     void *workspace, size_t workspace_bytes,
+                                     jl_stream_t stream);
+
 /*
  * jl_device_error -- synchronise `stream`, then read and clear the device
  * error word of the current device (0 = no fault reported).  *code receives

@@ -51,6 +51,8 @@ def lib():
         L.jlo_gauss.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
         L.jlo_f64_to_bf16.restype = ctypes.c_uint16
         L.jlo_f64_to_bf16.argtypes = [ctypes.c_double]
+        L.jlo_f64_to_bf16_array.restype = None
+        L.jlo_f64_to_bf16_array.argtypes = [ctypes.c_long, _f64p, _u16p]
         L.jlo_bf16_to_f64.restype = ctypes.c_double
         L.jlo_bf16_to_f64.argtypes = [ctypes.c_uint16]
         L.jlo_sketch_bf16.restype = None
@@ -115,6 +117,14 @@ def gauss(seed: int, e: int) -> float:
 
 def f64_to_bf16_bits(x: float) -> int:
     return int(lib().jlo_f64_to_bf16(float(x)))
+
+
+def f64_to_bf16_bits_array(x) -> np.ndarray:
+    """Elementwise f64_to_bf16_bits of an array (same C rounding)."""
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().jlo_f64_to_bf16_array(x.size, _ptr(x, _f64p), _ptr(out, _u16p))
+    return out
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:

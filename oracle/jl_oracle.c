@@ -115,6 +115,11 @@ uint16_t jlo_f64_to_bf16(double x)
     return code;
 }
 
+void jlo_f64_to_bf16_array(long n, const double *x, uint16_t *out)
+{
+    for (long i = 0; i < n; ++i) out[i] = jlo_f64_to_bf16(x[i]);
+}
+
 double jlo_bf16_to_f64(uint16_t code)
 {
     union { float f; uint32_t u; } cv;

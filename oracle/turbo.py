@@ -49,7 +49,7 @@ import math
 import numpy as np
 import scipy.special
 
-from . import _c, bf16_bits_to_f64, f64_to_bf16_bits, fp16_round_bits, gauss
+from . import _c, bf16_bits_to_f64, f64_to_bf16_bits_array, fp16_round_bits, gauss
 
 SQRT_HALF_PI = math.sqrt(math.pi / 2.0)
 
@@ -155,8 +155,7 @@ def rotation(d: int, seed: int) -> np.ndarray:
 
 def rotation_bf16_bits(d: int, seed: int) -> np.ndarray:
     """Pit: Pi rounded to bfloat16 (nearest, ties to even), row-major codes."""
-    P = rotation(d, seed)
-    return np.array([[f64_to_bf16_bits(float(v)) for v in row] for row in P], dtype=np.uint16)
+    return f64_to_bf16_bits_array(rotation(d, seed))
 
 
 def rotation_stored(d: int, seed: int) -> np.ndarray:
@@ -174,8 +173,7 @@ def query_map(Pit) -> np.ndarray:
 
 def _bf16_round(x) -> np.ndarray:
     """Round float64 values to the nearest bfloat16 (ties to even)."""
-    x = np.asarray(x, dtype=np.float64)
-    return np.array([bf16_bits_to_f64(f64_to_bf16_bits(float(v))) for v in x.ravel()]).reshape(x.shape)
+    return bf16_bits_to_f64(f64_to_bf16_bits_array(x))
 
 
 def _bf16_ulp(x) -> np.ndarray:
@@ -233,8 +231,7 @@ def quantize(K, Pit, c, S, round_residual: bool = True, band_abs: float = 0.0,
         frac = np.abs(R - Rt)
         amb = np.abs(ulp / 2 - frac) < band_abs
         out["r_amb"] = amb
-        out["sign_allow"] = band_rel * rnorm[:, None] + (np.abs(S)[None, :, :] *
-                                                         (amb * ulp)[:, None, :]).sum(axis=2)
+        out["sign_allow"] = band_rel * rnorm[:, None] + (amb * ulp) @ np.abs(S).T
     return out
 
 

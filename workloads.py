@@ -27,6 +27,9 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
            into bf16 keys of d=128 (codes made from gqa's keys).
   search   top-10 inner-product search of 128 bf16 N(0,1) queries over an index
            of 8,388,608 N(0,1) vectors (d=128) kept as QJL codes (m=256).
+  turbo-gqa  the gqa decode step with TurboQuant-prod keys: 2-bit cells of
+           the rotated key (rotation seed 1) plus QJL on the residual with a
+           128-row sketch (3 bits per coordinate plus two binary16 norms).
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -100,10 +103,16 @@ DEQUANT_GQA = GQA.with_(name="dequant-gqa")
 # search: 128 queries against an index of 8,388,608 vectors (as keys of one
 # sequence: B = Hkv = 1, T = index size; Hq = queries)
 SEARCH = Workload("search", 7, 1, 128, 1, 8388608, 128, 256, torch.bfloat16)
+# TurboQuant-prod decode over the gqa cache: the same keys, values and
+# queries, cells of 2 bits per rotated coordinate, a 128-row residual sketch
+# (seed 0) and the rotation of seed TURBO_ROTATION_SEED
+TURBO_GQA = GQA.with_(name="turbo-gqa", m=128)
+TURBO_MSE_BITS = 2
+TURBO_ROTATION_SEED = 1
 SEARCH_K = 10
 
 ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA,
-                           SEARCH)}
+                           SEARCH, TURBO_GQA)}
 
 
 def sweep_points():
