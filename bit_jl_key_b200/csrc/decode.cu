@@ -76,7 +76,9 @@ struct DecCfg {
   static constexpr int NC = CODE_BITS / KS;            // k slices
   static constexpr int NC_MSE = TB * D / KS;           // slices of the cell planes
   static constexpr int A_REGS = 4 * NC;
-  static constexpr bool A_SMEM = A_REGS > 64;          // A fragments in smem
+  // A fragments in smem when they would crowd the registers; the cell-plane
+  // codes keep theirs in registers (two CTAs per SM instead of one)
+  static constexpr bool A_SMEM = A_REGS > (TB ? 96 : 64);
   static constexpr int A_SMEM_BYTES = A_SMEM ? NC * 32 * 16 : 0;
   static constexpr int WARP_BYTES = STAGES * STAGE_BYTES + A_SMEM_BYTES;
   // per stage: the block's norms (TB > 0: two binary16 per key), with room

@@ -29,11 +29,15 @@
 //           A operand of
 //   MMA 2   D = rt S^T             (S resident; D reuses MMA 1's columns)
 //   epilogue B  sign words of D.
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 epilogue (TMEM lane quadrant
-// warp % 4).  Two accumulators: the epilogue runs A of tile t, then B of tile
-// t - 1, so MMA 2 of one tile overlaps epilogue A of the next.  Every wait is
-// bounded; a wait that runs out records DERR_TC_WAIT_TIMEOUT, tells the other
-// roles to stop, and the CTA drains its copies and frees its tensor memory.
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2-9 epilogue: warp w reads TMEM
+// lane quadrant w % 4 (32 keys) and column half (w - 2) / 4 (64 coordinates);
+// the two warps of a quadrant exchange their half sums of k^2 and rt^2
+// through shared memory.  Tensor memory: MMA 1 results double-buffered (so
+// MMA 1 runs a tile ahead), MMA 2 results single-buffered, residual rows
+// double-buffered.  The epilogue runs A of tile t, then B of tile t - 1, so
+// MMA 2 of one tile overlaps epilogue A of the next.  Every wait is bounded; a
+// wait that runs out records DERR_TC_WAIT_TIMEOUT, tells the other roles to
+// stop, and the CTA drains its copies and frees its tensor memory.
 #include "jl_common.cuh"
 #include "jl_internal.h"
 #include "jl_rng.cuh"
@@ -318,17 +322,21 @@ struct QCfg {
   static constexpr int W_CHUNK = 128 * 128;     // 128 rows x 64 columns of Pi or S
   static constexpr int W_BYTES = 128 * QD * 2;  // 32 KB
   static constexpr int STAGES = 4;
+  static constexpr int EPI_WARPS = 8;           // two per TMEM lane quadrant (column halves)
+  static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int OFF_PI = 0;
   static constexpr int OFF_S = W_BYTES;
   static constexpr int OFF_A = 2 * W_BYTES;
-  static constexpr int OFF_BAR = OFF_A + STAGES * A_STAGE;
-  static constexpr int NBAR = 2 * STAGES + 4 * 2 + 1;
+  static constexpr int OFF_X = OFF_A + STAGES * A_STAGE;   // half-row sums: [2][2][BM] float
+  static constexpr int OFF_BAR = OFF_X + 4 * BM * 4;
+  static constexpr int NBAR = 2 * STAGES + 2 + 2 + 1 + 1 + 1 + 4;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr int THREADS = 6 * 32;
   static constexpr int WORDS = TB * QD / 32 + QM / 32;
   static constexpr int PW = QD / 32;            // words per plane
   static constexpr int TMEM_COLS = 512;
-  static constexpr int A2_COL = 256;            // bf16 residual rows (64 columns each)
+  static constexpr int D1_COL = 0;              // rotated keys, two buffers of 128 columns
+  static constexpr int D2_COL = 256;            // residual projections, one buffer
+  static constexpr int A2_COL = 384;            // bf16 residual rows, two buffers of 64
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -385,14 +393,19 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *gbase = tq_smem_raw + (base - raw);
   const uint32_t sPi = base + C::OFF_PI, sS = base + C::OFF_S, sA = base + C::OFF_A;
+  float *xsum = reinterpret_cast<float *>(gbase + C::OFF_X);  // [k or r][half][row]
   const uint32_t bar0 = base + C::OFF_BAR;
   auto kfull = [&](int s) { return bar0 + 8u * s; };
   auto kempty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
   auto d1full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto afull = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
-  auto d2full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 4 + a); };
-  auto dempty = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 6 + a); };
-  const uint32_t wfull = bar0 + 8u * (2 * C::STAGES + 8);
+  const uint32_t d2full = bar0 + 8u * (2 * C::STAGES + 4);
+  const uint32_t d2empty = bar0 + 8u * (2 * C::STAGES + 5);
+  const uint32_t wfull = bar0 + 8u * (2 * C::STAGES + 6);
+  // the two epilogue warps of lane quadrant q exchange half-row sums through
+  // shared memory; each exchange is one phase of pairbar(q) (one arrival per
+  // warp), waited on with the same bound as every other wait
+  auto pairbar = [&](int q) { return bar0 + 8u * (2 * C::STAGES + 7 + q); };
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
   volatile int *abort_flag =
       reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
@@ -401,15 +414,16 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(kfull(s), 1);
-      mbar_init(kempty(s), 1 + 4);  // MMA commit + 4 epilogue warps (norms)
+      mbar_init(kempty(s), 1 + C::EPI_WARPS);  // MMA commit + epilogue warps (norms)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(d1full(a), 1);
-      mbar_init(afull(a), 4);
-      mbar_init(d2full(a), 1);
-      mbar_init(dempty(a), 4);
+      mbar_init(afull(a), C::EPI_WARPS);
     }
+    mbar_init(d2full, 1);
+    mbar_init(d2empty, C::EPI_WARPS);
     mbar_init(wfull, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(pairbar(q), 2);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -453,7 +467,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       tcx::drain_wait(wfull, 0);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: MMA 1 of tile t, then MMA 2 of tile t - 1
     if (lane == 0) {
       constexpr uint32_t idesc = tcx::idesc_f16(BM, 128, 1);
       bool ok = tcx::wait_phase(wfull, 0, abort_flag, p.err);
@@ -462,8 +476,10 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         if (t < cnt) {
           const int s = (int)(t % C::STAGES);
           const int a = (int)(t & 1);
+          // the key tile has landed; accumulator a was read by epilogue A of t - 2
           if (!tcx::wait_phase(kfull(s), (uint32_t)((t / C::STAGES) & 1), abort_flag, p.err) ||
-              !tcx::wait_phase(dempty(a), (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.err)) {
+              (t >= 2 && !tcx::wait_phase(afull(a), (uint32_t)(((t - 2) >> 1) & 1), abort_flag,
+                                          p.err))) {
             ok = false;
             break;
           }
@@ -473,7 +489,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
             const uint32_t koff = (uint32_t)(kk & 3) * 32u;
             const uint64_t ad = tcx::desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
             const uint64_t bd = tcx::desc_sw128(sPi + (kk >> 2) * C::W_CHUNK + koff);
-            tcx::mma_ss(tmem_base + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            tcx::mma_ss(tmem_base + C::D1_COL + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           tcx::commit(d1full(a));
           tcx::commit(kempty(s));
@@ -481,7 +497,9 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         if (t >= 1) {
           const int64_t u = t - 1;
           const int a = (int)(u & 1);
-          if (!tcx::wait_phase(afull(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err)) {
+          // residual rows of u written; the projection buffer read by B of u - 1
+          if (!tcx::wait_phase(afull(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err) ||
+              !tcx::wait_phase(d2empty, (uint32_t)((u & 1) ^ 1), abort_flag, p.err)) {
             ok = false;
             break;
           }
@@ -490,30 +508,37 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           for (int kk = 0; kk < QD / 16; ++kk) {
             const uint32_t koff = (uint32_t)(kk & 3) * 32u;
             const uint64_t bd = tcx::desc_sw128(sS + (kk >> 2) * C::W_CHUNK + koff);
-            tcx::mma_ts(tmem_base + a * 128, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
+            tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
                         kk > 0 ? 1u : 0u);
           }
-          tcx::commit(d2full(a));
+          tcx::commit(d2full);
           ++issued2;
         }
       }
       // the last products must be complete before tensor memory is freed
-      if (issued2 > 0) {
-        const int64_t u = issued2 - 1;
-        tcx::drain_wait(d2full((int)(u & 1)), (uint32_t)((u >> 1) & 1));
-      }
+      if (issued2 > 0) tcx::drain_wait(d2full, (uint32_t)((issued2 - 1) & 1));
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue: key row 32 * (warp % 4) + lane of each tile
+    // ---------------- epilogue: key row r = 32 (warp % 4) + lane, column
+    // half h (coordinates 64 h .. 64 h + 63) of each tile
     const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     const int r = 32 * q + lane;
-    const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16);
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
     float t[7], c[8];
 #pragma unroll
     for (int i = 0; i < 7; ++i) t[i] = p.thr[i];
 #pragma unroll
     for (int i = 0; i < 8; ++i) c[i] = p.cent[i];
+    float *xk = xsum;           // [2][BM] half sums of k^2
+    float *xr = xsum + 2 * BM;  // [2][BM] half sums of rt^2
+    uint32_t xchg = 0;          // exchanges done (phase index of pairbar(q))
+    auto exchange = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pairbar(q));
+      return tcx::wait_phase(pairbar(q), (xchg++) & 1u, abort_flag, p.err);
+    };
     bool ok = true;
     for (int64_t it = 0; ok && it <= cnt; ++it) {
       if (it < cnt) {
@@ -527,26 +552,28 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         }
         float ss0 = 0.f, ss1 = 0.f;
         {
-          const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + r * 128;
+          const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + h * C::A_CHUNK + r * 128;
 #pragma unroll
-          for (int kc = 0; kc < C::KCH; ++kc)
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ (r & 7)) << 4));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 v = *reinterpret_cast<const uint4 *>(rowp + kc * C::A_CHUNK +
-                                                               ((ch ^ (r & 7)) << 4));
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(w4[e] << 16);
-                const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
-                ss0 = fmaf(lo, lo, ss0);
-                ss1 = fmaf(hi, hi, ss1);
-              }
+            for (int e = 0; e < 4; ++e) {
+              const float lo = __uint_as_float(w4[e] << 16);
+              const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
+              ss0 = fmaf(lo, lo, ss0);
+              ss1 = fmaf(hi, hi, ss1);
             }
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(kempty(s));
-        const float nk = sqrtf(ss0 + ss1);
+        xk[h * BM + r] = ss0 + ss1;
+        if (!exchange()) {
+          ok = false;
+          break;
+        }
+        const float nk = sqrtf(xk[r] + xk[BM + r]);
         const float inv = nk > 0.f ? 1.f / nk : 0.f;
         if (!tcx::wait_phase(d1full(a), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) {
           ok = false;
@@ -554,11 +581,11 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         }
         __syncwarp();
         tcx::fence_after();
-        uint32_t planes[TB][C::PW];
+        uint32_t planes[TB][2];
         float rs0 = 0.f, rs1 = 0.f;
         uint32_t va[32], vb[32];
-        const uint32_t dcol = trow + (uint32_t)(a * 128);
-        const uint32_t acol = trow + (uint32_t)(C::A2_COL + a * 64);
+        const uint32_t dcol = tq + (uint32_t)(C::D1_COL + a * 128 + 64 * h);
+        const uint32_t acol = tq + (uint32_t)(C::A2_COL + a * 64 + 32 * h);
         auto chunk = [&](const uint32_t (&v)[32], int ch) {
           uint32_t pw[TB];
 #pragma unroll
@@ -579,64 +606,57 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           for (int pp = 0; pp < TB; ++pp) planes[pp][ch] = pw[pp];
         };
         tcx::ld32(dcol, va);
-        tcx::ld_wait(va);
         tcx::ld32(dcol + 32, vb);
+        tcx::ld_wait(va);
         chunk(va, 0);
         tcx::ld_wait(vb);
-        tcx::ld32(dcol + 64, va);
         chunk(vb, 1);
-        tcx::ld_wait(va);
-        tcx::ld32(dcol + 96, vb);
-        chunk(va, 2);
-        tcx::ld_wait(vb);
-        chunk(vb, 3);
         tcx::st_wait();
         tcx::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(afull(a));
+        xr[h * BM + r] = rs0 + rs1;
+        if (!exchange()) {
+          ok = false;
+          break;
+        }
         if (row < p.n) {
-          uint32_t *dst = p.codes + row * C::WORDS;
+          uint32_t *dst = p.codes + row * C::WORDS + 2 * h;
 #pragma unroll
           for (int pp = 0; pp < TB; ++pp)
-            *reinterpret_cast<uint4 *>(dst + pp * C::PW) =
-                make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
-          const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
-          const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
-          p.norms[row] = n16 | (r16 << 16);
+            *reinterpret_cast<uint2 *>(dst + pp * C::PW) = make_uint2(planes[pp][0], planes[pp][1]);
+          if (h == 0) {
+            const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
+            const uint32_t r16 =
+                __half_as_ushort(__float2half_rn(sqrtf(xr[r] + xr[BM + r])));
+            p.norms[row] = n16 | (r16 << 16);
+          }
         }
       }
       if (it >= 1) {
-        // ---- B: residual sign words of tile it - 1
+        // ---- B: residual sign words of tile it - 1 (this warp's half)
         const int64_t u = it - 1;
-        const int a = (int)(u & 1);
         const int64_t row = (blockIdx.x + u * gridDim.x) * BM + r;
-        if (!tcx::wait_phase(d2full(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err)) {
+        if (!tcx::wait_phase(d2full, (uint32_t)(u & 1), abort_flag, p.err)) {
           ok = false;
           break;
         }
         __syncwarp();
         tcx::fence_after();
-        uint32_t w[4];
         uint32_t va[32], vb[32];
-        const uint32_t dcol = trow + (uint32_t)(a * 128);
+        const uint32_t dcol = tq + (uint32_t)(C::D2_COL + 64 * h);
         tcx::ld32(dcol, va);
-        tcx::ld_wait(va);
         tcx::ld32(dcol + 32, vb);
-        w[0] = tcx::sign_word(va);
-        tcx::ld_wait(vb);
-        tcx::ld32(dcol + 64, va);
-        w[1] = tcx::sign_word(vb);
         tcx::ld_wait(va);
-        tcx::ld32(dcol + 96, vb);
-        w[2] = tcx::sign_word(va);
+        const uint32_t w0 = tcx::sign_word(va);
         tcx::ld_wait(vb);
-        w[3] = tcx::sign_word(vb);
+        const uint32_t w1 = tcx::sign_word(vb);
         tcx::fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(dempty(a));
+        if (lane == 0) mbar_arrive(d2empty);
         if (row < p.n)
-          *reinterpret_cast<uint4 *>(p.codes + row * C::WORDS + TB * C::PW) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint2 *>(p.codes + row * C::WORDS + TB * C::PW + 2 * h) =
+              make_uint2(w0, w1);
       }
     }
   }
