@@ -1,7 +1,7 @@
 """Benchmark: QJL key quantization + compressed-key decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search|turbo-gqa]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -20,6 +20,10 @@ step rewrites the same slots).
 The search workload times one jl_search_topk call: the top-10 index vectors
 of each of 128 queries over 8,388,608 compressed vectors (scores on the
 tensor cores; the roofline is the tensor peak).
+
+The turbo-gqa workload times the TurboQuant-prod step on the gqa cache:
+jl_turbo_quantize_keys over every key (rotation product and residual sketch on
+the tensor cores) and one jl_turbo_decode_attention call.
 
 The dequant-gqa workload times the explicit dequantizer: one
 jl_dequantize_keys call turning the gqa cache's codes and norms back into
@@ -573,9 +577,169 @@ def run_search(args, rank, world, local_rank):
     }
 
 
+def run_turbo(args, rank, world, local_rank):
+    """TurboQuant-prod step over the turbo-gqa cache: quantize every key
+    (rotation product, cells, residual QJL) and one decode step over the
+    cell-plane codes."""
+    import bit_jl_key_b200 as jl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload, args.batch)
+    bits = workloads.TURBO_MSE_BITS
+    peak, peak_kind = load_peaks()
+    Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED, device=dev)
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)
+    Kf = K.view(-1, w.d)
+    n_keys = Kf.shape[0]
+    words = jl.turbo_code_words(bits, w.m, w.d)
+    codes = torch.empty((n_keys, words), dtype=torch.int32, device=dev)
+    norms = torch.empty((n_keys, 2), dtype=torch.float16, device=dev)
+    V = workloads.values(w, dev)
+    Q = workloads.queries(w, dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((jl.jl_turbo_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d, bits),),
+                     dtype=torch.uint8, device=dev)
+    c4 = codes.view(w.B, w.Hkv, w.T, words)
+    n4 = norms.view(w.B, w.Hkv, w.T, 2)
+    stream = torch.cuda.current_stream(dev)
+
+    def quantize():
+        jl.jl_turbo_quantize_keys(Kf, Pi, S, bits, codes=codes, norms=norms)
+
+    def decode_call():
+        jl.jl_turbo_decode_attention(Q, Pinv, S, c4, n4, V, bits, softmax_scale=w.softmax_scale,
+                                     out=out, workspace=ws)
+
+    def step():
+        quantize()
+        decode_call()
+
+    def timed_loop(fn, n):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        _barrier(world, dev)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        _barrier(world, dev)
+        q_ms = timed_loop(quantize, args.steps)
+        d_ms = timed_loop(decode_call, args.steps)
+        _barrier(world, dev)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_step = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+
+    # estimator quality on sampled heads (untimed): normalised error of the
+    # scores against the exact inner products
+    score_err = None
+    if not args.no_score_error:
+        _, sc = jl.jl_turbo_decode_attention(Q, Pinv, S, c4, n4, V, bits, want_scores=True,
+                                             workspace=ws)
+        errs = []
+        for b in range(min(w.B, 2)):
+            for h in range(0, w.Hq, max(1, w.Hq // 4)):
+                kv = K[b, h // w.G].double()
+                q = Q[b, h].double()
+                exact = kv @ q
+                denom = kv.norm(dim=1) * q.norm()
+                errs.append(((sc[b, h].double() - exact) / denom).pow(2).mean().item())
+        score_err = {"rms_normalised_error": math.sqrt(sum(errs) / len(errs)),
+                     "heads_sampled": len(errs),
+                     "definition": "rms over sampled heads and all keys of "
+                                   "(score - <q,k>) / (||q|| ||k||)"}
+
+    e2e = None
+    if not args.no_e2e:
+        hK = K.cpu().pin_memory()
+        hV = V.cpu().pin_memory()
+        hQ = Q.cpu().pin_memory()
+        hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            Q.copy_(hQ, non_blocking=True)
+            step()
+            hOut.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        _barrier(world, dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e_steps = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        _barrier(world, dev)
+        e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+        e2e = {"value": whole_job_rate(n_keys, world, e_ms), "unit": "keys/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": (hK.numel() + hV.numel() + hQ.numel()) * 2,
+               "d2h_bytes_per_step": hOut.numel() * 2}
+
+    per_key = words * 4 + 4
+    qb = n_keys * (2 * w.d + per_key)
+    db = n_keys * (per_key + 2 * w.d) + w.B * w.Hq * w.d * 2 * 2
+    phases = {
+        "quantize": {"ms": q_ms, "keys_per_s": n_keys / (q_ms * 1e-3), "algorithmic_bytes": qb,
+                     "GB_per_s": qb / (q_ms * 1e-3) / 1e9,
+                     "tflops": n_keys * 2 * (w.d * w.d + w.m * w.d) / (q_ms * 1e-3) / 1e12},
+        "decode": {"ms": d_ms, "keys_scored_per_s": n_keys / (d_ms * 1e-3),
+                   "algorithmic_bytes": db, "GB_per_s": db / (d_ms * 1e-3) / 1e9},
+    }
+    for ph in phases.values():
+        ph["frac_of_hbm_peak"] = ph["GB_per_s"] / peak
+    dom = max(phases, key=lambda k: phases[k]["ms"])
+    kname = {"quantize": "jl_turbo_quantize_keys", "decode": "jl_turbo_decode_attention"}[dom]
+    traffic = ncu_traffic(("turbo_quantize" if dom == "quantize" else "turbo_decode") + ":" + w.name)
+    return {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": whole_job_rate(n_keys, world, ms_step), "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} d={w.d} "
+                               f"m={w.m}, {bits}-bit cells + 1-bit residual QJL",
+                   "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                   "l2": "inputs exceed L2 (126 MB); no flush"},
+        "phases": phases,
+        "phase_timing": "each phase alone: K back-to-back calls, CUDA events at the ends",
+        "roofline": {"kernel": kname, "bound": "hbm", "achieved": phases[dom]["GB_per_s"],
+                     "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": phases[dom]["GB_per_s"] / peak,
+                     "algorithmic_bytes_per_launch": phases[dom]["algorithmic_bytes"],
+                     "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
+        "score_error": score_err,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
+    if args.workload == "turbo-gqa":
+        return run_turbo(args, rank, world, local_rank)
     if args.workload == "search":
         return run_search(args, rank, world, local_rank)
     if args.workload == "paged-gqa":
@@ -799,6 +963,26 @@ def oracle_sample(w: workloads.Workload):
         def run():
             oracle.dequantize(sig, n64, S64)
         return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
+    if w.name == "turbo-gqa":
+        from oracle import turbo as tq
+        T = w.T
+        sub = w.with_(B=1, Hkv=1, Hq=w.G, T=T)
+        K = workloads.keys(sub).double().numpy().reshape(-1, w.d)
+        V = workloads.values(sub).double().numpy()
+        Q = workloads.queries(sub).double().numpy()
+        bits = workloads.TURBO_MSE_BITS
+        c = tq.lloyd_max(w.d, bits)                           # set-up, untimed
+        Pit = tq.rotation_stored(w.d, workloads.TURBO_ROTATION_SEED)
+
+        def run():
+            q = tq.quantize(K, Pit, c, S64)
+            tq.decode(Q, Pit, S64, c, q["cell"].reshape(1, 1, T, w.d),
+                      q["signs"].reshape(1, 1, T, -1),
+                      oracle.fp16_bits_to_f64(q["norm16"]).reshape(1, 1, T),
+                      oracle.fp16_bits_to_f64(q["rnorm16"]).reshape(1, 1, T), V,
+                      w.softmax_scale)
+        return run, T, (f"one (b, kv-head) unit: {T} keys, {w.G} query heads, "
+                        f"TurboQuant-prod quantize + decode in float64")
     if w.name == "prefill":
         n = 16384
         Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()
