@@ -26,21 +26,23 @@ Readings where the pages leave a step open:
     unique such Q), G[i][j] the standard normal of element i*d + j of the
     sketch generator with the rotation's own seed.  Pi is stored in bfloat16
     (Pit below); the key side uses Pit: y = Pit x.
-  * The cell of coordinate y_i is the number of boundaries strictly below it
-    (a value on a boundary goes to the lower cell); yhat_i = c[cell].  The
+  * The cell of coordinate y_i is that of the nearest centroid; a value
+    exactly on a boundary goes to the cell nearer zero (so the quantizer is
+    odd-symmetric; 0 goes to the cell just below it); yhat_i = c[cell].  The
     (b-1)-bit cell index is stored as b-1 bit planes, plane p holding bit p
     of every coordinate's index, each plane d bits LSB-first.
-  * Stage two works in the rotated frame: r = y - yhat, rounded to bfloat16
-    (rt, the vector the QJL stage is given), code sign(S rt) with an m x d
-    Gaussian sketch S (bit 1 for >= 0), and ||rt|| stored as binary16.  For
+  * Stage two works in the rotated frame on the residual r = y - yhat: its
+    code is sign(S rt) with rt = r rounded to bfloat16 (the precision of the
+    contraction's input; bit 1 for >= 0) and an m x d Gaussian sketch S, and
+    its norm ||r|| (of the residual itself) is stored as binary16.  For
     an exactly orthogonal Pi this is the pages' construction in distribution:
     S r = (S Pi^T)(Pi r) and S Pi^T is again an i.i.d. Gaussian matrix.
   * The query is mapped with the inverse transpose of the stored rotation,
     w = Pit^{-T} q, so that <w, y> = <q, x> holds exactly whatever rounding
     did to Pit; the estimate of <q, k> is
-        ||k|| * ( <w, yhat> + sqrt(pi/2)/m * ||rt|| * <S w, sign(S rt)> ),
-    whose expectation over S is ||k|| <w, yhat + rt>, i.e. <q, k> up to the
-    bfloat16 rounding of the residual and the binary16 norms.
+        ||k|| * ( <w, yhat> + sqrt(pi/2)/m * ||r|| * <S w, sign(S rt)> ),
+    whose expectation over S is ||k|| <w, yhat + rt ||r|| / ||rt||>, i.e.
+    <q, k> up to the bfloat16 rounding of the residual and the binary16 norms.
 """
 from __future__ import annotations
 
@@ -112,10 +114,17 @@ def lloyd_max(d: int, bits: int, tol: float = 1e-15, max_iter: int = 100000):
 
 
 def cell_of(Y, c):
-    """Cell of every value: the number of boundaries strictly below it."""
+    """Cell of every value: the cell of the nearest centroid; a value exactly
+    on a boundary goes to the cell nearer zero (0 goes to the cell just below
+    it), which keeps the quantizer odd-symmetric.  With L cells and the
+    positive boundaries t_+:  y > 0 -> L/2 + #{t in t_+ : t < y},
+    y <= 0 -> L/2 - 1 - #{t in t_+ : t < -y}."""
     t = boundaries(c)
+    L = len(c)
+    tpos = t[L // 2:]
     Y = np.asarray(Y, dtype=np.float64)
-    return np.sum(Y[..., None] > t, axis=-1).astype(np.uint8)
+    outer = np.sum(np.abs(Y)[..., None] > tpos, axis=-1)
+    return np.where(Y > 0, L // 2 + outer, L // 2 - 1 - outer).astype(np.uint8)
 
 
 def boundaries(c):
@@ -193,7 +202,7 @@ def quantize(K, Pit, c, S, round_residual: bool = True, band_abs: float = 0.0,
       r, rt   f64    [n, d]  residual y - c[cell], and as given to QJL
       signs   uint32 [n, m/32]  sign(S rt), LSB-first (bit 1 for >= 0)
       proj    f64    [n, m]  S rt
-      norm, rnorm  f64 [n]   ||k||, ||rt|| (exact)
+      norm, rnorm  f64 [n]   ||k||, ||r|| (exact)
       norm16, rnorm16 uint16 [n]  their binary16 codes
     With band_abs > 0 also:
       cell_band bool [n, d]  y within band_abs of a boundary
@@ -220,7 +229,7 @@ def quantize(K, Pit, c, S, round_residual: bool = True, band_abs: float = 0.0,
     signs = np.zeros((n, m // 32), dtype=np.uint64)
     for i in range(m):
         signs[:, i // 32] |= bits[:, i] << np.uint64(i % 32)
-    rnorm = np.sqrt(np.sum(Rt * Rt, axis=1))
+    rnorm = np.sqrt(np.sum(R * R, axis=1))
     out = {"cell": cell, "y": Y, "r": R, "rt": Rt, "signs": signs.astype(np.uint32),
            "proj": P, "norm": norm, "rnorm": rnorm,
            "norm16": fp16_round_bits(norm), "rnorm16": fp16_round_bits(rnorm)}

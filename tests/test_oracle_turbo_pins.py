@@ -174,11 +174,18 @@ def test_cells_are_nearest_centroids_brute_force():
             best = min(range(len(c)), key=lambda j: (dist[j], j))
             assert q["cell"][n, i] == best
             assert q["r"][n, i] == pytest.approx(y[i] - c[best], abs=1e-15)
-    # exactly on a boundary -> the lower cell
+    # exactly on a boundary -> the cell nearer zero; 0 -> the cell below it;
+    # the quantizer is odd-symmetric
     t = tq.boundaries(c)
     Y = np.array([[t[0], t[1], t[2], c[0], c[3], -1.0, 1.0, 0.0]])
     assert t[1] == 0.0
-    assert list(tq.cell_of(Y, c)[0]) == [0, 1, 2, 0, 3, 0, 3, 1]
+    assert list(tq.cell_of(Y, c)[0]) == [1, 1, 2, 0, 3, 0, 3, 1]
+    c3 = tq.lloyd_max(d, 3)
+    t3 = tq.boundaries(c3)
+    Y3 = np.concatenate([t3, -t3, c3, np.linspace(-0.9, 0.9, 37)])
+    cells = tq.cell_of(Y3, c3)
+    assert np.array_equal(c3[tq.cell_of(-Y3[Y3 != 0], c3)], -c3[cells[Y3 != 0]])
+    assert list(tq.cell_of(t3, c3)) == [1, 2, 3, 3, 4, 5, 6]
 
 
 def test_residual_code_is_qjl_of_the_rounded_residual():
@@ -195,7 +202,7 @@ def test_residual_code_is_qjl_of_the_rounded_residual():
     assert np.abs(q["rt"] - q["r"]).max() <= np.abs(q["r"]).max() * 2.0 ** -8
     signs, norms, _, _ = oracle.quantize(q["rt"], S)
     assert np.array_equal(signs, q["signs"])
-    assert np.allclose(norms, q["rnorm"], rtol=1e-15)
+    assert np.allclose(np.linalg.norm(q["r"], axis=1), q["rnorm"], rtol=1e-15)
     assert np.allclose(q["norm"], np.linalg.norm(K, axis=1), rtol=1e-15)
 
 
@@ -254,7 +261,7 @@ def test_prod_estimator_unbiased_over_sketches():
 
 
 def test_prod_variance_is_qjl_variance_of_the_residual():
-    # over sketches, Var = ||k||^2 ((pi/2) ||w||^2 ||rt||^2 - <w, rt>^2) / m
+    # over sketches, Var = (||k|| ||r|| / ||rt||)^2 ((pi/2) ||w||^2 ||rt||^2 - <w, rt>^2) / m
     rng = np.random.default_rng(12)
     d, m = 24, 64
     c = tq.lloyd_max(d, 1)
@@ -272,14 +279,16 @@ def test_prod_variance_is_qjl_variance_of_the_residual():
     est = np.array(est)
     rt = q0["rt"][0]
     nk = q0["norm"][0]
-    var = nk ** 2 * ((math.pi / 2) * (w @ w) * (rt @ rt) - (w @ rt) ** 2) / m
+    # the code is QJL of rt scaled by ||r|| (the residual's own norm)
+    sc = q0["rnorm"][0] / math.sqrt(rt @ rt)
+    var = (nk * sc) ** 2 * ((math.pi / 2) * (w @ w) * (rt @ rt) - (w @ rt) ** 2) / m
     n = est.size
     lo = scipy.stats.chi2.ppf(1e-4, n - 1) / (n - 1)
     hi = scipy.stats.chi2.ppf(1 - 1e-4, n - 1) / (n - 1)
     assert lo * var < est.var(ddof=1) < hi * var
-    # the mean is <w, yhat + rt> ||k||
+    # the mean is ||k|| <w, yhat + rt ||r|| / ||rt||>
     yhat = c[q0["cell"][0]]
-    mean = nk * (w @ (yhat + rt))
+    mean = nk * (w @ (yhat + sc * rt))
     assert abs(est.mean() - mean) < 4 * math.sqrt(var / n)
 
 
