@@ -23,10 +23,10 @@
 //
 // Quantizer (tensor cores), per tile of 128 keys:
 //   MMA 1   D = K Pi^T             (K: TMA-loaded bf16 tile; Pi resident)
-//   epilogue A  (one thread per key): y = D / ||k||; cells by a branch-free
-//           binary search over the boundaries (the cell bits are the code's
-//           planes); rt = bf16(y - c[cell]) written to tensor memory as the
-//           A operand of
+//   epilogue A  (one thread per key and column half): y = D / ||k||; cells by
+//           a branch-free search of |y| over the positive boundaries (the cell
+//           bits are the code's planes); r = y - c[cell], ||r||, and
+//           rt = bf16(r) written to tensor memory as the A operand of
 //   MMA 2   D = rt S^T             (S resident; D reuses MMA 1's columns)
 //   epilogue B  sign words of D.
 // Warp roles: 0 TMA producer, 1 MMA issuer, 2-9 epilogue: warp w reads TMEM
@@ -344,42 +344,62 @@ struct QParams {
   int64_t n;
   int64_t num_tiles;
   uint32_t *codes;
-  uint32_t *norms;  // (||k|| | ||rt|| << 16) binary16 pairs
+  uint32_t *norms;  // (||k|| | ||r|| << 16) binary16 pairs
   int *err;
-  float thr[7];
-  float cent[8];
+  float mag[4];      // centroid magnitudes a_0 < ... (positive half of the codebook)
+  float pos_thr[3];  // positive boundaries between them
 };
 
-// Cell of y by binary search over the boundaries (ties go to the lower cell);
-// the bits of the cell index go to the plane words at bit e; returns
-// y - c[cell].
+// Odd-symmetric cells.  With H = 2^(TB-1) centroid magnitudes a_0 < ... <
+// a_{H-1} (the positive half of the codebook) and the positive boundaries
+// p_0 < ... < p_{H-2} between them, a coordinate y lies in magnitude cell
+// mu = #{p_j < |y|} (a value on a boundary stays inward) on the side of its
+// sign (0 counts as negative), i.e. cell H + mu for y > 0 and H - 1 - mu
+// otherwise; its centroid is +-a_mu.  In bits: the top plane is [y > 0] and
+// plane k < TB-1 is bit k of mu when y > 0 and its complement otherwise, i.e.
+// XNOR(bit k of mu, [y > 0]).
+//
+// Every bit is the sign bit of a float formed on the FMA pipe, gathered into
+// code words by funnel shifts: [y > 0] = sign(0 - y) (0 - y is +0 for y = +-0)
+// and bit k of mu = sign(p - |y|) for the boundary p of that search level, so
+// the plane bit is the complement of sign((0 - y) (p - |y|)).
+struct Magnitudes {
+  float a[4];  // centroid magnitudes
+  float p[3];  // positive boundaries
+};
+
 template <int TB>
-__device__ __forceinline__ float cell_residual(float y, const float (&t)[7], const float (&c)[8],
-                                               uint32_t (&pw)[TB], int e) {
+struct PlaneChains {
+  uint32_t top[4];          // [y > 0], four chains of 8 bits
+  uint32_t mag[TB - 1 > 0 ? TB - 1 : 1][4];  // complemented magnitude planes
+};
+
+// residual of one coordinate; pushes its bits into chain g
+template <int TB>
+__device__ __forceinline__ float cell_residual(float y, const Magnitudes &mg, PlaneChains<TB> &ch,
+                                               int g) {
+  const float neg = 0.f - y;
+  ch.top[g] = __funnelshift_l(__float_as_uint(neg), ch.top[g], 1);
+  const float ay = fabsf(y);
+  float amag;
   if constexpr (TB == 1) {
-    const bool b0 = y > t[0];
-    pw[0] |= (uint32_t)b0 << e;
-    return y - (b0 ? c[1] : c[0]);
+    amag = mg.a[0];
   } else if constexpr (TB == 2) {
-    const bool b1 = y > t[1];
-    const bool b0 = y > (b1 ? t[2] : t[0]);
-    pw[1] |= (uint32_t)b1 << e;
-    pw[0] |= (uint32_t)b0 << e;
-    const float hi = b1 ? c[3] : c[1], lo = b1 ? c[2] : c[0];
-    return y - (b0 ? hi : lo);
+    const float d0 = mg.p[0] - ay;
+    ch.mag[0][g] = __funnelshift_l(__float_as_uint(neg * d0), ch.mag[0][g], 1);
+    amag = d0 < 0.f ? mg.a[1] : mg.a[0];
   } else {
-    const bool b2 = y > t[3];
-    const bool b1 = y > (b2 ? t[5] : t[1]);
-    const float t0 = b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]);
-    const bool b0 = y > t0;
-    pw[2] |= (uint32_t)b2 << e;
-    pw[1] |= (uint32_t)b1 << e;
-    pw[0] |= (uint32_t)b0 << e;
-    const float c01 = b0 ? c[1] : c[0], c23 = b0 ? c[3] : c[2];
-    const float c45 = b0 ? c[5] : c[4], c67 = b0 ? c[7] : c[6];
-    const float lo = b1 ? c23 : c01, hi = b1 ? c67 : c45;
-    return y - (b2 ? hi : lo);
+    const float d1 = mg.p[1] - ay;
+    const bool m1 = d1 < 0.f;
+    const float d0 = (m1 ? mg.p[2] : mg.p[0]) - ay;
+    ch.mag[1][g] = __funnelshift_l(__float_as_uint(neg * d1), ch.mag[1][g], 1);
+    ch.mag[0][g] = __funnelshift_l(__float_as_uint(neg * d0), ch.mag[0][g], 1);
+    const bool m0 = d0 < 0.f;
+    amag = m1 ? (m0 ? mg.a[3] : mg.a[2]) : (m0 ? mg.a[1] : mg.a[0]);
   }
+  // y - (+-a_mu): the centroid takes the sign of y, negative for y = +-0
+  const float sgn = __uint_as_float((__float_as_uint(neg) & 0x80000000u) | 0x3F800000u);
+  return fmaf(sgn, amag, y);
 }
 
 template <int TB>
@@ -526,11 +546,11 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
     const int h = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
-    float t[7], c[8];
+    Magnitudes mg;
 #pragma unroll
-    for (int i = 0; i < 7; ++i) t[i] = p.thr[i];
+    for (int i = 0; i < 4; ++i) mg.a[i] = p.mag[i];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = p.cent[i];
+    for (int i = 0; i < 3; ++i) mg.p[i] = p.pos_thr[i];
     float *xk = xsum;           // [2][BM] half sums of k^2
     float *xr = xsum + 2 * BM;  // [2][BM] half sums of rt^2
     uint32_t xchg = 0;          // exchanges done (phase index of pairbar(q))
@@ -586,24 +606,38 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         uint32_t va[32], vb[32];
         const uint32_t dcol = tq + (uint32_t)(C::D1_COL + a * 128 + 64 * h);
         const uint32_t acol = tq + (uint32_t)(C::A2_COL + a * 64 + 32 * h);
-        auto chunk = [&](const uint32_t (&v)[32], int ch) {
-          uint32_t pw[TB];
+        auto chunk = [&](uint32_t (&v)[32], int ch) {
+          PlaneChains<TB> pc;
 #pragma unroll
-          for (int pp = 0; pp < TB; ++pp) pw[pp] = 0u;
+          for (int g = 0; g < 4; ++g) {
+            pc.top[g] = 0u;
+#pragma unroll
+            for (int k = 0; k < (TB > 1 ? TB - 1 : 1); ++k) pc.mag[k][g] = 0u;
+          }
+          // coordinate 8 g + jj, highest first so that the funnel shifts
+          // leave bit jj of chain g at position jj
+#pragma unroll
+          for (int jj = 7; jj >= 0; --jj)
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int e = 8 * g + jj;
+              const float r = cell_residual<TB>(__uint_as_float(v[e]) * inv, mg, pc, g);
+              if (g & 1)
+                rs1 = fmaf(r, r, rs1);
+              else
+                rs0 = fmaf(r, r, rs0);
+              v[e] = __float_as_uint(r);
+            }
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float r0 = cell_residual<TB>(__uint_as_float(v[e]) * inv, t, c, pw, e);
-            const float r1 = cell_residual<TB>(__uint_as_float(v[e + 1]) * inv, t, c, pw, e + 1);
-            const uint32_t b = pack_bf16x2(r0, r1);
-            pk[e >> 1] = b;
-            const float lo = __uint_as_float(b << 16), hi = __uint_as_float(b & 0xFFFF0000u);
-            rs0 = fmaf(lo, lo, rs0);
-            rs1 = fmaf(hi, hi, rs1);
-          }
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
           tcx::st16(acol + 16 * ch, pk);
+          planes[TB - 1][ch] = pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
 #pragma unroll
-          for (int pp = 0; pp < TB; ++pp) planes[pp][ch] = pw[pp];
+          for (int k = 0; k < TB - 1; ++k)
+            planes[k][ch] = ~(pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
+                              (pc.mag[k][3] << 24));
         };
         tcx::ld32(dcol, va);
         tcx::ld32(dcol + 32, vb);
@@ -687,8 +721,9 @@ static cudaError_t launch_quantize_t(const uint16_t *K, int64_t n, int64_t ldk,
   p.norms = reinterpret_cast<uint32_t *>(norms);
   p.err = device_error_ptr();
   if (!p.err) return cudaErrorInvalidSymbol;
-  for (int i = 0; i < 7; ++i) p.thr[i] = i + 1 < cb.L ? cb.thr[i] : 0.f;
-  for (int i = 0; i < 8; ++i) p.cent[i] = i < cb.L ? cb.cf[i] : 0.f;
+  const int H = cb.L / 2;
+  for (int i = 0; i < 4; ++i) p.mag[i] = i < H ? cb.cf[H + i] : 0.f;
+  for (int i = 0; i < 3; ++i) p.pos_thr[i] = i + 1 < H ? cb.thr[H + i] : 0.f;
   cudaError_t e = cudaFuncSetAttribute(turbo_quantize_kernel<TB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

@@ -334,11 +334,12 @@ JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,
  *
  * Per key k (d = 128; the residual sketch S is m x d with m = 128):
  *   x = k / ||k||  (0 for k = 0),  y = Pi x  (Pi: the stored bf16 rotation)
- *   cell_i = number of codebook boundaries strictly below y_i
- *   rt = bf16(y - c[cell])           (nearest, ties to even)
- *   code = cell bit planes, then sign(S rt);  norms = (||k||, ||rt||) binary16
+ *   cell_i = the cell of the centroid nearest y_i (a value exactly on a
+ *            boundary goes to the cell nearer zero; 0 to the cell below it)
+ *   r = y - c[cell],  rt = bf16(r)   (nearest, ties to even)
+ *   code = cell bit planes, then sign(S rt);  norms = (||k||, ||r||) binary16
  * and per query q, with w = Pi^{-T} q (Pinv from jl_turbo_rotation_init):
- *   s(q, k) = ||k|| * ( <w, c[cell]> + sqrt(pi/2)/m * ||rt|| * <S w, sign(S rt)> ).
+ *   s(q, k) = ||k|| * ( <w, c[cell]> + sqrt(pi/2)/m * ||r|| * <S w, sign(S rt)> ).
  * For an exactly orthogonal Pi the QJL stage in this rotated frame is the
  * pages' construction in distribution (S Pi^T is again an i.i.d. Gaussian
  * matrix); mapping the query with the inverse transpose of the stored Pi
@@ -349,7 +350,7 @@ JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,
  * (p < mse_bits) is words [p*d/32, (p+1)*d/32) and holds bit p of every
  * coordinate's cell (coordinate i at bit i % 32 of word i / 32 of the
  * plane); the QJL code follows (jl_quantize_keys layout).  norms: n x 2
- * binary16, element 0 = ||k||, element 1 = ||rt||.
+ * binary16, element 0 = ||k||, element 1 = ||r||.
  * -------------------------------------------------------------------------*/
 #define JL_TURBO_MAX_MSE_BITS 3
 

@@ -13,9 +13,8 @@ Tolerances, from the arithmetic of the two sides:
     whose float64 projection is below the oracle's allowance: 1e-5 ||rt||
     plus |S_ij| ulp(r_j) for every residual coordinate within BAND_Y of a
     bf16 rounding midpoint.
-  * norms: ||k|| within 1 binary16 step; ||rt|| (keys whose cells agree)
-    within 1 step plus the change that residual coordinates near a bf16
-    midpoint can make: sum over them of ulp_j |r_j| / ||r||.
+  * norms: ||k||, and ||r|| for keys whose cells agree, within 1 binary16
+    step (fp32 against float64 sums before the rounding).
   * decode (the oracle's codes fed to both sides): scores within
     1e-3 max(|ref|, rms of the row); outputs within 2e-2.
 """
@@ -98,16 +97,7 @@ def _quantize_case(bits, K, rot_seed=1):
     assert not np.any(sdiff & ~allowed), int(np.count_nonzero(sdiff & ~allowed))
     gn = H.fp16_bits(norms).reshape(n, 2)
     assert H.fp16_ulp_diff(gn[:, 0], ref["norm16"]).max() <= 1
-    # ||rt||: one binary16 step, plus what the residual coordinates that may
-    # round to the other bf16 neighbour can move it: sum of ulp_j |r_j| / ||r||
-    r = ref["r"]
-    a = np.abs(r)
-    ulp = 2.0 ** (np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7)
-    move = (ref["r_amb"] * ulp * (a + ulp)).sum(axis=1) / np.maximum(ref["rnorm"], 1e-30)
-    gval = oracle.fp16_bits_to_f64(gn[:, 1])
-    step = np.spacing(ref["rnorm16"].view(np.float16).astype(np.float16)).astype(np.float64)
-    rerr = np.abs(gval - ref["rnorm"])
-    assert np.all((rerr <= step + move)[ok]), float(np.max((rerr - step - move)[ok]))
+    assert H.fp16_ulp_diff(gn[:, 1], ref["rnorm16"])[ok].max(initial=0) <= 1
     return int(cdiff.sum()), int(sdiff.sum()), int((~ok).sum())
 
 
