@@ -101,21 +101,30 @@ def test_paged_append_decode_matches_oracle(cfg):
         if T == 0:
             assert torch.count_nonzero(out[b]) == 0
             continue
-        # codes and norms as they sit in the pool (the appended key's were
-        # checked above against the oracle's quantization)
+        # the oracle decodes its own codes of the sequence's keys (the pool's
+        # cache part holds exactly those; the GPU's appended code was checked
+        # above against the oracle's within the band)
         pos = np.arange(T)
         pg, sl = table[b, pos // P], pos % P
-        sig = np.stack([sp_h[pg, h, sl] for h in range(Hkv)])
-        n16 = np.stack([np_h[pg, h, sl] for h in range(Hkv)])
+        ref = [oracle.quantize(H.f64(K[h]), S64) for h in range(Hkv)]
+        sig = np.stack([r[0] for r in ref])
+        n16 = np.stack([r[2] for r in ref])
         if lens[b]:
-            for h in range(Hkv):
-                ref_sig = oracle.quantize(H.f64(K[h, :lens[b]]), S64)[0]
-                assert np.array_equal(sig[h, :lens[b]], ref_sig)
+            pool_sig = np.stack([sp_h[pg, h, sl] for h in range(Hkv)])
+            assert np.array_equal(pool_sig[:, :lens[b]], sig[:, :lens[b]])
         ref_out, ref_sc = oracle.decode(H.f64(Q[b])[None], S64, sig[None],
                                         oracle.fp16_bits_to_f64(n16)[None], H.f64(V)[None],
                                         scale, want_scores=True)
         g_sc = H.f64(sc[b, :, :T])[None]
-        assert H.score_violations(g_sc, ref_sc) == 0, b
+        # the appended key's score only when its GPU code and norm equal the
+        # oracle's (an in-band flip or a 1-ulp norm moves that one score)
+        same = True
+        if append:
+            pa, sa = table[b, lens[b] // P], lens[b] % P
+            same = (np.array_equal(sp_h[pa, :, sa], sig[:, -1])
+                    and np.array_equal(np_h[pa, :, sa], n16[:, -1]))
+        upto = T if same else T - 1
+        assert H.score_violations(g_sc[..., :upto], ref_sc[..., :upto]) == 0, b
         mabs, rel = H.output_errors(H.f64(out[b])[None], ref_out)
         assert mabs <= H.OUT_ABS and rel <= 1e-2, (b, mabs, rel)
 
