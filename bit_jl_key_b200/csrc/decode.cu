@@ -93,7 +93,7 @@ struct DecCfg {
   static constexpr int SIGN_CHUNKS = SIGN_BYTES / SIGN_CHUNK;  // multiple of 32
   static constexpr int DT = D / 16;                    // 16-dim output tiles
   static_assert(SIGN_CHUNKS % 32 == 0, "sign chunks per lane");
-  static_assert(TB == 0 || (!S8 && D == 128 && M % 128 == 0), "cell-plane codes: bf16, d = 128");
+  static_assert(TB == 0 || (D == 128 && M % 128 == 0), "cell-plane codes: d = 128");
   static_assert(STAGE_BYTES % 1024 == 0 && WARP_BYTES % 1024 == 0, "swizzle atoms");
 };
 
@@ -245,22 +245,42 @@ __global__ void __launch_bounds__(PROJ_THREADS)
                        float wc1) {
   griddep_launch_dependents();
   constexpr int MT = TB * D + M;
+  constexpr int HALVES = PROJ_THREADS / D;  // threads per output coordinate
+  static_assert(PROJ_THREADS % D == 0 && D % HALVES == 0, "query map tiling");
+  __shared__ float qsm[PROJ_VECS * D];
+  __shared__ float part[HALVES][PROJ_VECS * D];
   __shared__ float wsm[PROJ_VECS * D];
   const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
   const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
   for (int e = threadIdx.x; e < PROJ_VECS * D; e += PROJ_THREADS) {
-    const int j = e / D, i = e - (e / D) * D;
-    float acc = 0.f;
-    if (j < nx) {
-      const int64_t qb = (x0 + j) * D;
+    const int j = e / D;
+    const int64_t src = x0 * D + e;
+    qsm[e] = j >= nx ? 0.f
+             : QF32  ? reinterpret_cast<const float *>(Q)[src]
+                     : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[src]);
+  }
+  __syncthreads();
+  {
+    // thread (i, h): partial sums over columns c of part h, all four queries
+    // at once so that each Pinv element is read once
+    const int i = threadIdx.x % D, h = threadIdx.x / D;
+    constexpr int CP = D / HALVES;
+    float acc[PROJ_VECS] = {};
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        const float qc = QF32 ? reinterpret_cast<const float *>(Q)[qb + c]
-                              : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[qb + c]);
-        acc = fmaf(__ldg(Pinv + c * D + i), qc, acc);
-      }
+    for (int c = h * CP; c < (h + 1) * CP; ++c) {
+      const float pv = __ldg(Pinv + c * D + i);
+#pragma unroll
+      for (int j = 0; j < PROJ_VECS; ++j) acc[j] = fmaf(pv, qsm[j * D + c], acc[j]);
     }
-    wsm[e] = acc;
+#pragma unroll
+    for (int j = 0; j < PROJ_VECS; ++j) part[h][j * D + i] = acc[j];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < PROJ_VECS * D; e += PROJ_THREADS) {
+    float w = 0.f;
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) w += part[h][e];
+    wsm[e] = w;
   }
   __syncthreads();
   project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TB * D, MT);
@@ -519,7 +539,7 @@ template <int M, int D, bool S8, int TB = 0>
 __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t,
                                              const Ring<M, D, S8, TB> &ring,
                                              uint32_t (&afr)[DecCfg<M, D, S8, TB>::A_SMEM ? 1 : DecCfg<M, D, S8, TB>::NC][4],
-                                             float &hscale, int &usum) {
+                                             float (&hscale)[2], int (&usum)[2]) {
   using C = DecCfg<M, D, S8, TB>;
   auto put = [&](int c, const uint32_t (&a4)[4]) {
     if constexpr (C::A_SMEM) {
@@ -582,6 +602,66 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
       }
     }
     (void)hscale; (void)usum;
+  } else if constexpr (TB > 0) {
+    // cell-plane codes: lane t owns code words 4 lw + t; runs lw < TB are
+    // cell planes (the codebook-weighted w), the others residual signs (S w):
+    // one scale per segment, u ~= hscale[s] (256 hi + lo), |256 hi + lo| <= 32000
+    float am[2] = {0.f, 0.f};
+    if (live) {
+#pragma unroll
+      for (int lw = 0; lw < C::LW; ++lw) {
+        const float *src = urow + 32 * (4 * lw + t);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 v = ldg4(src + 4 * k);
+          const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+          am[lw < TB ? 0 : 1] = fmaxf(am[lw < TB ? 0 : 1], a);
+        }
+      }
+    }
+    float inv[2];
+#pragma unroll
+    for (int sg = 0; sg < 2; ++sg) {
+      am[sg] = fmaxf(am[sg], __shfl_xor_sync(0xffffffffu, am[sg], 1));
+      am[sg] = fmaxf(am[sg], __shfl_xor_sync(0xffffffffu, am[sg], 2));
+      hscale[sg] = am[sg] > 0.f ? am[sg] / 32000.f : 0.f;
+      inv[sg] = am[sg] > 0.f ? 32000.f / am[sg] : 0.f;
+    }
+    int isum[2] = {0, 0};
+#pragma unroll
+    for (int lw = 0; lw < C::LW; ++lw) {
+      const int sg = lw < TB ? 0 : 1;
+      const float *src = urow + 32 * (4 * lw + t);
+      float4 x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
+      // byte register p of the word holds coordinates p + 8j, j = 0..3
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        uint32_t a4[4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int pp = 2 * c2 + r;
+          int hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int ui = __float2int_rn(f4c(x[(pp + 8 * j) >> 2], pp & 3) * inv[sg]);
+            isum[sg] += ui;
+            hi[j] = (ui + 128) >> 8;
+            lo[j] = ui - (hi[j] << 8);
+          }
+          a4[2 * r] = pack_s8x4(hi[0], hi[1], hi[2], hi[3]);
+          a4[2 * r + 1] = pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        put(4 * lw + c2, a4);
+      }
+    }
+#pragma unroll
+    for (int sg = 0; sg < 2; ++sg) {
+      isum[sg] += __shfl_xor_sync(0xffffffffu, isum[sg], 1);
+      isum[sg] += __shfl_xor_sync(0xffffffffu, isum[sg], 2);
+      usum[sg] = isum[sg];
+    }
   } else {
     // pass 1: the head's largest |u| (4 lanes of the quad together)
     float amax = 0.f;
@@ -607,7 +687,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
     }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    hscale = amax > 0.f ? amax / 32000.f : 0.f;
+    hscale[0] = amax > 0.f ? amax / 32000.f : 0.f;
     const float inv = amax > 0.f ? 32000.f / amax : 0.f;
     int isum = 0;
     auto quant = [&](float x, int &hi, int &lo) {
@@ -661,7 +741,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
     }
     isum += __shfl_xor_sync(0xffffffffu, isum, 1);
     isum += __shfl_xor_sync(0xffffffffu, isum, 2);
-    usum = isum;
+    usum[0] = isum;
   }
   if constexpr (C::A_SMEM) __syncwarp();
 }
@@ -751,8 +831,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   int64_t cur_u = -1, kv_base = 0;
   int Gg = 0, b_idx = 0, hq0 = 0;
   float mx = -INFINITY, lsum = 0.f;
-  float hscale = 0.f;   // int8 scoring: value of one unit of S q for head g
-  int usum = 0;         // int8 scoring: sum of the quantized S q of head g
+  // int8 scoring: value of one unit of the query row for head g and the sum
+  // of its quantized entries, per segment (cell planes, residual signs)
+  float hscale[2] = {0.f, 0.f};
+  int usum[2] = {0, 0};
   float acc[C::DT][4];
   uint32_t afr[C::A_SMEM ? 1 : C::NC][4];
   bool failed = false;
@@ -870,10 +952,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // (cell-plane codes: raw over the planes, rawq over the residual signs)
     float raw[4][2], rawq[4][2];
     if constexpr (S8) {
-      int sc[4][4];
+      int sc[4][4], sq[4][4];
 #pragma unroll
-      for (int kg = 0; kg < 4; ++kg) sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0;
-      const int pbase = (M >= 128) ? 0 : 4 * (t & 1);
+      for (int kg = 0; kg < 4; ++kg) {
+        sc[kg][0] = sc[kg][1] = sc[kg][2] = sc[kg][3] = 0;
+        sq[kg][0] = sq[kg][1] = sq[kg][2] = sq[kg][3] = 0;
+      }
+      const int pbase = (C::CODE_BITS >= 128) ? 0 : 4 * (t & 1);
 #pragma unroll
       for (int c = 0; c < C::NC; ++c) {
         uint32_t a0, a1, a2, a3;
@@ -889,7 +974,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
         for (int kg = 0; kg < 4; ++kg) {
           uint32_t w0, w1;
           int p0, p1;
-          if constexpr (M >= 128) {
+          if constexpr (C::CODE_BITS >= 128) {
             w0 = wd[kg][q0 >> 3]; p0 = q0 & 7;
             w1 = wd[kg][q1 >> 3]; p1 = q1 & 7;
           } else {
@@ -898,15 +983,21 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           // bytes j = bits p + 8j: {0, 1} per coordinate
           const uint32_t b0 = (w0 >> p0) & 0x01010101u;
           const uint32_t b1 = (w1 >> p1) & 0x01010101u;
-          mma_s8_16832(sc[kg], a0, a1, a2, a3, b0, b1);
+          if (TB > 0 && c >= C::NC_MSE)
+            mma_s8_16832(sq[kg], a0, a1, a2, a3, b0, b1);
+          else
+            mma_s8_16832(sc[kg], a0, a1, a2, a3, b0, b1);
         }
       }
       // sum_i u_i sign_i = hscale * (2 * sum_{bit=1} u_int - sum u_int)
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-          raw[kg][j] = hscale * (float)(2 * (sc[kg][j] * 256 + sc[kg][j + 2]) - usum);
+        for (int j = 0; j < 2; ++j) {
+          raw[kg][j] = hscale[0] * (float)(2 * (sc[kg][j] * 256 + sc[kg][j + 2]) - usum[0]);
+          if constexpr (TB > 0)
+            rawq[kg][j] = hscale[1] * (float)(2 * (sq[kg][j] * 256 + sq[kg][j + 2]) - usum[1]);
+        }
     } else {
       float sc[4][4], sq[4][4];
 #pragma unroll
@@ -1449,6 +1540,10 @@ bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int
   return true;
 }
 
+// Scoring MMA of the cell-plane codes: int8 (k = 32 coordinates per MMA,
+// four coordinates per expanded register) unless a bf16 build is forced.
+constexpr bool TURBO_S8 = JL_DECODE_SCORE != 1;
+
 template <int TB>
 static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bool q_f32,
                                          const float *Pinv, const uint16_t *S,
@@ -1462,7 +1557,7 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
   DecMaps maps;
   if (!make_maps(&maps, V, codes, norms, (int64_t)pl.B * pl.Hkv, pl.T, M, D,
-                 DecCfg<M, D, false, TB>::KEY_SIGN_BYTES, 4))
+                 DecCfg<M, D, TURBO_S8, TB>::KEY_SIGN_BYTES, 4))
     return cudaErrorInvalidValue;
   int *err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidSymbol;
@@ -1479,7 +1574,7 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, codes, norms, scores, softmax_scale, M, err);
-  return launch_scorer_combine<M, D, false, false, TB>(pl, p, maps, out, stream);
+  return launch_scorer_combine<M, D, TURBO_S8, false, TB>(pl, p, maps, out, stream);
 }
 
 cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, bool q_f32,
