@@ -236,3 +236,93 @@ def test_search_argument_errors(lib):
     need = jl.jl_search_workspace_bytes(4, 256, 128, 10)
     assert need > 0 and call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
     assert jl.jl_search_workspace_bytes(4, 256, 128, 17) == 0
+
+
+# --------------------------------------------------------------------------
+# TurboQuant-prod entry points
+
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_turbo_codebook_matches_oracle_on_host(lib, bits):
+    # the library computes its codebook on the host (its own quadrature); it
+    # must equal the oracle's Lloyd-Max centroids rounded to float
+    from oracle import turbo as tq
+    for d in (3, 64, 128, 1000):
+        got = np.array(jl.jl_turbo_codebook(d, bits), dtype=np.float32)
+        assert np.array_equal(got, tq.lloyd_max(d, bits).astype(np.float32)), d
+
+
+def test_turbo_codebook_argument_errors(lib):
+    buf = (ctypes.c_float * 8)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    assert lib.jl_turbo_codebook(128, 2, NULL) == jl.JL_ERR_INVALID_ARG
+    assert lib.jl_turbo_codebook(2, 2, p) == jl.JL_ERR_UNSUPPORTED
+    assert lib.jl_turbo_codebook(128, 0, p) == jl.JL_ERR_UNSUPPORTED
+    assert lib.jl_turbo_codebook(128, 4, p) == jl.JL_ERR_UNSUPPORTED
+    assert lib.jl_turbo_codebook(128, 3, p) == jl.JL_OK
+
+
+def test_turbo_rotation_argument_errors(lib):
+    f = lib.jl_turbo_rotation_init
+    need = jl.jl_turbo_rotation_workspace_bytes(128)
+    assert need == 4 * 128 * 128 * 8
+    assert jl.jl_turbo_rotation_workspace_bytes(96) == 0
+    assert f(FAKE, FAKE, 96, 1, FAKE, need, NULL) == jl.JL_ERR_UNSUPPORTED
+    assert f(NULL, FAKE, 128, 1, FAKE, need, NULL) == jl.JL_ERR_INVALID_ARG
+    assert f(FAKE, MISALIGNED, 128, 1, FAKE, need, NULL) == jl.JL_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 128, 1, NULL, need, NULL) == jl.JL_ERR_WORKSPACE
+    assert f(FAKE, FAKE, 128, 1, FAKE, need - 1, NULL) == jl.JL_ERR_WORKSPACE
+
+
+def test_turbo_quantize_argument_errors(lib):
+    f = lib.jl_turbo_quantize_keys
+    ok = dict(K=FAKE, kt=jl.JL_BF16, n=10, ld=128, Pi=FAKE, S=FAKE, m=128, d=128, bits=2,
+              codes=FAKE, norms=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["K"], a["kt"], a["n"], a["ld"], a["Pi"], a["S"], a["m"], a["d"], a["bits"],
+                 a["codes"], a["norms"], NULL)
+
+    assert call(n=0) == jl.JL_OK
+    assert call(n=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(kt=jl.JL_F32) == jl.JL_ERR_UNSUPPORTED
+    assert call(m=256) == jl.JL_ERR_UNSUPPORTED
+    assert call(d=64) == jl.JL_ERR_UNSUPPORTED
+    assert call(bits=0) == jl.JL_ERR_UNSUPPORTED
+    assert call(bits=4) == jl.JL_ERR_UNSUPPORTED
+    for k in ("K", "Pi", "S", "codes", "norms"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(ld=100) == jl.JL_ERR_INVALID_ARG
+    assert call(ld=132) == jl.JL_ERR_INVALID_ARG          # 264-byte rows: not 16-byte multiples
+    assert call(K=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(norms=ctypes.c_void_p((1 << 20) + 2)) == jl.JL_ERR_INVALID_ARG
+
+
+def test_turbo_decode_argument_errors(lib):
+    f = lib.jl_turbo_decode_attention
+    need = jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 2)
+    assert need > 0
+    assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 3) == 0
+    assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 256, 128, 2) == 0
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, Pinv=FAKE, S=FAKE, codes=FAKE, norms=FAKE, V=FAKE, B=2,
+              Hq=8, Hkv=2, T=64, m=128, d=128, bits=2, scale=0.088, out=FAKE, sc=NULL, ws=FAKE,
+              wsb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["Q"], a["qt"], a["Pinv"], a["S"], a["codes"], a["norms"], a["V"], a["B"],
+                 a["Hq"], a["Hkv"], a["T"], a["m"], a["d"], a["bits"],
+                 ctypes.c_float(a["scale"]), a["out"], a["sc"], a["ws"], a["wsb"], NULL)
+
+    assert call(B=0) == jl.JL_OK
+    assert call(B=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(T=0) == jl.JL_ERR_INVALID_ARG
+    assert call(Hq=6, Hkv=4) == jl.JL_ERR_INVALID_ARG
+    assert call(bits=3) == jl.JL_ERR_UNSUPPORTED
+    assert call(m=256) == jl.JL_ERR_UNSUPPORTED
+    assert call(scale=float("nan")) == jl.JL_ERR_INVALID_ARG
+    for k in ("Q", "Pinv", "S", "codes", "norms", "V", "out"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(codes=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
+    assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
