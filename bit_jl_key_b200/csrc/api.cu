@@ -337,7 +337,8 @@ int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv
                               jl_stream_t stream) {
   if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
-  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > 2) return JL_ERR_UNSUPPORTED;
+  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+    return JL_ERR_UNSUPPORTED;
   if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
   if (B == 0) return JL_OK;
   if (!Q || !Pinv || !S || !codes || !norms || !V || !out) return JL_ERR_INVALID_ARG;
@@ -349,7 +350,7 @@ int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv
   if (!jlk::make_turbo_decode_plan(B, Hq, Hkv, T, m, d, mse_bits, &p)) return JL_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
     return JL_ERR_WORKSPACE;
-  double walsh[3];
+  double walsh[4];
   if (!jlk::turbo_codebook(d, mse_bits, nullptr, walsh)) return JL_ERR_UNSUPPORTED;
   return from_cuda(jlk::launch_turbo_decode(p, mse_bits, Q, q_dtype == JL_F32, Pinv, S, codes,
                                             norms, V, walsh, softmax_scale, out, scores,

@@ -61,12 +61,16 @@ constexpr int DEC_NORM_AREA = 128; // per stage: 40 fp16 norms; bulk-tensor copi
 #endif
 
 // TB > 0: TurboQuant-prod codes, TB cell bit planes of D bits ahead of the M
-// residual sign bits, scored as TB + 1 sign contractions (see turbo_scores).
+// residual sign bits.  A symmetric codebook's centroid is a sum of +-1 terms
+// over the planes: one per plane for TB <= 2, and for TB = 3 the three planes
+// plus their product (whose bit is the XOR of the three), so a key is scored
+// as TERMS + 1 sign contractions.
 template <int M, int D, bool S8, int TB = 0>
 struct DecCfg {
   static constexpr int STAGES = 2;                     // blocks in the ring
-  static constexpr int CODE_BITS = TB * D + M;         // bits per key
-  static constexpr int KEY_SIGN_BYTES = CODE_BITS / 8;
+  static constexpr int TERMS = TB == 3 ? 4 : TB;       // +-1 plane terms
+  static constexpr int CODE_BITS = TERMS * D + M;      // coordinates contracted per key
+  static constexpr int KEY_SIGN_BYTES = (TB * D + M) / 8;  // bytes stored per key
   static constexpr int SIGN_BYTES = DEC_KB * KEY_SIGN_BYTES;
   static constexpr int V_BYTES = DEC_KB * D * 2;       // 4 or 8 KB
   static constexpr int V_BOX = DEC_KB * 128;           // one 64-column box
@@ -74,7 +78,7 @@ struct DecCfg {
   // scoring MMA: bf16 m16n8k16 (16 coordinates per slice) or s8 m16n8k32 (32)
   static constexpr int KS = S8 ? 32 : 16;
   static constexpr int NC = CODE_BITS / KS;            // k slices
-  static constexpr int NC_MSE = TB * D / KS;           // slices of the cell planes
+  static constexpr int NC_MSE = TERMS * D / KS;        // slices of the cell planes
   static constexpr int A_REGS = 4 * NC;
   // A fragments in smem when they would crowd the registers; the cell-plane
   // codes keep theirs in registers (two CTAs per SM instead of one)
@@ -232,19 +236,24 @@ __global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restr
 
 // TurboQuant-prod query rows, four queries per CTA: w = Pinv^T q (so that
 // <w, Pi x> = <q, x> for the stored bf16 Pi), then the row
-//   [wc_0 w, ..., wc_{TB-1} w, S w]
-// whose dot product with the +-1 expansion of a key's code [planes, signs]
-// gives the two raw sums of the score: the cell planes' part is
-// <w, c[cell]> because c_j = sum_p wc_p (2 bit_p(j) - 1) for the symmetric
-// codebook (its single-bit Walsh coefficients; the others vanish for
-// TB <= 2).
+//   [wc_0 w, ..., wc_{TERMS-1} w, S w]
+// whose dot product with the +-1 expansion of a key's code [plane terms,
+// signs] gives the two raw sums of the score: the plane terms' part is
+// <w, c[cell]> because a symmetric codebook is the sum of its odd Walsh
+// terms, c_j = sum_S wc_S prod_{p in S} (2 bit_p(j) - 1) over the odd subsets
+// S of the planes (the single planes, and for three planes also all three).
+struct WalshCoef {
+  float c[4];  // coefficients of the plane terms, in code order
+};
+
 template <int M, int D, int TB, bool QF32>
 __global__ void __launch_bounds__(PROJ_THREADS)
     turbo_qproj_kernel(const void *__restrict__ Q, const float *__restrict__ Pinv,
-                       const uint16_t *__restrict__ S, float *__restrict__ U, int nq, float wc0,
-                       float wc1) {
+                       const uint16_t *__restrict__ S, float *__restrict__ U, int nq,
+                       const WalshCoef wc) {
   griddep_launch_dependents();
-  constexpr int MT = TB * D + M;
+  constexpr int TERMS = TB == 3 ? 4 : TB;
+  constexpr int MT = TERMS * D + M;
   constexpr int HALVES = PROJ_THREADS / D;  // threads per output coordinate
   static_assert(PROJ_THREADS % D == 0 && D % HALVES == 0, "query map tiling");
   __shared__ float qsm[PROJ_VECS * D];
@@ -283,12 +292,12 @@ __global__ void __launch_bounds__(PROJ_THREADS)
     wsm[e] = w;
   }
   __syncthreads();
-  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TB * D, MT);
+  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TERMS * D, MT);
   for (int e = threadIdx.x; e < nx * D; e += PROJ_THREADS) {
     const int j = e / D, i = e - (e / D) * D;
     float *row = U + (x0 + j) * MT;
-    row[i] = wc0 * wsm[e];
-    if constexpr (TB > 1) row[D + i] = wc1 * wsm[e];
+#pragma unroll
+    for (int k = 0; k < TERMS; ++k) row[k * D + i] = wc.c[k] * wsm[e];
   }
 }
 
@@ -615,7 +624,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
         for (int k = 0; k < 8; ++k) {
           const float4 v = ldg4(src + 4 * k);
           const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-          am[lw < TB ? 0 : 1] = fmaxf(am[lw < TB ? 0 : 1], a);
+          am[lw < C::TERMS ? 0 : 1] = fmaxf(am[lw < C::TERMS ? 0 : 1], a);
         }
       }
     }
@@ -630,7 +639,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
     int isum[2] = {0, 0};
 #pragma unroll
     for (int lw = 0; lw < C::LW; ++lw) {
-      const int sg = lw < TB ? 0 : 1;
+      const int sg = lw < C::TERMS ? 0 : 1;
       const float *src = urow + 32 * (4 * lw + t);
       float4 x[8];
 #pragma unroll
@@ -929,7 +938,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
       const uint32_t kp = sg + (kg * 8 + g) * C::KEY_SIGN_BYTES;
-      if constexpr (TB > 0) {
+      if constexpr (TB == 3) {
+        // stored words: planes 0-2, then the residual signs; the product
+        // term's word is the XOR of the three planes
+#pragma unroll
+        for (int lw = 0; lw < 3; ++lw)
+          asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][lw]) : "r"(kp + (4 * lw + t) * 4));
+        asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][4]) : "r"(kp + (12 + t) * 4));
+        wd[kg][3] = wd[kg][0] ^ wd[kg][1] ^ wd[kg][2];
+      } else if constexpr (TB > 0) {
 #pragma unroll
         for (int lw = 0; lw < C::LW; ++lw)
           asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(wd[kg][lw]) : "r"(kp + (4 * lw + t) * 4));
@@ -1533,9 +1550,10 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
 
 bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int bits,
                             DecodePlan *pl) {
-  if (m != 128 || d != 128 || bits < 1 || bits > 2) return false;
+  if (m != 128 || d != 128 || bits < 1 || bits > 3) return false;
   if (!plan_common(B, Hq, Hkv, T, m, d, pl)) return false;
-  pl->u_bytes = round_up((size_t)B * Hq * (bits * d + m) * sizeof(float), 256);
+  const int terms = bits == 3 ? 4 : bits;
+  pl->u_bytes = round_up((size_t)B * Hq * (terms * d + m) * sizeof(float), 256);
   pl->total_bytes = pl->u_bytes + pl->partial_bytes;
   return true;
 }
@@ -1563,13 +1581,12 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
   if (err == nullptr) return cudaErrorInvalidSymbol;
   const int bh = pl.B * pl.Hq;
   const int qctas = (bh + PROJ_VECS - 1) / PROJ_VECS;
-  const float wc0 = (float)walsh[0], wc1 = (float)walsh[1];
+  WalshCoef wc;
+  for (int k = 0; k < 4; ++k) wc.c[k] = (float)walsh[k];
   if (q_f32)
-    turbo_qproj_kernel<M, D, TB, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh,
-                                                                          wc0, wc1);
+    turbo_qproj_kernel<M, D, TB, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc);
   else
-    turbo_qproj_kernel<M, D, TB, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh,
-                                                                           wc0, wc1);
+    turbo_qproj_kernel<M, D, TB, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecParams p;
@@ -1587,6 +1604,9 @@ cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, b
                                     softmax_scale, out, scores, workspace, stream);
   if (bits == 2)
     return launch_turbo_decode_t<2>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
+                                    softmax_scale, out, scores, workspace, stream);
+  if (bits == 3)
+    return launch_turbo_decode_t<3>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
                                     softmax_scale, out, scores, workspace, stream);
   return cudaErrorNotSupported;
 }

@@ -52,7 +52,7 @@ bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols,
 }
 
 // TurboQuant-prod (turbo_tc.cu): the stage-one codebook (host, cached; false
-// for unsupported d / bits), its single-bit Walsh coefficients, the rotation
+// for unsupported d / bits), its odd Walsh coefficients (walsh[4]), the rotation
 // and its inverse, and the tensor-core quantizer (d = m = 128, bf16 keys).
 bool turbo_codebook(int d, int bits, float *centroids, double *walsh);
 size_t turbo_rotation_workspace_bytes(int d);
@@ -82,7 +82,7 @@ bool make_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d,
 bool make_paged_plan(int B, int Hq, int Hkv, int64_t max_len, int m, int d,
                      DecodePlan *plan);
 
-// TurboQuant-prod decode (decode.cu): d = m = 128, bits 1 or 2.
+// TurboQuant-prod decode (decode.cu): d = m = 128, bits 1 to 3.
 bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int bits,
                             DecodePlan *plan);
 cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, bool q_f32,

@@ -153,7 +153,7 @@ struct Codebook {
   double c[8];      // centroids, ascending
   float cf[8];      // as float
   float thr[7];     // float((c_i + c_{i+1}) / 2)
-  double walsh[3];  // c_j = sum_p walsh[p] * (2 bit_p(j) - 1)  (bits <= 2)
+  double walsh[4];  // odd Walsh terms: single planes, then (3 bits) all three
 };
 
 static const Codebook *codebook(int d, int bits) {
@@ -173,13 +173,22 @@ static const Codebook *codebook(int d, int bits) {
   }
   for (int j = 0; j < cb.L; ++j) cb.cf[j] = (float)cb.c[j];
   for (int j = 0; j + 1 < cb.L; ++j) cb.thr[j] = (float)(0.5 * (cb.c[j] + cb.c[j + 1]));
-  // Walsh coefficients of the single-bit terms: (1/L) sum_j c_j e_p(j)
-  for (int p = 0; p < 3; ++p) {
+  // Walsh coefficients (1/L) sum_j c_j prod_{p in S} e_p(j), e_p = +-1 from
+  // bit p of j, for the odd subsets S (the even ones vanish for a symmetric
+  // codebook): {p} for each plane, then {0, 1, 2} with three planes
+  auto walsh_of = [&](int mask) {
     double s = 0.0;
-    if (p < bits)
-      for (int j = 0; j < cb.L; ++j) s += cb.c[j] * (((j >> p) & 1) ? 1.0 : -1.0);
-    cb.walsh[p] = s / cb.L;
-  }
+    for (int j = 0; j < cb.L; ++j) {
+      double e = 1.0;
+      for (int p = 0; p < bits; ++p)
+        if ((mask >> p) & 1) e *= ((j >> p) & 1) ? 1.0 : -1.0;
+      s += cb.c[j] * e;
+    }
+    return s / cb.L;
+  };
+  for (int k = 0; k < 4; ++k) cb.walsh[k] = 0.0;
+  for (int p = 0; p < bits; ++p) cb.walsh[p] = walsh_of(1 << p);
+  if (bits == 3) cb.walsh[3] = walsh_of(7);
   return &cache.emplace(key, cb).first->second;
 }
 
@@ -740,7 +749,7 @@ bool turbo_codebook(int d, int bits, float *centroids, double *walsh) {
   if (centroids)
     for (int j = 0; j < cb->L; ++j) centroids[j] = cb->cf[j];
   if (walsh)
-    for (int p = 0; p < 3; ++p) walsh[p] = cb->walsh[p];
+    for (int p = 0; p < 4; ++p) walsh[p] = cb->walsh[p];
   return true;
 }
 

@@ -425,7 +425,7 @@ JL_API size_t jl_turbo_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T,
  *   out    : out, device, B x Hq x d bf16.
  *   scores : optional out, B x Hq x T fp32 (s before softmax_scale).
  *   workspace : device scratch of jl_turbo_decode_workspace_bytes(...).
- * Supported: d = m = 128, mse_bits 1 or 2.  B == 0 is a no-op; T >= 1.
+ * Supported: d = m = 128, mse_bits 1 to 3.  B == 0 is a no-op; T >= 1.
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
  * JL_ERR_CUDA.
  */

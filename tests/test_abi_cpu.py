@@ -302,7 +302,8 @@ def test_turbo_decode_argument_errors(lib):
     f = lib.jl_turbo_decode_attention
     need = jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 2)
     assert need > 0
-    assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 3) == 0
+    assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 4) == 0
+    assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 128, 128, 3) > need
     assert jl.jl_turbo_decode_workspace_bytes(2, 8, 2, 64, 256, 128, 2) == 0
     ok = dict(Q=FAKE, qt=jl.JL_BF16, Pinv=FAKE, S=FAKE, codes=FAKE, norms=FAKE, V=FAKE, B=2,
               Hq=8, Hkv=2, T=64, m=128, d=128, bits=2, scale=0.088, out=FAKE, sc=NULL, ws=FAKE,
@@ -318,7 +319,7 @@ def test_turbo_decode_argument_errors(lib):
     assert call(B=-1) == jl.JL_ERR_INVALID_ARG
     assert call(T=0) == jl.JL_ERR_INVALID_ARG
     assert call(Hq=6, Hkv=4) == jl.JL_ERR_INVALID_ARG
-    assert call(bits=3) == jl.JL_ERR_UNSUPPORTED
+    assert call(bits=4) == jl.JL_ERR_UNSUPPORTED
     assert call(m=256) == jl.JL_ERR_UNSUPPORTED
     assert call(scale=float("nan")) == jl.JL_ERR_INVALID_ARG
     for k in ("Q", "Pinv", "S", "codes", "norms", "V", "out"):

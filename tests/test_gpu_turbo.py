@@ -156,7 +156,7 @@ def _decode_inputs(bits, B, Hq, Hkv, T, seed, qdtype=torch.bfloat16):
     return gpu_in, want
 
 
-@pytest.mark.parametrize("bits", [1, 2])
+@pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("B,Hq,Hkv,T", [(2, 8, 2, 300), (1, 4, 4, 1), (2, 32, 8, 4096),
                                         (1, 8, 1, 1001)])
 def test_decode_matches_oracle(bits, B, Hq, Hkv, T):
@@ -211,9 +211,75 @@ def test_end_to_end_library_rotation_and_codes():
 def test_decode_rejects_bad_arguments():
     torch.cuda.set_device(0)
     L = jl.load()
-    assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 128, 3) == 0
+    assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 128, 4) == 0
     assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 256, 128, 2) == 0
     assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 128, 2) > 0
     st = L.jl_turbo_quantize_keys(None, jl.JL_F32, 4, 128, None, None, 128, 128, 2, None, None,
                                   None)
     assert st == jl.JL_ERR_UNSUPPORTED
+
+
+def test_turbo_gqa_full_size_sampled_units():
+    # the turbo-gqa cache at full size, in the bench's launch configuration:
+    # library rotation, sketch and quantizer over all 2,097,152 keys, then one
+    # decode.  Sampled (b, kv-head) units: their codes are checked against the
+    # oracle's, then the oracle's codes are planted in the GPU cache so that
+    # the sampled heads' scores and outputs compare exactly-defined quantities.
+    torch.cuda.set_device(0)
+    w = workloads.TURBO_GQA
+    bits = workloads.TURBO_MSE_BITS
+    dev = "cuda"
+    Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED)
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed)
+    pit_bits = tq.rotation_bf16_bits(w.d, workloads.TURBO_ROTATION_SEED)
+    assert np.array_equal(Pi.cpu().view(torch.int16).numpy().view(np.uint16), pit_bits)
+    Pit = oracle.bf16_bits_to_f64(pit_bits)
+    S64 = oracle.sketch(w.m, w.d, w.sketch_seed)
+    c = tq.lloyd_max(w.d, bits)
+    K = workloads.keys(w, dev)
+    V = workloads.values(w, dev)
+    Q = workloads.queries(w, dev)
+    codes, norms = jl.jl_turbo_quantize_keys(K.view(-1, w.d), Pi, S, bits)
+    codes = codes.view(w.B, w.Hkv, w.T, -1)
+    norms = norms.view(w.B, w.Hkv, w.T, 2)
+    torch.cuda.synchronize()
+    assert jl.jl_device_error() == 0
+    units = [(0, 0), (7, 7), (3, 5)]
+    refs = {}
+    for (b, hk) in units:
+        ref = tq.quantize(H.f64(K[b, hk]), Pit, c, S64, band_abs=BAND_Y, band_rel=BAND_SIGN)
+        gw = H.u32(codes[b, hk])
+        gcell = tq.unpack_planes(gw[:, :bits * D // 32], D, bits)
+        cdiff = gcell != ref["cell"]
+        assert not np.any(cdiff & ~ref["cell_band"]), (b, hk)
+        ok = ~cdiff.any(axis=1)
+        sdiff = (H.code_bits(gw[:, bits * D // 32:], M) != H.code_bits(ref["signs"], M)) & ok[:, None]
+        assert not np.any(sdiff & ~(np.abs(ref["proj"]) < ref["sign_allow"])), (b, hk)
+        gn = H.fp16_bits(norms[b, hk])
+        assert H.fp16_ulp_diff(gn[:, 0], ref["norm16"]).max() <= 1
+        assert H.fp16_ulp_diff(gn[:, 1], ref["rnorm16"])[ok].max(initial=0) <= 1
+        rc = np.concatenate([tq.pack_planes(ref["cell"], bits), ref["signs"]], axis=1)
+        codes[b, hk] = torch.from_numpy(rc.view(np.int32)).to(dev)
+        norms[b, hk] = torch.from_numpy(
+            np.stack([ref["norm16"], ref["rnorm16"]], axis=1).view(np.float16)).to(dev)
+        refs[(b, hk)] = ref
+        print(f"turbo-gqa unit {(b, hk)}: {int(cdiff.sum())} in-band cells, "
+              f"{int(sdiff.sum())} allowed sign flips")
+    del K
+    out, sc = jl.jl_turbo_decode_attention(Q, Pinv, S, codes, norms, V, bits,
+                                           softmax_scale=w.softmax_scale, want_scores=True)
+    torch.cuda.synchronize()
+    assert jl.jl_device_error() == 0
+    for (b, hk) in units:
+        ref = refs[(b, hk)]
+        hqs = list(range(hk * w.G, (hk + 1) * w.G))
+        ref_out, ref_sc = tq.decode(H.f64(Q[b, hqs])[None], Pit, S64, c,
+                                    ref["cell"].reshape(1, 1, w.T, D),
+                                    ref["signs"].reshape(1, 1, w.T, -1),
+                                    oracle.fp16_bits_to_f64(ref["norm16"]).reshape(1, 1, w.T),
+                                    oracle.fp16_bits_to_f64(ref["rnorm16"]).reshape(1, 1, w.T),
+                                    H.f64(V[b, hk])[None, None], w.softmax_scale,
+                                    want_scores=True)
+        assert H.score_violations(H.f64(sc[b, hqs])[None], ref_sc) == 0, (b, hk)
+        mabs, rel = H.output_errors(H.f64(out[b, hqs])[None], ref_out)
+        assert mabs <= H.OUT_ABS and rel <= 1e-2, (b, hk, mabs, rel)
