@@ -28,10 +28,14 @@
 //   * An expander thread copies its code row of the tile two ahead into a
 //     shared-memory ring with cp.async while it expands the current one.
 //
-// One persistent CTA per SM, 9 warps with fixed roles:
-//   warps 0-3  expand: thread r owns code row r of the tile.
-//   warps 4-7  epilogue: warp w reads TMEM lane quadrant w % 4.
-//   warp 8     owns the TMEM allocation; lane 0 issues the MMAs of a tile
+// One persistent CTA per SM, 13 warps with fixed roles:
+//   warps 0-7  expand: warp w writes TMEM lane quadrant w % 4 (code rows
+//              32 (w % 4) .. + 31 of the tile) for part w / 4 of the tile's
+//              K-chunks (the first or the second half), so two warps expand
+//              each row at once; each thread copies its half of its code
+//              row two tiles ahead.
+//   warps 8-11 epilogue: warp w reads TMEM lane quadrant w % 4.
+//   warp 12    owns the TMEM allocation; lane 0 issues the MMAs of a tile
 //              into one of two accumulators and commits them to the barriers
 //              that free the Z chunks and publish the accumulator.
 // Every mbarrier wait is bounded (about 2 s of GPU time); a wait that runs
@@ -48,7 +52,8 @@ namespace dq {
 constexpr int BM = 128;          // codes per tile (MMA M)
 constexpr int CHUNK_K = 64;      // coordinates per Z chunk
 constexpr int CHUNK_COLS = CHUNK_K / 2;  // TMEM columns of a Z chunk (bf16 pairs)
-constexpr int EXP_WARPS = 4, EPI_WARPS = 4;
+constexpr int EXP_PARTS = 2;     // expander warps per TMEM lane quadrant
+constexpr int EXP_WARPS = 4 * EXP_PARTS, EPI_WARPS = 4;
 constexpr int MMA_WARP = EXP_WARPS + EPI_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int CODE_SLOTS = 3;    // code rows in flight: the tile and two ahead
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::RING; ++s) {
-      mbar_init(zfull_bar(s), EXP_WARPS);  // one arrive per expander warp
+      mbar_init(zfull_bar(s), 4);          // one arrive per quadrant's expander warp
       mbar_init(zempty_bar(s), 1);         // MMA commit
     }
     for (int a = 0; a < C::ACC; ++a) {
@@ -313,32 +318,48 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int64_t ntiles = p.num_tiles;
 
   if (warp < EXP_WARPS) {
-    // ---------------- expand: thread r owns row r of every tile; its code
-    // row of the tile two ahead is copied into shared memory meanwhile
-    const int r = threadIdx.x;
-    int64_t c = 0;  // chunks produced
-    bool ok = true;
-    const uint32_t crow = base + C::OFF_C + r * C::CODE_ROW;
+    // ---------------- expand: quadrant q = warp % 4 (row r = 32 q + lane),
+    // part pt = warp / 4: chunks [kc0, kc0 + nk) of every tile; the part's
+    // code words of the tile two ahead are copied meanwhile
+    const int q = warp & 3, pt = warp >> 2;
+    const int r = 32 * q + lane;
+    constexpr int KP = (C::KCH + EXP_PARTS - 1) / EXP_PARTS;  // chunks per part
+    const int kc0 = pt * KP;
+    const int nk = C::KCH - kc0 < KP ? C::KCH - kc0 : KP;
+    bool ok = nk > 0;
+    const uint32_t pbytes = (uint32_t)(KP * 8);             // 2 code words per chunk
+    const uint32_t crow = base + C::OFF_C + r * C::CODE_ROW + pt * pbytes;
     auto code_slot = [&](int64_t it) { return crow + (uint32_t)((it % CODE_SLOTS) * BM * C::CODE_ROW); };
-    for (int k = 0; k < CODE_SLOTS - 1; ++k) {
-      const int64_t row = ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BM + r;
-      copy_code_row<M>(code_slot(k), p.signs, row, row < p.n);
-    }
+    auto copy_part = [&](uint32_t dst, int64_t row) {
+      const bool live = row < p.n;
+      const uint8_t *src = reinterpret_cast<const uint8_t *>(p.signs + (live ? row : 0) * (M / 32)) +
+                           pt * pbytes;
+      if constexpr (KP * 8 >= 16) {
+#pragma unroll
+        for (int u = 0; u < KP * 8 / 16; ++u) cp_async_16(dst + 16 * u, src + 16 * u, live ? 16 : 0);
+      } else {
+        cp_async_8(dst, src, live ? 8 : 0);
+      }
+      cp_async_commit();
+    };
+    if (ok)
+      for (int k = 0; k < CODE_SLOTS - 1; ++k)
+        copy_part(code_slot(k), ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BM + r);
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
-      {
-        const int64_t row = (tile + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BM + r;
-        copy_code_row<M>(code_slot(it + CODE_SLOTS - 1), p.signs, row, row < p.n);
-      }
-      cp_async_wait<CODE_SLOTS - 1>();  // this tile's row has landed
-      uint32_t cur[C::CODE_WORDS];
+      copy_part(code_slot(it + CODE_SLOTS - 1),
+                (tile + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BM + r);
+      cp_async_wait<CODE_SLOTS - 1>();  // this tile's words have landed
+      uint32_t cur[2 * KP];
       {
         const uint8_t *src = gbase + (code_slot(it) - base);
 #pragma unroll
-        for (int i = 0; i < C::CODE_WORDS; ++i) cur[i] = reinterpret_cast<const uint32_t *>(src)[i];
+        for (int i = 0; i < 2 * KP; ++i) cur[i] = reinterpret_cast<const uint32_t *>(src)[i];
       }
 #pragma unroll
-      for (int kc = 0; kc < C::KCH; ++kc, ++c) {
+      for (int kk = 0; kk < KP; ++kk) {
+        if (kk >= nk) break;
+        const int64_t c = it * C::KCH + kc0 + kk;  // global chunk index
         const int s = (int)(c % C::RING);
         const uint32_t ph = (uint32_t)((c / C::RING) & 1);
         if (!wait_phase(zempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
@@ -350,12 +371,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t z[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const uint32_t w = cur[2 * kc + half];  // rows past the end expand a zero code
+          const uint32_t w = cur[2 * kk + half];  // rows past the end expand a zero code
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             z[16 * half + j] = ((w << (15 - j)) & 0x80008000u) ^ 0xBF80BF80u;
         }
-        tmem_st32(tmem_base + ((uint32_t)(32 * warp) << 16) +
+        tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) +
                       (uint32_t)(C::Z_COL0 + s * CHUNK_COLS), z);
         tmem_st_wait();
         tc_fence_before();
@@ -385,16 +406,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * D);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + c0, v);
-        tmem_ld_wait(v);
+      // 32 columns: scale, round to bf16, stage as 4 units of 16 B in box
+      // c0/64, row `lane`
+      auto emit = [&](const uint32_t (&v)[32], int c0) {
         uint32_t o[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * f, __uint_as_float(v[2 * e + 1]) * f);
-        // columns c0..c0+31 = 4 units of 16 B in box c0/64, row `lane`
         uint8_t *box = stage + (c0 >> 6) * C::OBOX + lane * 128;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -402,6 +420,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           *reinterpret_cast<uint4 *>(box + ((unit ^ (lane & 7)) << 4)) =
               make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
+      };
+      // the loads are double-buffered: group g + 1 is in flight while g is
+      // emitted
+      uint32_t va[32], vb[32];
+      tmem_ld32(trow, va);
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        tmem_ld_wait(va);
+        tmem_ld32(trow + c0 + 32, vb);
+        emit(va, c0);
+        tmem_ld_wait(vb);
+        if (c0 + 64 < D) tmem_ld32(trow + c0 + 64, va);
+        emit(vb, c0 + 32);
       }
       tc_fence_before();
       fence_async_smem();
