@@ -54,7 +54,8 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_decode_attention_paged", "jl_dequantize_keys", "jl_search_workspace_bytes",
             "jl_search_topk", "jl_turbo_codebook", "jl_turbo_rotation_workspace_bytes",
             "jl_turbo_rotation_init", "jl_turbo_quantize_keys", "jl_turbo_decode_workspace_bytes",
-            "jl_turbo_decode_attention")
+            "jl_turbo_decode_attention", "jl_turbo_decode_paged_workspace_bytes",
+            "jl_turbo_decode_attention_paged")
 
 _lib = None
 
@@ -120,6 +121,12 @@ def load():
     L.jl_turbo_decode_attention.restype = i32
     L.jl_turbo_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i64,
                                             i32, i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+    L.jl_turbo_decode_paged_workspace_bytes.restype = sz
+    L.jl_turbo_decode_paged_workspace_bytes.argtypes = [i32, i32, i32, i64, i32, i32, i32]
+    L.jl_turbo_decode_attention_paged.restype = i32
+    L.jl_turbo_decode_attention_paged.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32,
+                                                  i32, vp, i32, vp, i32, i32, i32, i64, i32, i32,
+                                                  i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.jl_bf16_from_f64.restype = ctypes.c_uint16
@@ -521,4 +528,57 @@ def jl_turbo_decode_attention(Q, Pinv, S, codes, norms, V, mse_bits, softmax_sca
                                        ctypes.c_float(softmax_scale), _ptr(out), _ptr(scores),
                                        _ptr(workspace), workspace.numel(), _stream(Q, stream)),
            "jl_turbo_decode_attention")
+    return (out, scores) if scores is not None else out
+
+
+def jl_turbo_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d, mse_bits) -> int:
+    return int(load().jl_turbo_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d, mse_bits))
+
+
+def jl_turbo_decode_attention_paged(Q, Pinv, S, code_pages, norm_pages, value_pages, block_table,
+                                    seq_lens, max_len, mse_bits, Pi=None, K_new=None, V_new=None,
+                                    softmax_scale=None, out=None, scores=None, want_scores=False,
+                                    workspace=None, stream=None):
+    """One decode step over a paged TurboQuant-prod cache of ragged sequences.
+
+    Pools: code_pages int32 [P_n, Hkv, P, words], norm_pages fp16 [P_n, Hkv,
+    P, 2], value_pages bf16 [P_n, Hkv, P, d].  With K_new / V_new [B, Hkv, d]
+    (and the rotation Pi) the new key of every sequence is quantized and stored
+    at position seq_lens[b] first.  Returns out [B, Hq, d] (and scores)."""
+    L = load()
+    B, Hq, d = Q.shape
+    num_pages, Hkv, P, words = code_pages.shape
+    m = S.shape[0]
+    assert words == turbo_code_words(mse_bits, m, d)
+    _need_cuda(Q, Pinv, S, code_pages, norm_pages, value_pages, block_table, seq_lens, K_new,
+               V_new, Pi)
+    assert norm_pages.shape == (num_pages, Hkv, P, 2) and norm_pages.dtype == torch.float16
+    assert value_pages.shape == (num_pages, Hkv, P, d) and value_pages.dtype == torch.bfloat16
+    assert block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.shape[0] == B
+    assert seq_lens.dtype == torch.int32 and seq_lens.shape == (B,)
+    for t in (Q, Pinv, S, code_pages, norm_pages, value_pages, block_table, seq_lens, K_new, V_new,
+              Pi):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("paged decode inputs must be contiguous")
+    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    kt = JL_BF16
+    if K_new is not None:
+        assert K_new.shape == (B, Hkv, d) and V_new is not None and V_new.shape == (B, Hkv, d)
+        assert Pi is not None and Pi.shape == (d, d) and Pi.dtype == torch.bfloat16
+        kt = JL_F32 if K_new.dtype == torch.float32 else JL_BF16
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=Q.device)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, max_len), dtype=torch.float32, device=Q.device)
+    need = jl_turbo_decode_paged_workspace_bytes(B, Hq, Hkv, max_len, m, d, mse_bits)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_turbo_decode_attention_paged(
+        _ptr(Q), qt, _ptr(K_new), kt, _ptr(V_new), _ptr(Pi), _ptr(Pinv), _ptr(S),
+        _ptr(code_pages), _ptr(norm_pages), _ptr(value_pages), num_pages, P, _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, max_len, m, d, mse_bits,
+        ctypes.c_float(softmax_scale), _ptr(out), _ptr(scores), _ptr(workspace),
+        workspace.numel(), _stream(Q, stream)), "jl_turbo_decode_attention_paged")
     return (out, scores) if scores is not None else out

@@ -357,6 +357,59 @@ int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv
                                             workspace, (cudaStream_t)stream));
 }
 
+size_t jl_turbo_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len, int m,
+                                             int d, int mse_bits) {
+  return jl_turbo_decode_workspace_bytes(B, Hq, Hkv, max_len, m, d, mse_bits);
+}
+
+int jl_turbo_decode_attention_paged(
+    const void *Q, jl_dtype q_dtype, const void *K_new, jl_dtype k_dtype, const uint16_t *V_new,
+    const uint16_t *Pi, const float *Pinv, const uint16_t *S, uint32_t *code_pages,
+    uint16_t *norm_pages, uint16_t *value_pages, int num_pages, int page_tokens,
+    const int32_t *block_table, int max_pages, const int32_t *seq_lens, int B, int Hq, int Hkv,
+    int64_t max_len, int m, int d, int mse_bits, float softmax_scale, uint16_t *out,
+    float *scores, void *workspace, size_t workspace_bytes, jl_stream_t stream) {
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (K_new && k_dtype != JL_BF16 && k_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || max_len < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
+  if (num_pages < 1 || max_pages < 1 || page_tokens < 32 || page_tokens % 32 != 0)
+    return JL_ERR_INVALID_ARG;
+  if ((int64_t)max_pages * page_tokens < max_len) return JL_ERR_INVALID_ARG;
+  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+    return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
+  if (B == 0) return JL_OK;
+  if (!Q || !Pinv || !S || !code_pages || !norm_pages || !value_pages || !block_table ||
+      !seq_lens || !out)
+    return JL_ERR_INVALID_ARG;
+  if (K_new && (!V_new || !Pi)) return JL_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(Pinv, 16) || !aligned(S, 16) || !aligned(code_pages, 16) ||
+      !aligned(norm_pages, 16) || !aligned(value_pages, 16) || !aligned(out, 4) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || (K_new && !aligned(K_new, 16)) ||
+      (V_new && !aligned(V_new, 16)) || (Pi && !aligned(Pi, 16)) ||
+      (scores && !aligned(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  jlk::DecodePlan p;
+  if (!jlk::make_turbo_decode_plan(B, Hq, Hkv, max_len, m, d, mse_bits, &p))
+    return JL_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
+    return JL_ERR_WORKSPACE;
+  jlk::TurboPagedArgs t;
+  t.Pi = Pi;
+  t.Pinv = Pinv;
+  if (!jlk::turbo_codebook(d, mse_bits, nullptr, t.walsh) ||
+      !jlk::turbo_magnitudes(d, mse_bits, t.mag, t.pos_thr))
+    return JL_ERR_UNSUPPORTED;
+  jlk::PagedArgs a;
+  a.Q = Q; a.q_f32 = q_dtype == JL_F32;
+  a.K_new = K_new; a.k_f32 = k_dtype == JL_F32; a.V_new = V_new; a.S = S;
+  a.sign_pages = code_pages; a.norm_pages = norm_pages; a.value_pages = value_pages;
+  a.num_pages = num_pages; a.page_tokens = page_tokens;
+  a.block_table = block_table; a.max_pages = max_pages; a.seq_lens = seq_lens;
+  a.softmax_scale = softmax_scale; a.out = out; a.scores = scores; a.workspace = workspace;
+  return from_cuda(jlk::launch_turbo_decode_paged(p, mse_bits, a, t, (cudaStream_t)stream));
+}
+
 int jl_device_error(int *code, jl_stream_t stream) {
   if (!code) return JL_ERR_INVALID_ARG;
   *code = 0;

@@ -247,11 +247,11 @@ struct WalshCoef {
 };
 
 template <int M, int D, int TB, bool QF32>
-__global__ void __launch_bounds__(PROJ_THREADS)
-    turbo_qproj_kernel(const void *__restrict__ Q, const float *__restrict__ Pinv,
-                       const uint16_t *__restrict__ S, float *__restrict__ U, int nq,
-                       const WalshCoef wc) {
-  griddep_launch_dependents();
+__device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
+                                                 const float *__restrict__ Pinv,
+                                                 const uint16_t *__restrict__ S,
+                                                 float *__restrict__ U, int nq,
+                                                 const WalshCoef &wc, int64_t x0) {
   constexpr int TERMS = TB == 3 ? 4 : TB;
   constexpr int MT = TERMS * D + M;
   constexpr int HALVES = PROJ_THREADS / D;  // threads per output coordinate
@@ -259,7 +259,6 @@ __global__ void __launch_bounds__(PROJ_THREADS)
   __shared__ float qsm[PROJ_VECS * D];
   __shared__ float part[HALVES][PROJ_VECS * D];
   __shared__ float wsm[PROJ_VECS * D];
-  const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
   const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
   for (int e = threadIdx.x; e < PROJ_VECS * D; e += PROJ_THREADS) {
     const int j = e / D;
@@ -299,6 +298,15 @@ __global__ void __launch_bounds__(PROJ_THREADS)
 #pragma unroll
     for (int k = 0; k < TERMS; ++k) row[k * D + i] = wc.c[k] * wsm[e];
   }
+}
+
+template <int M, int D, int TB, bool QF32>
+__global__ void __launch_bounds__(PROJ_THREADS)
+    turbo_qproj_kernel(const void *__restrict__ Q, const float *__restrict__ Pinv,
+                       const uint16_t *__restrict__ S, float *__restrict__ U, int nq,
+                       const WalshCoef wc) {
+  griddep_launch_dependents();
+  turbo_query_rows<M, D, TB, QF32>(Q, Pinv, S, U, nq, wc, (int64_t)blockIdx.x * PROJ_VECS);
 }
 
 // ---------------------------------------------------------------------------
@@ -1364,6 +1372,127 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
   }
 }
 
+// TurboQuant-prod paged step: the query rows (as turbo_qproj_kernel), then the
+// appended keys, four per CTA.  Per key: y = Pi k / ||k|| (the coalesced
+// projection routine on the bf16 rotation), its cells by the odd-symmetric
+// rule of the tensor-core quantizer (y > 0 picks the side, |y| against the
+// positive boundaries the magnitude; a value on a boundary stays inward),
+// r = y - c[cell] and ||r||, rt = bf16(r), then S rt (the same routine) and
+// its signs.  Plane and sign words come from warp ballots over the
+// coordinates.  The products are accumulated in fp32 in another order than
+// the tensor-core quantizer's, so a coordinate within that rounding of a
+// boundary (or a sign within it of 0) may come out either way.
+struct TurboPrepParams {
+  PrepParams pp;                // pp.sign_pages holds the full codes
+  const uint16_t *Pi;           // d x d bf16
+  const float *Pinv;            // d x d fp32
+  WalshCoef wc;
+  float mag[4];                 // centroid magnitudes (positive half)
+  float pos_thr[3];             // positive boundaries between them
+};
+
+template <int M, int D, int TB, bool QF32, bool KF32>
+__global__ void __launch_bounds__(PROJ_THREADS) turbo_paged_prep_kernel(const TurboPrepParams tp) {
+  constexpr int WORDS = (TB * D + M) / 32;
+  __shared__ float ys[PROJ_VECS][D];
+  __shared__ float rs[PROJ_VECS][D];
+  __shared__ float zs[PROJ_VECS][M];
+  const PrepParams &pp = tp.pp;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int bid = blockIdx.x;
+  const int qctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS;
+  if (bid < qctas) {
+    turbo_query_rows<M, D, TB, QF32>(pp.Q, tp.Pinv, pp.S, pp.U, pp.nq, tp.wc,
+                                      (int64_t)bid * PROJ_VECS);
+    return;
+  }
+  const int nkv = pp.B * pp.Hkv;
+  const int x0 = (bid - qctas) * PROJ_VECS;
+  if (!pp.append || x0 >= nkv) return;  // uniform over the CTA
+  const int nx = min(PROJ_VECS, nkv - x0);
+  const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;  // warp j: key x0 + j
+  project4<D, D, KF32>(tp.Pi, pp.K_new, x0, nx, &ys[0][0]);
+  __syncthreads();
+  uint32_t planes[TB][D / 32];
+  float nk = 0.f, rn = 0.f;
+  if (j < nx) {
+    const int kvi = x0 + j;
+    float ss = 0.f;
+    for (int c = lane; c < D; c += 32) {
+      const float x = KF32 ? reinterpret_cast<const float *>(pp.K_new)[(int64_t)kvi * D + c]
+                           : bf16_bits_to_f32(
+                                 reinterpret_cast<const uint16_t *>(pp.K_new)[(int64_t)kvi * D + c]);
+      ss = fmaf(x, x, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    nk = sqrtf(ss);
+    const float inv = nk > 0.f ? 1.f / nk : 0.f;
+    float rsq = 0.f;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) {
+      const int i = 32 * w + lane;
+      const float y = ys[j][i] * inv;
+      const bool top = y > 0.f;
+      const float ay = fabsf(y);
+      int mu = 0;  // magnitude cell: number of positive boundaries below |y|
+      if constexpr (TB == 2) {
+        mu = ay > tp.pos_thr[0];
+      } else if constexpr (TB == 3) {
+        const int hi = ay > tp.pos_thr[1];
+        mu = 2 * hi + (ay > (hi ? tp.pos_thr[2] : tp.pos_thr[0]));
+      }
+      const float amag = tp.mag[mu];
+      const float r = top ? y - amag : y + amag;
+      rsq = fmaf(r, r, rsq);
+      rs[j][i] = bf16_round_f32(r);
+      planes[TB - 1][w] = __ballot_sync(0xffffffffu, top);
+#pragma unroll
+      for (int k = 0; k < TB - 1; ++k)
+        planes[k][w] = __ballot_sync(0xffffffffu, (((mu >> k) & 1) != 0) == top);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rsq += __shfl_xor_sync(0xffffffffu, rsq, o);
+    rn = sqrtf(rsq);
+  } else {
+    for (int c = lane; c < D; c += 32) rs[j][c] = 0.f;
+  }
+  __syncthreads();
+  project4<M, D, true>(pp.S, &rs[0][0], 0, nx, &zs[0][0]);
+  __syncthreads();
+  if (j >= nx) return;
+  const int kvi = x0 + j;
+  const int b = kvi / pp.Hkv, hkv = kvi - b * pp.Hkv;
+  const int64_t pos = pp.seq_lens[b];
+  const int64_t pidx = pos / pp.page_tokens;
+  const int page = (pos >= 0 && pidx < pp.max_pages)
+                       ? pp.block_table[(int64_t)b * pp.max_pages + pidx] : -1;
+  if (page < 0 || page >= pp.num_pages || pos + 1 > pp.max_len) {
+    if (lane == 0) record_device_error(pp.err, DERR_DECODE_PLAN);
+    return;
+  }
+  const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
+  uint32_t *code = pp.sign_pages + slot * WORDS;
+#pragma unroll
+  for (int w = 0; w < M / 32; ++w) {
+    const uint32_t word = __ballot_sync(0xffffffffu, zs[j][w * 32 + lane] >= 0.f);
+    if (lane == 0) code[TB * (D / 32) + w] = word;
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < TB; ++k)
+#pragma unroll
+      for (int w = 0; w < D / 32; ++w) code[k * (D / 32) + w] = planes[k][w];
+    reinterpret_cast<uint32_t *>(pp.norm_pages)[slot] =
+        (uint32_t)__half_as_ushort(__float2half_rn(nk)) |
+        ((uint32_t)__half_as_ushort(__float2half_rn(rn)) << 16);
+  }
+  const uint32_t *vsrc = reinterpret_cast<const uint32_t *>(pp.V_new + (int64_t)kvi * D);
+  uint32_t *vdst = reinterpret_cast<uint32_t *>(pp.value_pages + slot * D);
+  for (int c = lane; c < D / 2; c += 32) vdst[c] = vsrc[c];
+}
+
 // ---------------------------------------------------------------------------
 // planning and launch
 static bool supported(int m, int d) {
@@ -1651,7 +1780,9 @@ cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
 
 // Paged pools: values [num_pages*Hkv][P][d], codes [num_pages*Hkv][P*m/8 bytes],
 // norms [num_pages*Hkv][P]; every block is one box inside one page.
-static bool make_paged_maps(DecMaps *mp, const PagedArgs &a, int Hkv, int m, int d) {
+static bool make_paged_maps(DecMaps *mp, const PagedArgs &a, int Hkv, int m, int d,
+                            int code_bytes = 0, int norm_bytes = 2) {
+  if (code_bytes == 0) code_bytes = m / 8;
   auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
   if (!fn) return false;
   const cuuint32_t estr[3] = {1, 1, 1};
@@ -1665,12 +1796,12 @@ static bool make_paged_maps(DecMaps *mp, const PagedArgs &a, int Hkv, int m, int
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
-  mp->sign_elem = (m > 256) ? 8 : 4;
+  mp->sign_elem = (DEC_KB * code_bytes / 4 > 256) ? 8 : 4;
   {
     const int es = mp->sign_elem;
-    cuuint64_t dims[2] = {(cuuint64_t)(P * (m / 8) / es), rows};
-    cuuint64_t strides[1] = {(cuuint64_t)(P * (m / 8))};
-    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * (m / 8) / es), 1};
+    cuuint64_t dims[2] = {(cuuint64_t)(P * code_bytes / es), rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(P * code_bytes)};
+    cuuint32_t box[2] = {(cuuint32_t)(DEC_KB * code_bytes / es), 1};
     if (fn(&mp->sign, es == 8 ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
            2, a.sign_pages, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -1679,9 +1810,11 @@ static bool make_paged_maps(DecMaps *mp, const PagedArgs &a, int Hkv, int m, int
   }
   {
     cuuint64_t dims[2] = {P, rows};
-    cuuint64_t strides[1] = {P * 2};
+    cuuint64_t strides[1] = {P * norm_bytes};
     cuuint32_t box[2] = {(cuuint32_t)DEC_KB, 1};
-    if (fn(&mp->norm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.norm_pages, dims, strides, box, estr,
+    if (fn(&mp->norm,
+           norm_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+           a.norm_pages, dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
@@ -1728,6 +1861,64 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
   return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);
+}
+
+template <int TB>
+static cudaError_t launch_turbo_paged_t(const DecodePlan &pl, const PagedArgs &a,
+                                        const TurboPagedArgs &t, cudaStream_t stream) {
+  constexpr int M = 128, D = 128;
+  uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
+  float *U = reinterpret_cast<float *>(ws);
+  float *partials = reinterpret_cast<float *>(ws + pl.u_bytes);
+  DecMaps maps;
+  if (!make_paged_maps(&maps, a, pl.Hkv, M, D, DecCfg<M, D, TURBO_S8, TB>::KEY_SIGN_BYTES, 4))
+    return cudaErrorInvalidValue;
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
+  TurboPrepParams tp;
+  PrepParams &pp = tp.pp;
+  pp.Q = a.Q; pp.S = a.S; pp.U = U; pp.nq = pl.B * pl.Hq;
+  pp.K_new = a.K_new; pp.V_new = a.V_new;
+  pp.sign_pages = a.sign_pages; pp.norm_pages = a.norm_pages; pp.value_pages = a.value_pages;
+  pp.num_pages = a.num_pages; pp.page_tokens = a.page_tokens; pp.max_pages = a.max_pages;
+  pp.block_table = a.block_table; pp.seq_lens = a.seq_lens;
+  pp.B = pl.B; pp.Hkv = pl.Hkv;
+  pp.append = a.K_new != nullptr;
+  pp.max_len = pl.T;
+  pp.err = err;
+  tp.Pi = t.Pi;
+  tp.Pinv = t.Pinv;
+  for (int k = 0; k < 4; ++k) {
+    tp.wc.c[k] = (float)t.walsh[k];
+    tp.mag[k] = t.mag[k];
+  }
+  for (int k = 0; k < 3; ++k) tp.pos_thr[k] = t.pos_thr[k];
+  const int nkv = pl.B * pl.Hkv;
+  const int prep_ctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS +
+                        (pp.append ? (nkv + PROJ_VECS - 1) / PROJ_VECS : 0);
+  const dim3 pg(prep_ctas), pb(PROJ_THREADS);
+  cudaError_t e;
+  if (a.q_f32)
+    e = a.k_f32 ? launch_pdl(turbo_paged_prep_kernel<M, D, TB, true, true>, pg, pb, 0, stream, tp)
+                : launch_pdl(turbo_paged_prep_kernel<M, D, TB, true, false>, pg, pb, 0, stream, tp);
+  else
+    e = a.k_f32 ? launch_pdl(turbo_paged_prep_kernel<M, D, TB, false, true>, pg, pb, 0, stream, tp)
+                : launch_pdl(turbo_paged_prep_kernel<M, D, TB, false, false>, pg, pb, 0, stream, tp);
+  if (e != cudaSuccess) return e;
+  DecParams p;
+  fill_params(p, pl, U, partials, nullptr, nullptr, a.scores, a.softmax_scale, M, err);
+  p.seq_lens = a.seq_lens; p.block_table = a.block_table;
+  p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
+  p.score_stride = pl.T;
+  return launch_scorer_combine<M, D, TURBO_S8, true, TB>(pl, p, maps, a.out, stream);
+}
+
+cudaError_t launch_turbo_decode_paged(const DecodePlan &pl, int bits, const PagedArgs &a,
+                                      const TurboPagedArgs &t, cudaStream_t stream) {
+  if (bits == 1) return launch_turbo_paged_t<1>(pl, a, t, stream);
+  if (bits == 2) return launch_turbo_paged_t<2>(pl, a, t, stream);
+  if (bits == 3) return launch_turbo_paged_t<3>(pl, a, t, stream);
+  return cudaErrorNotSupported;
 }
 
 cudaError_t launch_decode_paged(const DecodePlan &pl, const PagedArgs &a,

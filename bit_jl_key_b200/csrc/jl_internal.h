@@ -119,4 +119,19 @@ struct PagedArgs {
 cudaError_t launch_decode_paged(const DecodePlan &p, const PagedArgs &a,
                                 cudaStream_t stream);
 
+// TurboQuant-prod paged step (decode.cu): PagedArgs with sign_pages holding
+// the full codes ((bits d + m)/32 words per key) and norm_pages the binary16
+// (||k||, ||r||) pairs, plus the rotation, its query map and the codebook.
+struct TurboPagedArgs {
+  const uint16_t *Pi;
+  const float *Pinv;
+  double walsh[4];
+  float mag[4];      // centroid magnitudes, positive half
+  float pos_thr[3];  // positive boundaries between them
+};
+cudaError_t launch_turbo_decode_paged(const DecodePlan &p, int bits, const PagedArgs &a,
+                                      const TurboPagedArgs &t, cudaStream_t stream);
+// The codebook's centroid magnitudes and positive boundaries (float).
+bool turbo_magnitudes(int d, int bits, float *mag, float *pos_thr);
+
 }  // namespace jlk

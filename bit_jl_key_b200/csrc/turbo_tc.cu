@@ -753,6 +753,15 @@ bool turbo_codebook(int d, int bits, float *centroids, double *walsh) {
   return true;
 }
 
+bool turbo_magnitudes(int d, int bits, float *mag, float *pos_thr) {
+  if (d < 3 || d > 4096 || bits < 1 || bits > 3) return false;
+  const turbo::Codebook *cb = turbo::codebook(d, bits);
+  const int H = cb->L / 2;
+  for (int i = 0; i < 4; ++i) mag[i] = i < H ? cb->cf[H + i] : 0.f;
+  for (int i = 0; i < 3; ++i) pos_thr[i] = i + 1 < H ? cb->thr[H + i] : 0.f;
+  return true;
+}
+
 size_t turbo_rotation_workspace_bytes(int d) { return turbo::rotation_workspace_bytes(d); }
 
 cudaError_t launch_turbo_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t seed, void *ws,

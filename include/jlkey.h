@@ -437,6 +437,39 @@ JL_API int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const floa
                                      void *workspace, size_t workspace_bytes,
                                      jl_stream_t stream);
 
+/* Device scratch of jl_turbo_decode_attention_paged (0 for unsupported shapes). */
+JL_API size_t jl_turbo_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len,
+                                                    int m, int d, int mse_bits);
+
+/*
+ * jl_turbo_decode_attention_paged -- jl_decode_attention_paged for
+ * TurboQuant-prod keys: one decode step of a batch of sequences whose
+ * compressed cache lives in a pool of fixed-size pages, optionally appending
+ * each sequence's new key first (quantized as by jl_turbo_quantize_keys,
+ * with fp32 SIMT products instead of the tensor cores: a coordinate within
+ * that rounding of a cell boundary, or a sign within it of 0, may come out
+ * either way).  Same page, table, length and error rules as
+ * jl_decode_attention_paged; the logit is the TurboQuant-prod score of
+ * jl_turbo_decode_attention.
+ *   Pi          : in, d x d bf16 rotation (required with K_new).
+ *   Pinv        : in, d x d fp32 query map.
+ *   S           : in, m x d bf16 residual sketch.
+ *   code_pages  : in/out, num_pages x Hkv x page_tokens x ((mse_bits d + m)/32)
+ *                 uint32 (the jl_turbo_quantize_keys code layout).
+ *   norm_pages  : in/out, num_pages x Hkv x page_tokens x 2 binary16.
+ *   value_pages : in/out, num_pages x Hkv x page_tokens x d bf16.
+ * Supported: d = m = 128, mse_bits 1 to 3.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
+ * JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_decode_attention_paged(
+    const void *Q, jl_dtype q_dtype, const void *K_new, jl_dtype k_dtype, const uint16_t *V_new,
+    const uint16_t *Pi, const float *Pinv, const uint16_t *S, uint32_t *code_pages,
+    uint16_t *norm_pages, uint16_t *value_pages, int num_pages, int page_tokens,
+    const int32_t *block_table, int max_pages, const int32_t *seq_lens, int B, int Hq, int Hkv,
+    int64_t max_len, int m, int d, int mse_bits, float softmax_scale, uint16_t *out,
+    float *scores, void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
 /*
  * jl_device_error -- synchronise `stream`, then read and clear the device
  * error word of the current device (0 = no fault reported).  *code receives
