@@ -1,7 +1,8 @@
 """Benchmark: QJL key quantization + compressed-key decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search|turbo-gqa]
+                    [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search|turbo-gqa|
+                turbo-paged-gqa]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -264,12 +265,15 @@ def _barrier(world, dev):
 
 
 def run_paged(args, rank, world, local_rank):
-    """Serving step over a paged cache: append + decode in one call."""
+    """Serving step over a paged cache: append + decode in one call (QJL keys,
+    or TurboQuant-prod keys for turbo-paged-gqa)."""
     import bit_jl_key_b200 as jl
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = pick_workload(args.workload, args.batch)
+    turbo = w.name.startswith("turbo")
+    bits = workloads.TURBO_MSE_BITS
     peak, peak_kind = load_peaks()
     P = workloads.PAGE_TOKENS
     lens, table, num_pages = workloads.paged_layout(w, P)
@@ -277,9 +281,18 @@ def run_paged(args, rank, world, local_rank):
     # fill the pool (untimed): keys and values of every slot, quantized in place
     pool = w.with_(B=num_pages, T=P)
     Kp = workloads.keys(pool, dev)
-    sign_pages = torch.empty((num_pages, w.Hkv, P, w.m // 32), dtype=torch.int32, device=dev)
-    norm_pages = torch.empty((num_pages, w.Hkv, P), dtype=torch.float16, device=dev)
-    jl.jl_quantize_keys(Kp.view(-1, w.d), S, sign_pages.view(-1, w.m // 32), norm_pages.view(-1))
+    if turbo:
+        Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED, device=dev)
+        words = jl.turbo_code_words(bits, w.m, w.d)
+        sign_pages = torch.empty((num_pages, w.Hkv, P, words), dtype=torch.int32, device=dev)
+        norm_pages = torch.empty((num_pages, w.Hkv, P, 2), dtype=torch.float16, device=dev)
+        jl.jl_turbo_quantize_keys(Kp.view(-1, w.d), Pi, S, bits, codes=sign_pages.view(-1, words),
+                                  norms=norm_pages.view(-1, 2))
+    else:
+        words = w.m // 32
+        sign_pages = torch.empty((num_pages, w.Hkv, P, words), dtype=torch.int32, device=dev)
+        norm_pages = torch.empty((num_pages, w.Hkv, P), dtype=torch.float16, device=dev)
+        jl.jl_quantize_keys(Kp.view(-1, w.d), S, sign_pages.view(-1, words), norm_pages.view(-1))
     del Kp
     value_pages = workloads.values(pool, dev)
     Q = workloads.queries(w, dev)
@@ -287,15 +300,22 @@ def run_paged(args, rank, world, local_rank):
     seq = lens.to(dev)
     tab = table.to(dev)
     out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty((jl.jl_decode_paged_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d),),
-                     dtype=torch.uint8, device=dev)
+    wsb = (jl.jl_turbo_decode_paged_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d, bits)
+           if turbo else jl.jl_decode_paged_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d))
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     attended = int((lens.long() + 1).sum()) * w.Hkv     # KV keys scored per step
 
     def step():
-        jl.jl_decode_attention_paged(Q, S, sign_pages, norm_pages, value_pages, tab, seq,
-                                     w.T, K_new=Kn, V_new=Vn, softmax_scale=w.softmax_scale,
-                                     out=out, workspace=ws)
+        if turbo:
+            jl.jl_turbo_decode_attention_paged(Q, Pinv, S, sign_pages, norm_pages, value_pages,
+                                               tab, seq, w.T, bits, Pi=Pi, K_new=Kn, V_new=Vn,
+                                               softmax_scale=w.softmax_scale, out=out,
+                                               workspace=ws)
+        else:
+            jl.jl_decode_attention_paged(Q, S, sign_pages, norm_pages, value_pages, tab, seq,
+                                         w.T, K_new=Kn, V_new=Vn, softmax_scale=w.softmax_scale,
+                                         out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -351,7 +371,7 @@ def run_paged(args, rank, world, local_rank):
         e2e = {"value": whole_job_rate(attended, world, e_ms), "unit": "keys/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    per_key = w.m // 8 + 2 + 2 * w.d
+    per_key = (words * 4 + 4 if turbo else w.m // 8 + 2) + 2 * w.d
     db = attended * per_key
     gbs = db / (d_ms * 1e-3) / 1e9
     traffic = ncu_traffic("decode:" + w.name)
@@ -360,7 +380,8 @@ def run_paged(args, rank, world, local_rank):
                          "algorithmic_bytes": db, "GB_per_s": gbs,
                          "frac_of_hbm_peak": gbs / peak,
                          "appended_keys": w.B * w.Hkv}}
-    roof = {"kernel": "jl_decode_attention_paged", "bound": "hbm", "achieved": gbs,
+    roof = {"kernel": "jl_turbo_decode_attention_paged" if turbo else "jl_decode_attention_paged",
+            "bound": "hbm", "achieved": gbs,
             "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
             "frac": gbs / peak, "algorithmic_bytes_per_launch": db,
             "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
@@ -371,7 +392,8 @@ def run_paged(args, rank, world, local_rank):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
         "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} max_len={w.T} "
-                               f"d={w.d} m={w.m} page={P} lens={lens.tolist()} + 1 appended",
+                               f"d={w.d} m={w.m} page={P} lens={lens.tolist()} + 1 appended"
+                               + (f", {bits}-bit cells + 1-bit residual QJL" if turbo else ""),
                    "global_batch": w.B * world, "seq_len": w.T,
                    "parallelism": f"dp{world}",
                    "l2": "cache exceeds L2 (126 MB); no flush"},
@@ -742,7 +764,7 @@ def run_ours(args, rank, world, local_rank):
         return run_turbo(args, rank, world, local_rank)
     if args.workload == "search":
         return run_search(args, rank, world, local_rank)
-    if args.workload == "paged-gqa":
+    if args.workload in ("paged-gqa", "turbo-paged-gqa"):
         return run_paged(args, rank, world, local_rank)
     if args.workload == "dequant-gqa":
         return run_dequant(args, rank, world, local_rank)
@@ -963,7 +985,7 @@ def oracle_sample(w: workloads.Workload):
         def run():
             oracle.dequantize(sig, n64, S64)
         return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
-    if w.name == "turbo-gqa":
+    if w.name in ("turbo-gqa", "turbo-paged-gqa"):
         from oracle import turbo as tq
         T = w.T
         sub = w.with_(B=1, Hkv=1, Hq=w.G, T=T)

@@ -327,3 +327,38 @@ def test_turbo_decode_argument_errors(lib):
     assert call(codes=MISALIGNED) == jl.JL_ERR_INVALID_ARG
     assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
     assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
+
+
+def test_turbo_paged_argument_errors(lib):
+    f = lib.jl_turbo_decode_attention_paged
+    need = jl.jl_turbo_decode_paged_workspace_bytes(2, 8, 2, 256, 128, 128, 2)
+    assert need > 0
+    assert jl.jl_turbo_decode_paged_workspace_bytes(2, 8, 2, 256, 128, 128, 4) == 0
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, K=FAKE, kt=jl.JL_BF16, V=FAKE, Pi=FAKE, Pinv=FAKE, S=FAKE,
+              cp=FAKE, np_=FAKE, vp=FAKE, npages=20, P=64, tab=FAKE, maxp=4, lens=FAKE, B=2, Hq=8,
+              Hkv=2, max_len=256, m=128, d=128, bits=2, scale=0.088, out=FAKE, sc=NULL, ws=FAKE,
+              wsb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["Q"], a["qt"], a["K"], a["kt"], a["V"], a["Pi"], a["Pinv"], a["S"], a["cp"],
+                 a["np_"], a["vp"], a["npages"], a["P"], a["tab"], a["maxp"], a["lens"], a["B"],
+                 a["Hq"], a["Hkv"], a["max_len"], a["m"], a["d"], a["bits"],
+                 ctypes.c_float(a["scale"]), a["out"], a["sc"], a["ws"], a["wsb"], NULL)
+
+    assert call(B=0) == jl.JL_OK
+    assert call(P=48) == jl.JL_ERR_INVALID_ARG            # not a multiple of 32
+    assert call(maxp=3) == jl.JL_ERR_INVALID_ARG          # pages cannot hold max_len
+    assert call(bits=4) == jl.JL_ERR_UNSUPPORTED
+    assert call(m=256) == jl.JL_ERR_UNSUPPORTED
+    assert call(Pi=NULL) == jl.JL_ERR_INVALID_ARG         # appending needs the rotation
+    assert call(V=NULL) == jl.JL_ERR_INVALID_ARG          # key without its value
+    assert call(kt=9) == jl.JL_ERR_INVALID_ARG
+    assert call(Hq=6, Hkv=4) == jl.JL_ERR_INVALID_ARG
+    # without a new key neither the rotation nor the key dtype is looked at
+    assert call(K=NULL, V=NULL, Pi=NULL, kt=9, ws=NULL) == jl.JL_ERR_WORKSPACE
+    for k in ("Q", "Pinv", "S", "cp", "np_", "vp", "tab", "lens", "out"):
+        assert call(**{k: NULL}) == jl.JL_ERR_INVALID_ARG, k
+    assert call(cp=MISALIGNED) == jl.JL_ERR_INVALID_ARG
+    assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
+    assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE

@@ -30,6 +30,7 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
   turbo-gqa  the gqa decode step with TurboQuant-prod keys: 2-bit cells of
            the rotated key (rotation seed 1) plus QJL on the residual with a
            128-row sketch (3 bits per coordinate plus two binary16 norms).
+  turbo-paged-gqa  the paged-gqa serving step with TurboQuant-prod keys.
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -109,10 +110,12 @@ SEARCH = Workload("search", 7, 1, 128, 1, 8388608, 128, 256, torch.bfloat16)
 TURBO_GQA = GQA.with_(name="turbo-gqa", m=128)
 TURBO_MSE_BITS = 2
 TURBO_ROTATION_SEED = 1
+# the paged serving step of paged-gqa with TurboQuant-prod keys (same data)
+TURBO_PAGED_GQA = PAGED_GQA.with_(name="turbo-paged-gqa", m=128)
 SEARCH_K = 10
 
 ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA,
-                           SEARCH, TURBO_GQA)}
+                           SEARCH, TURBO_GQA, TURBO_PAGED_GQA)}
 
 
 def sweep_points():
