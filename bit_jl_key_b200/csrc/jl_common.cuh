@@ -45,6 +45,15 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
 // Pack two floats into a bf16x2 register (lo -> bits 0..15), round to nearest.
+// a0 += lo(w)^2 and a1 += hi(w)^2 for the two bf16 halves of w: one fma
+// with bf16 multiplicands and an fp32 addend each (exactly fmaf of the
+// widened halves; the widening is folded into the instruction)
+__device__ __forceinline__ void bf16x2_sq_acc(uint32_t w, float &a0, float &a1) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n"
+      " fma.rn.f32.bf16 %0, l, l, %0;\n fma.rn.f32.bf16 %1, h, h, %1;\n}\n"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w));
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

@@ -391,12 +391,7 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
               rowp + kc * C::A_CHUNK + ((c ^ (r & 7)) << 4));
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(w4[e] << 16);
-            const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
-            ss0 = fmaf(lo, lo, ss0);
-            ss1 = fmaf(hi, hi, ss1);
-          }
+          for (int e = 0; e < 4; ++e) bf16x2_sq_acc(w4[e], ss0, ss1);
         }
       }
       __syncwarp();

@@ -368,10 +368,11 @@ struct QParams {
 // plane k < TB-1 is bit k of mu when y > 0 and its complement otherwise, i.e.
 // XNOR(bit k of mu, [y > 0]).
 //
-// Every bit is the sign bit of a float formed on the FMA pipe, gathered into
-// code words by funnel shifts: [y > 0] = sign(0 - y) (0 - y is +0 for y = +-0)
-// and bit k of mu = sign(p - |y|) for the boundary p of that search level, so
-// the plane bit is the complement of sign((0 - y) (p - |y|)).
+// Every bit is the sign bit of a float, gathered into code words by funnel
+// shifts: [y > 0] = sign(-y) with -y formed as D (-1/||k||) + 0, which turns
+// -0 into +0, and bit k of mu = sign(p - |y|) for the boundary p of that
+// search level.  The plane word is then the complement of the XOR of the two
+// sign words (one logic op per 32 coordinates).
 struct Magnitudes {
   float a[4];  // centroid magnitudes
   float p[3];  // positive boundaries
@@ -380,35 +381,44 @@ struct Magnitudes {
 template <int TB>
 struct PlaneChains {
   uint32_t top[4];          // [y > 0], four chains of 8 bits
-  uint32_t mag[TB - 1 > 0 ? TB - 1 : 1][4];  // complemented magnitude planes
+  uint32_t mag[TB - 1 > 0 ? TB - 1 : 1][4];  // [p < |y|] of each search level
 };
 
-// residual of one coordinate; pushes its bits into chain g
+// -y = d * ninv + 0 with one rounding (ninv = -1/||k||): the product rounded
+// as y = d / ||k|| is, negated, and a -0 product becomes +0
+__device__ __forceinline__ float neg_scaled(float d, float ninv) {
+  float r;
+  asm("fma.rn.f32 %0, %1, %2, 0f00000000;\n" : "=f"(r) : "f"(d), "f"(ninv));
+  return r;
+}
+
+// residual of the coordinate whose accumulator value is d; pushes its bits
+// into chain g
 template <int TB>
-__device__ __forceinline__ float cell_residual(float y, const Magnitudes &mg, PlaneChains<TB> &ch,
-                                               int g) {
-  const float neg = 0.f - y;
+__device__ __forceinline__ float cell_residual(float d, float ninv, const Magnitudes &mg,
+                                               PlaneChains<TB> &ch, int g) {
+  const float neg = neg_scaled(d, ninv);
   ch.top[g] = __funnelshift_l(__float_as_uint(neg), ch.top[g], 1);
-  const float ay = fabsf(y);
+  const float ay = fabsf(neg);
   float amag;
   if constexpr (TB == 1) {
     amag = mg.a[0];
   } else if constexpr (TB == 2) {
     const float d0 = mg.p[0] - ay;
-    ch.mag[0][g] = __funnelshift_l(__float_as_uint(neg * d0), ch.mag[0][g], 1);
+    ch.mag[0][g] = __funnelshift_l(__float_as_uint(d0), ch.mag[0][g], 1);
     amag = d0 < 0.f ? mg.a[1] : mg.a[0];
   } else {
     const float d1 = mg.p[1] - ay;
     const bool m1 = d1 < 0.f;
     const float d0 = (m1 ? mg.p[2] : mg.p[0]) - ay;
-    ch.mag[1][g] = __funnelshift_l(__float_as_uint(neg * d1), ch.mag[1][g], 1);
-    ch.mag[0][g] = __funnelshift_l(__float_as_uint(neg * d0), ch.mag[0][g], 1);
+    ch.mag[1][g] = __funnelshift_l(__float_as_uint(d1), ch.mag[1][g], 1);
+    ch.mag[0][g] = __funnelshift_l(__float_as_uint(d0), ch.mag[0][g], 1);
     const bool m0 = d0 < 0.f;
     amag = m1 ? (m0 ? mg.a[3] : mg.a[2]) : (m0 ? mg.a[1] : mg.a[0]);
   }
   // y - (+-a_mu): the centroid takes the sign of y, negative for y = +-0
   const float sgn = __uint_as_float((__float_as_uint(neg) & 0x80000000u) | 0x3F800000u);
-  return fmaf(sgn, amag, y);
+  return fmaf(sgn, amag, -neg);
 }
 
 template <int TB>
@@ -587,12 +597,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
             const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ (r & 7)) << 4));
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float lo = __uint_as_float(w4[e] << 16);
-              const float hi = __uint_as_float(w4[e] & 0xFFFF0000u);
-              ss0 = fmaf(lo, lo, ss0);
-              ss1 = fmaf(hi, hi, ss1);
-            }
+            for (int e = 0; e < 4; ++e) bf16x2_sq_acc(w4[e], ss0, ss1);
           }
         }
         __syncwarp();
@@ -603,7 +608,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           break;
         }
         const float nk = sqrtf(xk[r] + xk[BM + r]);
-        const float inv = nk > 0.f ? 1.f / nk : 0.f;
+        const float ninv = nk > 0.f ? -1.f / nk : -0.f;
         if (!tcx::wait_phase(d1full(a), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) {
           ok = false;
           break;
@@ -630,7 +635,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const int e = 8 * g + jj;
-              const float r = cell_residual<TB>(__uint_as_float(v[e]) * inv, mg, pc, g);
+              const float r = cell_residual<TB>(__uint_as_float(v[e]), ninv, mg, pc, g);
               if (g & 1)
                 rs1 = fmaf(r, r, rs1);
               else
@@ -642,11 +647,13 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           for (int e = 0; e < 32; e += 2)
             pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
           tcx::st16(acol + 16 * ch, pk);
-          planes[TB - 1][ch] = pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
+          const uint32_t top =
+              pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
+          planes[TB - 1][ch] = top;
 #pragma unroll
           for (int k = 0; k < TB - 1; ++k)
-            planes[k][ch] = ~(pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
-                              (pc.mag[k][3] << 24));
+            planes[k][ch] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
+                                     (pc.mag[k][3] << 24)));
         };
         tcx::ld32(dcol, va);
         tcx::ld32(dcol + 32, vb);
