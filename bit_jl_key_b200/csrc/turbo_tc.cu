@@ -23,19 +23,20 @@
 //
 // Quantizer (tensor cores), per tile of 128 keys:
 //   MMA 1   D = K Pi^T             (K: TMA-loaded bf16 tile; Pi resident)
-//   epilogue A  (one thread per key and column half): y = D / ||k||; cells by
+//   epilogue A  (one thread per key): y = D / ||k||; cells by
 //           a branch-free search of |y| over the positive boundaries (the cell
 //           bits are the code's planes); r = y - c[cell], ||r||, and
 //           rt = bf16(r) written to tensor memory as the A operand of
 //   MMA 2   D = rt S^T             (S resident; D reuses MMA 1's columns)
 //   epilogue B  sign words of D.
 // Warp roles: 0 TMA producer, 1 MMA issuer, 2-9 epilogue: warp w reads TMEM
-// lane quadrant w % 4 (32 keys) and column half (w - 2) / 4 (64 coordinates);
-// the two warps of a quadrant exchange their half sums of k^2 and rt^2
-// through shared memory.  Tensor memory: MMA 1 results double-buffered (so
-// MMA 1 runs a tile ahead), MMA 2 results single-buffered, residual rows
-// double-buffered.  The epilogue runs A of tile t, then B of tile t - 1, so
-// MMA 2 of one tile overlaps epilogue A of the next.  Every wait is bounded; a
+// lane quadrant w % 4 (32 keys, whole rows) of the tiles of parity
+// (w - 2) / 4, running A then B of each.  The two epilogue warps that share a
+// quadrant (and a scheduler) thus work on different tiles and need no
+// exchange; one hides the other's waits.  Tensor memory: MMA 1 results and
+// residual rows double-buffered by tile parity, MMA 2 results single-buffered
+// (MMA 2 of a tile waits for epilogue B of the previous one, which the other
+// warp runs right after its A).  Every wait is bounded; a
 // wait that runs out records DERR_TC_WAIT_TIMEOUT, tells the other roles to
 // stop, and the CTA drains its copies and frees its tensor memory.
 #include "jl_common.cuh"
@@ -331,14 +332,13 @@ struct QCfg {
   static constexpr int W_CHUNK = 128 * 128;     // 128 rows x 64 columns of Pi or S
   static constexpr int W_BYTES = 128 * QD * 2;  // 32 KB
   static constexpr int STAGES = 4;
-  static constexpr int EPI_WARPS = 8;           // two per TMEM lane quadrant (column halves)
+  static constexpr int EPI_WARPS = 8;           // two per TMEM lane quadrant (tile parities)
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int OFF_PI = 0;
   static constexpr int OFF_S = W_BYTES;
   static constexpr int OFF_A = 2 * W_BYTES;
-  static constexpr int OFF_X = OFF_A + STAGES * A_STAGE;   // half-row sums: [2][2][BM] float
-  static constexpr int OFF_BAR = OFF_X + 4 * BM * 4;
-  static constexpr int NBAR = 2 * STAGES + 2 + 2 + 1 + 1 + 1 + 4;
+  static constexpr int OFF_BAR = OFF_A + STAGES * A_STAGE;
+  static constexpr int NBAR = 2 * STAGES + 2 + 2 + 2 + 1 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
   static constexpr int WORDS = TB * QD / 32 + QM / 32;
   static constexpr int PW = QD / 32;            // words per plane
@@ -347,6 +347,7 @@ struct QCfg {
   static constexpr int D2_COL = 256;            // residual projections, one buffer
   static constexpr int A2_COL = 384;            // bf16 residual rows, two buffers of 64
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(STAGES % 2 == 0, "a stage holds tiles of one parity");
 };
 
 struct QParams {
@@ -432,19 +433,16 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *gbase = tq_smem_raw + (base - raw);
   const uint32_t sPi = base + C::OFF_PI, sS = base + C::OFF_S, sA = base + C::OFF_A;
-  float *xsum = reinterpret_cast<float *>(gbase + C::OFF_X);  // [k or r][half][row]
   const uint32_t bar0 = base + C::OFF_BAR;
   auto kfull = [&](int s) { return bar0 + 8u * s; };
   auto kempty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
   auto d1full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto afull = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
-  const uint32_t d2full = bar0 + 8u * (2 * C::STAGES + 4);
-  const uint32_t d2empty = bar0 + 8u * (2 * C::STAGES + 5);
-  const uint32_t wfull = bar0 + 8u * (2 * C::STAGES + 6);
-  // the two epilogue warps of lane quadrant q exchange half-row sums through
-  // shared memory; each exchange is one phase of pairbar(q) (one arrival per
-  // warp), waited on with the same bound as every other wait
-  auto pairbar = [&](int q) { return bar0 + 8u * (2 * C::STAGES + 7 + q); };
+  // MMA 2 of tile u commits to d2full(u & 1), waited on only by the warps of
+  // that parity (so each of them sees every phase of it)
+  auto d2full = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 4 + a); };
+  const uint32_t d2empty = bar0 + 8u * (2 * C::STAGES + 6);
+  const uint32_t wfull = bar0 + 8u * (2 * C::STAGES + 7);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
   volatile int *abort_flag =
       reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
@@ -453,16 +451,15 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(kfull(s), 1);
-      mbar_init(kempty(s), 1 + C::EPI_WARPS);  // MMA commit + epilogue warps (norms)
+      mbar_init(kempty(s), 1 + C::EPI_WARPS / 2);  // MMA commit + the parity's warps (norms)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(d1full(a), 1);
-      mbar_init(afull(a), C::EPI_WARPS);
+      mbar_init(afull(a), C::EPI_WARPS / 2);
+      mbar_init(d2full(a), 1);
     }
-    mbar_init(d2full, 1);
-    mbar_init(d2empty, C::EPI_WARPS);
+    mbar_init(d2empty, C::EPI_WARPS / 2);
     mbar_init(wfull, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(pairbar(q), 2);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -550,17 +547,18 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
             tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
                         kk > 0 ? 1u : 0u);
           }
-          tcx::commit(d2full);
+          tcx::commit(d2full(a));
           ++issued2;
         }
       }
       // the last products must be complete before tensor memory is freed
-      if (issued2 > 0) tcx::drain_wait(d2full, (uint32_t)((issued2 - 1) & 1));
+      if (issued2 > 0)
+        tcx::drain_wait(d2full((int)((issued2 - 1) & 1)), (uint32_t)(((issued2 - 1) >> 1) & 1));
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue: key row r = 32 (warp % 4) + lane, column
-    // half h (coordinates 64 h .. 64 h + 63) of each tile
+    // ---------------- epilogue: key row r = 32 (warp % 4) + lane of the
+    // tiles of parity h
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
     const int r = 32 * q + lane;
@@ -570,144 +568,125 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
     for (int i = 0; i < 4; ++i) mg.a[i] = p.mag[i];
 #pragma unroll
     for (int i = 0; i < 3; ++i) mg.p[i] = p.pos_thr[i];
-    float *xk = xsum;           // [2][BM] half sums of k^2
-    float *xr = xsum + 2 * BM;  // [2][BM] half sums of rt^2
-    uint32_t xchg = 0;          // exchanges done (phase index of pairbar(q))
-    auto exchange = [&]() -> bool {
+    for (int64_t it = h; it < cnt; it += 2) {
+      // ---- A: norm, cells, residual (tile it uses stage s, buffers h)
+      const int s = (int)(it % C::STAGES);
+      const int64_t row = (blockIdx.x + it * gridDim.x) * BM + r;
+      if (!tcx::wait_phase(kfull(s), (uint32_t)((it / C::STAGES) & 1), abort_flag, p.err))
+        break;
+      float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < C::KCH; ++kc) {
+        const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + kc * C::A_CHUNK + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ (r & 7)) << 4));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bf16x2_sq_acc(w4[e], ss0, ss1);
+        }
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(pairbar(q));
-      return tcx::wait_phase(pairbar(q), (xchg++) & 1u, abort_flag, p.err);
-    };
-    bool ok = true;
-    for (int64_t it = 0; ok && it <= cnt; ++it) {
-      if (it < cnt) {
-        // ---- A: norm, cells, residual of tile it
-        const int s = (int)(it % C::STAGES);
-        const int a = (int)(it & 1);
-        const int64_t row = (blockIdx.x + it * gridDim.x) * BM + r;
-        if (!tcx::wait_phase(kfull(s), (uint32_t)((it / C::STAGES) & 1), abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        float ss0 = 0.f, ss1 = 0.f;
-        {
-          const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + h * C::A_CHUNK + r * 128;
+      if (lane == 0) mbar_arrive(kempty(s));
+      const float nk = sqrtf(ss0 + ss1);
+      const float ninv = nk > 0.f ? -1.f / nk : -0.f;
+      if (!tcx::wait_phase(d1full(h), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) break;
+      __syncwarp();
+      tcx::fence_after();
+      uint32_t planes[TB][4];
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t va[32], vb[32];
+      const uint32_t dcol = tq + (uint32_t)(C::D1_COL + h * 128);
+      const uint32_t acol = tq + (uint32_t)(C::A2_COL + h * 64);
+      auto chunk = [&](uint32_t (&v)[32], int ch) {
+        PlaneChains<TB> pc;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ (r & 7)) << 4));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        for (int g = 0; g < 4; ++g) {
+          pc.top[g] = 0u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) bf16x2_sq_acc(w4[e], ss0, ss1);
-          }
+          for (int k = 0; k < (TB > 1 ? TB - 1 : 1); ++k) pc.mag[k][g] = 0u;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(kempty(s));
-        xk[h * BM + r] = ss0 + ss1;
-        if (!exchange()) {
-          ok = false;
-          break;
-        }
-        const float nk = sqrtf(xk[r] + xk[BM + r]);
-        const float ninv = nk > 0.f ? -1.f / nk : -0.f;
-        if (!tcx::wait_phase(d1full(a), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        __syncwarp();
-        tcx::fence_after();
-        uint32_t planes[TB][2];
-        float rs0 = 0.f, rs1 = 0.f;
-        uint32_t va[32], vb[32];
-        const uint32_t dcol = tq + (uint32_t)(C::D1_COL + a * 128 + 64 * h);
-        const uint32_t acol = tq + (uint32_t)(C::A2_COL + a * 64 + 32 * h);
-        auto chunk = [&](uint32_t (&v)[32], int ch) {
-          PlaneChains<TB> pc;
+        // coordinate 8 g + jj, highest first so that the funnel shifts
+        // leave bit jj of chain g at position jj
+#pragma unroll
+        for (int jj = 7; jj >= 0; --jj)
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            pc.top[g] = 0u;
-#pragma unroll
-            for (int k = 0; k < (TB > 1 ? TB - 1 : 1); ++k) pc.mag[k][g] = 0u;
+            const int e = 8 * g + jj;
+            const float rr = cell_residual<TB>(__uint_as_float(v[e]), ninv, mg, pc, g);
+            if (g & 1)
+              rs1 = fmaf(rr, rr, rs1);
+            else
+              rs0 = fmaf(rr, rr, rs0);
+            v[e] = __float_as_uint(rr);
           }
-          // coordinate 8 g + jj, highest first so that the funnel shifts
-          // leave bit jj of chain g at position jj
+        uint32_t pk[16];
 #pragma unroll
-          for (int jj = 7; jj >= 0; --jj)
+        for (int e = 0; e < 32; e += 2)
+          pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        tcx::st16(acol + 16 * ch, pk);
+        const uint32_t top =
+            pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
+        planes[TB - 1][ch] = top;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int e = 8 * g + jj;
-              const float r = cell_residual<TB>(__uint_as_float(v[e]), ninv, mg, pc, g);
-              if (g & 1)
-                rs1 = fmaf(r, r, rs1);
-              else
-                rs0 = fmaf(r, r, rs0);
-              v[e] = __float_as_uint(r);
-            }
-          uint32_t pk[16];
+        for (int k = 0; k < TB - 1; ++k)
+          planes[k][ch] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
+                                   (pc.mag[k][3] << 24)));
+      };
+      // four chunks of 32 columns through two register sets: the load of the
+      // next chunk is in flight while one is processed
+      tcx::ld32(dcol, va);
+      tcx::ld32(dcol + 32, vb);
+      tcx::ld_wait(va);
+      chunk(va, 0);
+      tcx::ld32(dcol + 64, va);
+      tcx::ld_wait(vb);
+      chunk(vb, 1);
+      tcx::ld32(dcol + 96, vb);
+      tcx::ld_wait(va);
+      chunk(va, 2);
+      tcx::ld_wait(vb);
+      chunk(vb, 3);
+      tcx::st_wait();
+      tcx::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(afull(h));
+      if (row < p.n) {
+        uint32_t *dst = p.codes + row * C::WORDS;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-          tcx::st16(acol + 16 * ch, pk);
-          const uint32_t top =
-              pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
-          planes[TB - 1][ch] = top;
-#pragma unroll
-          for (int k = 0; k < TB - 1; ++k)
-            planes[k][ch] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
-                                     (pc.mag[k][3] << 24)));
-        };
-        tcx::ld32(dcol, va);
-        tcx::ld32(dcol + 32, vb);
-        tcx::ld_wait(va);
-        chunk(va, 0);
-        tcx::ld_wait(vb);
-        chunk(vb, 1);
-        tcx::st_wait();
-        tcx::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(afull(a));
-        xr[h * BM + r] = rs0 + rs1;
-        if (!exchange()) {
-          ok = false;
-          break;
-        }
-        if (row < p.n) {
-          uint32_t *dst = p.codes + row * C::WORDS + 2 * h;
-#pragma unroll
-          for (int pp = 0; pp < TB; ++pp)
-            *reinterpret_cast<uint2 *>(dst + pp * C::PW) = make_uint2(planes[pp][0], planes[pp][1]);
-          if (h == 0) {
-            const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
-            const uint32_t r16 =
-                __half_as_ushort(__float2half_rn(sqrtf(xr[r] + xr[BM + r])));
-            p.norms[row] = n16 | (r16 << 16);
-          }
-        }
+        for (int pp = 0; pp < TB; ++pp)
+          *reinterpret_cast<uint4 *>(dst + pp * C::PW) =
+              make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
+        const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
+        const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
+        p.norms[row] = n16 | (r16 << 16);
       }
-      if (it >= 1) {
-        // ---- B: residual sign words of tile it - 1 (this warp's half)
-        const int64_t u = it - 1;
-        const int64_t row = (blockIdx.x + u * gridDim.x) * BM + r;
-        if (!tcx::wait_phase(d2full, (uint32_t)(u & 1), abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        __syncwarp();
-        tcx::fence_after();
-        uint32_t va[32], vb[32];
-        const uint32_t dcol = tq + (uint32_t)(C::D2_COL + 64 * h);
-        tcx::ld32(dcol, va);
-        tcx::ld32(dcol + 32, vb);
+      // ---- B: residual sign words of tile it
+      if (!tcx::wait_phase(d2full(h), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) break;
+      __syncwarp();
+      tcx::fence_after();
+      uint32_t w[4];
+      {
+        const uint32_t d2 = tq + (uint32_t)C::D2_COL;
+        tcx::ld32(d2, va);
+        tcx::ld32(d2 + 32, vb);
         tcx::ld_wait(va);
-        const uint32_t w0 = tcx::sign_word(va);
+        w[0] = tcx::sign_word(va);
+        tcx::ld32(d2 + 64, va);
         tcx::ld_wait(vb);
-        const uint32_t w1 = tcx::sign_word(vb);
-        tcx::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(d2empty);
-        if (row < p.n)
-          *reinterpret_cast<uint2 *>(p.codes + row * C::WORDS + TB * C::PW + 2 * h) =
-              make_uint2(w0, w1);
+        w[1] = tcx::sign_word(vb);
+        tcx::ld32(d2 + 96, vb);
+        tcx::ld_wait(va);
+        w[2] = tcx::sign_word(va);
+        tcx::ld_wait(vb);
+        w[3] = tcx::sign_word(vb);
       }
+      tcx::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(d2empty);
+      if (row < p.n)
+        *reinterpret_cast<uint4 *>(p.codes + row * C::WORDS + TB * C::PW) =
+            make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 
