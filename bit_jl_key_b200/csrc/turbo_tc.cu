@@ -593,7 +593,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       if (!tcx::wait_phase(d1full(h), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) break;
       __syncwarp();
       tcx::fence_after();
-      uint32_t planes[TB][4];
+      uint32_t planes[TB][2];
       float rs0 = 0.f, rs1 = 0.f;
       uint32_t va[32], vb[32];
       const uint32_t dcol = tq + (uint32_t)(C::D1_COL + h * 128);
@@ -627,36 +627,35 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         tcx::st16(acol + 16 * ch, pk);
         const uint32_t top =
             pc.top[0] | (pc.top[1] << 8) | (pc.top[2] << 16) | (pc.top[3] << 24);
-        planes[TB - 1][ch] = top;
+        planes[TB - 1][ch & 1] = top;
 #pragma unroll
         for (int k = 0; k < TB - 1; ++k)
-          planes[k][ch] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) | (pc.mag[k][2] << 16) |
-                                   (pc.mag[k][3] << 24)));
+          planes[k][ch & 1] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) |
+                                       (pc.mag[k][2] << 16) | (pc.mag[k][3] << 24)));
       };
-      // four chunks of 32 columns through two register sets: the load of the
-      // next chunk is in flight while one is processed
-      tcx::ld32(dcol, va);
-      tcx::ld32(dcol + 32, vb);
-      tcx::ld_wait(va);
-      chunk(va, 0);
-      tcx::ld32(dcol + 64, va);
-      tcx::ld_wait(vb);
-      chunk(vb, 1);
-      tcx::ld32(dcol + 96, vb);
-      tcx::ld_wait(va);
-      chunk(va, 2);
-      tcx::ld_wait(vb);
-      chunk(vb, 3);
+      // four chunks of 32 columns, two per pass (a rolled loop keeps the
+      // code small); the second chunk's load is in flight during the first
+      uint32_t *dst = p.codes + row * C::WORDS;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        tcx::ld32(dcol + 64 * half, va);
+        tcx::ld32(dcol + 64 * half + 32, vb);
+        tcx::ld_wait(va);
+        chunk(va, 2 * half);
+        tcx::ld_wait(vb);
+        chunk(vb, 2 * half + 1);
+        if (row < p.n) {
+#pragma unroll
+          for (int pp = 0; pp < TB; ++pp)
+            *reinterpret_cast<uint2 *>(dst + pp * C::PW + 2 * half) =
+                make_uint2(planes[pp][0], planes[pp][1]);
+        }
+      }
       tcx::st_wait();
       tcx::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(afull(h));
       if (row < p.n) {
-        uint32_t *dst = p.codes + row * C::WORDS;
-#pragma unroll
-        for (int pp = 0; pp < TB; ++pp)
-          *reinterpret_cast<uint4 *>(dst + pp * C::PW) =
-              make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
         const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
         const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
         p.norms[row] = n16 | (r16 << 16);
@@ -665,28 +664,21 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       if (!tcx::wait_phase(d2full(h), (uint32_t)((it >> 1) & 1), abort_flag, p.err)) break;
       __syncwarp();
       tcx::fence_after();
-      uint32_t w[4];
-      {
-        const uint32_t d2 = tq + (uint32_t)C::D2_COL;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t d2 = tq + (uint32_t)(C::D2_COL + 64 * half);
         tcx::ld32(d2, va);
         tcx::ld32(d2 + 32, vb);
         tcx::ld_wait(va);
-        w[0] = tcx::sign_word(va);
-        tcx::ld32(d2 + 64, va);
+        const uint32_t w0 = tcx::sign_word(va);
         tcx::ld_wait(vb);
-        w[1] = tcx::sign_word(vb);
-        tcx::ld32(d2 + 96, vb);
-        tcx::ld_wait(va);
-        w[2] = tcx::sign_word(va);
-        tcx::ld_wait(vb);
-        w[3] = tcx::sign_word(vb);
+        const uint32_t w1 = tcx::sign_word(vb);
+        if (row < p.n)
+          *reinterpret_cast<uint2 *>(dst + TB * C::PW + 2 * half) = make_uint2(w0, w1);
       }
       tcx::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(d2empty);
-      if (row < p.n)
-        *reinterpret_cast<uint4 *>(p.codes + row * C::WORDS + TB * C::PW) =
-            make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 
