@@ -599,17 +599,37 @@ __device__ __forceinline__ bool better(float a, int32_t ia, float b, int32_t ib)
   return a > b || (a == b && (unsigned)ia < (unsigned)ib);
 }
 
+// The best (value, index, position) of a warp: each lane offers its own best
+// (position < 0 = none), the winner is broadcast to all lanes.
+__device__ __forceinline__ void warp_best(float &bv, int32_t &bi, int &bp) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    const int op = __shfl_xor_sync(0xffffffffu, bp, o);
+    if (op >= 0 && (bp < 0 || better(ov, oi, bv, bi))) {
+      bv = ov;
+      bi = oi;
+      bp = op;
+    }
+  }
+}
+
+// Two levels: each warp takes the k best of its slice of the candidates
+// (lane l owns slice entries l, l + 32, ...; the winning lane strikes its own
+// entry, so a round needs no block barrier), then warp 0 takes the k best of
+// the warps' lists.
 __global__ void __launch_bounds__(MERGE_THREADS) search_merge_kernel(
     const float *__restrict__ part_val, const int32_t *__restrict__ part_idx, int ctas, int kt,
     int k, const float *__restrict__ qscale, int32_t *__restrict__ out_idx,
     float *__restrict__ out_scores, unsigned *__restrict__ bound_out) {
+  constexpr int NW = MERGE_THREADS / 32;
   extern __shared__ uint8_t mg_smem[];
   const int ncand = ctas * LISTS * kt;
   float *cv = reinterpret_cast<float *>(mg_smem);
   int32_t *ci = reinterpret_cast<int32_t *>(cv + ncand);
-  __shared__ float wv[MERGE_THREADS / 32];
-  __shared__ int32_t wi[MERGE_THREADS / 32];
-  __shared__ int wpos[MERGE_THREADS / 32];
+  __shared__ float wv[NW * 16];
+  __shared__ int32_t wi[NW * 16];
   const int qi = blockIdx.x;
   for (int e = threadIdx.x; e < ncand; e += MERGE_THREADS) {
     const int list = e / kt, j = e - list * kt;  // list = cta * LISTS + half
@@ -619,52 +639,52 @@ __global__ void __launch_bounds__(MERGE_THREADS) search_merge_kernel(
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int per = (ncand + NW - 1) / NW;
+  const int e0 = w * per, e1 = min(ncand, e0 + per);
   for (int r = 0; r < k; ++r) {
     float bv = -INFINITY;
     int32_t bi = -1;
     int bp = -1;
-    for (int e = threadIdx.x; e < ncand; e += MERGE_THREADS)
+    for (int e = e0 + lane; e < e1; e += 32)
       if (ci[e] >= 0 && (bp < 0 || better(cv[e], ci[e], bv, bi))) {
         bv = cv[e];
         bi = ci[e];
         bp = e;
       }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      const int op = __shfl_xor_sync(0xffffffffu, bp, o);
-      if (op >= 0 && (bp < 0 || better(ov, oi, bv, bi))) {
-        bv = ov;
-        bi = oi;
-        bp = op;
-      }
-    }
+    const int mine = bp;
+    warp_best(bv, bi, bp);
+    if (bp >= 0 && bp == mine) ci[bp] = -1;  // the owner strikes the winner
     if (lane == 0) {
-      wv[w] = bv;
-      wi[w] = bi;
-      wpos[w] = bp;
+      wv[w * 16 + r] = bv;
+      wi[w * 16 + r] = bp >= 0 ? bi : -1;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float fv = -INFINITY;
-      int32_t fi = -1;
-      int fp = -1;
-      for (int x = 0; x < MERGE_THREADS / 32; ++x)
-        if (wpos[x] >= 0 && (fp < 0 || better(wv[x], wi[x], fv, fi))) {
-          fv = wv[x];
-          fi = wi[x];
-          fp = wpos[x];
-        }
-      if (bound_out) {
-        if (r == k - 1) bound_out[qi] = fp >= 0 ? ord_code(fv) : 0u;
-      } else {
-        out_idx[(int64_t)qi * k + r] = fi;
-        out_scores[(int64_t)qi * k + r] = fp >= 0 ? fv * qscale[qi] : -INFINITY;
+    __syncwarp();
+  }
+  __syncthreads();
+  if (w != 0) return;
+  // warp 0: NW lists of k, lane l owns entries l, l + 32, ... of the NW x 16 grid
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int32_t bi = -1;
+    int bp = -1;
+    for (int e = lane; e < NW * 16; e += 32)
+      if ((e & 15) < k && wi[e] >= 0 && (bp < 0 || better(wv[e], wi[e], bv, bi))) {
+        bv = wv[e];
+        bi = wi[e];
+        bp = e;
       }
-      if (fp >= 0) ci[fp] = -1;  // taken
+    const int mine = bp;
+    warp_best(bv, bi, bp);
+    if (bp >= 0 && bp == mine) wi[bp] = -1;
+    if (lane == 0) {
+      if (bound_out) {
+        if (r == k - 1) bound_out[qi] = bp >= 0 ? ord_code(bv) : 0u;
+      } else {
+        out_idx[(int64_t)qi * k + r] = bp >= 0 ? bi : -1;
+        out_scores[(int64_t)qi * k + r] = bp >= 0 ? bv * qscale[qi] : -INFINITY;
+      }
     }
-    __syncthreads();
+    __syncwarp();
   }
 }
 
