@@ -14,14 +14,20 @@
 // (M = 128, N = 256, K = m) on the tensor cores:
 //   * U = S q (projected by the query-projection kernel) is rounded to fp16
 //     with a power-of-two scale per query (relative error <= 2^-11 per
-//     coordinate) and written once into tensor memory as the A operand;
+//     coordinate) and written once as the A operand: into shared memory
+//     (128-byte swizzle, K-major) for m <= 256, so that tensor memory holds
+//     two accumulators and the MMAs of one tile overlap the epilogue of the
+//     previous one; into tensor memory beside a single accumulator for
+//     m = 512;
 //   * the B operand is Z scaled by each vector's norm, +-||x|| in fp16 (the
 //     norms are stored in binary16, and a product with the fp16 U is exact
 //     in fp32), expanded from the code bits into shared memory one K-chunk of
 //     64 coordinates (32 KB) at a time: an fp16 pair holds coordinates
 //     (p, p + 16) of a code word, ((w << (15 - p)) & 0x80008000) ^
 //     (0x80008000 | ||x|| ||x||), and U's columns use the same order;
-//   * the accumulator (256 fp32 columns) sits in tensor memory beside U.
+//   * each accumulator takes 256 fp32 columns of tensor memory.  (An MMA of
+//     N = 128 runs at about two thirds of the rate per flop of N = 256 here,
+//     so the tile stays 256 wide.)
 // Each epilogue lane owns one query and keeps its best KT scores (before the
 // query's positive output scale) in registers.  Per 32 columns the hot path
 // is the group maximum and one comparison with the list's bound: the larger
@@ -57,7 +63,7 @@ constexpr int CHUNK_K = 64;                    // coordinates per Z chunk
 constexpr int CHUNK_BYTES = BN * CHUNK_K * 2;  // 32 KB
 constexpr int EXP_WARPS = 4, EPI_WARPS = 4;
 constexpr int LISTS = 1;                       // lists per query and CTA
-constexpr int PARK_ROWS = 4;                   // groups a lane can park per tile
+constexpr int PARK_ROWS = 2;                   // groups a lane can park at once
 constexpr int MMA_WARP = EXP_WARPS + EPI_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int CODE_SLOTS = 3;
@@ -69,19 +75,23 @@ constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
 template <int M>
 struct Cfg {
   static constexpr int KCH = M / CHUNK_K;
-  static constexpr int U_COLS = M / 2;         // fp16 pairs
-  static constexpr int D_COL = U_COLS;         // accumulator columns [D_COL, D_COL + 256)
-  static constexpr int RING = M > 256 ? 3 : 4;
+  static constexpr bool U_SMEM = M <= 256;     // A operand in shared memory
+  static constexpr int U_COLS = U_SMEM ? 0 : M / 2;  // tensor-memory columns of U (fp16 pairs)
+  static constexpr int NACC = U_SMEM ? 2 : 1;  // accumulators of BN columns
+  static constexpr int D_COL = U_COLS;         // accumulator b: columns D_COL + BN b ...
+  static constexpr int RING = 3;
   static constexpr int CODE_ROW = M / 8;
   static constexpr int CODE_WORDS = M / 32;
-  static constexpr int OFF_Z = 0;
+  static constexpr int U_CHUNK = QM * 128;     // one 64-coordinate K-chunk of U
+  static constexpr int OFF_U = 0;
+  static constexpr int OFF_Z = OFF_U + (U_SMEM ? KCH * U_CHUNK : 0);
   static constexpr int OFF_C = OFF_Z + RING * CHUNK_BYTES;
   // per epilogue lane: PARK_ROWS rows of 33 floats (parked groups)
   static constexpr int OFF_P = OFF_C + CODE_SLOTS * BN * CODE_ROW;
   static constexpr int OFF_BAR = OFF_P + EPI_WARPS * 32 * PARK_ROWS * 33 * 4;
-  static constexpr int NBAR = 2 * RING + 2;
+  static constexpr int NBAR = 2 * RING + 2 * NACC;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static_assert(D_COL + BN <= TMEM_COLS, "tensor memory columns");
+  static_assert(D_COL + NACC * BN <= TMEM_COLS, "tensor memory columns");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -129,6 +139,16 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uin
       " setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D (tensor memory) += A (shared memory) * B (shared memory), fp16 inputs
+__device__ __forceinline__ void mma_f16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -237,6 +257,13 @@ __device__ __forceinline__ void expand_row(uint8_t *chunk, int r, uint32_t w0, u
   }
 }
 
+// max(a, b, c) in one instruction (three-input max.f32)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Order-preserving code of a float (larger float <-> larger code; never 0 for
 // a number), and back.
 __device__ __forceinline__ unsigned ord_code(float f) {
@@ -307,8 +334,8 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
   const uint32_t bar0 = base + C::OFF_BAR;
   auto zfull_bar = [&](int s) { return bar0 + 8u * s; };
   auto zempty_bar = [&](int s) { return bar0 + 8u * (C::RING + s); };
-  const uint32_t dfull_bar = bar0 + 8u * (2 * C::RING);
-  const uint32_t dempty_bar = bar0 + 8u * (2 * C::RING + 1);
+  auto dfull_bar = [&](int b) { return bar0 + 8u * (2 * C::RING + b); };
+  auto dempty_bar = [&](int b) { return bar0 + 8u * (2 * C::RING + C::NACC + b); };
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
   volatile int *abort_flag =
       reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
@@ -321,8 +348,10 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       mbar_init(zfull_bar(s), EXP_WARPS);
       mbar_init(zempty_bar(s), 1);
     }
-    mbar_init(dfull_bar, 1);
-    mbar_init(dempty_bar, EPI_WARPS);
+    for (int b = 0; b < C::NACC; ++b) {
+      mbar_init(dfull_bar(b), 1);
+      mbar_init(dempty_bar(b), EPI_WARPS);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -339,8 +368,10 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  // ---- U into tensor memory (warps 4-7, lane quadrant warp % 4): fp16 pairs
-  // (u_{32b+j}, u_{32b+j+16}) at column 16 b + j, scaled by 2^e per query
+  // ---- U (warps 4-7, query qi = 32 (warp % 4) + lane): fp16 pairs
+  // (u_{32b+j}, u_{32b+j+16}) as K positions 2 c, 2 c + 1 with c = 16 b + j,
+  // scaled by 2^e per query; into shared memory (word c of row qi in the
+  // swizzled K-chunk c / 32) or tensor memory (column c of lane qi)
   if (warp >= EXP_WARPS && warp < MMA_WARP) {
     const int q = warp & 3;
     const int qi = 32 * q + lane;
@@ -355,7 +386,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
     // output scale of the query's scores: sqrt(pi/2)/m * 2^-e
     if (blockIdx.x == 0) p.qscale[qi] = p.coef * ldexpf(1.f, ex - 15);
 #pragma unroll 1
-    for (int c0 = 0; c0 < C::U_COLS; c0 += 32) {
+    for (int c0 = 0; c0 < M / 2; c0 += 32) {
       uint32_t v[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
@@ -365,9 +396,19 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         __half2 h = __floats2half2_rn(lo, hi);
         v[e] = *reinterpret_cast<uint32_t *>(&h);
       }
-      tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+      if constexpr (C::U_SMEM) {
+        // 32 words = one 128-byte row of K-chunk c0 / 32: eight 16-byte units
+        uint8_t *rowp = gbase + C::OFF_U + (c0 / 32) * C::U_CHUNK + qi * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4 *>(rowp + ((u ^ (qi & 7)) << 4)) =
+              make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+      } else {
+        tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+      }
     }
-    tmem_st_wait();
+    if constexpr (C::U_SMEM) fence_async_smem();
+    else tmem_st_wait();
   }
   tc_fence_before();
   __syncthreads();
@@ -467,25 +508,30 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       const int nvalid = (int)((p.N - base_row) < BN ? (p.N - base_row) : BN);
       // the query's shared bound: scores below it cannot make the top KT
       const float gb = ord_float(*reinterpret_cast<volatile unsigned *>(p.gbound + qi));
-      if (!wait_phase(dfull_bar, (uint32_t)(tt & 1), abort_flag, p.err)) break;
+      const int ab = (int)(tt % C::NACC);
+      if (!wait_phase(dfull_bar(ab), (uint32_t)((tt / C::NACC) & 1), abort_flag, p.err)) break;
       __syncwarp();
       tc_fence_after();
-      const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)C::D_COL;
+      const uint32_t trow =
+          tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(C::D_COL + ab * BN);
       // the tile's 8 groups of 32 columns: while the accumulator is held only
       // the group maxima are taken; groups that may qualify are parked and
       // inserted once the accumulator is released (or when the rows are full)
       int np = 0;          // parked groups
       uint32_t pgs = 0;    // their group numbers, 4 bits each
-      // one group: its maximum (a tree, depth 5), parked if it may qualify
+      // one group: its maximum (a tree of three-input maxima, 17 steps),
+      // parked if it may qualify
       auto scan_group = [&](uint32_t (&v)[32], int g) {
-        float m16[16];
+        float t[11];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) m16[e] = fmaxf(__uint_as_float(v[e]), __uint_as_float(v[e + 16]));
-#pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) m16[e] = fmaxf(m16[e], m16[e + w]);
-        if (m16[0] > list.thr && m16[0] >= gb) {
+        for (int e = 0; e < 10; ++e)
+          t[e] = max3f(__uint_as_float(v[3 * e]), __uint_as_float(v[3 * e + 1]),
+                       __uint_as_float(v[3 * e + 2]));
+        t[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+        const float gm = fmaxf(max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]),
+                                     max3f(t[6], t[7], t[8])),
+                               fmaxf(t[9], t[10]));
+        if (gm > list.thr && gm >= gb) {
           float *row = park + np * 33;
 #pragma unroll
           for (int e = 0; e < 32; ++e) row[e] = __uint_as_float(v[e]);
@@ -517,7 +563,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         } else {  // the accumulator is read: free it
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(dempty_bar);
+          if (lane == 0) mbar_arrive(dempty_bar(ab));
         }
         scan_group(vb, g + 1);
         // at most two groups park per pair: flush before the rows run out,
@@ -549,7 +595,10 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       int64_t c = 0, tt = 0;
       bool ok = true;
       for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++tt) {
-        if (!wait_phase(dempty_bar, (uint32_t)((tt & 1) ^ 1), abort_flag, p.err)) break;
+        // accumulator ab was read by the epilogue of tile tt - NACC
+        const int ab = (int)(tt % C::NACC);
+        if (!wait_phase(dempty_bar(ab), (uint32_t)(((tt / C::NACC) & 1) ^ 1), abort_flag, p.err))
+          break;
         tc_fence_after();
         for (int kc = 0; kc < C::KCH; ++kc, ++c) {
           const int s = (int)(c % C::RING);
@@ -561,18 +610,24 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < CHUNK_K / 16; ++kk) {
-            const uint32_t atm = tmem_base + (uint32_t)(kc * 32 + kk * 8);
             const uint64_t bdesc = smem_desc_sw128(sZ + s * CHUNK_BYTES + kk * 32);
-            mma_f16_ts(tmem_base + C::D_COL, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t dt = tmem_base + (uint32_t)(C::D_COL + ab * BN);
+            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (C::U_SMEM)
+              mma_f16_ss(dt, smem_desc_sw128(base + C::OFF_U + kc * C::U_CHUNK + kk * 32), bdesc,
+                         idesc, acc);
+            else
+              mma_f16_ts(dt, tmem_base + (uint32_t)(kc * 32 + kk * 8), bdesc, idesc, acc);
           }
           mma_commit(zempty_bar(s));
         }
         if (!ok) break;
-        mma_commit(dfull_bar);
+        mma_commit(dfull_bar(ab));
       }
       if (tt > 0 && ok) {  // the last tile's MMAs complete before TMEM is freed
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(dfull_bar, (uint32_t)((tt - 1) & 1)) &&
+        const int lb = (int)((tt - 1) % C::NACC);
+        while (!mbar_try_wait(dfull_bar(lb), (uint32_t)(((tt - 1) / C::NACC) & 1)) &&
                globaltimer() - t0 < WAIT_NS) {
         }
       }
