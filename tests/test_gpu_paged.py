@@ -60,19 +60,20 @@ def _setup(B, Hq, Hkv, d, m, P, lens, max_len, seed, garbage=True):
 
 
 @pytest.mark.parametrize("cfg", [
-    # B, Hq, Hkv, d, m, P, lens, append
-    (4, 8, 2, 128, 256, 32, [0, 31, 100, 257], True),     # GQA, page = 1 block
-    (3, 4, 4, 64, 128, 64, [1, 64, 130], True),           # MHA (int8 scoring), 2 blocks/page
-    (2, 16, 1, 128, 256, 128, [500, 33], True),           # two head groups
-    (3, 2, 2, 128, 512, 32, [40, 0, 96], False),          # no append, one empty sequence
+    # B, Hq, Hkv, d, m, P, lens, append, query and new-key dtype
+    (4, 8, 2, 128, 256, 32, [0, 31, 100, 257], True, torch.bfloat16),  # GQA, page = 1 block
+    (3, 4, 4, 64, 128, 64, [1, 64, 130], True, torch.bfloat16),        # MHA (int8), 2 blocks/page
+    (2, 16, 1, 128, 256, 128, [500, 33], True, torch.bfloat16),        # two head groups
+    (3, 2, 2, 128, 512, 32, [40, 0, 96], False, torch.bfloat16),       # no append, one empty
+    (3, 8, 2, 128, 256, 64, [70, 1, 200], True, torch.float32),        # fp32 query and new key
 ])
 def test_paged_append_decode_matches_oracle(cfg):
     torch.cuda.set_device(0)
-    B, Hq, Hkv, d, m, P, lens, append = cfg
+    B, Hq, Hkv, d, m, P, lens, append, dt = cfg
     max_len = max(lens) + 1 + 7
     S, S64, table, (sp, npg, vp), keys, vals = _setup(B, Hq, Hkv, d, m, P, lens, max_len, 7)
-    Q = workloads.random_keys(B * Hq, d, 55, scale=2.0).reshape(B, Hq, d)
-    Kn = workloads.random_keys(B * Hkv, d, 56).reshape(B, Hkv, d)
+    Q = workloads.random_keys(B * Hq, d, 55, dtype=dt, scale=2.0).reshape(B, Hq, d)
+    Kn = workloads.random_keys(B * Hkv, d, 56, dtype=dt).reshape(B, Hkv, d)
     Vn = workloads.random_keys(B * Hkv, d, 57).reshape(B, Hkv, d)
     seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
     out, sc = jl.jl_decode_attention_paged(
@@ -88,7 +89,7 @@ def test_paged_append_decode_matches_oracle(cfg):
         K = keys[b]
         V = vals[b]
         if append:
-            K = torch.cat([K, Kn[b][:, None, :]], dim=1)
+            K = torch.cat([K.to(Kn.dtype), Kn[b][:, None, :]], dim=1)
             V = torch.cat([V, Vn[b][:, None, :]], dim=1)
             # the appended key: code (band rule), norm (1 ulp), value (bitwise)
             pg, sl = table[b, lens[b] // P], lens[b] % P

@@ -34,15 +34,16 @@ def _codes(ref, bits):
 
 
 @pytest.mark.parametrize("cfg", [
-    # B, Hq, Hkv, P, lens, append, bits
-    (4, 8, 2, 32, [0, 31, 100, 257], True, 2),
-    (3, 4, 4, 64, [1, 64, 130], True, 3),
-    (2, 16, 1, 128, [500, 33], True, 1),
-    (3, 8, 2, 32, [40, 0, 96], False, 2),
+    # B, Hq, Hkv, P, lens, append, bits, query and new-key dtype
+    (4, 8, 2, 32, [0, 31, 100, 257], True, 2, torch.bfloat16),
+    (3, 4, 4, 64, [1, 64, 130], True, 3, torch.bfloat16),
+    (2, 16, 1, 128, [500, 33], True, 1, torch.bfloat16),
+    (3, 8, 2, 32, [40, 0, 96], False, 2, torch.bfloat16),
+    (3, 8, 2, 64, [70, 1, 200], True, 2, torch.float32),
 ])
 def test_turbo_paged_append_decode_matches_oracle(cfg):
     torch.cuda.set_device(0)
-    B, Hq, Hkv, P, lens, append, bits = cfg
+    B, Hq, Hkv, P, lens, append, bits, dt = cfg
     rng = np.random.default_rng(B * 100 + P + bits)
     max_len = max(lens) + 1 + 7
     c = tq.lloyd_max(D, bits)
@@ -86,8 +87,8 @@ def test_turbo_paged_append_decode_matches_oracle(cfg):
     cp = torch.from_numpy(code_pool).cuda()
     npg = torch.from_numpy(norm_pool).cuda()
     vp = torch.from_numpy(val_pool).to(torch.bfloat16).cuda()
-    Q = workloads.random_keys(B * Hq, D, 55, scale=2.0).reshape(B, Hq, D)
-    Kn = workloads.random_keys(B * Hkv, D, 56).reshape(B, Hkv, D)
+    Q = workloads.random_keys(B * Hq, D, 55, dtype=dt, scale=2.0).reshape(B, Hq, D)
+    Kn = workloads.random_keys(B * Hkv, D, 56, dtype=dt).reshape(B, Hkv, D)
     Vn = workloads.random_keys(B * Hkv, D, 57).reshape(B, Hkv, D)
     seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
     out, sc = jl.jl_turbo_decode_attention_paged(
@@ -106,7 +107,7 @@ def test_turbo_paged_append_decode_matches_oracle(cfg):
         K, V = keys[b], vals[b]
         same = True
         if append:
-            K = torch.cat([K, Kn[b][:, None, :]], dim=1)
+            K = torch.cat([K.to(Kn.dtype), Kn[b][:, None, :]], dim=1)
             V = torch.cat([V, Vn[b][:, None, :]], dim=1)
             # the appended key: cells and signs within the bands, norms 1 step,
             # value bitwise
