@@ -62,6 +62,25 @@ def test_search_matches_oracle(m, d, N, nq):
     _check(gi.cpu().numpy(), gs.cpu().numpy(), allsc, k)
 
 
+@pytest.mark.parametrize("m,d,N,nq,k", [(256, 128, 50000, 40, 1), (256, 128, 50000, 40, 16),
+                                        (512, 128, 9000, 3, 1), (512, 128, 9000, 3, 16)])
+def test_search_k_extremes(m, d, N, nq, k):
+    # k = 1 and the largest k, on both operand paths (U in shared memory for
+    # m <= 256, in tensor memory for m = 512)
+    torch.cuda.set_device(0)
+    S = jl.jl_sketch_init(m, d, 0)
+    S64 = oracle.sketch(m, d, 0)
+    signs, n16 = _index(N, d, m, 800 + m + k, S64)
+    Q = workloads.random_keys(nq, d, 900 + k, scale=2.0)
+    gi, gs = jl.jl_search_topk(Q.cuda(), S, torch.from_numpy(signs.view(np.int32)).cuda(),
+                               torch.from_numpy(n16.view(np.float16)).cuda(), k)
+    torch.cuda.synchronize()
+    assert jl.jl_device_error() == 0
+    assert gi.shape == (nq, k)
+    _, _, allsc = oracle.search_topk(H.f64(Q), S64, signs, oracle.fp16_bits_to_f64(n16), k)
+    _check(gi.cpu().numpy(), gs.cpu().numpy(), allsc, k)
+
+
 def test_search_fp32_queries_duplicates_and_small_index():
     torch.cuda.set_device(0)
     m, d = 256, 128
