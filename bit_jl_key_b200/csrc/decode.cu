@@ -274,12 +274,16 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
     const int i = threadIdx.x % D, h = threadIdx.x / D;
     constexpr int CP = D / HALVES;
     float acc[PROJ_VECS] = {};
-#pragma unroll 8
-    for (int c = h * CP; c < (h + 1) * CP; ++c) {
-      const float pv = __ldg(Pinv + c * D + i);
+    // all of the thread's Pinv loads in flight at once (one L2 round trip,
+    // not one per group of eight)
+    float pv[CP];
 #pragma unroll
-      for (int j = 0; j < PROJ_VECS; ++j) acc[j] = fmaf(pv, qsm[j * D + c], acc[j]);
-    }
+    for (int cc = 0; cc < CP; ++cc) pv[cc] = __ldg(Pinv + (h * CP + cc) * D + i);
+#pragma unroll
+    for (int cc = 0; cc < CP; ++cc)
+#pragma unroll
+      for (int j = 0; j < PROJ_VECS; ++j)
+        acc[j] = fmaf(pv[cc], qsm[j * D + h * CP + cc], acc[j]);
 #pragma unroll
     for (int j = 0; j < PROJ_VECS; ++j) part[h][j * D + i] = acc[j];
   }
