@@ -362,3 +362,16 @@ def test_turbo_paged_argument_errors(lib):
     assert call(cp=MISALIGNED) == jl.JL_ERR_INVALID_ARG
     assert call(ws=NULL) == jl.JL_ERR_WORKSPACE
     assert call(wsb=need - 1) == jl.JL_ERR_WORKSPACE
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # no fallback: with the library absent, loading it raises instead of
+    # quietly running something else
+    import subprocess
+    import sys
+    env = dict(os.environ, JLKEY_LIBRARY=str(tmp_path / "absent" / "libjlkey.so"))
+    r = subprocess.run([sys.executable, "-c", "import bit_jl_key_b200 as jl; jl.load()"],
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "libjlkey" in (r.stderr + r.stdout)
