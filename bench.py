@@ -101,7 +101,7 @@ def pick_workload(name: str, batch: int = 0) -> workloads.Workload:
 
 
 def _pick(name: str) -> workloads.Workload:
-    if name.startswith("sweep"):
+    if name.startswith("sweep-"):
         # sweep-m<M>-d<D>
         m = int(name.split("-m")[1].split("-")[0])
         d = int(name.split("-d")[1])

@@ -1,0 +1,74 @@
+"""Host logic of bench.py: workload selection, byte accounting, the clock
+record, whole-job rates, and the stored ncu traffic (no GPU needed)."""
+import json
+import os
+
+import pytest
+import torch
+
+import bench
+import workloads
+
+
+def test_every_named_workload_is_selectable():
+    for name in workloads.ALL:
+        w = bench.pick_workload(name)
+        assert w.name == name
+    w = bench.pick_workload("sweep-m512-d64")
+    assert (w.m, w.d) == (512, 64)
+    assert bench.pick_workload("gqa", 2).B == 2
+
+
+def test_byte_accounting_matches_the_stated_per_key_sizes():
+    w = workloads.ALL["gqa"]
+    n = w.B * w.Hkv * w.T
+    # 256 B of bf16 key read, 32 B of code + 2 B of norm written per key
+    assert bench.quantize_bytes(w, n) == n * 290
+    # code + norm + bf16 value row per KV key
+    assert bench.decode_bytes(w) == n * 290
+    assert bench.decode_bytes(w) == 608174080
+
+
+def test_whole_job_rate_counts_every_rank():
+    # weak scaling: each rank's units over the slowest rank's time
+    assert bench.whole_job_rate(1000, 4, 2.0) == pytest.approx(2e6)
+    assert bench.reduce_max_over_ranks(3.5, 1, "cpu") == 3.5
+
+
+def test_clock_record_parsing():
+    s = bench.ClockSampler(0)
+    s.out = "\n".join([
+        "0, 1965, 1965, 240.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 250.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 245.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ])
+    r = s.summary()
+    assert r["sm_mhz"] == 1965 and r["sm_max_mhz"] == 1965
+    assert r["reasons"] == ["sw_power_cap"] and r["samples"] == 3
+    assert r["power_w_max"] == 250.0
+    s.out = "0, 1200, 1965, 500, 0x8, Active, Not Active, Active, Not Active"
+    assert s.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    s.out = ""
+    assert s.summary()["reasons"] == ["unavailable"]
+
+
+def test_stored_traffic_is_keyed_to_the_kernel_sources():
+    p = os.path.join(bench.ROOT, "profiles", "traffic.json")
+    with open(p) as f:
+        d = json.load(f)
+    assert d
+    for key, e in d.items():
+        assert e["dram_bytes_per_launch"] > 0 and e["how"], key
+        got = bench.ncu_traffic(key)
+        # an entry is served only while its sources are unchanged
+        fresh = e["source_hash"] == bench.kernel_source_hash(e["sources"])
+        assert (got is not None) == fresh, key
+    assert bench.ncu_traffic("no-such-kernel") is None
+
+
+def test_peaks_are_read_or_fall_back():
+    gbs, kind = bench.load_peaks()
+    assert gbs > 1000 and kind in ("measured", "fallback")
+    tf, tkind = bench.load_tensor_peak()
+    assert tf > 100 and tkind
