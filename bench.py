@@ -920,6 +920,12 @@ def run_ours(args, rank, world, local_rank):
                             "algorithmic_bytes": db,
                             "GB_per_s": db / (d_ms * 1e-3) / 1e9}
         phases["decode"]["frac_of_hbm_peak"] = phases["decode"]["GB_per_s"] / peak
+        # per-call bytes outside the per-key accounting: listed, not in GB/s
+        phases["decode"]["fixed_bytes_not_counted"] = {
+            "queries": Q.numel() * Q.element_size(),
+            "sketch": S.numel() * S.element_size(),
+            "out": out.numel() * out.element_size(),
+            "workspace (projections + partial states)": int(ws_bytes)}
     dom = max(phases, key=lambda k: phases[k]["ms"])
     traffic = ncu_traffic({"quantize": "quantize", "decode": "decode"}[dom] + ":" + w.name)
     roof = {"kernel": {"quantize": "jl_quantize_keys", "decode": "jl_decode_attention"}[dom],
