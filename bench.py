@@ -100,6 +100,12 @@ def pick_workload(name: str, batch: int = 0) -> workloads.Workload:
     return w.with_(B=batch) if batch else w
 
 
+def rank_workload(args, rank: int) -> workloads.Workload:
+    """This rank's batch: sequences [rank*B, (rank+1)*B) of the global batch
+    (every rank holds B sequences of its own; weak scaling)."""
+    return workloads.shard(pick_workload(args.workload, args.batch), rank)
+
+
 def _pick(name: str) -> workloads.Workload:
     if name.startswith("sweep-"):
         # sweep-m<M>-d<D>
@@ -271,7 +277,7 @@ def run_paged(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     turbo = w.name.startswith("turbo")
     bits = workloads.TURBO_MSE_BITS
     peak, peak_kind = load_peaks()
@@ -279,7 +285,8 @@ def run_paged(args, rank, world, local_rank):
     lens, table, num_pages = workloads.paged_layout(w, P)
     S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
     # fill the pool (untimed): keys and values of every slot, quantized in place
-    pool = w.with_(B=num_pages, T=P)
+    # pages of this rank's pool, seeded apart from every other rank's pool
+    pool = w.with_(B=num_pages, T=P, first_seq=rank * (w.B * -(-w.T // P) + 16))
     Kp = workloads.keys(pool, dev)
     if turbo:
         Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED, device=dev)
@@ -411,7 +418,7 @@ def run_dequant(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     peak, peak_kind = load_peaks()
     S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
     K = workloads.keys(w, dev)
@@ -505,7 +512,7 @@ def run_search(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     k = workloads.SEARCH_K
     hbm_peak, _ = load_peaks()
     tpeak, tkind = load_tensor_peak()
@@ -607,7 +614,7 @@ def run_turbo(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     bits = workloads.TURBO_MSE_BITS
     peak, peak_kind = load_peaks()
     Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED, device=dev)
@@ -757,6 +764,135 @@ def run_turbo(args, rank, world, local_rank):
     }
 
 
+def _timed_loop(stream, fn, n):
+    """Mean device time per call of n back-to-back calls (events at the ends
+    only: an event between calls would drain the stream)."""
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def phase_records(w, n_keys, q_ms, d_ms, peak, decode, extra_fixed=None):
+    """Per-phase rates and roofline fractions from event-timed durations."""
+    qb = quantize_bytes(w, n_keys)
+    phases = {"quantize": {"ms": q_ms, "keys_per_s": n_keys / (q_ms * 1e-3),
+                           "tokens_per_s": w.B * w.T / (q_ms * 1e-3),
+                           "algorithmic_bytes": qb,
+                           "GB_per_s": qb / (q_ms * 1e-3) / 1e9}}
+    phases["quantize"]["frac_of_hbm_peak"] = phases["quantize"]["GB_per_s"] / peak
+    if decode:
+        db = decode_bytes(w)
+        phases["decode"] = {"ms": d_ms, "keys_scored_per_s": n_keys / (d_ms * 1e-3),
+                            "head_key_pairs_per_s": w.B * w.Hq * w.T / (d_ms * 1e-3),
+                            "algorithmic_bytes": db,
+                            "GB_per_s": db / (d_ms * 1e-3) / 1e9}
+        phases["decode"]["frac_of_hbm_peak"] = phases["decode"]["GB_per_s"] / peak
+        if extra_fixed:
+            phases["decode"]["fixed_bytes_not_counted"] = extra_fixed
+    return phases
+
+
+PHASE_KERNEL = {"quantize": "jl_quantize_keys (quantize_tc_kernel)",
+                "decode": "jl_decode_attention (qproj + decode_scorer_kernel + combine)"}
+
+
+def roofline_of(phase, rec, w, peak, peak_kind):
+    """Roofline entry of one phase: its algorithmic bytes over its event-timed
+    duration, against the measured HBM copy bandwidth; DRAM traffic per launch
+    from the committed ncu summary when the kernel's source is unchanged."""
+    traffic = ncu_traffic(phase + ":" + w.name)
+    r = {"kernel": PHASE_KERNEL[phase], "bound": "hbm", "achieved": rec["GB_per_s"],
+         "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+         "frac": rec["GB_per_s"] / peak,
+         "algorithmic_bytes_per_launch": rec["algorithmic_bytes"],
+         "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
+    if traffic:
+        for k in ("dram_read_bytes_per_launch", "dram_write_bytes_per_launch",
+                  "write_side"):
+            if k in traffic:
+                r[k.replace("_per_launch", "")] = traffic[k]
+    return r
+
+
+def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error):
+    """One more workload on one GPU: quantize every key, then one decode step
+    over the compressed cache (prefill: quantize only).  Returns a record with
+    the step time, per-phase rates and rooflines (and, for the sketch-size
+    sweep, the estimator's error against the exact inner products)."""
+    stream = torch.cuda.current_stream(dev)
+    decode = w.name != "prefill"
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)
+    Kf = K.view(-1, w.d)
+    n_keys = Kf.shape[0]
+    W = w.m // 32
+    signs = torch.empty((n_keys, W), dtype=torch.int32, device=dev)
+    norms = torch.empty((n_keys,), dtype=torch.float16, device=dev)
+    if decode:
+        V = workloads.values(w, dev)
+        Q = workloads.queries(w, dev)
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((jl.jl_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.T, w.m, w.d),),
+                         dtype=torch.uint8, device=dev)
+        sg4 = signs.view(w.B, w.Hkv, w.T, W)
+        nr3 = norms.view(w.B, w.Hkv, w.T)
+
+    def quantize():
+        jl.jl_quantize_keys(Kf, S, signs, norms)
+
+    def decode_call():
+        jl.jl_decode_attention(Q, S, sg4, nr3, V, softmax_scale=w.softmax_scale,
+                               out=out, workspace=ws)
+
+    def step():
+        quantize()
+        if decode:
+            decode_call()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ms = _timed_loop(stream, step, steps)
+    q_ms = _timed_loop(stream, quantize, steps)
+    d_ms = _timed_loop(stream, decode_call, steps) if decode else 0.0
+    if jl.jl_device_error() != 0:
+        raise RuntimeError(f"device error in workload {w.name}")
+    phases = phase_records(w, n_keys, q_ms, d_ms, peak, decode)
+    rec = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} d={w.d} m={w.m}",
+           "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "keys_per_s": n_keys / (ms * 1e-3), "phases": phases,
+           "rooflines": {ph: roofline_of(ph, phases[ph], w, peak, peak_kind) for ph in phases},
+           "l2": "inputs exceed L2 (126 MB); no flush" if n_keys * w.d * 2 > 126e6
+                 else "inputs fit in L2; latency-bound parity workload"}
+    if w.name == "prefill":
+        rec["quantize_tokens_per_s"] = w.T / (q_ms * 1e-3)
+        rec["quantize_tokens_per_s_note"] = ("tokens of all 32 layers x 8 KV heads per second "
+                                             "(keys/s divided by layers x heads)")
+    if decode and with_score_error:
+        rec["score_error"] = score_error(jl, w, Q, S, sg4, nr3, V, K)
+    del K, signs, norms
+    if decode:
+        del V, Q, out, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+def other_configs():
+    """The workloads measured beside the headline one: the single-head parity
+    workload, long-context MHA decode, prefill quantization and the eight
+    points of the sketch-size sweep."""
+    return ([workloads.SINGLE, workloads.LONG, workloads.PREFILL] + workloads.sweep_points())
+
+
+def config_key(w) -> str:
+    return w.name if w.name != "sweep" else f"sweep-m{w.m}-d{w.d}"
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
@@ -770,7 +906,7 @@ def run_ours(args, rank, world, local_rank):
         return run_dequant(args, rank, world, local_rank)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     decode = w.name != "prefill"
     peak, peak_kind = load_peaks()
 
@@ -906,34 +1042,18 @@ def run_ours(args, rank, world, local_rank):
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
-    # ---- roofline of the dominant kernel
-    qb = quantize_bytes(w, n_keys)
-    phases = {"quantize": {"ms": q_ms, "keys_per_s": n_keys / (q_ms * 1e-3),
-                           "tokens_per_s": w.B * w.T / (q_ms * 1e-3),
-                           "algorithmic_bytes": qb,
-                           "GB_per_s": qb / (q_ms * 1e-3) / 1e9}}
-    phases["quantize"]["frac_of_hbm_peak"] = phases["quantize"]["GB_per_s"] / peak
+    # ---- roofline of the dominant kernel, and of both phases
+    fixed = None
     if decode:
-        db = decode_bytes(w)
-        phases["decode"] = {"ms": d_ms, "keys_scored_per_s": n_keys / (d_ms * 1e-3),
-                            "head_key_pairs_per_s": w.B * w.Hq * w.T / (d_ms * 1e-3),
-                            "algorithmic_bytes": db,
-                            "GB_per_s": db / (d_ms * 1e-3) / 1e9}
-        phases["decode"]["frac_of_hbm_peak"] = phases["decode"]["GB_per_s"] / peak
         # per-call bytes outside the per-key accounting: listed, not in GB/s
-        phases["decode"]["fixed_bytes_not_counted"] = {
-            "queries": Q.numel() * Q.element_size(),
-            "sketch": S.numel() * S.element_size(),
-            "out": out.numel() * out.element_size(),
-            "workspace (projections + partial states)": int(ws_bytes)}
+        fixed = {"queries": Q.numel() * Q.element_size(),
+                 "sketch": S.numel() * S.element_size(),
+                 "out": out.numel() * out.element_size(),
+                 "workspace (projections + partial states)": int(ws_bytes)}
+    phases = phase_records(w, n_keys, q_ms, d_ms, peak, decode, fixed)
+    rooflines = {ph: roofline_of(ph, phases[ph], w, peak, peak_kind) for ph in phases}
     dom = max(phases, key=lambda k: phases[k]["ms"])
-    traffic = ncu_traffic({"quantize": "quantize", "decode": "decode"}[dom] + ":" + w.name)
-    roof = {"kernel": {"quantize": "jl_quantize_keys", "decode": "jl_decode_attention"}[dom],
-            "bound": "hbm", "achieved": phases[dom]["GB_per_s"], "peak": peak,
-            "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
-            "frac": phases[dom]["GB_per_s"] / peak,
-            "algorithmic_bytes_per_launch": phases[dom]["algorithmic_bytes"],
-            "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
+    roof = rooflines[dom]
 
     clocks = clk.summary()
     line = {
@@ -950,6 +1070,7 @@ def run_ours(args, rank, world, local_rank):
         "phases": phases,
         "phase_timing": "each phase alone: K back-to-back calls, CUDA events at the ends",
         "roofline": roof,
+        "rooflines": rooflines,
         "score_error": score_err,
         "reconstruction_error": recon_err,
         "e2e": e2e,
@@ -957,6 +1078,25 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     return line
+
+
+def measure_other_configs(jl, dev, args, peak, peak_kind):
+    steps = max(3, min(args.steps, 10))
+    warmup = max(3, min(args.warmup, 5))
+    torch.cuda.empty_cache()
+    recs = {}
+    with ClockSampler(dev.index or 0) as clk:
+        for w in other_configs():
+            rec = measure_config(jl, w, dev, steps, warmup, peak, peak_kind,
+                                 with_score_error=(w.name == "sweep" and not args.no_score_error))
+            cb = getattr(args, "config_baselines", {}).get(config_key(w))
+            if cb is not None:
+                rec["cpu_baseline"] = cb
+            recs[config_key(w)] = rec
+    recs["clocks"] = clk.summary()
+    recs["note"] = ("each workload alone on one GPU, after the headline; steps and warm-up "
+                    "as listed per workload; rates and rooflines as the headline's")
+    return recs
 
 
 # --------------------------------------------------------------------------
@@ -1051,7 +1191,7 @@ def time_oracle(w, steps=1, warmup=0):
 
 
 def run_reference(args, rank, world):
-    w = pick_workload(args.workload, args.batch)
+    w = rank_workload(args, rank)
     if rank != 0:
         return None
     cb = time_oracle(w, steps=args.steps, warmup=args.warmup)
@@ -1086,6 +1226,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-score-error", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only the selected workload (default gqa runs also time "
+                         "the single, long, prefill and sweep workloads)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -1111,9 +1254,22 @@ def main():
     try:
         # the oracle runs before any GPU work on rank 0 (bounded sample)
         cb = None
+        args.config_baselines = {}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             cb = time_oracle(pick_workload(args.workload, args.batch), steps=1)
+            if args.workload == "gqa" and not args.no_configs:
+                for w in other_configs():
+                    c = time_oracle(w, steps=1)
+                    args.config_baselines[config_key(w)] = {
+                        k: c[k] for k in ("value", "unit", "cores", "kind", "sample")}
         line = run_ours(args, rank, world, local_rank)
+        if world == 1 and args.workload == "gqa" and not args.no_configs:
+            # the other workloads, each on its own, after the headline's
+            # tensors are released (weak-scaling runs skip them)
+            import bit_jl_key_b200 as jl
+            peak, peak_kind = load_peaks()
+            line["configs"] = measure_other_configs(
+                jl, torch.device("cuda", local_rank), args, peak, peak_kind)
         if cb is not None:
             line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
         if rank == 0:

@@ -273,6 +273,47 @@ def jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d) -> int:
     return int(load().jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d))
 
 
+def _decode_shapes(Q, S, signs, norms, V, out, scores):
+    """Shape, dtype and layout checks shared by the two decode wrappers: the
+    library sizes its copies from (B, Hq, Hkv, T, m, d), so a tensor shorter
+    than those shapes say would be read past its end.  Returns
+    (B, Hq, Hkv, T, m, d, query dtype code)."""
+    if Q.dim() != 3 or V.dim() != 4 or S.dim() != 2:
+        raise ValueError("Q must be [B, Hq, d], V [B, Hkv, T, d] and S [m, d]")
+    B, Hq, d = Q.shape
+    Bv, Hkv, T, dv = V.shape
+    m = S.shape[0]
+    if Q.dtype == torch.float32:
+        qt = JL_F32
+    elif Q.dtype == torch.bfloat16:
+        qt = JL_BF16
+    else:
+        raise TypeError(f"unsupported query dtype {Q.dtype}")
+    if Bv != B or dv != d:
+        raise ValueError(f"V {tuple(V.shape)} does not match Q {tuple(Q.shape)}")
+    if S.shape != (m, d) or S.dtype != torch.bfloat16:
+        raise ValueError(f"S must be bf16 [m, {d}], got {S.dtype} {tuple(S.shape)}")
+    if signs.shape != (B, Hkv, T, m // 32) or signs.dtype != torch.int32:
+        raise ValueError(f"signs must be int32 {(B, Hkv, T, m // 32)}, got "
+                         f"{signs.dtype} {tuple(signs.shape)}")
+    if norms.shape != (B, Hkv, T) or norms.dtype != torch.float16:
+        raise ValueError(f"norms must be float16 {(B, Hkv, T)}, got "
+                         f"{norms.dtype} {tuple(norms.shape)}")
+    if V.dtype != torch.bfloat16:
+        raise ValueError(f"V must be bf16, got {V.dtype}")
+    if out is not None and (out.shape != (B, Hq, d) or out.dtype != torch.bfloat16
+                            or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous bf16 {(B, Hq, d)} tensor")
+    if scores is not None and (scores.shape != (B, Hq, T) or scores.dtype != torch.float32
+                               or not scores.is_contiguous()):
+        raise ValueError(f"scores must be a contiguous float32 {(B, Hq, T)} tensor")
+    for t in (Q, S, signs, norms, V):
+        if not t.is_contiguous():
+            raise ValueError("decode inputs must be contiguous")
+    _need_cuda(Q, S, signs, norms, V, out, scores)
+    return B, Hq, Hkv, T, m, d, qt
+
+
 def jl_decode_attention(Q, S, signs, norms, V, softmax_scale=None, out=None,
                         scores=None, want_scores=False, workspace=None,
                         stream=None):
@@ -283,20 +324,7 @@ def jl_decode_attention(Q, S, signs, norms, V, softmax_scale=None, out=None,
     (out, scores [B, Hq, T] fp32) when ``want_scores`` (or ``scores`` given).
     """
     L = load()
-    B, Hq, d = Q.shape
-    Bv, Hkv, T, dv = V.shape
-    m = S.shape[0]
-    _need_cuda(Q, S, signs, norms, V)
-    assert Bv == B and dv == d
-    assert signs.shape == (B, Hkv, T, m // 32) and signs.dtype == torch.int32
-    assert norms.shape == (B, Hkv, T) and norms.dtype == torch.float16
-    assert V.dtype == torch.bfloat16
-    for t in (Q, S, signs, norms, V):
-        if not t.is_contiguous():
-            raise ValueError("decode inputs must be contiguous")
-    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
-    if Q.dtype not in (torch.float32, torch.bfloat16):
-        raise TypeError(f"unsupported query dtype {Q.dtype}")
+    B, Hq, Hkv, T, m, d, qt = _decode_shapes(Q, S, signs, norms, V, out, scores)
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -330,14 +358,7 @@ def jl_decode_attention_noalloc(Q, S, signs, norms, V, softmax_scale=None,
     tensors passed in are used as given; when ``out``/``scores`` are None this
     wrapper creates them with torch, as it would for any caller."""
     L = load()
-    B, Hq, d = Q.shape
-    _, Hkv, T, _ = V.shape
-    m = S.shape[0]
-    _need_cuda(Q, S, signs, norms, V)
-    for t in (Q, S, signs, norms, V):
-        if not t.is_contiguous():
-            raise ValueError("decode inputs must be contiguous")
-    qt = JL_F32 if Q.dtype == torch.float32 else JL_BF16
+    B, Hq, Hkv, T, m, d, qt = _decode_shapes(Q, S, signs, norms, V, out, scores)
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(d)
     if out is None:

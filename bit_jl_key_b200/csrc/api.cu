@@ -17,6 +17,7 @@ std::mutex g_attr_mu;
 int g_sm_count[kMaxDevices];
 int g_smem_optin[kMaxDevices];
 int *g_err_ptr[kMaxDevices];
+unsigned long long g_err_ctx[kMaxDevices];
 
 int current_device() {
   int dev = 0;
@@ -42,13 +43,41 @@ int device_sm_count() {
 int *device_error_ptr() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(g_attr_mu);
-  if (g_err_ptr[dev] == nullptr) {
+  if (g_err_ptr[dev] == nullptr || g_err_ctx[dev] != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
     g_err_ptr[dev] = static_cast<int *>(p);
+    g_err_ctx[dev] = ctx;
   }
   return g_err_ptr[dev];
+}
+
+unsigned long long current_context_id() {
+  using GetCurrent = int (*)(void **);
+  using GetId = int (*)(void *, unsigned long long *);
+  static std::once_flag once;
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  std::call_once(once, [] {
+    void *a = nullptr, *b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) ==
+            cudaSuccess && qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrent>(a);
+      get_id = reinterpret_cast<GetId>(b);
+    }
+  });
+  if (!get_current || !get_id) return 0;
+  // 0 also when no context is bound to this thread yet: the first lookup made
+  // under id 0 is then repeated once the runtime has bound one
+  void *ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != 0 || ctx == nullptr || get_id(ctx, &id) != 0) return 0;
+  return id;
 }
 
 void *tensor_map_encoder() {
@@ -77,6 +106,32 @@ int device_max_smem_optin() {
     g_smem_optin[dev] = v;
   }
   return g_smem_optin[dev];
+}
+
+int validate_decode(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                    const uint32_t *signs, const uint16_t *norms, const uint16_t *V,
+                    int B, int Hq, int Hkv, int64_t T, int m, int d, float softmax_scale,
+                    const uint16_t *out, const float *scores, DecodePlan *plan,
+                    bool *empty) {
+  auto al = [](const void *p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+  };
+  *empty = false;
+  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
+  if (!((d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512)))
+    return JL_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;  // NaN
+  if (B == 0) {
+    *empty = true;
+    return JL_OK;
+  }
+  if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
+  if (!al(Q, 16) || !al(S, 16) || !al(signs, 16) || !al(norms, 16) || !al(V, 16) ||
+      !al(out, 4) || (scores && !al(scores, 4)))
+    return JL_ERR_INVALID_ARG;
+  if (!make_decode_plan(B, Hq, Hkv, T, m, d, plan)) return JL_ERR_UNSUPPORTED;
+  return JL_OK;
 }
 
 }  // namespace jlk
@@ -214,19 +269,11 @@ int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
                         int m, int d, float softmax_scale, uint16_t *out,
                         float *scores, void *workspace, size_t workspace_bytes,
                         jl_stream_t stream) {
-  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
-  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0)
-    return JL_ERR_INVALID_ARG;
-  if (!supported_md(m, d)) return JL_ERR_UNSUPPORTED;
-  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;  // NaN
-  if (B == 0) return JL_OK;
-  if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
-  if (!aligned(Q, 16) || !aligned(S, 16) || !aligned(signs, 16) ||
-      !aligned(norms, 16) || !aligned(V, 16) || !aligned(out, 4) ||
-      (scores && !aligned(scores, 4)))
-    return JL_ERR_INVALID_ARG;
   jlk::DecodePlan p;
-  if (!jlk::make_decode_plan(B, Hq, Hkv, T, m, d, &p)) return JL_ERR_UNSUPPORTED;
+  bool empty = false;
+  const int st = jlk::validate_decode(Q, q_dtype, S, signs, norms, V, B, Hq, Hkv, T, m, d,
+                                      softmax_scale, out, scores, &p, &empty);
+  if (st != JL_OK || empty) return st;
   if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
     return JL_ERR_WORKSPACE;
   return from_cuda(jlk::launch_decode(p, Q, q_dtype == JL_F32, S, signs, norms,

@@ -17,7 +17,9 @@
 //  - shapes whose scratch would exceed the array are rejected before any
 //    launch;
 //  - the array's device address is looked up once per device, on the first
-//    call made with that device current.
+//    call made with that device current, and looked up again only if that
+//    device's context has been replaced since (cudaDeviceReset), so a reset
+//    never leaves a stale address behind.
 #include "jl_common.cuh"
 #include "jl_internal.h"
 
@@ -31,6 +33,7 @@ static __device__ __align__(256) unsigned char
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void *g_scratch_ptr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];
 
 // Device address of g_decode_scratch on the current device.  In host code the
 // array's name stands for a host-side shadow, not device memory, so kernels
@@ -40,12 +43,14 @@ cudaError_t scratch_address(void **out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = jlk::current_context_id();
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -58,25 +63,12 @@ extern "C" int jl_decode_attention_noalloc(
     const uint16_t *norms, const uint16_t *V, int B, int Hq, int Hkv,
     int64_t T, int m, int d, float softmax_scale, uint16_t *out,
     float *scores, jl_stream_t stream) {
-  // same argument checks as jl_decode_attention, minus the workspace
-  if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
-  if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0)
-    return JL_ERR_INVALID_ARG;
-  if (!((d == 64 || d == 128) &&
-        (m == 64 || m == 128 || m == 256 || m == 512)))
-    return JL_ERR_UNSUPPORTED;
-  if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
-  if (B == 0) return JL_OK;
-  if (!Q || !S || !signs || !norms || !V || !out) return JL_ERR_INVALID_ARG;
-  auto misaligned = [](const void *p, uintptr_t a) {
-    return (reinterpret_cast<uintptr_t>(p) % a) != 0;
-  };
-  if (misaligned(Q, 16) || misaligned(S, 16) || misaligned(signs, 16) ||
-      misaligned(norms, 16) || misaligned(V, 16) || misaligned(out, 4) ||
-      (scores && misaligned(scores, 4)))
-    return JL_ERR_INVALID_ARG;
+  // the checks of jl_decode_attention, minus the workspace
   jlk::DecodePlan p;
-  if (!jlk::make_decode_plan(B, Hq, Hkv, T, m, d, &p)) return JL_ERR_UNSUPPORTED;
+  bool empty = false;
+  const int st = jlk::validate_decode(Q, q_dtype, S, signs, norms, V, B, Hq, Hkv, T, m, d,
+                                      softmax_scale, out, scores, &p, &empty);
+  if (st != JL_OK || empty) return st;
   if (p.total_bytes > (size_t)JL_DECODE_STATIC_SCRATCH_BYTES)
     return JL_ERR_SCRATCH_LIMIT;
   void *scratch = nullptr;

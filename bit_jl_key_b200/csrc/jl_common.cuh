@@ -18,6 +18,11 @@ namespace jlk {
 // and returns early.  device_error_ptr() is the word's device address for the
 // current device.
 int *device_error_ptr();
+// Unique id of the CUDA context bound to the calling thread (0 if none is
+// bound yet or the driver cannot tell).  Caches of device addresses are keyed
+// by it, so a context torn down and created again (cudaDeviceReset) makes
+// them look the address up again instead of handing out a stale one.
+unsigned long long current_context_id();
 
 enum DeviceErr : int {
   DERR_NONE = 0,

@@ -91,6 +91,16 @@ cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, b
                                 float softmax_scale, uint16_t *out, float *scores,
                                 void *workspace, cudaStream_t stream);
 
+// Argument checks of jl_decode_attention that do not involve the workspace
+// (dtype, shapes, null pointers, alignment) and the work split they imply.
+// Returns JL_OK with *plan filled, or the status the entry point returns.
+// *empty is set when B == 0 (nothing to do).
+int validate_decode(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                    const uint32_t *signs, const uint16_t *norms, const uint16_t *V,
+                    int B, int Hq, int Hkv, int64_t T, int m, int d, float softmax_scale,
+                    const uint16_t *out, const float *scores, DecodePlan *plan,
+                    bool *empty);
+
 cudaError_t launch_decode(const DecodePlan &p, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,
                           const uint16_t *norms, const uint16_t *V,

@@ -312,7 +312,9 @@ JL_API int jl_decode_attention_paged(
  *    results: serialise them.
  *  - Set-up: the first call made with a given device current looks up the
  *    array's device address on that device; make that first call before any
- *    stream capture.
+ *    stream capture.  If that device's context is later destroyed and made
+ *    again (cudaDeviceReset), the next call sees the new context and looks
+ *    the address up again, so it never launches with a stale one.
  */
 #define JL_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,

@@ -62,6 +62,23 @@ def score_violations(gpu: np.ndarray, ref: np.ndarray) -> int:
     return int(np.count_nonzero(np.abs(gpu - ref) > tol))
 
 
+def key_match_mask(gpu_words: np.ndarray, ref_words: np.ndarray,
+                   gpu_norm_bits: np.ndarray, ref_norm_bits: np.ndarray) -> np.ndarray:
+    """[...] bool: keys whose GPU code and binary16 norm equal the oracle's
+    bit for bit (code words on the last axis)."""
+    same_code = np.all(gpu_words.astype(np.uint32) == ref_words.astype(np.uint32), axis=-1)
+    return same_code & (gpu_norm_bits.astype(np.uint16) == ref_norm_bits.astype(np.uint16))
+
+
+def masked_score_violations(gpu: np.ndarray, ref: np.ndarray, mask: np.ndarray) -> int:
+    """score_violations restricted to the entries where ``mask`` is set (the
+    rms that scales the tolerance still runs over every key of the row)."""
+    rms = np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True))
+    tol = SCORE_REL * np.maximum(np.abs(ref), rms)
+    bad = (np.abs(gpu - ref) > tol) & np.broadcast_to(mask, ref.shape)
+    return int(np.count_nonzero(bad))
+
+
 def output_errors(gpu: np.ndarray, ref: np.ndarray):
     """(max abs error, max over vectors of ||err|| / ||ref||)."""
     err = gpu - ref

@@ -140,6 +140,68 @@ def test_decode_argument_errors(lib):
     assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == jl.JL_ERR_WORKSPACE
 
 
+def test_noalloc_argument_errors_match_decode(lib):
+    # the no-alloc variant shares jl_decode_attention's checks (minus the
+    # workspace): every argument error gets the same status from both
+    f = lib.jl_decode_attention_noalloc
+    g = lib.jl_decode_attention
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, S=FAKE, signs=FAKE, norms=FAKE, V=FAKE,
+              B=2, Hq=8, Hkv=2, T=100, m=256, d=128, scale=0.1, out=FAKE,
+              scores=NULL)
+
+    def both(**kw):
+        a = dict(ok, **kw)
+        args = (a["Q"], a["qt"], a["S"], a["signs"], a["norms"], a["V"], a["B"], a["Hq"],
+                a["Hkv"], a["T"], a["m"], a["d"], ctypes.c_float(a["scale"]), a["out"],
+                a["scores"])
+        return f(*args, NULL), g(*args, FAKE, 1 << 40, NULL)
+
+    cases = [dict(B=0), dict(T=0), dict(Hq=6, Hkv=4), dict(Hkv=0), dict(qt=5), dict(m=48),
+             dict(d=256), dict(V=MISALIGNED), dict(signs=MISALIGNED),
+             dict(norms=ctypes.c_void_p((1 << 20) + 8)), dict(scale=float("nan")),
+             dict(scores=ctypes.c_void_p((1 << 20) + 2))]
+    cases += [{k: NULL} for k in ("Q", "S", "signs", "norms", "V", "out")]
+    for kw in cases:
+        na, ws = both(**kw)
+        assert na == ws, (kw, na, ws)
+        assert (na == jl.JL_OK) == (kw == dict(B=0)), kw
+
+
+@pytest.mark.parametrize("fn", ["jl_decode_attention", "jl_decode_attention_noalloc"])
+def test_decode_wrappers_check_shapes_and_dtypes(lib, fn):
+    # the library sizes its copies from the shapes, so the binding must refuse
+    # tensors that do not hold what those shapes say (checked before any
+    # device test: these tensors are on the host)
+    import torch
+    B, Hq, Hkv, T, m, d = 2, 8, 2, 64, 256, 128
+    Q = torch.zeros(B, Hq, d, dtype=torch.bfloat16)
+    S = torch.zeros(m, d, dtype=torch.bfloat16)
+    signs = torch.zeros(B, Hkv, T, m // 32, dtype=torch.int32)
+    norms = torch.zeros(B, Hkv, T, dtype=torch.float16)
+    V = torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16)
+    call = getattr(jl, fn)
+    bad = [
+        dict(signs=torch.zeros(B, Hkv, T - 1, m // 32, dtype=torch.int32)),
+        dict(signs=torch.zeros(B, Hkv, T, m // 64, dtype=torch.int32)),
+        dict(signs=signs.float()),
+        dict(norms=torch.zeros(B, Hkv, T - 1, dtype=torch.float16)),
+        dict(norms=norms.float()),
+        dict(V=V.half()),
+        dict(V=torch.zeros(B, Hkv, T, 64, dtype=torch.bfloat16)),
+        dict(S=torch.zeros(m, 64, dtype=torch.bfloat16)),
+        dict(S=S.float()),
+    ]
+    for kw in bad:
+        a = dict(Q=Q, S=S, signs=signs, norms=norms, V=V)
+        a.update(kw)
+        with pytest.raises(ValueError):
+            call(a["Q"], a["S"], a["signs"], a["norms"], a["V"])
+    with pytest.raises(TypeError):
+        call(Q.half(), S, signs, norms, V)
+    with pytest.raises(ValueError):          # well-formed, but on the host
+        call(Q, S, signs, norms, V)
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(ValueError):

@@ -2,10 +2,11 @@
 
 The GPU quantizes the whole cache and decodes it in the same launch
 configuration the bench times.  The oracle recomputes a sample: whole
-(b, kv-head) units for the decode workloads (their codes are compared with
-the band rule, then the oracle's codes for those units are written into the
-GPU cache so that the sampled outputs compare exactly-defined quantities),
-and random keys for the prefill workload.
+(b, kv-head) units for the decode workloads, and random keys for the prefill
+workload.  Each sampled unit is checked twice: the GPU chain (the GPU's own
+codes decoded on the GPU; scores compared on every key whose code and norm
+equal the oracle's, outputs whole), then with the oracle's codes written into
+the GPU cache (every score and output).
 """
 import math
 
@@ -41,16 +42,31 @@ def _decode_workload_check(w, units, q_scale=1.0):
     signs, norms = jl.jl_quantize_keys(K.view(-1, w.d), S)
     signs = signs.view(w.B, w.Hkv, w.T, W)
     norms = norms.view(w.B, w.Hkv, w.T)
-    report = []
+    # 1) the GPU chain: decode the GPU's own codes and norms
+    out, sc = jl.jl_decode_attention(Q, S, signs, norms, V,
+                                     softmax_scale=w.softmax_scale,
+                                     want_scores=True)
+    torch.cuda.synchronize()
+    chain = {}
+    for (b, hk) in units:
+        hqs = list(range(hk * w.G, (hk + 1) * w.G))
+        chain[(b, hk)] = (H.f64(sc[b, hqs])[None], H.f64(out[b, hqs])[None])
+    del out, sc
+    # 2) the oracle's codes for the sampled units: compared with the GPU's
+    # (band rule), then written into the cache for an all-keys decode check
+    report, refs = [], {}
     for (b, hk) in units:
         Kf = H.f64(K[b, hk])
         rsig, _, rn16, band = oracle.quantize(Kf, S64, band_rel=H.BAND_REL,
                                               want_band=True)
-        out_band, in_band = H.compare_codes(H.u32(signs[b, hk]), rsig, band, w.m)
+        g_words, g_norm = H.u32(signs[b, hk]), H.fp16_bits(norms[b, hk])
+        out_band, in_band = H.compare_codes(g_words, rsig, band, w.m)
         assert out_band == 0, (b, hk, out_band)
-        ulp = H.fp16_ulp_diff(H.fp16_bits(norms[b, hk]), rn16)
+        ulp = H.fp16_ulp_diff(g_norm, rn16)
         assert ulp.max() <= 1
-        report.append((b, hk, in_band, int((ulp > 0).sum())))
+        mask = H.key_match_mask(g_words, rsig, g_norm, rn16)
+        refs[(b, hk)] = mask
+        report.append((b, hk, in_band, int((ulp > 0).sum()), int((~mask).sum())))
         signs[b, hk] = torch.from_numpy(rsig.view(np.int32)).to(dev)
         norms[b, hk] = torch.from_numpy(rn16.view(np.float16)).to(dev)
     del K
@@ -66,12 +82,22 @@ def _decode_workload_check(w, units, q_scale=1.0):
         Vs = H.f64(V[b, hk])[None, None]
         ref_out, ref_sc = oracle.decode(Qs, S64, rsig, rn, Vs, w.softmax_scale,
                                         want_scores=True)
+        # planted codes: every score and output
         g_sc = H.f64(sc[b, hqs])[None]
         g_out = H.f64(out[b, hqs])[None]
         assert H.score_violations(g_sc, ref_sc) == 0, (b, hk)
         mabs, rel = H.output_errors(g_out, ref_out)
         assert mabs <= H.OUT_ABS and rel <= 1e-2, (b, hk, mabs, rel)
-    print(f"{w.name} m={w.m} d={w.d}: units (b, hkv, in-band flips, norm ulps) {report}")
+        # GPU chain: scores of the keys whose code and norm match the
+        # oracle's exactly; outputs of the whole chain
+        c_sc, c_out = chain[(b, hk)]
+        mask = refs[(b, hk)]
+        assert int((~mask).sum()) <= max(4, w.T // 100), (b, hk)
+        assert H.masked_score_violations(c_sc, ref_sc, mask) == 0, (b, hk)
+        mabs, _ = H.output_errors(c_out, ref_out)
+        assert mabs <= H.OUT_ABS, (b, hk, mabs)
+    print(f"{w.name} m={w.m} d={w.d}: units (b, hkv, in-band flips, norm ulps, "
+          f"keys left out of the chain's score check) {report}")
 
 
 def test_gqa_full_size():

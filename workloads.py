@@ -34,10 +34,16 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
-  * data seeds: workload index i (1..5) gives torch generator seeds
-    1000*i + {0: keys, 1: values, 2: queries, 3: outlier channels,
-    4: per-token norms, 5: sequence lengths, 6: page order, 7: appended
-    keys, 8: appended values};
+  * data seeds: workload index i and sequence g (the position of a batch
+    row in the global batch) give torch generator seeds
+    1000*i + k + 1000003*g with k in {0: keys, 1: values, 2: queries,
+    4: per-token norms, 5: sequence length, 7: appended key, 8: appended
+    value}; k = 3 (outlier channels) and k = 6 (page order) are drawn once
+    per workload (page order: per rank's pool);
+  * sharding: under data parallelism rank r holds sequences
+    [r*B, (r+1)*B) of the global batch (``shard``), so the ranks' batches
+    are distinct and together are exactly the global batch of B*world
+    sequences;
   * outlier channels: the first 4 entries of a seeded permutation of range(d);
   * queries are N(0,1) in the key dtype, scaled by ``q_scale`` (default 1);
   * softmax scale 1/sqrt(d).
@@ -53,7 +59,7 @@ import torch
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    index: int              # 1..5, selects the data seeds
+    index: int              # selects the data seeds
     B: int                  # batch
     Hq: int                 # query heads
     Hkv: int                # KV heads
@@ -64,6 +70,7 @@ class Workload:
     outliers: int = 0       # number of outlier channels scaled by 10
     lognormal_sigma: float = 0.0  # per-token norm spread (0 = none)
     sketch_seed: int = 0
+    first_seq: int = 0      # global index of this batch's first sequence
 
     @property
     def G(self) -> int:
@@ -128,6 +135,21 @@ def _gen(device, seed: int) -> torch.Generator:
     return g
 
 
+SEQ_SEED_STRIDE = 1000003
+
+
+def _seq_gen(w: Workload, kind: int, b: int, device) -> torch.Generator:
+    """Generator of draw ``kind`` for batch row b (global sequence
+    w.first_seq + b)."""
+    return _gen(device, 1000 * w.index + kind + SEQ_SEED_STRIDE * (w.first_seq + b))
+
+
+def shard(w: Workload, rank: int) -> Workload:
+    """Rank ``rank``'s batch under data parallelism: the B sequences starting
+    at global sequence rank*B (weak scaling: every rank holds B sequences)."""
+    return w.with_(first_seq=w.first_seq + rank * w.B)
+
+
 def outlier_channels(w: Workload) -> torch.Tensor:
     if w.outliers == 0:
         return torch.empty(0, dtype=torch.long)
@@ -151,32 +173,36 @@ def _fill_normal(out: torch.Tensor, gen: torch.Generator, rows_per_chunk: int,
 
 
 def keys(w: Workload, device="cpu", rows_per_chunk: int = 1 << 20):
-    """Keys [B, Hkv, T, d] in w.key_dtype."""
+    """Keys [B, Hkv, T, d] in w.key_dtype (each sequence from its own seed)."""
     K = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=w.key_dtype, device=device)
-    flat = K.view(-1, w.d)
-    row_scale = None
-    if w.lognormal_sigma > 0:
-        z = torch.randn(flat.shape[0], generator=_gen(device, 1000 * w.index + 4),
-                        device=device, dtype=torch.float32)
-        row_scale = torch.exp(w.lognormal_sigma * z)
-    _fill_normal(flat, _gen(device, 1000 * w.index + 0), rows_per_chunk,
-                 outlier_channels(w), row_scale)
+    cols = outlier_channels(w)
+    for b in range(w.B):
+        flat = K[b].view(-1, w.d)
+        row_scale = None
+        if w.lognormal_sigma > 0:
+            z = torch.randn(flat.shape[0], generator=_seq_gen(w, 4, b, device),
+                            device=device, dtype=torch.float32)
+            row_scale = torch.exp(w.lognormal_sigma * z)
+        _fill_normal(flat, _seq_gen(w, 0, b, device), rows_per_chunk, cols, row_scale)
     return K
 
 
 def values(w: Workload, device="cpu", rows_per_chunk: int = 1 << 20):
     """Values [B, Hkv, T, d] in bf16 (fp32 draws rounded to bf16)."""
     V = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.bfloat16, device=device)
-    _fill_normal(V.view(-1, w.d), _gen(device, 1000 * w.index + 1),
-                 rows_per_chunk, None)
+    for b in range(w.B):
+        _fill_normal(V[b].view(-1, w.d), _seq_gen(w, 1, b, device), rows_per_chunk, None)
     return V
 
 
 def queries(w: Workload, device="cpu", q_scale: float = 1.0):
     """One query token per (b, query head): [B, Hq, d] in w.key_dtype."""
-    Q = torch.randn((w.B, w.Hq, w.d), generator=_gen(device, 1000 * w.index + 2),
-                    device=device, dtype=torch.float32) * q_scale
-    return Q.to(w.key_dtype)
+    Q = torch.empty((w.B, w.Hq, w.d), dtype=w.key_dtype, device=device)
+    for b in range(w.B):
+        q = torch.randn((w.Hq, w.d), generator=_seq_gen(w, 2, b, device), device=device,
+                        dtype=torch.float32) * q_scale
+        Q[b].copy_(q)
+    return Q
 
 
 def random_keys(n: int, d: int, seed: int, dtype=torch.bfloat16, device="cpu",
@@ -191,16 +217,18 @@ def paged_layout(w: Workload, page_tokens: int = PAGE_TOKENS, spare_pages: int =
     """Sequence lengths and a shuffled block table for a paged cache.
 
     Lengths are uniform in [T/2, T-1) so that the appended key still fits the
-    bound T; sequence b owns ceil((len_b + 1) / page_tokens) pages, taken from
-    a seeded permutation of the pool.  Returns (lens int32 [B], block_table
-    int32 [B, max_pages] with -1 in unused entries, num_pages).
+    bound T (sequence g's length from its own seed); sequence b owns
+    ceil((len_b + 1) / page_tokens) pages, taken from a seeded permutation of
+    the pool.  Returns (lens int32 [B], block_table int32 [B, max_pages] with
+    -1 in unused entries, num_pages).
     """
-    g = _gen("cpu", 1000 * w.index + 5)
-    lens = torch.randint(w.T // 2, w.T - 1, (w.B,), generator=g, dtype=torch.int64)
+    lens = torch.cat([torch.randint(w.T // 2, w.T - 1, (1,), generator=_seq_gen(w, 5, b, "cpu"),
+                                    dtype=torch.int64) for b in range(w.B)])
     per_seq = [-(-(int(L) + 1) // page_tokens) for L in lens]
     max_pages = -(-w.T // page_tokens)
     num_pages = sum(per_seq) + spare_pages
-    perm = torch.randperm(num_pages, generator=_gen("cpu", 1000 * w.index + 6))
+    perm = torch.randperm(num_pages, generator=_gen("cpu", 1000 * w.index + 6 +
+                                                     SEQ_SEED_STRIDE * w.first_seq))
     table = torch.full((w.B, max_pages), -1, dtype=torch.int32)
     k = 0
     for b, n in enumerate(per_seq):
@@ -212,8 +240,10 @@ def paged_layout(w: Workload, page_tokens: int = PAGE_TOKENS, spare_pages: int =
 def new_tokens(w: Workload, device="cpu"):
     """The key and value each sequence appends in a decode step: [B, Hkv, d]
     each, drawn like the cache's keys (outlier channels included) and values."""
-    K = torch.empty((w.B * w.Hkv, w.d), dtype=w.key_dtype, device=device)
-    _fill_normal(K, _gen(device, 1000 * w.index + 7), 1 << 20, outlier_channels(w))
-    V = torch.empty((w.B * w.Hkv, w.d), dtype=torch.bfloat16, device=device)
-    _fill_normal(V, _gen(device, 1000 * w.index + 8), 1 << 20, None)
-    return K.view(w.B, w.Hkv, w.d), V.view(w.B, w.Hkv, w.d)
+    K = torch.empty((w.B, w.Hkv, w.d), dtype=w.key_dtype, device=device)
+    V = torch.empty((w.B, w.Hkv, w.d), dtype=torch.bfloat16, device=device)
+    cols = outlier_channels(w)
+    for b in range(w.B):
+        _fill_normal(K[b], _seq_gen(w, 7, b, device), 1 << 20, cols)
+        _fill_normal(V[b], _seq_gen(w, 8, b, device), 1 << 20, None)
+    return K, V
