@@ -55,7 +55,14 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_search_topk", "jl_turbo_codebook", "jl_turbo_rotation_workspace_bytes",
             "jl_turbo_rotation_init", "jl_turbo_quantize_keys", "jl_turbo_decode_workspace_bytes",
             "jl_turbo_decode_attention", "jl_turbo_decode_paged_workspace_bytes",
-            "jl_turbo_decode_attention_paged")
+            "jl_turbo_decode_attention_paged", "jl_test_drop_copies", "jl_build_flags")
+
+# device error codes (jl_device_error)
+JL_DERR_TC_WAIT_TIMEOUT = 1
+JL_DERR_DECODE_PLAN = 3
+JL_DERR_DECODE_WAIT_TIMEOUT = 4
+JL_DERR_INDEX = 5
+JL_BUILD_INDEX_CHECKS = 1
 
 _lib = None
 
@@ -129,6 +136,10 @@ def load():
                                                   i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
+    L.jl_build_flags.restype = i32
+    L.jl_build_flags.argtypes = []
+    L.jl_test_drop_copies.restype = i32
+    L.jl_test_drop_copies.argtypes = [i32, ctypes.c_uint64]
     L.jl_bf16_from_f64.restype = ctypes.c_uint16
     L.jl_bf16_from_f64.argtypes = [ctypes.c_double]
     _lib = L
@@ -439,6 +450,21 @@ def jl_device_error(stream=None) -> int:
     if st not in (JL_OK, JL_ERR_DEVICE):
         raise JLError(st, "jl_device_error")
     return int(code.value)
+
+
+def jl_test_drop_copies(enable: bool, wait_limit_ns: int = 0):
+    """Test hook: make the quantizer's and decode scorer's next launches start
+    no copy, with every wait bounded by ``wait_limit_ns`` (0 = default), so
+    that their bounded waits run out; ``jl_test_drop_copies(False)`` restores
+    normal operation.  See include/jlkey.h."""
+    _check(load().jl_test_drop_copies(1 if enable else 0, ctypes.c_uint64(wait_limit_ns)),
+           "jl_test_drop_copies")
+
+
+def jl_build_flags() -> int:
+    """JL_BUILD_* bits of the loaded library (JL_BUILD_INDEX_CHECKS for the
+    index-checking debug build)."""
+    return int(load().jl_build_flags())
 
 
 def jl_bf16_from_f64(x: float) -> int:

@@ -5,11 +5,20 @@
 #include "jl_common.cuh"
 #include "jl_internal.h"
 
+#include <atomic>
 #include <mutex>
 
 namespace jlk {
 
 __device__ int g_device_error = 0;
+
+namespace {
+std::atomic<int> g_drop_copies{0};
+std::atomic<unsigned long long> g_wait_limit_ns{WAIT_LIMIT_NS};
+}  // namespace
+
+bool test_drop_copies() { return g_drop_copies.load(std::memory_order_relaxed) != 0; }
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -455,6 +464,23 @@ int jl_turbo_decode_attention_paged(
   a.block_table = block_table; a.max_pages = max_pages; a.seq_lens = seq_lens;
   a.softmax_scale = softmax_scale; a.out = out; a.scores = scores; a.workspace = workspace;
   return from_cuda(jlk::launch_turbo_decode_paged(p, mse_bits, a, t, (cudaStream_t)stream));
+}
+
+int jl_test_drop_copies(int enable, uint64_t wait_limit_ns) {
+  if (enable != 0 && enable != 1) return JL_ERR_INVALID_ARG;
+  unsigned long long lim = wait_limit_ns ? (unsigned long long)wait_limit_ns : jlk::WAIT_LIMIT_NS;
+  if (lim < 1000ull || lim > jlk::WAIT_LIMIT_NS) return JL_ERR_INVALID_ARG;
+  jlk::g_wait_limit_ns.store(lim, std::memory_order_relaxed);
+  jlk::g_drop_copies.store(enable, std::memory_order_relaxed);
+  return JL_OK;
+}
+
+int jl_build_flags(void) {
+#ifdef JL_DEBUG_INDEX
+  return JL_BUILD_INDEX_CHECKS;
+#else
+  return 0;
+#endif
 }
 
 int jl_device_error(int *code, jl_stream_t stream) {

@@ -119,6 +119,8 @@ struct DecParams {
   const int32_t *seq_lens;  // [B]
   const int32_t *block_table;  // [B][max_pages]
   int max_pages, page_tokens, append, units, B, UH;
+  unsigned long long wait_ns;  // bound of every copy wait (WAIT_LIMIT_NS unless a test set one)
+  int drop_copies;             // test hook: the scorer issues no copy (its waits run out)
 };
 
 // Bulk-tensor maps of one decode call.  Values always go through `value`
@@ -163,10 +165,18 @@ __host__ __device__ __forceinline__ int warp_of_block(int64_t b, int64_t NB,
 constexpr int PROJ_THREADS = 256;
 constexpr int PROJ_VECS = 4;
 
+// Extents for the index checks of the debug build: X holds x_extent
+// elements, dst (from its start) dst_extent; err null = no checks.
+struct ProjLimits {
+  int *err = nullptr;
+  int64_t x_extent = 0, dst_extent = 0;
+};
+
 template <int M, int D, bool XF32>
 __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
                                          const void *__restrict__ X, int64_t x0,
-                                         int nx, float *dst, int dst_stride = M) {
+                                         int nx, float *dst, int dst_stride = M,
+                                         const ProjLimits lim = ProjLimits{}) {
   constexpr int CPL = D / 32;   // columns per lane
   constexpr int CH = 8;         // rows per chunk
   constexpr int RPW = M / 8;    // rows per warp
@@ -178,9 +188,11 @@ __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
       const int64_t e = (x0 + j) * D + lane * CPL + c;
-      x[j][c] = j >= nx ? 0.f
-                : XF32  ? reinterpret_cast<const float *>(X)[e]
-                        : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(X)[e]);
+      bool ok = j < nx;
+      if (ok && lim.err) ok = JL_IN_RANGE(lim.err, e, 1, lim.x_extent);
+      x[j][c] = !ok  ? 0.f
+                : XF32 ? reinterpret_cast<const float *>(X)[e]
+                       : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(X)[e]);
     }
 #pragma unroll
   for (int r0 = 0; r0 < RPW; r0 += CH) {
@@ -220,18 +232,21 @@ __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
       }
     }
     const int k = lane / PROJ_VECS, j = lane % PROJ_VECS;
-    if (j < nx) dst[(int64_t)j * dst_stride + warp + 8 * (r0 + k)] = v[0];
+    const int64_t di = (int64_t)j * dst_stride + warp + 8 * (r0 + k);
+    if (j < nx && (!lim.err || JL_IN_RANGE(lim.err, di, 1, lim.dst_extent))) dst[di] = v[0];
   }
 }
 
 template <int M, int D, bool QF32>
 __global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restrict__ Q,
                                                              const uint16_t *__restrict__ S,
-                                                             float *__restrict__ U, int nq) {
+                                                             float *__restrict__ U, int nq,
+                                                             int *err) {
   griddep_launch_dependents();  // let the scorer start its copies now
   const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
   const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
-  project4<M, D, QF32>(S, Q, x0, nx, U + x0 * M);
+  project4<M, D, QF32>(S, Q, x0, nx, U + x0 * M, M,
+                       ProjLimits{err, (int64_t)nq * D, ((int64_t)nq - x0) * M});
 }
 
 // TurboQuant-prod query rows, four queries per CTA: w = Pinv^T q (so that
@@ -251,7 +266,8 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
                                                  const float *__restrict__ Pinv,
                                                  const uint16_t *__restrict__ S,
                                                  float *__restrict__ U, int nq,
-                                                 const WalshCoef &wc, int64_t x0) {
+                                                 const WalshCoef &wc, int64_t x0,
+                                                 int *err) {
   constexpr int TERMS = TB == 3 ? 4 : TB;
   constexpr int MT = TERMS * D + M;
   constexpr int HALVES = PROJ_THREADS / D;  // threads per output coordinate
@@ -263,9 +279,9 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
   for (int e = threadIdx.x; e < PROJ_VECS * D; e += PROJ_THREADS) {
     const int j = e / D;
     const int64_t src = x0 * D + e;
-    qsm[e] = j >= nx ? 0.f
-             : QF32  ? reinterpret_cast<const float *>(Q)[src]
-                     : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[src]);
+    qsm[e] = (j >= nx || !JL_IN_RANGE(err, src, 1, (int64_t)nq * D)) ? 0.f
+             : QF32 ? reinterpret_cast<const float *>(Q)[src]
+                    : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(Q)[src]);
   }
   __syncthreads();
   {
@@ -295,12 +311,15 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
     wsm[e] = w;
   }
   __syncthreads();
-  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TERMS * D, MT);
+  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TERMS * D, MT,
+                       ProjLimits{err, PROJ_VECS * D, ((int64_t)nq - x0) * MT - TERMS * D});
   for (int e = threadIdx.x; e < nx * D; e += PROJ_THREADS) {
     const int j = e / D, i = e - (e / D) * D;
     float *row = U + (x0 + j) * MT;
 #pragma unroll
-    for (int k = 0; k < TERMS; ++k) row[k * D + i] = wc.c[k] * wsm[e];
+    for (int k = 0; k < TERMS; ++k)
+      if (JL_IN_RANGE(err, (x0 + j) * MT + k * D + i, 1, (int64_t)nq * MT))
+        row[k * D + i] = wc.c[k] * wsm[e];
   }
 }
 
@@ -308,9 +327,10 @@ template <int M, int D, int TB, bool QF32>
 __global__ void __launch_bounds__(PROJ_THREADS)
     turbo_qproj_kernel(const void *__restrict__ Q, const float *__restrict__ Pinv,
                        const uint16_t *__restrict__ S, float *__restrict__ U, int nq,
-                       const WalshCoef wc) {
+                       const WalshCoef wc, int *err) {
   griddep_launch_dependents();
-  turbo_query_rows<M, D, TB, QF32>(Q, Pinv, S, U, nq, wc, (int64_t)blockIdx.x * PROJ_VECS);
+  turbo_query_rows<M, D, TB, QF32>(Q, Pinv, S, U, nq, wc, (int64_t)blockIdx.x * PROJ_VECS,
+                                   err);
 }
 
 // ---------------------------------------------------------------------------
@@ -468,6 +488,7 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
                                             const Ring<M, D, S8, TB> &ring, const BlockPos &pos,
                                             int s, int lane) {
   using C = DecCfg<M, D, S8, TB>;
+  if (p.drop_copies) return;
   const int64_t kvi = pos.kvi;
   const int64_t key0 = pos.blk * DEC_KB;
   if (PAGED || maps.tma_codes) {
@@ -497,7 +518,9 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
   const uint32_t sdst = ring.sign(s);
 #pragma unroll
   for (int e = lane; e < C::SIGN_CHUNKS; e += 32) {
-    const bool ok = e * C::SIGN_CHUNK < nval * C::KEY_SIGN_BYTES;
+    const bool ok = e * C::SIGN_CHUNK < nval * C::KEY_SIGN_BYTES &&
+                    JL_IN_RANGE(p.err, gkey * C::KEY_SIGN_BYTES + e * C::SIGN_CHUNK,
+                                C::SIGN_CHUNK, p.n_keys * C::KEY_SIGN_BYTES);
     const void *src = ok ? (const void *)(sg + e * C::SIGN_CHUNK) : (const void *)p.signs;
     if constexpr (C::SIGN_CHUNK == 16)
       cp_async_16(sdst + e * 16, src, ok ? 16 : 0);
@@ -512,8 +535,10 @@ __device__ __forceinline__ void issue_block(const DecParams &p, const DecMaps &m
   if (lane < GROUPS) {
     const int64_t first = (gkey & ~(int64_t)(G - 1)) + G * lane;
     const int64_t avail = p.n_keys - first;
-    const bool ok = first < gkey + nval && avail > 0;
-    const int nbytes = ok ? (avail >= G ? 16 : (int)avail * C::NORM_BYTES) : 0;
+    bool ok = first < gkey + nval && avail > 0;
+    const int nbytes0 = ok ? (avail >= G ? 16 : (int)avail * C::NORM_BYTES) : 0;
+    if (ok) ok = JL_IN_RANGE(p.err, first * C::NORM_BYTES, nbytes0, p.n_keys * C::NORM_BYTES);
+    const int nbytes = ok ? nbytes0 : 0;
     const uint8_t *nb = reinterpret_cast<const uint8_t *>(p.norms);
     cp_async_16(ring.norm(s) + 16 * lane,
                 ok ? (const void *)(nb + first * C::NORM_BYTES) : (const void *)nb, nbytes);
@@ -858,7 +883,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   int usum[2] = {0, 0};
   float acc[C::DT][4];
   uint32_t afr[C::A_SMEM ? 1 : C::NC][4];
-  bool failed = false;
+  // a wait that ran out: bit 0 = it did; bits 1-2 = the block's index mod 4
+  // (its stage and phase); bit 3 = the next block was started too
+  int failed = 0;
 
   auto flush = [&](int64_t u) {
     float l = lsum;
@@ -916,13 +943,20 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       for (int dt = 0; dt < C::DT; ++dt)
         acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
       const float *urow = p.U + ((int64_t)b_idx * p.Hq + hq0 + g) * C::CODE_BITS;
-      build_afrags<M, D, S8, TB>(urow, g < Gg, t, ring, afr, hscale, usum);
+      const bool live =
+          g < Gg && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + g) * C::CODE_BITS,
+                                C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
+      build_afrags<M, D, S8, TB>(urow, live, t, ring, afr, hscale, usum);
       if constexpr (C::A_SMEM) __syncwarp();
     }
 
-    if (!mbar_wait_bounded(ring.bar(s), (uint32_t)((i / C::STAGES) & 1))) {
+    // the lanes wait converged, so they read the same barrier state and the
+    // same timer at the same instructions and agree on the outcome (the code
+    // below is warp-synchronous)
+    __syncwarp();
+    if (!mbar_wait_bounded(ring.bar(s), (uint32_t)((i / C::STAGES) & 1), p.wait_ns)) {
       record_device_error(p.err, DERR_DECODE_WAIT_TIMEOUT);
-      failed = true;
+      failed = 1 | ((int)(i & 3) << 1) | (i + 1 < nblk ? 8 : 0);
       break;
     }
     if constexpr (PAGED) {
@@ -1101,7 +1135,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           sval = (p.coef * nk) * raw[kg][j];
         }
         l2[kg][j] = sval * p.scale_log2;
-        if (p.scores != nullptr && key < nval && g < Gg)
+        if (p.scores != nullptr && key < nval && g < Gg &&
+            JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + g) * p.score_stride + key0 + key,
+                        1, (int64_t)p.B * p.Hq * p.score_stride))
           p.scores[((int64_t)b_idx * p.Hq + hq0 + g) * p.score_stride + key0 + key] = sval;
       }
     }
@@ -1169,12 +1205,16 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   }
   griddep_launch_dependents();
   if (failed) {
-    // let the copies already started land before the warp's smem goes away
-    for (int k = 0; k < C::STAGES; ++k) {
-      const unsigned long long t0 = globaltimer();
-      while (!mbar_try_wait(ring.bar(k), 0) && !mbar_try_wait(ring.bar(k), 1) &&
-             globaltimer() - t0 < WAIT_LIMIT_NS) {
-      }
+    // let the copies already started land before the warp's shared memory
+    // goes away: the ring (two stages) holds block i, whose wait ran out, and
+    // block i + 1 if it exists; block j sits in stage j % 2 and completes
+    // phase (j / 2) & 1 of its barrier
+    static_assert(C::STAGES == 2, "drain written for a two-stage ring");
+    if (!p.drop_copies) {
+      const int j = (failed >> 1) & 3;
+      mbar_wait_bounded(ring.bar(j & 1), (uint32_t)(j >> 1), p.wait_ns);
+      if (failed & 8)
+        mbar_wait_bounded(ring.bar((j + 1) & 1), (uint32_t)(((j + 1) >> 1) & 1), p.wait_ns);
     }
     return;
   }
@@ -1250,7 +1290,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
   griddep_wait();  // every partial state of the scorer is needed
   const int f = warp_of_block(first, NB, W);
   const int l = warp_of_block(last, NB, W);
-  const int n = min(l - f + 1, COMB_MAX_SLOTS);
+  int n = min(l - f + 1, COMB_MAX_SLOTS);
+  // the unit's records f + u .. f + u + n - 1 must lie in the workspace
+  if (!JL_IN_RANGE(p.err, (int64_t)f + u, n, p.slots)) n = 0;
   // records of unit u: warp w wrote record w + u (see the scorer's flush)
   const float *rec0 = partials + (size_t)((int64_t)f + u) * DEC_HPAD * (D + 2) +
                       (size_t)hh * (D + 2);
@@ -1288,7 +1330,8 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
 #pragma unroll
   for (int s = 0; s < 32; ++s) o = s < n ? fmaf(wts[s], v[s], o) : o;
   for (int s = 32; s < n; ++s) o = fmaf(wts[s], rec0[s * sstride + dim], o);
-  out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o * inv_l));
+  if (JL_IN_RANGE(p.err, (int64_t)bh * D + dim, 1, (int64_t)p.B * Hq * D))
+    out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o * inv_l));
 }
 
 // ---------------------------------------------------------------------------
@@ -1329,7 +1372,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
     // ---- query projections u = S q, four queries per CTA
     const int64_t x0 = (int64_t)bid * PROJ_VECS;
     const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)pp.nq - x0);
-    project4<M, D, QF32>(pp.S, pp.Q, x0, nx, pp.U + x0 * M);
+    project4<M, D, QF32>(pp.S, pp.Q, x0, nx, pp.U + x0 * M, M,
+                         ProjLimits{pp.err, (int64_t)pp.nq * D, ((int64_t)pp.nq - x0) * M});
     return;
   }
   const int nkv = pp.B * pp.Hkv;
@@ -1339,7 +1383,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
     // each at position seq_lens[b] of its sequence
     const int x0 = (bid - qctas) * PROJ_VECS;
     const int nx = min(PROJ_VECS, nkv - x0);
-    project4<M, D, KF32>(pp.S, pp.K_new, x0, nx, &ys[0][0]);
+    project4<M, D, KF32>(pp.S, pp.K_new, x0, nx, &ys[0][0], M,
+                         ProjLimits{pp.err, (int64_t)nkv * D, PROJ_VECS * M});
     __syncthreads();
     const int lane = i & 31, j = i >> 5;  // warp j stores key x0 + j
     if (j >= nx) return;
@@ -1354,6 +1399,7 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
       return;
     }
     const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
+    if (!JL_IN_RANGE(pp.err, slot, 1, (int64_t)pp.num_pages * pp.Hkv * pp.page_tokens)) return;
 #pragma unroll
     for (int w = 0; w < M / 32; ++w) {  // bit l of word w: coordinate 32w + l >= 0
       const uint32_t word = __ballot_sync(0xffffffffu, ys[j][w * 32 + lane] >= 0.f);
@@ -1408,7 +1454,7 @@ __global__ void __launch_bounds__(PROJ_THREADS) turbo_paged_prep_kernel(const Tu
   const int qctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS;
   if (bid < qctas) {
     turbo_query_rows<M, D, TB, QF32>(pp.Q, tp.Pinv, pp.S, pp.U, pp.nq, tp.wc,
-                                      (int64_t)bid * PROJ_VECS);
+                                      (int64_t)bid * PROJ_VECS, pp.err);
     return;
   }
   const int nkv = pp.B * pp.Hkv;
@@ -1416,7 +1462,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) turbo_paged_prep_kernel(const Tu
   if (!pp.append || x0 >= nkv) return;  // uniform over the CTA
   const int nx = min(PROJ_VECS, nkv - x0);
   const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;  // warp j: key x0 + j
-  project4<D, D, KF32>(tp.Pi, pp.K_new, x0, nx, &ys[0][0]);
+  project4<D, D, KF32>(tp.Pi, pp.K_new, x0, nx, &ys[0][0], D,
+                       ProjLimits{pp.err, (int64_t)nkv * D, PROJ_VECS * D});
   __syncthreads();
   uint32_t planes[TB][D / 32];
   float nk = 0.f, rn = 0.f;
@@ -1477,6 +1524,7 @@ __global__ void __launch_bounds__(PROJ_THREADS) turbo_paged_prep_kernel(const Tu
     return;
   }
   const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
+  if (!JL_IN_RANGE(pp.err, slot, 1, (int64_t)pp.num_pages * pp.Hkv * pp.page_tokens)) return;
   uint32_t *code = pp.sign_pages + slot * WORDS;
 #pragma unroll
   for (int w = 0; w < M / 32; ++w) {
@@ -1627,6 +1675,8 @@ static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *par
   p.units = pl.units;
   p.B = pl.B;
   p.UH = pl.Hkv * pl.HG;
+  p.wait_ns = wait_limit_ns();
+  p.drop_copies = 0;
 }
 
 // Launch the scorer (one wave, <= the plan's warp bound) and the combine.
@@ -1671,13 +1721,14 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   const int bh = pl.B * pl.Hq;
   const int qctas = (bh + PROJ_VECS - 1) / PROJ_VECS;
   if (q_f32)
-    qproj_kernel<M, D, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh);
+    qproj_kernel<M, D, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh, err);
   else
-    qproj_kernel<M, D, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh);
+    qproj_kernel<M, D, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, signs, norms, scores, softmax_scale, M, err);
+  p.drop_copies = test_drop_copies() ? 1 : 0;
   return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
 }
 
@@ -1717,9 +1768,11 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
   WalshCoef wc;
   for (int k = 0; k < 4; ++k) wc.c[k] = (float)walsh[k];
   if (q_f32)
-    turbo_qproj_kernel<M, D, TB, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc);
+    turbo_qproj_kernel<M, D, TB, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc,
+                                                                            err);
   else
-    turbo_qproj_kernel<M, D, TB, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc);
+    turbo_qproj_kernel<M, D, TB, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, Pinv, S, U, bh, wc,
+                                                                             err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecParams p;
@@ -1748,13 +1801,15 @@ cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S
                                     int nq, int m, int d, cudaStream_t stream) {
   if (nq <= 0) return cudaSuccess;
   const int ctas = (nq + PROJ_VECS - 1) / PROJ_VECS;
-#define JL_CASE(MM, DD)                                                              \
-  if (m == MM && d == DD) {                                                          \
-    if (q_f32)                                                                       \
-      qproj_kernel<MM, DD, true><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq);    \
-    else                                                                             \
-      qproj_kernel<MM, DD, false><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq);   \
-    return cudaGetLastError();                                                       \
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
+#define JL_CASE(MM, DD)                                                                \
+  if (m == MM && d == DD) {                                                            \
+    if (q_f32)                                                                         \
+      qproj_kernel<MM, DD, true><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err);  \
+    else                                                                               \
+      qproj_kernel<MM, DD, false><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err); \
+    return cudaGetLastError();                                                         \
   }
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)

@@ -233,22 +233,6 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k, int rows) {
   return (uint32_t)(kc * rows * 128 + r * 128 + ((((kin >> 3) ^ (r & 7)) << 4)) + (kin & 7) * 2);
 }
 
-// --------------------------------------------------------------------------
-// Start copying code row `row` (M/8 bytes) into shared memory at dst with
-// cp.async (zero fill when the row is past the end), as one commit group.
-template <int M>
-__device__ __forceinline__ void copy_code_row(uint32_t dst, const uint32_t *signs, int64_t row,
-                                              bool live) {
-  const uint8_t *src = reinterpret_cast<const uint8_t *>(signs + (live ? row : 0) * (M / 32));
-  if constexpr (M >= 128) {
-#pragma unroll
-    for (int q = 0; q < M / 128; ++q) cp_async_16(dst + 16 * q, src + 16 * q, live ? 16 : 0);
-  } else {
-    cp_async_8(dst, src, live ? 8 : 0);
-  }
-  cp_async_commit();
-}
-
 template <int M, int D>
 __global__ void __launch_bounds__(THREADS, 1)
     dequant_tc_kernel(const __grid_constant__ CUtensorMap tmap_out, const Params p) {
@@ -331,7 +315,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t crow = base + C::OFF_C + r * C::CODE_ROW + pt * pbytes;
     auto code_slot = [&](int64_t it) { return crow + (uint32_t)((it % CODE_SLOTS) * BM * C::CODE_ROW); };
     auto copy_part = [&](uint32_t dst, int64_t row) {
-      const bool live = row < p.n;
+      const bool live = row < p.n && JL_IN_RANGE(p.err, row * (M / 8) + pt * pbytes, KP * 8,
+                                                 p.n * (M / 8));
       const uint8_t *src = reinterpret_cast<const uint8_t *>(p.signs + (live ? row : 0) * (M / 32)) +
                            pt * pbytes;
       if constexpr (KP * 8 >= 16) {
@@ -395,7 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int a = (int)(t & 1);
       const uint32_t aph = (uint32_t)((t >> 1) & 1);
       const int64_t row = tile * BM + 32 * q + lane;
-      const bool live = row < p.n;
+      const bool live = row < p.n && JL_IN_RANGE(p.err, row, 1, p.n);
       const float f = live ? p.coef * __half2float(__ushort_as_half(__ldg(p.norms + row))) : 0.f;
       const int ob = (int)(t % C::OBUF);
       uint8_t *stage = gbase + C::OFF_O + (ew * C::OBUF + ob) * C::OWARP;

@@ -26,18 +26,48 @@ unsigned long long current_context_id();
 
 enum DeviceErr : int {
   DERR_NONE = 0,
-  DERR_TC_WAIT_TIMEOUT = 1,     // tensor-core quantizer: a pipeline wait ran out
-  DERR_TC_TMEM_ALLOC = 2,       // tensor-core quantizer: TMEM allocation failed
-  DERR_DECODE_PLAN = 3,         // decode: inconsistent work split
-  DERR_DECODE_WAIT_TIMEOUT = 4, // decode: a copy wait ran out
+  DERR_TC_WAIT_TIMEOUT = JL_DERR_TC_WAIT_TIMEOUT,  // tensor-core kernel: a pipeline wait ran out
+  DERR_TC_TMEM_ALLOC = 2,                          // tensor-core kernel: TMEM allocation failed
+  DERR_DECODE_PLAN = JL_DERR_DECODE_PLAN,          // decode: inconsistent work split
+  DERR_DECODE_WAIT_TIMEOUT = JL_DERR_DECODE_WAIT_TIMEOUT,  // decode: a copy wait ran out
+  DERR_INDEX = JL_DERR_INDEX,   // debug builds: an index left its buffer's extent
 };
 
 // Upper bound of every spin-wait in the library's kernels (GPU time).
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
 
+// Test hook set by jl_test_drop_copies (host side, api.cu): when on, the
+// tensor-core quantizer and the contiguous decode scorer launch without
+// issuing any copy, so their consumers' waits run out after
+// wait_limit_ns(); the kernels must then record the timeout, drain, free
+// tensor memory and return.  Off (the default) changes nothing.
+bool test_drop_copies();
+unsigned long long wait_limit_ns();
+
 __device__ __forceinline__ void record_device_error(int *err, int code) {
   atomicCAS(err, 0, code);
 }
+
+// Index checks of the debug build (compiled with -DJL_DEBUG_INDEX, which
+// `python -m bit_jl_key_b200.build --debug-index` does into
+// libjlkey_debug.so).  JL_IN_RANGE(err, first, count, extent) is true when
+// the elements [first, first + count) lie inside a buffer of `extent`
+// elements, the extent the call's shapes give that buffer; otherwise the
+// debug build records DERR_INDEX in the device error word and the caller
+// skips the access.  In the normal build it is the constant true and costs
+// nothing.
+#ifdef JL_DEBUG_INDEX
+__device__ __forceinline__ bool index_in_range(int *err, int64_t first, int64_t count,
+                                               int64_t extent) {
+  if (first >= 0 && count >= 0 && first + count <= extent) return true;
+  record_device_error(err, DERR_INDEX);
+  return false;
+}
+#define JL_IN_RANGE(err, first, count, extent)                                   \
+  ::jlk::index_in_range((err), (int64_t)(first), (int64_t)(count), (int64_t)(extent))
+#else
+#define JL_IN_RANGE(err, first, count, extent) true
+#endif
 
 // Number of SMs of the current device (cached per device, thread-safe).
 int device_sm_count();
@@ -162,14 +192,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
   return t;
 }
-// Wait for phase `parity` of `bar` for at most WAIT_LIMIT_NS; false if the
-// wait ran out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Wait for phase `parity` of `bar` for at most limit_ns of GPU time; false if
+// the wait ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+    if ((it & 63u) == 0 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map,

@@ -111,16 +111,19 @@ __device__ __forceinline__ uint32_t sign_word(const uint32_t (&v)[32]) {
 }
 
 // Bounded wait on a barrier phase; false when it ran out (the error word is
-// set and the shared abort flag raised) or another role gave up.
+// set and the shared abort flag raised) or another role gave up.  The bound
+// is limit_ns of GPU time (the library's default unless a launch was given a
+// shorter one).
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
-                                           volatile int *abort_flag, int *err) {
+                                           volatile int *abort_flag, int *err,
+                                           unsigned long long limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         record_device_error(err, DERR_TC_WAIT_TIMEOUT);
         return false;
@@ -129,9 +132,10 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
   }
 }
 // Bounded wait used while draining (no abort check): gives up silently.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
+                                           unsigned long long limit_ns = WAIT_LIMIT_NS) {
   const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < WAIT_LIMIT_NS) {
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < limit_ns) {
   }
 }
 

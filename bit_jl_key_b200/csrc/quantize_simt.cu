@@ -27,14 +27,16 @@ __global__ void __launch_bounds__(QS_WARPS * 32)
     quantize_simt_kernel(const void *__restrict__ K, int64_t n, int64_t ldk,
                          const uint16_t *__restrict__ S,
                          uint32_t *__restrict__ signs,
-                         uint16_t *__restrict__ norms) {
+                         uint16_t *__restrict__ norms, int *err) {
+  // extents the shapes give the buffers (debug index checks)
+  const int64_t k_extent = (n - 1) * ldk + D, s_extent = (int64_t)M * D;
   extern __shared__ __align__(16) uint8_t qsmem[];
   uint16_t *St = reinterpret_cast<uint16_t *>(qsmem);  // [D][M]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   float *kbuf = reinterpret_cast<float *>(qsmem + M * D * 2) + wid * D;
   for (int e = threadIdx.x; e < M * D; e += blockDim.x) {
     const int i = e / D, j = e - i * D;
-    St[j * M + i] = S[e];
+    St[j * M + i] = JL_IN_RANGE(err, e, 1, s_extent) ? S[e] : (uint16_t)0;
   }
   __syncthreads();
   constexpr int WORDS = M / 32;
@@ -42,9 +44,11 @@ __global__ void __launch_bounds__(QS_WARPS * 32)
        key += (int64_t)gridDim.x * QS_WARPS) {
     float ss = 0.f;
     for (int j = lane; j < D; j += 32) {
+      const int64_t ki = key * ldk + j;
       const float v =
-          F32 ? reinterpret_cast<const float *>(K)[key * ldk + j]
-              : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(K)[key * ldk + j]);
+          !JL_IN_RANGE(err, ki, 1, k_extent) ? 0.f
+          : F32 ? reinterpret_cast<const float *>(K)[ki]
+                : bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(K)[ki]);
       kbuf[j] = v;
       ss = fmaf(v, v, ss);
     }
@@ -62,11 +66,13 @@ __global__ void __launch_bounds__(QS_WARPS * 32)
 #pragma unroll
     for (int w = 0; w < WORDS; ++w) {
       const uint32_t word = __ballot_sync(0xffffffffu, acc[w] >= 0.f);
-      if (lane == w) signs[key * WORDS + w] = word;
+      if (lane == w && JL_IN_RANGE(err, key * WORDS + w, 1, n * WORDS))
+        signs[key * WORDS + w] = word;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) norms[key] = __half_as_ushort(__float2half_rn(sqrtf(ss)));
+    if (lane == 0 && JL_IN_RANGE(err, key, 1, n))
+      norms[key] = __half_as_ushort(__float2half_rn(sqrtf(ss)));
     __syncwarp();
   }
 }
@@ -83,7 +89,9 @@ static cudaError_t launch_qs(const void *K, bool f32, int64_t n, int64_t ldk,
   int64_t blocks = (n + QS_WARPS - 1) / QS_WARPS;
   const int64_t cap = (int64_t)device_sm_count() * 8;
   if (blocks > cap) blocks = cap;
-  kern<<<(int)blocks, QS_WARPS * 32, smem, stream>>>(K, n, ldk, S, signs, norms);
+  int *err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  kern<<<(int)blocks, QS_WARPS * 32, smem, stream>>>(K, n, ldk, S, signs, norms, err);
   return cudaGetLastError();
 }
 

@@ -30,6 +30,7 @@
 // roles to stop, and the CTA still drains its copies and frees its TMEM.
 #include "jl_common.cuh"
 #include "jl_internal.h"
+#include "jl_tc.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -45,7 +46,6 @@ constexpr int BM = 128;           // keys per tile (MMA M)
 #define JL_QTC_SIGN_WARPS 0
 #endif
 constexpr int SMEM_BUDGET = 220 * 1024;
-constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
 
 template <int M, int D>
 struct Cfg {
@@ -85,103 +85,11 @@ struct Params {
   uint32_t *signs;
   uint16_t *norms;
   int *err;
+  unsigned long long wait_ns;  // bound of every wait (WAIT_LIMIT_NS unless a test set one)
+  int drop_copies;             // test hook: issue no copy (every wait then runs out)
 };
 
-// --------------------------------------------------------------------------
-// PTX wrappers
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-// K-major operand, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);          // start address
-  d |= (uint64_t)1u << 16;                          // leading byte offset (unused)
-  d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset
-  d |= (uint64_t)1u << 46;                          // descriptor version
-  d |= (uint64_t)2u << 61;                          // SWIZZLE_128B
-  return d;
-}
-__device__ __forceinline__ void mma_bf16_ss(uint32_t tmem_d, uint64_t adesc,
-                                            uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-        "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
-        "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
-// The same wait, tied to the registers of one load: code that reads v after
-// it cannot be moved above it.
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
-                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
-                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
-                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
-               :
-               : "memory");
-}
-// Code word of 32 accumulator columns: bit j = 1 iff column j is >= 0
-// (sign bit clear).  One funnel shift per column moves its sign bit in; four
-// independent chains of 8 (one per byte) keep the dependency chain short.
-__device__ __forceinline__ uint32_t pack_signs(const uint32_t (&v)[32]) {
-  uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-#pragma unroll
-  for (int jj = 7; jj >= 0; --jj) {
-    c0 = __funnelshift_l(v[jj], c0, 1);
-    c1 = __funnelshift_l(v[8 + jj], c1, 1);
-    c2 = __funnelshift_l(v[16 + jj], c2, 1);
-    c3 = __funnelshift_l(v[24 + jj], c3, 1);
-  }
-  return ~(c0 | (c1 << 8) | (c2 << 16) | (c3 << 24));
-}
-
-// Bounded wait on a barrier phase; false when the wait ran out or another
-// role gave up (then the error word is set and the shared abort flag raised).
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
-                                           volatile int *abort_flag, int *err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > WAIT_NS) {
-        *abort_flag = 1;
-        record_device_error(err, DERR_TC_WAIT_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
+using namespace tcx;
 
 // --------------------------------------------------------------------------
 template <int M, int D>
@@ -232,15 +140,15 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
         "n"(C::TMEM_COLS)
         : "memory");
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
   const int64_t ntiles = p.num_tiles;
   if (warp == 0) {
     // ---------------- TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !p.drop_copies) {
       mbar_expect_tx(sfull_bar, C::S_BYTES);
       for (int kc = 0; kc < C::KCH; ++kc)
         for (int h = 0; h < C::NH; ++h)
@@ -250,7 +158,7 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
       for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
         const int s = (int)(i % C::STAGES);
         const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
-        if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.err)) break;
+        if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.err, p.wait_ns)) break;
         mbar_expect_tx(full_bar(s), C::A_STAGE);
         for (int kc = 0; kc < C::KCH; ++kc)
           tma_load_2d(sA + s * C::A_STAGE + kc * C::A_CHUNK, &tmap_k, kc * 64,
@@ -262,12 +170,12 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
         const int s = (int)(j % C::STAGES);
         const uint32_t ph = (uint32_t)((j / C::STAGES) & 1);
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(full_bar(s), ph) && globaltimer() - t0 < WAIT_NS) {
+        while (!mbar_try_wait(full_bar(s), ph) && globaltimer() - t0 < p.wait_ns) {
         }
       }
       {
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(sfull_bar, 0) && globaltimer() - t0 < WAIT_NS) {
+        while (!mbar_try_wait(sfull_bar, 0) && globaltimer() - t0 < p.wait_ns) {
         }
       }
     }
@@ -278,40 +186,40 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
                                  | (1u << 7) | (1u << 10)  // A, B: bf16
                                  | ((uint32_t)(C::NMMA >> 3) << 17)  // N
                                  | ((uint32_t)(BM >> 4) << 24);      // M
-      bool ok = wait_phase(sfull_bar, 0, abort_flag, p.err);
+      bool ok = wait_phase(sfull_bar, 0, abort_flag, p.err, p.wait_ns);
       int64_t i = 0, j = 0;  // tiles and items (tile x N-half) issued
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
         const int s = (int)(i % C::STAGES);
         const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
-        if (!wait_phase(full_bar(s), ph, abort_flag, p.err)) break;
+        if (!wait_phase(full_bar(s), ph, abort_flag, p.err, p.wait_ns)) break;
         for (int h = 0; h < C::NH; ++h, ++j) {
           const int a = (int)(j & 1);
           const uint32_t aph = (uint32_t)((j >> 1) & 1);
-          if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err)) {
+          if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
-          tc_fence_after();
+          fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t koff = (uint32_t)(kk & 3) * 32u;
             const uint64_t adesc =
-                smem_desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
+                desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
             const uint64_t bdesc =
-                smem_desc_sw128(sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
-            mma_bf16_ss(tmem_base + a * C::NMMA, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                desc_sw128(sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
+            mma_ss(tmem_base + a * C::NMMA, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
           }
-          mma_commit(tfull_bar(a));
+          commit(tfull_bar(a));
         }
         if (!ok) break;
-        mma_commit(empty_bar(s));
+        commit(empty_bar(s));
       }
       // drain: the last accumulator's MMAs must be complete before TMEM is freed
       if (j > 0) {
         const int64_t jl = j - 1;
         const unsigned long long t0 = globaltimer();
         while (!mbar_try_wait(tfull_bar((int)(jl & 1)), (uint32_t)((jl >> 1) & 1)) &&
-               globaltimer() - t0 < WAIT_NS) {
+               globaltimer() - t0 < p.wait_ns) {
         }
       }
     }
@@ -331,12 +239,12 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
       for (int h = 0; h < C::NH; ++h, ++j) {
         const int a = (int)(j & 1);
         const uint32_t aph = (uint32_t)((j >> 1) & 1);
-        if (!wait_phase(tfull_bar(a), aph, abort_flag, p.err)) {
+        // the lanes decide together (the tensor-memory loads are warp-wide)
+        if (!__all_sync(0xffffffffu, wait_phase(tfull_bar(a), aph, abort_flag, p.err, p.wait_ns))) {
           ok = false;
           break;
         }
-        __syncwarp();
-        tc_fence_after();
+        fence_after();
         const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * C::NMMA);
         uint32_t *dst = p.signs + row * C::WORDS + h * C::WORDS_ITEM + k * WPW;
         // this warp's WPW code words; the TMEM loads are double-buffered so
@@ -344,19 +252,20 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
         uint32_t words[WPW];
         uint32_t va[32], vb[32];
         const uint32_t tcol = trow + 32 * (k * WPW);
-        tmem_ld32(tcol, va);
+        ld32(tcol, va);
 #pragma unroll
         for (int w = 0; w < WPW; w += 2) {
-          tmem_ld_wait(va);
-          if (w + 1 < WPW) tmem_ld32(tcol + 32 * (w + 1), vb);
-          words[w] = pack_signs(va);
+          ld_wait(va);
+          if (w + 1 < WPW) ld32(tcol + 32 * (w + 1), vb);
+          words[w] = sign_word(va);
           if (w + 1 < WPW) {
-            tmem_ld_wait(vb);
-            if (w + 2 < WPW) tmem_ld32(tcol + 32 * (w + 2), va);
-            words[w + 1] = pack_signs(vb);
+            ld_wait(vb);
+            if (w + 2 < WPW) ld32(tcol + 32 * (w + 2), va);
+            words[w + 1] = sign_word(vb);
           }
         }
-        if (live) {
+        if (live && JL_IN_RANGE(p.err, row * C::WORDS + h * C::WORDS_ITEM + k * WPW, WPW,
+                                p.n * C::WORDS)) {
 #pragma unroll
           for (int w = 0; w < WPW; w += GW) {
             if constexpr (GW == 1)
@@ -368,7 +277,7 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
                   make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
           }
         }
-        tc_fence_before();
+        fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty_bar(a));
       }
@@ -380,7 +289,8 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = (int)(i % C::STAGES);
       const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
-      if (!wait_phase(full_bar(s), ph, abort_flag, p.err)) break;
+      if (!__all_sync(0xffffffffu, wait_phase(full_bar(s), ph, abort_flag, p.err, p.wait_ns)))
+        break;
       float ss0 = 0.f, ss1 = 0.f;
       const uint8_t *rowp = gbase + C::OFF_A + s * C::A_STAGE + r * 128;
 #pragma unroll
@@ -397,14 +307,15 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
       const int64_t row = tile * BM + r;
-      if (row < p.n) p.norms[row] = __half_as_ushort(__float2half_rn(sqrtf(ss0 + ss1)));
+      if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n))
+        p.norms[row] = __half_as_ushort(__float2half_rn(sqrtf(ss0 + ss1)));
     }
   }
 
-  tc_fence_before();
+  fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
+    fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
                  "n"(C::TMEM_COLS)
                  : "memory");
@@ -442,7 +353,8 @@ cudaError_t launch_t(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *
   if (!make_map(&ms, S, M, D, D, (uint32_t)C::NMMA)) return cudaErrorInvalidValue;
   int *err = device_error_ptr();
   if (!err) return cudaErrorInvalidSymbol;
-  Params p{n, (n + BM - 1) / BM, signs, norms, err};
+  Params p{n, (n + BM - 1) / BM, signs, norms, err, wait_limit_ns(),
+           test_drop_copies() ? 1 : 0};
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<M, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

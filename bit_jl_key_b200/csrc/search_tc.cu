@@ -217,11 +217,11 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
 // with cp.async, zero fill past the end, as one commit group.
 template <int M>
 __device__ __forceinline__ void copy_code_rows(uint32_t dst0, uint32_t dst1, const uint32_t *signs,
-                                               int64_t row0, int64_t N) {
+                                               int64_t row0, int64_t N, int *err) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int64_t row = row0 + 128 * h;
-    const bool live = row < N;
+    const bool live = row < N && JL_IN_RANGE(err, row * (M / 8), M / 8, N * (M / 8));
     const uint32_t dst = h ? dst1 : dst0;
     const uint8_t *src = reinterpret_cast<const uint8_t *>(signs + (live ? row : 0) * (M / 32));
     if constexpr (M >= 128) {
@@ -423,13 +423,14 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
     auto slot0 = [&](int64_t it) { return crow0 + (uint32_t)((it % CODE_SLOTS) * BN * C::CODE_ROW); };
     for (int k = 0; k < CODE_SLOTS - 1; ++k) {
       const int64_t row0 = tile_at((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BN + t;
-      copy_code_rows<M>(slot0(k), slot0(k) + 128 * C::CODE_ROW, p.signs, row0, p.N);
+      copy_code_rows<M>(slot0(k), slot0(k) + 128 * C::CODE_ROW, p.signs, row0, p.N, p.err);
     }
     int64_t c = 0, it = 0;
     bool ok = true;
     // the two rows' norms (0 past the end), one tile ahead: B holds +-||x||
     auto norm_of = [&](int64_t row) -> uint32_t {
-      return row < p.N ? (uint32_t)__ldg(p.norms + row) & 0x7FFFu : 0u;
+      return (row < p.N && JL_IN_RANGE(p.err, row, 1, p.N))
+                 ? (uint32_t)__ldg(p.norms + row) & 0x7FFFu : 0u;
     };
     uint32_t n0 = norm_of(tile_at(blockIdx.x) * BN + t), n1 = norm_of(tile_at(blockIdx.x) * BN + t + 128);
     for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++it) {
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       {
         const int64_t row0 = tile_at(j + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BN + t;
         const uint32_t d0 = slot0(it + CODE_SLOTS - 1);
-        copy_code_rows<M>(d0, d0 + 128 * C::CODE_ROW, p.signs, row0, p.N);
+        copy_code_rows<M>(d0, d0 + 128 * C::CODE_ROW, p.signs, row0, p.N, p.err);
       }
       const uint32_t x0 = 0x80008000u | (n0 << 16) | n0;
       const uint32_t x1 = 0x80008000u | (n1 << 16) | n1;

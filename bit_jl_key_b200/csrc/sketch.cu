@@ -17,10 +17,10 @@
 namespace jlk {
 
 __global__ void sketch_kernel(uint16_t *__restrict__ S, int64_t total,
-                              uint64_t seed) {
+                              uint64_t seed, int *err) {
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
-    S[e] = bf16_from_f64_bits(gauss_at(seed, (uint64_t)e));
+    if (JL_IN_RANGE(err, e, 1, total)) S[e] = bf16_from_f64_bits(gauss_at(seed, (uint64_t)e));
   }
 }
 
@@ -29,7 +29,9 @@ cudaError_t launch_sketch(uint16_t *S, int m, int d, uint64_t seed,
   const int64_t total = (int64_t)m * d;
   const int threads = 256;
   const int blocks = (int)((total + threads - 1) / threads);
-  sketch_kernel<<<blocks, threads, 0, stream>>>(S, total, seed);
+  int *err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  sketch_kernel<<<blocks, threads, 0, stream>>>(S, total, seed, err);
   return cudaGetLastError();
 }
 

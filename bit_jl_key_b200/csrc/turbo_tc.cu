@@ -644,7 +644,8 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         chunk(va, 2 * half);
         tcx::ld_wait(vb);
         chunk(vb, 2 * half + 1);
-        if (row < p.n) {
+        if (row < p.n &&
+            JL_IN_RANGE(p.err, row * C::WORDS + 2 * half, (TB - 1) * C::PW + 2, p.n * C::WORDS)) {
 #pragma unroll
           for (int pp = 0; pp < TB; ++pp)
             *reinterpret_cast<uint2 *>(dst + pp * C::PW + 2 * half) =
@@ -655,7 +656,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       tcx::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(afull(h));
-      if (row < p.n) {
+      if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n)) {
         const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
         const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
         p.norms[row] = n16 | (r16 << 16);
@@ -673,7 +674,8 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
         const uint32_t w0 = tcx::sign_word(va);
         tcx::ld_wait(vb);
         const uint32_t w1 = tcx::sign_word(vb);
-        if (row < p.n)
+        if (row < p.n &&
+            JL_IN_RANGE(p.err, row * C::WORDS + TB * C::PW + 2 * half, 2, p.n * C::WORDS))
           *reinterpret_cast<uint2 *>(dst + TB * C::PW + 2 * half) = make_uint2(w0, w1);
       }
       tcx::fence_before();

@@ -41,7 +41,7 @@
  *  - Supported shapes: d in {64, 128}; m in {64, 128, 256, 512}.
  *  - Thread safety: entry points may be called concurrently from several host
  *    threads; the only process-wide state is a per-device cache of device
- *    attributes.
+ *    attributes and addresses, and the test hook of jl_test_drop_copies.
  */
 #ifndef JLKEY_H
 #define JLKEY_H
@@ -476,9 +476,47 @@ JL_API int jl_turbo_decode_attention_paged(
  * jl_device_error -- synchronise `stream`, then read and clear the device
  * error word of the current device (0 = no fault reported).  *code receives
  * the word.  Returns JL_OK, JL_ERR_DEVICE when the word was non-zero, or
- * JL_ERR_CUDA.
+ * JL_ERR_CUDA.  Codes: JL_DERR_TC_WAIT_TIMEOUT (a tensor-core kernel's
+ * pipeline wait ran out), JL_DERR_DECODE_PLAN (a decode work split or a
+ * paged length did not fit), JL_DERR_DECODE_WAIT_TIMEOUT (a decode copy wait
+ * ran out), JL_DERR_INDEX (see below).
  */
+enum {
+    JL_DERR_TC_WAIT_TIMEOUT = 1,
+    JL_DERR_DECODE_PLAN = 3,
+    JL_DERR_DECODE_WAIT_TIMEOUT = 4,
+    JL_DERR_INDEX = 5 /* index-checking debug build only: a kernel computed an
+                         index outside the extent the call's shapes give a
+                         buffer, and skipped that access */
+};
 JL_API int jl_device_error(int *code, jl_stream_t stream);
+
+/*
+ * jl_test_drop_copies -- failure detection test hook (not part of the
+ * method; for tests only).  Every wait inside the library's kernels is
+ * bounded; when one runs out the kernel records a code in the device error
+ * word, lets the copies it started land, frees its tensor memory and returns,
+ * leaving the context usable.  To exercise that path without any GPU fault,
+ * enable = 1 makes the launches that follow of the tensor-core quantizer
+ * (jl_quantize_keys, bf16 keys) and of the contiguous decode scorer
+ * (jl_decode_attention, jl_decode_attention_noalloc) start no copy at all,
+ * so their waits run out; their outputs are then undefined.  wait_limit_ns
+ * (1e3 .. 2e9, 0 = the default 2e9) bounds, in GPU time, every wait of those
+ * two kernels launched after the call.  enable = 0 with wait_limit_ns = 0
+ * restores normal operation.  Process-wide; calls made while it is on from
+ * other threads are affected too.  Returns JL_OK or JL_ERR_INVALID_ARG.
+ */
+JL_API int jl_test_drop_copies(int enable, uint64_t wait_limit_ns);
+
+/*
+ * jl_build_flags -- how this copy of the library was built (not part of the
+ * method): a bit set of JL_BUILD_* flags.  JL_BUILD_INDEX_CHECKS: the
+ * index-checking debug build, whose kernels check every global access they
+ * make through a raw pointer against the extent the call's shapes give that
+ * buffer, skip one that falls outside and report JL_DERR_INDEX.
+ */
+enum { JL_BUILD_INDEX_CHECKS = 1 };
+JL_API int jl_build_flags(void);
 
 /*
  * jl_bf16_from_f64 -- host helper: the bf16 code (round to nearest, ties to

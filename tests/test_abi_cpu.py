@@ -202,6 +202,17 @@ def test_decode_wrappers_check_shapes_and_dtypes(lib, fn):
         call(Q, S, signs, norms, V)
 
 
+def test_drop_copies_hook_arguments(lib):
+    f = lib.jl_test_drop_copies
+    assert f(0, 0) == jl.JL_OK
+    assert f(1, 1_000_000) == jl.JL_OK
+    assert f(1, 0) == jl.JL_OK                 # default bound
+    assert f(2, 0) == jl.JL_ERR_INVALID_ARG
+    assert f(1, 999) == jl.JL_ERR_INVALID_ARG   # below 1 us
+    assert f(1, 2_000_000_001) == jl.JL_ERR_INVALID_ARG
+    assert f(0, 0) == jl.JL_OK                 # left off for the other tests
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(ValueError):
