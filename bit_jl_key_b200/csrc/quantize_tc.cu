@@ -14,10 +14,10 @@
 // One persistent CTA per SM, 10 warps with fixed roles:
 //   warp 0     TMA producer: S once, then one 128 x d key tile per stage of
 //              a STAGES-deep shared-memory ring.
-//   warp 1     owns the TMEM allocation; lane 0 issues the MMAs of a tile
-//              into one of two TMEM accumulators (one for m = 512) and
-//              commits them to the barriers that free the key stage and
-//              publish the accumulator.
+//   warp 1     owns the TMEM allocation; one elected lane issues the MMAs
+//              of each work item (a tile, or half of one at m = 512) into one
+//              of two TMEM accumulators and commits them to the barriers that
+//              free the key stage and publish the accumulator.
 //   warps 2-5  sign epilogue: warp w reads TMEM lanes 32*(w%4).. (its lane
 //              quadrant), 32 columns per tcgen05.ld, and packs the 32 sign
 //              bits of a word with one funnel shift per value; then releases
@@ -155,14 +155,18 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
           tma_load_2d(sS + kc * C::S_CHUNK + h * C::NMMA * 128, &tmap_s, kc * 64,
                       h * C::NMMA, sfull_bar);
       int64_t i = 0;
+      int s = 0;          // stage of tile i and the phase it completes next
+      uint32_t ph = 0;
       for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-        const int s = (int)(i % C::STAGES);
-        const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
         if (!wait_phase(empty_bar(s), ph ^ 1u, abort_flag, p.err, p.wait_ns)) break;
         mbar_expect_tx(full_bar(s), C::A_STAGE);
         for (int kc = 0; kc < C::KCH; ++kc)
           tma_load_2d(sA + s * C::A_STAGE + kc * C::A_CHUNK, &tmap_k, kc * 64,
                       (int)(tile * BM), full_bar(s));
+        if (++s == C::STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       // drain: the last stages issued must have landed before the CTA exits
       const int64_t issued = i;
@@ -180,50 +184,74 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
+    // ---------------- MMA issuer: the whole warp runs the loop (its waits and
+    // counters stay warp-uniform) and one elected lane issues the MMAs and
+    // commits.  The operand descriptors differ only in their start address
+    // (bits 0-13 of the low word, address / 16), and every operand lies below
+    // 256 KB of shared memory: an operand is the base descriptor plus one
+    // 32-bit add.  This warp shares its sub-partition with epilogue warps
+    // that keep the integer pipe busy, so its per-tile integer work is kept
+    // to a few instructions.
+    {
       constexpr uint32_t idesc = (1u << 4)                 // D: fp32
                                  | (1u << 7) | (1u << 10)  // A, B: bf16
                                  | ((uint32_t)(C::NMMA >> 3) << 17)  // N
                                  | ((uint32_t)(BM >> 4) << 24);      // M
-      bool ok = wait_phase(sfull_bar, 0, abort_flag, p.err, p.wait_ns);
-      int64_t i = 0, j = 0;  // tiles and items (tile x N-half) issued
-      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
-        const int s = (int)(i % C::STAGES);
-        const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
-        if (!wait_phase(full_bar(s), ph, abort_flag, p.err, p.wait_ns)) break;
-        for (int h = 0; h < C::NH; ++h, ++j) {
-          const int a = (int)(j & 1);
-          const uint32_t aph = (uint32_t)((j >> 1) & 1);
-          if (!wait_phase(tempty_bar(a), aph ^ 1u, abort_flag, p.err, p.wait_ns)) {
+      const uint64_t a0 = desc_sw128(sA), b0 = desc_sw128(sS);
+      const uint32_t a_hi = (uint32_t)(a0 >> 32), a_lo0 = (uint32_t)a0;
+      const uint32_t b_hi = (uint32_t)(b0 >> 32), b_lo0 = (uint32_t)b0;
+      bool ok = __all_sync(0xffffffffu, wait_phase(sfull_bar, 0, abort_flag, p.err, p.wait_ns));
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t j = 0;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        if (!__all_sync(0xffffffffu, wait_phase(full_bar(s), ph, abort_flag, p.err, p.wait_ns)))
+          break;
+        const uint32_t a_lo = a_lo0 + (uint32_t)s * (uint32_t)(C::A_STAGE >> 4);
+#pragma unroll
+        for (int h = 0; h < C::NH; ++h) {
+          const uint32_t a = j & 1u;
+          const uint32_t aph = (j >> 1) & 1u;
+          if (!__all_sync(0xffffffffu,
+                          wait_phase(tempty_bar((int)a), aph ^ 1u, abort_flag, p.err, p.wait_ns))) {
             ok = false;
             break;
           }
           fence_after();
+          const uint32_t tmem_d = tmem_base + a * (uint32_t)C::NMMA;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-            const uint64_t adesc =
-                desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
-            const uint64_t bdesc =
-                desc_sw128(sS + (kk >> 2) * C::S_CHUNK + h * C::NMMA * 128 + koff);
-            mma_ss(tmem_base + a * C::NMMA, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (uint32_t)(kk & 3) * 32u;
+              const uint32_t aoff = ((uint32_t)(kk >> 2) * C::A_CHUNK + koff) >> 4;
+              const uint32_t boff =
+                  ((uint32_t)(kk >> 2) * C::S_CHUNK + (uint32_t)h * C::NMMA * 128u + koff) >> 4;
+              const uint64_t adesc = ((uint64_t)a_hi << 32) | (uint64_t)(a_lo + aoff);
+              const uint64_t bdesc = ((uint64_t)b_hi << 32) | (uint64_t)(b_lo0 + boff);
+              mma_ss(tmem_d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            }
+            commit(tfull_bar((int)a));
           }
-          commit(tfull_bar(a));
+          __syncwarp();
+          ++j;
         }
         if (!ok) break;
-        commit(empty_bar(s));
+        if (elect_one()) commit(empty_bar(s));
+        __syncwarp();
+        if (++s == C::STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
-      // drain: the last accumulator's MMAs must be complete before TMEM is freed
-      if (j > 0) {
-        const int64_t jl = j - 1;
+      if (j > 0 && lane == 0) {
+        const uint32_t jl = j - 1;
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(tfull_bar((int)(jl & 1)), (uint32_t)((jl >> 1) & 1)) &&
+        while (!mbar_try_wait(tfull_bar((int)(jl & 1)), (jl >> 1) & 1) &&
                globaltimer() - t0 < p.wait_ns) {
         }
       }
+      __syncwarp();
     }
-    __syncwarp();
   } else if (warp < C::FIRST_NORM_WARP) {
     // ---------------- sign epilogue: TMEM lane quadrant warp % 4, and the
     // k-th of the quadrant's SQ shares of each item's code words
@@ -285,10 +313,9 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
   } else {
     // ---------------- norm epilogue: rows 32*(warp-6) .. +31 of each tile
     const int r = 32 * (warp - C::FIRST_NORM_WARP) + lane;
-    int64_t i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-      const int s = (int)(i % C::STAGES);
-      const uint32_t ph = (uint32_t)((i / C::STAGES) & 1);
+    int s = 0;            // stage of this tile and the phase it completes next
+    uint32_t ph = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
       if (!__all_sync(0xffffffffu, wait_phase(full_bar(s), ph, abort_flag, p.err, p.wait_ns)))
         break;
       float ss0 = 0.f, ss1 = 0.f;
@@ -309,6 +336,10 @@ __global__ void __launch_bounds__(Cfg<M, D>::THREADS, 1)
       const int64_t row = tile * BM + r;
       if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n))
         p.norms[row] = __half_as_ushort(__float2half_rn(sqrtf(ss0 + ss1)));
+      if (++s == C::STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
   }
 

@@ -79,8 +79,10 @@ def _shard_worker(rank, world, port, out_q):
             gathered[name] = parts
         ms = bench.reduce_max_over_ranks([4.0, 2.0][rank], world, torch.device("cpu"))
         rate = bench.whole_job_rate(w.n_keys, world, ms)
+        # numpy arrays travel through the queue by value (torch tensors would
+        # be shared through file descriptors that die with this process)
         out_q.put((rank, w.first_seq, w.n_keys, rate,
-                   {k: [p.clone() for p in v] for k, v in gathered.items()}
+                   {k: [p.numpy().copy() for p in v] for k, v in gathered.items()}
                    if rank == 0 else None))
     finally:
         dist.destroy_process_group()
@@ -105,7 +107,7 @@ def test_ranks_hold_distinct_shards_of_the_global_batch():
             "Q": workloads.queries(glob).float(),
             "lens": workloads.paged_layout(glob.with_(T=4096))[0].float(),
             "Kn": workloads.new_tokens(glob)[0].float()}
-    parts = res[0][4]
+    parts = {k: [torch.from_numpy(a) for a in v] for k, v in res[0][4].items()}
     for name, full in want.items():
         assert not torch.equal(parts[name][0], parts[name][1]), name
         assert torch.equal(torch.cat(parts[name]), full), name
