@@ -801,19 +801,56 @@ PHASE_KERNEL = {"quantize": "jl_quantize_keys (quantize_tc_kernel)",
                 "decode": "jl_decode_attention (qproj + decode_scorer_kernel + combine)"}
 
 
-def roofline_of(phase, rec, w, peak, peak_kind):
-    """Roofline entry of one phase: its algorithmic bytes over its event-timed
-    duration, against the measured HBM copy bandwidth; DRAM traffic per launch
-    from the committed ncu summary when the kernel's source is unchanged."""
-    traffic = ncu_traffic(phase + ":" + w.name)
+def load_tensor_peaks():
+    """(burst, sustained) dense bf16 TFLOP/s from MEASURED_PEAKS.json, else the
+    fallback burst figure for both."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return (float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    "measured")
+    return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def quantize_flops(w, n_keys):
+    """The projection K S^T: 2 m d flops per key."""
+    return 2 * w.m * w.d * n_keys
+
+
+def roofline_of(phase, rec, w, peak, peak_kind, full_size=True, n_keys=None):
+    """Roofline entry of one phase: its algorithmic bytes (or, for a quantizer
+    whose flops per byte exceed the ridge of the measured peaks, its flops)
+    over its event-timed duration, against the measured HBM copy bandwidth
+    (or the measured bf16 tensor peak).  DRAM traffic per launch comes from
+    the committed ncu summary when the kernel's source is unchanged and the
+    workload is the full-size one the summary was scaled to."""
+    traffic = ncu_traffic(phase + ":" + w.name) if full_size else None
     r = {"kernel": PHASE_KERNEL[phase], "bound": "hbm", "achieved": rec["GB_per_s"],
          "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
          "frac": rec["GB_per_s"] / peak,
          "algorithmic_bytes_per_launch": rec["algorithmic_bytes"],
          "traffic": traffic["dram_bytes_per_launch"] if traffic else None}
+    if phase == "quantize" and n_keys:
+        t_burst, t_sus, t_kind = load_tensor_peaks()
+        flops = quantize_flops(w, n_keys)
+        intensity = flops / rec["algorithmic_bytes"]
+        ridge = t_burst * 1e12 / (peak * 1e9)
+        tf = flops / (rec["ms"] * 1e-3) / 1e12
+        r["flops_per_launch"] = flops
+        r["flop_per_byte"] = intensity
+        r["ridge_flop_per_byte"] = ridge
+        r["tensor_tflops"] = tf
+        r["frac_of_bf16_burst"] = tf / t_burst
+        r["frac_of_bf16_sustained"] = tf / t_sus
+        if intensity > ridge:
+            r.update({"bound": "tensor", "achieved": tf, "peak": t_burst,
+                      "peak_kind": f"{t_kind} bf16_tflops (burst; the phase is timed alone)",
+                      "unit": "TFLOP/s", "frac": tf / t_burst})
     if traffic:
         for k in ("dram_read_bytes_per_launch", "dram_write_bytes_per_launch",
-                  "write_side"):
+                  "l2_write_bytes_per_launch", "write_side"):
             if k in traffic:
                 r[k.replace("_per_launch", "")] = traffic[k]
     return r
@@ -866,7 +903,8 @@ def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error)
     rec = {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} T={w.T} d={w.d} m={w.m}",
            "steps": steps, "warmup": warmup, "ms_per_step": ms,
            "keys_per_s": n_keys / (ms * 1e-3), "phases": phases,
-           "rooflines": {ph: roofline_of(ph, phases[ph], w, peak, peak_kind) for ph in phases},
+           "rooflines": {ph: roofline_of(ph, phases[ph], w, peak, peak_kind, n_keys=n_keys)
+                         for ph in phases},
            "l2": "inputs exceed L2 (126 MB); no flush" if n_keys * w.d * 2 > 126e6
                  else "inputs fit in L2; latency-bound parity workload"}
     if w.name == "prefill":
@@ -1051,7 +1089,8 @@ def run_ours(args, rank, world, local_rank):
                  "out": out.numel() * out.element_size(),
                  "workspace (projections + partial states)": int(ws_bytes)}
     phases = phase_records(w, n_keys, q_ms, d_ms, peak, decode, fixed)
-    rooflines = {ph: roofline_of(ph, phases[ph], w, peak, peak_kind) for ph in phases}
+    rooflines = {ph: roofline_of(ph, phases[ph], w, peak, peak_kind, full_size=not args.batch,
+                                 n_keys=n_keys) for ph in phases}
     dom = max(phases, key=lambda k: phases[k]["ms"])
     roof = rooflines[dom]
 

@@ -172,15 +172,19 @@ struct ProjLimits {
   int64_t x_extent = 0, dst_extent = 0;
 };
 
-template <int M, int D, bool XF32>
+// RS > 1 splits the m sketch rows over RS CTAs: this CTA projects rows
+// [split * m / RS, (split + 1) * m / RS) only (a launch of RS times as many,
+// shorter CTAs; the routine is latency-bound, so the split cuts its time).
+template <int M, int D, bool XF32, int RS = 1>
 __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
                                          const void *__restrict__ X, int64_t x0,
                                          int nx, float *dst, int dst_stride = M,
-                                         const ProjLimits lim = ProjLimits{}) {
-  constexpr int CPL = D / 32;   // columns per lane
-  constexpr int CH = 8;         // rows per chunk
-  constexpr int RPW = M / 8;    // rows per warp
-  static_assert(CH * PROJ_VECS == 32 && RPW % CH == 0, "projection tiling");
+                                         const ProjLimits lim = ProjLimits{}, int split = 0) {
+  constexpr int CPL = D / 32;        // columns per lane
+  constexpr int CH = 8;              // rows per chunk
+  constexpr int RPW = M / (8 * RS);  // rows per warp
+  static_assert(CH * PROJ_VECS == 32 && RPW % CH == 0 && RPW >= CH, "projection tiling");
+  const int rbase = split * (M / RS);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float x[PROJ_VECS][CPL];
 #pragma unroll
@@ -199,7 +203,7 @@ __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
     uint32_t sw[CH][CPL / 2];
 #pragma unroll
     for (int k = 0; k < CH; ++k) {
-      const uint16_t *row = S + (int64_t)(warp + 8 * (r0 + k)) * D + lane * CPL;
+      const uint16_t *row = S + (int64_t)(rbase + warp + 8 * (r0 + k)) * D + lane * CPL;
       if constexpr (CPL == 4) {
         const uint2 t = __ldg(reinterpret_cast<const uint2 *>(row));
         sw[k][0] = t.x;
@@ -232,9 +236,15 @@ __device__ __forceinline__ void project4(const uint16_t *__restrict__ S,
       }
     }
     const int k = lane / PROJ_VECS, j = lane % PROJ_VECS;
-    const int64_t di = (int64_t)j * dst_stride + warp + 8 * (r0 + k);
+    const int64_t di = (int64_t)j * dst_stride + rbase + warp + 8 * (r0 + k);
     if (j < nx && (!lim.err || JL_IN_RANGE(lim.err, di, 1, lim.dst_extent))) dst[di] = v[0];
   }
+}
+
+// Row splits of the query projection: one 8-row chunk per warp.
+template <int M>
+constexpr int proj_splits() {
+  return M / 64;
 }
 
 template <int M, int D, bool QF32>
@@ -245,8 +255,9 @@ __global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restr
   griddep_launch_dependents();  // let the scorer start its copies now
   const int64_t x0 = (int64_t)blockIdx.x * PROJ_VECS;
   const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)nq - x0);
-  project4<M, D, QF32>(S, Q, x0, nx, U + x0 * M, M,
-                       ProjLimits{err, (int64_t)nq * D, ((int64_t)nq - x0) * M});
+  project4<M, D, QF32, proj_splits<M>()>(S, Q, x0, nx, U + x0 * M, M,
+                                         ProjLimits{err, (int64_t)nq * D, ((int64_t)nq - x0) * M},
+                                         (int)blockIdx.y);
 }
 
 // TurboQuant-prod query rows, four queries per CTA: w = Pinv^T q (so that
@@ -792,10 +803,75 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
   if constexpr (C::A_SMEM) __syncwarp();
 }
 
-template <int M, int D, bool S8, bool PAGED, int TB = 0>
+// Query fragments of the int8 scoring with the keys as the MMA's rows (one
+// query head per KV head): the B operand of m16n8k32 is the head's quantised
+// u, column 0 the high limbs and column 1 the low limbs, the other six columns
+// zero.  u is quantised exactly as build_afrags does it (per head to +-32000,
+// two limbs, the same coordinate order: k slot 4t + i of slice c is bit
+// (2c & 7) + 8i of the lane's word t * WORDS + c / 4, and slot 16 + 4t + i bit
+// (2c & 7) + 1 + 8i), so column g of lane (g, t) needs the limbs of head 0:
+// lanes g = 0 and 1 both quantise head 0's row and keep one limb each.
+template <int M>
+__device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool live, int g, int t,
+                                                     uint32_t (&bfr)[M / 32][2],
+                                                     float (&hscale)[2], int (&usum)[2]) {
+  static_assert(M >= 128, "keys-as-rows scoring: m >= 128");
+  constexpr int WORDS = LaneRuns<M>::WORDS;
+  float amax = 0.f;
+  if (live) {
+#pragma unroll
+    for (int lw = 0; lw < WORDS; ++lw) {
+      const float *src = urow + 32 * (t * WORDS + lw);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 v = ldg4(src + 4 * k);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+    }
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  hscale[0] = amax > 0.f ? amax / 32000.f : 0.f;
+  const float inv = amax > 0.f ? 32000.f / amax : 0.f;
+  int isum = 0;
+#pragma unroll
+  for (int lw = 0; lw < WORDS; ++lw) {
+    const float *src = urow + 32 * (t * WORDS + lw);
+    float4 x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
+#pragma unroll
+    for (int c2 = 0; c2 < 4; ++c2) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int pp = 2 * c2 + r;
+        int hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int ui = __float2int_rn(f4c(x[(pp + 8 * j) >> 2], pp & 3) * inv);
+          isum += ui;
+          hi[j] = (ui + 128) >> 8;
+          lo[j] = ui - (hi[j] << 8);
+        }
+        bfr[4 * lw + c2][r] = g == 0   ? pack_s8x4(hi[0], hi[1], hi[2], hi[3])
+                              : g == 1 ? pack_s8x4(lo[0], lo[1], lo[2], lo[3])
+                                       : 0u;
+      }
+    }
+  }
+  isum += __shfl_xor_sync(0xffffffffu, isum, 1);
+  isum += __shfl_xor_sync(0xffffffffu, isum, 2);
+  usum[0] = isum;
+}
+
+// KR: int8 scoring with the keys as the MMA's rows (one query head per KV
+// head, m >= 128, QJL codes): 16 keys per m16n8k32 instead of 8 heads, half
+// the MMAs of the head-rows form when only one head row is live.
+template <int M, int D, bool S8, bool PAGED, int TB = 0, bool KR = false>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
     decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
   using C = DecCfg<M, D, S8, TB>;
+  static_assert(!KR || (S8 && TB == 0 && M >= 128), "keys-as-rows scoring: int8, QJL codes, m >= 128");
   extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -882,7 +958,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
   float hscale[2] = {0.f, 0.f};
   int usum[2] = {0, 0};
   float acc[C::DT][4];
-  uint32_t afr[C::A_SMEM ? 1 : C::NC][4];
+  uint32_t afr[(C::A_SMEM || KR) ? 1 : C::NC][4];
+  uint32_t bfr[KR ? C::NC : 1][2];
   // a wait that ran out: bit 0 = it did; bits 1-2 = the block's index mod 4
   // (its stage and phase); bit 3 = the next block was started too
   int failed = 0;
@@ -946,7 +1023,18 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       const bool live =
           g < Gg && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + g) * C::CODE_BITS,
                                 C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
-      build_afrags<M, D, S8, TB>(urow, live, t, ring, afr, hscale, usum);
+      if constexpr (KR) {
+        // one head: lanes g = 0 and 1 quantise head 0's row (one limb each)
+        const float *urow0 = p.U + ((int64_t)b_idx * p.Hq + hq0) * C::CODE_BITS;
+        const bool live0 =
+            g < 2 && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0) * C::CODE_BITS,
+                                 C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
+        build_bfrags_keyrows<M>(urow0, live0, g, t, bfr, hscale, usum);
+        (void)urow;
+        (void)live;
+      } else {
+        build_afrags<M, D, S8, TB>(urow, live, t, ring, afr, hscale, usum);
+      }
       if constexpr (C::A_SMEM) __syncwarp();
     }
 
@@ -1014,7 +1102,47 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
     // ---- raw estimator sum_i u_i sign_i for head g, keys kg*8 + 2t + j
     // (cell-plane codes: raw over the planes, rawq over the residual signs)
     float raw[4][2], rawq[4][2];
-    if constexpr (S8) {
+    if constexpr (KR) {
+      // rows: keys kb*16 + g (code words wd[2 kb]) and kb*16 + g + 8 (wd[2 kb + 1]);
+      // columns 0 / 1: the high / low limb sums; two accumulators per key
+      // block (even and odd slices) for independent MMA chains
+      int sc[2][2][4];
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int par = 0; par < 2; ++par)
+          sc[kb][par][0] = sc[kb][par][1] = sc[kb][par][2] = sc[kb][par][3] = 0;
+#pragma unroll
+      for (int c = 0; c < C::NC; ++c) {
+        const int q0 = 2 * c, q1 = 2 * c + 1;
+        const int p0 = q0 & 7, p1 = q1 & 7;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          const uint32_t wr0 = wd[2 * kb][q0 >> 3], wr8 = wd[2 * kb + 1][q0 >> 3];
+          const uint32_t a0 = (wr0 >> p0) & 0x01010101u;
+          const uint32_t a1 = (wr8 >> p0) & 0x01010101u;
+          const uint32_t a2 = (wr0 >> p1) & 0x01010101u;
+          const uint32_t a3 = (wr8 >> p1) & 0x01010101u;
+          mma_s8_16832(sc[kb][c & 1], a0, a1, a2, a3, bfr[c][0], bfr[c][1]);
+        }
+      }
+      // lane (g, 0) holds sum_{bit=1} u_int of keys kb*16 + g (v[kb][0]) and
+      // kb*16 + g + 8 (v[kb][1]); key kg*8 + 2t + j sits in lane (2t + j, 0)
+      int v[2][2];
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        v[kb][0] = (sc[kb][0][0] + sc[kb][1][0]) * 256 + (sc[kb][0][1] + sc[kb][1][1]);
+        v[kb][1] = (sc[kb][0][2] + sc[kb][1][2]) * 256 + (sc[kb][0][3] + sc[kb][1][3]);
+      }
+#pragma unroll
+      for (int kg = 0; kg < 4; ++kg)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int si = __shfl_sync(0xffffffffu, v[kg >> 1][kg & 1], (2 * t + j) * 4);
+          raw[kg][j] = hscale[0] * (float)(2 * si - usum[0]);
+        }
+      (void)rawq;
+    } else if constexpr (S8) {
       int sc[4][4], sq[4][4];
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg) {
@@ -1337,7 +1465,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
 // ---------------------------------------------------------------------------
 // 4. paged calls: one prep launch of 256-thread CTAs does the query
 // projections (four queries per CTA) and, when keys are given, appends each
-// sequence's new key (four keys per CTA).  The scorer and the combine derive
+// sequence's new key (four keys per CTA); each group of four is split over
+// m / 64 CTAs by sketch rows (blockIdx.y), the first of which also stores
+// the key's norm and value row.  The scorer and the combine derive
 // the work split from seq_lens themselves.
 struct PrepParams {
   const void *Q;
@@ -1365,6 +1495,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
   // scorer be scheduled; it waits for this grid's results where it needs them
   griddep_wait();
   griddep_launch_dependents();
+  constexpr int RS = proj_splits<M>();  // blockIdx.y: this CTA's rows of S
+  const int split = (int)blockIdx.y;
   const int bid = blockIdx.x;
   const int i = threadIdx.x;
   const int qctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS;
@@ -1372,8 +1504,9 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
     // ---- query projections u = S q, four queries per CTA
     const int64_t x0 = (int64_t)bid * PROJ_VECS;
     const int nx = (int)min((int64_t)PROJ_VECS, (int64_t)pp.nq - x0);
-    project4<M, D, QF32>(pp.S, pp.Q, x0, nx, pp.U + x0 * M, M,
-                         ProjLimits{pp.err, (int64_t)pp.nq * D, ((int64_t)pp.nq - x0) * M});
+    project4<M, D, QF32, RS>(pp.S, pp.Q, x0, nx, pp.U + x0 * M, M,
+                             ProjLimits{pp.err, (int64_t)pp.nq * D, ((int64_t)pp.nq - x0) * M},
+                             split);
     return;
   }
   const int nkv = pp.B * pp.Hkv;
@@ -1383,8 +1516,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
     // each at position seq_lens[b] of its sequence
     const int x0 = (bid - qctas) * PROJ_VECS;
     const int nx = min(PROJ_VECS, nkv - x0);
-    project4<M, D, KF32>(pp.S, pp.K_new, x0, nx, &ys[0][0], M,
-                         ProjLimits{pp.err, (int64_t)nkv * D, PROJ_VECS * M});
+    project4<M, D, KF32, RS>(pp.S, pp.K_new, x0, nx, &ys[0][0], M,
+                             ProjLimits{pp.err, (int64_t)nkv * D, PROJ_VECS * M}, split);
     __syncthreads();
     const int lane = i & 31, j = i >> 5;  // warp j stores key x0 + j
     if (j >= nx) return;
@@ -1400,11 +1533,14 @@ __global__ void __launch_bounds__(PROJ_THREADS) paged_prep_kernel(const PrepPara
     }
     const int64_t slot = ((int64_t)page * pp.Hkv + hkv) * pp.page_tokens + (pos % pp.page_tokens);
     if (!JL_IN_RANGE(pp.err, slot, 1, (int64_t)pp.num_pages * pp.Hkv * pp.page_tokens)) return;
+    // this CTA's code words: rows [split * M / RS, (split + 1) * M / RS)
 #pragma unroll
-    for (int w = 0; w < M / 32; ++w) {  // bit l of word w: coordinate 32w + l >= 0
+    for (int w = split * (M / RS / 32); w < (split + 1) * (M / RS / 32); ++w) {
+      // bit l of word w: coordinate 32w + l >= 0
       const uint32_t word = __ballot_sync(0xffffffffu, ys[j][w * 32 + lane] >= 0.f);
       if (lane == 0) pp.sign_pages[slot * (M / 32) + w] = word;
     }
+    if (split != 0) return;  // the first split stores the norm and the value row
     float ss = 0.f;
     for (int c = lane; c < D; c += 32) {
       const float x = KF32 ? reinterpret_cast<const float *>(pp.K_new)[(int64_t)kvi * D + c]
@@ -1680,11 +1816,11 @@ static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *par
 }
 
 // Launch the scorer (one wave, <= the plan's warp bound) and the combine.
-template <int M, int D, bool S8, bool PAGED, int TB = 0>
+template <int M, int D, bool S8, bool PAGED, int TB = 0, bool KR = false>
 static cudaError_t launch_scorer_combine(const DecodePlan &pl, DecParams &p, const DecMaps &maps,
                                          uint16_t *out, cudaStream_t stream) {
   using C = DecCfg<M, D, S8, TB>;
-  auto kern = decode_scorer_kernel<M, D, S8, PAGED, TB>;
+  auto kern = decode_scorer_kernel<M, D, S8, PAGED, TB, KR>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::CTA_BYTES);
   if (e != cudaSuccess) return e;
@@ -1721,14 +1857,22 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   const int bh = pl.B * pl.Hq;
   const int qctas = (bh + PROJ_VECS - 1) / PROJ_VECS;
   if (q_f32)
-    qproj_kernel<M, D, true><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh, err);
+    qproj_kernel<M, D, true><<<dim3(qctas, proj_splits<M>()), PROJ_THREADS, 0, stream>>>(Q, S, U,
+                                                                                        bh, err);
   else
-    qproj_kernel<M, D, false><<<qctas, PROJ_THREADS, 0, stream>>>(Q, S, U, bh, err);
+    qproj_kernel<M, D, false><<<dim3(qctas, proj_splits<M>()), PROJ_THREADS, 0, stream>>>(Q, S, U,
+                                                                                         bh, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, signs, norms, scores, softmax_scale, M, err);
   p.drop_copies = test_drop_copies() ? 1 : 0;
+  // one head per KV head and a code at least twice the value row's bytes
+  // (m >= 4d): the keys-as-rows int8 scoring (half the MMAs; measured faster
+  // there, slightly slower at m = 2d)
+  if constexpr (S8 && M >= 4 * D) {
+    if (pl.G == 1) return launch_scorer_combine<M, D, true, false, 0, true>(pl, p, maps, out, stream);
+  }
   return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
 }
 
@@ -1803,13 +1947,14 @@ cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S
   const int ctas = (nq + PROJ_VECS - 1) / PROJ_VECS;
   int *err = device_error_ptr();
   if (err == nullptr) return cudaErrorInvalidSymbol;
-#define JL_CASE(MM, DD)                                                                \
-  if (m == MM && d == DD) {                                                            \
-    if (q_f32)                                                                         \
-      qproj_kernel<MM, DD, true><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err);  \
-    else                                                                               \
-      qproj_kernel<MM, DD, false><<<ctas, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err); \
-    return cudaGetLastError();                                                         \
+#define JL_CASE(MM, DD)                                                                  \
+  if (m == MM && d == DD) {                                                              \
+    const dim3 grid(ctas, proj_splits<MM>());                                            \
+    if (q_f32)                                                                           \
+      qproj_kernel<MM, DD, true><<<grid, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err);    \
+    else                                                                                 \
+      qproj_kernel<MM, DD, false><<<grid, PROJ_THREADS, 0, stream>>>(Q, S, U, nq, err);   \
+    return cudaGetLastError();                                                           \
   }
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
@@ -1905,7 +2050,7 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   const int nkv = pl.B * pl.Hkv;
   const int prep_ctas = (pp.nq + PROJ_VECS - 1) / PROJ_VECS +
                         (pp.append ? (nkv + PROJ_VECS - 1) / PROJ_VECS : 0);
-  const dim3 pg(prep_ctas), pb(PROJ_THREADS);
+  const dim3 pg(prep_ctas, proj_splits<M>()), pb(PROJ_THREADS);
   cudaError_t e;
   if (a.q_f32)
     e = a.k_f32 ? launch_pdl(paged_prep_kernel<M, D, true, true>, pg, pb, 0, stream, pp)
@@ -1919,6 +2064,9 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   p.seq_lens = a.seq_lens; p.block_table = a.block_table;
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
+  if constexpr (S8 && M >= 4 * D) {  // as the contiguous call
+    if (pl.G == 1) return launch_scorer_combine<M, D, true, true, 0, true>(pl, p, maps, a.out, stream);
+  }
   return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);
 }
 

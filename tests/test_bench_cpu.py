@@ -72,3 +72,27 @@ def test_peaks_are_read_or_fall_back():
     assert gbs > 1000 and kind in ("measured", "fallback")
     tf, tkind = bench.load_tensor_peak()
     assert tf > 100 and tkind
+
+
+def test_quantizer_roofline_bound_follows_the_ridge():
+    # 2 m d flops over (2 d + m/8 + 2) bytes per key: m = 512, d = 64 sits above
+    # the ridge of the measured peaks (tensor-bound), the headline shape below
+    peak = 6457.7
+    t_burst, _, _ = bench.load_tensor_peaks()
+    for (m, d), bound in (((512, 64), "tensor"), ((256, 128), "hbm"), ((64, 64), "hbm")):
+        w = workloads.SWEEP_BASE.with_(m=m, d=d)
+        n = w.n_keys
+        qb = bench.quantize_bytes(w, n)
+        ms = 1.0
+        rec = {"ms": ms, "algorithmic_bytes": qb, "GB_per_s": qb / 1e-3 / 1e9}
+        r = bench.roofline_of("quantize", rec, w, peak, "measured", full_size=False, n_keys=n)
+        ridge = t_burst * 1e12 / (peak * 1e9)
+        assert (2 * m * d / (2 * d + m // 8 + 2) > ridge) == (bound == "tensor")
+        assert r["bound"] == bound, (m, d)
+        assert r["traffic"] is None               # scaled-down workloads carry none
+        if bound == "tensor":
+            assert r["unit"] == "TFLOP/s"
+            assert r["achieved"] == pytest.approx(2 * m * d * n / 1e-3 / 1e12)
+            assert r["frac"] == pytest.approx(r["achieved"] / t_burst)
+        else:
+            assert r["unit"] == "GB/s" and r["frac"] == pytest.approx(rec["GB_per_s"] / peak)

@@ -144,6 +144,9 @@ DECODE_CASES = [
     (1, 4, 4, 1001, 128, 64, torch.bfloat16, 1.0),
     (1, 2, 2, 512, 512, 128, torch.bfloat16, 2.0),
     (2, 4, 1, 777, 512, 64, torch.bfloat16, 1.0),
+    # one head per KV head with m >= 4d: keys as the int8 MMA's rows
+    (2, 3, 3, 999, 256, 64, torch.float32, 2.0),
+    (1, 2, 2, 4097, 512, 128, torch.bfloat16, 3.0),
 ]
 
 
