@@ -35,7 +35,7 @@
 //              each row at once; each thread copies its half of its code
 //              row two tiles ahead.
 //   warps 8-11 epilogue: warp w reads TMEM lane quadrant w % 4.
-//   warp 12    owns the TMEM allocation; lane 0 issues the MMAs of a tile
+//   warp 12    owns the TMEM allocation; one elected lane issues the MMAs of a tile
 //              into one of two accumulators and commits them to the barriers
 //              that free the Z chunks and publish the accumulator.
 // Every mbarrier wait is bounded (about 2 s of GPU time); a wait that runs
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = nk > 0;
     const uint32_t pbytes = (uint32_t)(KP * 8);             // 2 code words per chunk
     const uint32_t crow = base + C::OFF_C + r * C::CODE_ROW + pt * pbytes;
-    auto code_slot = [&](int64_t it) { return crow + (uint32_t)((it % CODE_SLOTS) * BM * C::CODE_ROW); };
+    auto code_slot = [&](int slot) { return crow + (uint32_t)(slot * BM * C::CODE_ROW); };
     auto copy_part = [&](uint32_t dst, int64_t row) {
       const bool live = row < p.n && JL_IN_RANGE(p.err, row * (M / 8) + pt * pbytes, KP * 8,
                                                  p.n * (M / 8));
@@ -330,23 +330,30 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok)
       for (int k = 0; k < CODE_SLOTS - 1; ++k)
         copy_part(code_slot(k), ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BM + r);
-    int64_t it = 0;
-    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
-      copy_part(code_slot(it + CODE_SLOTS - 1),
+    int cs = 0;                    // code slot of this tile's words
+    // ring slot and phase of this part's first chunk of the tile: global
+    // chunk it * KCH + kc0, advanced by KCH per tile without a division
+    int rs0 = kc0 % C::RING;
+    uint32_t rph0 = (uint32_t)((kc0 / C::RING) & 1);
+    for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      copy_part(code_slot(cs == 0 ? CODE_SLOTS - 1 : cs - 1),
                 (tile + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BM + r);
       cp_async_wait<CODE_SLOTS - 1>();  // this tile's words have landed
       uint32_t cur[2 * KP];
       {
-        const uint8_t *src = gbase + (code_slot(it) - base);
+        const uint8_t *src = gbase + (code_slot(cs) - base);
 #pragma unroll
         for (int i = 0; i < 2 * KP; ++i) cur[i] = reinterpret_cast<const uint32_t *>(src)[i];
       }
+      int s = rs0;
+      uint32_t ph = rph0;
 #pragma unroll
       for (int kk = 0; kk < KP; ++kk) {
         if (kk >= nk) break;
-        const int64_t c = it * C::KCH + kc0 + kk;  // global chunk index
-        const int s = (int)(c % C::RING);
-        const uint32_t ph = (uint32_t)((c / C::RING) & 1);
+        if (kk > 0 && ++s == C::RING) {  // global chunk it * KCH + kc0 + kk
+          s = 0;
+          ph ^= 1u;
+        }
         if (!wait_phase(zempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
           ok = false;
           break;
@@ -368,6 +375,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(zfull_bar(s));
       }
+      // next tile: its first chunk of this part is KCH chunks later
+      rs0 += C::KCH;
+      while (rs0 >= C::RING) {
+        rs0 -= C::RING;
+        rph0 ^= 1u;
+      }
+      if (++cs == CODE_SLOTS) cs = 0;
     }
     cp_async_wait<0>();  // no copy outlives the CTA
   } else if (warp < MMA_WARP) {
@@ -434,48 +448,69 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) bulk_wait_all();  // stores complete before the CTA exits
     __syncwarp();
   } else {
-    // ---------------- MMA issuer
-    if (lane == 0) {
+    // ---------------- MMA issuer: the whole warp runs the loop, one elected
+    // lane issues; the B descriptor is the base plus a 32-bit start-address add
+    {
       constexpr uint32_t idesc = (1u << 4)                  // D: fp32
                                  | (1u << 7) | (1u << 10)   // A, B: bf16
                                  | ((uint32_t)(D >> 3) << 17)   // N
                                  | ((uint32_t)(BM >> 4) << 24); // M
-      int64_t c = 0, t = 0;
+      const uint64_t b0 = smem_desc_sw128(sST);
+      const uint32_t b_hi = (uint32_t)(b0 >> 32), b_lo0 = (uint32_t)b0;
+      int rs = 0;
+      uint32_t rph = 0;
+      uint32_t t = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++t) {
-        const int a = (int)(t & 1);
-        const uint32_t aph = (uint32_t)((t >> 1) & 1);
-        if (!wait_phase(aempty_bar(a), aph ^ 1u, abort_flag, p.err)) break;
+        const int a = (int)(t & 1u);
+        const uint32_t aph = (t >> 1) & 1u;
+        if (!__all_sync(0xffffffffu, wait_phase(aempty_bar(a), aph ^ 1u, abort_flag, p.err)))
+          break;
         tc_fence_after();
-        for (int kc = 0; kc < C::KCH; ++kc, ++c) {
-          const int s = (int)(c % C::RING);
-          const uint32_t ph = (uint32_t)((c / C::RING) & 1);
-          if (!wait_phase(zfull_bar(s), ph, abort_flag, p.err)) {
+        for (int kc = 0; kc < C::KCH; ++kc) {
+          const int s = rs;
+          const uint32_t ph = rph;
+          if (++rs == C::RING) {
+            rs = 0;
+            rph ^= 1u;
+          }
+          if (!__all_sync(0xffffffffu, wait_phase(zfull_bar(s), ph, abort_flag, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          uint32_t el;
+          asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
+                       : "=r"(el));
+          if (el) {
+            const uint32_t blo = b_lo0 + (uint32_t)kc * (uint32_t)(C::ST_CHUNK >> 4);
 #pragma unroll
-          for (int kk = 0; kk < CHUNK_K / 16; ++kk) {  // K = 16: 8 columns of A
-            const uint32_t atm = tmem_base + (uint32_t)(C::Z_COL0 + s * CHUNK_COLS + kk * 8);
-            const uint64_t bdesc = smem_desc_sw128(sST + kc * C::ST_CHUNK + kk * 32);
-            mma_bf16_ts(tmem_base + a * D, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < CHUNK_K / 16; ++kk) {  // K = 16: 8 columns of A
+              const uint32_t atm = tmem_base + (uint32_t)(C::Z_COL0 + s * CHUNK_COLS + kk * 8);
+              const uint64_t bdesc = ((uint64_t)b_hi << 32) | (uint64_t)(blo + (uint32_t)(kk * 2));
+              mma_bf16_ts(tmem_base + a * D, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(zempty_bar(s));
           }
-          mma_commit(zempty_bar(s));
+          __syncwarp();
         }
         if (!ok) break;
-        mma_commit(afull_bar(a));
+        uint32_t el2;
+        asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
+                     : "=r"(el2));
+        if (el2) mma_commit(afull_bar(a));
+        __syncwarp();
       }
       // drain: the last accumulator's MMAs must be complete before TMEM is freed
-      if (t > 0 && ok) {
-        const int64_t tl = t - 1;
+      if (t > 0 && ok && lane == 0) {
+        const uint32_t tl = t - 1;
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(afull_bar((int)(tl & 1)), (uint32_t)((tl >> 1) & 1)) &&
+        while (!mbar_try_wait(afull_bar((int)(tl & 1u)), (tl >> 1) & 1u) &&
                globaltimer() - t0 < WAIT_NS) {
         }
       }
+      __syncwarp();
     }
-    __syncwarp();
   }
 
   tc_fence_before();

@@ -46,7 +46,9 @@
 //   warps 0-3  expand: thread t owns rows t and t + 128 of every tile.
 //   warps 4-7  U into tensor memory first, then the epilogue: lane quadrant
 //              warp % 4 = queries 32 (warp % 4) .. + 31, one list per query.
-//   warp 8     owns the TMEM allocation; lane 0 issues the MMAs.
+//   warp 8     owns the TMEM allocation; the whole warp runs the MMA loop
+//              and one elected lane issues the MMAs (descriptors are
+//              precomputed: an operand is the base plus a 32-bit add).
 // Every mbarrier wait is bounded; a wait that runs out records
 // DERR_TC_WAIT_TIMEOUT and the CTA still frees its TMEM.
 #include "jl_common.cuh"
@@ -420,12 +422,14 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
     // ---------------- expand: rows t and t + 128 of every tile
     const int t = threadIdx.x;
     const uint32_t crow0 = base + C::OFF_C + t * C::CODE_ROW;
-    auto slot0 = [&](int64_t it) { return crow0 + (uint32_t)((it % CODE_SLOTS) * BN * C::CODE_ROW); };
+    auto slot0 = [&](int slot) { return crow0 + (uint32_t)(slot * BN * C::CODE_ROW); };
     for (int k = 0; k < CODE_SLOTS - 1; ++k) {
       const int64_t row0 = tile_at((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * BN + t;
       copy_code_rows<M>(slot0(k), slot0(k) + 128 * C::CODE_ROW, p.signs, row0, p.N, p.err);
     }
-    int64_t c = 0, it = 0;
+    int rs = 0;                 // ring slot of the next chunk and its phase
+    uint32_t rph = 0;
+    int cs = 0;                 // code slot of this tile's rows
     bool ok = true;
     // the two rows' norms (0 past the end), one tile ahead: B holds +-||x||
     auto norm_of = [&](int64_t row) -> uint32_t {
@@ -433,12 +437,12 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
                  ? (uint32_t)__ldg(p.norms + row) & 0x7FFFu : 0u;
     };
     uint32_t n0 = norm_of(tile_at(blockIdx.x) * BN + t), n1 = norm_of(tile_at(blockIdx.x) * BN + t + 128);
-    for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++it) {
+    for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x) {
       const int64_t nrow = tile_at(j + gridDim.x) * BN + t;
       const uint32_t nn0 = norm_of(nrow), nn1 = norm_of(nrow + 128);
       {
         const int64_t row0 = tile_at(j + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BN + t;
-        const uint32_t d0 = slot0(it + CODE_SLOTS - 1);
+        const uint32_t d0 = slot0(cs == 0 ? CODE_SLOTS - 1 : cs - 1);
         copy_code_rows<M>(d0, d0 + 128 * C::CODE_ROW, p.signs, row0, p.N, p.err);
       }
       const uint32_t x0 = 0x80008000u | (n0 << 16) | n0;
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       cp_async_wait<CODE_SLOTS - 1>();
       uint32_t c0w[C::CODE_WORDS], c1w[C::CODE_WORDS];
       {
-        const uint32_t *s0 = reinterpret_cast<const uint32_t *>(gbase + (slot0(it) - base));
+        const uint32_t *s0 = reinterpret_cast<const uint32_t *>(gbase + (slot0(cs) - base));
         const uint32_t *s1 = s0 + 128 * (C::CODE_ROW / 4);
 #pragma unroll
         for (int i = 0; i < C::CODE_WORDS; ++i) {
@@ -455,9 +459,13 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         }
       }
 #pragma unroll
-      for (int kc = 0; kc < C::KCH; ++kc, ++c) {
-        const int s = (int)(c % C::RING);
-        const uint32_t ph = (uint32_t)((c / C::RING) & 1);
+      for (int kc = 0; kc < C::KCH; ++kc) {
+        const int s = rs;
+        const uint32_t ph = rph;
+        if (++rs == C::RING) {
+          rs = 0;
+          rph ^= 1u;
+        }
         if (!wait_phase(zempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
           ok = false;
           break;
@@ -471,6 +479,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       }
       n0 = nn0;
       n1 = nn1;
+      if (++cs == CODE_SLOTS) cs = 0;
     }
     cp_async_wait<0>();
   } else if (warp < MMA_WARP) {
@@ -503,14 +512,14 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         if (sc > list.thr) list.insert(sc, (int32_t)(base_row + 32 * g + e));
       }
     };
-    int64_t tt = 0;
+    uint32_t tt = 0;
     for (int64_t j = blockIdx.x; j < ntiles; j += gridDim.x, ++tt) {
       const int64_t base_row = tile_at(j) * BN;
       const int nvalid = (int)((p.N - base_row) < BN ? (p.N - base_row) : BN);
       // the query's shared bound: scores below it cannot make the top KT
       const float gb = ord_float(*reinterpret_cast<volatile unsigned *>(p.gbound + qi));
-      const int ab = (int)(tt % C::NACC);
-      if (!wait_phase(dfull_bar(ab), (uint32_t)((tt / C::NACC) & 1), abort_flag, p.err)) break;
+      const int ab = (int)(tt % (uint32_t)C::NACC);
+      if (!wait_phase(dfull_bar(ab), (tt / (uint32_t)C::NACC) & 1u, abort_flag, p.err)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t trow =
@@ -587,53 +596,78 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       p.part_idx[o + e] = list.idx[e];
     }
   } else {
-    // ---------------- MMA issuer
-    if (lane == 0) {
+    // ---------------- MMA issuer: the whole warp runs the loop, one elected
+    // lane issues; descriptors are the base plus a 32-bit start-address add
+    {
       constexpr uint32_t idesc = (1u << 4)                        // D: fp32
                                  | (0u << 7) | (0u << 10)         // A, B: fp16
                                  | ((uint32_t)(BN >> 3) << 17)    // N
                                  | ((uint32_t)(QM >> 4) << 24);   // M
-      int64_t c = 0, tt = 0;
+      const uint64_t z0 = smem_desc_sw128(sZ);
+      const uint64_t u0 = smem_desc_sw128(base + C::OFF_U);
+      const uint32_t z_hi = (uint32_t)(z0 >> 32), z_lo0 = (uint32_t)z0;
+      const uint32_t u_hi = (uint32_t)(u0 >> 32), u_lo0 = (uint32_t)u0;
+      int rs = 0;
+      uint32_t rph = 0;
+      uint32_t tt = 0;
       bool ok = true;
       for (int64_t j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++tt) {
         // accumulator ab was read by the epilogue of tile tt - NACC
-        const int ab = (int)(tt % C::NACC);
-        if (!wait_phase(dempty_bar(ab), (uint32_t)(((tt / C::NACC) & 1) ^ 1), abort_flag, p.err))
+        const uint32_t ab = tt % (uint32_t)C::NACC;
+        if (!__all_sync(0xffffffffu, wait_phase(dempty_bar((int)ab),
+                                                ((tt / (uint32_t)C::NACC) & 1u) ^ 1u,
+                                                abort_flag, p.err)))
           break;
         tc_fence_after();
-        for (int kc = 0; kc < C::KCH; ++kc, ++c) {
-          const int s = (int)(c % C::RING);
-          const uint32_t ph = (uint32_t)((c / C::RING) & 1);
-          if (!wait_phase(zfull_bar(s), ph, abort_flag, p.err)) {
+        const uint32_t dt = tmem_base + (uint32_t)C::D_COL + ab * (uint32_t)BN;
+        for (int kc = 0; kc < C::KCH; ++kc) {
+          const int s = rs;
+          const uint32_t ph = rph;
+          if (++rs == C::RING) {
+            rs = 0;
+            rph ^= 1u;
+          }
+          if (!__all_sync(0xffffffffu, wait_phase(zfull_bar(s), ph, abort_flag, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const uint32_t zlo = z_lo0 + (uint32_t)s * (uint32_t)(CHUNK_BYTES >> 4);
+          const uint32_t ulo = u_lo0 + (uint32_t)kc * (uint32_t)(C::U_CHUNK >> 4);
+          uint32_t el;
+          asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
+                       : "=r"(el));
+          if (el) {
 #pragma unroll
-          for (int kk = 0; kk < CHUNK_K / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(sZ + s * CHUNK_BYTES + kk * 32);
-            const uint32_t dt = tmem_base + (uint32_t)(C::D_COL + ab * BN);
-            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-            if constexpr (C::U_SMEM)
-              mma_f16_ss(dt, smem_desc_sw128(base + C::OFF_U + kc * C::U_CHUNK + kk * 32), bdesc,
-                         idesc, acc);
-            else
-              mma_f16_ts(dt, tmem_base + (uint32_t)(kc * 32 + kk * 8), bdesc, idesc, acc);
+            for (int kk = 0; kk < CHUNK_K / 16; ++kk) {
+              const uint64_t bdesc = ((uint64_t)z_hi << 32) | (uint64_t)(zlo + (uint32_t)(kk * 2));
+              const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (C::U_SMEM)
+                mma_f16_ss(dt, ((uint64_t)u_hi << 32) | (uint64_t)(ulo + (uint32_t)(kk * 2)),
+                           bdesc, idesc, acc);
+              else
+                mma_f16_ts(dt, tmem_base + (uint32_t)(kc * 32 + kk * 8), bdesc, idesc, acc);
+            }
+            mma_commit(zempty_bar(s));
           }
-          mma_commit(zempty_bar(s));
+          __syncwarp();
         }
         if (!ok) break;
-        mma_commit(dfull_bar(ab));
+        uint32_t el2;
+        asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
+                     : "=r"(el2));
+        if (el2) mma_commit(dfull_bar((int)ab));
+        __syncwarp();
       }
-      if (tt > 0 && ok) {  // the last tile's MMAs complete before TMEM is freed
+      if (tt > 0 && ok && lane == 0) {  // the last tile's MMAs complete before TMEM is freed
         const unsigned long long t0 = globaltimer();
         const int lb = (int)((tt - 1) % C::NACC);
-        while (!mbar_try_wait(dfull_bar(lb), (uint32_t)(((tt - 1) / C::NACC) & 1)) &&
+        while (!mbar_try_wait(dfull_bar(lb), ((tt - 1) / (uint32_t)C::NACC) & 1u) &&
                globaltimer() - t0 < WAIT_NS) {
         }
       }
+      __syncwarp();
     }
-    __syncwarp();
   }
 
   tc_fence_before();

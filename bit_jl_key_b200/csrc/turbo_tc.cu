@@ -503,56 +503,82 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       tcx::drain_wait(wfull, 0);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer: MMA 1 of tile t, then MMA 2 of tile t - 1
-    if (lane == 0) {
+    // ---------------- MMA issuer: MMA 1 of tile t, then MMA 2 of tile t - 1.
+    // The whole warp runs the loop (waits and counters warp-uniform) and one
+    // elected lane issues; descriptors are the base plus a 32-bit start-address
+    // add (every operand lies below 256 KB of shared memory).
+    {
       constexpr uint32_t idesc = tcx::idesc_f16(BM, 128, 1);
-      bool ok = tcx::wait_phase(wfull, 0, abort_flag, p.err);
+      const uint64_t da = tcx::desc_sw128(sA), dpi = tcx::desc_sw128(sPi), ds = tcx::desc_sw128(sS);
+      const uint32_t a_hi = (uint32_t)(da >> 32), a_lo0 = (uint32_t)da;
+      const uint32_t pi_hi = (uint32_t)(dpi >> 32), pi_lo = (uint32_t)dpi;
+      const uint32_t s_hi = (uint32_t)(ds >> 32), s_lo = (uint32_t)ds;
+      bool ok = __all_sync(0xffffffffu, tcx::wait_phase(wfull, 0, abort_flag, p.err));
       int64_t issued2 = 0;
+      int ks = 0;          // key stage of tile t and the phase it completes next
+      uint32_t kph = 0;
       for (int64_t t = 0; ok && t <= cnt; ++t) {
         if (t < cnt) {
-          const int s = (int)(t % C::STAGES);
+          const int s = ks;
           const int a = (int)(t & 1);
           // the key tile has landed; accumulator a was read by epilogue A of t - 2
-          if (!tcx::wait_phase(kfull(s), (uint32_t)((t / C::STAGES) & 1), abort_flag, p.err) ||
-              (t >= 2 && !tcx::wait_phase(afull(a), (uint32_t)(((t - 2) >> 1) & 1), abort_flag,
-                                          p.err))) {
+          const bool got = tcx::wait_phase(kfull(s), kph, abort_flag, p.err) &&
+                           (t < 2 || tcx::wait_phase(afull(a), (uint32_t)(((t - 2) >> 1) & 1),
+                                                     abort_flag, p.err));
+          if (!__all_sync(0xffffffffu, got)) {
             ok = false;
             break;
           }
           tcx::fence_after();
+          if (tcx::elect_one()) {
+            const uint32_t alo = a_lo0 + (uint32_t)s * (uint32_t)(C::A_STAGE >> 4);
 #pragma unroll
-          for (int kk = 0; kk < QD / 16; ++kk) {
-            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-            const uint64_t ad = tcx::desc_sw128(sA + s * C::A_STAGE + (kk >> 2) * C::A_CHUNK + koff);
-            const uint64_t bd = tcx::desc_sw128(sPi + (kk >> 2) * C::W_CHUNK + koff);
-            tcx::mma_ss(tmem_base + C::D1_COL + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < QD / 16; ++kk) {
+              const uint32_t off =
+                  ((uint32_t)(kk >> 2) * (uint32_t)C::A_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+              const uint32_t woff =
+                  ((uint32_t)(kk >> 2) * (uint32_t)C::W_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+              const uint64_t ad = ((uint64_t)a_hi << 32) | (uint64_t)(alo + off);
+              const uint64_t bd = ((uint64_t)pi_hi << 32) | (uint64_t)(pi_lo + woff);
+              tcx::mma_ss(tmem_base + C::D1_COL + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            tcx::commit(d1full(a));
+            tcx::commit(kempty(s));
           }
-          tcx::commit(d1full(a));
-          tcx::commit(kempty(s));
+          __syncwarp();
+          if (++ks == C::STAGES) {
+            ks = 0;
+            kph ^= 1u;
+          }
         }
         if (t >= 1) {
           const int64_t u = t - 1;
           const int a = (int)(u & 1);
           // residual rows of u written; the projection buffer read by B of u - 1
-          if (!tcx::wait_phase(afull(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err) ||
-              !tcx::wait_phase(d2empty, (uint32_t)((u & 1) ^ 1), abort_flag, p.err)) {
+          const bool got = tcx::wait_phase(afull(a), (uint32_t)((u >> 1) & 1), abort_flag, p.err) &&
+                           tcx::wait_phase(d2empty, (uint32_t)((u & 1) ^ 1), abort_flag, p.err);
+          if (!__all_sync(0xffffffffu, got)) {
             ok = false;
             break;
           }
           tcx::fence_after();
+          if (tcx::elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < QD / 16; ++kk) {
-            const uint32_t koff = (uint32_t)(kk & 3) * 32u;
-            const uint64_t bd = tcx::desc_sw128(sS + (kk >> 2) * C::W_CHUNK + koff);
-            tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
-                        kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < QD / 16; ++kk) {
+              const uint32_t woff =
+                  ((uint32_t)(kk >> 2) * (uint32_t)C::W_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+              const uint64_t bd = ((uint64_t)s_hi << 32) | (uint64_t)(s_lo + woff);
+              tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
+                          kk > 0 ? 1u : 0u);
+            }
+            tcx::commit(d2full(a));
           }
-          tcx::commit(d2full(a));
+          __syncwarp();
           ++issued2;
         }
       }
       // the last products must be complete before tensor memory is freed
-      if (issued2 > 0)
+      if (issued2 > 0 && lane == 0)
         tcx::drain_wait(d2full((int)((issued2 - 1) & 1)), (uint32_t)(((issued2 - 1) >> 1) & 1));
     }
     __syncwarp();
