@@ -286,6 +286,37 @@ def scores(Q, Pit, S, c, cell, signs, norms, rnorms):
     return np.asarray(norms, dtype=np.float64)[None, :] * (mse + qjl)
 
 
+def dequantize(cell, signs, norms, rnorms, Pit, S, c):
+    """Q_prod^-1 of each code, float64 [n, d]: stage one's reconstruction plus
+    the QJL dequantizer of the residual code ("TurboQuant: bridging MSE and
+    inner product, in two stages": the QJL estimate is added back to xhat),
+    taken in the rotated frame and mapped back with the inverse of the
+    stored rotation, then scaled by the key norm:
+        khat = ||k|| * Pit^{-1} ( c[cell] + sqrt(pi/2)/m * ||r|| * S^T z ),
+    z_i = +1 where code bit i is set, else -1.  For every q,
+    <q, khat> = ||k|| (<w, c[cell]> + sqrt(pi/2)/m ||r|| <S w, z>) with
+    w = Pit^{-T} q, the estimate `scores` gives.
+
+    cell uint8 [n, d]; signs uint32 [n, m/32]; norms, rnorms [n] (float64
+    values of the stored norms or exact ones); Pit [d, d]; S [m, d]; c the
+    centroids."""
+    cell = np.asarray(cell)
+    sg = np.asarray(signs, dtype=np.uint64)
+    S = np.asarray(S, dtype=np.float64)
+    c = np.asarray(c, dtype=np.float64)
+    m, d = S.shape
+    n = cell.shape[0]
+    assert cell.shape == (n, d) and sg.shape == (n, m // 32)
+    z = np.empty((n, m))
+    for i in range(m):
+        z[:, i] = 2.0 * ((sg[:, i // 32] >> np.uint64(i % 32)) & np.uint64(1)).astype(np.float64) - 1.0
+    rn = np.asarray(rnorms, dtype=np.float64).reshape(n)
+    nk = np.asarray(norms, dtype=np.float64).reshape(n)
+    yrec = c[cell] + (SQRT_HALF_PI / m) * rn[:, None] * (z @ S)   # rows c[cell] + a S^T z
+    Pinv = np.linalg.inv(np.asarray(Pit, dtype=np.float64))
+    return nk[:, None] * (yrec @ Pinv.T)
+
+
 def decode(Q, Pit, S, c, cell, signs, norms, rnorms, V, softmax_scale: float,
            want_scores=False):
     """Decode attention with TurboQuant-prod scores.

@@ -346,6 +346,102 @@ def test_scores_equal_dequantized_inner_product():
             assert sc[j, n] == pytest.approx(Qm[j] @ krec, rel=1e-12, abs=1e-12)
 
 
+# --------------------------------------------------------------------------
+# the prod dequantizer
+
+@pytest.mark.parametrize("d,m,bits", [(16, 32, 1), (24, 64, 2), (32, 32, 3)])
+def test_dequantized_inner_product_is_the_estimator(d, m, bits):
+    # <q, Q_prod^-1(code)> is the estimate of <q, k> that scores() computes
+    # the other way round (query mapped, centroids and sketch products)
+    rng = np.random.default_rng(40 + bits)
+    c = tq.lloyd_max(d, bits)
+    Pit = tq.rotation_stored(d, 17)
+    S = oracle.sketch(m, d, 18)
+    K = rng.standard_normal((7, d)) * 1.3
+    Qm = rng.standard_normal((4, d))
+    q = tq.quantize(K, Pit, c, S)
+    nk = oracle.fp16_bits_to_f64(q["norm16"])
+    nr = oracle.fp16_bits_to_f64(q["rnorm16"])
+    khat = tq.dequantize(q["cell"], q["signs"], nk, nr, Pit, S, c)
+    assert khat.shape == K.shape
+    sc = tq.scores(Qm, Pit, S, c, q["cell"], q["signs"], nk, nr)
+    assert np.allclose(Qm @ khat.T, sc, rtol=1e-11, atol=1e-12)
+
+
+def test_dequantized_residual_part_is_the_qjl_dequantizer():
+    # khat / ||k|| mapped into the rotated frame is c[cell] plus the QJL
+    # dequantizer (the C oracle) of the residual code with the norm ||r||
+    rng = np.random.default_rng(41)
+    d, m = 32, 64
+    c = tq.lloyd_max(d, 2)
+    Pit = tq.rotation_stored(d, 19)
+    S = oracle.sketch(m, d, 20)
+    K = rng.standard_normal((6, d))
+    q = tq.quantize(K, Pit, c, S)
+    nk, nr = q["norm"], q["rnorm"]
+    khat = tq.dequantize(q["cell"], q["signs"], nk, nr, Pit, S, c)
+    qjl = oracle.dequantize(q["signs"], nr, S)
+    want = nk[:, None] * np.linalg.solve(Pit, (c[q["cell"]] + qjl).T).T
+    assert np.allclose(khat, want, rtol=1e-11, atol=1e-13)
+
+
+def test_dequantized_key_is_unbiased_over_sketches():
+    # E_S[khat] = k (exact residual, exact norms), coordinate by coordinate
+    rng = np.random.default_rng(42)
+    d = m = 32
+    c = tq.lloyd_max(d, 2)
+    Pit = tq.rotation_stored(d, 23)
+    k = rng.standard_normal(d) * 0.8
+    est = []
+    for S in _sketches(m, d, 3000, 31000):
+        q = tq.quantize(k[None, :], Pit, c, S, round_residual=False)
+        est.append(tq.dequantize(q["cell"], q["signs"], q["norm"], q["rnorm"], Pit, S, c)[0])
+    est = np.array(est)
+    se = est.std(axis=0, ddof=1) / math.sqrt(est.shape[0])
+    assert np.all(np.abs(est.mean(axis=0) - k) < 4.5 * se)
+    # stage one alone is biased: the mean is not c[cell] mapped back
+    q = tq.quantize(k[None, :], Pit, c, _sketches(m, d, 1, 31000)[0], round_residual=False)
+    mse_only = q["norm"][0] * np.linalg.solve(Pit, c[q["cell"][0]])
+    assert np.max(np.abs(mse_only - k) / se) > 10
+
+
+def test_dequantized_error_is_the_qjl_distortion_of_the_residual():
+    # exact rotation P: E_S ||k - khat||^2 = ||k||^2 ||r||^2 ((pi/2) d - 1) / m,
+    # the QJL reconstruction error of the residual (r does not depend on S)
+    rng = np.random.default_rng(43)
+    d, m = 16, 64
+    c = tq.lloyd_max(d, 1)
+    P = tq.rotation(d, 24)
+    k = rng.standard_normal(d) * 2.0
+    err2 = []
+    r2 = None
+    for S in _sketches(m, d, 3000, 41000):
+        q = tq.quantize(k[None, :], P, c, S, round_residual=False)
+        khat = tq.dequantize(q["cell"], q["signs"], q["norm"], q["rnorm"], P, S, c)[0]
+        err2.append(float(np.sum((k - khat) ** 2)))
+        r2 = float(q["rnorm"][0] ** 2)
+    err2 = np.array(err2)
+    pred = float(k @ k) * r2 * ((math.pi / 2) * d - 1) / m
+    assert abs(err2.mean() - pred) < 4.5 * err2.std(ddof=1) / math.sqrt(err2.size)
+
+
+def test_dequantized_zero_key_and_norm_scaling():
+    d, m = 16, 32
+    c = tq.lloyd_max(d, 2)
+    Pit = tq.rotation_stored(d, 25)
+    S = oracle.sketch(m, d, 26)
+    K = np.zeros((2, d))
+    K[1] = np.linspace(-1, 1, d)
+    q = tq.quantize(K, Pit, c, S)
+    khat = tq.dequantize(q["cell"], q["signs"], q["norm"], q["rnorm"], Pit, S, c)
+    assert np.all(khat[0] == 0)
+    # the code of 5 k is the code of k; khat scales with the norm
+    q5 = tq.quantize(5 * K[1:], Pit, c, S)
+    assert np.array_equal(q5["cell"], q["cell"][1:]) and np.array_equal(q5["signs"], q["signs"][1:])
+    k5 = tq.dequantize(q5["cell"], q5["signs"], q5["norm"], q5["rnorm"], Pit, S, c)
+    assert np.allclose(k5[0], 5 * khat[1], rtol=1e-12)
+
+
 def test_decode_invariants():
     rng = np.random.default_rng(14)
     d, m = 16, 32
