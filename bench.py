@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search|turbo-gqa|
-                turbo-paged-gqa]
+                turbo-paged-gqa|turbo-dequant-gqa]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -28,7 +28,9 @@ the tensor cores) and one jl_turbo_decode_attention call.
 
 The dequant-gqa workload times the explicit dequantizer: one
 jl_dequantize_keys call turning the gqa cache's codes and norms back into
-bf16 keys.
+bf16 keys.  turbo-dequant-gqa does the same for the turbo-gqa cache's
+TurboQuant-prod codes (one jl_turbo_dequantize_keys call; the reconstruction
+matrix is built once, untimed).
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload
 (independent sequences, no data-path collective), timing is the max over ranks
@@ -412,18 +414,50 @@ def run_paged(args, rank, world, local_rank):
     }
 
 
+def turbo_reconstruction_error(jl, w, codes, norms, R, bits, K, rows=65536):
+    """Measured reconstruction error of the TurboQuant-prod dequantizer on the
+    first rows of the cache, mean over keys of ||k - khat||^2, beside the QJL
+    error of the residual, mean of ||k||^2 ||r||^2 ((pi/2) d - 1) / m (its
+    expectation over Gaussian sketches).  Measurement only."""
+    n = min(rows, codes.shape[0])
+    khat = jl.jl_turbo_dequantize_keys(codes[:n], norms[:n], R, bits).double()
+    k = K.reshape(-1, w.d)[:n].double()
+    meas = ((khat - k) ** 2).sum(1)
+    nk = norms[:n, 0].double()
+    nr = norms[:n, 1].double()
+    pred = (nk * nr) ** 2 * ((math.pi / 2) * w.d - 1) / w.m
+    return {"mean_sq_error": float(meas.mean()), "predicted": float(pred.mean()),
+            "mean_rel_sq_error": float((meas / (k * k).sum(1)).mean()), "samples": n}
+
+
 def run_dequant(args, rank, world, local_rank):
-    """Explicit dequantizer over the gqa cache's codes: khat in bf16."""
+    """Explicit dequantizer over a cache's codes: khat in bf16 (QJL codes of
+    the gqa cache, or TurboQuant-prod codes of the turbo-gqa cache)."""
     import bit_jl_key_b200 as jl
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = rank_workload(args, rank)
+    turbo = w.name == "turbo-dequant-gqa"
     peak, peak_kind = load_peaks()
     S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
     K = workloads.keys(w, dev)
-    signs, norms = jl.jl_quantize_keys(K.view(-1, w.d), S)      # untimed set-up
-    recon = None if args.no_score_error else reconstruction_error(jl, w, S, signs, norms, K)
+    if turbo:                                                   # untimed set-up
+        bits = workloads.TURBO_MSE_BITS
+        Pi, Pinv = jl.jl_turbo_rotation_init(w.d, workloads.TURBO_ROTATION_SEED, device=dev)
+        signs, norms = jl.jl_turbo_quantize_keys(K.view(-1, w.d), Pi, S, bits)
+        R = jl.jl_turbo_dequant_basis(Pinv, S)
+        recon = (None if args.no_score_error
+                 else turbo_reconstruction_error(jl, w, signs, norms, R, bits, K))
+        code_bytes = (bits * w.d + w.m) // 8 + 4
+        kdim = w.d + w.m
+        api = "jl_turbo_dequantize_keys"
+    else:
+        signs, norms = jl.jl_quantize_keys(K.view(-1, w.d), S)
+        recon = None if args.no_score_error else reconstruction_error(jl, w, S, signs, norms, K)
+        code_bytes = w.m // 8 + 2
+        kdim = w.m
+        api = "jl_dequantize_keys"
     del K
     torch.cuda.empty_cache()
     n = signs.shape[0]
@@ -431,7 +465,10 @@ def run_dequant(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        jl.jl_dequantize_keys(signs, norms, S, out=out)
+        if turbo:
+            jl.jl_turbo_dequantize_keys(signs, norms, R, bits, out=out)
+        else:
+            jl.jl_dequantize_keys(signs, norms, S, out=out)
 
     for _ in range(args.warmup):
         step()
@@ -479,7 +516,7 @@ def run_dequant(args, rank, world, local_rank):
                "h2d_bytes_per_step": hS.numel() * 4 + hN.numel() * 2,
                "d2h_bytes_per_step": hOut.numel() * 2}
 
-    nbytes = n * (w.m // 8 + 2 + 2 * w.d)
+    nbytes = n * (code_bytes + 2 * w.d)
     gbs = nbytes / (ms * 1e-3) / 1e9
     traffic = ncu_traffic("dequant:" + w.name)
     return {
@@ -488,14 +525,15 @@ def run_dequant(args, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
-        "config": {"workload": f"{w.name}: {n} codes, m={w.m}, d={w.d} -> bf16 keys",
+        "config": {"workload": (f"{w.name}: {n} codes, m={w.m}, d={w.d}"
+                                + (f", {bits}-bit cells" if turbo else "") + " -> bf16 keys"),
                    "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
                    "l2": "inputs and outputs exceed L2 (126 MB); no flush"},
         "phases": {"dequantize": {"ms": ms, "keys_per_s": n / (ms * 1e-3),
                                   "algorithmic_bytes": nbytes, "GB_per_s": gbs,
                                   "frac_of_hbm_peak": gbs / peak,
-                                  "tflops": n * 2 * w.m * w.d / (ms * 1e-3) / 1e12}},
-        "roofline": {"kernel": "jl_dequantize_keys", "bound": "hbm", "achieved": gbs,
+                                  "tflops": n * 2 * kdim * w.d / (ms * 1e-3) / 1e12}},
+        "roofline": {"kernel": api, "bound": "hbm", "achieved": gbs,
                      "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
                      "frac": gbs / peak, "algorithmic_bytes_per_launch": nbytes,
                      "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
@@ -940,7 +978,7 @@ def run_ours(args, rank, world, local_rank):
         return run_search(args, rank, world, local_rank)
     if args.workload in ("paged-gqa", "turbo-paged-gqa"):
         return run_paged(args, rank, world, local_rank)
-    if args.workload == "dequant-gqa":
+    if args.workload in ("dequant-gqa", "turbo-dequant-gqa"):
         return run_dequant(args, rank, world, local_rank)
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -1169,6 +1207,20 @@ def oracle_sample(w: workloads.Workload):
 
         def run():
             oracle.dequantize(sig, n64, S64)
+        return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
+    if w.name == "turbo-dequant-gqa":
+        from oracle import turbo as tq
+        n = 131072
+        bits = workloads.TURBO_MSE_BITS
+        Kf = workloads.keys(w.with_(B=1, Hkv=1, T=n)).view(-1, w.d).double().numpy()
+        c = tq.lloyd_max(w.d, bits)                           # set-up, untimed
+        Pit = tq.rotation_stored(w.d, workloads.TURBO_ROTATION_SEED)
+        q = tq.quantize(Kf, Pit, c, S64)
+        nk = oracle.fp16_bits_to_f64(q["norm16"])
+        nr = oracle.fp16_bits_to_f64(q["rnorm16"])
+
+        def run():
+            tq.dequantize(q["cell"], q["signs"], nk, nr, Pit, S64, c)
         return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
     if w.name in ("turbo-gqa", "turbo-paged-gqa"):
         from oracle import turbo as tq

@@ -55,7 +55,8 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_search_topk", "jl_turbo_codebook", "jl_turbo_rotation_workspace_bytes",
             "jl_turbo_rotation_init", "jl_turbo_quantize_keys", "jl_turbo_decode_workspace_bytes",
             "jl_turbo_decode_attention", "jl_turbo_decode_paged_workspace_bytes",
-            "jl_turbo_decode_attention_paged", "jl_test_drop_copies", "jl_build_flags")
+            "jl_turbo_decode_attention_paged", "jl_turbo_dequant_basis",
+            "jl_turbo_dequantize_keys", "jl_test_drop_copies", "jl_build_flags")
 
 # device error codes (jl_device_error)
 JL_DERR_TC_WAIT_TIMEOUT = 1
@@ -134,6 +135,10 @@ def load():
     L.jl_turbo_decode_attention_paged.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32,
                                                   i32, vp, i32, vp, i32, i32, i32, i64, i32, i32,
                                                   i32, ctypes.c_float, vp, vp, vp, sz, vp]
+    L.jl_turbo_dequant_basis.restype = i32
+    L.jl_turbo_dequant_basis.argtypes = [vp, vp, i32, i32, vp, vp]
+    L.jl_turbo_dequantize_keys.restype = i32
+    L.jl_turbo_dequantize_keys.argtypes = [vp, vp, i64, vp, i32, i32, i32, vp, vp]
     L.jl_device_error.restype = i32
     L.jl_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.jl_build_flags.restype = i32
@@ -533,6 +538,49 @@ def jl_turbo_quantize_keys(K, Pi, S, mse_bits: int, codes=None, norms=None, stre
                                     _ptr(S), m, d, mse_bits, _ptr(codes), _ptr(norms),
                                     _stream(K, stream)), "jl_turbo_quantize_keys")
     return codes, norms
+
+
+def jl_turbo_dequant_basis(Pinv, S, out=None, stream=None):
+    """R = [Pinv | Pinv S^T] as binary16 [d, d + m]: the reconstruction matrix
+    of jl_turbo_dequantize_keys."""
+    L = load()
+    m, d = S.shape
+    _need_cuda(Pinv, S, out)
+    assert Pinv.dtype == torch.float32 and Pinv.shape == (d, d) and Pinv.is_contiguous()
+    assert S.dtype == torch.bfloat16 and S.is_contiguous()
+    if out is None:
+        out = torch.empty((d, d + m), dtype=torch.float16, device=S.device)
+    assert out.dtype == torch.float16 and out.shape == (d, d + m) and out.is_contiguous()
+    _check(L.jl_turbo_dequant_basis(_ptr(Pinv), _ptr(S), m, d, _ptr(out), _stream(S, stream)),
+           "jl_turbo_dequant_basis")
+    return out
+
+
+def jl_turbo_dequantize_keys(codes, norms, basis, mse_bits: int, out=None, stream=None):
+    """khat = ||k|| Pi^{-1} (c[cell] + sqrt(pi/2)/m ||r|| S^T z) for each
+    TurboQuant-prod code (codes int32 [..., words], norms fp16 [..., 2],
+    basis from jl_turbo_dequant_basis): [n, d] bf16."""
+    L = load()
+    d = basis.shape[0]
+    m = basis.shape[1] - d
+    words = turbo_code_words(mse_bits, m, d)
+    _need_cuda(codes, norms, basis, out)
+    assert codes.dtype == torch.int32 and codes.shape[-1] == words
+    assert norms.dtype == torch.float16 and norms.shape[-1] == 2
+    assert basis.dtype == torch.float16
+    codes2 = codes.reshape(-1, words)
+    n = codes2.shape[0]
+    assert norms.numel() == 2 * n
+    for t in (codes2, norms, basis):
+        if not t.is_contiguous():
+            raise ValueError("dequantize inputs must be contiguous")
+    if out is None:
+        out = torch.empty((n, d), dtype=torch.bfloat16, device=codes.device)
+    assert out.dtype == torch.bfloat16 and out.numel() == n * d and out.is_contiguous()
+    _check(L.jl_turbo_dequantize_keys(_ptr(codes2), _ptr(norms), n, _ptr(basis), m, d, mse_bits,
+                                      _ptr(out), _stream(codes, stream)),
+           "jl_turbo_dequantize_keys")
+    return out
 
 
 def jl_turbo_decode_workspace_bytes(B, Hq, Hkv, T, m, d, mse_bits) -> int:

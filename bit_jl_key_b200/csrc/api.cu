@@ -466,6 +466,29 @@ int jl_turbo_decode_attention_paged(
   return from_cuda(jlk::launch_turbo_decode_paged(p, mse_bits, a, t, (cudaStream_t)stream));
 }
 
+int jl_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
+                           uint16_t *basis, jl_stream_t stream) {
+  if (m != 128 || d != 128) return JL_ERR_UNSUPPORTED;
+  if (!Pinv || !S || !basis) return JL_ERR_INVALID_ARG;
+  if (!aligned(Pinv, 16) || !aligned(S, 16) || !aligned(basis, 16)) return JL_ERR_INVALID_ARG;
+  return from_cuda(jlk::launch_turbo_dequant_basis(Pinv, S, m, d, basis, (cudaStream_t)stream));
+}
+
+int jl_turbo_dequantize_keys(const uint32_t *codes, const uint16_t *norms, int64_t n_keys,
+                             const uint16_t *basis, int m, int d, int mse_bits, uint16_t *out,
+                             jl_stream_t stream) {
+  if (n_keys < 0) return JL_ERR_INVALID_ARG;
+  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+    return JL_ERR_UNSUPPORTED;
+  if (n_keys == 0) return JL_OK;
+  if (!codes || !norms || !basis || !out) return JL_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(norms, 4) || !aligned(basis, 16) || !aligned(out, 16))
+    return JL_ERR_INVALID_ARG;
+  if (n_keys >= ((int64_t)1 << 40)) return JL_ERR_UNSUPPORTED;
+  return from_cuda(jlk::launch_turbo_dequantize(codes, norms, n_keys, basis, m, d, mse_bits, out,
+                                                (cudaStream_t)stream));
+}
+
 int jl_test_drop_copies(int enable, uint64_t wait_limit_ns) {
   if (enable != 0 && enable != 1) return JL_ERR_INVALID_ARG;
   unsigned long long lim = wait_limit_ns ? (unsigned long long)wait_limit_ns : jlk::WAIT_LIMIT_NS;

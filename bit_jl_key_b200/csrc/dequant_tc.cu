@@ -1,179 +1,143 @@
-// dequant_tc.cu -- explicit QJL dequantizer on the 5th-generation tensor cores.
+// dequant_tc.cu -- explicit dequantizers on the 5th-generation tensor cores.
 //
-// Dequantizer Q^-1(z) = sqrt(pi/2)/d * S^T z of "The Geometry of Forgetting:
-// How Three Papers Cracked KV Cache Quantization", section "QJL: one bit, zero
-// parameters, unbiased inner products", taken with m sketch rows and with the
-// stored norm restoring the magnitude (same page, "PolarQuant" section):
+// QJL codes: the dequantizer Q^-1(z) = sqrt(pi/2)/d * S^T z of "The Geometry
+// of Forgetting: How Three Papers Cracked KV Cache Quantization", section
+// "QJL: one bit, zero parameters, unbiased inner products", taken with m
+// sketch rows and with the stored norm restoring the magnitude (same page,
+// "PolarQuant" section):
 //     khat = sqrt(pi/2)/m * ||k|| * S^T z,   z_i = +1 if code bit i is set.
 // The reconstruction error E||k - khat||^2 is the page's D_mse for this
 // quantizer.
 //
-// For a tile of 128 codes, Khat = Z S is a dense bf16 contraction (M = 128
-// codes, N = d, K = m): tcgen05.mma with Z read from tensor memory, S^T from
+// TurboQuant-prod codes (same page, "TurboQuant: bridging MSE and inner
+// product, in two stages": the QJL estimate of the residual is added back to
+// the stage-one reconstruction), in the rotated frame, mapped back with the
+// inverse of the stored rotation and scaled by the key norm:
+//     khat = ||k|| * Pi^{-1} ( c[cell] + sqrt(pi/2)/m * ||r|| * S^T z )
+//          = ||k|| * R a,   R = [Pi^{-1} | Pi^{-1} S^T]  (d x (d + m)),
+//     a = [c[cell_0 .. cell_{d-1}] ; alpha z],  alpha = sqrt(pi/2)/m * ||r||.
+// R is built once (turbo_basis_kernel); a holds binary16 centroids and
+// +-alpha, so a key costs one fp16 contraction of length d + m.
+//
+// For a tile of 128 codes, Khat = A B is a dense contraction (M = 128 codes,
+// N = d, K = m or d + m): tcgen05.mma with A read from tensor memory, B from
 // shared memory (128-byte swizzle, K-major) and the fp32 accumulator in
 // tensor memory.
-//   * Z (the A operand) is expanded from the code bits by threads straight
-//     into tensor memory, one K-chunk of 64 coordinates (32 columns of bf16
-//     pairs, one tcgen05.st per thread) at a time, into a ring of chunks; it
-//     never passes through shared memory.  A bf16 pair holds coordinates
-//     (p, p + 16) of a 32-bit code word, built with one shift and one LOP3:
-//     ((w << (15 - p)) & 0x80008000) ^ 0xBF80BF80.
-//   * S^T (the B operand, N = d rows of K = m) stays resident; its K order is
-//     the same permutation of each 32-coordinate block, so the contraction is
-//     unchanged.
-//   * The epilogue scales row r by sqrt(pi/2)/m * ||k_r||, rounds to bf16,
-//     writes its 32 rows into a 128-byte-swizzled staging tile in shared
-//     memory and stores them with bulk-tensor copies (which also clip rows
-//     past the last code).
-//   * An expander thread copies its code row of the tile two ahead into a
-//     shared-memory ring with cp.async while it expands the current one.
+//   * A is expanded from the code bits by threads straight into tensor
+//     memory, one K-chunk of 64 coordinates (32 columns of 16-bit pairs, one
+//     tcgen05.st per thread) at a time, into a ring of chunks; it never
+//     passes through shared memory.  A pair holds coordinates (p, p + 16) of
+//     a 32-bit code word.  QJL: bf16 +-1 with one shift and one LOP3,
+//     ((w << (15 - p)) & 0x80008000) ^ 0xBF80BF80.  TurboQuant: the cell's
+//     centroid as binary16, its magnitude chosen by the XNOR of each lower
+//     plane with the top plane (the codebook is odd-symmetric) and its sign
+//     by the top plane; then the residual signs as +-alpha.
+//   * B (S^T, or R^T for TurboQuant) stays resident; its K order is the same
+//     permutation of each 32-coordinate block, so the contraction is
+//     unchanged.  TurboQuant interleaves its K-chunks (centroid chunk i at
+//     2 i, sign chunk i at 2 i + 1) so both expander parts do equal work.
+//   * The epilogue scales row r by sqrt(pi/2)/m * ||k_r|| (QJL) or ||k_r||
+//     (TurboQuant), rounds to bf16, writes its 32 rows into a
+//     128-byte-swizzled staging tile in shared memory and stores them with
+//     bulk-tensor copies (which also clip rows past the last code).
+//   * An expander thread copies its part of its code row of the tile two
+//     ahead into a shared-memory ring with cp.async while it expands the
+//     current one.
 //
 // One persistent CTA per SM, 13 warps with fixed roles:
 //   warps 0-7  expand: warp w writes TMEM lane quadrant w % 4 (code rows
 //              32 (w % 4) .. + 31 of the tile) for part w / 4 of the tile's
 //              K-chunks (the first or the second half), so two warps expand
-//              each row at once; each thread copies its half of its code
+//              each row at once; each thread copies its part of its code
 //              row two tiles ahead.
 //   warps 8-11 epilogue: warp w reads TMEM lane quadrant w % 4.
 //   warp 12    owns the TMEM allocation; one elected lane issues the MMAs of a tile
 //              into one of two accumulators and commits them to the barriers
-//              that free the Z chunks and publish the accumulator.
+//              that free the A chunks and publish the accumulator.
 // Every mbarrier wait is bounded (about 2 s of GPU time); a wait that runs
 // out records DERR_TC_WAIT_TIMEOUT, raises a shared abort flag, and the CTA
 // still frees its TMEM.
 #include "jl_common.cuh"
 #include "jl_internal.h"
+#include "jl_tc.cuh"
 
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 namespace jlk {
+
+using namespace tcx;
 namespace dq {
 
 constexpr int BM = 128;          // codes per tile (MMA M)
-constexpr int CHUNK_K = 64;      // coordinates per Z chunk
-constexpr int CHUNK_COLS = CHUNK_K / 2;  // TMEM columns of a Z chunk (bf16 pairs)
+constexpr int CHUNK_K = 64;      // coordinates per A chunk
+constexpr int CHUNK_COLS = CHUNK_K / 2;  // TMEM columns of an A chunk (16-bit pairs)
 constexpr int EXP_PARTS = 2;     // expander warps per TMEM lane quadrant
 constexpr int EXP_WARPS = 4 * EXP_PARTS, EPI_WARPS = 4;
 constexpr int MMA_WARP = EXP_WARPS + EPI_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int CODE_SLOTS = 3;    // code rows in flight: the tile and two ahead
-constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
+constexpr uint32_t SIGN2 = 0x80008000u;  // sign bits of a 16-bit pair
 
-template <int M, int D>
+// TB = 0: QJL codes (m/32 sign words, one binary16 norm per key).
+// TB = 1..3: TurboQuant-prod codes (TB cell planes of d bits, then m sign
+// bits; a binary16 (||k||, ||r||) pair per key); d = m = 128.
+template <int M, int D, int TB>
 struct Cfg {
-  static constexpr int KCH = M / CHUNK_K;             // Z chunks per tile (>= 1)
-  static constexpr int ST_CHUNK = D * 128;            // one K-chunk of S^T
-  static constexpr int ST_BYTES = M * D * 2;
+  static constexpr bool TURBO = TB > 0;
+  static constexpr int K = TURBO ? D + M : M;         // contraction length
+  static constexpr int KCH = K / CHUNK_K;             // A chunks per tile (>= 1)
+  static constexpr int B_CHUNK = D * 128;             // one K-chunk of B
+  static constexpr int B_BYTES = K * D * 2;
   // output staging: per epilogue warp, 32 rows x d bf16 as D/64 swizzled
-  // boxes of 32 x 128 B; two buffers per warp when they fit beside 4 Z chunks
+  // boxes of 32 x 128 B, two buffers per warp
   static constexpr int OBOX = 32 * 128;
   static constexpr int OWARP = (D / 64) * OBOX;
-  static constexpr int CODE_ROW = M / 8;              // bytes per code
+  static constexpr int KP = (KCH + EXP_PARTS - 1) / EXP_PARTS;  // chunks per part
+  // code bytes of one part of a row in the ring: QJL, the part's 2 words per
+  // chunk; TurboQuant, 8 bytes of every cell plane and of the sign words,
+  // then the norm pair (padded to 8)
+  static constexpr int PART_BYTES = TURBO ? 8 * (TB + 1) + 8 : KP * 8;
+  static constexpr int CODE_ROW = TURBO ? EXP_PARTS * PART_BYTES : M / 8;
+  static constexpr int CODE_BYTES_G = TURBO ? (TB * D + M) / 8 : M / 8;  // per key in HBM
   static constexpr int C_BYTES = CODE_SLOTS * BM * CODE_ROW;
   static constexpr int OBUF = 2;
   static constexpr int O_BYTES = EPI_WARPS * OBUF * OWARP;
-  // tensor memory: accumulators at columns [0, 2d), Z chunks after them
+  // tensor memory: accumulators at columns [0, 2d), A chunks after them
   static constexpr int ACC = 2;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int Z_COL0 = ACC * D;
-  static constexpr int RING_RAW = (TMEM_COLS - Z_COL0) / CHUNK_COLS;
+  static constexpr int A_COL0 = ACC * D;
+  static constexpr int RING_RAW = (TMEM_COLS - A_COL0) / CHUNK_COLS;
   static constexpr int RING = RING_RAW > 8 ? 8 : RING_RAW;
-  static constexpr int OFF_O = ST_BYTES;
+  static constexpr int OFF_O = B_BYTES;
   static constexpr int OFF_C = OFF_O + O_BYTES;
   static constexpr int OFF_BAR = OFF_C + C_BYTES;
   static constexpr int NBAR = 2 * RING + 2 * ACC;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + align slack
-  static_assert(M % CHUNK_K == 0 && RING >= 2, "Z ring");
-  static_assert(Z_COL0 + RING * CHUNK_COLS <= TMEM_COLS, "tensor memory columns");
-  static constexpr int CODE_WORDS = M / 32;
+  static_assert(K % CHUNK_K == 0 && RING >= 2, "A ring");
+  static_assert(A_COL0 + RING * CHUNK_COLS <= TMEM_COLS, "tensor memory columns");
+  static_assert(!TURBO || (D == 128 && M == 128 && TB <= 3), "TurboQuant shapes");
+  static_assert(!TURBO || KCH == 2 * EXP_PARTS, "one centroid and one sign chunk per part");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 struct Params {
-  const uint32_t *signs;  // n x m/32
-  const uint16_t *norms;  // n binary16
-  const uint16_t *S;      // m x d bf16
+  const uint32_t *codes;  // n x code words
+  const uint16_t *norms;  // n binary16 (QJL) or n x 2 (TurboQuant)
+  const uint16_t *B;      // QJL: S, m x d bf16; TurboQuant: R, d x (d + m) binary16
   int64_t n, num_tiles;
   float coef;             // sqrt(pi/2) / m
+  uint32_t mag[4];        // TurboQuant: centroid magnitudes a_0 < .. (binary16 pairs)
+  uint32_t dmag01, dmag23;  // a_0 ^ a_1, a_2 ^ a_3 (binary16 bits)
   int *err;
 };
 
-// --------------------------------------------------------------------------
-// PTX wrappers
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-// generic-proxy writes to shared memory -> visible to the tensor core
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-// K-major operand, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;
-  d |= (uint64_t)(1024u >> 4) << 32;
-  d |= (uint64_t)1u << 46;
-  d |= (uint64_t)2u << 61;
-  return d;
-}
-// D (tensor memory) += A (tensor memory, one row per lane) * B (shared memory)
-__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 32 consecutive columns of this thread's lane <- v
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
-      "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
-      "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-        "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
-        "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-// wait for this thread's TMEM loads, tied to the registers of one load
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
-                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
-                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
-                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
-               :
+
+// 4-byte async copy global -> shared; src_bytes < 4 zero-fills.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src,
+                                           int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst),
+               "l"(src), "r"(src_bytes)
                : "memory");
 }
 
@@ -199,27 +163,9 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
 }
 
-// Bounded wait on a barrier phase; false when the wait ran out or another
-// role gave up (then the error word is set and the shared abort flag raised).
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
-                                           volatile int *abort_flag, int *err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > WAIT_NS) {
-        *abort_flag = 1;
-        record_device_error(err, DERR_TC_WAIT_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
 
 // Position of coordinate i of a 32-coordinate block in the operand's K
-// order: bf16 pair j holds coordinates j (low half) and j + 16 (high half).
+// order: 16-bit pair j holds coordinates j (low half) and j + 16 (high half).
 __host__ __device__ __forceinline__ int k_slot(int i) {
   const int j = i & 15, h = (i >> 4) & 1;
   return (i & ~31) + 2 * j + h;
@@ -233,20 +179,53 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k, int rows) {
   return (uint32_t)(kc * rows * 128 + r * 128 + ((((kin >> 3) ^ (r & 7)) << 4)) + (kin & 7) * 2);
 }
 
-template <int M, int D>
+// TurboQuant centroid pairs of one code word per plane: pair j holds the
+// binary16 centroids of coordinates j and j + 16 of the 32 the words cover.
+// The cell's top plane bit gives the sign (set: positive); each lower plane
+// bit XNOR the top one gives a bit of the magnitude's index (the codebook is
+// c[H + i] = a_i, c[H - 1 - i] = -a_i).
+template <int TB>
+__device__ __forceinline__ void centroid_pairs(const uint32_t (&w)[TB], const Params &p,
+                                               uint32_t *z) {
+  if constexpr (TB == 1) {
+    const uint32_t k = SIGN2 | p.mag[0];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) z[j] = ((w[0] << (15 - j)) & SIGN2) ^ k;
+  } else if constexpr (TB == 2) {
+    const uint32_t x = ~(w[0] ^ w[1]);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t mag = p.mag[0] ^ (((x >> j) & 0x00010001u) * p.dmag01);
+      z[j] = mag ^ (((w[1] << (15 - j)) & SIGN2) ^ SIGN2);
+    }
+  } else {
+    const uint32_t x0 = ~(w[0] ^ w[2]), x1 = ~(w[1] ^ w[2]);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t u0 = (x0 >> j) & 0x00010001u;
+      const uint32_t lo = p.mag[0] ^ (u0 * p.dmag01);
+      const uint32_t hi = p.mag[2] ^ (u0 * p.dmag23);
+      const uint32_t sel = ((x1 >> j) & 0x00010001u) * 0xFFFFu;
+      const uint32_t mag = (hi & sel) | (lo & ~sel);
+      z[j] = mag ^ (((w[2] << (15 - j)) & SIGN2) ^ SIGN2);
+    }
+  }
+}
+
+template <int M, int D, int TB>
 __global__ void __launch_bounds__(THREADS, 1)
     dequant_tc_kernel(const __grid_constant__ CUtensorMap tmap_out, const Params p) {
-  using C = Cfg<M, D>;
+  using C = Cfg<M, D, TB>;
   extern __shared__ uint8_t dq_smem_raw[];
   const uint32_t raw = smem_u32(dq_smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *gbase = dq_smem_raw + (base - raw);
-  const uint32_t sST = base;
+  const uint32_t sB = base;
   const uint32_t bar0 = base + C::OFF_BAR;
-  auto zfull_bar = [&](int s) { return bar0 + 8u * s; };
-  auto zempty_bar = [&](int s) { return bar0 + 8u * (C::RING + s); };
-  auto afull_bar = [&](int a) { return bar0 + 8u * (2 * C::RING + a); };
-  auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * C::RING + C::ACC + a); };
+  auto afull_bar = [&](int s) { return bar0 + 8u * s; };               // A chunk written
+  auto aempty_bar = [&](int s) { return bar0 + 8u * (C::RING + s); };  // A chunk consumed
+  auto accfull_bar = [&](int a) { return bar0 + 8u * (2 * C::RING + a); };
+  auto accempty_bar = [&](int a) { return bar0 + 8u * (2 * C::RING + C::ACC + a); };
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(gbase + C::OFF_BAR + C::NBAR * 8);
   volatile int *abort_flag =
       reinterpret_cast<volatile int *>(gbase + C::OFF_BAR + C::NBAR * 8 + 4);
@@ -256,12 +235,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::RING; ++s) {
-      mbar_init(zfull_bar(s), 4);          // one arrive per quadrant's expander warp
-      mbar_init(zempty_bar(s), 1);         // MMA commit
+      mbar_init(afull_bar(s), 4);            // one arrive per quadrant's expander warp
+      mbar_init(aempty_bar(s), 1);           // MMA commit
     }
     for (int a = 0; a < C::ACC; ++a) {
-      mbar_init(afull_bar(a), 1);          // MMA commit
-      mbar_init(aempty_bar(a), EPI_WARPS); // epilogue warps
+      mbar_init(accfull_bar(a), 1);          // MMA commit
+      mbar_init(accempty_bar(a), EPI_WARPS); // epilogue warps
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -274,30 +253,51 @@ __global__ void __launch_bounds__(THREADS, 1)
         "n"(C::TMEM_COLS)
         : "memory");
   }
-  // S^T into shared memory, once: 16-byte unit (row n, K positions 8u..8u+7)
-  // per thread and step; K position k holds coordinate i with k_slot(i) = k
-  for (int e = threadIdx.x; e < D * (M / 8); e += THREADS) {
-    const int n = e % D, u = e / D;
-    uint32_t pk[4];
+  // B into shared memory, once: 16-byte unit (row n, K positions 8u..8u+7)
+  // per thread and step; K position k of a chunk holds coordinate i with
+  // k_slot(i) = k
+  if constexpr (!C::TURBO) {
+    for (int e = threadIdx.x; e < D * (M / 8); e += THREADS) {
+      const int n = e % D, u = e / D;
+      uint32_t pk[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint16_t h2[2];
+      for (int q = 0; q < 4; ++q) {
+        uint16_t h2[2];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int k = 8 * u + 2 * q + hh;           // K position
-        const int blk = k & ~31, jj = (k & 31) >> 1, h = k & 1;
-        const int i = blk + jj + 16 * h;            // coordinate at k
-        h2[hh] = __ldg(p.S + (int64_t)i * D + n);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int k = 8 * u + 2 * q + hh;           // K position
+          const int blk = k & ~31, jj = (k & 31) >> 1, h = k & 1;
+          const int i = blk + jj + 16 * h;            // coordinate at k
+          h2[hh] = __ldg(p.B + (int64_t)i * D + n);   // S[i][n]
+        }
+        pk[q] = (uint32_t)h2[0] | ((uint32_t)h2[1] << 16);
       }
-      pk[q] = (uint32_t)h2[0] | ((uint32_t)h2[1] << 16);
+      *reinterpret_cast<uint4 *>(gbase + sw128_offset(n, 8 * u, D)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    *reinterpret_cast<uint4 *>(gbase + sw128_offset(n, 8 * u, D)) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  } else {
+    // R row n is K-contiguous: the unit's low halves are 4 consecutive
+    // columns, its high halves the 4 columns 16 later
+    for (int e = threadIdx.x; e < D * (C::K / 8); e += THREADS) {
+      const int n = e % D, ug = e / D;
+      const int kc = ug >> 3, u = ug & 7;
+      const int col0 = ((kc & 1) ? D + 64 * (kc >> 1) : 64 * (kc >> 1)) + 32 * (u >> 2) +
+                       4 * (u & 3);
+      const int64_t off = (int64_t)n * (D + M) + col0;
+      uint2 lo = make_uint2(0u, 0u), hi = make_uint2(0u, 0u);
+      if (JL_IN_RANGE(p.err, off, 20, (int64_t)D * (D + M))) {
+        lo = __ldg(reinterpret_cast<const uint2 *>(p.B + off));
+        hi = __ldg(reinterpret_cast<const uint2 *>(p.B + off + 16));
+      }
+      *reinterpret_cast<uint4 *>(gbase + sw128_offset(n, 8 * ug, D)) =
+          make_uint4(__byte_perm(lo.x, hi.x, 0x5410), __byte_perm(lo.x, hi.x, 0x7632),
+                     __byte_perm(lo.y, hi.y, 0x5410), __byte_perm(lo.y, hi.y, 0x7632));
+    }
   }
   fence_async_smem();
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int64_t ntiles = p.num_tiles;
 
@@ -307,23 +307,38 @@ __global__ void __launch_bounds__(THREADS, 1)
     // code words of the tile two ahead are copied meanwhile
     const int q = warp & 3, pt = warp >> 2;
     const int r = 32 * q + lane;
-    constexpr int KP = (C::KCH + EXP_PARTS - 1) / EXP_PARTS;  // chunks per part
+    constexpr int KP = C::KP;
     const int kc0 = pt * KP;
     const int nk = C::KCH - kc0 < KP ? C::KCH - kc0 : KP;
     bool ok = nk > 0;
-    const uint32_t pbytes = (uint32_t)(KP * 8);             // 2 code words per chunk
-    const uint32_t crow = base + C::OFF_C + r * C::CODE_ROW + pt * pbytes;
+    const uint32_t crow =
+        base + C::OFF_C + r * C::CODE_ROW + pt * (C::TURBO ? C::PART_BYTES : KP * 8);
     auto code_slot = [&](int slot) { return crow + (uint32_t)(slot * BM * C::CODE_ROW); };
     auto copy_part = [&](uint32_t dst, int64_t row) {
-      const bool live = row < p.n && JL_IN_RANGE(p.err, row * (M / 8) + pt * pbytes, KP * 8,
-                                                 p.n * (M / 8));
-      const uint8_t *src = reinterpret_cast<const uint8_t *>(p.signs + (live ? row : 0) * (M / 32)) +
-                           pt * pbytes;
-      if constexpr (KP * 8 >= 16) {
+      if constexpr (!C::TURBO) {
+        const bool live = row < p.n && JL_IN_RANGE(p.err, row * (M / 8) + pt * KP * 8, KP * 8,
+                                                   p.n * (M / 8));
+        const uint8_t *src =
+            reinterpret_cast<const uint8_t *>(p.codes + (live ? row : 0) * (M / 32)) + pt * KP * 8;
+        if constexpr (KP * 8 >= 16) {
 #pragma unroll
-        for (int u = 0; u < KP * 8 / 16; ++u) cp_async_16(dst + 16 * u, src + 16 * u, live ? 16 : 0);
+          for (int u = 0; u < KP * 8 / 16; ++u) cp_async_16(dst + 16 * u, src + 16 * u, live ? 16 : 0);
+        } else {
+          cp_async_8(dst, src, live ? 8 : 0);
+        }
       } else {
-        cp_async_8(dst, src, live ? 8 : 0);
+        // 8 bytes (the part's 64 coordinates) of each cell plane and of the
+        // sign words, then the norm pair
+        const bool live = row < p.n &&
+                          JL_IN_RANGE(p.err, row * C::CODE_BYTES_G, C::CODE_BYTES_G,
+                                      p.n * C::CODE_BYTES_G) &&
+                          JL_IN_RANGE(p.err, 2 * row, 2, 2 * p.n);
+        const int64_t rr = live ? row : 0;
+        const uint8_t *src =
+            reinterpret_cast<const uint8_t *>(p.codes) + rr * C::CODE_BYTES_G + 8 * pt;
+#pragma unroll
+        for (int pl = 0; pl <= TB; ++pl) cp_async_8(dst + 8 * pl, src + pl * (D / 8), live ? 8 : 0);
+        cp_async_4(dst + 8 * (TB + 1), p.norms + 2 * rr, live ? 4 : 0);
       }
       cp_async_commit();
     };
@@ -335,15 +350,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     // chunk it * KCH + kc0, advanced by KCH per tile without a division
     int rs0 = kc0 % C::RING;
     uint32_t rph0 = (uint32_t)((kc0 / C::RING) & 1);
+    constexpr int NW = C::TURBO ? 2 * TB + 3 : 2 * KP;  // words of a part's slot
     for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
       copy_part(code_slot(cs == 0 ? CODE_SLOTS - 1 : cs - 1),
                 (tile + (int64_t)(CODE_SLOTS - 1) * gridDim.x) * BM + r);
       cp_async_wait<CODE_SLOTS - 1>();  // this tile's words have landed
-      uint32_t cur[2 * KP];
+      uint32_t cur[NW];
       {
         const uint8_t *src = gbase + (code_slot(cs) - base);
 #pragma unroll
-        for (int i = 0; i < 2 * KP; ++i) cur[i] = reinterpret_cast<const uint32_t *>(src)[i];
+        for (int i = 0; i < NW; ++i) cur[i] = reinterpret_cast<const uint32_t *>(src)[i];
+      }
+      // TurboQuant: +-alpha pairs for the sign chunk, alpha = sqrt(pi/2)/m ||r||
+      // rounded to binary16 (rows past the end have a zero norm pair)
+      uint32_t kalpha = 0;
+      if constexpr (C::TURBO) {
+        const float alpha =
+            p.coef * __half2float(__ushort_as_half((uint16_t)(cur[2 * TB + 2] >> 16)));
+        const uint32_t a16 = (uint32_t)__half_as_ushort(__float2half_rn(alpha));
+        kalpha = SIGN2 | (a16 << 16) | a16;
       }
       int s = rs0;
       uint32_t ph = rph0;
@@ -354,26 +379,43 @@ __global__ void __launch_bounds__(THREADS, 1)
           s = 0;
           ph ^= 1u;
         }
-        if (!wait_phase(zempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
+        if (!wait_phase(aempty_bar(s), ph ^ 1u, abort_flag, p.err)) {
           ok = false;
           break;
         }
         // the chunk's 32 TMEM columns of row r: column 16 h + j holds the
-        // pair (j, j + 16) of code word 2 kc + h
+        // pair (j, j + 16) of the chunk's code word h
         uint32_t z[32];
+        if constexpr (!C::TURBO) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t w = cur[2 * kk + half];  // rows past the end expand a zero code
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t w = cur[2 * kk + half];  // rows past the end expand a zero code
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            z[16 * half + j] = ((w << (15 - j)) & 0x80008000u) ^ 0xBF80BF80u;
+            for (int j = 0; j < 16; ++j)
+              z[16 * half + j] = ((w << (15 - j)) & SIGN2) ^ 0xBF80BF80u;
+          }
+        } else if (kk == 0) {                       // centroid chunk pt
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t w[TB];
+#pragma unroll
+            for (int pl = 0; pl < TB; ++pl) w[pl] = cur[2 * pl + half];
+            centroid_pairs<TB>(w, p, z + 16 * half);
+          }
+        } else {                                    // sign chunk pt
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t w = cur[2 * TB + half];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) z[16 * half + j] = ((w << (15 - j)) & SIGN2) ^ kalpha;
+          }
         }
-        tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) +
-                      (uint32_t)(C::Z_COL0 + s * CHUNK_COLS), z);
-        tmem_st_wait();
-        tc_fence_before();
+        st32(tmem_base + ((uint32_t)(32 * q) << 16) +
+                      (uint32_t)(C::A_COL0 + s * CHUNK_COLS), z);
+        st_wait();
+        fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(zfull_bar(s));
+        if (lane == 0) mbar_arrive(afull_bar(s));
       }
       // next tile: its first chunk of this part is KCH chunks later
       rs0 += C::KCH;
@@ -394,16 +436,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int a = (int)(t & 1);
       const uint32_t aph = (uint32_t)((t >> 1) & 1);
       const int64_t row = tile * BM + 32 * q + lane;
-      const bool live = row < p.n && JL_IN_RANGE(p.err, row, 1, p.n);
-      const float f = live ? p.coef * __half2float(__ushort_as_half(__ldg(p.norms + row))) : 0.f;
+      float f = 0.f;
+      if constexpr (!C::TURBO) {
+        if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n))
+          f = p.coef * __half2float(__ushort_as_half(__ldg(p.norms + row)));
+      } else {
+        if (row < p.n && JL_IN_RANGE(p.err, 2 * row, 1, 2 * p.n))
+          f = __half2float(__ushort_as_half(__ldg(p.norms + 2 * row)));
+      }
       const int ob = (int)(t % C::OBUF);
       uint8_t *stage = gbase + C::OFF_O + (ew * C::OBUF + ob) * C::OWARP;
       // the staging buffer's previous stores must have read it
       if (lane == 0) bulk_wait_read<C::OBUF - 1>();
       __syncwarp();
-      if (!wait_phase(afull_bar(a), aph, abort_flag, p.err)) break;
+      if (!wait_phase(accfull_bar(a), aph, abort_flag, p.err)) break;
       __syncwarp();
-      tc_fence_after();
+      fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * D);
       // 32 columns: scale, round to bf16, stage as 4 units of 16 B in box
       // c0/64, row `lane`
@@ -423,21 +471,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       // the loads are double-buffered: group g + 1 is in flight while g is
       // emitted
       uint32_t va[32], vb[32];
-      tmem_ld32(trow, va);
+      ld32(trow, va);
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 64) {
-        tmem_ld_wait(va);
-        tmem_ld32(trow + c0 + 32, vb);
+        ld_wait(va);
+        ld32(trow + c0 + 32, vb);
         emit(va, c0);
-        tmem_ld_wait(vb);
-        if (c0 + 64 < D) tmem_ld32(trow + c0 + 64, va);
+        ld_wait(vb);
+        if (c0 + 64 < D) ld32(trow + c0 + 64, va);
         emit(vb, c0 + 32);
       }
-      tc_fence_before();
+      fence_before();
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(aempty_bar(a));
+        mbar_arrive(accempty_bar(a));
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
           tma_store_2d(&tmap_out, smem_u32(stage + bx * C::OBOX), bx * 64,
@@ -451,11 +499,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------- MMA issuer: the whole warp runs the loop, one elected
     // lane issues; the B descriptor is the base plus a 32-bit start-address add
     {
-      constexpr uint32_t idesc = (1u << 4)                  // D: fp32
-                                 | (1u << 7) | (1u << 10)   // A, B: bf16
-                                 | ((uint32_t)(D >> 3) << 17)   // N
-                                 | ((uint32_t)(BM >> 4) << 24); // M
-      const uint64_t b0 = smem_desc_sw128(sST);
+      constexpr uint32_t idesc = idesc_f16(BM, D, C::TURBO ? 0 : 1);  // fp16 or bf16
+      const uint64_t b0 = desc_sw128(sB);
       const uint32_t b_hi = (uint32_t)(b0 >> 32), b_lo0 = (uint32_t)b0;
       int rs = 0;
       uint32_t rph = 0;
@@ -464,9 +509,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++t) {
         const int a = (int)(t & 1u);
         const uint32_t aph = (t >> 1) & 1u;
-        if (!__all_sync(0xffffffffu, wait_phase(aempty_bar(a), aph ^ 1u, abort_flag, p.err)))
+        if (!__all_sync(0xffffffffu, wait_phase(accempty_bar(a), aph ^ 1u, abort_flag, p.err)))
           break;
-        tc_fence_after();
+        fence_after();
         for (int kc = 0; kc < C::KCH; ++kc) {
           const int s = rs;
           const uint32_t ph = rph;
@@ -474,49 +519,43 @@ __global__ void __launch_bounds__(THREADS, 1)
             rs = 0;
             rph ^= 1u;
           }
-          if (!__all_sync(0xffffffffu, wait_phase(zfull_bar(s), ph, abort_flag, p.err))) {
+          if (!__all_sync(0xffffffffu, wait_phase(afull_bar(s), ph, abort_flag, p.err))) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          uint32_t el;
-          asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
-                       : "=r"(el));
-          if (el) {
-            const uint32_t blo = b_lo0 + (uint32_t)kc * (uint32_t)(C::ST_CHUNK >> 4);
+          fence_after();
+          if (elect_one()) {
+            const uint32_t blo = b_lo0 + (uint32_t)kc * (uint32_t)(C::B_CHUNK >> 4);
 #pragma unroll
             for (int kk = 0; kk < CHUNK_K / 16; ++kk) {  // K = 16: 8 columns of A
-              const uint32_t atm = tmem_base + (uint32_t)(C::Z_COL0 + s * CHUNK_COLS + kk * 8);
+              const uint32_t atm = tmem_base + (uint32_t)(C::A_COL0 + s * CHUNK_COLS + kk * 8);
               const uint64_t bdesc = ((uint64_t)b_hi << 32) | (uint64_t)(blo + (uint32_t)(kk * 2));
-              mma_bf16_ts(tmem_base + a * D, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem_base + a * D, atm, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(zempty_bar(s));
+            commit(aempty_bar(s));
           }
           __syncwarp();
         }
         if (!ok) break;
-        uint32_t el2;
-        asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
-                     : "=r"(el2));
-        if (el2) mma_commit(afull_bar(a));
+        if (elect_one()) commit(accfull_bar(a));
         __syncwarp();
       }
       // drain: the last accumulator's MMAs must be complete before TMEM is freed
       if (t > 0 && ok && lane == 0) {
         const uint32_t tl = t - 1;
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(afull_bar((int)(tl & 1u)), (tl >> 1) & 1u) &&
-               globaltimer() - t0 < WAIT_NS) {
+        while (!mbar_try_wait(accfull_bar((int)(tl & 1u)), (tl >> 1) & 1u) &&
+               globaltimer() - t0 < WAIT_LIMIT_NS) {
         }
       }
       __syncwarp();
     }
   }
 
-  tc_fence_before();
+  fence_before();
   __syncthreads();
   if (warp == MMA_WARP) {
-    tc_fence_after();
+    fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
                  "n"(C::TMEM_COLS)
                  : "memory");
@@ -536,23 +575,43 @@ static bool make_out_map(CUtensorMap *map, uint16_t *out, int64_t n, int d) {
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int M, int D>
-cudaError_t launch_t(const uint32_t *signs, const uint16_t *norms, int64_t n,
-                     const uint16_t *S, uint16_t *out, cudaStream_t stream) {
-  using C = Cfg<M, D>;
-  int *err = device_error_ptr();
-  if (!err) return cudaErrorInvalidSymbol;
+template <int M, int D, int TB>
+cudaError_t launch_t(Params p, uint16_t *out, cudaStream_t stream) {
+  using C = Cfg<M, D, TB>;
+  p.err = device_error_ptr();
+  if (!p.err) return cudaErrorInvalidSymbol;
   CUtensorMap tmap;
-  if (!make_out_map(&tmap, out, n, D)) return cudaErrorInvalidValue;
-  Params p{signs, norms, S, n, (n + BM - 1) / BM,
-           (float)(1.2533141373155002512 / (double)M), err};
-  cudaError_t e = cudaFuncSetAttribute(dequant_tc_kernel<M, D>,
+  if (!make_out_map(&tmap, out, p.n, D)) return cudaErrorInvalidValue;
+  p.num_tiles = (p.n + BM - 1) / BM;
+  p.coef = (float)(1.2533141373155002512 / (double)M);
+  cudaError_t e = cudaFuncSetAttribute(dequant_tc_kernel<M, D, TB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t sms = device_sm_count();
   const int64_t grid = p.num_tiles < sms ? p.num_tiles : sms;
-  dequant_tc_kernel<M, D><<<(int)grid, THREADS, C::SMEM, stream>>>(tmap, p);
+  dequant_tc_kernel<M, D, TB><<<(int)grid, THREADS, C::SMEM, stream>>>(tmap, p);
   return cudaGetLastError();
+}
+
+// R = [Pinv | Pinv S^T] rounded to binary16: one thread per element, the
+// products accumulated in fp32
+constexpr int BASIS_THREADS = 256;
+__global__ void __launch_bounds__(BASIS_THREADS)
+    turbo_basis_kernel(const float *__restrict__ Pinv, const uint16_t *__restrict__ S, int m,
+                       int d, uint16_t *__restrict__ basis, int *err) {
+  const int idx = blockIdx.x * BASIS_THREADS + threadIdx.x;
+  const int cols = d + m;
+  if (idx >= d * cols) return;
+  const int j = idx / cols, c = idx % cols;
+  float v = 0.f;
+  if (c < d) {
+    if (JL_IN_RANGE(err, j * d + c, 1, d * d)) v = Pinv[j * d + c];
+  } else {
+    const int l = c - d;
+    if (JL_IN_RANGE(err, j * d, d, d * d) && JL_IN_RANGE(err, l * d, d, m * d))
+      for (int i = 0; i < d; ++i) v = fmaf(Pinv[j * d + i], bf16_bits_to_f32(S[l * d + i]), v);
+  }
+  if (JL_IN_RANGE(err, idx, 1, d * cols)) basis[idx] = __half_as_ushort(__float2half_rn(v));
 }
 
 }  // namespace dq
@@ -560,12 +619,54 @@ cudaError_t launch_t(const uint32_t *signs, const uint16_t *norms, int64_t n,
 cudaError_t launch_dequantize_tc(const uint32_t *signs, const uint16_t *norms, int64_t n,
                                  const uint16_t *S, int m, int d, uint16_t *out,
                                  cudaStream_t stream) {
+  dq::Params p{};
+  p.codes = signs;
+  p.norms = norms;
+  p.B = S;
+  p.n = n;
 #define JL_CASE(MM, DD) \
-  if (m == MM && d == DD) return dq::launch_t<MM, DD>(signs, norms, n, S, out, stream);
+  if (m == MM && d == DD) return dq::launch_t<MM, DD, 0>(p, out, stream);
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
 #undef JL_CASE
   return cudaErrorNotSupported;
+}
+
+cudaError_t launch_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
+                                       uint16_t *basis, cudaStream_t stream) {
+  if (m != 128 || d != 128) return cudaErrorNotSupported;
+  int *err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  const int total = d * (d + m);
+  dq::turbo_basis_kernel<<<(total + dq::BASIS_THREADS - 1) / dq::BASIS_THREADS,
+                           dq::BASIS_THREADS, 0, stream>>>(Pinv, S, m, d, basis, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_turbo_dequantize(const uint32_t *codes, const uint16_t *norms, int64_t n,
+                                    const uint16_t *basis, int m, int d, int bits,
+                                    uint16_t *out, cudaStream_t stream) {
+  if (m != 128 || d != 128) return cudaErrorNotSupported;
+  float mag[4], thr[3];
+  if (!turbo_magnitudes(d, bits, mag, thr)) return cudaErrorNotSupported;
+  dq::Params p{};
+  p.codes = codes;
+  p.norms = norms;
+  p.B = basis;
+  p.n = n;
+  uint32_t h[4];
+  for (int i = 0; i < 4; ++i) {
+    h[i] = (uint32_t)__half_as_ushort(__float2half_rn(mag[i]));
+    p.mag[i] = h[i] | (h[i] << 16);
+  }
+  p.dmag01 = h[0] ^ h[1];
+  p.dmag23 = h[2] ^ h[3];
+  switch (bits) {
+    case 1: return dq::launch_t<128, 128, 1>(p, out, stream);
+    case 2: return dq::launch_t<128, 128, 2>(p, out, stream);
+    case 3: return dq::launch_t<128, 128, 3>(p, out, stream);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 }  // namespace jlk

@@ -33,6 +33,15 @@ cudaError_t launch_dequantize_tc(const uint32_t *signs, const uint16_t *norms, i
                                  const uint16_t *S, int m, int d, uint16_t *out,
                                  cudaStream_t stream);
 
+// TurboQuant-prod dequantizer (dequant_tc.cu): the reconstruction matrix
+// R = [Pinv | Pinv S^T] in binary16 (d x (d + m)), and khat = ||k|| R a on
+// the tensor cores (d = m = 128).
+cudaError_t launch_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
+                                       uint16_t *basis, cudaStream_t stream);
+cudaError_t launch_turbo_dequantize(const uint32_t *codes, const uint16_t *norms, int64_t n,
+                                    const uint16_t *basis, int m, int d, int bits,
+                                    uint16_t *out, cudaStream_t stream);
+
 // u = S q for nq queries (fp32 [nq][m]).
 cudaError_t launch_query_projection(const void *Q, bool q_f32, const uint16_t *S, float *U,
                                     int nq, int m, int d, cudaStream_t stream);

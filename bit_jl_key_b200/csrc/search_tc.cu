@@ -53,11 +53,14 @@
 // DERR_TC_WAIT_TIMEOUT and the CTA still frees its TMEM.
 #include "jl_common.cuh"
 #include "jl_internal.h"
+#include "jl_tc.cuh"
 
 #include <math.h>
 
 namespace jlk {
 namespace srch {
+
+using namespace tcx;
 
 constexpr int QM = 128;                        // queries per pass (MMA M)
 constexpr int BN = 256;                        // index vectors per tile (MMA N)
@@ -72,7 +75,6 @@ constexpr int CODE_SLOTS = 3;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_CTAS = 256;                  // bounds the per-CTA lists
 constexpr int MERGE_THREADS = 256;
-constexpr unsigned long long WAIT_NS = WAIT_LIMIT_NS;
 
 template <int M>
 struct Cfg {
@@ -113,107 +115,7 @@ struct Params {
   int *err;
 };
 
-// --------------------------------------------------------------------------
-// PTX wrappers
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;
-  d |= (uint64_t)(1024u >> 4) << 32;
-  d |= (uint64_t)1u << 46;
-  d |= (uint64_t)2u << 61;
-  return d;
-}
-// D (tensor memory) += A (tensor memory) * B (shared memory), fp16 inputs
-__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D (tensor memory) += A (shared memory) * B (shared memory), fp16 inputs
-__device__ __forceinline__ void mma_f16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-        "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-        "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
-        "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]),
-                 "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
-                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]),
-                 "+r"(v[27]), "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
-               :
-               : "memory");
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
-      "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
-      "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-}
 
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity,
-                                           volatile int *abort_flag, int *err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > WAIT_NS) {
-        *abort_flag = 1;
-        record_device_error(err, DERR_TC_WAIT_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
 
 // Copy code rows `row0` and `row0 + 128` (M/8 bytes each) into shared memory
 // with cp.async, zero fill past the end, as one commit group.
@@ -365,9 +267,9 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         "n"(TMEM_COLS)
         : "memory");
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
   // ---- U (warps 4-7, query qi = 32 (warp % 4) + lane): fp16 pairs
@@ -406,15 +308,15 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
           *reinterpret_cast<uint4 *>(rowp + ((u ^ (qi & 7)) << 4)) =
               make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
       } else {
-        tmem_st32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        st32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
       }
     }
     if constexpr (C::U_SMEM) fence_async_smem();
-    else tmem_st_wait();
+    else st_wait();
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
 
   const int64_t ntiles = p.num_tiles;
   auto tile_at = [&](int64_t j) { return p.tile0 + j * p.tile_step; };  // rows past N: zero codes
@@ -521,7 +423,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       const int ab = (int)(tt % (uint32_t)C::NACC);
       if (!wait_phase(dfull_bar(ab), (tt / (uint32_t)C::NACC) & 1u, abort_flag, p.err)) break;
       __syncwarp();
-      tc_fence_after();
+      fence_after();
       const uint32_t trow =
           tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(C::D_COL + ab * BN);
       // the tile's 8 groups of 32 columns: while the accumulator is held only
@@ -561,17 +463,17 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
       // taken; groups that may qualify are parked and inserted after the
       // accumulator is released (or when all rows are in use)
       uint32_t va[32], vb[32];
-      tmem_ld32(trow, va);
+      ld32(trow, va);
 #pragma unroll 1
       for (int g = 0; g < BN / 32; g += 2) {
-        tmem_ld_wait(va);
-        tmem_ld32(trow + 32 * (g + 1), vb);
+        ld_wait(va);
+        ld32(trow + 32 * (g + 1), vb);
         scan_group(va, g);
-        tmem_ld_wait(vb);
+        ld_wait(vb);
         if (g + 2 < BN / 32) {
-          tmem_ld32(trow + 32 * (g + 2), va);
+          ld32(trow + 32 * (g + 2), va);
         } else {  // the accumulator is read: free it
-          tc_fence_before();
+          fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(dempty_bar(ab));
         }
@@ -603,8 +505,8 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
                                  | (0u << 7) | (0u << 10)         // A, B: fp16
                                  | ((uint32_t)(BN >> 3) << 17)    // N
                                  | ((uint32_t)(QM >> 4) << 24);   // M
-      const uint64_t z0 = smem_desc_sw128(sZ);
-      const uint64_t u0 = smem_desc_sw128(base + C::OFF_U);
+      const uint64_t z0 = desc_sw128(sZ);
+      const uint64_t u0 = desc_sw128(base + C::OFF_U);
       const uint32_t z_hi = (uint32_t)(z0 >> 32), z_lo0 = (uint32_t)z0;
       const uint32_t u_hi = (uint32_t)(u0 >> 32), u_lo0 = (uint32_t)u0;
       int rs = 0;
@@ -618,7 +520,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
                                                 ((tt / (uint32_t)C::NACC) & 1u) ^ 1u,
                                                 abort_flag, p.err)))
           break;
-        tc_fence_after();
+        fence_after();
         const uint32_t dt = tmem_base + (uint32_t)C::D_COL + ab * (uint32_t)BN;
         for (int kc = 0; kc < C::KCH; ++kc) {
           const int s = rs;
@@ -631,7 +533,7 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
             ok = false;
             break;
           }
-          tc_fence_after();
+          fence_after();
           const uint32_t zlo = z_lo0 + (uint32_t)s * (uint32_t)(CHUNK_BYTES >> 4);
           const uint32_t ulo = u_lo0 + (uint32_t)kc * (uint32_t)(C::U_CHUNK >> 4);
           uint32_t el;
@@ -643,12 +545,12 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
               const uint64_t bdesc = ((uint64_t)z_hi << 32) | (uint64_t)(zlo + (uint32_t)(kk * 2));
               const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
               if constexpr (C::U_SMEM)
-                mma_f16_ss(dt, ((uint64_t)u_hi << 32) | (uint64_t)(ulo + (uint32_t)(kk * 2)),
+                mma_ss(dt, ((uint64_t)u_hi << 32) | (uint64_t)(ulo + (uint32_t)(kk * 2)),
                            bdesc, idesc, acc);
               else
-                mma_f16_ts(dt, tmem_base + (uint32_t)(kc * 32 + kk * 8), bdesc, idesc, acc);
+                mma_ts(dt, tmem_base + (uint32_t)(kc * 32 + kk * 8), bdesc, idesc, acc);
             }
-            mma_commit(zempty_bar(s));
+            commit(zempty_bar(s));
           }
           __syncwarp();
         }
@@ -656,24 +558,24 @@ __global__ void __launch_bounds__(THREADS, 1) search_tc_kernel(const Params p) {
         uint32_t el2;
         asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
                      : "=r"(el2));
-        if (el2) mma_commit(dfull_bar((int)ab));
+        if (el2) commit(dfull_bar((int)ab));
         __syncwarp();
       }
       if (tt > 0 && ok && lane == 0) {  // the last tile's MMAs complete before TMEM is freed
         const unsigned long long t0 = globaltimer();
         const int lb = (int)((tt - 1) % C::NACC);
         while (!mbar_try_wait(dfull_bar(lb), ((tt - 1) / (uint32_t)C::NACC) & 1u) &&
-               globaltimer() - t0 < WAIT_NS) {
+               globaltimer() - t0 < WAIT_LIMIT_NS) {
         }
       }
       __syncwarp();
     }
   }
 
-  tc_fence_before();
+  fence_before();
   __syncthreads();
   if (warp == MMA_WARP) {
-    tc_fence_after();
+    fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem_base),
                  "n"(TMEM_COLS)
                  : "memory");

@@ -473,6 +473,54 @@ JL_API int jl_turbo_decode_attention_paged(
     float *scores, void *workspace, size_t workspace_bytes, jl_stream_t stream);
 
 /*
+ * jl_turbo_dequant_basis -- the reconstruction matrix of the TurboQuant-prod
+ * dequantizer, R = [Pi^{-1} | Pi^{-1} S^T] (d x (d + m)), so that
+ *     khat = ||k|| * R [ c[cell_0 .. cell_{d-1}] ; sqrt(pi/2)/m ||r|| z ]
+ * (jl_turbo_dequantize_keys).  Build it once per (rotation, sketch) pair.
+ *   Pinv  : in, device, d x d fp32 query map of jl_turbo_rotation_init
+ *           (the inverse of the stored bf16 Pi), 16-byte aligned.
+ *   S     : in, device, m x d bf16 residual sketch, 16-byte aligned.
+ *   basis : out, device, d x (d + m) binary16, row-major: basis[j][i] =
+ *           Pinv[j][i] for i < d, basis[j][d + l] = sum_i Pinv[j][i] S[l][i]
+ *           (fp32 products and sums), each rounded to nearest binary16;
+ *           16-byte aligned, d (d + m) elements.
+ * Supported: d = m = 128.
+ * Errors: JL_ERR_INVALID_ARG (null or misaligned pointer), JL_ERR_UNSUPPORTED
+ * (d, m), JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
+                                  uint16_t *basis, jl_stream_t stream);
+
+/*
+ * jl_turbo_dequantize_keys -- explicit TurboQuant-prod dequantizer Q_prod^-1.
+ * Defines: "The Geometry of Forgetting: How Three Papers Cracked KV Cache
+ * Quantization", section "TurboQuant: bridging MSE and inner product, in two
+ * stages" (the QJL estimate of the residual added back to the stage-one
+ * reconstruction), in the rotated frame, mapped back with the inverse of the
+ * stored rotation and scaled by the key norm:
+ *     khat_t = ||k_t|| * Pi^{-1} ( c[cell_t] + sqrt(pi/2)/m ||r_t|| S^T z_t ),
+ * z_ti = +1 if residual bit i is set, so <q, khat_t> is the TurboQuant-prod
+ * estimate s(q, k_t) of jl_turbo_decode_attention.  Computed as
+ * ||k_t|| * basis a_t on the tensor cores (binary16 operands, fp32
+ * accumulation) with a_t = [ binary16(c[cell_ti]) ; binary16(sqrt(pi/2)/m
+ * ||r_t||) z_t ] (the centroids of jl_turbo_codebook rounded to binary16;
+ * ||r_t|| the stored binary16 norm, the product in fp32 then rounded).
+ *   codes : in, device, n_keys x ((mse_bits d + m)/32) uint32
+ *           (jl_turbo_quantize_keys layout), 16-byte aligned.
+ *   norms : in, device, n_keys x 2 binary16 (||k||, ||r||), 4-byte aligned.
+ *   basis : in, device, d x (d + m) binary16 from jl_turbo_dequant_basis,
+ *           16-byte aligned.
+ *   out   : out, device, n_keys x d bf16 (round to nearest), 16-byte aligned.
+ * Supported: d = m = 128, mse_bits 1 to JL_TURBO_MAX_MSE_BITS.  n_keys == 0
+ * is a no-op.
+ * Errors: JL_ERR_INVALID_ARG (null or misaligned pointer, n_keys < 0),
+ * JL_ERR_UNSUPPORTED (d, m, mse_bits, n_keys >= 2^40), JL_ERR_CUDA.
+ */
+JL_API int jl_turbo_dequantize_keys(const uint32_t *codes, const uint16_t *norms,
+                                    int64_t n_keys, const uint16_t *basis, int m, int d,
+                                    int mse_bits, uint16_t *out, jl_stream_t stream);
+
+/*
  * jl_device_error -- synchronise `stream`, then read and clear the device
  * error word of the current device (0 = no fault reported).  *code receives
  * the word.  Returns JL_OK, JL_ERR_DEVICE when the word was non-zero, or

@@ -25,3 +25,16 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_error_after_gpu_test(request):
+    """Every GPU test ends with the library's device error word clear: a
+    kernel that recorded an error (an expired wait, or an out-of-range index
+    in the index-checking build) fails the test that launched it."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import bit_jl_key_b200 as jl
+    if jl._lib is not None:
+        assert jl.jl_device_error() == 0, "device error word set after the test"

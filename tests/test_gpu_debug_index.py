@@ -4,8 +4,8 @@ The debug build (``python -m bit_jl_key_b200.build --debug-index``, compiled
 with -DJL_DEBUG_INDEX into libjlkey_debug.so) checks every global access its
 kernels make through a raw pointer against the extent that the call's shapes
 give that buffer; an access outside it is skipped and reported as
-JL_DERR_INDEX through jl_device_error.  Each parity module asserts at teardown
-that jl_device_error() is 0, so a pass here means the small cases of every
+JL_DERR_INDEX through jl_device_error.  Every GPU test asserts at teardown
+(tests/conftest.py) that jl_device_error() is 0, so a pass here means the small cases of every
 kernel touched memory only inside the buffers they were given, and still
 matched the oracle.  (Tensor-map copies are bounded by the hardware against
 their maps and need no software check.)  The full-size cases are left out.
@@ -21,7 +21,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 pytestmark = pytest.mark.gpu
 
 SUITES = ["tests/test_gpu_parity.py", "tests/test_gpu_paged.py", "tests/test_gpu_dequant.py",
-          "tests/test_gpu_search.py", "tests/test_gpu_turbo.py", "tests/test_gpu_turbo_paged.py"]
+          "tests/test_gpu_search.py", "tests/test_gpu_turbo.py", "tests/test_gpu_turbo_paged.py",
+          "tests/test_gpu_turbo_dequant.py"]
 
 
 def test_parity_suites_pass_under_index_checks():

@@ -31,6 +31,8 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
            the rotated key (rotation seed 1) plus QJL on the residual with a
            128-row sketch (3 bits per coordinate plus two binary16 norms).
   turbo-paged-gqa  the paged-gqa serving step with TurboQuant-prod keys.
+  turbo-dequant-gqa  the turbo-gqa cache's 2,097,152 TurboQuant-prod codes
+           (2-bit cells, m=128) and norm pairs turned back into bf16 keys.
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -119,10 +121,12 @@ TURBO_MSE_BITS = 2
 TURBO_ROTATION_SEED = 1
 # the paged serving step of paged-gqa with TurboQuant-prod keys (same data)
 TURBO_PAGED_GQA = PAGED_GQA.with_(name="turbo-paged-gqa", m=128)
+# the turbo-gqa cache's codes turned back into bf16 keys (same data)
+TURBO_DEQUANT_GQA = TURBO_GQA.with_(name="turbo-dequant-gqa")
 SEARCH_K = 10
 
 ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA,
-                           SEARCH, TURBO_GQA, TURBO_PAGED_GQA)}
+                           SEARCH, TURBO_GQA, TURBO_PAGED_GQA, TURBO_DEQUANT_GQA)}
 
 
 def sweep_points():
