@@ -393,21 +393,39 @@ __device__ __forceinline__ float neg_scaled(float d, float ninv) {
   return r;
 }
 
-// residual of the coordinate whose accumulator value is d; pushes its bits
-// into chain g
+// Two fp32 lanes in one 64-bit register (Blackwell's packed fp32 pipe:
+// one instruction rounds each lane exactly as the scalar form would).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// magnitude of the centroid of -y = neg (pushing the magnitude bits of its
+// search levels into chain g)
 template <int TB>
-__device__ __forceinline__ float cell_residual(float d, float ninv, const Magnitudes &mg,
-                                               PlaneChains<TB> &ch, int g) {
-  const float neg = neg_scaled(d, ninv);
-  ch.top[g] = __funnelshift_l(__float_as_uint(neg), ch.top[g], 1);
+__device__ __forceinline__ float cell_magnitude(float neg, const Magnitudes &mg,
+                                                PlaneChains<TB> &ch, int g) {
   const float ay = fabsf(neg);
-  float amag;
   if constexpr (TB == 1) {
-    amag = mg.a[0];
+    return mg.a[0];
   } else if constexpr (TB == 2) {
     const float d0 = mg.p[0] - ay;
     ch.mag[0][g] = __funnelshift_l(__float_as_uint(d0), ch.mag[0][g], 1);
-    amag = d0 < 0.f ? mg.a[1] : mg.a[0];
+    return d0 < 0.f ? mg.a[1] : mg.a[0];
   } else {
     const float d1 = mg.p[1] - ay;
     const bool m1 = d1 < 0.f;
@@ -415,11 +433,32 @@ __device__ __forceinline__ float cell_residual(float d, float ninv, const Magnit
     ch.mag[1][g] = __funnelshift_l(__float_as_uint(d1), ch.mag[1][g], 1);
     ch.mag[0][g] = __funnelshift_l(__float_as_uint(d0), ch.mag[0][g], 1);
     const bool m0 = d0 < 0.f;
-    amag = m1 ? (m0 ? mg.a[3] : mg.a[2]) : (m0 ? mg.a[1] : mg.a[0]);
+    return m1 ? (m0 ? mg.a[3] : mg.a[2]) : (m0 ? mg.a[1] : mg.a[0]);
   }
-  // y - (+-a_mu): the centroid takes the sign of y, negative for y = +-0
-  const float sgn = __uint_as_float((__float_as_uint(neg) & 0x80000000u) | 0x3F800000u);
-  return fmaf(sgn, amag, -neg);
+}
+
+// Cell and residual of the adjacent coordinates (jj, jj + 1) of chain g with
+// packed fp32 arithmetic: -y of both from one fma, both residuals from one
+// subtraction (the centroid carries the sign of y, so y - c = +-a - neg),
+// and both squares into the residual norm's two lanes; the bits go into the
+// chains higher coordinate first, as the scalar order does.  Returns the
+// residual pair (lane 0: coordinate jj).
+template <int TB>
+__device__ __forceinline__ uint64_t cell_residual_pair(uint64_t d2, uint64_t ninv2,
+                                                       const Magnitudes &mg, PlaneChains<TB> &ch,
+                                                       int g, uint64_t &rs2) {
+  const uint64_t neg2 = f32x2_fma(d2, ninv2, 0ull);  // + (+0, +0): a -0 product becomes +0
+  float n0, n1;
+  f32x2_unpack(neg2, n0, n1);
+  ch.top[g] = __funnelshift_l(__float_as_uint(n1), ch.top[g], 1);
+  const float a1 = cell_magnitude<TB>(n1, mg, ch, g);
+  ch.top[g] = __funnelshift_l(__float_as_uint(n0), ch.top[g], 1);
+  const float a0 = cell_magnitude<TB>(n0, mg, ch, g);
+  const float s0 = __uint_as_float(__float_as_uint(a0) | (__float_as_uint(n0) & 0x80000000u));
+  const float s1 = __uint_as_float(__float_as_uint(a1) | (__float_as_uint(n1) & 0x80000000u));
+  const uint64_t rr2 = f32x2_sub(f32x2_pack(s0, s1), neg2);
+  rs2 = f32x2_fma(rr2, rr2, rs2);
+  return rr2;
 }
 
 template <int TB>
@@ -620,7 +659,8 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       __syncwarp();
       tcx::fence_after();
       uint32_t planes[TB][2];
-      float rs0 = 0.f, rs1 = 0.f;
+      uint64_t rs2 = 0ull;                       // residual sum of squares, two lanes
+      const uint64_t ninv2 = f32x2_pack(ninv, ninv);
       uint32_t va[32], vb[32];
       const uint32_t dcol = tq + (uint32_t)(C::D1_COL + h * 128);
       const uint32_t acol = tq + (uint32_t)(C::A2_COL + h * 64);
@@ -632,19 +672,20 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < (TB > 1 ? TB - 1 : 1); ++k) pc.mag[k][g] = 0u;
         }
-        // coordinate 8 g + jj, highest first so that the funnel shifts
-        // leave bit jj of chain g at position jj
+        // coordinates 8 g + jj and 8 g + jj + 1, highest first so that the
+        // funnel shifts leave bit jj of chain g at position jj
 #pragma unroll
-        for (int jj = 7; jj >= 0; --jj)
+        for (int jj = 6; jj >= 0; jj -= 2)
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const int e = 8 * g + jj;
-            const float rr = cell_residual<TB>(__uint_as_float(v[e]), ninv, mg, pc, g);
-            if (g & 1)
-              rs1 = fmaf(rr, rr, rs1);
-            else
-              rs0 = fmaf(rr, rr, rs0);
-            v[e] = __float_as_uint(rr);
+            const uint64_t rr2 = cell_residual_pair<TB>(
+                f32x2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), ninv2, mg, pc, g,
+                rs2);
+            float r0, r1;
+            f32x2_unpack(rr2, r0, r1);
+            v[e] = __float_as_uint(r0);
+            v[e + 1] = __float_as_uint(r1);
           }
         uint32_t pk[16];
 #pragma unroll
@@ -684,6 +725,8 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       if (lane == 0) mbar_arrive(afull(h));
       if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n)) {
         const uint32_t n16 = __half_as_ushort(__float2half_rn(nk));
+        float rs0, rs1;
+        f32x2_unpack(rs2, rs0, rs1);
         const uint32_t r16 = __half_as_ushort(__float2half_rn(sqrtf(rs0 + rs1)));
         p.norms[row] = n16 | (r16 << 16);
       }
