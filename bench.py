@@ -59,6 +59,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -142,16 +143,45 @@ def ncu_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """nvidia-smi clock/throttle samples (every 100 ms, read by a thread) for
+    the timed region.  ``region_start`` / ``region_end`` bracket the region
+    (host times taken after a device synchronize on both sides, so they bound
+    the device's work).  A region shorter than a few sampling intervals gets
+    at most one sample of its own; ``region_end(top_up=fn)`` then keeps the
+    GPU under the same load, running fn (one untimed step) until the region
+    and its continuation hold ``min_samples`` samples.  The summary says how
+    many samples fell inside the region and how many in the continuation."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
         self.proc = None
-        self.out = None
+        self.samples = []          # (host time, parsed sample)
+        self.lock = threading.Lock()
+        self.thread = None
+        self.t0 = self.t1 = None
+        self.t_end = None
+
+    def feed(self, line: str, t=None):
+        """Parse one nvidia-smi CSV line (ignored when malformed)."""
+        c = [x.strip() for x in line.split(",")]
+        if len(c) < 9:
+            return
+        try:
+            smp = (float(c[1]), float(c[2]), float(c[3]),
+                   [n for n, v in zip(self.NAMES, c[5:9]) if v.lower().startswith("active")])
+        except ValueError:
+            return
+        with self.lock:
+            self.samples.append((time.monotonic() if t is None else t, smp))
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            self.feed(line)
 
     def __enter__(self):
         try:
@@ -161,41 +191,61 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
-        time.sleep(0.3)
+            return self
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        deadline = time.monotonic() + 5.0      # the first sample: nvidia-smi is up
+        while time.monotonic() < deadline and not self._count(0.0, None):
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+            if self.thread is not None:
+                self.thread.join(timeout=5)
+
+    def _count(self, t_from, t_to):
+        with self.lock:
+            return sum(1 for t, _ in self.samples if t >= t_from and (t_to is None or t <= t_to))
+
+    def region_start(self):
+        self.t0 = time.monotonic()
+        self.t1 = self.t_end = None
+
+    def region_end(self, top_up=None, min_samples=3, max_s=3.0):
+        self.t1 = time.monotonic()
+        if top_up is not None and self.proc is not None:
+            stop = self.t1 + max_s
+            while self._count(self.t0, None) < min_samples and time.monotonic() < stop:
+                top_up()
+                torch.cuda.synchronize()
+        self.t_end = time.monotonic()
 
     def summary(self):
-        if not self.out:
+        with self.lock:
+            samples = list(self.samples)
+        if self.t0 is not None:
+            t1 = self.t1 if self.t1 is not None else float("inf")
+            t_end = self.t_end if self.t_end is not None else t1
+            inside = [x for t, x in samples if self.t0 <= t <= t1]
+            after = [x for t, x in samples if t1 < t <= t_end]
+        else:
+            inside, after = [x for _, x in samples], []
+        used = inside + after
+        if not used:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sms, maxs, reasons, power = [], [], set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.strip().splitlines():
-            c = [x.strip() for x in line.split(",")]
-            if len(c) < 9:
-                continue
-            try:
-                sms.append(float(c[1]))
-                maxs.append(float(c[2]))
-                power.append(float(c[3]))
-            except ValueError:
-                continue
-            for n, v in zip(names, c[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sms:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
-                "reasons": sorted(reasons), "samples": len(sms),
-                "power_w_max": max(power) if power else None}
+        reasons = sorted({n for x in used for n in x[3]})
+        return {"sm_mhz": statistics.median(x[0] for x in used),
+                "sm_max_mhz": max(x[1] for x in used), "reasons": reasons,
+                "samples": len(used), "samples_in_region": len(inside),
+                "samples_same_load_after": len(after), "interval_ms": 100,
+                "power_w_max": max(x[2] for x in used)}
 
 
 def reduce_max_over_ranks(x: float, world: int, device) -> float:
@@ -338,11 +388,13 @@ def run_paged(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         _barrier(world, dev)
+        clk.region_start()
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         _barrier(world, dev)
+        clk.region_end(top_up=step)
     ms_step = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
     d_ms = ms_step
     if jl.jl_device_error() != 0:
@@ -479,11 +531,13 @@ def run_dequant(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         _barrier(world, dev)
+        clk.region_start()
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         _barrier(world, dev)
+        clk.region_end(top_up=step)
     ms = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
     if jl.jl_device_error() != 0:
         raise RuntimeError("device error in the timed region")
@@ -579,11 +633,13 @@ def run_search(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         _barrier(world, dev)
+        clk.region_start()
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         _barrier(world, dev)
+        clk.region_end(top_up=step)
     ms = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
     if jl.jl_device_error() != 0:
         raise RuntimeError("device error in the timed region")
@@ -702,11 +758,13 @@ def run_turbo(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         _barrier(world, dev)
+        clk.region_start()
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         _barrier(world, dev)
+        clk.region_end(top_up=step)
         q_ms = timed_loop(quantize, args.steps)
         d_ms = timed_loop(decode_call, args.steps)
         _barrier(world, dev)
@@ -894,7 +952,7 @@ def roofline_of(phase, rec, w, peak, peak_kind, full_size=True, n_keys=None):
     return r
 
 
-def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error):
+def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error, clk=None):
     """One more workload on one GPU: quantize every key, then one decode step
     over the compressed cache (prefill: quantize only).  Returns a record with
     the step time, per-phase rates and rooflines (and, for the sketch-size
@@ -932,7 +990,11 @@ def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
+    if clk is not None:
+        clk.region_start()
     ms = _timed_loop(stream, step, steps)
+    if clk is not None:
+        clk.region_end(top_up=step)
     q_ms = _timed_loop(stream, quantize, steps)
     d_ms = _timed_loop(stream, decode_call, steps) if decode else 0.0
     if jl.jl_device_error() != 0:
@@ -945,6 +1007,8 @@ def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error)
                          for ph in phases},
            "l2": "inputs exceed L2 (126 MB); no flush" if n_keys * w.d * 2 > 126e6
                  else "inputs fit in L2; latency-bound parity workload"}
+    if clk is not None:
+        rec["clocks"] = clk.summary()
     if w.name == "prefill":
         rec["quantize_tokens_per_s"] = w.T / (q_ms * 1e-3)
         rec["quantize_tokens_per_s_note"] = ("tokens of all 32 layers x 8 KV heads per second "
@@ -1045,11 +1109,13 @@ def run_ours(args, rank, world, local_rank):
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         barrier()
+        clk.region_start()
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         barrier()
+        clk.region_end(top_up=step)
         q_ms = timed_loop(quantize, args.steps)
         d_ms = timed_loop(decode_call, args.steps) if decode else 0.0
         barrier()
@@ -1165,14 +1231,15 @@ def measure_other_configs(jl, dev, args, peak, peak_kind):
     with ClockSampler(dev.index or 0) as clk:
         for w in other_configs():
             rec = measure_config(jl, w, dev, steps, warmup, peak, peak_kind,
-                                 with_score_error=(w.name == "sweep" and not args.no_score_error))
+                                 with_score_error=(w.name == "sweep" and not args.no_score_error),
+                                 clk=clk)
             cb = getattr(args, "config_baselines", {}).get(config_key(w))
             if cb is not None:
                 rec["cpu_baseline"] = cb
             recs[config_key(w)] = rec
-    recs["clocks"] = clk.summary()
     recs["note"] = ("each workload alone on one GPU, after the headline; steps and warm-up "
-                    "as listed per workload; rates and rooflines as the headline's")
+                    "as listed per workload; rates and rooflines as the headline's; clocks "
+                    "per workload from its own timed region")
     return recs
 
 

@@ -37,20 +37,36 @@ def test_whole_job_rate_counts_every_rank():
 
 def test_clock_record_parsing():
     s = bench.ClockSampler(0)
-    s.out = "\n".join([
-        "0, 1965, 1965, 240.1, 0x0, Not Active, Not Active, Not Active, Not Active",
-        "0, 1950, 1965, 250.0, 0x4, Not Active, Not Active, Not Active, Active",
-        "0, 1965, 1965, 245.0, 0x0, Not Active, Not Active, Not Active, Not Active",
-        "garbage line",
-    ])
+    for i, line in enumerate([
+            "0, 1965, 1965, 240.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+            "0, 1950, 1965, 250.0, 0x4, Not Active, Not Active, Not Active, Active",
+            "0, 1965, 1965, 245.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+            "garbage line"]):
+        s.feed(line, t=float(i))
     r = s.summary()
     assert r["sm_mhz"] == 1965 and r["sm_max_mhz"] == 1965
     assert r["reasons"] == ["sw_power_cap"] and r["samples"] == 3
     assert r["power_w_max"] == 250.0
-    s.out = "0, 1200, 1965, 500, 0x8, Active, Not Active, Active, Not Active"
+    s = bench.ClockSampler(0)
+    s.feed("0, 1200, 1965, 500, 0x8, Active, Not Active, Active, Not Active", t=0.0)
     assert s.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
-    s.out = ""
-    assert s.summary()["reasons"] == ["unavailable"]
+    assert bench.ClockSampler(0).summary()["reasons"] == ["unavailable"]
+
+
+def test_clock_samples_are_taken_from_the_region_and_its_continuation():
+    # idle samples before the region are left out; samples after it count
+    # only up to the end of the top-up that kept the same load
+    s = bench.ClockSampler(0)
+    line = "0, {mhz}, 1965, 300, 0x0, Not Active, Not Active, Not Active, Not Active"
+    s.feed(line.format(mhz=345), t=0.5)               # idle, before the region
+    s.t0, s.t1, s.t_end = 1.0, 1.05, 1.4
+    s.feed(line.format(mhz=1965), t=1.02)             # inside
+    s.feed(line.format(mhz=1950), t=1.2)              # same load, after
+    s.feed(line.format(mhz=1965), t=1.3)
+    s.feed(line.format(mhz=400), t=2.0)               # after the top-up ended
+    r = s.summary()
+    assert r["samples_in_region"] == 1 and r["samples_same_load_after"] == 2
+    assert r["samples"] == 3 and r["sm_mhz"] == 1965
 
 
 def test_stored_traffic_is_keyed_to_the_kernel_sources():
