@@ -143,28 +143,39 @@ def ncu_traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples (every 100 ms, read by a thread) for
-    the timed region.  ``region_start`` / ``region_end`` bracket the region
-    (host times taken after a device synchronize on both sides, so they bound
-    the device's work).  A region shorter than a few sampling intervals gets
-    at most one sample of its own; ``region_end(top_up=fn)`` then keeps the
-    GPU under the same load, running fn (one untimed step) until the region
-    and its continuation hold ``min_samples`` samples.  The summary says how
-    many samples fell inside the region and how many in the continuation."""
+    """SM clock, power and throttle-reason samples for the timed region, read
+    by a thread: from NVML every 5 ms (nvidia-smi every 100 ms where NVML
+    cannot be loaded).  Reading only: nothing is set.  ``region_start`` /
+    ``region_end`` bracket the region (host times taken after a device
+    synchronize on both sides, so they bound the device's work).  A region
+    shorter than a few sampling intervals holds few samples of its own;
+    ``region_end(top_up=fn)`` then keeps the GPU under the same load, running
+    fn (one untimed step) until the region and its continuation hold
+    ``min_samples``.  The summary says how many samples fell inside the
+    region and how many in the continuation."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # NVML clocks-event reason bits -> the names above
+    NVML_BITS = ((0x8, "hw_slowdown"), (0x80, "hw_slowdown"), (0x40, "hw_thermal_slowdown"),
+                 (0x20, "sw_thermal_slowdown"), (0x4, "sw_power_cap"))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, min_samples: int = 3):
         self.gpu_index = gpu_index
+        self.min_samples = min_samples
         self.proc = None
-        self.samples = []          # (host time, parsed sample)
+        self.nvml = None
+        self.samples = []          # (host time, (sm MHz, max sm MHz, power W, reasons))
         self.lock = threading.Lock()
+        self.stop = threading.Event()
         self.thread = None
+        self.source = None
+        self.interval_ms = None
         self.t0 = self.t1 = None
         self.t_end = None
+        self.power_limit = None
 
     def feed(self, line: str, t=None):
         """Parse one nvidia-smi CSV line (ignored when malformed)."""
@@ -179,27 +190,96 @@ class ClockSampler:
         with self.lock:
             self.samples.append((time.monotonic() if t is None else t, smp))
 
-    def _reader(self):
+    def _smi_reader(self):
         for line in self.proc.stdout:
             self.feed(line)
 
-    def __enter__(self):
+    def _nvml_poller(self, h, max_mhz):
+        nv = self.nvml
+        while not self.stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                try:
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except AttributeError:
+                    bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                reasons = sorted({n for b, n in self.NVML_BITS if bits & b})
+                with self.lock:
+                    self.samples.append((time.monotonic(), (mhz, max_mhz, watts, reasons)))
+            except Exception:  # noqa: BLE001 -- a failed read is a missing sample
+                pass
+            self.stop.wait(0.005)
+
+    def _device_uuid(self):
+        try:
+            u = str(torch.cuda.get_device_properties(self.gpu_index).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:  # noqa: BLE001
+            return None
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+        except Exception:  # noqa: BLE001
+            return False
+        self.nvml = nv
+        try:
+            uuid = self._device_uuid()
+            h = (nv.nvmlDeviceGetHandleByUUID(uuid) if uuid
+                 else nv.nvmlDeviceGetHandleByIndex(self.gpu_index))
+            max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            try:
+                self.power_limit = (nv.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0,
+                                    nv.nvmlDeviceGetPowerManagementLimitConstraints(h)[1] / 1000.0)
+            except Exception:  # noqa: BLE001
+                self.power_limit = None
+        except Exception:  # noqa: BLE001
+            nv.nvmlShutdown()
+            self.nvml = None
+            return False
+        self.source, self.interval_ms = "nvml", 5
+        self.min_samples = max(self.min_samples, 10)
+        self.thread = threading.Thread(target=self._nvml_poller, args=(h, max_mhz), daemon=True)
+        self.thread.start()
+        return True
+
+    def _start_smi(self):
+        uuid = self._device_uuid()
+        gid = uuid or str(self.gpu_index)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
-            return self
-        self.thread = threading.Thread(target=self._reader, daemon=True)
+            return
+        try:
+            q = subprocess.run(["nvidia-smi", f"--id={gid}",
+                                "--query-gpu=enforced.power.limit,power.max_limit",
+                                "--format=csv,noheader,nounits"],
+                               capture_output=True, text=True, timeout=10)
+            lim = [x.strip() for x in q.stdout.strip().split(",")]
+            self.power_limit = (float(lim[0]), float(lim[1]))
+        except (OSError, ValueError, IndexError, subprocess.SubprocessError):
+            self.power_limit = None
+        self.source, self.interval_ms = "nvidia-smi", 100
+        self.thread = threading.Thread(target=self._smi_reader, daemon=True)
         self.thread.start()
-        deadline = time.monotonic() + 5.0      # the first sample: nvidia-smi is up
-        while time.monotonic() < deadline and not self._count(0.0, None):
-            time.sleep(0.02)
+
+    def __enter__(self):
+        if not self._start_nvml():
+            self._start_smi()
+        deadline = time.monotonic() + 5.0      # the first sample has arrived
+        while self.thread is not None and time.monotonic() < deadline \
+                and not self._count(0.0, None):
+            time.sleep(0.01)
         return self
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -207,8 +287,13 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 self.proc.wait()
-            if self.thread is not None:
-                self.thread.join(timeout=5)
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
 
     def _count(self, t_from, t_to):
         with self.lock:
@@ -218,11 +303,18 @@ class ClockSampler:
         self.t0 = time.monotonic()
         self.t1 = self.t_end = None
 
-    def region_end(self, top_up=None, min_samples=3, max_s=3.0):
+    def region_end(self, top_up=None, max_s=3.0):
         self.t1 = time.monotonic()
-        if top_up is not None and self.proc is not None:
-            stop = self.t1 + max_s
-            while self._count(self.t0, None) < min_samples and time.monotonic() < stop:
+        self.t_end = self.t1
+        if top_up is not None:
+            self.extend(top_up, max_s)
+
+    def extend(self, top_up, max_s=3.0):
+        """Keep sampling, running top_up() (the same step, untimed), until the
+        region and everything since hold min_samples samples."""
+        if self.thread is not None:
+            stop = time.monotonic() + max_s
+            while self._count(self.t0, None) < self.min_samples and time.monotonic() < stop:
                 top_up()
                 torch.cuda.synchronize()
         self.t_end = time.monotonic()
@@ -241,11 +333,17 @@ class ClockSampler:
         if not used:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         reasons = sorted({n for x in used for n in x[3]})
-        return {"sm_mhz": statistics.median(x[0] for x in used),
-                "sm_max_mhz": max(x[1] for x in used), "reasons": reasons,
-                "samples": len(used), "samples_in_region": len(inside),
-                "samples_same_load_after": len(after), "interval_ms": 100,
-                "power_w_max": max(x[2] for x in used)}
+        rec = {"sm_mhz": statistics.median(x[0] for x in used),
+               "sm_max_mhz": max(x[1] for x in used), "reasons": reasons,
+               "samples": len(used), "samples_in_region": len(inside),
+               "samples_same_load_after": len(after), "source": self.source,
+               "interval_ms": self.interval_ms,
+               "power_w_max": max(x[2] for x in used),
+               "power_limit_w": self.power_limit[0] if self.power_limit else None,
+               "power_max_limit_w": self.power_limit[1] if self.power_limit else None}
+        if inside:
+            rec["sm_mhz_in_region"] = statistics.median(x[0] for x in inside)
+        return rec
 
 
 def reduce_max_over_ranks(x: float, world: int, device) -> float:
@@ -764,10 +862,11 @@ def run_turbo(args, rank, world, local_rank):
             step()
         t1.record(stream)
         _barrier(world, dev)
-        clk.region_end(top_up=step)
+        clk.region_end()
         q_ms = timed_loop(quantize, args.steps)
         d_ms = timed_loop(decode_call, args.steps)
         _barrier(world, dev)
+        clk.extend(top_up=step)
     if jl.jl_device_error() != 0:
         raise RuntimeError("device error in the timed region")
     ms_step = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
@@ -994,9 +1093,11 @@ def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error,
         clk.region_start()
     ms = _timed_loop(stream, step, steps)
     if clk is not None:
-        clk.region_end(top_up=step)
+        clk.region_end()
     q_ms = _timed_loop(stream, quantize, steps)
     d_ms = _timed_loop(stream, decode_call, steps) if decode else 0.0
+    if clk is not None:
+        clk.extend(top_up=step)
     if jl.jl_device_error() != 0:
         raise RuntimeError(f"device error in workload {w.name}")
     phases = phase_records(w, n_keys, q_ms, d_ms, peak, decode)
@@ -1115,10 +1216,11 @@ def run_ours(args, rank, world, local_rank):
             step()
         t1.record(stream)
         barrier()
-        clk.region_end(top_up=step)
+        clk.region_end()
         q_ms = timed_loop(quantize, args.steps)
         d_ms = timed_loop(decode_call, args.steps) if decode else 0.0
         barrier()
+        clk.extend(top_up=step)
     ms_total = t0.elapsed_time(t1)
     if jl.jl_device_error() != 0:
         raise RuntimeError("device error in the timed region")
