@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload gqa|long|prefill|single|sweep-m<M>-d<D>|paged-gqa|dequant-gqa|search|turbo-gqa|
-                turbo-paged-gqa|turbo-dequant-gqa]
+                turbo-paged-gqa|turbo-dequant-gqa|turbo-gqa-d64]
 
 A step is one pass of the whole hot path over one batch of the workload:
 quantize every key of the batch (sign code + fp16 norm, jl_quantize_keys) and
@@ -1137,7 +1137,7 @@ def config_key(w) -> str:
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
-    if args.workload == "turbo-gqa":
+    if args.workload in ("turbo-gqa", "turbo-gqa-d64"):
         return run_turbo(args, rank, world, local_rank)
     if args.workload == "search":
         return run_search(args, rank, world, local_rank)
@@ -1391,7 +1391,7 @@ def oracle_sample(w: workloads.Workload):
         def run():
             tq.dequantize(q["cell"], q["signs"], nk, nr, Pit, S64, c)
         return run, n, f"first {n} codes of the workload's recipe (dequantize only)"
-    if w.name in ("turbo-gqa", "turbo-paged-gqa"):
+    if w.name in ("turbo-gqa", "turbo-paged-gqa", "turbo-gqa-d64"):
         from oracle import turbo as tq
         T = w.T
         sub = w.with_(B=1, Hkv=1, Hq=w.G, T=T)

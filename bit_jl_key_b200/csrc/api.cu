@@ -155,6 +155,9 @@ bool supported_md(int m, int d) {
   return (d == 64 || d == 128) && (m == 64 || m == 128 || m == 256 || m == 512);
 }
 
+// TurboQuant-prod shapes: one residual bit per coordinate, m = d = 64 or 128
+static bool turbo_md(int m, int d) { return m == d && (d == 64 || d == 128); }
+
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? JL_OK : JL_ERR_CUDA; }
 
 int validate_quantize(const void *K, jl_dtype kt, int64_t n, int64_t ldk,
@@ -363,7 +366,7 @@ int jl_turbo_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
                            jl_stream_t stream) {
   if (key_dtype != JL_BF16 && key_dtype != JL_F32) return JL_ERR_INVALID_ARG;
   if (n_keys < 0) return JL_ERR_INVALID_ARG;
-  if (key_dtype != JL_BF16 || m != 128 || d != 128 || mse_bits < 1 ||
+  if (key_dtype != JL_BF16 || !turbo_md(m, d) || mse_bits < 1 ||
       mse_bits > JL_TURBO_MAX_MSE_BITS)
     return JL_ERR_UNSUPPORTED;
   if (n_keys == 0) return JL_OK;
@@ -393,7 +396,7 @@ int jl_turbo_decode_attention(const void *Q, jl_dtype q_dtype, const float *Pinv
                               jl_stream_t stream) {
   if (q_dtype != JL_BF16 && q_dtype != JL_F32) return JL_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0) return JL_ERR_INVALID_ARG;
-  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+  if (!turbo_md(m, d) || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
     return JL_ERR_UNSUPPORTED;
   if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
   if (B == 0) return JL_OK;
@@ -431,7 +434,7 @@ int jl_turbo_decode_attention_paged(
   if (num_pages < 1 || max_pages < 1 || page_tokens < 32 || page_tokens % 32 != 0)
     return JL_ERR_INVALID_ARG;
   if ((int64_t)max_pages * page_tokens < max_len) return JL_ERR_INVALID_ARG;
-  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+  if (!turbo_md(m, d) || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
     return JL_ERR_UNSUPPORTED;
   if (!(softmax_scale == softmax_scale)) return JL_ERR_INVALID_ARG;
   if (B == 0) return JL_OK;
@@ -468,7 +471,7 @@ int jl_turbo_decode_attention_paged(
 
 int jl_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
                            uint16_t *basis, jl_stream_t stream) {
-  if (m != 128 || d != 128) return JL_ERR_UNSUPPORTED;
+  if (!turbo_md(m, d)) return JL_ERR_UNSUPPORTED;
   if (!Pinv || !S || !basis) return JL_ERR_INVALID_ARG;
   if (!aligned(Pinv, 16) || !aligned(S, 16) || !aligned(basis, 16)) return JL_ERR_INVALID_ARG;
   return from_cuda(jlk::launch_turbo_dequant_basis(Pinv, S, m, d, basis, (cudaStream_t)stream));
@@ -478,7 +481,7 @@ int jl_turbo_dequantize_keys(const uint32_t *codes, const uint16_t *norms, int64
                              const uint16_t *basis, int m, int d, int mse_bits, uint16_t *out,
                              jl_stream_t stream) {
   if (n_keys < 0) return JL_ERR_INVALID_ARG;
-  if (m != 128 || d != 128 || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
+  if (!turbo_md(m, d) || mse_bits < 1 || mse_bits > JL_TURBO_MAX_MSE_BITS)
     return JL_ERR_UNSUPPORTED;
   if (n_keys == 0) return JL_OK;
   if (!codes || !norms || !basis || !out) return JL_ERR_INVALID_ARG;

@@ -64,12 +64,26 @@ constexpr int DEC_NORM_AREA = 128; // per stage: 40 fp16 norms; bulk-tensor copi
 // residual sign bits.  A symmetric codebook's centroid is a sum of +-1 terms
 // over the planes: one per plane for TB <= 2, and for TB = 3 the three planes
 // plus their product (whose bit is the XOR of the three), so a key is scored
-// as TERMS + 1 sign contractions.
+// as TERMS + 1 sign contractions.  The scorer contracts code words four at a
+// time (128 coordinates, one integer scale per segment), so each segment --
+// the plane terms' TERMS * D coordinates, then the M residual signs -- is
+// padded to whole runs of 128 coordinates whose query weights are zero (at
+// D = 128 nothing is padded).
+template <int M, int D, int TB>
+struct TurboRow {
+  static constexpr int TERMS = TB == 3 ? 4 : TB;
+  static constexpr int MSE = (TERMS * D + 127) / 128 * 128;  // padded plane-term segment
+  static constexpr int QJL = (M + 127) / 128 * 128;          // padded residual segment
+  static constexpr int LEN = MSE + QJL;                      // query row length
+};
+
 template <int M, int D, bool S8, int TB = 0>
 struct DecCfg {
   static constexpr int STAGES = 2;                     // blocks in the ring
   static constexpr int TERMS = TB == 3 ? 4 : TB;       // +-1 plane terms
-  static constexpr int CODE_BITS = TERMS * D + M;      // coordinates contracted per key
+  // coordinates contracted per key (TurboQuant: the padded query row)
+  static constexpr int CODE_BITS = TB ? TurboRow<M, D, TB>::LEN : M;
+  static constexpr int MSE_RUNS = TB ? TurboRow<M, D, TB>::MSE / 128 : 0;  // plane-term runs
   static constexpr int KEY_SIGN_BYTES = (TB * D + M) / 8;  // bytes stored per key
   static constexpr int SIGN_BYTES = DEC_KB * KEY_SIGN_BYTES;
   static constexpr int V_BYTES = DEC_KB * D * 2;       // 4 or 8 KB
@@ -78,7 +92,7 @@ struct DecCfg {
   // scoring MMA: bf16 m16n8k16 (16 coordinates per slice) or s8 m16n8k32 (32)
   static constexpr int KS = S8 ? 32 : 16;
   static constexpr int NC = CODE_BITS / KS;            // k slices
-  static constexpr int NC_MSE = TERMS * D / KS;        // slices of the cell planes
+  static constexpr int NC_MSE = MSE_RUNS * 128 / KS;   // slices of the cell planes
   static constexpr int A_REGS = 4 * NC;
   // A fragments in smem when they would crowd the registers; the cell-plane
   // codes keep theirs in registers (two CTAs per SM instead of one)
@@ -97,7 +111,7 @@ struct DecCfg {
   static constexpr int SIGN_CHUNKS = SIGN_BYTES / SIGN_CHUNK;  // multiple of 32
   static constexpr int DT = D / 16;                    // 16-dim output tiles
   static_assert(SIGN_CHUNKS % 32 == 0, "sign chunks per lane");
-  static_assert(TB == 0 || (D == 128 && M % 128 == 0), "cell-plane codes: d = 128");
+  static_assert(TB == 0 || ((D == 128 || D == 64) && M == D), "cell-plane codes: m = d = 64 or 128");
   static_assert(STAGE_BYTES % 1024 == 0 && WARP_BYTES % 1024 == 0, "swizzle atoms");
 };
 
@@ -262,7 +276,8 @@ __global__ void __launch_bounds__(PROJ_THREADS) qproj_kernel(const void *__restr
 
 // TurboQuant-prod query rows, four queries per CTA: w = Pinv^T q (so that
 // <w, Pi x> = <q, x> for the stored bf16 Pi), then the row
-//   [wc_0 w, ..., wc_{TERMS-1} w, S w]
+//   [wc_0 w, ..., wc_{TERMS-1} w, 0..., S w, 0...]
+// (each segment zero-padded to whole 128-coordinate runs, TurboRow)
 // whose dot product with the +-1 expansion of a key's code [plane terms,
 // signs] gives the two raw sums of the score: the plane terms' part is
 // <w, c[cell]> because a symmetric codebook is the sum of its odd Walsh
@@ -279,8 +294,9 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
                                                  float *__restrict__ U, int nq,
                                                  const WalshCoef &wc, int64_t x0,
                                                  int *err) {
-  constexpr int TERMS = TB == 3 ? 4 : TB;
-  constexpr int MT = TERMS * D + M;
+  using R = TurboRow<M, D, TB>;
+  constexpr int TERMS = R::TERMS;
+  constexpr int MT = R::LEN;
   constexpr int HALVES = PROJ_THREADS / D;  // threads per output coordinate
   static_assert(PROJ_THREADS % D == 0 && D % HALVES == 0, "query map tiling");
   __shared__ float qsm[PROJ_VECS * D];
@@ -322,8 +338,8 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
     wsm[e] = w;
   }
   __syncthreads();
-  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + TERMS * D, MT,
-                       ProjLimits{err, PROJ_VECS * D, ((int64_t)nq - x0) * MT - TERMS * D});
+  project4<M, D, true>(S, wsm, 0, nx, U + x0 * MT + R::MSE, MT,
+                       ProjLimits{err, PROJ_VECS * D, ((int64_t)nq - x0) * MT - R::MSE});
   for (int e = threadIdx.x; e < nx * D; e += PROJ_THREADS) {
     const int j = e / D, i = e - (e / D) * D;
     float *row = U + (x0 + j) * MT;
@@ -331,6 +347,15 @@ __device__ __forceinline__ void turbo_query_rows(const void *__restrict__ Q,
     for (int k = 0; k < TERMS; ++k)
       if (JL_IN_RANGE(err, (x0 + j) * MT + k * D + i, 1, (int64_t)nq * MT))
         row[k * D + i] = wc.c[k] * wsm[e];
+  }
+  if constexpr (R::MSE > TERMS * D || R::QJL > M) {
+    // the padding of both segments
+    constexpr int P1 = R::MSE - TERMS * D, P2 = R::QJL - M;
+    for (int e = threadIdx.x; e < nx * (P1 + P2); e += PROJ_THREADS) {
+      const int j = e / (P1 + P2), c = e - j * (P1 + P2);
+      const int col = c < P1 ? TERMS * D + c : R::MSE + M + (c - P1);
+      if (JL_IN_RANGE(err, (x0 + j) * MT + col, 1, (int64_t)nq * MT)) U[(x0 + j) * MT + col] = 0.f;
+    }
   }
 }
 
@@ -672,7 +697,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
         for (int k = 0; k < 8; ++k) {
           const float4 v = ldg4(src + 4 * k);
           const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-          am[lw < C::TERMS ? 0 : 1] = fmaxf(am[lw < C::TERMS ? 0 : 1], a);
+          am[lw < C::MSE_RUNS ? 0 : 1] = fmaxf(am[lw < C::MSE_RUNS ? 0 : 1], a);
         }
       }
     }
@@ -687,7 +712,7 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
     int isum[2] = {0, 0};
 #pragma unroll
     for (int lw = 0; lw < C::LW; ++lw) {
-      const int sg = lw < C::TERMS ? 0 : 1;
+      const int sg = lw < C::MSE_RUNS ? 0 : 1;
       const float *src = urow + 32 * (4 * lw + t);
       float4 x[8];
 #pragma unroll
@@ -1072,7 +1097,35 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
 #pragma unroll
     for (int kg = 0; kg < 4; ++kg) {
       const uint32_t kp = sg + (kg * 8 + g) * C::KEY_SIGN_BYTES;
-      if constexpr (TB == 3) {
+      if constexpr (TB > 0 && D == 64) {
+        // run lw, lane t: logical word L = 4 lw + t of the padded row; plane
+        // words are stored first (2 per plane), then the residual signs; the
+        // product term's word (TB = 3) is the XOR of the three planes'; a
+        // padding word is 0 (its query weights are 0)
+        constexpr int PW = D / 32;
+#pragma unroll
+        for (int lw = 0; lw < C::LW; ++lw) {
+          const int L = 4 * lw + t;
+          uint32_t w = 0u;
+          if (lw < C::MSE_RUNS) {
+            if (L < TB * PW) {
+              asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(w) : "r"(kp + L * 4));
+            } else if (TB == 3 && L < C::TERMS * PW) {
+              const int x = L - 3 * PW;
+              uint32_t w0, w1, w2;
+              asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(w0) : "r"(kp + x * 4));
+              asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(w1) : "r"(kp + (PW + x) * 4));
+              asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(w2) : "r"(kp + (2 * PW + x) * 4));
+              w = w0 ^ w1 ^ w2;
+            }
+          } else {
+            const int jw = L - 4 * C::MSE_RUNS;
+            if (jw < M / 32)
+              asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(w) : "r"(kp + (TB * PW + jw) * 4));
+          }
+          wd[kg][lw] = w;
+        }
+      } else if constexpr (TB == 3) {
         // stored words: planes 0-2, then the residual signs; the product
         // term's word is the XOR of the three planes
 #pragma unroll
@@ -1878,10 +1931,11 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
 
 bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int bits,
                             DecodePlan *pl) {
-  if (m != 128 || d != 128 || bits < 1 || bits > 3) return false;
+  if (!((m == 128 && d == 128) || (m == 64 && d == 64)) || bits < 1 || bits > 3) return false;
   if (!plan_common(B, Hq, Hkv, T, m, d, pl)) return false;
   const int terms = bits == 3 ? 4 : bits;
-  pl->u_bytes = round_up((size_t)B * Hq * (terms * d + m) * sizeof(float), 256);
+  const size_t row = (size_t)(terms * d + 127) / 128 * 128 + (size_t)(m + 127) / 128 * 128;
+  pl->u_bytes = round_up((size_t)B * Hq * row * sizeof(float), 256);
   pl->total_bytes = pl->u_bytes + pl->partial_bytes;
   return true;
 }
@@ -1890,14 +1944,14 @@ bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int
 // four coordinates per expanded register) unless a bf16 build is forced.
 constexpr bool TURBO_S8 = JL_DECODE_SCORE != 1;
 
-template <int TB>
+template <int TB, int D>
 static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bool q_f32,
                                          const float *Pinv, const uint16_t *S,
                                          const uint32_t *codes, const uint16_t *norms,
                                          const uint16_t *V, const double *walsh,
                                          float softmax_scale, uint16_t *out, float *scores,
                                          void *workspace, cudaStream_t stream) {
-  constexpr int M = 128, D = 128;
+  constexpr int M = D;
   float *U = reinterpret_cast<float *>(workspace);
   float *partials =
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
@@ -1929,15 +1983,12 @@ cudaError_t launch_turbo_decode(const DecodePlan &pl, int bits, const void *Q, b
                                 const uint16_t *norms, const uint16_t *V, const double *walsh,
                                 float softmax_scale, uint16_t *out, float *scores,
                                 void *workspace, cudaStream_t stream) {
-  if (bits == 1)
-    return launch_turbo_decode_t<1>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
-                                    softmax_scale, out, scores, workspace, stream);
-  if (bits == 2)
-    return launch_turbo_decode_t<2>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
-                                    softmax_scale, out, scores, workspace, stream);
-  if (bits == 3)
-    return launch_turbo_decode_t<3>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,
-                                    softmax_scale, out, scores, workspace, stream);
+#define JL_CASE(TB, DD)                                                                   \
+  if (bits == TB && pl.d == DD && pl.m == DD)                                              \
+    return launch_turbo_decode_t<TB, DD>(pl, Q, q_f32, Pinv, S, codes, norms, V, walsh,     \
+                                         softmax_scale, out, scores, workspace, stream);
+  JL_CASE(1, 128) JL_CASE(2, 128) JL_CASE(3, 128) JL_CASE(1, 64) JL_CASE(2, 64) JL_CASE(3, 64)
+#undef JL_CASE
   return cudaErrorNotSupported;
 }
 
@@ -2070,10 +2121,10 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);
 }
 
-template <int TB>
+template <int TB, int D>
 static cudaError_t launch_turbo_paged_t(const DecodePlan &pl, const PagedArgs &a,
                                         const TurboPagedArgs &t, cudaStream_t stream) {
-  constexpr int M = 128, D = 128;
+  constexpr int M = D;
   uint8_t *ws = reinterpret_cast<uint8_t *>(a.workspace);
   float *U = reinterpret_cast<float *>(ws);
   float *partials = reinterpret_cast<float *>(ws + pl.u_bytes);
@@ -2122,9 +2173,10 @@ static cudaError_t launch_turbo_paged_t(const DecodePlan &pl, const PagedArgs &a
 
 cudaError_t launch_turbo_decode_paged(const DecodePlan &pl, int bits, const PagedArgs &a,
                                       const TurboPagedArgs &t, cudaStream_t stream) {
-  if (bits == 1) return launch_turbo_paged_t<1>(pl, a, t, stream);
-  if (bits == 2) return launch_turbo_paged_t<2>(pl, a, t, stream);
-  if (bits == 3) return launch_turbo_paged_t<3>(pl, a, t, stream);
+#define JL_CASE(TB, DD) \
+  if (bits == TB && pl.d == DD && pl.m == DD) return launch_turbo_paged_t<TB, DD>(pl, a, t, stream);
+  JL_CASE(1, 128) JL_CASE(2, 128) JL_CASE(3, 128) JL_CASE(1, 64) JL_CASE(2, 64) JL_CASE(3, 64)
+#undef JL_CASE
   return cudaErrorNotSupported;
 }
 

@@ -35,7 +35,8 @@
 //   * B (S^T, or R^T for TurboQuant) stays resident; its K order is the same
 //     permutation of each 32-coordinate block, so the contraction is
 //     unchanged.  TurboQuant interleaves its K-chunks (centroid chunk i at
-//     2 i, sign chunk i at 2 i + 1) so both expander parts do equal work.
+//     2 i, sign chunk i at 2 i + 1); at d = 128 each expander part thus
+//     expands one chunk of each kind.
 //   * The epilogue scales row r by sqrt(pi/2)/m * ||k_r|| (QJL) or ||k_r||
 //     (TurboQuant), rounds to bf16, writes its 32 rows into a
 //     128-byte-swizzled staging tile in shared memory and stores them with
@@ -81,7 +82,7 @@ constexpr uint32_t SIGN2 = 0x80008000u;  // sign bits of a 16-bit pair
 
 // TB = 0: QJL codes (m/32 sign words, one binary16 norm per key).
 // TB = 1..3: TurboQuant-prod codes (TB cell planes of d bits, then m sign
-// bits; a binary16 (||k||, ||r||) pair per key); d = m = 128.
+// bits; a binary16 (||k||, ||r||) pair per key); d = m = 64 or 128.
 template <int M, int D, int TB>
 struct Cfg {
   static constexpr bool TURBO = TB > 0;
@@ -116,8 +117,8 @@ struct Cfg {
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + align slack
   static_assert(K % CHUNK_K == 0 && RING >= 2, "A ring");
   static_assert(A_COL0 + RING * CHUNK_COLS <= TMEM_COLS, "tensor memory columns");
-  static_assert(!TURBO || (D == 128 && M == 128 && TB <= 3), "TurboQuant shapes");
-  static_assert(!TURBO || KCH == 2 * EXP_PARTS, "one centroid and one sign chunk per part");
+  static_assert(!TURBO || ((D == 128 || D == 64) && M == D && TB <= 3), "TurboQuant shapes");
+  static_assert(!TURBO || KCH % EXP_PARTS == 0, "whole chunks per part");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -327,15 +328,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           cp_async_8(dst, src, live ? 8 : 0);
         }
       } else {
-        // 8 bytes (the part's 64 coordinates) of each cell plane and of the
-        // sign words, then the norm pair
+        // 8 bytes (the 64 coordinates of the part's chunk index kc0 / 2) of
+        // each cell plane and of the sign words, then the norm pair
         const bool live = row < p.n &&
                           JL_IN_RANGE(p.err, row * C::CODE_BYTES_G, C::CODE_BYTES_G,
                                       p.n * C::CODE_BYTES_G) &&
                           JL_IN_RANGE(p.err, 2 * row, 2, 2 * p.n);
         const int64_t rr = live ? row : 0;
         const uint8_t *src =
-            reinterpret_cast<const uint8_t *>(p.codes) + rr * C::CODE_BYTES_G + 8 * pt;
+            reinterpret_cast<const uint8_t *>(p.codes) + rr * C::CODE_BYTES_G + 8 * (kc0 >> 1);
 #pragma unroll
         for (int pl = 0; pl <= TB; ++pl) cp_async_8(dst + 8 * pl, src + pl * (D / 8), live ? 8 : 0);
         cp_async_4(dst + 8 * (TB + 1), p.norms + 2 * rr, live ? 4 : 0);
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 16; ++j)
               z[16 * half + j] = ((w << (15 - j)) & SIGN2) ^ 0xBF80BF80u;
           }
-        } else if (kk == 0) {                       // centroid chunk pt
+        } else if (((kc0 + kk) & 1) == 0) {         // centroid chunk (kc0 + kk) / 2
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t w[TB];
@@ -402,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int pl = 0; pl < TB; ++pl) w[pl] = cur[2 * pl + half];
             centroid_pairs<TB>(w, p, z + 16 * half);
           }
-        } else {                                    // sign chunk pt
+        } else {                                    // sign chunk (kc0 + kk) / 2
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             const uint32_t w = cur[2 * TB + half];
@@ -634,7 +635,7 @@ cudaError_t launch_dequantize_tc(const uint32_t *signs, const uint16_t *norms, i
 
 cudaError_t launch_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, int d,
                                        uint16_t *basis, cudaStream_t stream) {
-  if (m != 128 || d != 128) return cudaErrorNotSupported;
+  if (m != d || (d != 64 && d != 128)) return cudaErrorNotSupported;
   int *err = device_error_ptr();
   if (!err) return cudaErrorInvalidSymbol;
   const int total = d * (d + m);
@@ -646,7 +647,7 @@ cudaError_t launch_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int
 cudaError_t launch_turbo_dequantize(const uint32_t *codes, const uint16_t *norms, int64_t n,
                                     const uint16_t *basis, int m, int d, int bits,
                                     uint16_t *out, cudaStream_t stream) {
-  if (m != 128 || d != 128) return cudaErrorNotSupported;
+  if (m != d || (d != 64 && d != 128)) return cudaErrorNotSupported;
   float mag[4], thr[3];
   if (!turbo_magnitudes(d, bits, mag, thr)) return cudaErrorNotSupported;
   dq::Params p{};
@@ -661,12 +662,11 @@ cudaError_t launch_turbo_dequantize(const uint32_t *codes, const uint16_t *norms
   }
   p.dmag01 = h[0] ^ h[1];
   p.dmag23 = h[2] ^ h[3];
-  switch (bits) {
-    case 1: return dq::launch_t<128, 128, 1>(p, out, stream);
-    case 2: return dq::launch_t<128, 128, 2>(p, out, stream);
-    case 3: return dq::launch_t<128, 128, 3>(p, out, stream);
-    default: return cudaErrorNotSupported;
-  }
+#define JL_CASE(TB, DD) \
+  if (bits == TB && d == DD) return dq::launch_t<DD, DD, TB>(p, out, stream);
+  JL_CASE(1, 128) JL_CASE(2, 128) JL_CASE(3, 128) JL_CASE(1, 64) JL_CASE(2, 64) JL_CASE(3, 64)
+#undef JL_CASE
+  return cudaErrorNotSupported;
 }
 
 }  // namespace jlk

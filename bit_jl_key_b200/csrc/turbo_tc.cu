@@ -318,34 +318,38 @@ cudaError_t launch_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t seed, voi
 }
 
 // --------------------------------------------------------------------------
-// quantizer (tensor cores), d = m = 128
+// quantizer (tensor cores), d = m = 64 or 128
 
 constexpr int BM = 128;
-constexpr int QD = 128;   // head dim = rotation size
-constexpr int QM = 128;   // residual sketch rows
 
-template <int TB>
+// TB cell planes, head dim D = rotation size = residual sketch rows M
+template <int TB, int D>
 struct QCfg {
-  static constexpr int KCH = QD / 64;
+  static constexpr int M = D;
+  static constexpr int KCH = D / 64;
   static constexpr int A_CHUNK = BM * 128;      // one 64-column swizzle column of a tile
-  static constexpr int A_STAGE = BM * QD * 2;   // 32 KB
-  static constexpr int W_CHUNK = 128 * 128;     // 128 rows x 64 columns of Pi or S
-  static constexpr int W_BYTES = 128 * QD * 2;  // 32 KB
+  static constexpr int A_STAGE = BM * D * 2;    // 32 or 16 KB
+  static constexpr int PI_CHUNK = D * 128;      // D rows x 64 columns of Pi
+  static constexpr int S_CHUNK = M * 128;       // M rows x 64 columns of S
+  static constexpr int PI_BYTES = D * D * 2;
+  static constexpr int S_BYTES = M * D * 2;
   static constexpr int STAGES = 4;
   static constexpr int EPI_WARPS = 8;           // two per TMEM lane quadrant (tile parities)
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int OFF_PI = 0;
-  static constexpr int OFF_S = W_BYTES;
-  static constexpr int OFF_A = 2 * W_BYTES;
+  static constexpr int OFF_S = PI_BYTES;
+  static constexpr int OFF_A = PI_BYTES + S_BYTES;
   static constexpr int OFF_BAR = OFF_A + STAGES * A_STAGE;
   static constexpr int NBAR = 2 * STAGES + 2 + 2 + 2 + 1 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr int WORDS = TB * QD / 32 + QM / 32;
-  static constexpr int PW = QD / 32;            // words per plane
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int D1_COL = 0;              // rotated keys, two buffers of 128 columns
-  static constexpr int D2_COL = 256;            // residual projections, one buffer
-  static constexpr int A2_COL = 384;            // bf16 residual rows, two buffers of 64
+  static constexpr int WORDS = TB * D / 32 + M / 32;
+  static constexpr int PW = D / 32;             // words per plane
+  static constexpr int TMEM_COLS = 4 * D;       // 512 or 256
+  static constexpr int D1_COL = 0;              // rotated keys, two buffers of D columns
+  static constexpr int D2_COL = 2 * D;          // residual projections, one buffer of M
+  static constexpr int A2_COL = 2 * D + M;      // bf16 residual rows, two buffers of D / 2
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(OFF_S % 1024 == 0 && OFF_A % 1024 == 0, "swizzle atoms");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(STAGES % 2 == 0, "a stage holds tiles of one parity");
 };
@@ -461,12 +465,12 @@ __device__ __forceinline__ uint64_t cell_residual_pair(uint64_t d2, uint64_t nin
   return rr2;
 }
 
-template <int TB>
-__global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
+template <int TB, int D>
+__global__ void __launch_bounds__(QCfg<TB, D>::THREADS, 1)
     turbo_quantize_kernel(const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_pi,
                           const __grid_constant__ CUtensorMap tmap_s, const QParams p) {
-  using C = QCfg<TB>;
+  using C = QCfg<TB, D>;
   extern __shared__ uint8_t tq_smem_raw[];
   const uint32_t raw = smem_u32(tq_smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -521,10 +525,10 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      mbar_expect_tx(wfull, 2 * C::W_BYTES);
+      mbar_expect_tx(wfull, C::PI_BYTES + C::S_BYTES);
       for (int kc = 0; kc < C::KCH; ++kc) {
-        tma_load_2d(sPi + kc * C::W_CHUNK, &tmap_pi, kc * 64, 0, wfull);
-        tma_load_2d(sS + kc * C::W_CHUNK, &tmap_s, kc * 64, 0, wfull);
+        tma_load_2d(sPi + kc * C::PI_CHUNK, &tmap_pi, kc * 64, 0, wfull);
+        tma_load_2d(sS + kc * C::S_CHUNK, &tmap_s, kc * 64, 0, wfull);
       }
       int64_t t = 0;
       for (; t < cnt; ++t) {
@@ -547,7 +551,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
     // elected lane issues; descriptors are the base plus a 32-bit start-address
     // add (every operand lies below 256 KB of shared memory).
     {
-      constexpr uint32_t idesc = tcx::idesc_f16(BM, 128, 1);
+      constexpr uint32_t idesc = tcx::idesc_f16(BM, D, 1);  // N = D = M
       const uint64_t da = tcx::desc_sw128(sA), dpi = tcx::desc_sw128(sPi), ds = tcx::desc_sw128(sS);
       const uint32_t a_hi = (uint32_t)(da >> 32), a_lo0 = (uint32_t)da;
       const uint32_t pi_hi = (uint32_t)(dpi >> 32), pi_lo = (uint32_t)dpi;
@@ -572,14 +576,14 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           if (tcx::elect_one()) {
             const uint32_t alo = a_lo0 + (uint32_t)s * (uint32_t)(C::A_STAGE >> 4);
 #pragma unroll
-            for (int kk = 0; kk < QD / 16; ++kk) {
+            for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off =
                   ((uint32_t)(kk >> 2) * (uint32_t)C::A_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
               const uint32_t woff =
-                  ((uint32_t)(kk >> 2) * (uint32_t)C::W_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+                  ((uint32_t)(kk >> 2) * (uint32_t)C::PI_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
               const uint64_t ad = ((uint64_t)a_hi << 32) | (uint64_t)(alo + off);
               const uint64_t bd = ((uint64_t)pi_hi << 32) | (uint64_t)(pi_lo + woff);
-              tcx::mma_ss(tmem_base + C::D1_COL + a * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+              tcx::mma_ss(tmem_base + C::D1_COL + a * D, ad, bd, idesc, kk > 0 ? 1u : 0u);
             }
             tcx::commit(d1full(a));
             tcx::commit(kempty(s));
@@ -603,12 +607,12 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           tcx::fence_after();
           if (tcx::elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < QD / 16; ++kk) {
+            for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t woff =
-                  ((uint32_t)(kk >> 2) * (uint32_t)C::W_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+                  ((uint32_t)(kk >> 2) * (uint32_t)C::S_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
               const uint64_t bd = ((uint64_t)s_hi << 32) | (uint64_t)(s_lo + woff);
-              tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * 64 + kk * 8, bd, idesc,
-                          kk > 0 ? 1u : 0u);
+              tcx::mma_ts(tmem_base + C::D2_COL, tmem_base + C::A2_COL + a * (D / 2) + kk * 8, bd,
+                          idesc, kk > 0 ? 1u : 0u);
             }
             tcx::commit(d2full(a));
           }
@@ -662,8 +666,8 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       uint64_t rs2 = 0ull;                       // residual sum of squares, two lanes
       const uint64_t ninv2 = f32x2_pack(ninv, ninv);
       uint32_t va[32], vb[32];
-      const uint32_t dcol = tq + (uint32_t)(C::D1_COL + h * 128);
-      const uint32_t acol = tq + (uint32_t)(C::A2_COL + h * 64);
+      const uint32_t dcol = tq + (uint32_t)(C::D1_COL + h * D);
+      const uint32_t acol = tq + (uint32_t)(C::A2_COL + h * (D / 2));
       auto chunk = [&](uint32_t (&v)[32], int ch) {
         PlaneChains<TB> pc;
 #pragma unroll
@@ -700,11 +704,11 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
           planes[k][ch & 1] = ~(top ^ (pc.mag[k][0] | (pc.mag[k][1] << 8) |
                                        (pc.mag[k][2] << 16) | (pc.mag[k][3] << 24)));
       };
-      // four chunks of 32 columns, two per pass (a rolled loop keeps the
+      // D / 32 chunks of 32 columns, two per pass (a rolled loop keeps the
       // code small); the second chunk's load is in flight during the first
       uint32_t *dst = p.codes + row * C::WORDS;
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < D / 64; ++half) {
         tcx::ld32(dcol + 64 * half, va);
         tcx::ld32(dcol + 64 * half + 32, vb);
         tcx::ld_wait(va);
@@ -735,7 +739,7 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
       __syncwarp();
       tcx::fence_after();
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < C::M / 64; ++half) {
         const uint32_t d2 = tq + (uint32_t)(C::D2_COL + 64 * half);
         tcx::ld32(d2, va);
         tcx::ld32(d2 + 32, vb);
@@ -763,14 +767,14 @@ __global__ void __launch_bounds__(QCfg<TB>::THREADS, 1)
   }
 }
 
-template <int TB>
+template <int TB, int D>
 static cudaError_t launch_quantize_t(const uint16_t *K, int64_t n, int64_t ldk,
                                      const uint16_t *Pi, const uint16_t *S, const Codebook &cb,
                                      uint32_t *codes, uint16_t *norms, cudaStream_t stream) {
-  using C = QCfg<TB>;
+  using C = QCfg<TB, D>;
   CUtensorMap mk, mpi, ms;
-  if (!tc::make_map(&mk, K, (uint64_t)n, QD, (uint64_t)ldk, BM) ||
-      !tc::make_map(&mpi, Pi, QD, QD, QD, 128) || !tc::make_map(&ms, S, QM, QD, QD, 128))
+  if (!tc::make_map(&mk, K, (uint64_t)n, D, (uint64_t)ldk, BM) ||
+      !tc::make_map(&mpi, Pi, D, D, D, D) || !tc::make_map(&ms, S, C::M, D, D, C::M))
     return cudaErrorInvalidValue;
   QParams p{};
   p.n = n;
@@ -782,11 +786,11 @@ static cudaError_t launch_quantize_t(const uint16_t *K, int64_t n, int64_t ldk,
   const int H = cb.L / 2;
   for (int i = 0; i < 4; ++i) p.mag[i] = i < H ? cb.cf[H + i] : 0.f;
   for (int i = 0; i < 3; ++i) p.pos_thr[i] = i + 1 < H ? cb.thr[H + i] : 0.f;
-  cudaError_t e = cudaFuncSetAttribute(turbo_quantize_kernel<TB>,
+  cudaError_t e = cudaFuncSetAttribute(turbo_quantize_kernel<TB, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  turbo_quantize_kernel<TB><<<(int)grid, C::THREADS, C::SMEM, stream>>>(mk, mpi, ms, p);
+  turbo_quantize_kernel<TB, D><<<(int)grid, C::THREADS, C::SMEM, stream>>>(mk, mpi, ms, p);
   return cudaGetLastError();
 }
 
@@ -821,14 +825,14 @@ cudaError_t launch_turbo_rotation(uint16_t *Pi, float *Pinv, int d, uint64_t see
 cudaError_t launch_turbo_quantize(const uint16_t *K, int64_t n, int64_t ldk, const uint16_t *Pi,
                                   const uint16_t *S, int m, int d, int bits, uint32_t *codes,
                                   uint16_t *norms, cudaStream_t stream) {
-  if (m != turbo::QM || d != turbo::QD) return cudaErrorNotSupported;
+  if (m != d || (d != 64 && d != 128)) return cudaErrorNotSupported;
   const turbo::Codebook *cb = turbo::codebook(d, bits);
-  switch (bits) {
-    case 1: return turbo::launch_quantize_t<1>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
-    case 2: return turbo::launch_quantize_t<2>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
-    case 3: return turbo::launch_quantize_t<3>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
-    default: return cudaErrorNotSupported;
-  }
+#define JL_CASE(TB, DD)                                                                        \
+  if (bits == TB && d == DD)                                                                   \
+    return turbo::launch_quantize_t<TB, DD>(K, n, ldk, Pi, S, *cb, codes, norms, stream);
+  JL_CASE(1, 128) JL_CASE(2, 128) JL_CASE(3, 128) JL_CASE(1, 64) JL_CASE(2, 64) JL_CASE(3, 64)
+#undef JL_CASE
+  return cudaErrorNotSupported;
 }
 
 }  // namespace jlk

@@ -334,7 +334,8 @@ JL_API int jl_decode_attention_noalloc(const void *Q, jl_dtype q_dtype,
  * and inner product, in two stages" (b-1 bits per coordinate from the
  * Lloyd-Max codebook of f, one more bit from QJL on the residual; unbiased).
  *
- * Per key k (d = 128; the residual sketch S is m x d with m = 128):
+ * Per key k (d = 64 or 128; the residual sketch S is m x d with m = d: one
+ * residual bit per coordinate):
  *   x = k / ||k||  (0 for k = 0),  y = Pi x  (Pi: the stored bf16 rotation)
  *   cell_i = the cell of the centroid nearest y_i (a value exactly on a
  *            boundary goes to the cell nearer zero; 0 to the cell below it)
@@ -402,7 +403,7 @@ JL_API int jl_turbo_rotation_init(uint16_t *Pi, float *Pinv, int d, uint64_t see
  * either cell; a residual coordinate within that error of a bf16 rounding
  * midpoint may round either way, and a sign within the resulting error of 0
  * either sign.  n_keys == 0 is a no-op.
- * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED (d, m not 128; key dtype
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED (d, m not equal 64 or 128; key dtype
  * not bf16; mse_bits outside [1, JL_TURBO_MAX_MSE_BITS]), JL_ERR_CUDA.
  */
 JL_API int jl_turbo_quantize_keys(const void *K, jl_dtype key_dtype, int64_t n_keys,
@@ -427,7 +428,7 @@ JL_API size_t jl_turbo_decode_workspace_bytes(int B, int Hq, int Hkv, int64_t T,
  *   out    : out, device, B x Hq x d bf16.
  *   scores : optional out, B x Hq x T fp32 (s before softmax_scale).
  *   workspace : device scratch of jl_turbo_decode_workspace_bytes(...).
- * Supported: d = m = 128, mse_bits 1 to 3.  B == 0 is a no-op; T >= 1.
+ * Supported: d = m = 64 or 128, mse_bits 1 to 3.  B == 0 is a no-op; T >= 1.
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
  * JL_ERR_CUDA.
  */
@@ -460,7 +461,7 @@ JL_API size_t jl_turbo_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int6
  *                 uint32 (the jl_turbo_quantize_keys code layout).
  *   norm_pages  : in/out, num_pages x Hkv x page_tokens x 2 binary16.
  *   value_pages : in/out, num_pages x Hkv x page_tokens x d bf16.
- * Supported: d = m = 128, mse_bits 1 to 3.
+ * Supported: d = m = 64 or 128, mse_bits 1 to 3.
  * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_WORKSPACE,
  * JL_ERR_CUDA.
  */
@@ -484,7 +485,7 @@ JL_API int jl_turbo_decode_attention_paged(
  *           Pinv[j][i] for i < d, basis[j][d + l] = sum_i Pinv[j][i] S[l][i]
  *           (fp32 products and sums), each rounded to nearest binary16;
  *           16-byte aligned, d (d + m) elements.
- * Supported: d = m = 128.
+ * Supported: d = m = 64 or 128.
  * Errors: JL_ERR_INVALID_ARG (null or misaligned pointer), JL_ERR_UNSUPPORTED
  * (d, m), JL_ERR_CUDA.
  */
@@ -511,7 +512,7 @@ JL_API int jl_turbo_dequant_basis(const float *Pinv, const uint16_t *S, int m, i
  *   basis : in, device, d x (d + m) binary16 from jl_turbo_dequant_basis,
  *           16-byte aligned.
  *   out   : out, device, n_keys x d bf16 (round to nearest), 16-byte aligned.
- * Supported: d = m = 128, mse_bits 1 to JL_TURBO_MAX_MSE_BITS.  n_keys == 0
+ * Supported: d = m = 64 or 128, mse_bits 1 to JL_TURBO_MAX_MSE_BITS.  n_keys == 0
  * is a no-op.
  * Errors: JL_ERR_INVALID_ARG (null or misaligned pointer, n_keys < 0),
  * JL_ERR_UNSUPPORTED (d, m, mse_bits, n_keys >= 2^40), JL_ERR_CUDA.

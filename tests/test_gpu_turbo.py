@@ -39,11 +39,11 @@ def _bf16_tensor(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def _setup(bits, rot_seed=1, sk_seed=0):
-    c = tq.lloyd_max(D, bits)
-    pit_bits = tq.rotation_bf16_bits(D, rot_seed)
+def _setup(bits, rot_seed=1, sk_seed=0, d=D):
+    c = tq.lloyd_max(d, bits)
+    pit_bits = tq.rotation_bf16_bits(d, rot_seed)
     Pit = oracle.bf16_bits_to_f64(pit_bits)
-    s_bits = oracle.sketch_bf16_bits(M, D, sk_seed)
+    s_bits = oracle.sketch_bf16_bits(d, d, sk_seed)
     S64 = oracle.bf16_bits_to_f64(s_bits)
     return c, pit_bits, Pit, s_bits, S64
 
@@ -77,7 +77,8 @@ def test_codebook_matches_oracle(bits):
 
 
 def _quantize_case(bits, K, rot_seed=1):
-    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed)
+    d = m = K.shape[1]
+    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed, d=d)
     n = K.shape[0]
     codes, norms = jl.jl_turbo_quantize_keys(K.cuda(), _bf16_tensor(pit_bits), _bf16_tensor(s_bits),
                                              bits)
@@ -85,13 +86,13 @@ def _quantize_case(bits, K, rot_seed=1):
     assert jl.jl_device_error() == 0
     ref = tq.quantize(H.f64(K), Pit, c, S64, band_abs=BAND_Y, band_rel=BAND_SIGN)
     gw = H.u32(codes).reshape(n, -1)
-    pw = bits * D // 32
-    gcell = tq.unpack_planes(gw[:, :pw], D, bits)
+    pw = bits * d // 32
+    gcell = tq.unpack_planes(gw[:, :pw], d, bits)
     cdiff = gcell != ref["cell"]
     assert not np.any(cdiff & ~ref["cell_band"]), int(np.count_nonzero(cdiff & ~ref["cell_band"]))
     ok = ~cdiff.any(axis=1)
-    gz = H.code_bits(gw[:, pw:], M)
-    rz = H.code_bits(ref["signs"], M)
+    gz = H.code_bits(gw[:, pw:], m)
+    rz = H.code_bits(ref["signs"], m)
     sdiff = (gz != rz) & ok[:, None]
     allowed = np.abs(ref["proj"]) < ref["sign_allow"]
     assert not np.any(sdiff & ~allowed), int(np.count_nonzero(sdiff & ~allowed))
@@ -101,21 +102,23 @@ def _quantize_case(bits, K, rot_seed=1):
     return int(cdiff.sum()), int(sdiff.sum()), int((~ok).sum())
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("n", [1, 300, 4099])
-def test_quantize_matches_oracle(bits, n):
+def test_quantize_matches_oracle(bits, n, d):
     torch.cuda.set_device(0)
-    K = workloads.random_keys(n, D, 900 + n + bits, scale=1.3)
+    K = workloads.random_keys(n, d, 900 + n + bits + d, scale=1.3)
     cf, sf, kf = _quantize_case(bits, K)
-    print(f"turbo quantize bits={bits} n={n}: {cf} in-band cells, {sf} allowed sign flips, "
-          f"{kf} keys skipped for the residual check")
+    print(f"turbo quantize d={d} bits={bits} n={n}: {cf} in-band cells, {sf} allowed sign "
+          f"flips, {kf} keys skipped for the residual check")
 
 
-def test_quantize_edge_keys():
+@pytest.mark.parametrize("d", [128, 64])
+def test_quantize_edge_keys(d):
     # a zero key (norm 0, y = 0: every coordinate in the cell just below 0),
     # huge and tiny keys, outlier channels
     torch.cuda.set_device(0)
-    K = workloads.random_keys(256, D, 31)
+    K = workloads.random_keys(256, d, 31)
     K[0] = 0
     K[1] *= 3000
     K[2] *= 1e-3
@@ -133,19 +136,19 @@ def test_quantize_gqa_keys_sampled():
     print(f"turbo-gqa keys: {cf} in-band cells, {sf} allowed sign flips, {kf} keys skipped")
 
 
-def _decode_inputs(bits, B, Hq, Hkv, T, seed, qdtype=torch.bfloat16):
-    c, pit_bits, Pit, s_bits, S64 = _setup(bits)
-    K = workloads.random_keys(B * Hkv * T, D, seed, scale=1.0)
-    V = workloads.random_keys(B * Hkv * T, D, seed + 1).reshape(B, Hkv, T, D)
-    Q = workloads.random_keys(B * Hq, D, seed + 2, dtype=qdtype).reshape(B, Hq, D)
+def _decode_inputs(bits, B, Hq, Hkv, T, seed, qdtype=torch.bfloat16, d=D):
+    c, pit_bits, Pit, s_bits, S64 = _setup(bits, d=d)
+    K = workloads.random_keys(B * Hkv * T, d, seed, scale=1.0)
+    V = workloads.random_keys(B * Hkv * T, d, seed + 1).reshape(B, Hkv, T, d)
+    Q = workloads.random_keys(B * Hq, d, seed + 2, dtype=qdtype).reshape(B, Hq, d)
     ref = tq.quantize(H.f64(K), Pit, c, S64)
     planes = tq.pack_planes(ref["cell"], bits)
     codes = np.concatenate([planes, ref["signs"]], axis=1).reshape(B, Hkv, T, -1)
     norms = np.stack([ref["norm16"], ref["rnorm16"]], axis=1).reshape(B, Hkv, T, 2)
     nk = oracle.fp16_bits_to_f64(ref["norm16"]).reshape(B, Hkv, T)
     nr = oracle.fp16_bits_to_f64(ref["rnorm16"]).reshape(B, Hkv, T)
-    want = tq.decode(H.f64(Q), Pit, S64, c, ref["cell"].reshape(B, Hkv, T, D),
-                     ref["signs"].reshape(B, Hkv, T, -1), nk, nr, H.f64(V), 1 / np.sqrt(D),
+    want = tq.decode(H.f64(Q), Pit, S64, c, ref["cell"].reshape(B, Hkv, T, d),
+                     ref["signs"].reshape(B, Hkv, T, -1), nk, nr, H.f64(V), 1 / np.sqrt(d),
                      want_scores=True)
     gpu_in = dict(Q=Q.cuda(),
                   Pinv=torch.from_numpy(np.linalg.inv(Pit).astype(np.float32)).cuda(),
@@ -157,11 +160,13 @@ def _decode_inputs(bits, B, Hq, Hkv, T, seed, qdtype=torch.bfloat16):
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3])
-@pytest.mark.parametrize("B,Hq,Hkv,T", [(2, 8, 2, 300), (1, 4, 4, 1), (2, 32, 8, 4096),
-                                        (1, 8, 1, 1001)])
-def test_decode_matches_oracle(bits, B, Hq, Hkv, T):
+@pytest.mark.parametrize("B,Hq,Hkv,T,d", [(2, 8, 2, 300, 128), (1, 4, 4, 1, 128),
+                                          (2, 32, 8, 4096, 128), (1, 8, 1, 1001, 128),
+                                          (2, 8, 2, 300, 64), (1, 4, 4, 1, 64),
+                                          (2, 16, 4, 2048, 64), (1, 8, 1, 1001, 64)])
+def test_decode_matches_oracle(bits, B, Hq, Hkv, T, d):
     torch.cuda.set_device(0)
-    gi, (ref_out, ref_sc) = _decode_inputs(bits, B, Hq, Hkv, T, 4000 + T + B)
+    gi, (ref_out, ref_sc) = _decode_inputs(bits, B, Hq, Hkv, T, 4000 + T + B + d, d=d)
     out, sc = jl.jl_turbo_decode_attention(gi["Q"], gi["Pinv"], gi["S"], gi["codes"], gi["norms"],
                                            gi["V"], bits, want_scores=True)
     torch.cuda.synchronize()
@@ -169,7 +174,8 @@ def test_decode_matches_oracle(bits, B, Hq, Hkv, T):
     assert H.score_violations(H.f64(sc), ref_sc) == 0
     mabs, rel = H.output_errors(H.f64(out), ref_out)
     assert mabs <= H.OUT_ABS, mabs
-    print(f"turbo decode bits={bits} {B}x{Hq}/{Hkv}x{T}: out err {mabs:.2e} (rel {rel:.2e})")
+    print(f"turbo decode d={d} bits={bits} {B}x{Hq}/{Hkv}x{T}: out err {mabs:.2e} "
+          f"(rel {rel:.2e})")
 
 
 def test_decode_fp32_queries():
@@ -182,28 +188,29 @@ def test_decode_fp32_queries():
     assert H.output_errors(H.f64(out), ref_out)[0] <= H.OUT_ABS
 
 
-def test_end_to_end_library_rotation_and_codes():
+@pytest.mark.parametrize("d", [128, 64])
+def test_end_to_end_library_rotation_and_codes(d):
     # rotation, quantization and decode all from the library; the oracle
     # decodes its own codes of the same keys
     torch.cuda.set_device(0)
     bits, B, Hq, Hkv, T = 2, 2, 8, 2, 2048
-    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=5)
-    Pi, Pinv = jl.jl_turbo_rotation_init(D, 5)
-    S = jl.jl_sketch_init(M, D, 0)
-    K = workloads.random_keys(B * Hkv * T, D, 123)
-    V = workloads.random_keys(B * Hkv * T, D, 124).reshape(B, Hkv, T, D)
-    Q = workloads.random_keys(B * Hq, D, 125).reshape(B, Hq, D)
+    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=5, d=d)
+    Pi, Pinv = jl.jl_turbo_rotation_init(d, 5)
+    S = jl.jl_sketch_init(d, d, 0)
+    K = workloads.random_keys(B * Hkv * T, d, 123)
+    V = workloads.random_keys(B * Hkv * T, d, 124).reshape(B, Hkv, T, d)
+    Q = workloads.random_keys(B * Hq, d, 125).reshape(B, Hq, d)
     codes, norms = jl.jl_turbo_quantize_keys(K.cuda(), Pi, S, bits)
     out = jl.jl_turbo_decode_attention(Q.cuda(), Pinv, S, codes.reshape(B, Hkv, T, -1),
                                        norms.reshape(B, Hkv, T, 2), V.cuda(), bits)
     torch.cuda.synchronize()
     assert jl.jl_device_error() == 0
     ref = tq.quantize(H.f64(K), Pit, c, S64)
-    ref_out, _ = tq.decode(H.f64(Q), Pit, S64, c, ref["cell"].reshape(B, Hkv, T, D),
+    ref_out, _ = tq.decode(H.f64(Q), Pit, S64, c, ref["cell"].reshape(B, Hkv, T, d),
                            ref["signs"].reshape(B, Hkv, T, -1),
                            oracle.fp16_bits_to_f64(ref["norm16"]).reshape(B, Hkv, T),
                            oracle.fp16_bits_to_f64(ref["rnorm16"]).reshape(B, Hkv, T),
-                           H.f64(V), 1 / np.sqrt(D))
+                           H.f64(V), 1 / np.sqrt(d))
     mabs, rel = H.output_errors(H.f64(out), ref_out)
     assert mabs <= H.OUT_ABS, mabs
 
@@ -214,6 +221,8 @@ def test_decode_rejects_bad_arguments():
     assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 128, 4) == 0
     assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 256, 128, 2) == 0
     assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 128, 2) > 0
+    assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 64, 64, 2) > 0
+    assert jl.jl_turbo_decode_workspace_bytes(1, 8, 2, 64, 128, 64, 2) == 0   # m = d only
     st = L.jl_turbo_quantize_keys(None, jl.JL_F32, 4, 128, None, None, 128, 128, 2, None, None,
                                   None)
     assert st == jl.JL_ERR_UNSUPPORTED

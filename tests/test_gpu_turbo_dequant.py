@@ -46,11 +46,11 @@ def _bf16_tensor(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def _setup(bits, rot_seed=1, sk_seed=0):
-    c = tq.lloyd_max(D, bits)
-    pit_bits = tq.rotation_bf16_bits(D, rot_seed)
+def _setup(bits, rot_seed=1, sk_seed=0, d=D):
+    c = tq.lloyd_max(d, bits)
+    pit_bits = tq.rotation_bf16_bits(d, rot_seed)
     Pit = oracle.bf16_bits_to_f64(pit_bits)
-    s_bits = oracle.sketch_bf16_bits(M, D, sk_seed)
+    s_bits = oracle.sketch_bf16_bits(d, d, sk_seed)
     S64 = oracle.bf16_bits_to_f64(s_bits)
     return c, pit_bits, Pit, s_bits, S64
 
@@ -62,8 +62,9 @@ def _oracle_pinv32(Pit):
 def _tolerance(cell, signs, norms, rnorms, Pinv, S64, c, ref, eps_pinv=0.0):
     """Element-wise bound on |gpu - ref| (see the module docstring)."""
     n = cell.shape[0]
+    m, d = S64.shape
     nk = np.asarray(norms, dtype=np.float64)[:, None]
-    alpha = (SQRT_HALF_PI / M) * np.asarray(rnorms, dtype=np.float64)[:, None]
+    alpha = (SQRT_HALF_PI / m) * np.asarray(rnorms, dtype=np.float64)[:, None]
     aP = np.abs(Pinv)
     PS = Pinv @ S64.T                                    # d x m
     s1 = np.abs(c[cell]) @ aP.T                          # [n, d]
@@ -73,8 +74,8 @@ def _tolerance(cell, signs, norms, rnorms, Pinv, S64, c, ref, eps_pinv=0.0):
     sc = np.abs(c[cell]).sum(axis=1)[:, None]
     ss = np.abs(S64).sum()
     e = nk * ((2.0 ** -10 + 2.0 ** -20) * (s1 + s2) + 2.0 ** -25 * sps + 2.0 ** -16 * (s1 + s2)
-              + 128 * 2.0 ** -24 * s2b + eps_pinv * (sc + alpha * ss))
-    assert e.shape == (n, D)
+              + d * 2.0 ** -24 * s2b + eps_pinv * (sc + alpha * ss))
+    assert e.shape == (n, d)
     return e + 2.0 ** -8 * (np.abs(ref) + e) + 1e-30
 
 
@@ -87,7 +88,7 @@ def _check(out, ref, tol):
 
 
 def _oracle_case(bits, K, rot_seed=1, sk_seed=0):
-    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed, sk_seed)
+    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed, sk_seed, d=K.shape[1])
     ref = tq.quantize(H.f64(K), Pit, c, S64)
     codes = np.concatenate([tq.pack_planes(ref["cell"], bits), ref["signs"]], axis=1)
     norms = np.stack([ref["norm16"], ref["rnorm16"]], axis=1)
@@ -115,13 +116,14 @@ def test_basis_matches_oracle():
     assert np.array_equal(R[:, :D].cpu().numpy(), P32.astype(np.float16))
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("n", [1, 300, 4099])
-def test_dequantize_matches_oracle(bits, n):
+def test_dequantize_matches_oracle(bits, n, d):
     # oracle codes of seeded keys; n = 300 is two full tiles and a ragged 44,
     # 4099 spans 33 tiles (several per CTA) with a ragged 3
     torch.cuda.set_device(0)
-    K = workloads.random_keys(n, D, 1300 + n + bits, scale=1.4)
+    K = workloads.random_keys(n, d, 1300 + n + bits + d, scale=1.4)
     c, Pit, s_bits, S64, ref, codes, norms, nk, nr = _oracle_case(bits, K)
     P32 = _oracle_pinv32(Pit)
     R = jl.jl_turbo_dequant_basis(torch.from_numpy(P32).cuda(), _bf16_tensor(s_bits))
@@ -132,18 +134,19 @@ def test_dequantize_matches_oracle(bits, n):
     want = tq.dequantize(ref["cell"], ref["signs"], nk, nr, Pit, S64, c)
     tol = _tolerance(ref["cell"], ref["signs"], nk, nr, np.linalg.inv(Pit), S64, c, want)
     worst = _check(out, want, tol)
-    print(f"turbo dequantize bits={bits} n={n}: worst error {worst:.3f} of the bound")
+    print(f"turbo dequantize d={d} bits={bits} n={n}: worst error {worst:.3f} of the bound")
 
 
-def test_dequantize_random_codes_and_edge_norms():
+@pytest.mark.parametrize("d", [128, 64])
+def test_dequantize_random_codes_and_edge_norms(d):
     # random code bits and norms, zero norms (a zero key), a tiny ||r|| whose
     # binary16 alpha is subnormal, and large ||k||
     torch.cuda.set_device(0)
-    rng = np.random.default_rng(8)
+    rng = np.random.default_rng(8 + d)
     for bits in (1, 2, 3):
-        c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=3, sk_seed=4)
+        c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=3, sk_seed=4, d=d)
         n = 260
-        words = (bits * D + M) // 32
+        words = (bits * d + d) // 32
         codes = rng.integers(0, 2 ** 32, size=(n, words), dtype=np.uint64).astype(np.uint32)
         nk16 = rng.uniform(0.01, 60.0, size=n).astype(np.float16)
         nr16 = rng.uniform(0.0, 0.6, size=n).astype(np.float16)
@@ -158,8 +161,8 @@ def test_dequantize_random_codes_and_edge_norms():
                                           torch.from_numpy(norms).cuda(), R, bits)
         torch.cuda.synchronize()
         assert jl.jl_device_error() == 0
-        cell = tq.unpack_planes(codes[:, :bits * D // 32], D, bits)
-        signs = codes[:, bits * D // 32:]
+        cell = tq.unpack_planes(codes[:, :bits * d // 32], d, bits)
+        signs = codes[:, bits * d // 32:]
         nk = nk16.astype(np.float64)
         nr = nr16.astype(np.float64)
         want = tq.dequantize(cell, signs, nk, nr, Pit, S64, c)
@@ -197,17 +200,18 @@ def test_dequantize_empty_and_bad_arguments():
     assert L.jl_turbo_dequant_basis(None, None, 128, 64, None, None) == jl.JL_ERR_UNSUPPORTED
 
 
-def test_end_to_end_library_rotation_quantizer_and_basis():
+@pytest.mark.parametrize("d", [128, 64])
+def test_end_to_end_library_rotation_quantizer_and_basis(d):
     # rotation, sketch, codes and basis all from the library; compared with
     # the oracle's dequantization of its own codes for the keys whose codes
     # and norms agree bit for bit (the others differ only within the
     # quantizer's stated bands, which its own tests check)
     torch.cuda.set_device(0)
     bits, n = 2, 4096
-    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=5)
-    Pi, Pinv = jl.jl_turbo_rotation_init(D, 5)
-    S = jl.jl_sketch_init(M, D, 0)
-    K = workloads.random_keys(n, D, 321)
+    c, pit_bits, Pit, s_bits, S64 = _setup(bits, rot_seed=5, d=d)
+    Pi, Pinv = jl.jl_turbo_rotation_init(d, 5)
+    S = jl.jl_sketch_init(d, d, 0)
+    K = workloads.random_keys(n, d, 321)
     codes, norms = jl.jl_turbo_quantize_keys(K.cuda(), Pi, S, bits)
     R = jl.jl_turbo_dequant_basis(Pinv, S)
     out = jl.jl_turbo_dequantize_keys(codes, norms, R, bits)

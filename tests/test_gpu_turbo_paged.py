@@ -34,16 +34,20 @@ def _codes(ref, bits):
 
 
 @pytest.mark.parametrize("cfg", [
-    # B, Hq, Hkv, P, lens, append, bits, query and new-key dtype
-    (4, 8, 2, 32, [0, 31, 100, 257], True, 2, torch.bfloat16),
-    (3, 4, 4, 64, [1, 64, 130], True, 3, torch.bfloat16),
-    (2, 16, 1, 128, [500, 33], True, 1, torch.bfloat16),
-    (3, 8, 2, 32, [40, 0, 96], False, 2, torch.bfloat16),
-    (3, 8, 2, 64, [70, 1, 200], True, 2, torch.float32),
+    # B, Hq, Hkv, P, lens, append, bits, query and new-key dtype, d = m
+    (4, 8, 2, 32, [0, 31, 100, 257], True, 2, torch.bfloat16, 128),
+    (3, 4, 4, 64, [1, 64, 130], True, 3, torch.bfloat16, 128),
+    (2, 16, 1, 128, [500, 33], True, 1, torch.bfloat16, 128),
+    (3, 8, 2, 32, [40, 0, 96], False, 2, torch.bfloat16, 128),
+    (3, 8, 2, 64, [70, 1, 200], True, 2, torch.float32, 128),
+    (4, 8, 2, 32, [0, 31, 100, 257], True, 2, torch.bfloat16, 64),
+    (3, 4, 4, 64, [1, 64, 130], True, 3, torch.bfloat16, 64),
+    (2, 16, 1, 64, [500, 33], True, 1, torch.float32, 64),
 ])
 def test_turbo_paged_append_decode_matches_oracle(cfg):
     torch.cuda.set_device(0)
-    B, Hq, Hkv, P, lens, append, bits, dt = cfg
+    B, Hq, Hkv, P, lens, append, bits, dt, D = cfg
+    M = D
     rng = np.random.default_rng(B * 100 + P + bits)
     max_len = max(lens) + 1 + 7
     c = tq.lloyd_max(D, bits)

@@ -33,6 +33,8 @@ Workloads (keys/values/queries are synthetic; there are no model weights):
   turbo-paged-gqa  the paged-gqa serving step with TurboQuant-prod keys.
   turbo-dequant-gqa  the turbo-gqa cache's 2,097,152 TurboQuant-prod codes
            (2-bit cells, m=128) and norm pairs turned back into bf16 keys.
+  turbo-gqa-d64  turbo-gqa with 64-dimension heads: d = m = 64 (keys drawn
+           as gqa's, with d = 64).
 
 Recipe details that the workload descriptions leave open:
   * the sketch seed is 0 for every workload;
@@ -123,10 +125,13 @@ TURBO_ROTATION_SEED = 1
 TURBO_PAGED_GQA = PAGED_GQA.with_(name="turbo-paged-gqa", m=128)
 # the turbo-gqa cache's codes turned back into bf16 keys (same data)
 TURBO_DEQUANT_GQA = TURBO_GQA.with_(name="turbo-dequant-gqa")
+# turbo-gqa with 64-dimension heads (one residual bit per coordinate: m = d)
+TURBO_GQA_D64 = TURBO_GQA.with_(name="turbo-gqa-d64", d=64, m=64)
 SEARCH_K = 10
 
 ALL = {w.name: w for w in (SINGLE, GQA, LONG, PREFILL, SWEEP_BASE, PAGED_GQA, DEQUANT_GQA,
-                           SEARCH, TURBO_GQA, TURBO_PAGED_GQA, TURBO_DEQUANT_GQA)}
+                           SEARCH, TURBO_GQA, TURBO_PAGED_GQA, TURBO_DEQUANT_GQA,
+                           TURBO_GQA_D64)}
 
 
 def sweep_points():
