@@ -5,8 +5,10 @@
 // unbiased inner products"), plus the key norm stored beside the code (same
 // page, "PolarQuant" section: one radius per vector in floating point).
 //
-// One warp per key.  S sits transposed in shared memory (St[j][i]) so that
-// lane l reads sketch rows 32w + l of column j conflict-free; lane l then
+// One warp per key.  S sits transposed in shared memory (St[j][i], rows of
+// M + 2 halves so that the transposing stores of consecutive columns j fall
+// in different banks) so that lane l reads sketch rows 32w + l of column j
+// conflict-free; lane l then
 // holds (S k)_{32w + l} for every word w, and a ballot over the warp yields
 // code word w directly (bit l = lane l's sign).  Products are fp32 FMA of the
 // bf16 sketch with the key as stored (bf16 or fp32).
@@ -16,10 +18,11 @@
 namespace jlk {
 
 constexpr int QS_WARPS = 8;
+constexpr int QS_PAD = 2;  // halves of padding per transposed row
 
 template <int M, int D>
 constexpr int qs_smem_bytes() {
-  return M * D * 2 + QS_WARPS * D * 4;
+  return ((D * (M + QS_PAD) * 2 + 15) / 16) * 16 + QS_WARPS * D * 4;
 }
 
 template <int M, int D, bool F32>
@@ -30,13 +33,15 @@ __global__ void __launch_bounds__(QS_WARPS * 32)
                          uint16_t *__restrict__ norms, int *err) {
   // extents the shapes give the buffers (debug index checks)
   const int64_t k_extent = (n - 1) * ldk + D, s_extent = (int64_t)M * D;
+  constexpr int LDT = M + QS_PAD;  // transposed row pitch (halves)
   extern __shared__ __align__(16) uint8_t qsmem[];
-  uint16_t *St = reinterpret_cast<uint16_t *>(qsmem);  // [D][M]
+  uint16_t *St = reinterpret_cast<uint16_t *>(qsmem);  // [D][LDT]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  float *kbuf = reinterpret_cast<float *>(qsmem + M * D * 2) + wid * D;
+  float *kbuf =
+      reinterpret_cast<float *>(qsmem + ((D * LDT * 2 + 15) / 16) * 16) + wid * D;
   for (int e = threadIdx.x; e < M * D; e += blockDim.x) {
     const int i = e / D, j = e - i * D;
-    St[j * M + i] = JL_IN_RANGE(err, e, 1, s_extent) ? S[e] : (uint16_t)0;
+    St[j * LDT + i] = JL_IN_RANGE(err, e, 1, s_extent) ? S[e] : (uint16_t)0;
   }
   __syncthreads();
   constexpr int WORDS = M / 32;
@@ -61,7 +66,7 @@ __global__ void __launch_bounds__(QS_WARPS * 32)
       const float kv = kbuf[j];
 #pragma unroll
       for (int w = 0; w < WORDS; ++w)
-        acc[w] = fmaf(bf16_bits_to_f32(St[j * M + 32 * w + lane]), kv, acc[w]);
+        acc[w] = fmaf(bf16_bits_to_f32(St[j * LDT + 32 * w + lane]), kv, acc[w]);
     }
 #pragma unroll
     for (int w = 0; w < WORDS; ++w) {
