@@ -828,14 +828,15 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
   if constexpr (C::A_SMEM) __syncwarp();
 }
 
-// Query fragments of the int8 scoring with the keys as the MMA's rows (one
-// query head per KV head): the B operand of m16n8k32 is the head's quantised
-// u, column 0 the high limbs and column 1 the low limbs, the other six columns
-// zero.  u is quantised exactly as build_afrags does it (per head to +-32000,
-// two limbs, the same coordinate order: k slot 4t + i of slice c is bit
-// (2c & 7) + 8i of the lane's word t * WORDS + c / 4, and slot 16 + 4t + i bit
-// (2c & 7) + 1 + 8i), so column g of lane (g, t) needs the limbs of head 0:
-// lanes g = 0 and 1 both quantise head 0's row and keep one limb each.
+// Query fragments of the int8 scoring with the keys as the MMA's rows (at
+// most four query heads per KV head): the B operand of m16n8k32 holds head
+// h's quantised u in columns 2h (high limbs) and 2h + 1 (low limbs), columns
+// of absent heads zero.  u is quantised exactly as build_afrags does it (per
+// head to +-32000, two limbs, the same coordinate order: k slot 4t + i of
+// slice c is bit (2c & 7) + 8i of the lane's word t * WORDS + c / 4, and slot
+// 16 + 4t + i bit (2c & 7) + 1 + 8i), so column g of lane (g, t) needs the
+// limbs of head g / 2: lanes 2h and 2h + 1 both quantise head h's row (urow,
+// live) and keep one limb each; hscale / usum come back per lane group.
 template <int M>
 __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool live, int g, int t,
                                                      uint32_t (&bfr)[M / 32][2],
@@ -878,9 +879,10 @@ __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool liv
           hi[j] = (ui + 128) >> 8;
           lo[j] = ui - (hi[j] << 8);
         }
-        bfr[4 * lw + c2][r] = g == 0   ? pack_s8x4(hi[0], hi[1], hi[2], hi[3])
-                              : g == 1 ? pack_s8x4(lo[0], lo[1], lo[2], lo[3])
-                                       : 0u;
+        // column g: head g / 2, the high (g even) or low (g odd) limb
+        bfr[4 * lw + c2][r] = !live        ? 0u
+                              : (g & 1) == 0 ? pack_s8x4(hi[0], hi[1], hi[2], hi[3])
+                                             : pack_s8x4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
   }
@@ -889,14 +891,16 @@ __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool liv
   usum[0] = isum;
 }
 
-// KR: int8 scoring with the keys as the MMA's rows (one query head per KV
-// head, m >= 128, QJL codes): 16 keys per m16n8k32 instead of 8 heads, half
-// the MMAs of the head-rows form when only one head row is live.
+// KR: int8 scoring with the keys as the MMA's rows (at most four query heads
+// per KV head, m >= 128, QJL codes): 16 keys per m16n8k32, the eight columns
+// the two limbs of each head; half the MMAs of the head-rows form, whose
+// 16 rows then hold at most eight live limb rows.
 template <int M, int D, bool S8, bool PAGED, int TB = 0, bool KR = false>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
     decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
   using C = DecCfg<M, D, S8, TB>;
   static_assert(!KR || (S8 && TB == 0 && M >= 128), "keys-as-rows scoring: int8, QJL codes, m >= 128");
+  // (a keys-as-rows launch has at most four heads per unit: p.G <= 4)
   extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -1049,12 +1053,16 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           g < Gg && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + g) * C::CODE_BITS,
                                 C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
       if constexpr (KR) {
-        // one head: lanes g = 0 and 1 quantise head 0's row (one limb each)
-        const float *urow0 = p.U + ((int64_t)b_idx * p.Hq + hq0) * C::CODE_BITS;
-        const bool live0 =
-            g < 2 && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0) * C::CODE_BITS,
-                                 C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
-        build_bfrags_keyrows<M>(urow0, live0, g, t, bfr, hscale, usum);
+        // lanes 2h and 2h + 1 quantise head h's row (one limb each); lane
+        // (g, t) then takes head g's scale and sum for the softmax layout
+        const int hb = g >> 1;
+        const float *urowb = p.U + ((int64_t)b_idx * p.Hq + hq0 + hb) * C::CODE_BITS;
+        const bool liveb =
+            hb < Gg && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + hb) * C::CODE_BITS,
+                                   C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
+        build_bfrags_keyrows<M>(urowb, liveb, g, t, bfr, hscale, usum);
+        hscale[0] = __shfl_sync(0xffffffffu, hscale[0], (8 * g) & 31);
+        usum[0] = __shfl_sync(0xffffffffu, usum[0], (8 * g) & 31);
         (void)urow;
         (void)live;
       } else {
@@ -1179,8 +1187,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           mma_s8_16832(sc[kb][c & 1], a0, a1, a2, a3, bfr[c][0], bfr[c][1]);
         }
       }
-      // lane (g, 0) holds sum_{bit=1} u_int of keys kb*16 + g (v[kb][0]) and
-      // kb*16 + g + 8 (v[kb][1]); key kg*8 + 2t + j sits in lane (2t + j, 0)
+      // lane (g, t) holds head t's sum_{bit=1} u_int of keys kb*16 + g
+      // (v[kb][0]) and kb*16 + g + 8 (v[kb][1]); head g's key kg*8 + 2t + j
+      // sits in lane (2t + j, g)
       int v[2][2];
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
@@ -1191,7 +1200,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       for (int kg = 0; kg < 4; ++kg)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int si = __shfl_sync(0xffffffffu, v[kg >> 1][kg & 1], (2 * t + j) * 4);
+          const int si = __shfl_sync(0xffffffffu, v[kg >> 1][kg & 1], (2 * t + j) * 4 + (g & 3));
           raw[kg][j] = hscale[0] * (float)(2 * si - usum[0]);
         }
       (void)rawq;
@@ -1833,6 +1842,18 @@ static bool decode_use_s8(int G, int m) {
   return G == 1 || m > 256;
 }
 
+// The keys-as-rows int8 scoring (m >= 128, at most four heads per KV head).
+// Measured against the head-rows form on one box (B = 8, T = 32768):
+//   G = 1: faster for m >= 4d, slightly slower at m = 2d;
+//   G = 4: d = 128, m = 512: 137.5 -> 120.7 us; m = 256: 113.0 -> 115.0 us
+//          (slower); m = 128: 106.4 -> 105 us; d = 64, m = 128 / 256 / 512:
+//          75.2 -> 71.2, 102.0 -> 77.4, 108.0 -> 104.0 us.
+static bool decode_use_keyrows(int G, int m, int d) {
+  if (JL_DECODE_SCORE == 1 || m < 128) return false;
+  if (G == 1) return m >= 4 * d;
+  return G <= 4 && (m >= 4 * d || d == 64);
+}
+
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args &&...args) {
@@ -1923,8 +1944,9 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   // one head per KV head and a code at least twice the value row's bytes
   // (m >= 4d): the keys-as-rows int8 scoring (half the MMAs; measured faster
   // there, slightly slower at m = 2d)
-  if constexpr (S8 && M >= 4 * D) {
-    if (pl.G == 1) return launch_scorer_combine<M, D, true, false, 0, true>(pl, p, maps, out, stream);
+  if constexpr (M >= 128) {
+    if (decode_use_keyrows(pl.G, M, D))
+      return launch_scorer_combine<M, D, true, false, 0, true>(pl, p, maps, out, stream);
   }
   return launch_scorer_combine<M, D, S8, false>(pl, p, maps, out, stream);
 }
@@ -2115,8 +2137,9 @@ static cudaError_t launch_paged_t(const DecodePlan &pl, const PagedArgs &a,
   p.seq_lens = a.seq_lens; p.block_table = a.block_table;
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
-  if constexpr (S8 && M >= 4 * D) {  // as the contiguous call
-    if (pl.G == 1) return launch_scorer_combine<M, D, true, true, 0, true>(pl, p, maps, a.out, stream);
+  if constexpr (M >= 128) {  // as the contiguous call
+    if (decode_use_keyrows(pl.G, M, D))
+      return launch_scorer_combine<M, D, true, true, 0, true>(pl, p, maps, a.out, stream);
   }
   return launch_scorer_combine<M, D, S8, true>(pl, p, maps, a.out, stream);
 }

@@ -67,6 +67,8 @@ def _setup(B, Hq, Hkv, d, m, P, lens, max_len, seed, garbage=True):
     (3, 2, 2, 128, 512, 32, [40, 0, 96], False, torch.bfloat16),       # no append, one empty
     (3, 8, 2, 128, 256, 64, [70, 1, 200], True, torch.float32),        # fp32 query and new key
     (2, 2, 2, 64, 256, 32, [95, 31], True, torch.bfloat16),            # MHA, m = 4d: keys as MMA rows
+    (3, 8, 2, 64, 256, 64, [300, 0, 77], True, torch.bfloat16),        # GQA, keys as MMA rows
+    (2, 8, 4, 128, 512, 32, [129, 64], True, torch.float32),           # 2 heads/KV head, m = 4d
 ])
 def test_paged_append_decode_matches_oracle(cfg):
     torch.cuda.set_device(0)

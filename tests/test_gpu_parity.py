@@ -147,6 +147,11 @@ DECODE_CASES = [
     # one head per KV head with m >= 4d: keys as the int8 MMA's rows
     (2, 3, 3, 999, 256, 64, torch.float32, 2.0),
     (1, 2, 2, 4097, 512, 128, torch.bfloat16, 3.0),
+    # two to four heads per KV head, keys as rows (m >= 4d, or d = 64)
+    (2, 8, 2, 1500, 256, 64, torch.bfloat16, 2.0),
+    (1, 6, 2, 700, 128, 64, torch.float32, 1.0),
+    (2, 8, 4, 1000, 512, 128, torch.bfloat16, 3.0),
+    (1, 12, 4, 4096, 512, 64, torch.bfloat16, 1.0),
 ]
 
 
