@@ -837,32 +837,44 @@ __device__ __forceinline__ void build_afrags(const float *urow, bool live, int t
 // 16 + 4t + i bit (2c & 7) + 1 + 8i), so column g of lane (g, t) needs the
 // limbs of head g / 2: lanes 2h and 2h + 1 both quantise head h's row (urow,
 // live) and keep one limb each; hscale / usum come back per lane group.
-template <int M>
+template <int M, int D, int TB = 0>
 __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool live, int g, int t,
-                                                     uint32_t (&bfr)[M / 32][2],
+                                                     uint32_t (&bfr)[DecCfg<M, D, true, TB>::NC][2],
                                                      float (&hscale)[2], int (&usum)[2]) {
-  static_assert(M >= 128, "keys-as-rows scoring: m >= 128");
-  constexpr int WORDS = LaneRuns<M>::WORDS;
-  float amax = 0.f;
+  using C = DecCfg<M, D, true, TB>;
+  static_assert(TB > 0 || M >= 128, "keys-as-rows scoring: m >= 128");
+  // runs of 32-coordinate words the lane reads: contiguous (QJL codes) or,
+  // for cell-plane codes, word 4 lw + t with segment (planes, residual signs)
+  // by run, as build_afrags
+  constexpr int RUNS = TB ? C::LW : LaneRuns<M>::WORDS;
+  auto word_of = [&](int lw) { return TB ? 4 * lw + t : t * RUNS + lw; };
+  auto seg_of = [&](int lw) { return (TB && lw >= C::MSE_RUNS) ? 1 : 0; };
+  float am[2] = {0.f, 0.f};
   if (live) {
 #pragma unroll
-    for (int lw = 0; lw < WORDS; ++lw) {
-      const float *src = urow + 32 * (t * WORDS + lw);
+    for (int lw = 0; lw < RUNS; ++lw) {
+      const float *src = urow + 32 * word_of(lw);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 v = ldg4(src + 4 * k);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        am[seg_of(lw)] = fmaxf(am[seg_of(lw)],
+                               fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
     }
   }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  hscale[0] = amax > 0.f ? amax / 32000.f : 0.f;
-  const float inv = amax > 0.f ? 32000.f / amax : 0.f;
-  int isum = 0;
+  float inv[2];
 #pragma unroll
-  for (int lw = 0; lw < WORDS; ++lw) {
-    const float *src = urow + 32 * (t * WORDS + lw);
+  for (int sg = 0; sg < 2; ++sg) {
+    am[sg] = fmaxf(am[sg], __shfl_xor_sync(0xffffffffu, am[sg], 1));
+    am[sg] = fmaxf(am[sg], __shfl_xor_sync(0xffffffffu, am[sg], 2));
+    hscale[sg] = am[sg] > 0.f ? am[sg] / 32000.f : 0.f;
+    inv[sg] = am[sg] > 0.f ? 32000.f / am[sg] : 0.f;
+  }
+  int isum[2] = {0, 0};
+#pragma unroll
+  for (int lw = 0; lw < RUNS; ++lw) {
+    const int sg = seg_of(lw);
+    const float *src = urow + 32 * word_of(lw);
     float4 x[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) x[k] = live ? ldg4(src + 4 * k) : make_float4(0, 0, 0, 0);
@@ -874,8 +886,8 @@ __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool liv
         int hi[4], lo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int ui = __float2int_rn(f4c(x[(pp + 8 * j) >> 2], pp & 3) * inv);
-          isum += ui;
+          const int ui = __float2int_rn(f4c(x[(pp + 8 * j) >> 2], pp & 3) * inv[sg]);
+          isum[sg] += ui;
           hi[j] = (ui + 128) >> 8;
           lo[j] = ui - (hi[j] << 8);
         }
@@ -886,9 +898,12 @@ __device__ __forceinline__ void build_bfrags_keyrows(const float *urow, bool liv
       }
     }
   }
-  isum += __shfl_xor_sync(0xffffffffu, isum, 1);
-  isum += __shfl_xor_sync(0xffffffffu, isum, 2);
-  usum[0] = isum;
+#pragma unroll
+  for (int sg = 0; sg < 2; ++sg) {
+    isum[sg] += __shfl_xor_sync(0xffffffffu, isum[sg], 1);
+    isum[sg] += __shfl_xor_sync(0xffffffffu, isum[sg], 2);
+    usum[sg] = isum[sg];
+  }
 }
 
 // KR: int8 scoring with the keys as the MMA's rows (at most four query heads
@@ -899,7 +914,7 @@ template <int M, int D, bool S8, bool PAGED, int TB = 0, bool KR = false>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
     decode_scorer_kernel(const __grid_constant__ DecMaps maps, const DecParams p) {
   using C = DecCfg<M, D, S8, TB>;
-  static_assert(!KR || (S8 && TB == 0 && M >= 128), "keys-as-rows scoring: int8, QJL codes, m >= 128");
+  static_assert(!KR || (S8 && (TB > 0 || M >= 128)), "keys-as-rows scoring: int8, m >= 128");
   // (a keys-as-rows launch has at most four heads per unit: p.G <= 4)
   extern __shared__ uint8_t dsmem_raw[];
   const int lane = threadIdx.x & 31;
@@ -1060,9 +1075,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
         const bool liveb =
             hb < Gg && JL_IN_RANGE(p.err, ((int64_t)b_idx * p.Hq + hq0 + hb) * C::CODE_BITS,
                                    C::CODE_BITS, (int64_t)p.B * p.Hq * C::CODE_BITS);
-        build_bfrags_keyrows<M>(urowb, liveb, g, t, bfr, hscale, usum);
-        hscale[0] = __shfl_sync(0xffffffffu, hscale[0], (8 * g) & 31);
-        usum[0] = __shfl_sync(0xffffffffu, usum[0], (8 * g) & 31);
+        build_bfrags_keyrows<M, D, TB>(urowb, liveb, g, t, bfr, hscale, usum);
+#pragma unroll
+        for (int sg = 0; sg < (TB ? 2 : 1); ++sg) {
+          hscale[sg] = __shfl_sync(0xffffffffu, hscale[sg], (8 * g) & 31);
+          usum[sg] = __shfl_sync(0xffffffffu, usum[sg], (8 * g) & 31);
+        }
         (void)urow;
         (void)live;
       } else {
@@ -1167,12 +1185,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
       // rows: keys kb*16 + g (code words wd[2 kb]) and kb*16 + g + 8 (wd[2 kb + 1]);
       // columns 0 / 1: the high / low limb sums; two accumulators per key
       // block (even and odd slices) for independent MMA chains
-      int sc[2][2][4];
+      // (cell-plane codes: sq for the residual-sign slices, c >= NC_MSE)
+      int sc[2][2][4], sq[2][2][4];
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int par = 0; par < 2; ++par)
+        for (int par = 0; par < 2; ++par) {
           sc[kb][par][0] = sc[kb][par][1] = sc[kb][par][2] = sc[kb][par][3] = 0;
+          sq[kb][par][0] = sq[kb][par][1] = sq[kb][par][2] = sq[kb][par][3] = 0;
+        }
 #pragma unroll
       for (int c = 0; c < C::NC; ++c) {
         const int q0 = 2 * c, q1 = 2 * c + 1;
@@ -1184,26 +1205,37 @@ __global__ void __launch_bounds__(DEC_WARPS * 32)
           const uint32_t a1 = (wr8 >> p0) & 0x01010101u;
           const uint32_t a2 = (wr0 >> p1) & 0x01010101u;
           const uint32_t a3 = (wr8 >> p1) & 0x01010101u;
-          mma_s8_16832(sc[kb][c & 1], a0, a1, a2, a3, bfr[c][0], bfr[c][1]);
+          if (TB > 0 && c >= C::NC_MSE)
+            mma_s8_16832(sq[kb][c & 1], a0, a1, a2, a3, bfr[c][0], bfr[c][1]);
+          else
+            mma_s8_16832(sc[kb][c & 1], a0, a1, a2, a3, bfr[c][0], bfr[c][1]);
         }
       }
       // lane (g, t) holds head t's sum_{bit=1} u_int of keys kb*16 + g
       // (v[kb][0]) and kb*16 + g + 8 (v[kb][1]); head g's key kg*8 + 2t + j
       // sits in lane (2t + j, g)
-      int v[2][2];
+      int v[2][2], vq[2][2];
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
         v[kb][0] = (sc[kb][0][0] + sc[kb][1][0]) * 256 + (sc[kb][0][1] + sc[kb][1][1]);
         v[kb][1] = (sc[kb][0][2] + sc[kb][1][2]) * 256 + (sc[kb][0][3] + sc[kb][1][3]);
+        vq[kb][0] = (sq[kb][0][0] + sq[kb][1][0]) * 256 + (sq[kb][0][1] + sq[kb][1][1]);
+        vq[kb][1] = (sq[kb][0][2] + sq[kb][1][2]) * 256 + (sq[kb][0][3] + sq[kb][1][3]);
       }
 #pragma unroll
       for (int kg = 0; kg < 4; ++kg)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int si = __shfl_sync(0xffffffffu, v[kg >> 1][kg & 1], (2 * t + j) * 4 + (g & 3));
+          const int src = (2 * t + j) * 4 + (g & 3);
+          const int si = __shfl_sync(0xffffffffu, v[kg >> 1][kg & 1], src);
           raw[kg][j] = hscale[0] * (float)(2 * si - usum[0]);
+          if constexpr (TB > 0) {
+            const int sj = __shfl_sync(0xffffffffu, vq[kg >> 1][kg & 1], src);
+            rawq[kg][j] = hscale[1] * (float)(2 * sj - usum[1]);
+          }
         }
-      (void)rawq;
+      (void)sq;
+      (void)vq;
     } else if constexpr (S8) {
       int sc[4][4], sq[4][4];
 #pragma unroll
@@ -1966,6 +1998,16 @@ bool make_turbo_decode_plan(int B, int Hq, int Hkv, int64_t T, int m, int d, int
 // four coordinates per expanded register) unless a bf16 build is forced.
 constexpr bool TURBO_S8 = JL_DECODE_SCORE != 1;
 
+// Keys-as-rows scoring of cell-plane codes (at most four heads per KV head;
+// two accumulator sets and two scales per head, planes and residual signs).
+// Measured against the head-rows form on one box (G = 4, B = 8, T = 32768,
+// b-1 = 2): d = 128 119.8 -> 116.0 us, d = 64 82.5 -> 77.5 us; the paged
+// step within noise (114.5 -> 111.0 / 115.3 us).
+static bool turbo_use_keyrows(int G, int d) {
+  (void)d;
+  return G <= 4;
+}
+
 template <int TB, int D>
 static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bool q_f32,
                                          const float *Pinv, const uint16_t *S,
@@ -1997,6 +2039,8 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, codes, norms, scores, softmax_scale, M, err);
+  if (TURBO_S8 && turbo_use_keyrows(pl.G, D))
+    return launch_scorer_combine<M, D, true, false, TB, true>(pl, p, maps, out, stream);
   return launch_scorer_combine<M, D, TURBO_S8, false, TB>(pl, p, maps, out, stream);
 }
 
@@ -2191,6 +2235,8 @@ static cudaError_t launch_turbo_paged_t(const DecodePlan &pl, const PagedArgs &a
   p.seq_lens = a.seq_lens; p.block_table = a.block_table;
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
+  if (TURBO_S8 && turbo_use_keyrows(pl.G, D))
+    return launch_scorer_combine<M, D, true, true, TB, true>(pl, p, maps, a.out, stream);
   return launch_scorer_combine<M, D, TURBO_S8, true, TB>(pl, p, maps, a.out, stream);
 }
 
