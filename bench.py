@@ -696,6 +696,17 @@ def run_dequant(args, rank, world, local_rank):
     }
 
 
+def search_launches_per_call(N, nq, sms=148):
+    """Kernels one jl_search_topk call launches: per pass of 128 queries the
+    query projection, the warm-start sample pass and its merge (when the
+    index has at least eight tiles of 256 per CTA), the full pass and the
+    final merge."""
+    tiles = -(-N // 256)
+    grid = min(sms, tiles)
+    per_pass = 3 + (2 if tiles // (grid * 4) >= 2 else 0)
+    return per_pass * -(-nq // 128)
+
+
 def run_search(args, rank, world, local_rank):
     """Top-k inner-product search over a compressed index."""
     import bit_jl_key_b200 as jl
@@ -793,7 +804,8 @@ def run_search(args, rank, world, local_rank):
                      "frac": tflops / tpeak, "algorithmic_flops_per_launch": flops,
                      "traffic": None},
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": search_launches_per_call(
+            N, nq, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "clocks": clk.summary(),
     }
 

@@ -112,3 +112,13 @@ def test_quantizer_roofline_bound_follows_the_ridge():
             assert r["frac"] == pytest.approx(r["achieved"] / t_burst)
         else:
             assert r["unit"] == "GB/s" and r["frac"] == pytest.approx(rec["GB_per_s"] / peak)
+
+
+def test_search_launch_count_follows_the_call_plan():
+    # projection + full pass + merge, plus the sample pass and its merge when
+    # the index has at least 8 tiles of 256 vectors per CTA; per 128 queries
+    assert bench.search_launches_per_call(8388608, 128) == 5
+    assert bench.search_launches_per_call(1000, 128) == 3
+    assert bench.search_launches_per_call(8388608, 129) == 10
+    assert bench.search_launches_per_call(148 * 256 * 8, 1, sms=148) == 5
+    assert bench.search_launches_per_call(148 * 256 * 8 - 256, 1, sms=148) == 3
