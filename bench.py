@@ -1485,17 +1485,26 @@ def unit_of(w) -> str:
     return "query-vector pairs/s" if w.name == "search" else "keys/s"
 
 
-def time_oracle(w, steps=1, warmup=0):
+def time_oracle(w, steps=1, warmup=0, min_seconds=0.0):
+    """The oracle on the host cores over its bounded sample of the workload:
+    `steps` runs of the sample, repeated until at least min_seconds of CPU
+    work have been timed."""
     import oracle
     run, keys, desc = oracle_sample(w)
     for _ in range(warmup):
         run()
     t = time.perf_counter()
-    for _ in range(steps):
-        run()
-    dt = (time.perf_counter() - t) / steps
+    n = 0
+    while True:
+        for _ in range(steps):
+            run()
+        n += steps
+        if time.perf_counter() - t >= min_seconds:
+            break
+    dt = (time.perf_counter() - t) / n
     return {"value": keys / dt, "unit": unit_of(w), "cores": oracle.max_threads(),
-            "kind": "oracle", "sample": desc, "s_per_step": dt}
+            "kind": "oracle", "sample": desc + (f", repeated {n} times" if n > 1 else ""),
+            "s_per_step": dt, "seconds_timed": dt * n}
 
 
 def run_reference(args, rank, world):
@@ -1564,10 +1573,13 @@ def main():
         cb = None
         args.config_baselines = {}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cb = time_oracle(pick_workload(args.workload, args.batch), steps=1)
+            # about 10 s of oracle work for the line's own baseline, 2 s for
+            # each other config's (the default run stays within minutes)
+            cb = time_oracle(pick_workload(args.workload, args.batch), steps=1,
+                             min_seconds=10.0)
             if args.workload == "gqa" and not args.no_configs:
                 for w in other_configs():
-                    c = time_oracle(w, steps=1)
+                    c = time_oracle(w, steps=1, min_seconds=2.0)
                     args.config_baselines[config_key(w)] = {
                         k: c[k] for k in ("value", "unit", "cores", "kind", "sample")}
         line = run_ours(args, rank, world, local_rank)
