@@ -1127,6 +1127,11 @@ def measure_config(jl, w, dev, steps, warmup, peak, peak_kind, with_score_error,
         if decode:
             decode_call()
 
+    # each workload starts from an idle GPU, as the headline does: the
+    # previous config's sustained load can leave the power controller
+    # holding the clocks down for a while
+    torch.cuda.synchronize(dev)
+    time.sleep(1.0)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
