@@ -432,19 +432,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     // in shared memory (128-byte swizzle) and written by bulk-tensor stores
     const int q = warp & 3;
     const int ew = warp - EXP_WARPS;
+    // the row's stored norm (||k||), 0 past the end; loaded a tile ahead, so
+    // that its latency hides behind the current tile rather than stalling
+    // the warp once the accumulator is ready
+    constexpr int NSTRIDE = C::TURBO ? 2 : 1;  // binary16s per key
+    auto load_norm = [&](int64_t tl) -> uint16_t {
+      const int64_t row = tl * BM + 32 * q + lane;
+      uint16_t h = 0;
+      if (tl < ntiles && row < p.n && JL_IN_RANGE(p.err, NSTRIDE * row, 1, NSTRIDE * p.n))
+        h = __ldg(p.norms + NSTRIDE * row);
+      return h;
+    };
+    uint16_t nrm_next = load_norm(blockIdx.x);
     int64_t t = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++t) {
       const int a = (int)(t & 1);
       const uint32_t aph = (uint32_t)((t >> 1) & 1);
-      const int64_t row = tile * BM + 32 * q + lane;
-      float f = 0.f;
-      if constexpr (!C::TURBO) {
-        if (row < p.n && JL_IN_RANGE(p.err, row, 1, p.n))
-          f = p.coef * __half2float(__ushort_as_half(__ldg(p.norms + row)));
-      } else {
-        if (row < p.n && JL_IN_RANGE(p.err, 2 * row, 1, 2 * p.n))
-          f = __half2float(__ushort_as_half(__ldg(p.norms + 2 * row)));
-      }
+      const uint16_t nrm = nrm_next;
+      nrm_next = load_norm(tile + gridDim.x);
+      const float f = (C::TURBO ? 1.f : p.coef) * __half2float(__ushort_as_half(nrm));
       const int ob = (int)(t % C::OBUF);
       uint8_t *stage = gbase + C::OFF_O + (ew * C::OBUF + ob) * C::OWARP;
       // the staging buffer's previous stores must have read it
