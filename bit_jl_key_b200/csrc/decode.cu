@@ -2003,10 +2003,7 @@ constexpr bool TURBO_S8 = JL_DECODE_SCORE != 1;
 // Measured against the head-rows form on one box (G = 4, B = 8, T = 32768,
 // b-1 = 2): d = 128 119.8 -> 116.0 us, d = 64 82.5 -> 77.5 us; the paged
 // step within noise (114.5 -> 111.0 / 115.3 us).
-static bool turbo_use_keyrows(int G, int d) {
-  (void)d;
-  return G <= 4;
-}
+static bool turbo_use_keyrows(int G) { return G <= 4; }
 
 template <int TB, int D>
 static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bool q_f32,
@@ -2039,7 +2036,7 @@ static cudaError_t launch_turbo_decode_t(const DecodePlan &pl, const void *Q, bo
   if (e != cudaSuccess) return e;
   DecParams p;
   fill_params(p, pl, U, partials, codes, norms, scores, softmax_scale, M, err);
-  if (TURBO_S8 && turbo_use_keyrows(pl.G, D))
+  if (TURBO_S8 && turbo_use_keyrows(pl.G))
     return launch_scorer_combine<M, D, true, false, TB, true>(pl, p, maps, out, stream);
   return launch_scorer_combine<M, D, TURBO_S8, false, TB>(pl, p, maps, out, stream);
 }
@@ -2235,7 +2232,7 @@ static cudaError_t launch_turbo_paged_t(const DecodePlan &pl, const PagedArgs &a
   p.seq_lens = a.seq_lens; p.block_table = a.block_table;
   p.max_pages = a.max_pages; p.page_tokens = a.page_tokens; p.append = pp.append;
   p.score_stride = pl.T;
-  if (TURBO_S8 && turbo_use_keyrows(pl.G, D))
+  if (TURBO_S8 && turbo_use_keyrows(pl.G))
     return launch_scorer_combine<M, D, true, true, TB, true>(pl, p, maps, a.out, stream);
   return launch_scorer_combine<M, D, TURBO_S8, true, TB>(pl, p, maps, a.out, stream);
 }
