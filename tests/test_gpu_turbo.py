@@ -163,7 +163,9 @@ def _decode_inputs(bits, B, Hq, Hkv, T, seed, qdtype=torch.bfloat16, d=D):
 @pytest.mark.parametrize("B,Hq,Hkv,T,d", [(2, 8, 2, 300, 128), (1, 4, 4, 1, 128),
                                           (2, 32, 8, 4096, 128), (1, 8, 1, 1001, 128),
                                           (2, 8, 2, 300, 64), (1, 4, 4, 1, 64),
-                                          (2, 16, 4, 2048, 64), (1, 8, 1, 1001, 64)])
+                                          (2, 16, 4, 2048, 64), (1, 8, 1, 1001, 64),
+                                          # three heads per KV head (keys as MMA rows)
+                                          (2, 6, 2, 777, 128), (1, 9, 3, 1500, 64)])
 def test_decode_matches_oracle(bits, B, Hq, Hkv, T, d):
     torch.cuda.set_device(0)
     gi, (ref_out, ref_sc) = _decode_inputs(bits, B, Hq, Hkv, T, 4000 + T + B + d, d=d)
@@ -178,9 +180,10 @@ def test_decode_matches_oracle(bits, B, Hq, Hkv, T, d):
           f"(rel {rel:.2e})")
 
 
-def test_decode_fp32_queries():
+@pytest.mark.parametrize("d", [128, 64])
+def test_decode_fp32_queries(d):
     torch.cuda.set_device(0)
-    gi, (ref_out, ref_sc) = _decode_inputs(2, 1, 8, 2, 640, 77, qdtype=torch.float32)
+    gi, (ref_out, ref_sc) = _decode_inputs(2, 1, 8, 2, 640, 77 + d, qdtype=torch.float32, d=d)
     out, sc = jl.jl_turbo_decode_attention(gi["Q"], gi["Pinv"], gi["S"], gi["codes"], gi["norms"],
                                            gi["V"], 2, want_scores=True)
     torch.cuda.synchronize()
