@@ -110,6 +110,9 @@ def rank_workload(args, rank: int) -> workloads.Workload:
 
 
 def _pick(name: str) -> workloads.Workload:
+    if name == "long-cp":
+        # the long workload, its context split across the ranks
+        return workloads.ALL["long"]
     if name.startswith("sweep-"):
         # sweep-m<M>-d<D>
         m = int(name.split("-m")[1].split("-")[0])
@@ -1187,9 +1190,136 @@ def config_key(w) -> str:
     return w.name if w.name != "sweep" else f"sweep-m{w.m}-d{w.d}"
 
 
+def run_context_parallel(args, rank, world, local_rank):
+    """--workload long-cp: one sequence's context split across the ranks
+    (strong scaling).  Rank r holds keys context_range(T, world, r) of every
+    head; a step quantizes the rank's slice of keys, decodes it to softmax
+    states, all-gathers the states and merges them (the output is the same on
+    every rank).  value = all keys of the context over the slowest rank's
+    step time."""
+    import bit_jl_key_b200 as jl
+    from bit_jl_key_b200.context_parallel import context_range, decode_context_parallel
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = pick_workload(args.workload, args.batch)
+    a, b = context_range(w.T, world, rank)
+    wl = w.with_(T=b - a)                       # this rank's share, for the byte counts
+    peak, peak_kind = load_peaks()
+    S = jl.jl_sketch_init(w.m, w.d, w.sketch_seed, device=dev)
+    K = workloads.keys(w, dev)[:, :, a:b].contiguous()
+    V = workloads.values(w, dev)[:, :, a:b].contiguous()
+    torch.cuda.empty_cache()
+    Q = workloads.queries(w, dev)
+    W = w.m // 32
+    n_keys = wl.B * wl.Hkv * wl.T
+    signs = torch.empty((wl.B, wl.Hkv, wl.T, W), dtype=torch.int32, device=dev)
+    norms = torch.empty((wl.B, wl.Hkv, wl.T), dtype=torch.float16, device=dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ws_bytes = jl.jl_decode_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.T, wl.m, wl.d)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def quantize():
+        jl.jl_quantize_keys(K.view(-1, w.d), S, signs.view(-1, W), norms.view(-1))
+
+    def decode_call():
+        decode_context_parallel(Q, S, signs, norms, V, w.softmax_scale, out=out, workspace=ws)
+
+    def step():
+        quantize()
+        decode_call()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        clk.region_start()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        barrier()
+        clk.region_end()
+        q_ms = _timed_loop(stream, quantize, args.steps)
+        d_ms = _timed_loop(stream, decode_call, args.steps)
+        barrier()
+        clk.extend(top_up=step)
+    if jl.jl_device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_step = reduce_max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    q_ms = reduce_max_over_ranks(q_ms, world, dev)
+    d_ms = reduce_max_over_ranks(d_ms, world, dev)
+    keys_all = w.B * w.Hkv * w.T
+
+    # ---- end to end: the rank's keys, values and the queries from pinned
+    # host memory, the output back
+    e2e = None
+    if not args.no_e2e:
+        hK, hV, hQ = (t.cpu().pin_memory() for t in (K, V, Q))
+        hOut = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ))
+
+        def e2e_step():
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            Q.copy_(hQ, non_blocking=True)
+            step()
+            hOut.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        barrier()
+        e_steps = max(3, args.steps // 4)
+        e_ms = _timed_loop(stream, e2e_step, e_steps)
+        barrier()
+        e_ms = reduce_max_over_ranks(e_ms, world, dev)
+        e2e = {"value": keys_all / (e_ms * 1e-3), "unit": "keys/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hOut.numel() * 2}
+    phases = phase_records(wl, n_keys, q_ms, d_ms, peak, True,
+                           {"states exchanged per rank": w.B * w.Hq * (w.d + 2) * 4})
+    rooflines = {ph: roofline_of(ph, phases[ph], wl, peak, peak_kind, full_size=False,
+                                 n_keys=n_keys) for ph in phases}
+    rooflines["decode"]["kernel"] = ("jl_decode_attention_state (qproj + decode_scorer_kernel "
+                                     "+ combine) + all-gather + merge_states_kernel")
+    dom = max(phases, key=lambda k: phases[k]["ms"])
+    return {
+        "metric": "decode keys scored/s and achieved HBM GB/s (% peak); quantize tokens/s",
+        "value": keys_all / (ms_step * 1e-3), "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": f"{w.name} context split over {world} rank(s): B={w.B} "
+                               f"Hq={w.Hq} Hkv={w.Hkv} T={w.T} (this rank {wl.T}) "
+                               f"d={w.d} m={w.m}",
+                   "global_batch": w.B, "seq_len": w.T, "parallelism": f"cp{world}",
+                   "l2": "inputs exceed L2 (126 MB) at up to 8 ranks; no flush"},
+        "phases": phases,
+        "phase_timing": "each phase alone: K back-to-back calls, CUDA events at the ends; "
+                        "max over ranks",
+        "roofline": rooflines[dom],
+        "rooflines": rooflines,
+        "e2e": e2e,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import bit_jl_key_b200 as jl
 
+    if args.workload == "long-cp":
+        return run_context_parallel(args, rank, world, local_rank)
     if args.workload in ("turbo-gqa", "turbo-gqa-d64"):
         return run_turbo(args, rank, world, local_rank)
     if args.workload == "search":

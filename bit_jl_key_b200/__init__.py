@@ -56,7 +56,8 @@ EXPORTED = ("jl_status_string", "jl_sketch_init", "jl_quantize_keys",
             "jl_turbo_rotation_init", "jl_turbo_quantize_keys", "jl_turbo_decode_workspace_bytes",
             "jl_turbo_decode_attention", "jl_turbo_decode_paged_workspace_bytes",
             "jl_turbo_decode_attention_paged", "jl_turbo_dequant_basis",
-            "jl_turbo_dequantize_keys", "jl_test_drop_copies", "jl_build_flags")
+            "jl_turbo_dequantize_keys", "jl_test_drop_copies", "jl_build_flags",
+            "jl_decode_attention_state", "jl_merge_attention_states")
 
 # device error codes (jl_device_error)
 JL_DERR_TC_WAIT_TIMEOUT = 1
@@ -99,6 +100,10 @@ def load():
     L.jl_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32,
                                       i64, i32, i32, ctypes.c_float, vp, vp,
                                       vp, sz, vp]
+    L.jl_decode_attention_state.restype = i32
+    L.jl_decode_attention_state.argtypes = list(L.jl_decode_attention.argtypes)
+    L.jl_merge_attention_states.restype = i32
+    L.jl_merge_attention_states.argtypes = [vp, i32, i64, i32, vp, vp]
     L.jl_decode_attention_noalloc.restype = i32
     L.jl_decode_attention_noalloc.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32,
                                               i32, i64, i32, i32, ctypes.c_float,
@@ -359,6 +364,64 @@ def jl_decode_attention(Q, S, signs, norms, V, softmax_scale=None, out=None,
            "jl_decode_attention")
     if scores is not None:
         return out, scores
+    return out
+
+
+def jl_decode_attention_state(Q, S, signs, norms, V, softmax_scale=None, state=None,
+                              scores=None, want_scores=False, workspace=None,
+                              stream=None):
+    """jl_decode_attention over one part of a context, returning the softmax
+    state of every (b, query head) instead of the output: state [B, Hq, d + 2]
+    fp32 holding (acc[d], max, sum), for jl_merge_attention_states.  Returns
+    state, or (state, scores [B, Hq, T]) when ``want_scores``."""
+    L = load()
+    B, Hq, Hkv, T, m, d, qt = _decode_shapes(Q, S, signs, norms, V, None, scores)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if state is None:
+        state = torch.empty((B, Hq, d + 2), dtype=torch.float32, device=Q.device)
+    elif (state.shape != (B, Hq, d + 2) or state.dtype != torch.float32
+          or not state.is_contiguous()):
+        raise ValueError(f"state must be a contiguous float32 {(B, Hq, d + 2)} tensor")
+    _need_cuda(state)
+    if want_scores and scores is None:
+        scores = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
+    need = jl_decode_workspace_bytes(B, Hq, Hkv, T, m, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Q.device)
+    _check(L.jl_decode_attention_state(_ptr(Q), qt, _ptr(S), _ptr(signs), _ptr(norms),
+                                       _ptr(V), B, Hq, Hkv, T, m, d,
+                                       ctypes.c_float(softmax_scale), _ptr(state),
+                                       _ptr(scores), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(Q, stream)),
+           "jl_decode_attention_state")
+    if scores is not None:
+        return state, scores
+    return state
+
+
+def jl_merge_attention_states(states, out=None, stream=None):
+    """Attention output [..., d] bf16 from the states [R, ..., d + 2] fp32 of R
+    disjoint parts of each row's context (jl_decode_attention_state)."""
+    L = load()
+    if states.dim() < 2 or states.dtype != torch.float32 or not states.is_contiguous():
+        raise ValueError("states must be a contiguous float32 [R, ..., d + 2] tensor")
+    R = states.shape[0]
+    d = states.shape[-1] - 2
+    lead = tuple(states.shape[1:-1])
+    rows = 1
+    for n in lead:
+        rows *= n
+    if out is None:
+        out = torch.empty(lead + (d,), dtype=torch.bfloat16, device=states.device)
+    elif (tuple(out.shape) != lead + (d,) or out.dtype != torch.bfloat16
+          or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous bf16 {lead + (d,)} tensor")
+    _need_cuda(states, out)
+    _check(L.jl_merge_attention_states(_ptr(states), R, rows, d, _ptr(out),
+                                       _stream(states, stream)),
+           "jl_merge_attention_states")
     return out
 
 

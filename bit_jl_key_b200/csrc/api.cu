@@ -293,6 +293,35 @@ int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *S,
                                       (cudaStream_t)stream));
 }
 
+int jl_decode_attention_state(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                              const uint32_t *signs, const uint16_t *norms,
+                              const uint16_t *V, int B, int Hq, int Hkv, int64_t T,
+                              int m, int d, float softmax_scale, float *state,
+                              float *scores, void *workspace, size_t workspace_bytes,
+                              jl_stream_t stream) {
+  jlk::DecodePlan p;
+  bool empty = false;
+  // the state buffer takes the output's checks (non-null, 4-byte aligned)
+  const int st = jlk::validate_decode(Q, q_dtype, S, signs, norms, V, B, Hq, Hkv, T, m, d,
+                                      softmax_scale, reinterpret_cast<const uint16_t *>(state),
+                                      scores, &p, &empty);
+  if (st != JL_OK || empty) return st;
+  if (!workspace || workspace_bytes < p.total_bytes || !aligned(workspace, 256))
+    return JL_ERR_WORKSPACE;
+  return from_cuda(jlk::launch_decode(p, Q, q_dtype == JL_F32, S, signs, norms, V,
+                                      softmax_scale, nullptr, scores, workspace,
+                                      (cudaStream_t)stream, state));
+}
+
+int jl_merge_attention_states(const float *states, int R, int64_t rows, int d,
+                              uint16_t *out, jl_stream_t stream) {
+  if (R < 1 || R > 65536 || rows < 0 || rows >= ((int64_t)1 << 31)) return JL_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return JL_ERR_UNSUPPORTED;
+  if (rows == 0) return JL_OK;
+  if (!states || !out || !aligned(states, 4) || !aligned(out, 4)) return JL_ERR_INVALID_ARG;
+  return from_cuda(jlk::launch_merge_states(states, R, rows, d, out, (cudaStream_t)stream));
+}
+
 size_t jl_decode_paged_workspace_bytes(int B, int Hq, int Hkv, int64_t max_len, int m,
                                        int d) {
   jlk::DecodePlan p;

@@ -135,6 +135,7 @@ struct DecParams {
   int max_pages, page_tokens, append, units, B, UH;
   unsigned long long wait_ns;  // bound of every copy wait (WAIT_LIMIT_NS unless a test set one)
   int drop_copies;             // test hook: the scorer issues no copy (its waits run out)
+  float *state;                // nullable [B][Hq][D + 2]: the merged state instead of out
 };
 
 // Bulk-tensor maps of one decode call.  Values always go through `value`
@@ -1455,7 +1456,7 @@ template <int D, bool PAGED>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
                                                            uint16_t *__restrict__ out) {
   __shared__ float wts[COMB_MAX_SLOTS];
-  __shared__ float inv_l;
+  __shared__ float inv_l, comb_mx, comb_l;
   __shared__ int64_t red[2][D / 32];
   const float *__restrict__ partials = p.partials;
   const int Hq = p.Hq, G = p.G;
@@ -1540,7 +1541,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) inv_l = 1.f / L;
+    if (lane == 0) {
+      inv_l = 1.f / L;
+      comb_mx = mx;
+      comb_l = L;
+    }
   }
   __syncthreads();
   const int dim = threadIdx.x;
@@ -1552,8 +1557,67 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecParams p,
 #pragma unroll
   for (int s = 0; s < 32; ++s) o = s < n ? fmaf(wts[s], v[s], o) : o;
   for (int s = 32; s < n; ++s) o = fmaf(wts[s], rec0[s * sstride + dim], o);
+  if (p.state) {
+    // the unit's state as one record of the same form: (acc, max, sum)
+    const int64_t at = (int64_t)bh * (D + 2);
+    if (JL_IN_RANGE(p.err, at, D + 2, (int64_t)p.B * Hq * (D + 2))) {
+      p.state[at + dim] = o;
+      if (dim == 0) {
+        p.state[at + D] = comb_mx;
+        p.state[at + D + 1] = comb_l;
+      }
+    }
+    return;
+  }
   if (JL_IN_RANGE(p.err, (int64_t)bh * D + dim, 1, (int64_t)p.B * Hq * D))
     out[(int64_t)bh * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(o * inv_l));
+}
+
+// ---------------------------------------------------------------------------
+// 3b. merge of attention states computed over disjoint parts of one context
+// (as the combine leaves them with a state buffer: acc[D], max, sum, softmax
+// weights 2^(x - max)).  The same log-sum-exp merge as the combine: every
+// part is rescaled to the largest max; parts with no keys (sum 0) drop out,
+// and a row with none is zero.  One CTA of D threads per row.
+template <int D>
+__global__ void __launch_bounds__(D) merge_states_kernel(const float *__restrict__ states,
+                                                         int R, int64_t rows,
+                                                         uint16_t *__restrict__ out, int *err) {
+  const int64_t row = blockIdx.x;
+  const int dim = threadIdx.x;
+  const size_t pstride = (size_t)rows * (D + 2);
+  const float *rec = states + (size_t)row * (D + 2);
+  float mx = -INFINITY;
+  for (int r = 0; r < R; ++r) {
+    const float l = __ldg(rec + r * pstride + D + 1);
+    if (l > 0.f) mx = fmaxf(mx, __ldg(rec + r * pstride + D));
+  }
+  float L = 0.f, o = 0.f;
+  if (mx > -INFINITY) {
+    for (int r = 0; r < R; ++r) {
+      const float l = __ldg(rec + r * pstride + D + 1);
+      if (l > 0.f) {
+        const float w = fast_exp2(__ldg(rec + r * pstride + D) - mx);
+        L = fmaf(w, l, L);
+        o = fmaf(w, __ldg(rec + r * pstride + dim), o);
+      }
+    }
+  }
+  if (JL_IN_RANGE(err, row * D + dim, 1, rows * D))
+    out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L > 0.f ? o / L : 0.f));
+}
+
+cudaError_t launch_merge_states(const float *states, int R, int64_t rows, int d,
+                                uint16_t *out, cudaStream_t stream) {
+  int *err = device_error_ptr();
+  if (err == nullptr) return cudaErrorInvalidSymbol;
+  if (d == 128)
+    merge_states_kernel<128><<<(unsigned)rows, 128, 0, stream>>>(states, R, rows, out, err);
+  else if (d == 64)
+    merge_states_kernel<64><<<(unsigned)rows, 64, 0, stream>>>(states, R, rows, out, err);
+  else
+    return cudaErrorNotSupported;
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -1919,6 +1983,7 @@ static void fill_params(DecParams &p, const DecodePlan &pl, float *U, float *par
   p.UH = pl.Hkv * pl.HG;
   p.wait_ns = wait_limit_ns();
   p.drop_copies = 0;
+  p.state = nullptr;
 }
 
 // Launch the scorer (one wave, <= the plan's warp bound) and the combine.
@@ -1951,7 +2016,7 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
                                    const uint32_t *signs, const uint16_t *norms,
                                    const uint16_t *V, float softmax_scale,
                                    uint16_t *out, float *scores,
-                                   void *workspace, cudaStream_t stream) {
+                                   void *workspace, cudaStream_t stream, float *state) {
   float *U = reinterpret_cast<float *>(workspace);
   float *partials =
       reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + pl.u_bytes);
@@ -1973,6 +2038,7 @@ static cudaError_t launch_decode_t(const DecodePlan &pl, const void *Q,
   DecParams p;
   fill_params(p, pl, U, partials, signs, norms, scores, softmax_scale, M, err);
   p.drop_copies = test_drop_copies() ? 1 : 0;
+  p.state = state;
   // one head per KV head and a code at least twice the value row's bytes
   // (m >= 4d): the keys-as-rows int8 scoring (half the MMAs; measured faster
   // there, slightly slower at m = 2d)
@@ -2080,16 +2146,16 @@ cudaError_t launch_decode(const DecodePlan &pl, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,
                           const uint16_t *norms, const uint16_t *V,
                           float softmax_scale, uint16_t *out, float *scores,
-                          void *workspace, cudaStream_t stream) {
+                          void *workspace, cudaStream_t stream, float *state) {
   const bool s8 = decode_use_s8(pl.G, pl.m);
 #define JL_CASE(MM, DD)                                                         \
   if (pl.m == MM && pl.d == DD)                                                 \
     return s8 ? launch_decode_t<MM, DD, true>(pl, Q, q_f32, S, signs, norms, V, \
                                               softmax_scale, out, scores,       \
-                                              workspace, stream)                \
+                                              workspace, stream, state)         \
               : launch_decode_t<MM, DD, false>(pl, Q, q_f32, S, signs, norms, V, \
                                                softmax_scale, out, scores,      \
-                                               workspace, stream);
+                                               workspace, stream, state);
   JL_CASE(64, 64) JL_CASE(128, 64) JL_CASE(256, 64) JL_CASE(512, 64)
   JL_CASE(64, 128) JL_CASE(128, 128) JL_CASE(256, 128) JL_CASE(512, 128)
 #undef JL_CASE

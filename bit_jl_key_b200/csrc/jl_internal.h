@@ -114,7 +114,12 @@ cudaError_t launch_decode(const DecodePlan &p, const void *Q, bool q_f32,
                           const uint16_t *S, const uint32_t *signs,
                           const uint16_t *norms, const uint16_t *V,
                           float softmax_scale, uint16_t *out, float *scores,
-                          void *workspace, cudaStream_t stream);
+                          void *workspace, cudaStream_t stream, float *state = nullptr);
+
+// Merge R attention states per row ([R][rows][d + 2], each (acc, max, sum))
+// into bf16 rows [rows][d].
+cudaError_t launch_merge_states(const float *states, int R, int64_t rows, int d,
+                                uint16_t *out, cudaStream_t stream);
 
 struct PagedArgs {
   const void *Q;

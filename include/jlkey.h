@@ -166,6 +166,48 @@ JL_API int jl_decode_attention(const void *Q, jl_dtype q_dtype, const uint16_t *
                         jl_stream_t stream);
 
 /*
+ * jl_decode_attention_state -- jl_decode_attention over one part of a context
+ * whose keys are spread over several buffers (or GPUs), stopping before the
+ * final division: the softmax state of each (b, query head), for
+ * jl_merge_attention_states to combine with the other parts' states.
+ * Defines: the same estimator, logit and value sum as jl_decode_attention;
+ * softmax over a union of disjoint key sets as the log-sum-exp merge of the
+ * sets' states (plain algebra of the softmax; the pages do not treat it).
+ *   All arguments as jl_decode_attention, for this part's T keys, except:
+ *   state    : out, device, B x Hq x (d + 2) fp32, 4-byte aligned (replaces
+ *              `out`).  Record (b, h) holds acc[0..d-1], mx, l with
+ *              weights w_t = 2^(log2(e) * logit_t - mx): acc = sum_t w_t v_t
+ *              and l = sum_t w_t, so the part's output is acc / l.  Only
+ *              acc / l and mx + log2(l) are fixed; mx is the kernel's
+ *              running maximum.
+ *   scores   : optional, B x Hq x T as in jl_decode_attention (this part).
+ * Errors: as jl_decode_attention.
+ */
+JL_API int jl_decode_attention_state(const void *Q, jl_dtype q_dtype, const uint16_t *S,
+                              const uint32_t *signs, const uint16_t *norms,
+                              const uint16_t *V, int B, int Hq, int Hkv, int64_t T,
+                              int m, int d, float softmax_scale, float *state,
+                              float *scores, void *workspace, size_t workspace_bytes,
+                              jl_stream_t stream);
+
+/*
+ * jl_merge_attention_states -- the attention output of a context split into
+ * R parts, from the parts' states (jl_decode_attention_state).
+ * Defines: softmax over the union of the parts: with M = max over parts of
+ * mx_r, out = sum_r 2^(mx_r - M) acc_r / sum_r 2^(mx_r - M) l_r.  A part
+ * whose l is 0 (no keys) contributes nothing; a row with no part left is 0.
+ *   states   : in, device, R x rows x (d + 2) fp32 (part r's records at
+ *              r * rows * (d + 2)), 4-byte aligned.
+ *   R        : number of parts, 1 <= R <= 65536.
+ *   rows     : records per part (B x Hq), 0 <= rows < 2^31; 0 is a no-op.
+ *   d        : 64 or 128.
+ *   out      : out, device, rows x d bf16 (nearest), 4-byte aligned.
+ * Errors: JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED (d), JL_ERR_CUDA.
+ */
+JL_API int jl_merge_attention_states(const float *states, int R, int64_t rows, int d,
+                              uint16_t *out, jl_stream_t stream);
+
+/*
  * jl_dequantize_keys -- explicit dequantizer of the codes.
  * Defines: Q^-1(z) = sqrt(pi/2)/d * S^T z ("The Geometry of Forgetting: How
  * Three Papers Cracked KV Cache Quantization", section "QJL: one bit, zero

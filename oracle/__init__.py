@@ -270,6 +270,35 @@ def decode(Q, S, signs, norms, V, softmax_scale: float, want_scores=False):
     return out, sc
 
 
+def decode_state(Q, S, signs, norms, V, softmax_scale: float):
+    """Softmax state of decode attention over one part of a context.
+
+    The pages say nothing about splitting a context; this is the plain
+    algebra of the softmax.  For a part holding keys t, with logits
+    x_t = softmax_scale * s_t (s the estimator, as in ``decode``), returns
+    (out [B,Hq,d], lse2 [B,Hq]): the part's own attention output and
+    lse2 = log2 sum_t exp(x_t).  Both are unique, whatever running maximum
+    an implementation keeps.
+    """
+    out, sc = decode(Q, S, signs, norms, V, softmax_scale, want_scores=True)
+    x = softmax_scale * sc                                  # [B,Hq,T]
+    mx = x.max(axis=-1, keepdims=True)
+    lse2 = (mx[..., 0] + np.log(np.exp(x - mx).sum(axis=-1))) / math.log(2.0)
+    return out, lse2
+
+
+def merge_states(outs, lse2s):
+    """Attention output of a context split into R parts from the parts'
+    states (``decode_state``): each part's output weighted by its share
+    2^lse2_r / sum_r 2^lse2_r of the softmax mass.  outs [R,...,d],
+    lse2s [R,...]."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lse2s = np.asarray(lse2s, dtype=np.float64)
+    top = lse2s.max(axis=0, keepdims=True)
+    w = np.exp2(lse2s - top)                                # [R,...]
+    return (w[..., None] * outs).sum(axis=0) / w.sum(axis=0)[..., None]
+
+
 def exact_attention(Q, K, V, softmax_scale: float, want_scores=False):
     """Attention with the unquantized keys (context only)."""
     Q = _c(Q, np.float64)

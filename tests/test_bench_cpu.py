@@ -17,6 +17,8 @@ def test_every_named_workload_is_selectable():
     w = bench.pick_workload("sweep-m512-d64")
     assert (w.m, w.d) == (512, 64)
     assert bench.pick_workload("gqa", 2).B == 2
+    # the context-split run times the long workload, its context over the ranks
+    assert bench.pick_workload("long-cp") == workloads.ALL["long"]
 
 
 def test_byte_accounting_matches_the_stated_per_key_sizes():

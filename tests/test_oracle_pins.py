@@ -296,6 +296,55 @@ def test_decode_identical_keys_average_values():
     np.testing.assert_allclose(out[0, 0], V[0, 0].mean(0), rtol=1e-12, atol=1e-14)
 
 
+def test_decode_state_of_known_scores():
+    # S = I as above: the part's lse2 is log2 of the library's sum of exps of
+    # the known logits, and its output is the plain decode of the part
+    rng = np.random.default_rng(21)
+    d = m = 32
+    T = 11
+    q = rng.standard_normal(d) * 3.0
+    codes = rng.integers(0, 2 ** 32, size=T, dtype=np.uint64).astype(np.uint32)
+    norms = rng.uniform(0.5, 3.0, size=T)
+    bits = (codes[:, None] >> np.arange(32)[None, :]) & 1
+    s = math.sqrt(math.pi / 2) / m * norms * (np.where(bits, 1.0, -1.0) @ q)
+    V = rng.standard_normal((T, d))
+    scale = 0.61
+    out, lse2 = oracle.decode_state(q[None, None, :], _identity_sketch(d),
+                                    codes.reshape(1, 1, T, 1), norms[None, None, :],
+                                    V[None, None], scale)
+    assert lse2.shape == (1, 1)
+    np.testing.assert_allclose(lse2[0, 0], scipy.special.logsumexp(scale * s) / math.log(2),
+                               rtol=1e-13)
+    np.testing.assert_allclose(out[0, 0], scipy.special.softmax(scale * s) @ V, rtol=1e-12,
+                               atol=1e-13)
+
+
+@pytest.mark.parametrize("cuts", [(1,), (20, 21), (5, 17, 30, 39), (40,)])
+def test_merge_of_split_states_equals_whole_decode(cuts):
+    # softmax over a union of disjoint key sets: merging the parts' states
+    # must give the C decode over the whole context (GQA, peaked logits)
+    rng = np.random.default_rng(22)
+    B, Hq, Hkv, T, m, d = 2, 4, 2, 41, 64, 16
+    S = rng.standard_normal((m, d))
+    K = rng.standard_normal((B * Hkv * T, d)) * 2.0
+    signs, norms, _, _ = oracle.quantize(K, S)
+    signs = signs.reshape(B, Hkv, T, m // 32)
+    norms = norms.reshape(B, Hkv, T)
+    V = rng.standard_normal((B, Hkv, T, d))
+    Q = rng.standard_normal((B, Hq, d)) * 2.0
+    scale = 0.9
+    whole, _ = oracle.decode(Q, S, signs, norms, V, scale)
+    edges = (0,) + tuple(cuts) + (T,)
+    parts = [oracle.decode_state(Q, S, signs[:, :, a:b], norms[:, :, a:b], V[:, :, a:b],
+                                 scale) for a, b in zip(edges[:-1], edges[1:])]
+    merged = oracle.merge_states([p[0] for p in parts], [p[1] for p in parts])
+    np.testing.assert_allclose(merged, whole, rtol=1e-11, atol=1e-12)
+    # the parts' softmax masses add up to the whole's
+    _, lse_whole = oracle.decode_state(Q, S, signs, norms, V, scale)
+    tot = np.log2(sum(np.exp2(p[1]) for p in parts))
+    np.testing.assert_allclose(tot, lse_whole, rtol=1e-12)
+
+
 def test_decode_grouped_query_head_mapping():
     # Hq = 6, Hkv = 2: heads 0..2 read KV head 0, heads 3..5 read KV head 1
     rng = np.random.default_rng(6)
