@@ -167,6 +167,71 @@ def test_noalloc_argument_errors_match_decode(lib):
         assert (na == jl.JL_OK) == (kw == dict(B=0)), kw
 
 
+def test_state_decode_argument_errors_match_decode(lib):
+    # the state variant takes jl_decode_attention's checks, the state buffer
+    # standing in for the output
+    f = lib.jl_decode_attention_state
+    g = lib.jl_decode_attention
+    ok = dict(Q=FAKE, qt=jl.JL_BF16, S=FAKE, signs=FAKE, norms=FAKE, V=FAKE,
+              B=2, Hq=8, Hkv=2, T=100, m=256, d=128, scale=0.1, out=FAKE,
+              scores=NULL, ws=FAKE, wsb=1 << 40)
+
+    def both(**kw):
+        a = dict(ok, **kw)
+        args = (a["Q"], a["qt"], a["S"], a["signs"], a["norms"], a["V"], a["B"], a["Hq"],
+                a["Hkv"], a["T"], a["m"], a["d"], ctypes.c_float(a["scale"]), a["out"],
+                a["scores"], a["ws"], a["wsb"], NULL)
+        return f(*args), g(*args)
+
+    cases = [dict(B=0), dict(T=0), dict(Hq=6, Hkv=4), dict(Hkv=0), dict(qt=5), dict(m=48),
+             dict(d=256), dict(V=MISALIGNED), dict(signs=MISALIGNED),
+             dict(out=ctypes.c_void_p((1 << 20) + 2)), dict(scale=float("nan")),
+             dict(ws=NULL), dict(wsb=jl.jl_decode_workspace_bytes(2, 8, 2, 100, 256, 128) - 1)]
+    cases += [{k: NULL} for k in ("Q", "S", "signs", "norms", "V", "out")]
+    for kw in cases:
+        st, dec = both(**kw)
+        assert st == dec, (kw, st, dec)
+        assert (st == jl.JL_OK) == (kw == dict(B=0)), kw
+
+
+def test_merge_states_argument_errors(lib):
+    f = lib.jl_merge_attention_states
+
+    def call(states=FAKE, R=2, rows=16, d=128, out=FAKE):
+        return f(states, R, rows, d, out, NULL)
+
+    assert call(rows=0) == jl.JL_OK                   # nothing to merge
+    assert call(R=0) == jl.JL_ERR_INVALID_ARG
+    assert call(R=65537) == jl.JL_ERR_INVALID_ARG
+    assert call(rows=-1) == jl.JL_ERR_INVALID_ARG
+    assert call(rows=1 << 31) == jl.JL_ERR_INVALID_ARG
+    assert call(d=96) == jl.JL_ERR_UNSUPPORTED
+    assert call(states=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(out=NULL) == jl.JL_ERR_INVALID_ARG
+    assert call(states=ctypes.c_void_p((1 << 20) + 2)) == jl.JL_ERR_INVALID_ARG
+    assert call(out=ctypes.c_void_p((1 << 20) + 2)) == jl.JL_ERR_INVALID_ARG
+
+
+def test_state_wrappers_refuse_bad_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):             # well-formed, but on the host
+        jl.jl_merge_attention_states(torch.zeros(2, 4, 130))
+    with pytest.raises(ValueError):
+        jl.jl_merge_attention_states(torch.zeros(2, 4, 130, dtype=torch.float64))
+    with pytest.raises(ValueError):
+        jl.jl_merge_attention_states(torch.zeros(2, 4, 130),
+                                     out=torch.zeros(4, 64, dtype=torch.bfloat16))
+    B, Hq, Hkv, T, m, d = 1, 4, 2, 64, 256, 128
+    args = (torch.zeros(B, Hq, d, dtype=torch.bfloat16), torch.zeros(m, d, dtype=torch.bfloat16),
+            torch.zeros(B, Hkv, T, m // 32, dtype=torch.int32),
+            torch.zeros(B, Hkv, T, dtype=torch.float16),
+            torch.zeros(B, Hkv, T, d, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):             # state of the wrong width
+        jl.jl_decode_attention_state(*args, state=torch.zeros(B, Hq, d))
+    with pytest.raises(ValueError):
+        jl.jl_decode_attention_state(*args)
+
+
 @pytest.mark.parametrize("fn", ["jl_decode_attention", "jl_decode_attention_noalloc"])
 def test_decode_wrappers_check_shapes_and_dtypes(lib, fn):
     # the library sizes its copies from the shapes, so the binding must refuse
